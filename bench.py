@@ -1,0 +1,429 @@
+"""Benchmark: tree-packed KDA forward + backward on one or more B200s.
+
+One step = the whole hot path (planned rounds: forward and backward of the
+tree-packed chunkwise KDA layer) over one synthetic rollout tree: the
+single-fork tree (8192-token prefix -> 16 branches of U[512, 2048] tokens),
+H = 16, d_k = d_v = 128, chunk 64, bf16 inputs with fp32 state.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tpc|reference]
+
+N > 1 runs under torchrun: each rank processes its own tree (weak scaling, no
+data-path collective); the time is the max over ranks.  Rank 0 prints one
+JSON line.  ``--impl reference`` times the fp64 CPU oracle on bounded samples
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "tree-packed KDA fwd+bwd tokens/s (unique & expanded); % of TC/HBM roofline"
+WORKLOAD = "single_fork"
+
+# algorithmic FLOP per processed token-head of each kernel (chunk C, head dim d), see the design doc
+def kernel_flops(name, C, d):
+    Cd, dd = C * d, d * d
+    return {"kda_fwd_prep": 6 * Cd, "kda_fwd_scan": 4 * dd, "kda_fwd_out": 4 * Cd + 2 * dd,
+            "kda_bwd_prep": 2 * Cd + 4 * dd, "kda_bwd_scan": 4 * dd, "kda_bwd_dq": 6 * Cd + 4 * dd,
+            "kda_bwd_dkv": 10 * Cd + 2 * dd}.get(name, 0)
+
+
+# algorithmic HBM bytes per token-head of the whole step (bf16 I/O): forward reads q,k,v,g (8d)
+# + beta (2) and writes o (2d); backward reads those and dO and writes dq,dk,dv (6d), dg (4d), dbeta (4)
+def step_bytes_per_token_head(d):
+    return (8 * d + 2 + 2 * d) + (8 * d + 2 + 2 * d + 6 * d + 4 * d + 4)
+
+
+def step_flops_per_token_head(C, d):
+    return 3 * (10 * C * d + 6 * d * d)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"], sustained=j.get("bf16_tflops_sustained"),
+                    sm_max_mhz=j.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def setup_dist():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "tree_packed_chunkwise_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel):
+    """dram bytes per launch from a committed ncu capture, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(kernel)
+    if not e or e.get("source_hash") != source_hash(["kda_kernels.cuh", "common.cuh"]):
+        return None
+    return e["bytes_per_launch"]
+
+
+# ------------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, n_tokens, seed):
+    """fp64 oracle fwd+bwd on a bounded sample: the first n_tokens of the first trajectory."""
+    from oracle import kda as okda
+    t = w.tree
+    rows = t.trajectory_rows(t.leaves()[0])[:n_tokens]
+    inp = synth.kda_inputs(seed, rows, w.H, w.dk, w.dv, w.dtype)
+    d_o = synth.rows_normal(seed, synth.STREAM["d_o"], rows, w.H * w.dv, w.dtype).reshape(len(rows), w.H, w.dv)
+    t0 = time.perf_counter()
+    okda.forward(*inp)
+    okda.backward(*inp, d_o)
+    return time.perf_counter() - t0, len(rows)
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def run_reference(args, ws, rank):
+    w = synth.workload(WORKLOAD)
+    if rank != 0:
+        return
+    n_tok = args.ref_tokens
+    oracle_sample(w, 8, w.seed)  # warm caches / imports
+    for _ in range(args.warmup):
+        oracle_sample(w, 16, w.seed)
+    tot_t, tot_n = 0.0, 0
+    for _ in range(args.steps):
+        dt, n = oracle_sample(w, n_tok, w.seed)
+        tot_t += dt
+        tot_n += n
+    rate = tot_n / tot_t
+    sample = f"first {n_tok} tokens of trajectory 0 (H={w.H}, d={w.dk}) fwd+bwd per step, fp64 numpy"
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "sample_tokens_per_step": n_tok},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------ GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="tpc", choices=["tpc", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=192)
+    ap.add_argument("--cpu-tokens", type=int, default=768)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-expanded", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "tpc" else args.warmup
+
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, ws, rank)
+        return
+
+    import torch
+    import tree_packed_chunkwise_b200 as tpc
+
+    world, rank, local = setup_dist()
+    w = synth.workload(WORKLOAD)
+    t = w.tree
+    seed = w.seed + 1000 * rank
+    plan = tpc.Plan(t.parent, t.length, w.chunk).upload()
+    info = plan.info
+    N, H, d = info["n_unique"], w.H, w.dk
+    st = t.node_start()
+    # inputs drawn on the device by the generator twin (same bits as synth's host generator)
+    import synth.gpu as sgpu
+    src_rows = torch.tensor(plan.compact_source_rows(st, t.length), dtype=torch.int32, device="cuda")
+    bf = torch.bfloat16
+    dev = dict(zip(("q", "k", "v", "g", "beta"), sgpu.kda_inputs(seed, src_rows, H, d, d, w.dtype)))
+    dev["d_o"] = sgpu.normal_rows(seed, synth.STREAM["d_o"], src_rows, H * d, w.dtype).view(N, H, d)
+    dev["d_final"] = sgpu.normal_rows(seed, synth.STREAM["d_final"], None, H * d * d, "f32",
+                                      shape=(info["n_leaves"],)).view(info["n_leaves"], H, d, d)
+    host = {k: v.cpu().pin_memory() for k, v in dev.items()}
+    shape = tpc.kda_shape(H, d, tpc.TPC_BF16, tpc.TPC_BF16)
+    wsb = tpc.alloc_workspace(plan, shape)
+    outs = dict(o=torch.empty(N, H, d, dtype=bf, device="cuda"),
+                final=torch.empty(info["n_leaves"], H, d, d, dtype=torch.float32, device="cuda"))
+    grads = dict(dq=torch.empty(N, H, d, dtype=bf, device="cuda"), dk=torch.empty(N, H, d, dtype=bf, device="cuda"),
+                 dv=torch.empty(N, H, d, dtype=bf, device="cuda"),
+                 dg=torch.empty(N, H, d, dtype=torch.float32, device="cuda"),
+                 dbeta=torch.empty(N, H, dtype=torch.float32, device="cuda"), d_init=None)
+    stream = torch.cuda.current_stream()
+
+    def step(x):
+        tpc.tpc_kda_forward(plan, x["q"], x["k"], x["v"], x["g"], x["beta"], ws=wsb, o=outs["o"],
+                            final_state=outs["final"], out_dtype=bf)
+        tpc.tpc_kda_backward(plan, wsb, x["q"], x["k"], x["v"], x["g"], x["beta"], x["d_o"], x["d_final"],
+                             out_dtype=bf, grads=grads)
+
+    for _ in range(args.warmup):
+        step(dev)
+    torch.cuda.synchronize()
+    tpc.tpc_status(plan, wsb, H, d)
+
+    # ---- timed region: K steps, inputs + workspace (> 1 GB) far larger than L2
+    n0 = tpc.tpc_launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(dev)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    launches = tpc.tpc_launch_count() - n0
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    ms_step = ms / args.steps
+    value = world * N / (ms_step / 1e3)
+    value_exp = world * info["n_expanded"] / (ms_step / 1e3)
+
+    # ---- per-kernel durations (CUDA events around each launch, separate pass)
+    tpc.tpc_profile_enable(True)
+    for _ in range(args.steps):
+        step(dev)
+    torch.cuda.synchronize()
+    prof = tpc.tpc_profile_read()
+    tpc.tpc_profile_enable(False)
+    tokens_proc = info["n_seq_tokens"]
+    kern = {}
+    for name, (n, tot) in prof.items():
+        per = tot / n
+        fl = kernel_flops(name, w.chunk, d)
+        units = tokens_proc * H if name not in ("kda_fwd_scan", "kda_bwd_scan") else tokens_proc * H / info["n_rounds"]
+        kern[name] = {"launches_per_step": n / args.steps, "ms_per_launch": per, "share": 0.0,
+                      "gflop_per_launch": fl * units / 1e9}
+    total_ms = sum(v["ms_per_launch"] * v["launches_per_step"] for v in kern.values())
+    for v in kern.values():
+        v["share"] = v["ms_per_launch"] * v["launches_per_step"] / total_ms
+    dom = max(kern, key=lambda k: kern[k]["share"])
+    peaks = load_peaks()
+    clocks = clk.summary()
+    sm_max = clocks.get("sm_max_mhz") or peaks["sm_max_mhz"]
+    alu_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12  # fp32 FMA lanes x 2 FLOP x max SM clock, TFLOP/s
+    dk = kern[dom]
+    achieved = dk["gflop_per_launch"] / dk["ms_per_launch"]  # GFLOP/ms == TFLOP/s
+    roofline = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                "frac": achieved / alu_peak, "traffic": committed_traffic(dom),
+                "peak_source": "148 SMs x 128 fp32 lanes x 2 x max SM clock"}
+    step_bytes = step_bytes_per_token_head(d) * tokens_proc * H
+    step_flops = step_flops_per_token_head(w.chunk, d) * tokens_proc * H
+    step_roof = {"hbm_frac": (step_bytes / (ms_step / 1e3)) / (peaks["hbm_gbs"] * 1e9),
+                 "tc_frac": (step_flops / (ms_step / 1e3)) / (peaks["bf16_tflops"] * 1e12),
+                 "algorithmic_bytes": step_bytes, "algorithmic_flops": step_flops, "peak_source": peaks["source"]}
+
+    # ---- trajectory-expanded comparator: the same kernels, one sequence per trajectory
+    expanded = None
+    if not args.no_expanded:
+        tb = plan.tables()
+        lens = np.diff(tb["traj_offset"]).astype(np.int32)
+        eplan = tpc.Plan(np.full(len(lens), -1, np.int32), lens, w.chunk).upload()
+        xe = {k: tpc.tpc_gather_expanded(plan, dev[k]) for k in ("q", "k", "v", "g", "beta", "d_o")}
+        xe["d_final"] = dev["d_final"]
+        NE = eplan.info["n_unique"]
+        ews = tpc.alloc_workspace(eplan, shape)
+        eo = torch.empty(NE, H, d, dtype=bf, device="cuda")
+        ef = torch.empty(eplan.info["n_leaves"], H, d, d, dtype=torch.float32, device="cuda")
+        eg = {k: torch.empty_like(xe["q"]) for k in ("dq", "dk", "dv")}
+        eg.update(dg=torch.empty(NE, H, d, dtype=torch.float32, device="cuda"),
+                  dbeta=torch.empty(NE, H, dtype=torch.float32, device="cuda"), d_init=None)
+
+        def estep():
+            tpc.tpc_kda_forward(eplan, xe["q"], xe["k"], xe["v"], xe["g"], xe["beta"], ws=ews, o=eo, final_state=ef,
+                                out_dtype=bf)
+            tpc.tpc_kda_backward(eplan, ews, xe["q"], xe["k"], xe["v"], xe["g"], xe["beta"], xe["d_o"], xe["d_final"],
+                                 out_dtype=bf, grads=eg)
+
+        for _ in range(2):
+            estep()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ek = max(2, args.steps // 4)
+        e0.record(stream)
+        for _ in range(ek):
+            estep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), world) / ek
+        expanded = {"ms_per_step": ems, "expanded_tokens_per_s": world * info["n_expanded"] / (ems / 1e3),
+                    "speedup_tree_vs_expanded": ems / ms_step,
+                    "target_speedup": info["n_expanded"] / info["n_seq_tokens"]}
+        del ews, xe, eg
+
+    # ---- end to end through the C ABI with host buffers: H2D inputs, fwd+bwd, D2H results
+    e2e = None
+    if not args.no_e2e:
+        hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in
+                [("o", outs["o"]), ("final", outs["final"])] + [(k, grads[k]) for k in ("dq", "dk", "dv", "dg", "dbeta")]}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+
+        def e2e_step():
+            for k in host:
+                dev[k].copy_(host[k], non_blocking=True)
+            step(dev)
+            hout["o"].copy_(outs["o"], non_blocking=True)
+            hout["final"].copy_(outs["final"], non_blocking=True)
+            for k in ("dq", "dk", "dv", "dg", "dbeta"):
+                hout[k].copy_(grads[k], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ams = max_over_ranks(a0.elapsed_time(a1), world) / args.steps
+        e2e = {"value": world * N / (ams / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ams}
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, n = oracle_sample(w, args.cpu_tokens, seed)
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"first {n} tokens of trajectory 0 (H={H}, d={d}) fwd+bwd, fp64 numpy, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16 in/out, fp32 state and accumulation", "data": "synthetic",
+                "config": {"workload": w.name, "n_unique": N, "n_expanded": info["n_expanded"],
+                           "replay_rows": info["replay_total"], "rounds": info["n_rounds"], "chunk": w.chunk,
+                           "heads": H, "head_dim": d, "parallelism": f"dp{world} (independent trees)",
+                           "l2": "inputs+workspace > 1 GB per step, larger than L2"},
+                "value_expanded": value_exp, "roofline": roofline, "step_roofline": step_roof,
+                "kernels": kern, "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+                "expanded_path": expanded}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

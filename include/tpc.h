@@ -1,0 +1,231 @@
+/*
+ * tpc.h -- C ABI of the B200 (sm_100a) tree-packed chunkwise KDA library.
+ *
+ * The operation: chunkwise gated delta-rule ("KDA") linear attention,
+ * forward and backward, run once over a prefix-shared rollout tree instead
+ * of once per root-to-leaf trajectory (HARTS: "A Prefix-Sharing Training
+ * System for Agentic RL with Hybrid-Attention Models", abstract; Figure 1;
+ * Figure 2; Figure C.1).  Per token t and head, with g_t = log(alpha_t):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * Conventions shared by every call
+ *  - Trees are parent-pointer forests of fork-free segments (HARTS Figure
+ *    2(a)).  parent[i] = -1 (root) or a smaller id; length[i] >= 1.  The
+ *    trajectories are the root-to-leaf paths, ordered by leaf id.
+ *  - Token tensors use the plan's compact layout (HARTS Figure C.1(a): one
+ *    physical row per unique token): segment v occupies rows
+ *    row_offset[v] .. row_offset[v] + length[v] - 1 (tpc_plan_export).
+ *    Row-major [N_unique, H, d]; beta is [N_unique, H].
+ *  - All device memory (tensors, plan tables, workspace) is owned by the
+ *    caller and passed as raw pointers.  The library owns only the opaque
+ *    host-side plan object.
+ *  - Device calls are asynchronous on the given stream and never
+ *    synchronise; a zero stream means the legacy default stream.
+ *  - Every call returns a status code (TPC_OK = 0).  tpc_last_error()
+ *    gives a message for the calling thread.  Nothing aborts and no C++
+ *    exception crosses this boundary.  Kernel-side checks (gate range,
+ *    table bounds) record a code in the workspace status word; read it with
+ *    tpc_status().
+ */
+#ifndef TPC_H_
+#define TPC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tpc_stream_t; /* == cudaStream_t */
+
+enum tpc_status_code {
+  TPC_OK = 0,
+  TPC_ERR_INVALID_TREE = 1, /* parent order, range or zero-length segment */
+  TPC_ERR_BAD_SHAPE = 2,    /* inconsistent sizes */
+  TPC_ERR_UNSUPPORTED = 3,  /* head dims / chunk size not built */
+  TPC_ERR_NULL = 4,         /* required pointer is NULL */
+  TPC_ERR_WORKSPACE = 5,    /* workspace too small or misaligned */
+  TPC_ERR_CUDA = 6,         /* a CUDA runtime call failed */
+  TPC_ERR_DEVICE_CHECK = 7, /* a kernel-side check failed (see tpc_status) */
+  TPC_ERR_TIMEOUT = 8,      /* a bounded device wait ran out */
+  TPC_ERR_RANGE = 9,        /* gates outside the supported range */
+  TPC_ERR_STATE = 10        /* plan not uploaded / wrong call order */
+};
+
+enum tpc_dtype { TPC_F32 = 0, TPC_BF16 = 1 };
+
+/* Returns the message of the last failed call on this thread ("" if none). */
+const char* tpc_last_error(void);
+/* Library version string. */
+const char* tpc_version(void);
+
+/* ------------------------------------------------------------------ plan */
+typedef struct tpc_plan tpc_plan;
+
+/*
+ * Round planner (HARTS abstract: a linear-time planner reaching the minimum
+ * number of sequential packed linear-attention calls; Figure 2: direct
+ * continuations, replay-started side sequences, a boundary state usable
+ * only by a later call).  Runs on the host in O(n_nodes + tokens/chunk).
+ *   parent, length: host arrays of n_nodes int32 (see conventions).
+ *   chunk: chunk size C (16, 32 or 64).
+ *   *out: receives a new plan; free it with tpc_plan_destroy.
+ * Errors: TPC_ERR_NULL, TPC_ERR_INVALID_TREE, TPC_ERR_UNSUPPORTED.
+ */
+int tpc_plan_create(const int32_t* parent, const int32_t* length, int32_t n_nodes,
+                    int32_t chunk, tpc_plan** out);
+void tpc_plan_destroy(tpc_plan* plan);
+
+typedef struct tpc_plan_info {
+  int64_t n_unique;     /* unique token rows N */
+  int64_t n_expanded;   /* sum of trajectory lengths */
+  int64_t replay_total; /* replayed rows over all sequences (R) */
+  int64_t n_seq_tokens; /* rows processed by the packed calls = N + R */
+  int32_t n_nodes, n_rounds, n_seqs, n_chunks, n_slots, n_leaves, n_roots, chunk;
+  int32_t max_seq_chunks; /* longest sequence, in chunks */
+  int32_t n_replay_targets;
+} tpc_plan_info;
+int tpc_plan_get_info(const tpc_plan* plan, tpc_plan_info* info);
+
+/*
+ * Host tables (bit-exact comparison surface).  Every member is a
+ * caller-owned host array or NULL (skipped).  Sizes: per node n_nodes,
+ * leaves n_leaves, expanded_rows n_expanded, traj_offset n_leaves + 1.
+ *   round        1-based round of the packed call that computes the node
+ *   is_cont      1 if the node continues its parent's sequence
+ *   anchor       node holding token b_v - 1 (b_v = floor(s_v/C)*C), -1 if b_v = 0
+ *   replay_start first position of a sequence head (b_v, 0 for roots), -1 otherwise
+ *   replay_len   replayed rows of a sequence head (s_v - b_v), -1 otherwise
+ *   row_offset   first compact row of the node
+ *   occurrence   number of trajectories through the node (HARTS Figure 1: q_B)
+ *   leaves       leaf node ids in trajectory order
+ *   expanded_rows compact row of every trajectory position, trajectories concatenated
+ *   traj_offset  start of each trajectory in expanded_rows
+ */
+typedef struct tpc_plan_tables {
+  int32_t* round;
+  int32_t* is_cont;
+  int32_t* anchor;
+  int32_t* replay_start;
+  int32_t* replay_len;
+  int64_t* row_offset;
+  int32_t* occurrence;
+  int32_t* leaves;
+  int64_t* expanded_rows;
+  int64_t* traj_offset;
+} tpc_plan_tables;
+int tpc_plan_export(const tpc_plan* plan, tpc_plan_tables* tables);
+
+/*
+ * Device index tables: bytes needed, and the upload.  The caller allocates
+ * `bytes` of device memory (256-byte aligned); tpc_plan_upload copies the
+ * sequence, chunk, slot and replay tables there (async on `stream`) and
+ * records the address in the plan, which every later device call uses.
+ * The memory must stay valid while the plan is used.
+ */
+size_t tpc_plan_device_bytes(const tpc_plan* plan);
+int tpc_plan_upload(tpc_plan* plan, void* dev, size_t bytes, tpc_stream_t stream);
+
+/* ------------------------------------------------------------------ KDA */
+typedef struct tpc_kda_shape {
+  int32_t H;          /* heads */
+  int32_t dk, dv;     /* head dims; dk == dv in {32, 64, 128} */
+  int32_t in_dtype;   /* tpc_dtype of q, k, v, g, beta, d_o */
+  int32_t out_dtype;  /* tpc_dtype of o, dq, dk, dv */
+} tpc_kda_shape;
+
+/*
+ * Workspace bytes for tpc_kda_forward + tpc_kda_backward on this plan.
+ * The forward leaves in it what the backward reads (chunk-start states,
+ * U, W, boundary-state slots); do not reuse it in between.  256-byte
+ * aligned.  Returns 0 for an unsupported shape.
+ */
+size_t tpc_kda_workspace_bytes(const tpc_plan* plan, const tpc_kda_shape* shape);
+
+typedef struct tpc_kda_fwd_io {
+  const void* q;          /* [N, H, dk] in_dtype */
+  const void* k;          /* [N, H, dk] in_dtype, any norm */
+  const void* v;          /* [N, H, dv] in_dtype */
+  const void* g;          /* [N, H, dk] in_dtype, log(alpha) <= 0 */
+  const void* beta;       /* [N, H]     in_dtype */
+  const float* init_state;/* [n_roots, H, dk, dv] fp32 or NULL (= 0) */
+  void* o;                /* [N, H, dv] out_dtype */
+  float* final_state;     /* [n_leaves, H, dk, dv] fp32 or NULL */
+} tpc_kda_fwd_io;
+
+/*
+ * Tree-packed forward: for each round, one packed launch over every
+ * sequence of the round (HARTS Figure 2(c)); sequences start from the
+ * initial state or from a boundary state exported by an earlier round and
+ * replay the rows between the aligned boundary and their first own row
+ * without writing outputs (Figure C.1(b)).  Outputs equal the per-trajectory
+ * recurrence (the chunk grid is aligned to trajectory positions).
+ * Errors: TPC_ERR_NULL, TPC_ERR_STATE (plan not uploaded),
+ * TPC_ERR_UNSUPPORTED, TPC_ERR_WORKSPACE, TPC_ERR_CUDA.
+ */
+int tpc_kda_forward(const tpc_plan* plan, const tpc_kda_shape* shape, const tpc_kda_fwd_io* io,
+                    void* ws, size_t ws_bytes, tpc_stream_t stream);
+
+typedef struct tpc_kda_bwd_io {
+  const void* q; const void* k; const void* v; const void* g; const void* beta; /* as forward */
+  const float* init_state;  /* as forward */
+  const void* d_o;          /* [N, H, dv] in_dtype: output gradient per unique row */
+  const float* d_final;     /* [n_leaves, H, dk, dv] fp32 or NULL */
+  void* dq; void* dk; void* dv; /* [N, H, d] out_dtype */
+  float* dg;                /* [N, H, dk] fp32 (gradient w.r.t. log alpha) */
+  float* dbeta;             /* [N, H] fp32 */
+  float* d_init;            /* [n_roots, H, dk, dv] fp32 or NULL */
+} tpc_kda_bwd_io;
+
+/*
+ * Backward of sum <d_o, o> + sum <d_final, final_state>: rounds in reverse;
+ * the gradient of each boundary state is the sum of its consumers'
+ * gradients, in a fixed order, added before the producer's reverse scan
+ * crosses that boundary (HARTS abstract: gradients from dependent work
+ * accumulate before one backward pass through the shared prefix).
+ * Replayed rows contribute to the gradients of their own rows in a fixed
+ * order; results are bitwise reproducible.  Requires the workspace of a
+ * tpc_kda_forward on the same inputs.
+ */
+int tpc_kda_backward(const tpc_plan* plan, const tpc_kda_shape* shape, const tpc_kda_bwd_io* io,
+                     void* ws, size_t ws_bytes, tpc_stream_t stream);
+
+/*
+ * Reads (after synchronising `stream`) and clears the status word that
+ * kernels write in `ws`.  Returns TPC_OK or the first recorded error.
+ */
+int tpc_status(const tpc_plan* plan, const tpc_kda_shape* shape, void* ws, tpc_stream_t stream);
+
+/* ------------------------------------------------------------------ row maps */
+/*
+ * Deterministic occurrence sum (HARTS Figure 1: one row serves every
+ * trajectory through it): x_unique[r] = sum over occurrences of r, in
+ * trajectory order, of x_exp[j].  x_exp is [n_expanded, width] and
+ * x_unique [N, width], both fp32.
+ */
+int tpc_reduce_expanded_to_unique(const tpc_plan* plan, const float* x_exp, float* x_unique,
+                                  int64_t width, tpc_stream_t stream);
+/* Gather to the trajectory-expanded layout: x_exp[j] = x_unique[expanded_rows[j]];
+ * elem_bytes 2 or 4, width elements per row. */
+int tpc_gather_expanded(const tpc_plan* plan, const void* x_unique, void* x_exp, int64_t width,
+                        int32_t elem_bytes, tpc_stream_t stream);
+/* Occurrence count per compact row (int32 [N]). */
+int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t stream);
+
+/* ------------------------------------------------------------------ diagnostics */
+/* Per-kernel timing: when enabled, every launch is bracketed by CUDA events recorded on
+ * its stream (adds a few microseconds per launch).  Not thread safe. */
+void tpc_profile_enable(int on);
+/* Synchronises the recorded events and writes "name launches total_ms" lines into buf
+ * (truncated to len), then clears the records. */
+int tpc_profile_read(char* buf, size_t len);
+/* Number of kernels this library has launched in the process. */
+long long tpc_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TPC_H_ */

@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI library (no GPU needed): every declared symbol is
+exported, and the C++ planner's tables equal the oracle planner's bit for bit."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import planner as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def tpc():
+    from tree_packed_chunkwise_b200 import build
+    build.build()
+    import tree_packed_chunkwise_b200 as t
+    t.lib()
+    return t
+
+
+def declared_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(tpc_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported(tpc):
+    names = declared_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(tpc.lib(), n), n
+    assert names <= set(tpc.SIGNATURES), names - set(tpc.SIGNATURES)
+
+
+def compare(tpc, parent, length, C):
+    ref = P.plan(parent, length, C)
+    pl = tpc.Plan(parent, length, C)
+    tb = pl.tables()
+    assert pl.info["n_rounds"] == ref.n_rounds
+    assert np.array_equal(tb["round"], ref.round)
+    assert np.array_equal(tb["is_cont"], ref.cont)
+    assert np.array_equal(tb["anchor"], ref.anchor)
+    assert np.array_equal(tb["replay_start"], ref.replay_start)
+    assert np.array_equal(tb["replay_len"], ref.replay_len)
+    assert np.array_equal(tb["row_offset"], ref.row_offset)
+    assert np.array_equal(tb["occurrence"], ref.occurrence)
+    assert np.array_equal(tb["leaves"], ref.leaves)
+    rows, offs = P.expanded_rows(ref)
+    assert np.array_equal(tb["expanded_rows"], rows)
+    assert np.array_equal(tb["traj_offset"], offs)
+    assert pl.info["replay_total"] == ref.replay_total
+    assert pl.info["n_slots"] == len(ref.slots)
+    assert pl.info["n_seqs"] == len(ref.seqs)
+    return pl
+
+
+@pytest.mark.parametrize("cfg", ["fig1", "single_fork", "agentic", "agentic_small", "wide"])
+def test_planner_bit_exact_on_workloads(tpc, cfg):
+    w = synth.workload(cfg)
+    compare(tpc, w.tree.parent, w.tree.length, w.chunk)
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+def test_planner_bit_exact_random(tpc, C):
+    rng = np.random.default_rng(C)
+    for _ in range(400):
+        n = int(rng.integers(1, 40))
+        parent = [-1] + [(-1 if rng.random() < 0.05 else int(rng.integers(0, i))) for i in range(1, n)]
+        length = rng.integers(1, 4 * C, size=n)
+        compare(tpc, parent, length, C)
+
+
+def test_fig1_chunk_table(tpc):
+    w = synth.workload("fig1")
+    pl = tpc.Plan(w.tree.parent, w.tree.length, 16)
+    assert pl.info["n_chunks"] == 9 and pl.info["n_rounds"] == 2 and pl.info["replay_total"] == 8
+    assert pl.info["n_unique"] == 121 and pl.info["n_expanded"] == 225
+
+
+def test_invalid_inputs_return_status(tpc):
+    with pytest.raises(tpc.TpcError) as e:
+        tpc.Plan([-1, 2, 0], [1, 1, 1], 16)
+    assert e.value.code == 1
+    with pytest.raises(tpc.TpcError) as e:
+        tpc.Plan([-1, 0], [4, 0], 16)
+    assert e.value.code == 1
+    with pytest.raises(tpc.TpcError) as e:
+        tpc.Plan([-1], [4], 48)
+    assert e.value.code == 3
+    assert tpc.lib().tpc_plan_device_bytes(None) == 0

@@ -1,0 +1,297 @@
+"""Python binding of ``libtpc.so``: tree-packed chunkwise KDA on B200 (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  PyTorch provides device memory and streams.  The
+functions keep the C names of ``include/tpc.h``.  There is no CPU fallback:
+without the built library or a CUDA device the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtpc.so")
+
+TPC_F32, TPC_BF16 = 0, 1
+_STATUS = {0: "TPC_OK", 1: "TPC_ERR_INVALID_TREE", 2: "TPC_ERR_BAD_SHAPE", 3: "TPC_ERR_UNSUPPORTED",
+           4: "TPC_ERR_NULL", 5: "TPC_ERR_WORKSPACE", 6: "TPC_ERR_CUDA", 7: "TPC_ERR_DEVICE_CHECK",
+           8: "TPC_ERR_TIMEOUT", 9: "TPC_ERR_RANGE", 10: "TPC_ERR_STATE"}
+
+i32p = ctypes.POINTER(ctypes.c_int32)
+i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+class TpcError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{_STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("n_unique", ctypes.c_int64), ("n_expanded", ctypes.c_int64), ("replay_total", ctypes.c_int64),
+                ("n_seq_tokens", ctypes.c_int64), ("n_nodes", ctypes.c_int32), ("n_rounds", ctypes.c_int32),
+                ("n_seqs", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("n_slots", ctypes.c_int32),
+                ("n_leaves", ctypes.c_int32), ("n_roots", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("max_seq_chunks", ctypes.c_int32), ("n_replay_targets", ctypes.c_int32)]
+
+
+class PlanTables(ctypes.Structure):
+    _fields_ = [("round", i32p), ("is_cont", i32p), ("anchor", i32p), ("replay_start", i32p),
+                ("replay_len", i32p), ("row_offset", i64p), ("occurrence", i32p), ("leaves", i32p),
+                ("expanded_rows", i64p), ("traj_offset", i64p)]
+
+
+class KdaShape(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
+                ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
+class KdaFwdIO(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("g", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("init_state", ctypes.c_void_p), ("o", ctypes.c_void_p),
+                ("final_state", ctypes.c_void_p)]
+
+
+class KdaBwdIO(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("g", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("init_state", ctypes.c_void_p), ("d_o", ctypes.c_void_p),
+                ("d_final", ctypes.c_void_p), ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p),
+                ("dv", ctypes.c_void_p), ("dg", ctypes.c_void_p), ("dbeta", ctypes.c_void_p),
+                ("d_init", ctypes.c_void_p)]
+
+
+# exported symbols of include/tpc.h: name -> (restype, argtypes)
+_V, _P = ctypes.c_void_p, ctypes.POINTER
+SIGNATURES = {
+    "tpc_last_error": (ctypes.c_char_p, []),
+    "tpc_version": (ctypes.c_char_p, []),
+    "tpc_plan_create": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int32, _P(_V)]),
+    "tpc_plan_destroy": (None, [_V]),
+    "tpc_plan_get_info": (ctypes.c_int, [_V, _P(PlanInfo)]),
+    "tpc_plan_export": (ctypes.c_int, [_V, _P(PlanTables)]),
+    "tpc_plan_device_bytes": (ctypes.c_size_t, [_V]),
+    "tpc_plan_upload": (ctypes.c_int, [_V, _V, ctypes.c_size_t, _V]),
+    "tpc_kda_workspace_bytes": (ctypes.c_size_t, [_V, _P(KdaShape)]),
+    "tpc_kda_forward": (ctypes.c_int, [_V, _P(KdaShape), _P(KdaFwdIO), _V, ctypes.c_size_t, _V]),
+    "tpc_kda_backward": (ctypes.c_int, [_V, _P(KdaShape), _P(KdaBwdIO), _V, ctypes.c_size_t, _V]),
+    "tpc_status": (ctypes.c_int, [_V, _P(KdaShape), _V, _V]),
+    "tpc_reduce_expanded_to_unique": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, _V]),
+    "tpc_gather_expanded": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int32, _V]),
+    "tpc_occurrence_counts": (ctypes.c_int, [_V, _V, _V]),
+    "tpc_profile_enable": (None, [ctypes.c_int]),
+    "tpc_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t]),
+    "tpc_launch_count": (ctypes.c_longlong, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run tree_packed_chunkwise_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != 0:
+        raise TpcError(rc, lib().tpc_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ------------------------------------------------------------------------------------ plan
+class Plan:
+    """Round plan of a rollout tree (host object; ``upload`` places its tables on the device)."""
+
+    def __init__(self, parent, length, chunk: int):
+        parent = np.ascontiguousarray(parent, np.int32)
+        length = np.ascontiguousarray(length, np.int32)
+        h = ctypes.c_void_p()
+        _check(lib().tpc_plan_create(parent.ctypes.data_as(i32p), length.ctypes.data_as(i32p),
+                                     int(parent.shape[0]), int(chunk), ctypes.byref(h)))
+        self._h = h
+        self.n_nodes = int(parent.shape[0])
+        info = PlanInfo()
+        _check(lib().tpc_plan_get_info(self._h, ctypes.byref(info)))
+        self.info = {f: getattr(info, f) for f, _ in PlanInfo._fields_}
+        self.dev_tables = None
+
+    def __del__(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.tpc_plan_destroy(self._h)
+            self._h = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    def tables(self) -> dict:
+        n, nl, ne = self.n_nodes, self.info["n_leaves"], self.info["n_expanded"]
+        out = {k: np.zeros(n, np.int32) for k in ("round", "is_cont", "anchor", "replay_start", "replay_len",
+                                                  "occurrence")}
+        out["row_offset"] = np.zeros(n, np.int64)
+        out["leaves"] = np.zeros(nl, np.int32)
+        out["expanded_rows"] = np.zeros(ne, np.int64)
+        out["traj_offset"] = np.zeros(nl + 1, np.int64)
+        t = PlanTables(**{k: v.ctypes.data_as(i64p if v.dtype == np.int64 else i32p) for k, v in out.items()})
+        _check(lib().tpc_plan_export(self._h, ctypes.byref(t)))
+        return out
+
+    def upload(self, device="cuda", stream=None):
+        import torch
+        nbytes = int(lib().tpc_plan_device_bytes(self._h))
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _check(lib().tpc_plan_upload(self._h, _ptr(buf), nbytes, _stream_ptr(stream)))
+        self.dev_tables = buf
+        return self
+
+    def compact_source_rows(self, node_start: np.ndarray, length: np.ndarray) -> np.ndarray:
+        """For every compact row, the node-order row (rows of node 0, node 1, ...) it holds."""
+        tb = self.tables()
+        perm = np.empty(int(length.sum()), np.int64)
+        for v in range(self.n_nodes):
+            perm[tb["row_offset"][v]:tb["row_offset"][v] + length[v]] = np.arange(node_start[v], node_start[v] + length[v])
+        return perm
+
+    def to_compact(self, node_rows_array: np.ndarray, node_start: np.ndarray, length: np.ndarray) -> np.ndarray:
+        """Reorders a node-order row array to the compact layout."""
+        return node_rows_array[self.compact_source_rows(node_start, length)]
+
+
+# ------------------------------------------------------------------------------------ KDA
+def _dtype_code(t):
+    import torch
+    return TPC_BF16 if t.dtype == torch.bfloat16 else TPC_F32
+
+
+def kda_shape(H, d, in_dtype, out_dtype) -> KdaShape:
+    return KdaShape(H, d, d, in_dtype, out_dtype)
+
+
+def tpc_kda_workspace_bytes(plan: Plan, shape: KdaShape) -> int:
+    return int(lib().tpc_kda_workspace_bytes(plan.handle, ctypes.byref(shape)))
+
+
+def alloc_workspace(plan: Plan, shape: KdaShape, device="cuda"):
+    import torch
+    n = tpc_kda_workspace_bytes(plan, shape)
+    if n == 0:
+        raise TpcError(3, "unsupported shape for this plan")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def tpc_kda_forward(plan: Plan, q, k, v, g, beta, init_state=None, out_dtype=None, ws=None, o=None,
+                    final_state=None, want_final=True, stream=None):
+    """Tree-packed forward.  Tensors in compact row order; returns (o, final_state, ws)."""
+    import torch
+    N, H, d = q.shape
+    out_dtype = out_dtype or q.dtype
+    shape = kda_shape(H, d, _dtype_code(q), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
+    if ws is None:
+        ws = alloc_workspace(plan, shape, q.device)
+    if o is None:
+        o = torch.empty(N, H, d, dtype=out_dtype, device=q.device)
+    if final_state is None and want_final:
+        final_state = torch.empty(plan.info["n_leaves"], H, d, d, dtype=torch.float32, device=q.device)
+    io = KdaFwdIO(_ptr(q).value, _ptr(k).value, _ptr(v).value, _ptr(g).value, _ptr(beta).value,
+                  None if init_state is None else init_state.data_ptr(), o.data_ptr(),
+                  None if final_state is None else final_state.data_ptr())
+    _check(lib().tpc_kda_forward(plan.handle, ctypes.byref(shape), ctypes.byref(io), _ptr(ws), ws.numel(),
+                                 _stream_ptr(stream)))
+    return o, final_state, ws
+
+
+def tpc_kda_backward(plan: Plan, ws, q, k, v, g, beta, d_o, d_final=None, init_state=None, out_dtype=None,
+                     want_d_init=True, grads=None, stream=None):
+    """Backward; returns dict(dq, dk, dv, dg, dbeta, d_init)."""
+    import torch
+    N, H, d = q.shape
+    out_dtype = out_dtype or q.dtype
+    shape = kda_shape(H, d, _dtype_code(q), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
+    if grads is None:
+        dev = q.device
+        grads = dict(dq=torch.empty(N, H, d, dtype=out_dtype, device=dev),
+                     dk=torch.empty(N, H, d, dtype=out_dtype, device=dev),
+                     dv=torch.empty(N, H, d, dtype=out_dtype, device=dev),
+                     dg=torch.empty(N, H, d, dtype=torch.float32, device=dev),
+                     dbeta=torch.empty(N, H, dtype=torch.float32, device=dev),
+                     d_init=torch.empty(plan.info["n_roots"], H, d, d, dtype=torch.float32, device=dev)
+                     if want_d_init else None)
+    io = KdaBwdIO(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
+                  None if init_state is None else init_state.data_ptr(), d_o.data_ptr(),
+                  None if d_final is None else d_final.data_ptr(),
+                  grads["dq"].data_ptr(), grads["dk"].data_ptr(), grads["dv"].data_ptr(), grads["dg"].data_ptr(),
+                  grads["dbeta"].data_ptr(), None if grads.get("d_init") is None else grads["d_init"].data_ptr())
+    _check(lib().tpc_kda_backward(plan.handle, ctypes.byref(shape), ctypes.byref(io), _ptr(ws), ws.numel(),
+                                  _stream_ptr(stream)))
+    return grads
+
+
+def tpc_status(plan: Plan, ws, H, d, stream=None):
+    shape = kda_shape(H, d, 0, 0)
+    _check(lib().tpc_status(plan.handle, ctypes.byref(shape), _ptr(ws), _stream_ptr(stream)))
+
+
+def tpc_reduce_expanded_to_unique(plan: Plan, x_exp, stream=None):
+    import torch
+    width = int(np.prod(x_exp.shape[1:]))
+    out = torch.empty((plan.info["n_unique"],) + tuple(x_exp.shape[1:]), dtype=torch.float32, device=x_exp.device)
+    _check(lib().tpc_reduce_expanded_to_unique(plan.handle, _ptr(x_exp), _ptr(out), width, _stream_ptr(stream)))
+    return out
+
+
+def tpc_gather_expanded(plan: Plan, x_unique, stream=None):
+    import torch
+    width = int(np.prod(x_unique.shape[1:]))
+    out = torch.empty((plan.info["n_expanded"],) + tuple(x_unique.shape[1:]), dtype=x_unique.dtype,
+                      device=x_unique.device)
+    _check(lib().tpc_gather_expanded(plan.handle, _ptr(x_unique), _ptr(out), width, x_unique.element_size(),
+                                     _stream_ptr(stream)))
+    return out
+
+
+def tpc_occurrence_counts(plan: Plan, device="cuda", stream=None):
+    import torch
+    out = torch.empty(plan.info["n_unique"], dtype=torch.int32, device=device)
+    _check(lib().tpc_occurrence_counts(plan.handle, _ptr(out), _stream_ptr(stream)))
+    return out
+
+
+# ------------------------------------------------------------------------------------ diagnostics
+def tpc_profile_enable(on: bool):
+    lib().tpc_profile_enable(1 if on else 0)
+
+
+def tpc_profile_read() -> dict:
+    """{kernel name: (launches, total ms)} of the launches recorded since the last read."""
+    buf = ctypes.create_string_buffer(1 << 16)
+    _check(lib().tpc_profile_read(buf, len(buf)))
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, n, ms = line.split()
+        out[name] = (int(n), float(ms))
+    return out
+
+
+def tpc_launch_count() -> int:
+    return int(lib().tpc_launch_count())

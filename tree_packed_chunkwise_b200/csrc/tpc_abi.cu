@@ -1,0 +1,428 @@
+// C ABI of the tree-packed chunkwise KDA library (declarations and contracts in include/tpc.h).
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/tpc.h"
+#include "kda_kernels.cuh"
+#include "plan.h"
+#include "rowmap_kernels.cuh"
+
+struct tpc_plan {
+  tpc::Plan p;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+
+#define TPC_CUDA(call)                                                                  \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess) return fail(TPC_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Optional per-kernel timing: CUDA events around every launch (on the launching stream).
+struct Profiler {
+  bool on = false;
+  long long launches = 0;
+  struct Rec { const char* name; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+};
+Profiler g_prof;
+
+#define TPC_LAUNCH(NAME, STREAM, ...)                                     \
+  do {                                                                    \
+    cudaEvent_t a_ = nullptr, b_ = nullptr;                               \
+    if (g_prof.on) {                                                      \
+      TPC_CUDA(cudaEventCreate(&a_));                                     \
+      TPC_CUDA(cudaEventCreate(&b_));                                     \
+      TPC_CUDA(cudaEventRecord(a_, STREAM));                              \
+    }                                                                     \
+    __VA_ARGS__;                                                          \
+    TPC_CUDA(cudaGetLastError());                                         \
+    ++g_prof.launches;                                                    \
+    if (g_prof.on) {                                                      \
+      TPC_CUDA(cudaEventRecord(b_, STREAM));                              \
+      g_prof.recs.push_back({NAME, a_, b_});                              \
+    }                                                                     \
+  } while (0)
+
+// workspace layout (bytes) for a plan + shape
+struct WsLayout {
+  size_t status, W, U, Khat, decay, S0, slot, dU, dS, dS0seq, pdk, pdG, rdk, rdv, rdg, rdb, tdk, tdv, tdg, tdb, total;
+};
+
+WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
+  WsLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o += a256(bytes); return r; };
+  const size_t nc = p.chunks.size(), cd = (size_t)C * D, dd = (size_t)D * D;
+  const size_t R = (size_t)p.replay_total, T = p.tgt_row.size();
+  L.status = take(256);
+  L.W = take(nc * H * cd * 4);
+  L.U = take(nc * H * cd * 4);
+  L.Khat = take(nc * H * cd * 4);
+  L.decay = take(nc * H * D * 4);
+  L.S0 = take(nc * H * dd * 4);
+  L.slot = take(p.slots.size() * H * dd * 4);
+  L.dU = take(nc * H * cd * 4);
+  L.dS = take(nc * H * dd * 4);
+  L.dS0seq = take(p.seqs.size() * H * dd * 4);
+  L.pdk = take(nc * H * cd * 4);
+  L.pdG = take(nc * H * cd * 4);
+  L.rdk = take(R * H * D * 4);
+  L.rdv = take(R * H * D * 4);
+  L.rdg = take(R * H * D * 4);
+  L.rdb = take(R * H * 4);
+  L.tdk = take(T * H * D * 4);
+  L.tdv = take(T * H * D * 4);
+  L.tdg = take(T * H * D * 4);
+  L.tdb = take(T * H * 4);
+  L.total = o;
+  return L;
+}
+
+tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
+  char* b = static_cast<char*>(ws);
+  tpc::KdaWs w;
+  w.status = reinterpret_cast<int*>(b + L.status);
+  auto f = [&](size_t off) { return reinterpret_cast<float*>(b + off); };
+  w.W = f(L.W); w.U = f(L.U); w.Khat = f(L.Khat); w.decay = f(L.decay); w.S0 = f(L.S0); w.slot = f(L.slot);
+  w.dU = f(L.dU); w.dS = f(L.dS); w.dS0seq = f(L.dS0seq); w.pdk = f(L.pdk); w.pdG = f(L.pdG);
+  w.rdk = f(L.rdk); w.rdv = f(L.rdv); w.rdg = f(L.rdg); w.rdb = f(L.rdb);
+  w.tdk = f(L.tdk); w.tdv = f(L.tdv); w.tdg = f(L.tdg); w.tdb = f(L.tdb);
+  return w;
+}
+
+bool shape_supported(int C, int D) { return (C == 16 && D == 32) || (C == 64 && D == 128) || (C == 32 && D == 64); }
+
+int check_shape(const tpc_plan* plan, const tpc_kda_shape* s) {
+  if (!plan || !s) return fail(TPC_ERR_NULL, "plan or shape is NULL");
+  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded (tpc_plan_upload)");
+  if (s->H < 1 || s->dk < 1 || s->dv < 1) return fail(TPC_ERR_BAD_SHAPE, "H, dk, dv must be >= 1");
+  if (s->dk != s->dv) return fail(TPC_ERR_UNSUPPORTED, "dk != dv is not built");
+  if (!shape_supported(plan->p.C, s->dk))
+    return fail(TPC_ERR_UNSUPPORTED, "built (chunk, d) pairs: (16,32), (32,64), (64,128)");
+  if ((s->in_dtype != TPC_F32 && s->in_dtype != TPC_BF16) || (s->out_dtype != TPC_F32 && s->out_dtype != TPC_BF16))
+    return fail(TPC_ERR_UNSUPPORTED, "dtype must be TPC_F32 or TPC_BF16");
+  return TPC_OK;
+}
+
+template <class KernelT>
+cudaError_t set_smem(KernelT k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int C, int D, typename Tin, typename Tout>
+int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_io* io, void* ws, cudaStream_t st) {
+  using namespace tpc;
+  constexpr int DVT = D < 32 ? D : 32;
+  const int H = s->H;
+  const WsLayout L = ws_layout(p, H, C, D);
+  KdaWs w = ws_view(L, ws);
+  const int nc = (int)p.chunks.size();
+  TPC_CUDA(cudaMemsetAsync(w.status, 0, 4, st));
+  TPC_CUDA(set_smem(kda_fwd_prep<C, D, Tin>, fwd_prep_smem<C, D>()));
+  TPC_CUDA(set_smem(kda_fwd_scan<C, D, DVT>, scan_smem<C, D, DVT>()));
+  TPC_CUDA(set_smem(kda_fwd_out<C, D, Tin, Tout>, out_smem<C, D>()));
+  const Tin* q = static_cast<const Tin*>(io->q);
+  const Tin* k = static_cast<const Tin*>(io->k);
+  const Tin* v = static_cast<const Tin*>(io->v);
+  const Tin* g = static_cast<const Tin*>(io->g);
+  const Tin* b = static_cast<const Tin*>(io->beta);
+  TPC_LAUNCH("kda_fwd_prep", st,
+             (kda_fwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, fwd_prep_smem<C, D>(), st>>>(p.dt, H, k, v, g, b, w)));
+  for (int r = 1; r <= p.n_rounds; ++r) {
+    const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+    TPC_LAUNCH("kda_fwd_scan", st,
+               (kda_fwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads, scan_smem<C, D, DVT>(), st>>>(
+                   p.dt, s0, H, io->init_state, io->final_state, w)));
+  }
+  TPC_LAUNCH("kda_fwd_out", st,
+             (kda_fwd_out<C, D, Tin, Tout><<<dim3(nc, H), kThreads, out_smem<C, D>(), st>>>(
+                 p.dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
+  return TPC_OK;
+}
+
+template <int C, int D, typename Tin, typename Tout>
+int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_io* io, void* ws, cudaStream_t st) {
+  using namespace tpc;
+  constexpr int DVT = D < 32 ? D : 32;
+  const int H = s->H;
+  const WsLayout L = ws_layout(p, H, C, D);
+  KdaWs w = ws_view(L, ws);
+  const int nc = (int)p.chunks.size();
+  TPC_CUDA(set_smem(kda_bwd_prep<C, D, Tin>, bprep_smem<C, D>()));
+  TPC_CUDA(set_smem(kda_bwd_scan<C, D, DVT>, scan_smem<C, D, DVT>() + sizeof(float) * D * (DVT + 1)));
+  TPC_CUDA(set_smem(kda_bwd_dq<C, D, Tin, Tout>, bdq_smem<C, D>()));
+  TPC_CUDA(set_smem(kda_bwd_dkv<C, D, Tin, Tout>, bdkv_smem<C, D>()));
+  const Tin* q = static_cast<const Tin*>(io->q);
+  const Tin* k = static_cast<const Tin*>(io->k);
+  const Tin* v = static_cast<const Tin*>(io->v);
+  const Tin* g = static_cast<const Tin*>(io->g);
+  const Tin* b = static_cast<const Tin*>(io->beta);
+  const Tin* dO = static_cast<const Tin*>(io->d_o);
+  TPC_LAUNCH("kda_bwd_prep", st,
+             (kda_bwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, bprep_smem<C, D>(), st>>>(p.dt, H, q, k, g, dO, w)));
+  for (int r = p.n_rounds; r >= 1; --r) {
+    const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+    TPC_LAUNCH("kda_bwd_scan", st,
+               (kda_bwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads,
+                                          scan_smem<C, D, DVT>() + sizeof(float) * D * (DVT + 1), st>>>(
+                   p.dt, s0, H, io->d_final, w)));
+  }
+  TPC_LAUNCH("kda_bwd_dq", st,
+             (kda_bwd_dq<C, D, Tin, Tout><<<dim3(nc, H), kThreads, bdq_smem<C, D>(), st>>>(
+                 p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w)));
+  TPC_LAUNCH("kda_bwd_dkv", st,
+             (kda_bwd_dkv<C, D, Tin, Tout><<<dim3(nc, H), kThreads, bdkv_smem<C, D>(), st>>>(
+                 p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg, io->dbeta,
+                 w)));
+  if (!p.tgt_row.empty()) {
+    TPC_LAUNCH("kda_replay_reduce", st,
+               (kda_replay_reduce<D, Tout><<<dim3((unsigned)p.tgt_row.size(), H), 128, 0, st>>>(
+                   p.dt, H, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg, io->dbeta, w)));
+  }
+  if (io->d_init) {
+    TPC_LAUNCH("kda_init_reduce", st,
+               (kda_init_reduce<D><<<dim3((unsigned)p.roots.size(), H), 256, 0, st>>>(p.dt, H, io->d_init, w)));
+  }
+  return TPC_OK;
+}
+
+template <class F>
+int dispatch(const tpc_plan* plan, const tpc_kda_shape* s, F&& f) {
+  const int C = plan->p.C, D = s->dk;
+  const bool ib = s->in_dtype == TPC_BF16, ob = s->out_dtype == TPC_BF16;
+#define TPC_CASE(CC, DD)                                                                         \
+  if (C == CC && D == DD) {                                                                      \
+    if (ib && ob) return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{}, \
+                           __nv_bfloat16{}, __nv_bfloat16{});                                    \
+    if (ib) return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{},       \
+                     __nv_bfloat16{}, float{});                                                  \
+    if (ob) return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{},       \
+                     float{}, __nv_bfloat16{});                                                  \
+    return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{}, float{}, float{}); \
+  }
+  TPC_CASE(16, 32)
+  TPC_CASE(32, 64)
+  TPC_CASE(64, 128)
+#undef TPC_CASE
+  return fail(TPC_ERR_UNSUPPORTED, "unsupported (chunk, d)");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tpc_last_error(void) { return g_err.c_str(); }
+const char* tpc_version(void) { return "tpc 0.1 (sm_100a)"; }
+
+int tpc_plan_create(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, tpc_plan** out) {
+  if (!parent || !length || !out) return fail(TPC_ERR_NULL, "parent, length and out must be non-NULL");
+  *out = nullptr;
+  tpc_plan* p = new (std::nothrow) tpc_plan();
+  if (!p) return fail(TPC_ERR_CUDA, "out of host memory");
+  std::string err;
+  try {
+    err = tpc::build_plan(parent, length, n_nodes, chunk, p->p);
+  } catch (const std::exception& e) {
+    err = std::string("planner: ") + e.what();
+  }
+  if (!err.empty()) {
+    delete p;
+    const bool unsup = err.find("chunk size") != std::string::npos;
+    return fail(unsup ? TPC_ERR_UNSUPPORTED : TPC_ERR_INVALID_TREE, err);
+  }
+  *out = p;
+  return TPC_OK;
+}
+
+void tpc_plan_destroy(tpc_plan* plan) { delete plan; }
+
+int tpc_plan_get_info(const tpc_plan* plan, tpc_plan_info* info) {
+  if (!plan || !info) return fail(TPC_ERR_NULL, "plan or info is NULL");
+  const tpc::Plan& p = plan->p;
+  info->n_unique = p.n_unique;
+  info->n_expanded = p.n_expanded;
+  info->replay_total = p.replay_total;
+  info->n_seq_tokens = p.n_unique + p.replay_total;
+  info->n_nodes = p.n;
+  info->n_rounds = p.n_rounds;
+  info->n_seqs = (int32_t)p.seqs.size();
+  info->n_chunks = (int32_t)p.chunks.size();
+  info->n_slots = (int32_t)p.slots.size();
+  info->n_leaves = (int32_t)p.leaves.size();
+  info->n_roots = (int32_t)p.roots.size();
+  info->chunk = p.C;
+  info->max_seq_chunks = p.max_seq_chunks;
+  info->n_replay_targets = (int32_t)p.tgt_row.size();
+  return TPC_OK;
+}
+
+int tpc_plan_export(const tpc_plan* plan, tpc_plan_tables* t) {
+  if (!plan || !t) return fail(TPC_ERR_NULL, "plan or tables is NULL");
+  const tpc::Plan& p = plan->p;
+  auto cp = [](auto* dst, const auto& src) {
+    if (dst) for (size_t i = 0; i < src.size(); ++i) dst[i] = src[i];
+  };
+  cp(t->round, p.round);
+  cp(t->is_cont, p.is_cont);
+  cp(t->anchor, p.anchor);
+  cp(t->replay_start, p.replay_start);
+  cp(t->replay_len, p.replay_len);
+  cp(t->row_offset, p.row_offset);
+  cp(t->occurrence, p.occurrence);
+  cp(t->leaves, p.leaves);
+  cp(t->expanded_rows, p.exp_rows64);
+  cp(t->traj_offset, p.traj_offset);
+  return TPC_OK;
+}
+
+size_t tpc_plan_device_bytes(const tpc_plan* plan) {
+  if (!plan) return 0;
+  std::vector<size_t> off;
+  return tpc::device_layout(plan->p, off);
+}
+
+int tpc_plan_upload(tpc_plan* plan, void* dev, size_t bytes, tpc_stream_t stream) {
+  if (!plan || !dev) return fail(TPC_ERR_NULL, "plan or device buffer is NULL");
+  if (reinterpret_cast<uintptr_t>(dev) % 256) return fail(TPC_ERR_WORKSPACE, "device table buffer must be 256-byte aligned");
+  std::vector<size_t> off;
+  const size_t need = tpc::device_layout(plan->p, off);
+  if (bytes < need) return fail(TPC_ERR_WORKSPACE, "device table buffer too small");
+  std::vector<uint8_t> blob;
+  tpc::pack_device_blob(plan->p, off, blob);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TPC_CUDA(cudaMemcpyAsync(dev, blob.data(), need, cudaMemcpyHostToDevice, st));
+  // the pageable source is copied before cudaMemcpyAsync returns for host->device staging,
+  // but make it explicit so that `blob` can be released
+  TPC_CUDA(cudaStreamSynchronize(st));
+  plan->p.dev = dev;
+  plan->p.dev_bytes = bytes;
+  plan->p.blob_offsets = off;
+  plan->p.dt = tpc::device_view(plan->p, dev, off);
+  return TPC_OK;
+}
+
+size_t tpc_kda_workspace_bytes(const tpc_plan* plan, const tpc_kda_shape* s) {
+  if (!plan || !s || s->dk != s->dv || !shape_supported(plan->p.C, s->dk) || s->H < 1) return 0;
+  return ws_layout(plan->p, s->H, plan->p.C, s->dk).total;
+}
+
+int tpc_kda_forward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_fwd_io* io, void* ws, size_t ws_bytes,
+                    tpc_stream_t stream) {
+  if (int rc = check_shape(plan, s)) return rc;
+  if (!io || !io->q || !io->k || !io->v || !io->g || !io->beta || !io->o || !ws)
+    return fail(TPC_ERR_NULL, "forward: q, k, v, g, beta, o and ws are required");
+  if (ws_bytes < tpc_kda_workspace_bytes(plan, s)) return fail(TPC_ERR_WORKSPACE, "workspace too small");
+  if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(TPC_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout) {
+    return forward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout)>(plan->p, s, io, ws, st);
+  });
+}
+
+int tpc_kda_backward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_bwd_io* io, void* ws, size_t ws_bytes,
+                     tpc_stream_t stream) {
+  if (int rc = check_shape(plan, s)) return rc;
+  if (!io || !io->q || !io->k || !io->v || !io->g || !io->beta || !io->d_o || !io->dq || !io->dk || !io->dv ||
+      !io->dg || !io->dbeta || !ws)
+    return fail(TPC_ERR_NULL, "backward: inputs, d_o, gradient outputs and ws are required");
+  if (ws_bytes < tpc_kda_workspace_bytes(plan, s)) return fail(TPC_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout) {
+    return backward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout)>(plan->p, s, io, ws, st);
+  });
+}
+
+int tpc_status(const tpc_plan* plan, const tpc_kda_shape* s, void* ws, tpc_stream_t stream) {
+  if (!plan || !s || !ws) return fail(TPC_ERR_NULL, "plan, shape or ws is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int code = 0;
+  TPC_CUDA(cudaStreamSynchronize(st));
+  TPC_CUDA(cudaMemcpy(&code, ws, 4, cudaMemcpyDeviceToHost));
+  TPC_CUDA(cudaMemset(ws, 0, 4));
+  if (code == TPC_ERR_RANGE) return fail(TPC_ERR_RANGE, "gate decay inside a 16-row sub-block exceeds 80 (log units)");
+  if (code) return fail(TPC_ERR_DEVICE_CHECK, "kernel-side check failed with code " + std::to_string(code));
+  return TPC_OK;
+}
+
+int tpc_reduce_expanded_to_unique(const tpc_plan* plan, const float* x_exp, float* x_unique, int64_t width,
+                                  tpc_stream_t stream) {
+  if (!plan || !x_exp || !x_unique) return fail(TPC_ERR_NULL, "plan or buffers NULL");
+  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
+  if (width < 1) return fail(TPC_ERR_BAD_SHAPE, "width must be >= 1");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = plan->p.n_unique;
+  TPC_LAUNCH("reduce_expanded", st,
+             (tpc::reduce_expanded_kernel<<<(unsigned)N, 128, 0, st>>>(plan->p.dt, x_exp, x_unique, width)));
+  return TPC_OK;
+}
+
+int tpc_gather_expanded(const tpc_plan* plan, const void* x_unique, void* x_exp, int64_t width, int32_t elem_bytes,
+                        tpc_stream_t stream) {
+  if (!plan || !x_unique || !x_exp) return fail(TPC_ERR_NULL, "plan or buffers NULL");
+  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
+  if (width < 1 || (elem_bytes != 2 && elem_bytes != 4)) return fail(TPC_ERR_BAD_SHAPE, "width >= 1, elem_bytes 2 or 4");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t M = plan->p.n_expanded;
+  if (elem_bytes == 2)
+    TPC_LAUNCH("gather_expanded", st,
+               (tpc::gather_rows_kernel<uint16_t><<<(unsigned)M, 128, 0, st>>>(
+                   plan->p.dt, (const uint16_t*)x_unique, (uint16_t*)x_exp, width)));
+  else
+    TPC_LAUNCH("gather_expanded", st,
+               (tpc::gather_rows_kernel<uint32_t><<<(unsigned)M, 128, 0, st>>>(
+                   plan->p.dt, (const uint32_t*)x_unique, (uint32_t*)x_exp, width)));
+  return TPC_OK;
+}
+
+int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t stream) {
+  if (!plan || !counts) return fail(TPC_ERR_NULL, "plan or counts NULL");
+  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = plan->p.n_unique;
+  TPC_LAUNCH("occurrence_count", st,
+             (tpc::occurrence_count_kernel<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(plan->p.dt, counts, N)));
+  return TPC_OK;
+}
+
+void tpc_profile_enable(int on) { g_prof.on = on != 0; }
+
+long long tpc_launch_count(void) { return g_prof.launches; }
+
+int tpc_profile_read(char* buf, size_t len) {
+  if (!buf || len == 0) return fail(TPC_ERR_NULL, "buffer is NULL");
+  std::vector<std::pair<std::string, std::pair<long long, double>>> acc;
+  for (auto& r : g_prof.recs) {
+    TPC_CUDA(cudaEventSynchronize(r.b));
+    float ms = 0.f;
+    TPC_CUDA(cudaEventElapsedTime(&ms, r.a, r.b));
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+    bool found = false;
+    for (auto& e : acc)
+      if (e.first == r.name) { e.second.first++; e.second.second += ms; found = true; }
+    if (!found) acc.push_back({r.name, {1, (double)ms}});
+  }
+  g_prof.recs.clear();
+  std::string out;
+  for (auto& e : acc) out += e.first + " " + std::to_string(e.second.first) + " " + std::to_string(e.second.second) + "\n";
+  std::snprintf(buf, len, "%s", out.c_str());
+  return TPC_OK;
+}
+
+}  // extern "C"
