@@ -194,7 +194,7 @@ def cpu_threads():
 
 
 def run_reference(args, ws, rank):
-    w = synth.workload(WORKLOAD)
+    w = synth.workload(args.workload)
     if rank != 0:
         return
     n_tok = args.ref_tokens
@@ -230,6 +230,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-expanded", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, help="single_fork (default), agentic, agentic_small")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "tpc" else args.warmup
 
@@ -243,7 +244,7 @@ def main():
     import tree_packed_chunkwise_b200 as tpc
 
     world, rank, local = setup_dist()
-    w = synth.workload(WORKLOAD)
+    w = synth.workload(args.workload)
     t = w.tree
     seed = w.seed + 1000 * rank
     plan = tpc.Plan(t.parent, t.length, w.chunk).upload()
