@@ -215,6 +215,32 @@ int tpc_gather_expanded(const tpc_plan* plan, const void* x_unique, void* x_exp,
 /* Occurrence count per compact row (int32 [N]). */
 int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t stream);
 
+/* ------------------------------------------------------------------ allocation-free forward */
+/* Bytes of device scratch built into the library for tpc_kda_forward_static (64 MiB). */
+#define TPC_STATIC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * tpc_kda_forward with no device allocation at all (the HARTS pages have no counterpart; this is
+ * a deployment convenience).  It is for callers that may not allocate device memory themselves:
+ * code running inside a host runtime whose own pool owns the whole device, or a latency-critical
+ * path that must not pay the device-wide synchronisation a fresh cudaMalloc can cause.  The plan
+ * tables and the forward workspace go into one device array of TPC_STATIC_SCRATCH_BYTES that is
+ * compiled into this library, so every GPU that loads the library holds those bytes until the
+ * process exits.  The plan does not need tpc_plan_upload for this call.
+ *   io: as tpc_kda_forward (caller-owned inputs and outputs); the call allocates nothing and calls
+ *       no allocating routine.
+ *   Sizes: problems whose tables + workspace exceed TPC_STATIC_SCRATCH_BYTES are rejected with
+ *       TPC_ERR_WORKSPACE and a message giving the bytes needed.
+ *   Set-up: the first call on a device looks up the array's device address (with that device
+ *       current); make that first call before any stream capture.
+ *   Sharing: every call uses the same array and it keeps the previous call's contents; the call
+ *       clears its status word itself.  Calls that overlap on the GPU (other streams, other host
+ *       threads) race on the array: serialise them.  tpc_kda_backward cannot follow this call (the
+ *       workspace it needs is not kept).
+ */
+int tpc_kda_forward_static(const tpc_plan* plan, const tpc_kda_shape* shape, const tpc_kda_fwd_io* io,
+                           tpc_stream_t stream);
+
 /* ------------------------------------------------------------------ diagnostics */
 /* Per-kernel timing: when enabled, every launch is bracketed by CUDA events recorded on
  * its stream (adds a few microseconds per launch).  Not thread safe. */

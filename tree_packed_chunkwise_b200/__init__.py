@@ -81,6 +81,7 @@ SIGNATURES = {
     "tpc_reduce_expanded_to_unique": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, _V]),
     "tpc_gather_expanded": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int32, _V]),
     "tpc_occurrence_counts": (ctypes.c_int, [_V, _V, _V]),
+    "tpc_kda_forward_static": (ctypes.c_int, [_V, _P(KdaShape), _P(KdaFwdIO), _V]),
     "tpc_profile_enable": (None, [ctypes.c_int]),
     "tpc_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t]),
     "tpc_launch_count": (ctypes.c_longlong, []),
@@ -219,6 +220,25 @@ def tpc_kda_forward(plan: Plan, q, k, v, g, beta, init_state=None, out_dtype=Non
     _check(lib().tpc_kda_forward(plan.handle, ctypes.byref(shape), ctypes.byref(io), _ptr(ws), ws.numel(),
                                  _stream_ptr(stream)))
     return o, final_state, ws
+
+
+def tpc_kda_forward_static(plan: Plan, q, k, v, g, beta, init_state=None, out_dtype=None, o=None,
+                           final_state=None, want_final=True, stream=None):
+    """Forward that allocates nothing on the device: tables and workspace live in the library's
+    built-in scratch array (see include/tpc.h).  Returns (o, final_state)."""
+    import torch
+    N, H, d = q.shape
+    out_dtype = out_dtype or q.dtype
+    shape = kda_shape(H, d, _dtype_code(q), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
+    if o is None:
+        o = torch.empty(N, H, d, dtype=out_dtype, device=q.device)
+    if final_state is None and want_final:
+        final_state = torch.empty(plan.info["n_leaves"], H, d, d, dtype=torch.float32, device=q.device)
+    io = KdaFwdIO(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
+                  None if init_state is None else init_state.data_ptr(), o.data_ptr(),
+                  None if final_state is None else final_state.data_ptr())
+    _check(lib().tpc_kda_forward_static(plan.handle, ctypes.byref(shape), ctypes.byref(io), _stream_ptr(stream)))
+    return o, final_state
 
 
 def tpc_kda_backward(plan: Plan, ws, q, k, v, g, beta, d_o, d_final=None, init_state=None, out_dtype=None,

@@ -3,6 +3,7 @@
 
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -223,6 +224,69 @@ int dispatch(const tpc_plan* plan, const tpc_kda_shape* s, F&& f) {
   return fail(TPC_ERR_UNSUPPORTED, "unsupported (chunk, d)");
 }
 
+// ------------------------------------------------------------------------------------------------
+// Allocation-free forward (tpc_kda_forward_static).  Its plan tables and workspace live in one
+// file-scope device array, so a caller that may not allocate device memory can still run the
+// forward pass.  Host code must not pass the array's name to a kernel: in host code that name is a
+// host-side stand-in, not a device address.  The device address is looked up once per device with
+// cudaGetSymbolAddress and cached.
+static __device__ __align__(256) unsigned char g_static_scratch[TPC_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void* g_static_ptr[kMaxDevices] = {};
+cudaError_t g_static_rc[kMaxDevices] = {};
+std::once_flag g_static_once[kMaxDevices];
+
+// forward-only workspace: status word, W, U, Khat, decay, S0 and slot states
+size_t static_ws_layout(const tpc::Plan& p, int H, int C, int D, size_t base, tpc::KdaWs* w, char* dev) {
+  size_t o = base;
+  auto take = [&](size_t bytes) { size_t r = o; o += a256(bytes); return r; };
+  const size_t nc = p.chunks.size(), cd = (size_t)C * D, dd = (size_t)D * D;
+  const size_t st = take(256), W = take(nc * H * cd * 4), U = take(nc * H * cd * 4), K = take(nc * H * cd * 4);
+  const size_t dec = take(nc * H * D * 4), S0 = take(nc * H * dd * 4), sl = take(p.slots.size() * H * dd * 4);
+  if (w && dev) {
+    *w = tpc::KdaWs{};
+    w->status = reinterpret_cast<int*>(dev + st);
+    w->W = reinterpret_cast<float*>(dev + W);
+    w->U = reinterpret_cast<float*>(dev + U);
+    w->Khat = reinterpret_cast<float*>(dev + K);
+    w->decay = reinterpret_cast<float*>(dev + dec);
+    w->S0 = reinterpret_cast<float*>(dev + S0);
+    w->slot = reinterpret_cast<float*>(dev + sl);
+  }
+  return o;
+}
+
+template <int C, int D, typename Tin, typename Tout>
+int forward_static_impl(const tpc::Plan& p, const tpc::DevTables& dt, tpc::KdaWs w, const tpc_kda_shape* s,
+                        const tpc_kda_fwd_io* io, cudaStream_t st) {
+  using namespace tpc;
+  constexpr int DVT = D < 32 ? D : 32;
+  const int H = s->H;
+  const int nc = (int)p.chunks.size();
+  TPC_CUDA(cudaMemsetAsync(w.status, 0, 4, st));  // the array keeps the previous call's contents
+  TPC_CUDA(set_smem(kda_fwd_prep<C, D, Tin>, fwd_prep_smem<C, D>()));
+  TPC_CUDA(set_smem(kda_fwd_scan<C, D, DVT>, scan_smem<C, D, DVT>()));
+  TPC_CUDA(set_smem(kda_fwd_out<C, D, Tin, Tout>, out_smem<C, D>()));
+  const Tin* q = static_cast<const Tin*>(io->q);
+  const Tin* k = static_cast<const Tin*>(io->k);
+  const Tin* v = static_cast<const Tin*>(io->v);
+  const Tin* g = static_cast<const Tin*>(io->g);
+  const Tin* b = static_cast<const Tin*>(io->beta);
+  TPC_LAUNCH("kda_fwd_prep", st,
+             (kda_fwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, fwd_prep_smem<C, D>(), st>>>(dt, H, k, v, g, b, w)));
+  for (int r = 1; r <= p.n_rounds; ++r) {
+    const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+    TPC_LAUNCH("kda_fwd_scan", st,
+               (kda_fwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads, scan_smem<C, D, DVT>(), st>>>(
+                   dt, s0, H, io->init_state, io->final_state, w)));
+  }
+  TPC_LAUNCH("kda_fwd_out", st,
+             (kda_fwd_out<C, D, Tin, Tout><<<dim3(nc, H), kThreads, out_smem<C, D>(), st>>>(
+                 dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
+  return TPC_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -423,6 +487,46 @@ int tpc_profile_read(char* buf, size_t len) {
   for (auto& e : acc) out += e.first + " " + std::to_string(e.second.first) + " " + std::to_string(e.second.second) + "\n";
   std::snprintf(buf, len, "%s", out.c_str());
   return TPC_OK;
+}
+
+int tpc_kda_forward_static(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_fwd_io* io,
+                           tpc_stream_t stream) {
+  if (!plan || !s) return fail(TPC_ERR_NULL, "plan or shape is NULL");
+  if (s->H < 1 || s->dk != s->dv) return fail(TPC_ERR_BAD_SHAPE, "H >= 1 and dk == dv required");
+  if (!shape_supported(plan->p.C, s->dk)) return fail(TPC_ERR_UNSUPPORTED, "unsupported (chunk, d)");
+  if ((s->in_dtype != TPC_F32 && s->in_dtype != TPC_BF16) || (s->out_dtype != TPC_F32 && s->out_dtype != TPC_BF16))
+    return fail(TPC_ERR_UNSUPPORTED, "dtype must be TPC_F32 or TPC_BF16");
+  if (!io || !io->q || !io->k || !io->v || !io->g || !io->beta || !io->o)
+    return fail(TPC_ERR_NULL, "forward: q, k, v, g, beta and o are required");
+  const tpc::Plan& p = plan->p;
+  std::vector<size_t> off;
+  const size_t table_bytes = tpc::device_layout(p, off);
+  const size_t need = static_ws_layout(p, s->H, p.C, s->dk, a256(table_bytes), nullptr, nullptr);
+  if (need > (size_t)TPC_STATIC_SCRATCH_BYTES)
+    return fail(TPC_ERR_WORKSPACE, "problem needs " + std::to_string(need) + " bytes of device scratch; the "
+                "allocation-free forward holds at most " + std::to_string((size_t)TPC_STATIC_SCRATCH_BYTES));
+  int dev = 0;
+  TPC_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(TPC_ERR_UNSUPPORTED, "device ordinal out of range");
+  // once per device, with that device current: the device address of the scratch array
+  std::call_once(g_static_once[dev], [dev] {
+    g_static_rc[dev] = cudaGetSymbolAddress(&g_static_ptr[dev], g_static_scratch);
+  });
+  if (g_static_rc[dev] != cudaSuccess || !g_static_ptr[dev])
+    return fail(TPC_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(g_static_rc[dev]));
+  char* base = static_cast<char*>(g_static_ptr[dev]);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // plan tables at the start of the array (pageable source: staged before cudaMemcpyAsync returns)
+  std::vector<uint8_t> blob;
+  tpc::pack_device_blob(p, off, blob);
+  TPC_CUDA(cudaMemcpyAsync(base, blob.data(), table_bytes, cudaMemcpyHostToDevice, st));
+  const tpc::DevTables dt = tpc::device_view(p, base, off);
+  tpc::KdaWs w;
+  static_ws_layout(p, s->H, p.C, s->dk, a256(table_bytes), &w, base);
+  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout) {
+    return forward_static_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout)>(p, dt, w, s, io,
+                                                                                                        st);
+  });
 }
 
 }  // extern "C"
