@@ -1,0 +1,709 @@
+// Tensor-core (tcgen05) per-chunk kernels of the tree-packed chunkwise KDA path, chunk C = 64,
+// head dim D = 128.
+//
+// Every contraction of the chunkwise form runs on the 5th-generation tensor cores with fp32
+// accumulators in TMEM.  Operands that are not raw bf16 inputs (gated keys, the WY factors, the
+// state, U, P ...) carry ~16 significant bits as a bf16 pair x = hi + lo, and a product of two such
+// operands is hi*hi + lo*hi + hi*lo (three MMA chains into one accumulator); against a raw bf16
+// input two chains suffice.  Single-pass bf16 or fp16 operands miss the 2e-3 max-error bound.
+//
+// The intra-chunk gated products gated(a, b)_ri = sum_c a_rc b_ic e^{G_rc - G_ic} use the chunk's
+// first row as the reference of every channel: a_rc e^{G_rc - G_0c} (<= 1) and b_ic e^{G_0c - G_ic}
+// (>= 1) are single dense operands.  The reference is causal: nothing computed for row r depends on
+// a later row of the chunk, so a row shared by several trajectories gets the same bits whether its
+// chunk continues into one branch or another (each trajectory keeps its chunkwise numerical path).
+// Factors stay within e^{+-80} while a channel decays by at most kMaxChunkDecay over one chunk
+// (checked; TPC_ERR_RANGE otherwise).
+#pragma once
+#include <type_traits>
+
+#include "kda_kernels.cuh"
+#include "tc.cuh"
+
+namespace tpc {
+
+constexpr int kTcC = 64, kTcD = 128;
+constexpr float kMaxChunkDecay = 80.f;  // G_first - G_last per channel over one chunk
+enum : int { kStatusTimeout = 8 };
+
+namespace tck {
+
+using namespace tc;
+
+// A x B tile (b contiguous) of bf16 hi (and lo) values val(a, b); 16-byte stores, one 8-wide
+// chunk of b per thread and step; neighbouring threads take neighbouring a (conflict-free).
+template <int A, int B, bool SPLIT, class F>
+__device__ __forceinline__ void build_tile(uint8_t* hi, uint8_t* lo, F val) {
+  for (int e = threadIdx.x; e < A * (B / 8); e += blockDim.x) {
+    const int a = e % A, b0 = (e / A) * 8;
+    __align__(16) __nv_bfloat16 h[8];
+    __align__(16) __nv_bfloat16 l[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x = val(a, b0 + j);
+      if (SPLIT) split_bf16(x, h[j], l[j]);
+      else h[j] = __float2bfloat16_rn(x);
+    }
+    *reinterpret_cast<uint4*>(hi + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(h);
+    if (SPLIT) *reinterpret_cast<uint4*>(lo + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(l);
+  }
+}
+
+// Reads an M x N fp32 accumulator (N a multiple of 32) starting at TMEM column col0:
+// f(m, n0, v) gets 16 consecutive columns n0 .. n0+15 of row m.  Warp w reads the lanes of
+// sub-partition w % 4; the two groups of four warps take alternating 16-column chunks.
+template <int M, int N, class F>
+__device__ __forceinline__ void acc_read(uint32_t tbase, int col0, F f) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, sp = w & 3, grp = (w >> 2) & 1;
+  for (int c = grp * 16; c < N; c += 32) {
+    float v[16];
+    tmem_ld16(tbase + ((uint32_t)(32 * sp) << 16) + (uint32_t)(col0 + c), v);
+    const int m = (M == 128) ? 32 * sp + lane : (lane < 16 ? 16 * sp + lane : -1);
+    if (m >= 0) f(m, c, v);
+  }
+}
+
+// Writes 16 values (one row chunk) into a K-major/MN-major tile as bf16 hi/lo at (a, b0..b0+15).
+template <int A, bool SPLIT>
+__device__ __forceinline__ void put16(uint8_t* hi, uint8_t* lo, int a, int b0, const float* v) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    __align__(16) __nv_bfloat16 h[8];
+    __align__(16) __nv_bfloat16 l[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (SPLIT) split_bf16(v[8 * half + j], h[j], l[j]);
+      else h[j] = __float2bfloat16_rn(v[8 * half + j]);
+    }
+    *reinterpret_cast<uint4*>(hi + cm_off(a, b0 + 8 * half, A)) = *reinterpret_cast<const uint4*>(h);
+    if (SPLIT) *reinterpret_cast<uint4*>(lo + cm_off(a, b0 + 8 * half, A)) = *reinterpret_cast<const uint4*>(l);
+  }
+}
+
+struct Sync {
+  uint64_t* bar;
+  uint32_t phase;
+  int* status;
+};
+
+// Makes the threads' shared-memory writes visible to the tensor core, lets thread 0 issue the
+// MMAs and commit, and waits (bounded) for their completion.  Returns false on every thread if
+// any thread's wait ran out (CTA-wide vote), after recording TPC_ERR_TIMEOUT.
+template <class F>
+__device__ __forceinline__ bool run(Sync& s, F issue) {
+  fence_async_smem();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (threadIdx.x == 0) {
+    issue();
+    commit(s.bar);
+  }
+  const bool ok = mbar_wait(s.bar, s.phase);
+  const int failed = __syncthreads_or(ok ? 0 : 1);
+  if (failed) {
+    if (threadIdx.x == 0) set_status(s.status, kStatusTimeout);
+    mbar_wait(s.bar, s.phase, 200000000ull);  // give MMAs still in flight a last bounded chance
+    return false;
+  }
+  s.phase ^= 1u;
+  fence_after_sync();
+  return true;
+}
+
+// three chains: hi*hi + lo*hi + hi*lo (both operands split) or two (b exact: lo of b absent)
+__device__ __forceinline__ void mma3(uint32_t d, const Op& ah, const Op& al, const Op& bh, const Op& bl, int K,
+                                     uint32_t id, bool acc, bool b_exact) {
+  mma_chain(d, ah, bh, K, id, acc);
+  mma_chain(d, al, bh, K, id, true);
+  if (!b_exact) mma_chain(d, ah, bl, K, id, true);
+}
+
+// hi/lo product with either operand possibly exact (its lo part is zero and skipped)
+__device__ __forceinline__ void mma4(uint32_t d, const Op& ah, const Op& al, const Op& bh, const Op& bl, int K,
+                                     uint32_t id, bool acc, bool a_exact, bool b_exact) {
+  mma_chain(d, ah, bh, K, id, acc);
+  if (!a_exact) mma_chain(d, al, bh, K, id, true);
+  if (!b_exact) mma_chain(d, ah, bl, K, id, true);
+}
+
+// T = (I + L)^{-1} for strictly lower-triangular L (64 x 64, pitch LC), fp32, in smem.
+// Diagonal 16 x 16 blocks: (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) (N^16 = 0);
+// off-diagonal blocks: T_pq = -T_pp sum_{q <= s < p} L_ps T_sq, by increasing p - q.
+// W1, W2: 4 scratch 16 x 16 blocks each (pitch 17).
+template <int LC>
+__device__ __forceinline__ void block_inverse(float* T, const float* L, float* W1, float* W2) {
+  constexpr int B = 16, P = 17, BB = B * P;
+  const int tid = threadIdx.x;
+  // diagonal blocks, all four at once: element e -> (block, row, col)
+  auto blk = [&](int e, int& p, int& r, int& c) { p = e >> 8; r = (e >> 4) & 15; c = e & 15; };
+  // W1_p = N_p (strict lower), T_pp = I - N_p
+  for (int e = tid; e < 4 * 256; e += blockDim.x) {
+    int p, r, c;
+    blk(e, p, r, c);
+    const float n = (c < r) ? L[(16 * p + r) * LC + 16 * p + c] : 0.f;
+    W1[p * BB + r * P + c] = n;
+    T[(16 * p + r) * LC + 16 * p + c] = (r == c ? 1.f : 0.f) - n;
+  }
+  __syncthreads();
+  for (int level = 0; level < 3; ++level) {
+    // W2 = W1 * W1  (N^2, N^4, N^8)
+    for (int e = tid; e < 4 * 256; e += blockDim.x) {
+      int p, r, c;
+      blk(e, p, r, c);
+      float acc = 0.f;
+      for (int k = c + 1; k < r; ++k) acc = fmaf(W1[p * BB + r * P + k], W1[p * BB + k * P + c], acc);
+      W2[p * BB + r * P + c] = acc;
+    }
+    __syncthreads();
+    // T_pp <- T_pp (I + W2): row r of T times (I + W2)
+    float out[4];
+    int cnt = 0;
+    for (int e = tid; e < 4 * 256; e += blockDim.x, ++cnt) {
+      int p, r, c;
+      blk(e, p, r, c);
+      float acc = T[(16 * p + r) * LC + 16 * p + c];
+      for (int k = c + 1; k <= r; ++k) acc = fmaf(T[(16 * p + r) * LC + 16 * p + k], W2[p * BB + k * P + c], acc);
+      out[cnt] = acc;
+    }
+    __syncthreads();
+    cnt = 0;
+    for (int e = tid; e < 4 * 256; e += blockDim.x, ++cnt) {
+      int p, r, c;
+      blk(e, p, r, c);
+      T[(16 * p + r) * LC + 16 * p + c] = out[cnt];
+    }
+    for (int e = tid; e < 4 * 256; e += blockDim.x) {
+      int p, r, c;
+      blk(e, p, r, c);
+      W1[p * BB + r * P + c] = W2[p * BB + r * P + c];
+    }
+    __syncthreads();
+  }
+  // off-diagonal blocks by distance d = p - q: T_pq = -T_pp * (sum_s L_ps T_sq)
+  for (int d = 1; d < 4; ++d) {
+    const int nb = 4 - d;  // blocks (p, p - d), p = d .. 3
+    // W1[j] = sum_{s=q}^{p-1} L_ps T_sq
+    for (int e = tid; e < nb * 256; e += blockDim.x) {
+      const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+      const int p = d + j, q = j;
+      float acc = 0.f;
+      for (int s = q; s < p; ++s)
+        for (int k = 0; k < 16; ++k)
+          acc = fmaf(L[(16 * p + r) * LC + 16 * s + k], T[(16 * s + k) * LC + 16 * q + c], acc);
+      W1[j * BB + r * P + c] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < nb * 256; e += blockDim.x) {
+      const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+      const int p = d + j, q = j;
+      float acc = 0.f;
+      for (int k = 0; k <= r; ++k) acc = fmaf(T[(16 * p + r) * LC + 16 * p + k], W1[j * BB + k * P + c], acc);
+      T[(16 * p + r) * LC + 16 * q + c] = -acc;
+    }
+    __syncthreads();
+  }
+  // upper blocks are zero
+  for (int e = tid; e < 64 * 64; e += blockDim.x) {
+    const int r = e >> 6, c = e & 63;
+    if ((c >> 4) > (r >> 4)) T[r * LC + c] = 0.f;
+  }
+  __syncthreads();
+}
+
+// G <- inclusive cumulative gate over the chunk's rows (rows >= n repeat row n - 1); the reference
+// (row 0) goes to ref[c].  Flags TPC_ERR_RANGE when a channel decays by more than kMaxChunkDecay.
+__device__ __forceinline__ void cumsum_ref(float* G, int LD, int n, float* ref, int* status) {
+  for (int c = threadIdx.x; c < kTcD; c += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < kTcC; ++i) {
+      if (i < n) acc += G[i * LD + c];
+      G[i * LD + c] = acc;
+    }
+    ref[c] = G[c];
+    if (status && !(G[c] - G[(n - 1) * LD + c] <= kMaxChunkDecay)) set_status(status, kStatusRange);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_in(const T* base, const int* rows, int H, int h, int n, int r, int c) {
+  return r < n ? to_f(base[((size_t)rows[r] * H + h) * kTcD + c]) : 0.f;
+}
+
+}  // namespace tck
+
+// --------------------------------------------------------------------------------- forward prep
+// per (chunk, head): Atilde = gated(k, k) (strict lower), T = (I + diag(beta) Atilde)^{-1},
+// W = T diag(beta) Kbar, U' = T diag(beta) V, Khat = k e^{G_C - G}, decay = e^{G_C}.
+struct PrepTcSmem {
+  static constexpr int C = kTcC, D = kTcD, LD = D + 1, LC = C + 1;
+  static constexpr size_t G = 0;
+  static constexpr size_t A = G + sizeof(float) * C * LD;
+  static constexpr size_t T = A + sizeof(float) * C * LC;
+  static constexpr size_t W1 = T + sizeof(float) * C * LC;
+  static constexpr size_t W2 = W1 + sizeof(float) * 4 * 16 * 17;
+  static constexpr size_t vec = W2 + sizeof(float) * 4 * 16 * 17;       // beta[C], ref[D], gC[D]
+  static constexpr size_t tiles = (vec + sizeof(float) * (C + 2 * D) + 1023) & ~size_t(1023);
+  // phase 1: af hi/lo, bf hi/lo (C x D each); phase 2: T' hi/lo (C x C), Kbar hi/lo, V hi/lo (C x D)
+  static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2;
+  static constexpr size_t total = tiles + 2 * CCb + 4 * CDb;
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads, 1)
+    kda_fwd_prep_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
+                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, KdaWs ws) {
+  using namespace tck;
+  using S = PrepTcSmem;
+  constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
+  constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
+  const int ci = blockIdx.x, h = blockIdx.y;
+  const ChunkRec ch = t.chunks[ci];
+  const int n = ch.n_rows;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  float* sG = reinterpret_cast<float*>(tsm + S::G);
+  float* sA = reinterpret_cast<float*>(tsm + S::A);
+  float* sT = reinterpret_cast<float*>(tsm + S::T);
+  float* sW1 = reinterpret_cast<float*>(tsm + S::W1);
+  float* sW2 = reinterpret_cast<float*>(tsm + S::W2);
+  float* sb = reinterpret_cast<float*>(tsm + S::vec);
+  float* sref = sb + C;
+  uint8_t* tl = tsm + S::tiles;
+  __shared__ int srow[C];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < C; i += blockDim.x) {
+    srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
+  }
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
+  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  __syncthreads();
+  cumsum_ref(sG, LD, n, sref, ws.status);
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  Sync sy{&bar, 0u, ws.status};
+  bool ok = true;
+  // phase 1: Atilde = af bf^T with af = k e^{G - ref}, bf = k e^{ref - G}
+  {
+    uint8_t *afh = tl, *afl = tl + S::CDb, *bfh = tl + 2 * S::CDb, *bfl = tl + 3 * S::CDb;
+    build_tile<C, D, true>(afh, afl, [&](int r, int c) {
+      return ld_in(k_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
+    });
+    build_tile<C, D, true>(bfh, bfl, [&](int i, int c) {
+      return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
+    });
+    const tc::Op ah{tc::smem_u32(afh), C, false}, al{tc::smem_u32(afl), C, false};
+    const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
+    ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
+    if (ok) {
+      acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
+        for (int j = 0; j < 16; ++j) {
+          const int i = i0 + j;
+          sA[r * LC + i] = (i < r) ? sb[r] * v[j] : 0.f;  // L = diag(beta) Atilde, strict lower
+        }
+      });
+    }
+  }
+  if (ok) {
+    __syncthreads();
+    block_inverse<LC>(sT, sA, sW1, sW2);
+    // phase 2: W = T' Kbar and U' = T' V with T' = T diag(beta)
+    uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
+            *vl = vh + S::CDb;
+    build_tile<C, C, true>(th, tlo, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
+    build_tile<C, D, true>(kh, kl, [&](int i, int c) {
+      return ld_in(k_, srow, H, h, n, i, c) * expf(sG[i * LD + c]);
+    });
+    build_tile<C, D, !EX>(vh, vl, [&](int i, int c) { return ld_in(v_, srow, H, h, n, i, c); });
+    const tc::Op tH{tc::smem_u32(th), C, false}, tL{tc::smem_u32(tlo), C, false};
+    const tc::Op kH{tc::smem_u32(kh), C, true}, kL{tc::smem_u32(kl), C, true};
+    const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
+    const uint32_t id = tc::idesc_bf16(C, D, false, true);
+    ok = run(sy, [&] {
+      mma3(tb + 64, tH, tL, kH, kL, C, id, false, false);
+      mma3(tb + 192, tH, tL, vH, vL, C, id, false, EX);
+    });
+    if (ok) {
+      const size_t base = (size_t)ci * H + h;
+      float* W = ws.W + base * C * D;
+      float* U = ws.U + base * C * D;
+      acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) {
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(W + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      });
+      acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) {
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(U + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      });
+      float* Kh = ws.Khat + base * C * D;
+      for (int e = tid; e < C * D; e += blockDim.x) {
+        const int i = e / D, c = e % D;
+        Kh[e] = ld_in(k_, srow, H, h, n, i, c) * expf(sG[(n - 1) * LD + c] - sG[i * LD + c]);
+      }
+      for (int c = tid; c < D; c += blockDim.x) ws.decay[base * D + c] = expf(sG[(n - 1) * LD + c]);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
+}
+
+// --------------------------------------------------------------------------------- forward output
+// per (chunk, head): P = lower_incl(gated(q, k)), O = Qbar S0 + P U (own rows only)
+struct OutTcSmem {
+  static constexpr int C = kTcC, D = kTcD, LD = D + 1;
+  static constexpr size_t G = 0;
+  static constexpr size_t vec = G + sizeof(float) * C * LD;  // ref[D]
+  static constexpr size_t tiles = (vec + sizeof(float) * D + 1023) & ~size_t(1023);
+  static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2, DDb = size_t(D) * D * 2;
+  // region R (4 CDb): phase 1 qf hi/lo + bf hi/lo; phase 2: P hi/lo (2 CCb) + U hi/lo (2 CDb)
+  static constexpr size_t R = tiles;
+  static constexpr size_t Qb = R + 4 * CDb;     // Qbar hi/lo
+  static constexpr size_t S0 = Qb + 2 * CDb;    // S0 hi/lo (D x D)
+  static constexpr size_t total = S0 + 2 * DDb;
+};
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads, 1)
+    kda_fwd_out_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
+                   const Tin* __restrict__ g_, Tout* __restrict__ o_, KdaWs ws) {
+  using namespace tck;
+  using S = OutTcSmem;
+  constexpr int C = S::C, D = S::D, LD = S::LD;
+  const int ci = blockIdx.x, h = blockIdx.y;
+  const ChunkRec ch = t.chunks[ci];
+  const int n = ch.n_rows;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  float* sG = reinterpret_cast<float*>(tsm + S::G);
+  float* sref = reinterpret_cast<float*>(tsm + S::vec);
+  __shared__ int srow[C];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 256);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  __syncthreads();
+  cumsum_ref(sG, LD, n, sref, nullptr);
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  Sync sy{&bar, 0u, ws.status};
+  const size_t base = (size_t)ci * H + h;
+  uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
+  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *s0h = tsm + S::S0, *s0l = s0h + S::DDb;
+  build_tile<C, D, true>(qfh, qfl, [&](int r, int c) {
+    return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
+  });
+  build_tile<C, D, true>(bfh, bfl, [&](int i, int c) {
+    return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
+  });
+  build_tile<C, D, true>(qbh, qbl, [&](int r, int c) { return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c]); });
+  const float* S0g = ws.S0 + base * D * D;
+  build_tile<D, D, true>(s0h, s0l, [&](int c, int j) { return S0g[c * D + j]; });
+  bool ok = run(sy, [&] {
+    const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
+    const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
+    mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false);
+  });
+  if (ok) {
+    uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
+    acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
+      float m[16];
+      for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+      put16<C, true>(ph, pl, r, i0, m);
+    });
+    const float* Ug = ws.U + base * C * D;
+    build_tile<C, D, true>(uh, ul, [&](int i, int j) { return Ug[i * D + j]; });
+    ok = run(sy, [&] {
+      const uint32_t id = tc::idesc_bf16(C, D, false, true);
+      const tc::Op qH{tc::smem_u32(qbh), C, false}, qL{tc::smem_u32(qbl), C, false};
+      const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
+      const tc::Op pH{tc::smem_u32(ph), C, false}, pL{tc::smem_u32(pl), C, false};
+      const tc::Op uH{tc::smem_u32(uh), C, true}, uL{tc::smem_u32(ul), C, true};
+      mma3(tb + 64, qH, qL, sH, sL, D, id, false, false);
+      mma3(tb + 64, pH, pL, uH, uL, C, id, true, false);
+    });
+    if (ok) {
+      acc_read<C, D>(tb, 64, [&](int r, int j0, const float* v) {
+        if (r >= ch.n_replay && r < n) {
+          Tout* dst = o_ + ((size_t)srow[r] * H + h) * D + j0;
+          for (int j = 0; j < 16; ++j) dst[j] = from_f<Tout>(v[j]);
+        }
+      });
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 256);
+}
+
+}  // namespace tpc
+
+namespace tpc {
+
+// --------------------------------------------------------------------------------- backward prep
+// per (chunk, head): dU0 = P^T dO and X = Qbar^T dO - W^T dU0 (the state-independent parts of the
+// reverse scan).  dO rows of replayed rows are zero.
+struct BprepTcSmem {
+  static constexpr int C = kTcC, D = kTcD, LD = D + 1;
+  static constexpr size_t G = 0;
+  static constexpr size_t vec = G + sizeof(float) * C * LD;
+  static constexpr size_t tiles = (vec + sizeof(float) * D + 1023) & ~size_t(1023);
+  static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2;
+  static constexpr size_t R = tiles;             // qf, bf (4 CDb) -> P (2 CCb) + dU0 (2 CDb)
+  static constexpr size_t Qb = R + 4 * CDb;      // Qbar, MN-major
+  static constexpr size_t dO = Qb + 2 * CDb;     // dO, MN-major
+  static constexpr size_t Wt = dO + 2 * CDb;     // -W, MN-major
+  static constexpr size_t total = Wt + 2 * CDb;
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads, 1)
+    kda_bwd_prep_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
+                    const Tin* __restrict__ g_, const Tin* __restrict__ do_, KdaWs ws) {
+  using namespace tck;
+  using S = BprepTcSmem;
+  constexpr int C = S::C, D = S::D, LD = S::LD;
+  constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
+  const int ci = blockIdx.x, h = blockIdx.y;
+  const ChunkRec ch = t.chunks[ci];
+  const int n = ch.n_rows;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  float* sG = reinterpret_cast<float*>(tsm + S::G);
+  float* sref = reinterpret_cast<float*>(tsm + S::vec);
+  __shared__ int srow[C];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  __syncthreads();
+  cumsum_ref(sG, LD, n, sref, nullptr);
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  Sync sy{&bar, 0u, ws.status};
+  const size_t base = (size_t)ci * H + h;
+  uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
+  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *doh = tsm + S::dO, *dol = doh + S::CDb;
+  uint8_t *wh = tsm + S::Wt, *wl = wh + S::CDb;
+  build_tile<C, D, true>(qfh, qfl, [&](int r, int c) {
+    return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
+  });
+  build_tile<C, D, true>(bfh, bfl, [&](int i, int c) {
+    return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
+  });
+  build_tile<C, D, true>(qbh, qbl, [&](int r, int c) { return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c]); });
+  build_tile<C, D, !EX>(doh, dol, [&](int r, int j) {
+    return r >= ch.n_replay ? ld_in(do_, srow, H, h, n, r, j) : 0.f;
+  });
+  const float* Wg = ws.W + base * C * D;
+  build_tile<C, D, true>(wh, wl, [&](int r, int c) { return -Wg[r * D + c]; });
+  bool ok = run(sy, [&] {
+    const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
+    const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
+    mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false);
+  });
+  uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *duh = pl + S::CCb, *dul = duh + S::CDb;
+  if (ok) {
+    acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
+      float m[16];
+      for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+      put16<C, true>(ph, pl, r, i0, m);  // element (r, i): MN-major operand P^T (k = r, m = i)
+    });
+    ok = run(sy, [&] {
+      const tc::Op pH{tc::smem_u32(ph), C, true}, pL{tc::smem_u32(pl), C, true};
+      const tc::Op oH{tc::smem_u32(doh), C, true}, oL{tc::smem_u32(dol), C, true};
+      mma3(tb + 64, pH, pL, oH, oL, C, tc::idesc_bf16(C, D, true, true), false, EX);
+    });
+  }
+  if (ok) {
+    float* dU = ws.dU + base * C * D;
+    acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(dU + i * D + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      put16<C, true>(duh, dul, i, j0, v);  // element (i, j): MN-major operand (k = i, n = j)
+    });
+    ok = run(sy, [&] {
+      const uint32_t id = tc::idesc_bf16(D, D, true, true);
+      const tc::Op qH{tc::smem_u32(qbh), C, true}, qL{tc::smem_u32(qbl), C, true};
+      const tc::Op oH{tc::smem_u32(doh), C, true}, oL{tc::smem_u32(dol), C, true};
+      const tc::Op wH{tc::smem_u32(wh), C, true}, wL{tc::smem_u32(wl), C, true};
+      const tc::Op uH{tc::smem_u32(duh), C, true}, uL{tc::smem_u32(dul), C, true};
+      mma3(tb + 192, qH, qL, oH, oL, C, id, false, EX);
+      mma3(tb + 192, wH, wL, uH, uL, C, id, true, false);
+    });
+  }
+  if (ok) {
+    float* X = ws.dS + base * D * D;
+    acc_read<D, D>(tb, 192, [&](int c, int j0, const float* v) {
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(X + c * D + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    });
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
+}
+
+// --------------------------------------------------------------------------------- backward dq
+// per (chunk, head), with S0 (chunk start state), dS (gradient of the chunk end state) and U:
+//   dP = lower_incl(dO U^T), Tq = dO S0^T, T1 = U dS^T,
+//   RS = dP bf (bf = k e^{G_0 - G}),  CS = dP^T qf (qf = q e^{G - G_0})
+//   dq  = e^G Tq + e^{G - G_0} RS                         (final)
+//   pdk = e^{G_C - G} T1 + e^{G_0 - G} CS                 (partial dk)
+//   pdG = q dq - k pdk,  pdG[n-1] += sum_i k_i e^{G_C - G_i} T1_i + e^{G_C} rowsum(dS * S0)
+struct BdqTcSmem {
+  static constexpr int C = kTcC, D = kTcD, LD = D + 1;
+  static constexpr size_t G = 0;
+  static constexpr size_t vec = G + sizeof(float) * C * LD;  // ref[D]
+  static constexpr size_t tiles = (vec + sizeof(float) * D + 1023) & ~size_t(1023);
+  static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2, DDb = size_t(D) * D * 2;
+  // phase 1: dO (K-major) | U (K-major) | S0 (K-major D x D); phase 2: dS in the S0 slot;
+  // phase 3: dP | bf (MN) | qf (MN) over the dO/U/S0 space; epilogue row buffer (C x LD fp32) after.
+  static constexpr size_t R = tiles;
+  static constexpr size_t total = R + 4 * CDb + 2 * DDb;
+};
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads, 1)
+    kda_bwd_dq_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
+                  const Tin* __restrict__ g_, const Tin* __restrict__ do_, Tout* __restrict__ dq_, KdaWs ws) {
+  using namespace tck;
+  using S = BdqTcSmem;
+  constexpr int C = S::C, D = S::D, LD = S::LD;
+  constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
+  const int ci = blockIdx.x, h = blockIdx.y;
+  const ChunkRec ch = t.chunks[ci];
+  const int n = ch.n_rows;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  float* sG = reinterpret_cast<float*>(tsm + S::G);
+  float* sref = reinterpret_cast<float*>(tsm + S::vec);
+  __shared__ int srow[C];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  __syncthreads();
+  cumsum_ref(sG, LD, n, sref, nullptr);
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  Sync sy{&bar, 0u, ws.status};
+  const size_t base = (size_t)ci * H + h;
+  const float* S0g = ws.S0 + base * D * D;
+  const float* dSg = ws.dS + base * D * D;
+  const float* Ug = ws.U + base * C * D;
+  // TMEM columns: Tq [0,128), T1 [128,256), RS [256,384), dP [384,448) then CS [384,512)
+  constexpr int cTq = 0, cT1 = 128, cRS = 256, cCS = 384;
+  uint8_t *doh = tsm + S::R, *dol = doh + S::CDb, *uh = dol + S::CDb, *ul = uh + S::CDb;
+  uint8_t *sh = ul + S::CDb, *sl = sh + S::DDb;
+  build_tile<C, D, !EX>(doh, dol, [&](int r, int j) {
+    return r >= ch.n_replay ? ld_in(do_, srow, H, h, n, r, j) : 0.f;
+  });
+  build_tile<C, D, true>(uh, ul, [&](int i, int j) { return Ug[i * D + j]; });
+  build_tile<D, D, true>(sh, sl, [&](int c, int j) { return S0g[c * D + j]; });
+  const tc::Op oH{tc::smem_u32(doh), C, false}, oL{tc::smem_u32(dol), C, false};
+  const tc::Op uH{tc::smem_u32(uh), C, false}, uL{tc::smem_u32(ul), C, false};
+  const tc::Op sH{tc::smem_u32(sh), D, false}, sL{tc::smem_u32(sl), D, false};
+  bool ok = run(sy, [&] {
+    mma4(tb + cCS, oH, oL, uH, uL, D, tc::idesc_bf16(C, C, false, false), false, EX, false);   // dP (raw)
+    mma4(tb + cTq, oH, oL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, EX, false);  // Tq
+  });
+  if (ok) {
+    build_tile<D, D, true>(sh, sl, [&](int c, int j) { return dSg[c * D + j]; });
+    ok = run(sy, [&] { mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false); });
+  }
+  uint8_t *pH8 = tsm + S::R, *pL8 = pH8 + S::CCb, *bh = pL8 + S::CCb, *bl = bh + S::CDb, *qh = bl + S::CDb,
+          *ql = qh + S::CDb;
+  if (ok) {
+    acc_read<C, C>(tb, cCS, [&](int r, int i0, const float* v) {
+      float m[16];
+      for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+      put16<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
+    });
+    build_tile<C, D, true>(bh, bl, [&](int i, int c) {
+      return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
+    });
+    build_tile<C, D, true>(qh, ql, [&](int r, int c) {
+      return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
+    });
+    ok = run(sy, [&] {
+      const uint32_t id = tc::idesc_bf16(C, D, false, true), idT = tc::idesc_bf16(C, D, true, true);
+      const tc::Op pK{tc::smem_u32(pH8), C, false}, pKl{tc::smem_u32(pL8), C, false};  // dP (r, i), K-major
+      const tc::Op pM{tc::smem_u32(pH8), C, true}, pMl{tc::smem_u32(pL8), C, true};    // dP^T (i, r), MN-major
+      const tc::Op bH{tc::smem_u32(bh), C, true}, bL{tc::smem_u32(bl), C, true};
+      const tc::Op qH{tc::smem_u32(qh), C, true}, qL{tc::smem_u32(ql), C, true};
+      mma4(tb + cRS, pK, pKl, bH, bL, C, id, false, false, false);
+      mma4(tb + cCS, pM, pMl, qH, qL, C, idT, false, false, false);
+    });
+  }
+  if (ok) {
+    float* pdk = ws.pdk + base * C * D;
+    float* pdG = ws.pdG + base * C * D;
+    float* sbuf = reinterpret_cast<float*>(tsm + S::R);  // [C][LD]: k e^{G_C - G} T1 per row
+    const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
+    const int r = lane < 16 ? 16 * sp + lane : -1;
+    const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
+    for (int c0 = grp * 16; c0 < D; c0 += 32) {
+      float tq[16], t1[16], rs[16], cs[16];
+      tc::tmem_ld16(la + cTq + c0, tq);
+      tc::tmem_ld16(la + cT1 + c0, t1);
+      tc::tmem_ld16(la + cRS + c0, rs);
+      tc::tmem_ld16(la + cCS + c0, cs);
+      if (r < 0) continue;
+      for (int j = 0; j < 16; ++j) {
+        const int c = c0 + j;
+        const float Gr = sG[r * LD + c], G0 = sref[c], GC = sG[(n - 1) * LD + c];
+        const float qv = ld_in(q_, srow, H, h, n, r, c), kv = ld_in(k_, srow, H, h, n, r, c);
+        const float dq = expf(Gr) * tq[j] + expf(Gr - G0) * rs[j];
+        const float dks = expf(GC - Gr) * t1[j];
+        const float dk = dks + expf(G0 - Gr) * cs[j];
+        pdk[r * D + c] = dk;
+        pdG[r * D + c] = qv * dq - kv * dk;
+        sbuf[r * LD + c] = r < n ? kv * dks : 0.f;
+        if (r >= ch.n_replay && r < n) dq_[((size_t)srow[r] * H + h) * D + c] = from_f<Tout>(dq);
+      }
+    }
+    __syncthreads();
+    for (int c = tid; c < D; c += blockDim.x) {
+      float acc = 0.f;
+      for (int i = 0; i < n; ++i) acc += sbuf[i * LD + c];
+      float acc2 = 0.f;
+      for (int j = 0; j < D; ++j) acc2 = fmaf(dSg[c * D + j], S0g[c * D + j], acc2);
+      pdG[(n - 1) * D + c] += acc + expf(sG[(n - 1) * LD + c]) * acc2;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
+}
+
+}  // namespace tpc

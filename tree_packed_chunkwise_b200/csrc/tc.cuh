@@ -1,0 +1,140 @@
+// Fifth-generation tensor-core (tcgen05) helpers for sm_100a: shared-memory operand descriptors,
+// MMA issue with TMEM accumulators, completion through an mbarrier (bounded wait), TMEM
+// allocation and loads.  Operands are bf16 tiles in the canonical no-swizzle "core matrix" layout:
+// 8 x 8 element blocks of 128 contiguous bytes (8 rows of 16 bytes).
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace tpc {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Byte offset of element (a, b) in a core-matrix tile: b is the contiguous index (8 elements per
+// 16-byte row of a core matrix), a the strided index with extent A (multiple of 8).
+__host__ __device__ __forceinline__ uint32_t cm_off(int a, int b, int A) {
+  return (uint32_t)(((((b >> 3) * (A >> 3)) + (a >> 3)) << 7) + ((a & 7) << 4) + ((b & 7) << 1));
+}
+
+// Shared-memory matrix descriptor (no swizzle, descriptor version 1 for sm_100).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// An operand tile: shared address, extent of its strided index, and whether the contiguous index
+// is M/N (mn = true, "MN-major") or K (mn = false, "K-major").
+//   K-major : element (row r in M or N, k) at cm_off(r, k, A = rows)
+//   MN-major: element (k, column n in M or N) at cm_off(k, n, A = K extent of the tile)
+struct Op {
+  uint32_t base;
+  int A;
+  bool mn;
+};
+
+// descriptor for the 16-wide K step s of the operand
+__device__ __forceinline__ uint64_t op_desc(const Op& o, int s) {
+  const uint32_t grp = (uint32_t)(o.A >> 3) * 128u;
+  if (!o.mn) return smem_desc(o.base + (uint32_t)(2 * s) * grp, grp, 128u);  // LBO: K chunk, SBO: 8 rows
+  return smem_desc(o.base + (uint32_t)(2 * s) * 128u, 128u, grp);             // LBO: 8 K rows, SBO: 8 columns
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, M in {64, 128}, N multiple of 8 (M = 64) or 16 (M = 128).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn, bool neg_a = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((neg_a ? 1u : 0u) << 13) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// D (+)= A (M x K) * B (K x N), K a multiple of 16; issued by one thread.
+__device__ __forceinline__ void mma_chain(uint32_t d_tmem, const Op& a, const Op& b, int K, uint32_t idesc,
+                                          bool accumulate) {
+  for (int s = 0; s < K / 16; ++s) mma_bf16(d_tmem, op_desc(a, s), op_desc(b, s), idesc, (accumulate || s) ? 1u : 0u);
+}
+
+// The mbarrier arrives once all tcgen05 operations issued so far by this thread have completed.
+__device__ __forceinline__ void commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity; false once timeout_ns has passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = 1000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > timeout_ns) return false;
+  return true;
+}
+
+// writes by threads to shared memory become visible to the tensor core (async proxy)
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// TMEM allocation by one whole warp; the address is written to *slot (shared memory).
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane (warp-collective; lanes of the warp's
+// sub-partition).  taddr = (lane << 16) | column.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// TMEM lane holding row m of an M-row accumulator (M = 128: lane m; M = 64: first half of each
+// 32-lane sub-partition).
+__host__ __device__ __forceinline__ int acc_lane(int m, int M) { return M == 128 ? m : (m & 15) + 32 * (m >> 4); }
+
+// bf16 hi/lo split of an fp32 value: x ~= hi + lo with |x - hi - lo| <= 2^-16 |x| (approximately)
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+}  // namespace tc
+}  // namespace tpc

@@ -10,6 +10,7 @@
 
 #include "../../include/tpc.h"
 #include "kda_kernels.cuh"
+#include "kda_tc.cuh"
 #include "plan.h"
 #include "rowmap_kernels.cuh"
 
@@ -143,17 +144,31 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
   const Tin* v = static_cast<const Tin*>(io->v);
   const Tin* g = static_cast<const Tin*>(io->g);
   const Tin* b = static_cast<const Tin*>(io->beta);
-  TPC_LAUNCH("kda_fwd_prep", st,
-             (kda_fwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, fwd_prep_smem<C, D>(), st>>>(p.dt, H, k, v, g, b, w)));
+  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  if constexpr (kTensorCores) {
+    TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmem::total));
+    TPC_LAUNCH("kda_fwd_prep_tc", st,
+               (kda_fwd_prep_tc<Tin><<<dim3(nc, H), kThreads, PrepTcSmem::total, st>>>(p.dt, H, k, v, g, b, w)));
+  } else {
+    TPC_LAUNCH("kda_fwd_prep", st,
+               (kda_fwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, fwd_prep_smem<C, D>(), st>>>(p.dt, H, k, v, g, b, w)));
+  }
   for (int r = 1; r <= p.n_rounds; ++r) {
     const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
     TPC_LAUNCH("kda_fwd_scan", st,
                (kda_fwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads, scan_smem<C, D, DVT>(), st>>>(
                    p.dt, s0, H, io->init_state, io->final_state, w)));
   }
-  TPC_LAUNCH("kda_fwd_out", st,
-             (kda_fwd_out<C, D, Tin, Tout><<<dim3(nc, H), kThreads, out_smem<C, D>(), st>>>(
-                 p.dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
+  if constexpr (kTensorCores) {
+    TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
+    TPC_LAUNCH("kda_fwd_out_tc", st,
+               (kda_fwd_out_tc<Tin, Tout><<<dim3(nc, H), kThreads, OutTcSmem::total, st>>>(
+                   p.dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
+  } else {
+    TPC_LAUNCH("kda_fwd_out", st,
+               (kda_fwd_out<C, D, Tin, Tout><<<dim3(nc, H), kThreads, out_smem<C, D>(), st>>>(
+                   p.dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
+  }
   return TPC_OK;
 }
 
