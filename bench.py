@@ -37,6 +37,7 @@ WORKLOAD = "single_fork"
 # algorithmic FLOP per processed token-head of each kernel (chunk C, head dim d), see the design doc
 def kernel_flops(name, C, d):
     Cd, dd = C * d, d * d
+    name = name[:-3] if name.endswith("_tc") else name
     return {"kda_fwd_prep": 6 * Cd, "kda_fwd_scan": 4 * dd, "kda_fwd_out": 4 * Cd + 2 * dd,
             "kda_bwd_prep": 2 * Cd + 4 * dd, "kda_bwd_scan": 4 * dd, "kda_bwd_dq": 6 * Cd + 4 * dd,
             "kda_bwd_dkv": 10 * Cd + 2 * dd}.get(name, 0)

@@ -706,4 +706,291 @@ __global__ void __launch_bounds__(kThreads, 1)
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
 }
 
+// --------------------------------------------------------------------------------- backward dk/dv
+// per (chunk, head), the WY part of the backward:
+//   Atilde = gated(k, k) (strict lower), T = (I + diag(beta) Atilde)^{-1}, X = [W | U'] = T diag(beta) [Kbar | V]
+//   dX = [-dU S0^T | dU],  dB = T^T dX,  dA = -strict_lower(dB X^T),  dAt = diag(beta) dA
+//   dk  = pdk + e^G beta dB_k + e^{G-G_0} (dAt bf) + e^{G_0-G} (dAt^T af)
+//   dG  = pdG + Kbar beta dB_k + k (e^{G-G_0} (dAt bf) - e^{G_0-G} (dAt^T af)),  dg = reverse cumsum of dG
+//   dv  = beta dB_v,  dbeta = rowsum(dB_k Kbar + dB_v v + dA Atilde)
+// Replayed rows go to the replay partials, rows replayed elsewhere to the target staging.
+struct BdkvTcSmem {
+  static constexpr int C = kTcC, D = kTcD, LD = D + 1, LC = C + 1;
+  static constexpr size_t G = 0;
+  static constexpr size_t At = G + sizeof(float) * C * LD;        // Atilde fp32 [C][LC]
+  static constexpr size_t vec = At + sizeof(float) * C * LC;      // beta[C], ref[D], dbeta parts[6][C]
+  static constexpr size_t Tt = (vec + sizeof(float) * (C + D + 6 * C) + 1023) & ~size_t(1023);  // T tile (MN)
+  static constexpr size_t CCb = size_t(C) * C * 2, CDb = size_t(C) * D * 2, DDb = size_t(D) * D * 2;
+  static constexpr size_t R = Tt + 2 * CCb;
+  static constexpr size_t Rbytes = 128 * 1024;
+  static constexpr size_t total = R + Rbytes;
+  // offsets inside R by phase
+  static constexpr size_t p1_af = 0, p1_bf = 2 * CDb;                                 // K-major af, bf
+  static constexpr size_t inv_L = 0, inv_T = inv_L + sizeof(float) * C * LC;           // fp32 L, T
+  static constexpr size_t inv_W1 = inv_T + sizeof(float) * C * LC, inv_W2 = inv_W1 + sizeof(float) * 4 * 16 * 17;
+  static constexpr size_t p2_Tp = 44 * 1024, p2_Kb = p2_Tp + 2 * CCb, p2_V = p2_Kb + 2 * CDb;  // T', Kbar, V
+  static constexpr size_t p2_dU = 0, p2_S0 = 2 * CDb;                                  // dU (K), S0 (K)
+  static constexpr size_t p3_X = 0, p3_dX = 4 * CDb;                                   // X (K, C x 2D), dX (MN)
+  static constexpr size_t p4_dB = 4 * CDb;                                             // dB (K, C x 2D)
+  static constexpr size_t p5_dA = 0, p5_bf = 2 * CCb, p5_af = p5_bf + 2 * CDb;         // dAt, bf (MN), af (MN)
+  static_assert(p2_V + 2 * CDb <= Rbytes && p2_S0 + 2 * DDb <= Rbytes && p3_dX + 4 * CDb <= Rbytes, "R");
+  static_assert(inv_W2 + sizeof(float) * 4 * 16 * 17 <= p2_Tp, "inverse scratch overlaps T'");
+};
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads, 1)
+    kda_bwd_dkv_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
+                   const Tin* __restrict__ g_, const Tin* __restrict__ beta_, Tout* __restrict__ dk_,
+                   Tout* __restrict__ dv_, float* __restrict__ dg_, float* __restrict__ dbeta_, KdaWs ws) {
+  using namespace tck;
+  using S = BdkvTcSmem;
+  constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
+  constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
+  const int ci = blockIdx.x, h = blockIdx.y;
+  const ChunkRec ch = t.chunks[ci];
+  const int n = ch.n_rows;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  float* sG = reinterpret_cast<float*>(tsm + S::G);
+  float* sAt = reinterpret_cast<float*>(tsm + S::At);
+  float* sb = reinterpret_cast<float*>(tsm + S::vec);
+  float* sref = sb + C;
+  float* sdb = sref + D;  // [6][C] partial dbeta (dB_k, dB_v, dA parts per warp group), fixed-order sum
+  uint8_t* tTh = tsm + S::Tt;
+  uint8_t* tTl = tTh + S::CCb;
+  uint8_t* R = tsm + S::R;
+  __shared__ int srow[C];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
+  for (int e = tid; e < 6 * C; e += blockDim.x) sdb[e] = 0.f;
+  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  __syncthreads();
+  cumsum_ref(sG, LD, n, sref, nullptr);
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  Sync sy{&bar, 0u, ws.status};
+  const size_t base = (size_t)ci * H + h;
+  const float* S0g = ws.S0 + base * D * D;
+  const float* dUg = ws.dU + base * C * D;
+  float* pdk = ws.pdk + base * C * D;
+  float* pdG = ws.pdG + base * C * D;
+  auto kin = [&](int r, int c) { return ld_in(k_, srow, H, h, n, r, c); };
+  const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
+  const int myrow = lane < 16 ? 16 * sp + lane : -1;  // M = 64 accumulator row of this thread
+  const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
+  // TMEM columns
+  constexpr int cA = 0, cW = 64, cU = 192, cdW = 320, cdB = 0, cdA = 256, cRS = 320, cCS = 0;
+
+  // ---- phase 1: Atilde
+  {
+    uint8_t *afh = R + S::p1_af, *afl = afh + S::CDb, *bfh = R + S::p1_bf, *bfl = bfh + S::CDb;
+    build_tile<C, D, true>(afh, afl, [&](int r, int c) { return kin(r, c) * expf(sG[r * LD + c] - sref[c]); });
+    build_tile<C, D, true>(bfh, bfl, [&](int i, int c) { return kin(i, c) * expf(sref[c] - sG[i * LD + c]); });
+  }
+  bool ok = run(sy, [&] {
+    const tc::Op ah{tc::smem_u32(R + S::p1_af), C, false}, al{tc::smem_u32(R + S::p1_af + S::CDb), C, false};
+    const tc::Op bh{tc::smem_u32(R + S::p1_bf), C, false}, bl{tc::smem_u32(R + S::p1_bf + S::CDb), C, false};
+    mma4(tb + cA, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false, false);
+  });
+  if (ok) {
+    float* sL = reinterpret_cast<float*>(R + S::inv_L);
+    float* sT = reinterpret_cast<float*>(R + S::inv_T);
+    acc_read<C, C>(tb, cA, [&](int r, int i0, const float* v) {
+      for (int j = 0; j < 16; ++j) {
+        const int i = i0 + j;
+        const float a = (i < r) ? v[j] : 0.f;
+        sAt[r * LC + i] = a;
+        sL[r * LC + i] = sb[r] * a;
+      }
+    });
+    __syncthreads();
+    block_inverse<LC>(sT, sL, reinterpret_cast<float*>(R + S::inv_W1), reinterpret_cast<float*>(R + S::inv_W2));
+    // ---- phase 2a: W = T' Kbar, U' = T' V (T' = T diag(beta)); the T tile for T^T dX
+    uint8_t *tph = R + S::p2_Tp, *tpl = tph + S::CCb, *kbh = R + S::p2_Kb, *kbl = kbh + S::CDb, *vh = R + S::p2_V,
+            *vl = vh + S::CDb;
+    build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
+    build_tile<C, C, true>(tTh, tTl, [&](int r, int i) { return sT[r * LC + i]; });
+    build_tile<C, D, true>(kbh, kbl, [&](int i, int c) { return kin(i, c) * expf(sG[i * LD + c]); });
+    build_tile<C, D, !EX>(vh, vl, [&](int i, int c) { return ld_in(v_, srow, H, h, n, i, c); });
+    ok = run(sy, [&] {
+      const uint32_t id = tc::idesc_bf16(C, D, false, true);
+      const tc::Op tH{tc::smem_u32(tph), C, false}, tL{tc::smem_u32(tpl), C, false};
+      const tc::Op kH{tc::smem_u32(kbh), C, true}, kL{tc::smem_u32(kbl), C, true};
+      const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
+      mma4(tb + cW, tH, tL, kH, kL, C, id, false, false, false);
+      mma4(tb + cU, tH, tL, vH, vL, C, id, false, false, EX);
+    });
+  }
+  if (ok) {
+    // ---- phase 2b: dW' = dU S0^T
+    uint8_t *duh = R + S::p2_dU, *dul = duh + S::CDb, *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
+    build_tile<C, D, true>(duh, dul, [&](int r, int j) { return dUg[r * D + j]; });
+    build_tile<D, D, true>(s0h, s0l, [&](int c, int j) { return S0g[c * D + j]; });
+    ok = run(sy, [&] {
+      const tc::Op aH{tc::smem_u32(duh), C, false}, aL{tc::smem_u32(dul), C, false};
+      const tc::Op bH{tc::smem_u32(s0h), D, false}, bL{tc::smem_u32(s0l), D, false};
+      mma4(tb + cdW, aH, aL, bH, bL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
+    });
+  }
+  if (ok) {
+    // ---- phase 3: X (K-major, rows i, columns n in [0, 2D)) and dX (MN-major, k = r, n)
+    uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb, *dxh = R + S::p3_dX, *dxl = dxh + 2 * S::CDb;
+    acc_read<C, D>(tb, cW, [&](int i, int c0, const float* v) { put16<C, true>(xh, xl, i, c0, v); });
+    acc_read<C, D>(tb, cU, [&](int i, int c0, const float* v) { put16<C, true>(xh, xl, i, D + c0, v); });
+    acc_read<C, D>(tb, cdW, [&](int r, int c0, const float* v) {
+      float m[16];
+      for (int j = 0; j < 16; ++j) m[j] = -v[j];
+      put16<C, true>(dxh, dxl, r, c0, m);
+    });
+    build_tile<C, D, true>(dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), [&](int r, int j) {
+      return dUg[r * D + j];
+    });
+    ok = run(sy, [&] {
+      const tc::Op aH{tc::smem_u32(tTh), C, true}, aL{tc::smem_u32(tTl), C, true};
+      const tc::Op bH{tc::smem_u32(dxh), C, true}, bL{tc::smem_u32(dxl), C, true};
+      mma4(tb + cdB, aH, aL, bH, bL, C, tc::idesc_bf16(C, 2 * D, true, true), false, false, false);
+    });
+  }
+  if (ok) {
+    // ---- read dB: dB tile for dA; dv; dk / dG / dbeta contributions
+    uint8_t *dbh = R + S::p4_dB, *dbl = dbh + 2 * S::CDb;
+    for (int c0 = grp * 16; c0 < 2 * D; c0 += 32) {
+      float v[16];
+      tc::tmem_ld16(la + cdB + c0, v);
+      if (myrow < 0) continue;
+      const int i = myrow;
+      put16<C, true>(dbh, dbl, i, c0, v);
+      float part = 0.f;
+      if (c0 < D) {
+        for (int j = 0; j < 16; ++j) {
+          const int c = c0 + j;
+          const float eg = expf(sG[i * LD + c]);
+          const float kv = kin(i, c);
+          const float bdb = sb[i] * v[j];
+          pdk[i * D + c] += eg * bdb;
+          pdG[i * D + c] += kv * eg * bdb;
+          part = fmaf(v[j], kv * eg, part);
+        }
+      } else if (i < n) {
+        for (int j = 0; j < 16; ++j) {
+          const int c = c0 - D + j;
+          const float vv = ld_in(v_, srow, H, h, n, i, c);
+          part = fmaf(v[j], vv, part);
+          const float val = sb[i] * v[j];
+          if (i < ch.n_replay) {
+            ws.rdv[((size_t)(ch.replay_base + i) * H + h) * D + c] = val;
+          } else {
+            const int tg = t.row_tgt[srow[i]];
+            if (tg >= 0) ws.tdv[((size_t)tg * H + h) * D + c] = val;
+            else dv_[((size_t)srow[i] * H + h) * D + c] = from_f<Tout>(val);
+          }
+        }
+      }
+      sdb[((c0 < D ? 0 : 2) + grp) * C + i] += part;  // one slot per (half, warp group)
+    }
+    uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb;
+    ok = run(sy, [&] {
+      const tc::Op aH{tc::smem_u32(dbh), C, false}, aL{tc::smem_u32(dbl), C, false};
+      const tc::Op bH{tc::smem_u32(xh), C, false}, bL{tc::smem_u32(xl), C, false};
+      mma4(tb + cdA, aH, aL, bH, bL, 2 * D, tc::idesc_bf16(C, C, false, false), false, false, false);
+    });
+  }
+  if (ok) {
+    // ---- dA = -(dB X^T) strict lower; dAt = beta dA (tile); dbeta += rowsum(dA Atilde)
+    uint8_t *dah = R + S::p5_dA, *dal = dah + S::CCb;
+    for (int c0 = grp * 16; c0 < C; c0 += 32) {
+      float v[16];
+      tc::tmem_ld16(la + cdA + c0, v);
+      if (myrow < 0) continue;
+      const int r = myrow;
+      float m[16], part = 0.f;
+      for (int j = 0; j < 16; ++j) {
+        const int i = c0 + j;
+        const float dA = (i < r) ? -v[j] : 0.f;
+        part = fmaf(dA, sAt[r * LC + i], part);
+        m[j] = sb[r] * dA;
+      }
+      put16<C, true>(dah, dal, r, c0, m);  // element (r, i)
+      sdb[(4 + grp) * C + r] += part;
+    }
+    // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
+    uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
+    build_tile<C, D, true>(bfh, bfl, [&](int i, int c) { return kin(i, c) * expf(sref[c] - sG[i * LD + c]); });
+    build_tile<C, D, true>(afh, afl, [&](int r, int c) { return kin(r, c) * expf(sG[r * LD + c] - sref[c]); });
+    ok = run(sy, [&] {
+      const tc::Op pK{tc::smem_u32(dah), C, false}, pKl{tc::smem_u32(dal), C, false};
+      const tc::Op pM{tc::smem_u32(dah), C, true}, pMl{tc::smem_u32(dal), C, true};
+      const tc::Op bH{tc::smem_u32(bfh), C, true}, bL{tc::smem_u32(bfl), C, true};
+      const tc::Op aH{tc::smem_u32(afh), C, true}, aL{tc::smem_u32(afl), C, true};
+      mma4(tb + cRS, pK, pKl, bH, bL, C, tc::idesc_bf16(C, D, false, true), false, false, false);
+      mma4(tb + cCS, pM, pMl, aH, aL, C, tc::idesc_bf16(C, D, true, true), false, false, false);
+    });
+  }
+  if (ok) {
+    // ---- final: dk, dG = partials + gated terms; dG staged for the reverse cumulative sum
+    float* sdG = reinterpret_cast<float*>(R);  // [C][LD]
+    for (int c0 = grp * 16; c0 < D; c0 += 32) {
+      float rs[16], cs[16];
+      tc::tmem_ld16(la + cRS + c0, rs);
+      tc::tmem_ld16(la + cCS + c0, cs);
+      if (myrow < 0) continue;
+      const int r = myrow;
+      for (int j = 0; j < 16; ++j) {
+        const int c = c0 + j;
+        const float Gr = sG[r * LD + c], G0 = sref[c];
+        const float a = expf(Gr - G0) * rs[j], b = expf(G0 - Gr) * cs[j];
+        const float kv = kin(r, c);
+        const float dkv = pdk[r * D + c] + a + b;
+        sdG[r * LD + c] = r < n ? pdG[r * D + c] + kv * (a - b) : 0.f;
+        if (r < n) {
+          if (r < ch.n_replay) {
+            ws.rdk[((size_t)(ch.replay_base + r) * H + h) * D + c] = dkv;
+          } else {
+            const int tg = t.row_tgt[srow[r]];
+            if (tg >= 0) ws.tdk[((size_t)tg * H + h) * D + c] = dkv;
+            else dk_[((size_t)srow[r] * H + h) * D + c] = from_f<Tout>(dkv);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    for (int c = tid; c < D; c += blockDim.x) {
+      float acc = 0.f;
+      for (int r = n - 1; r >= 0; --r) {
+        acc += sdG[r * LD + c];
+        if (r < ch.n_replay) {
+          ws.rdg[((size_t)(ch.replay_base + r) * H + h) * D + c] = acc;
+        } else {
+          const int tg = t.row_tgt[srow[r]];
+          if (tg >= 0) ws.tdg[((size_t)tg * H + h) * D + c] = acc;
+          else dg_[((size_t)srow[r] * H + h) * D + c] = acc;
+        }
+      }
+    }
+    for (int r = tid; r < n; r += blockDim.x) {
+      const float db = ((sdb[0 * C + r] + sdb[1 * C + r]) + (sdb[2 * C + r] + sdb[3 * C + r])) +
+                       (sdb[4 * C + r] + sdb[5 * C + r]);
+      if (r < ch.n_replay) {
+        ws.rdb[(size_t)(ch.replay_base + r) * H + h] = db;
+      } else {
+        const int tg = t.row_tgt[srow[r]];
+        if (tg >= 0) ws.tdb[(size_t)tg * H + h] = db;
+        else dbeta_[(size_t)srow[r] * H + h] = db;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
+}
+
 }  // namespace tpc

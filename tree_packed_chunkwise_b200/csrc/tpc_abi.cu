@@ -190,8 +190,15 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   const Tin* g = static_cast<const Tin*>(io->g);
   const Tin* b = static_cast<const Tin*>(io->beta);
   const Tin* dO = static_cast<const Tin*>(io->d_o);
-  TPC_LAUNCH("kda_bwd_prep", st,
-             (kda_bwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, bprep_smem<C, D>(), st>>>(p.dt, H, q, k, g, dO, w)));
+  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  if constexpr (kTensorCores) {
+    TPC_CUDA(set_smem(kda_bwd_prep_tc<Tin>, BprepTcSmem::total));
+    TPC_LAUNCH("kda_bwd_prep_tc", st,
+               (kda_bwd_prep_tc<Tin><<<dim3(nc, H), kThreads, BprepTcSmem::total, st>>>(p.dt, H, q, k, g, dO, w)));
+  } else {
+    TPC_LAUNCH("kda_bwd_prep", st,
+               (kda_bwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, bprep_smem<C, D>(), st>>>(p.dt, H, q, k, g, dO, w)));
+  }
   for (int r = p.n_rounds; r >= 1; --r) {
     const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
     TPC_LAUNCH("kda_bwd_scan", st,
@@ -199,13 +206,25 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
                                           scan_smem<C, D, DVT>() + sizeof(float) * D * (DVT + 1), st>>>(
                    p.dt, s0, H, io->d_final, w)));
   }
-  TPC_LAUNCH("kda_bwd_dq", st,
-             (kda_bwd_dq<C, D, Tin, Tout><<<dim3(nc, H), kThreads, bdq_smem<C, D>(), st>>>(
-                 p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w)));
-  TPC_LAUNCH("kda_bwd_dkv", st,
-             (kda_bwd_dkv<C, D, Tin, Tout><<<dim3(nc, H), kThreads, bdkv_smem<C, D>(), st>>>(
-                 p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg, io->dbeta,
-                 w)));
+  if constexpr (kTensorCores) {
+    TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
+    TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmem::total));
+    TPC_LAUNCH("kda_bwd_dq_tc", st,
+               (kda_bwd_dq_tc<Tin, Tout><<<dim3(nc, H), kThreads, BdqTcSmem::total, st>>>(
+                   p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w)));
+    TPC_LAUNCH("kda_bwd_dkv_tc", st,
+               (kda_bwd_dkv_tc<Tin, Tout><<<dim3(nc, H), kThreads, BdkvTcSmem::total, st>>>(
+                   p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg, io->dbeta,
+                   w)));
+  } else {
+    TPC_LAUNCH("kda_bwd_dq", st,
+               (kda_bwd_dq<C, D, Tin, Tout><<<dim3(nc, H), kThreads, bdq_smem<C, D>(), st>>>(
+                   p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w)));
+    TPC_LAUNCH("kda_bwd_dkv", st,
+               (kda_bwd_dkv<C, D, Tin, Tout><<<dim3(nc, H), kThreads, bdkv_smem<C, D>(), st>>>(
+                   p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg, io->dbeta,
+                   w)));
+  }
   if (!p.tgt_row.empty()) {
     TPC_LAUNCH("kda_replay_reduce", st,
                (kda_replay_reduce<D, Tout><<<dim3((unsigned)p.tgt_row.size(), H), 128, 0, st>>>(
