@@ -21,6 +21,7 @@ struct KdaWs {
   float *dU, *dS, *dS0seq, *pdk, *pdG;                     // backward
   float *rdk, *rdv, *rdg, *rdb;                            // replay partials [R][H][D] / [R][H]
   float *tdk, *tdv, *tdg, *tdb;                            // own part of replay-target rows
+  float *Mt, *Bc;  // tensor-core path: per-chunk state transition M (bf16 hi/lo operand tile) and B (fp32)
 };
 
 template <int C, int D>

@@ -23,6 +23,7 @@
 namespace tpc {
 
 constexpr int kTcC = 64, kTcD = 128;
+constexpr uint32_t kMtileBytes = 2u * kTcD * kTcD * 2u;  // state transition tile: hi + lo bf16, 128 x 128
 constexpr float kMaxChunkDecay = 80.f;  // G_first - G_last per channel over one chunk
 enum : int { kStatusTimeout = 8 };
 
@@ -46,6 +47,59 @@ __device__ __forceinline__ void build_tile(uint8_t* hi, uint8_t* lo, F val) {
     }
     *reinterpret_cast<uint4*>(hi + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(h);
     if (SPLIT) *reinterpret_cast<uint4*>(lo + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(l);
+  }
+}
+
+// Same tile from a row-major global matrix: row a starts at rowp(a) (nullptr -> zeros), columns b
+// contiguous.  Every thread first issues all of its 16-byte loads (8 bf16 or 2 x 4 fp32 per step),
+// then converts; f(a, b, x) transforms each loaded value.
+template <typename T>
+__device__ __forceinline__ void ld8(const T* p, float (&x)[8]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 w = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+  } else {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(b2[j]);
+      x[2 * j] = f.x;
+      x[2 * j + 1] = f.y;
+    }
+  }
+}
+
+template <int A, int B, bool SPLIT, typename T, class RP, class F>
+__device__ __forceinline__ void build_tile_ld(uint8_t* hi, uint8_t* lo, RP rowp, F f) {
+  constexpr int NCH = A * (B / 8);
+  static_assert(NCH % kThreads == 0, "tile chunks must be a multiple of the CTA size");
+  constexpr int IT = NCH / kThreads;
+  float x[IT][8];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * kThreads, a = e % A, b0 = (e / A) * 8;
+    const T* p = rowp(a);
+    if (p) ld8(p + b0, x[it]);
+    else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[it][j] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * kThreads, a = e % A, b0 = (e / A) * 8;
+    __align__(16) __nv_bfloat16 hh[8];
+    __align__(16) __nv_bfloat16 ll[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float y = f(a, b0 + j, x[it][j]);
+      if (SPLIT) split_bf16(y, hh[j], ll[j]);
+      else hh[j] = __float2bfloat16_rn(y);
+    }
+    *reinterpret_cast<uint4*>(hi + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(hh);
+    if (SPLIT) *reinterpret_cast<uint4*>(lo + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(ll);
   }
 }
 
@@ -246,7 +300,7 @@ struct PrepTcSmem {
   static constexpr size_t tiles = (vec + sizeof(float) * (C + 2 * D) + 1023) & ~size_t(1023);
   // phase 1: af hi/lo, bf hi/lo (C x D each); phase 2: T' hi/lo (C x C), Kbar hi/lo, V hi/lo (C x D)
   static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2;
-  static constexpr size_t total = tiles + 2 * CCb + 4 * CDb;
+  static constexpr size_t total = tiles + 6 * CDb;  // phase 3: W, U' (MN) and Khat (MN) hi/lo
 };
 
 template <typename Tin>
@@ -290,16 +344,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
+  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   bool ok = true;
   // phase 1: Atilde = af bf^T with af = k e^{G - ref}, bf = k e^{ref - G}
   {
     uint8_t *afh = tl, *afl = tl + S::CDb, *bfh = tl + 2 * S::CDb, *bfl = tl + 3 * S::CDb;
-    build_tile<C, D, true>(afh, afl, [&](int r, int c) {
-      return ld_in(k_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
-    });
-    build_tile<C, D, true>(bfh, bfl, [&](int i, int c) {
-      return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
-    });
+    build_tile_ld<C, D, true, Tin>(afh, afl, row_k, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
+    build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
     const tc::Op ah{tc::smem_u32(afh), C, false}, al{tc::smem_u32(afl), C, false};
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
     ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
@@ -319,10 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
             *vl = vh + S::CDb;
     build_tile<C, C, true>(th, tlo, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
-    build_tile<C, D, true>(kh, kl, [&](int i, int c) {
-      return ld_in(k_, srow, H, h, n, i, c) * expf(sG[i * LD + c]);
-    });
-    build_tile<C, D, !EX>(vh, vl, [&](int i, int c) { return ld_in(v_, srow, H, h, n, i, c); });
+    build_tile_ld<C, D, true, Tin>(kh, kl, row_k, [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); });
+    build_tile_ld<C, D, !EX, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
     const tc::Op tH{tc::smem_u32(th), C, false}, tL{tc::smem_u32(tlo), C, false};
     const tc::Op kH{tc::smem_u32(kh), C, true}, kL{tc::smem_u32(kl), C, true};
     const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
@@ -332,23 +382,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma3(tb + 192, tH, tL, vH, vL, C, id, false, EX);
     });
     if (ok) {
+      // phase 3: the chunk's state transition S_end = M S_0 + B with M = Diag(e^{G_C}) - Khat^T W and
+      // B = Khat^T U' (Khat = k e^{G_C - G})
       const size_t base = (size_t)ci * H + h;
-      float* W = ws.W + base * C * D;
-      float* U = ws.U + base * C * D;
+      float* Wg = ws.W + base * C * D;
+      float* Ug = ws.U + base * C * D;
+      uint8_t *wth = tl, *wtl = tl + S::CDb, *uth = tl + 2 * S::CDb, *utl = tl + 3 * S::CDb, *khh = tl + 4 * S::CDb,
+              *khl = tl + 5 * S::CDb;
       acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) {
         for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(W + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          *reinterpret_cast<float4*>(Wg + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        put16<C, true>(wth, wtl, r, c0, v);  // element (i, c): MN-major (k = i)
       });
       acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) {
         for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(U + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          *reinterpret_cast<float4*>(Ug + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        put16<C, true>(uth, utl, r, c0, v);
       });
-      float* Kh = ws.Khat + base * C * D;
-      for (int e = tid; e < C * D; e += blockDim.x) {
-        const int i = e / D, c = e % D;
-        Kh[e] = ld_in(k_, srow, H, h, n, i, c) * expf(sG[(n - 1) * LD + c] - sG[i * LD + c]);
+      const float* gC = sG + (n - 1) * LD;
+      build_tile_ld<C, D, true, Tin>(khh, khl, row_k, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
+      ok = run(sy, [&] {
+        const uint32_t id = tc::idesc_bf16(D, D, true, true);
+        const tc::Op kH{tc::smem_u32(khh), C, true}, kL{tc::smem_u32(khl), C, true};
+        const tc::Op wH{tc::smem_u32(wth), C, true}, wL{tc::smem_u32(wtl), C, true};
+        const tc::Op uH{tc::smem_u32(uth), C, true}, uL{tc::smem_u32(utl), C, true};
+        mma4(tb, kH, kL, wH, wL, C, id, false, false, false);        // Khat^T W
+        mma4(tb + 128, kH, kL, uH, uL, C, id, false, false, false);  // Khat^T U'
+      });
+      if (ok) {
+        uint8_t* Mt = reinterpret_cast<uint8_t*>(ws.Mt) + base * kMtileBytes;
+        float* Bg = ws.Bc + base * D * D;
+        acc_read<D, D>(tb, 0, [&](int c, int c0, const float* v) {
+          float m[16];
+          const float gam = expf(gC[c]);
+          for (int j = 0; j < 16; ++j) m[j] = (c0 + j == c ? gam : 0.f) - v[j];
+          put16<D, true>(Mt, Mt + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
+        });
+        acc_read<D, D>(tb, 128, [&](int c, int j0, const float* v) {
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(Bg + c * D + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        });
       }
-      for (int c = tid; c < D; c += blockDim.x) ws.decay[base * D + c] = expf(sG[(n - 1) * LD + c]);
     }
   }
   tc::fence_before_sync();
@@ -357,17 +431,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // --------------------------------------------------------------------------------- forward output
-// per (chunk, head): P = lower_incl(gated(q, k)), O = Qbar S0 + P U (own rows only)
+// per (chunk, head), with the chunk-start state S0 from the scan:
+//   U = U' - W S0 (written back for the backward),  P = lower_incl(gated(q, k)),  O = Qbar S0 + P U
 struct OutTcSmem {
   static constexpr int C = kTcC, D = kTcD, LD = D + 1;
   static constexpr size_t G = 0;
   static constexpr size_t vec = G + sizeof(float) * C * LD;  // ref[D]
   static constexpr size_t tiles = (vec + sizeof(float) * D + 1023) & ~size_t(1023);
   static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2, DDb = size_t(D) * D * 2;
-  // region R (4 CDb): phase 1 qf hi/lo + bf hi/lo; phase 2: P hi/lo (2 CCb) + U hi/lo (2 CDb)
+  // R (4 CDb): run 1 qf + bf; run 2 P (2 CCb) + U (2 CDb).  Wq (2 CDb): run 1 W, run 2 Qbar.
   static constexpr size_t R = tiles;
-  static constexpr size_t Qb = R + 4 * CDb;     // Qbar hi/lo
-  static constexpr size_t S0 = Qb + 2 * CDb;    // S0 hi/lo (D x D)
+  static constexpr size_t Wq = R + 4 * CDb;
+  static constexpr size_t S0 = Wq + 2 * CDb;    // S0 hi/lo (D x D, MN-major)
   static constexpr size_t total = S0 + 2 * DDb;
 };
 
@@ -389,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
   for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
-  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 256);
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
   if (tid == 0) {
     tc::mbar_init(&bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -402,43 +477,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
+  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   const size_t base = (size_t)ci * H + h;
-  uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
-  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *s0h = tsm + S::S0, *s0l = s0h + S::DDb;
-  build_tile<C, D, true>(qfh, qfl, [&](int r, int c) {
-    return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
-  });
-  build_tile<C, D, true>(bfh, bfl, [&](int i, int c) {
-    return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
-  });
-  build_tile<C, D, true>(qbh, qbl, [&](int r, int c) { return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c]); });
   const float* S0g = ws.S0 + base * D * D;
-  build_tile<D, D, true>(s0h, s0l, [&](int c, int j) { return S0g[c * D + j]; });
+  const float* Wg = ws.W + base * C * D;
+  float* Ug = ws.U + base * C * D;
+  // TMEM: P [0,64), W S0 [64,192), O [192,320)
+  uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
+  uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb, *s0h = tsm + S::S0, *s0l = s0h + S::DDb;
+  build_tile_ld<C, D, true, Tin>(qfh, qfl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
+  build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
+  build_tile_ld<C, D, true, float>(wh, wl, [&](int r) { return Wg + r * D; }, [&](int, int, float x) { return x; });
+  build_tile_ld<D, D, true, float>(s0h, s0l, [&](int c) { return S0g + c * D; }, [&](int, int, float x) { return x; });
+  const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
   bool ok = run(sy, [&] {
     const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
-    mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false);
+    const tc::Op wH{tc::smem_u32(wh), C, false}, wL{tc::smem_u32(wl), C, false};
+    mma4(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false, false);
+    mma4(tb + 64, wH, wL, sH, sL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
   });
+  uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
+  uint8_t *qbh = wh, *qbl = wl;
   if (ok) {
-    uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
     acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
       float m[16];
       for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
       put16<C, true>(ph, pl, r, i0, m);
     });
-    const float* Ug = ws.U + base * C * D;
-    build_tile<C, D, true>(uh, ul, [&](int i, int j) { return Ug[i * D + j]; });
+    acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
+      float u[16];
+      for (int j = 0; j < 16; j += 4) {
+        const float4 up = *reinterpret_cast<const float4*>(Ug + i * D + j0 + j);
+        u[j] = up.x - v[j]; u[j + 1] = up.y - v[j + 1]; u[j + 2] = up.z - v[j + 2]; u[j + 3] = up.w - v[j + 3];
+        *reinterpret_cast<float4*>(Ug + i * D + j0 + j) = make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
+      }
+      put16<C, true>(uh, ul, i, j0, u);  // element (i, j): MN-major (k = i)
+    });
+    build_tile_ld<C, D, true, Tin>(qbh, qbl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c]); });
     ok = run(sy, [&] {
       const uint32_t id = tc::idesc_bf16(C, D, false, true);
       const tc::Op qH{tc::smem_u32(qbh), C, false}, qL{tc::smem_u32(qbl), C, false};
-      const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
       const tc::Op pH{tc::smem_u32(ph), C, false}, pL{tc::smem_u32(pl), C, false};
       const tc::Op uH{tc::smem_u32(uh), C, true}, uL{tc::smem_u32(ul), C, true};
-      mma3(tb + 64, qH, qL, sH, sL, D, id, false, false);
-      mma3(tb + 64, pH, pL, uH, uL, C, id, true, false);
+      mma4(tb + 192, qH, qL, sH, sL, D, id, false, false, false);
+      mma4(tb + 192, pH, pL, uH, uL, C, id, true, false, false);
     });
     if (ok) {
-      acc_read<C, D>(tb, 64, [&](int r, int j0, const float* v) {
+      acc_read<C, D>(tb, 192, [&](int r, int j0, const float* v) {
         if (r >= ch.n_replay && r < n) {
           Tout* dst = o_ + ((size_t)srow[r] * H + h) * D + j0;
           for (int j = 0; j < 16; ++j) dst[j] = from_f<Tout>(v[j]);
@@ -448,12 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 256);
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
 }
-
-}  // namespace tpc
-
-namespace tpc {
 
 // --------------------------------------------------------------------------------- backward prep
 // per (chunk, head): dU0 = P^T dO and X = Qbar^T dO - W^T dU0 (the state-independent parts of the
@@ -503,22 +586,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
+  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_do = [&](int a) -> const Tin* {
+    return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
+  };
   const size_t base = (size_t)ci * H + h;
   uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
   uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *doh = tsm + S::dO, *dol = doh + S::CDb;
   uint8_t *wh = tsm + S::Wt, *wl = wh + S::CDb;
-  build_tile<C, D, true>(qfh, qfl, [&](int r, int c) {
-    return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
-  });
-  build_tile<C, D, true>(bfh, bfl, [&](int i, int c) {
-    return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
-  });
-  build_tile<C, D, true>(qbh, qbl, [&](int r, int c) { return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c]); });
-  build_tile<C, D, !EX>(doh, dol, [&](int r, int j) {
-    return r >= ch.n_replay ? ld_in(do_, srow, H, h, n, r, j) : 0.f;
-  });
+  build_tile_ld<C, D, true, Tin>(qfh, qfl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
+  build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
+  build_tile_ld<C, D, true, Tin>(qbh, qbl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c]); });
+  build_tile_ld<C, D, !EX, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
   const float* Wg = ws.W + base * C * D;
-  build_tile<C, D, true>(wh, wl, [&](int r, int c) { return -Wg[r * D + c]; });
+  build_tile_ld<C, D, true, float>(wh, wl, [&](int r) { return Wg + r * D; }, [&](int, int, float x) { return -x; });
   bool ok = run(sy, [&] {
     const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
@@ -617,6 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
+  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_do = [&](int a) -> const Tin* {
+    return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
+  };
   const size_t base = (size_t)ci * H + h;
   const float* S0g = ws.S0 + base * D * D;
   const float* dSg = ws.dS + base * D * D;
@@ -625,11 +712,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int cTq = 0, cT1 = 128, cRS = 256, cCS = 384;
   uint8_t *doh = tsm + S::R, *dol = doh + S::CDb, *uh = dol + S::CDb, *ul = uh + S::CDb;
   uint8_t *sh = ul + S::CDb, *sl = sh + S::DDb;
-  build_tile<C, D, !EX>(doh, dol, [&](int r, int j) {
-    return r >= ch.n_replay ? ld_in(do_, srow, H, h, n, r, j) : 0.f;
-  });
-  build_tile<C, D, true>(uh, ul, [&](int i, int j) { return Ug[i * D + j]; });
-  build_tile<D, D, true>(sh, sl, [&](int c, int j) { return S0g[c * D + j]; });
+  build_tile_ld<C, D, !EX, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
+  build_tile_ld<C, D, true, float>(uh, ul, [&](int i) { return Ug + i * D; }, [&](int, int, float x) { return x; });
+  build_tile_ld<D, D, true, float>(sh, sl, [&](int c) { return S0g + c * D; }, [&](int, int, float x) { return x; });
   const tc::Op oH{tc::smem_u32(doh), C, false}, oL{tc::smem_u32(dol), C, false};
   const tc::Op uH{tc::smem_u32(uh), C, false}, uL{tc::smem_u32(ul), C, false};
   const tc::Op sH{tc::smem_u32(sh), D, false}, sL{tc::smem_u32(sl), D, false};
@@ -638,8 +723,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma4(tb + cTq, oH, oL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, EX, false);  // Tq
   });
   if (ok) {
-    build_tile<D, D, true>(sh, sl, [&](int c, int j) { return dSg[c * D + j]; });
-    ok = run(sy, [&] { mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false); });
+    // phase 2: T1 = U dS^T and dU = dU0 + Khat dS (Khat = k e^{G_C - G}, K-major in the dO slot)
+    build_tile_ld<D, D, true, float>(sh, sl, [&](int c) { return dSg + c * D; }, [&](int, int, float x) { return x; });
+    const float* gC = sG + (n - 1) * LD;
+    build_tile_ld<C, D, true, Tin>(doh, dol, row_k, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
+    ok = run(sy, [&] {
+      mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
+      const tc::Op kH{tc::smem_u32(doh), C, false}, kL{tc::smem_u32(dol), C, false};
+      const tc::Op dH{tc::smem_u32(sh), D, true}, dL{tc::smem_u32(sl), D, true};
+      mma4(tb + cRS, kH, kL, dH, dL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
+    });
+    if (ok) {
+      float* dUg = ws.dU + base * C * D;
+      acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) {
+        for (int j = 0; j < 16; j += 4) {
+          float4 u = *reinterpret_cast<const float4*>(dUg + i * D + j0 + j);
+          u.x += v[j]; u.y += v[j + 1]; u.z += v[j + 2]; u.w += v[j + 3];
+          *reinterpret_cast<float4*>(dUg + i * D + j0 + j) = u;
+        }
+      });
+    }
   }
   uint8_t *pH8 = tsm + S::R, *pL8 = pH8 + S::CCb, *bh = pL8 + S::CCb, *bl = bh + S::CDb, *qh = bl + S::CDb,
           *ql = qh + S::CDb;
@@ -649,12 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
       put16<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
     });
-    build_tile<C, D, true>(bh, bl, [&](int i, int c) {
-      return ld_in(k_, srow, H, h, n, i, c) * expf(sref[c] - sG[i * LD + c]);
-    });
-    build_tile<C, D, true>(qh, ql, [&](int r, int c) {
-      return ld_in(q_, srow, H, h, n, r, c) * expf(sG[r * LD + c] - sref[c]);
-    });
+    build_tile_ld<C, D, true, Tin>(bh, bl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
+    build_tile_ld<C, D, true, Tin>(qh, ql, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
     ok = run(sy, [&] {
       const uint32_t id = tc::idesc_bf16(C, D, false, true), idT = tc::idesc_bf16(C, D, true, true);
       const tc::Op pK{tc::smem_u32(pH8), C, false}, pKl{tc::smem_u32(pL8), C, false};  // dP (r, i), K-major
@@ -778,6 +877,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
+  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   const size_t base = (size_t)ci * H + h;
   const float* S0g = ws.S0 + base * D * D;
   const float* dUg = ws.dU + base * C * D;
@@ -793,8 +894,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- phase 1: Atilde
   {
     uint8_t *afh = R + S::p1_af, *afl = afh + S::CDb, *bfh = R + S::p1_bf, *bfl = bfh + S::CDb;
-    build_tile<C, D, true>(afh, afl, [&](int r, int c) { return kin(r, c) * expf(sG[r * LD + c] - sref[c]); });
-    build_tile<C, D, true>(bfh, bfl, [&](int i, int c) { return kin(i, c) * expf(sref[c] - sG[i * LD + c]); });
+    build_tile_ld<C, D, true, Tin>(afh, afl, row_k, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
+    build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
   }
   bool ok = run(sy, [&] {
     const tc::Op ah{tc::smem_u32(R + S::p1_af), C, false}, al{tc::smem_u32(R + S::p1_af + S::CDb), C, false};
@@ -819,8 +920,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             *vl = vh + S::CDb;
     build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
     build_tile<C, C, true>(tTh, tTl, [&](int r, int i) { return sT[r * LC + i]; });
-    build_tile<C, D, true>(kbh, kbl, [&](int i, int c) { return kin(i, c) * expf(sG[i * LD + c]); });
-    build_tile<C, D, !EX>(vh, vl, [&](int i, int c) { return ld_in(v_, srow, H, h, n, i, c); });
+    build_tile_ld<C, D, true, Tin>(kbh, kbl, row_k, [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); });
+    build_tile_ld<C, D, !EX, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
     ok = run(sy, [&] {
       const uint32_t id = tc::idesc_bf16(C, D, false, true);
       const tc::Op tH{tc::smem_u32(tph), C, false}, tL{tc::smem_u32(tpl), C, false};
@@ -833,8 +934,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // ---- phase 2b: dW' = dU S0^T
     uint8_t *duh = R + S::p2_dU, *dul = duh + S::CDb, *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
-    build_tile<C, D, true>(duh, dul, [&](int r, int j) { return dUg[r * D + j]; });
-    build_tile<D, D, true>(s0h, s0l, [&](int c, int j) { return S0g[c * D + j]; });
+    build_tile_ld<C, D, true, float>(duh, dul, [&](int r) { return dUg + r * D; }, [&](int, int, float x) { return x; });
+    build_tile_ld<D, D, true, float>(s0h, s0l, [&](int c) { return S0g + c * D; }, [&](int, int, float x) { return x; });
     ok = run(sy, [&] {
       const tc::Op aH{tc::smem_u32(duh), C, false}, aL{tc::smem_u32(dul), C, false};
       const tc::Op bH{tc::smem_u32(s0h), D, false}, bL{tc::smem_u32(s0l), D, false};
@@ -851,9 +952,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) m[j] = -v[j];
       put16<C, true>(dxh, dxl, r, c0, m);
     });
-    build_tile<C, D, true>(dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), [&](int r, int j) {
-      return dUg[r * D + j];
-    });
+    build_tile_ld<C, D, true, float>(dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), [&](int r) { return dUg + r * D; }, [&](int, int, float x) { return x; });
     ok = run(sy, [&] {
       const tc::Op aH{tc::smem_u32(tTh), C, true}, aL{tc::smem_u32(tTl), C, true};
       const tc::Op bH{tc::smem_u32(dxh), C, true}, bL{tc::smem_u32(dxl), C, true};
@@ -924,8 +1023,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
     uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
-    build_tile<C, D, true>(bfh, bfl, [&](int i, int c) { return kin(i, c) * expf(sref[c] - sG[i * LD + c]); });
-    build_tile<C, D, true>(afh, afl, [&](int r, int c) { return kin(r, c) * expf(sG[r * LD + c] - sref[c]); });
+    build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
+    build_tile_ld<C, D, true, Tin>(afh, afl, row_k, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
     ok = run(sy, [&] {
       const tc::Op pK{tc::smem_u32(dah), C, false}, pKl{tc::smem_u32(dal), C, false};
       const tc::Op pM{tc::smem_u32(dah), C, true}, pMl{tc::smem_u32(dal), C, true};

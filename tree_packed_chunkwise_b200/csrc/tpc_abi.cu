@@ -11,6 +11,7 @@
 #include "../../include/tpc.h"
 #include "kda_kernels.cuh"
 #include "kda_tc.cuh"
+#include "kda_scan_tc.cuh"
 #include "plan.h"
 #include "rowmap_kernels.cuh"
 
@@ -63,7 +64,8 @@ Profiler g_prof;
 
 // workspace layout (bytes) for a plan + shape
 struct WsLayout {
-  size_t status, W, U, Khat, decay, S0, slot, dU, dS, dS0seq, pdk, pdG, rdk, rdv, rdg, rdb, tdk, tdv, tdg, tdb, total;
+  size_t status, W, U, Khat, decay, S0, slot, dU, dS, dS0seq, pdk, pdG, rdk, rdv, rdg, rdb, tdk, tdv, tdg, tdb, Mt, Bc,
+      total;
 };
 
 WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
@@ -92,6 +94,9 @@ WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
   L.tdv = take(T * H * D * 4);
   L.tdg = take(T * H * D * 4);
   L.tdb = take(T * H * 4);
+  const bool tensor_cores = (C == tpc::kTcC && D == tpc::kTcD);
+  L.Mt = take(tensor_cores ? nc * H * (size_t)tpc::kMtileBytes : 0);
+  L.Bc = take(tensor_cores ? nc * H * dd * 4 : 0);
   L.total = o;
   return L;
 }
@@ -105,6 +110,7 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
   w.dU = f(L.dU); w.dS = f(L.dS); w.dS0seq = f(L.dS0seq); w.pdk = f(L.pdk); w.pdG = f(L.pdG);
   w.rdk = f(L.rdk); w.rdv = f(L.rdv); w.rdg = f(L.rdg); w.rdb = f(L.rdb);
   w.tdk = f(L.tdk); w.tdv = f(L.tdv); w.tdg = f(L.tdg); w.tdb = f(L.tdb);
+  w.Mt = f(L.Mt); w.Bc = f(L.Bc);
   return w;
 }
 
@@ -153,11 +159,18 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     TPC_LAUNCH("kda_fwd_prep", st,
                (kda_fwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, fwd_prep_smem<C, D>(), st>>>(p.dt, H, k, v, g, b, w)));
   }
+  if constexpr (kTensorCores) TPC_CUDA(set_smem(kda_scan_tc<false>, ScanTcSmem::total));
   for (int r = 1; r <= p.n_rounds; ++r) {
     const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-    TPC_LAUNCH("kda_fwd_scan", st,
-               (kda_fwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads, scan_smem<C, D, DVT>(), st>>>(
-                   p.dt, s0, H, io->init_state, io->final_state, w)));
+    if constexpr (kTensorCores) {
+      TPC_LAUNCH("kda_fwd_scan_tc", st,
+                 (kda_scan_tc<false><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
+                     p.dt, s0, H, io->init_state, io->final_state, nullptr, w)));
+    } else {
+      TPC_LAUNCH("kda_fwd_scan", st,
+                 (kda_fwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads, scan_smem<C, D, DVT>(), st>>>(
+                     p.dt, s0, H, io->init_state, io->final_state, w)));
+    }
   }
   if constexpr (kTensorCores) {
     TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
@@ -199,12 +212,19 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
     TPC_LAUNCH("kda_bwd_prep", st,
                (kda_bwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, bprep_smem<C, D>(), st>>>(p.dt, H, q, k, g, dO, w)));
   }
+  if constexpr (kTensorCores) TPC_CUDA(set_smem(kda_scan_tc<true>, ScanTcSmem::total));
   for (int r = p.n_rounds; r >= 1; --r) {
     const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-    TPC_LAUNCH("kda_bwd_scan", st,
-               (kda_bwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads,
-                                          scan_smem<C, D, DVT>() + sizeof(float) * D * (DVT + 1), st>>>(
-                   p.dt, s0, H, io->d_final, w)));
+    if constexpr (kTensorCores) {
+      TPC_LAUNCH("kda_bwd_scan_tc", st,
+                 (kda_scan_tc<true><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
+                     p.dt, s0, H, nullptr, nullptr, io->d_final, w)));
+    } else {
+      TPC_LAUNCH("kda_bwd_scan", st,
+                 (kda_bwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads,
+                                            scan_smem<C, D, DVT>() + sizeof(float) * D * (DVT + 1), st>>>(
+                     p.dt, s0, H, io->d_final, w)));
+    }
   }
   if constexpr (kTensorCores) {
     TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
