@@ -103,6 +103,95 @@ __device__ __forceinline__ void build_tile_ld(uint8_t* hi, uint8_t* lo, RP rowp,
   }
 }
 
+// Gate rows of the chunk into G (fp32, pitch LD): every thread issues its 16-byte loads first;
+// neighbouring threads take neighbouring rows (conflict-free stores).  Rows >= n are zero.
+template <typename T>
+__device__ __forceinline__ void load_gate(float* G, int LD, const T* g_, const int* rows, int H, int h, int n) {
+  constexpr int NCH = kTcC * (kTcD / 8), IT = NCH / kThreads;
+  float x[IT][8];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * kThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
+    if (a < n) ld8(g_ + ((size_t)rows[a] * H + h) * kTcD + b0, x[it]);
+    else
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[it][j] = 0.f;
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * kThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) G[a * LD + b0 + j] = x[it][j];
+  }
+}
+
+// Copy of the chunk's rows of an input (row pitch kTcD + 8 elements) in shared memory.
+constexpr int kStagePitch = kTcD + 8;
+template <typename T>
+__device__ __forceinline__ void stage_rows(T* dst, const T* src, const int* rows, int H, int h, int n) {
+  constexpr int VEC = 16 / sizeof(T), NCH = kTcC * (kTcD / VEC), IT = NCH / kThreads;
+  uint4 x[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * kThreads, a = e / (kTcD / VEC), b0 = (e % (kTcD / VEC)) * VEC;
+    x[it] = a < n ? __ldg(reinterpret_cast<const uint4*>(src + ((size_t)rows[a] * H + h) * kTcD + b0))
+                  : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * kThreads, a = e / (kTcD / VEC), b0 = (e % (kTcD / VEC)) * VEC;
+    *reinterpret_cast<uint4*>(dst + a * kStagePitch + b0) = x[it];
+  }
+}
+
+// 16 consecutive values of a staged row as fp32
+template <typename T>
+__device__ __forceinline__ void staged16(const T* st, int r, int c0, float (&v)[16]) {
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) {
+      const float4 u = *reinterpret_cast<const float4*>(st + r * kStagePitch + c0 + j);
+      v[j] = u.x; v[j + 1] = u.y; v[j + 2] = u.z; v[j + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; j += 8) {
+      const uint4 u = *reinterpret_cast<const uint4*>(st + r * kStagePitch + c0 + j);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(b2[k]);
+        v[j + 2 * k] = f.x;
+        v[j + 2 * k + 1] = f.y;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void ld16g(const float* p, float (&v)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 4) {
+    const float4 u = *reinterpret_cast<const float4*>(p + j);
+    v[j] = u.x; v[j + 1] = u.y; v[j + 2] = u.z; v[j + 3] = u.w;
+  }
+}
+__device__ __forceinline__ void st16g(float* p, const float (&v)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(p + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+}
+template <typename T>
+__device__ __forceinline__ void st16_out(T* p, const float (&v)[16]) {
+  if constexpr (sizeof(T) == 4) {
+    st16g(reinterpret_cast<float*>(p), v);
+  } else {
+    __align__(16) __nv_bfloat16 b[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) b[j] = __float2bfloat16_rn(v[j]);
+    reinterpret_cast<uint4*>(p)[0] = reinterpret_cast<const uint4*>(b)[0];
+    reinterpret_cast<uint4*>(p)[1] = reinterpret_cast<const uint4*>(b)[1];
+  }
+}
+
 // Reads an M x N fp32 accumulator (N a multiple of 32) starting at TMEM column col0:
 // f(m, n0, v) gets 16 consecutive columns n0 .. n0+15 of row m.  Warp w reads the lanes of
 // sub-partition w % 4; the two groups of four warps take alternating 16-column chunks.
@@ -337,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
-  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, ws.status);
   __syncthreads();
@@ -470,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
   __syncthreads();
@@ -579,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
   __syncthreads();
@@ -692,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
   __syncthreads();
@@ -768,6 +857,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* pdk = ws.pdk + base * C * D;
     float* pdG = ws.pdG + base * C * D;
     float* sbuf = reinterpret_cast<float*>(tsm + S::R);  // [C][LD]: k e^{G_C - G} T1 per row
+    Tin* sq = reinterpret_cast<Tin*>(tsm + S::R + sizeof(float) * C * LD);
+    Tin* sk = sq + C * kStagePitch;
+    stage_rows(sq, q_, srow, H, h, n);
+    stage_rows(sk, k_, srow, H, h, n);
+    __syncthreads();
     const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
     const int r = lane < 16 ? 16 * sp + lane : -1;
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
@@ -778,25 +872,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_ld16(la + cRS + c0, rs);
       tc::tmem_ld16(la + cCS + c0, cs);
       if (r < 0) continue;
+      float qv[16], kv[16], dq[16], dk[16], dG[16];
+      staged16(sq, r, c0, qv);
+      staged16(sk, r, c0, kv);
+#pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int c = c0 + j;
         const float Gr = sG[r * LD + c], G0 = sref[c], GC = sG[(n - 1) * LD + c];
-        const float qv = ld_in(q_, srow, H, h, n, r, c), kv = ld_in(k_, srow, H, h, n, r, c);
-        const float dq = expf(Gr) * tq[j] + expf(Gr - G0) * rs[j];
+        dq[j] = expf(Gr) * tq[j] + expf(Gr - G0) * rs[j];
         const float dks = expf(GC - Gr) * t1[j];
-        const float dk = dks + expf(G0 - Gr) * cs[j];
-        pdk[r * D + c] = dk;
-        pdG[r * D + c] = qv * dq - kv * dk;
-        sbuf[r * LD + c] = r < n ? kv * dks : 0.f;
-        if (r >= ch.n_replay && r < n) dq_[((size_t)srow[r] * H + h) * D + c] = from_f<Tout>(dq);
+        dk[j] = dks + expf(G0 - Gr) * cs[j];
+        dG[j] = qv[j] * dq[j] - kv[j] * dk[j];
+        sbuf[r * LD + c] = r < n ? kv[j] * dks : 0.f;
       }
+      st16g(pdk + r * D + c0, dk);
+      st16g(pdG + r * D + c0, dG);
+      if (r >= ch.n_replay && r < n) st16_out(dq_ + ((size_t)srow[r] * H + h) * D + c0, dq);
     }
     __syncthreads();
     for (int c = tid; c < D; c += blockDim.x) {
       float acc = 0.f;
       for (int i = 0; i < n; ++i) acc += sbuf[i * LD + c];
       float acc2 = 0.f;
-      for (int j = 0; j < D; ++j) acc2 = fmaf(dSg[c * D + j], S0g[c * D + j], acc2);
+      for (int j = 0; j < D; j += 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(dSg + c * D + j));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(S0g + c * D + j));
+        acc2 = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc2))));
+      }
       pdG[(n - 1) * D + c] += acc + expf(sG[(n - 1) * LD + c]) * acc2;
     }
   }
@@ -818,7 +920,8 @@ struct BdkvTcSmem {
   static constexpr size_t G = 0;
   static constexpr size_t At = G + sizeof(float) * C * LD;        // Atilde fp32 [C][LC]
   static constexpr size_t vec = At + sizeof(float) * C * LC;      // beta[C], ref[D], dbeta parts[6][C]
-  static constexpr size_t Tt = (vec + sizeof(float) * (C + D + 6 * C) + 1023) & ~size_t(1023);  // T tile (MN)
+  static constexpr size_t Ks = (vec + sizeof(float) * (C + D + 6 * C) + 15) & ~size_t(15);      // staged k rows
+  static constexpr size_t Tt = (Ks + sizeof(__nv_bfloat16) * C * tck::kStagePitch + 1023) & ~size_t(1023);  // T tile
   static constexpr size_t CCb = size_t(C) * C * 2, CDb = size_t(C) * D * 2, DDb = size_t(D) * D * 2;
   static constexpr size_t R = Tt + 2 * CCb;
   static constexpr size_t Rbytes = 128 * 1024;
@@ -870,7 +973,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
   for (int e = tid; e < 6 * C; e += blockDim.x) sdb[e] = 0.f;
-  load_rows<C, D>(sG, g_, srow, H, h, 0, n);
+  Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
+  stage_rows(sk, k_, srow, H, h, n);
+  load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
   __syncthreads();
@@ -884,7 +989,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const float* dUg = ws.dU + base * C * D;
   float* pdk = ws.pdk + base * C * D;
   float* pdG = ws.pdG + base * C * D;
-  auto kin = [&](int r, int c) { return ld_in(k_, srow, H, h, n, r, c); };
   const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
   const int myrow = lane < 16 ? 16 * sp + lane : -1;  // M = 64 accumulator row of this thread
   const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
@@ -970,28 +1074,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       put16<C, true>(dbh, dbl, i, c0, v);
       float part = 0.f;
       if (c0 < D) {
+        float kv[16], a[16], b[16];
+        staged16(sk, i, c0, kv);
+        ld16g(pdk + i * D + c0, a);
+        ld16g(pdG + i * D + c0, b);
+#pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const int c = c0 + j;
-          const float eg = expf(sG[i * LD + c]);
-          const float kv = kin(i, c);
+          const float eg = expf(sG[i * LD + c0 + j]);
           const float bdb = sb[i] * v[j];
-          pdk[i * D + c] += eg * bdb;
-          pdG[i * D + c] += kv * eg * bdb;
-          part = fmaf(v[j], kv * eg, part);
+          a[j] += eg * bdb;
+          b[j] += kv[j] * eg * bdb;
+          part = fmaf(v[j], kv[j] * eg, part);
         }
+        st16g(pdk + i * D + c0, a);
+        st16g(pdG + i * D + c0, b);
       } else if (i < n) {
-        for (int j = 0; j < 16; ++j) {
-          const int c = c0 - D + j;
-          const float vv = ld_in(v_, srow, H, h, n, i, c);
-          part = fmaf(v[j], vv, part);
-          const float val = sb[i] * v[j];
-          if (i < ch.n_replay) {
-            ws.rdv[((size_t)(ch.replay_base + i) * H + h) * D + c] = val;
-          } else {
-            const int tg = t.row_tgt[srow[i]];
-            if (tg >= 0) ws.tdv[((size_t)tg * H + h) * D + c] = val;
-            else dv_[((size_t)srow[i] * H + h) * D + c] = from_f<Tout>(val);
+        const int c1 = c0 - D;
+        float vv[16], val[16];
+        if constexpr (sizeof(Tin) == 2) {
+          const uint4* src = reinterpret_cast<const uint4*>(v_ + ((size_t)srow[i] * H + h) * D + c1);
+          const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+          const __nv_bfloat162* b0 = reinterpret_cast<const __nv_bfloat162*>(&u0);
+          const __nv_bfloat162* b1 = reinterpret_cast<const __nv_bfloat162*>(&u1);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f0 = __bfloat1622float2(b0[k]), f1 = __bfloat1622float2(b1[k]);
+            vv[2 * k] = f0.x; vv[2 * k + 1] = f0.y; vv[8 + 2 * k] = f1.x; vv[8 + 2 * k + 1] = f1.y;
           }
+        } else {
+          ld16g(reinterpret_cast<const float*>(v_) + ((size_t)srow[i] * H + h) * D + c1, vv);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          part = fmaf(v[j], vv[j], part);
+          val[j] = sb[i] * v[j];
+        }
+        if (i < ch.n_replay) {
+          st16g(ws.rdv + ((size_t)(ch.replay_base + i) * H + h) * D + c1, val);
+        } else {
+          const int tg = t.row_tgt[srow[i]];
+          if (tg >= 0) st16g(ws.tdv + ((size_t)tg * H + h) * D + c1, val);
+          else st16_out(dv_ + ((size_t)srow[i] * H + h) * D + c1, val);
         }
       }
       sdb[((c0 < D ? 0 : 2) + grp) * C + i] += part;  // one slot per (half, warp group)
@@ -1043,21 +1166,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_ld16(la + cCS + c0, cs);
       if (myrow < 0) continue;
       const int r = myrow;
+      float kv[16], dkv[16], pg[16];
+      staged16(sk, r, c0, kv);
+      ld16g(pdk + r * D + c0, dkv);
+      ld16g(pdG + r * D + c0, pg);
+#pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int c = c0 + j;
         const float Gr = sG[r * LD + c], G0 = sref[c];
         const float a = expf(Gr - G0) * rs[j], b = expf(G0 - Gr) * cs[j];
-        const float kv = kin(r, c);
-        const float dkv = pdk[r * D + c] + a + b;
-        sdG[r * LD + c] = r < n ? pdG[r * D + c] + kv * (a - b) : 0.f;
-        if (r < n) {
-          if (r < ch.n_replay) {
-            ws.rdk[((size_t)(ch.replay_base + r) * H + h) * D + c] = dkv;
-          } else {
-            const int tg = t.row_tgt[srow[r]];
-            if (tg >= 0) ws.tdk[((size_t)tg * H + h) * D + c] = dkv;
-            else dk_[((size_t)srow[r] * H + h) * D + c] = from_f<Tout>(dkv);
-          }
+        dkv[j] += a + b;
+        sdG[r * LD + c] = r < n ? pg[j] + kv[j] * (a - b) : 0.f;
+      }
+      if (r < n) {
+        if (r < ch.n_replay) {
+          st16g(ws.rdk + ((size_t)(ch.replay_base + r) * H + h) * D + c0, dkv);
+        } else {
+          const int tg = t.row_tgt[srow[r]];
+          if (tg >= 0) st16g(ws.tdk + ((size_t)tg * H + h) * D + c0, dkv);
+          else st16_out(dk_ + ((size_t)srow[r] * H + h) * D + c0, dkv);
         }
       }
     }

@@ -94,7 +94,7 @@ WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
   L.tdv = take(T * H * D * 4);
   L.tdg = take(T * H * D * 4);
   L.tdb = take(T * H * 4);
-  const bool tensor_cores = (C == tpc::kTcC && D == tpc::kTcD);
+  const bool tensor_cores = (C == tpc::kTcC && D == tpc::kTcD);  // (bf16 inputs; sized for either)
   L.Mt = take(tensor_cores ? nc * H * (size_t)tpc::kMtileBytes : 0);
   L.Bc = take(tensor_cores ? nc * H * dd * 4 : 0);
   L.total = o;
@@ -150,7 +150,8 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
   const Tin* v = static_cast<const Tin*>(io->v);
   const Tin* g = static_cast<const Tin*>(io->g);
   const Tin* b = static_cast<const Tin*>(io->beta);
-  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
+  constexpr bool kTensorCores = (C == kTcC && D == kTcD && std::is_same<Tin, __nv_bfloat16>::value);
   if constexpr (kTensorCores) {
     TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmem::total));
     TPC_LAUNCH("kda_fwd_prep_tc", st,
@@ -203,7 +204,8 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   const Tin* g = static_cast<const Tin*>(io->g);
   const Tin* b = static_cast<const Tin*>(io->beta);
   const Tin* dO = static_cast<const Tin*>(io->d_o);
-  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
+  constexpr bool kTensorCores = (C == kTcC && D == kTcD && std::is_same<Tin, __nv_bfloat16>::value);
   if constexpr (kTensorCores) {
     TPC_CUDA(set_smem(kda_bwd_prep_tc<Tin>, BprepTcSmem::total));
     TPC_LAUNCH("kda_bwd_prep_tc", st,
