@@ -215,6 +215,46 @@ int tpc_gather_expanded(const tpc_plan* plan, const void* x_unique, void* x_exp,
 /* Occurrence count per compact row (int32 [N]). */
 int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t stream);
 
+/* ------------------------------------------------------------------ dense products */
+/*
+ * bf16 GEMM on tensor cores (the projections of the hybrid layer group and the vocabulary
+ * products of log-probability recovery, HARTS Figure C.1(d)):
+ *   C = alpha * op(A) op(B) + beta * C,  op(A) M x K, op(B) K x N, fp32 accumulation.
+ *   a_mn = 0: A stored [M][lda] (K contiguous); a_mn = 1: A stored [K][lda] (M contiguous).
+ *   b_mn = 0: B stored [N][ldb] (K contiguous); b_mn = 1: B stored [K][ldb] (N contiguous).
+ *   C: [M][ldc], c_dtype TPC_F32 (beta allowed) or TPC_BF16 (beta must be 0).
+ *   A, B 16-byte aligned with lda, ldb multiples of 8.  status: optional device int receiving
+ *   TPC_ERR_TIMEOUT if a bounded pipeline wait runs out.
+ */
+int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                  int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype, float alpha, float beta, int32_t* status,
+                  tpc_stream_t stream);
+
+/* ------------------------------------------------------------------ log-probability recovery */
+/*
+ * Log-probabilities of every original trajectory position from one logit row per unique row
+ * (HARTS abstract: log-probabilities recovered for each original trajectory position; Figure 1:
+ * one logit row z_B supplies every trajectory's target log-probability; Figure C.1(d): no
+ * expanded vocabulary-sized logits).  For compact row u with hidden state h_u and output matrix
+ * W [V][Dh]: z_u = W h_u, lse_u = log sum exp z_u, and for each occurrence j of u (trajectory
+ * order, tpc_plan_export's expanded_rows) with target y_j: logp_j = z_u[y_j] - lse_u.
+ *   h: bf16 [N_unique][Dh] (compact order), W: bf16 [V][Dh], targets: int32 [n_expanded] in [0, V).
+ *   logp: fp32 [n_expanded], lse: fp32 [N_unique].  V and Dh multiples of 8.
+ *   scratch: caller device memory of tpc_logprob_scratch_bytes(V, chunk_rows) bytes (256-aligned);
+ *   logits exist only for chunk_rows unique rows at a time.
+ *   status: optional device int; a target outside [0, V) records TPC_ERR_DEVICE_CHECK.
+ * Backward of sum_j dlogp_j logp_j: dh fp32 [N_unique][Dh] and dW fp32 [V][Dh] (overwritten),
+ * from the forward's lse.  Deterministic (fixed chunk and occurrence order).
+ */
+size_t tpc_logprob_scratch_bytes(int64_t V, int32_t chunk_rows);
+int tpc_logprob_forward(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh,
+                        const int32_t* targets, float* logp, float* lse, void* scratch, size_t scratch_bytes,
+                        int32_t chunk_rows, int32_t* status, tpc_stream_t stream);
+int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh,
+                         const int32_t* targets, const float* dlogp, const float* lse, float* dh, float* dW,
+                         void* scratch, size_t scratch_bytes, int32_t chunk_rows, int32_t* status,
+                         tpc_stream_t stream);
+
 /* ------------------------------------------------------------------ allocation-free forward */
 /* Bytes of device scratch built into the library for tpc_kda_forward_static (64 MiB). */
 #define TPC_STATIC_SCRATCH_BYTES (64u << 20)

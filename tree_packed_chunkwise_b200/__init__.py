@@ -82,6 +82,14 @@ SIGNATURES = {
     "tpc_gather_expanded": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int32, _V]),
     "tpc_occurrence_counts": (ctypes.c_int, [_V, _V, _V]),
     "tpc_kda_forward_static": (ctypes.c_int, [_V, _P(KdaShape), _P(KdaFwdIO), _V]),
+    "tpc_gemm_bf16": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                     ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_float, ctypes.c_float, _V, _V]),
+    "tpc_logprob_scratch_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int32]),
+    "tpc_logprob_forward": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V, _V, _V, _V, ctypes.c_size_t,
+                                           ctypes.c_int32, _V, _V]),
+    "tpc_logprob_backward": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V, _V, _V, _V, _V, _V,
+                                            ctypes.c_size_t, ctypes.c_int32, _V, _V]),
     "tpc_profile_enable": (None, [ctypes.c_int]),
     "tpc_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t]),
     "tpc_launch_count": (ctypes.c_longlong, []),
@@ -315,3 +323,55 @@ def tpc_profile_read() -> dict:
 
 def tpc_launch_count() -> int:
     return int(lib().tpc_launch_count())
+
+
+# ------------------------------------------------------------------------------------ dense products
+def tpc_gemm_bf16(a, b, c=None, a_mn=False, b_mn=False, out_dtype=None, alpha=1.0, beta=0.0, status=None, stream=None):
+    """C = alpha op(A) op(B) + beta C on tensor cores.  a: [M, K] (or [K, M] with a_mn), b: [N, K] (or [K, N]
+    with b_mn), bf16, last dimension contiguous.  Returns C [M, N] (fp32 unless out_dtype is bf16)."""
+    import torch
+    M = a.shape[1] if a_mn else a.shape[0]
+    K = a.shape[0] if a_mn else a.shape[1]
+    N = b.shape[1] if b_mn else b.shape[0]
+    if c is None:
+        c = torch.empty(M, N, dtype=out_dtype or torch.float32, device=a.device)
+    code = TPC_BF16 if c.dtype == torch.bfloat16 else TPC_F32
+    _check(lib().tpc_gemm_bf16(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, a.stride(0), b.stride(0),
+                               c.stride(0), int(a_mn), int(b_mn), code, float(alpha), float(beta),
+                               None if status is None else status.data_ptr(), _stream_ptr(stream)))
+    return c
+
+
+# ------------------------------------------------------------------------------------ log-probabilities
+def logprob_scratch(V, chunk_rows, device="cuda"):
+    import torch
+    n = int(lib().tpc_logprob_scratch_bytes(V, chunk_rows))
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def tpc_logprob_forward(plan: Plan, h, W, targets, chunk_rows=2048, scratch=None, status=None, stream=None):
+    """Per-occurrence log-probabilities (fp32 [n_expanded]) and per-row lse (fp32 [N_unique])."""
+    import torch
+    V, Dh = W.shape
+    chunk_rows = min(chunk_rows, plan.info["n_unique"])
+    scratch = scratch if scratch is not None else logprob_scratch(V, chunk_rows, h.device)
+    logp = torch.empty(plan.info["n_expanded"], dtype=torch.float32, device=h.device)
+    lse = torch.empty(plan.info["n_unique"], dtype=torch.float32, device=h.device)
+    _check(lib().tpc_logprob_forward(plan.handle, _ptr(h), _ptr(W), V, Dh, _ptr(targets), _ptr(logp), _ptr(lse),
+                                     _ptr(scratch), scratch.numel(), chunk_rows, _ptr(status), _stream_ptr(stream)))
+    return logp, lse
+
+
+def tpc_logprob_backward(plan: Plan, h, W, targets, dlogp, lse, chunk_rows=2048, scratch=None, status=None,
+                         stream=None):
+    """Gradients (fp32) of sum(dlogp * logp) w.r.t. h [N_unique, Dh] and W [V, Dh]."""
+    import torch
+    V, Dh = W.shape
+    chunk_rows = min(chunk_rows, plan.info["n_unique"])
+    scratch = scratch if scratch is not None else logprob_scratch(V, chunk_rows, h.device)
+    dh = torch.empty(plan.info["n_unique"], Dh, dtype=torch.float32, device=h.device)
+    dW = torch.empty(V, Dh, dtype=torch.float32, device=h.device)
+    _check(lib().tpc_logprob_backward(plan.handle, _ptr(h), _ptr(W), V, Dh, _ptr(targets), _ptr(dlogp), _ptr(lse),
+                                      _ptr(dh), _ptr(dW), _ptr(scratch), scratch.numel(), chunk_rows, _ptr(status),
+                                      _stream_ptr(stream)))
+    return dh, dW

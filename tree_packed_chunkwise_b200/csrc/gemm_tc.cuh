@@ -1,0 +1,133 @@
+// bf16 GEMM on 5th-generation tensor cores: C = alpha * op(A) op(B) (+ beta * C), fp32 accumulation
+// in TMEM.  A is M x K and B is K x N; each is given either K-major (K contiguous: A as [M][K], B
+// as [N][K]) or MN-major (M resp. N contiguous: A as [K][M], B as [K][N]).
+//
+// One CTA per 128 x 256 output tile, K in steps of 64 through a 4-stage shared-memory pipeline:
+// a producer thread issues TMA loads (one 16-byte-wide box per 8-element core-matrix column of the
+// no-swizzle canonical layout), an MMA thread issues tcgen05.mma and frees stages by tcgen05.commit,
+// all 128 threads run the epilogue (thread = row).  All waits are bounded.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace tpc {
+
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4, kGemmThreads = 128;
+
+struct GemmSmem {
+  static constexpr size_t Ab = size_t(kGemmBM) * kGemmBK * 2, Bb = size_t(kGemmBN) * kGemmBK * 2;
+  static constexpr size_t stage = Ab + Bb;
+  static constexpr size_t total = kGemmStages * stage;
+};
+
+struct GemmArgs {
+  int M, N, K;
+  int a_mn, b_mn;     // 1: MN-major
+  int c_dtype;        // 0 fp32, 1 bf16
+  long long ldc;      // elements
+  float alpha, beta;  // beta != 0 reads C (fp32 only)
+  void* C;
+  int* status;
+};
+
+template <int C_BF16>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, GemmArgs g) {
+  using namespace tc;
+  extern __shared__ __align__(1024) uint8_t gsm[];
+  __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], accb;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * kGemmBN;
+  const int KT = (g.K + kGemmBK - 1) / kGemmBK;
+  if (w == 0) tmem_alloc(&tslot, 256);
+  if (tid == 0) {
+    for (int s = 0; s < kGemmStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&accb, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = tslot;
+  bool ok = true;
+  if (w == 0 && lane == 0) {
+    // producer
+    for (int kt = 0; kt < KT && ok; ++kt) {
+      const int s = kt % kGemmStages;
+      if (kt >= kGemmStages && !mbar_wait(&empty[s], ((kt / kGemmStages) - 1) & 1)) {
+        set_status(g.status, 8);
+        ok = false;
+        break;
+      }
+      uint8_t* sa = gsm + s * GemmSmem::stage;
+      uint8_t* sb = sa + GemmSmem::Ab;
+      mbar_arrive_expect_tx(&full[s], (uint32_t)GemmSmem::stage);
+      const int k0 = kt * kGemmBK;
+      if (!g.a_mn) {
+        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sa + j * (kGemmBM / 8) * 128, &tma_a, k0 + 8 * j, m0, &full[s]);
+      } else {
+        for (int j = 0; j < kGemmBM / 8; ++j) tma_load_2d(sa + j * (kGemmBK / 8) * 128, &tma_a, m0 + 8 * j, k0, &full[s]);
+      }
+      if (!g.b_mn) {
+        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sb + j * (kGemmBN / 8) * 128, &tma_b, k0 + 8 * j, n0, &full[s]);
+      } else {
+        for (int j = 0; j < kGemmBN / 8; ++j) tma_load_2d(sb + j * (kGemmBK / 8) * 128, &tma_b, n0 + 8 * j, k0, &full[s]);
+      }
+    }
+  } else if (w == 1 && lane == 0) {
+    // MMA issuer
+    const uint32_t id = idesc_bf16(kGemmBM, kGemmBN, g.a_mn != 0, g.b_mn != 0);
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % kGemmStages;
+      if (!mbar_wait(&full[s], (kt / kGemmStages) & 1)) {
+        set_status(g.status, 8);
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      const uint8_t* sa = gsm + s * GemmSmem::stage;
+      const Op a{smem_u32(sa), g.a_mn ? kGemmBK : kGemmBM, g.a_mn != 0};
+      const Op b{smem_u32(sa + GemmSmem::Ab), g.b_mn ? kGemmBK : kGemmBN, g.b_mn != 0};
+      mma_chain(tb, a, b, kGemmBK, id, kt > 0);
+      commit(&empty[s]);
+    }
+    commit(&accb);
+  }
+  // epilogue: every thread waits for the accumulator (bounded)
+  const bool done = mbar_wait(&accb, 0, 4000000000ull);
+  const int failed = __syncthreads_or(done ? 0 : 1);
+  __syncwarp();
+  if (!failed) {
+    fence_after_sync();
+    const int m = m0 + 32 * w + lane;
+    const uint32_t la = tb + ((uint32_t)(32 * w) << 16);
+    for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+      float v[16];
+      tmem_ld16(la + c0, v);
+      if (m >= g.M || n0 + c0 >= g.N) continue;
+      const int nn = min(16, g.N - (n0 + c0));
+      if (C_BF16) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.C) + (size_t)m * g.ldc + n0 + c0;
+        for (int j = 0; j < nn; ++j) dst[j] = __float2bfloat16_rn(g.alpha * v[j]);
+      } else {
+        float* dst = static_cast<float*>(g.C) + (size_t)m * g.ldc + n0 + c0;
+        if (g.beta != 0.f)
+          for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j] + g.beta * dst[j];
+        else
+          for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j];
+      }
+    }
+  } else if (tid == 0) {
+    set_status(g.status, 8);
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (w == 0) tmem_dealloc(tb, 256);
+}
+
+}  // namespace tpc

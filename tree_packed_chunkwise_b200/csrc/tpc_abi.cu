@@ -12,6 +12,9 @@
 #include "kda_kernels.cuh"
 #include "kda_tc.cuh"
 #include "kda_scan_tc.cuh"
+#include "gemm_tc.cuh"
+#include "logprob_kernels.cuh"
+#include <cudaTypedefs.h>
 #include "plan.h"
 #include "rowmap_kernels.cuh"
 
@@ -343,6 +346,30 @@ int forward_static_impl(const tpc::Plan& p, const tpc::DevTables& dt, tpc::KdaWs
   return TPC_OK;
 }
 
+// ------------------------------------------------------------------------------------------------
+// TMA tensor maps (driver entry point looked up through the runtime; no link against libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems,
+                uint32_t box_rows) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void**>(&g_encode), cudaEnableDefault,
+                                &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      g_encode = nullptr;
+  });
+  if (!g_encode) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld_elems * 2};
+  cuuint32_t box[2] = {8, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -517,6 +544,105 @@ int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t st
   const int64_t N = plan->p.n_unique;
   TPC_LAUNCH("occurrence_count", st,
              (tpc::occurrence_count_kernel<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(plan->p.dt, counts, N)));
+  return TPC_OK;
+}
+
+int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                  int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype, float alpha, float beta, int32_t* status,
+                  tpc_stream_t stream) {
+  if (!A || !B || !C) return fail(TPC_ERR_NULL, "gemm: A, B and C are required");
+  if (M < 1 || N < 1 || K < 1 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30))
+    return fail(TPC_ERR_BAD_SHAPE, "gemm: sizes must be in [1, 2^30]");
+  if ((lda % 8) || (ldb % 8) || (reinterpret_cast<uintptr_t>(A) % 16) || (reinterpret_cast<uintptr_t>(B) % 16))
+    return fail(TPC_ERR_BAD_SHAPE, "gemm: A and B need 16-byte aligned bases and leading dimensions multiple of 8");
+  if (c_dtype != TPC_F32 && c_dtype != TPC_BF16) return fail(TPC_ERR_UNSUPPORTED, "gemm: C is fp32 or bf16");
+  if (c_dtype == TPC_BF16 && beta != 0.f) return fail(TPC_ERR_UNSUPPORTED, "gemm: beta needs an fp32 C");
+  if (a_mn ? (lda < M) : (lda < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: lda too small");
+  if (b_mn ? (ldb < N) : (ldb < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldb too small");
+  if (ldc < N) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldc too small");
+  CUtensorMap ta, tb;
+  const bool ok_a = a_mn ? tensor_map(&ta, A, M, K, lda, tpc::kGemmBK) : tensor_map(&ta, A, K, M, lda, tpc::kGemmBM);
+  const bool ok_b = b_mn ? tensor_map(&tb, B, N, K, ldb, tpc::kGemmBK) : tensor_map(&tb, B, K, N, ldb, tpc::kGemmBN);
+  if (!ok_a || !ok_b) return fail(TPC_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
+  tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid((unsigned)((N + tpc::kGemmBN - 1) / tpc::kGemmBN), (unsigned)((M + tpc::kGemmBM - 1) / tpc::kGemmBM));
+  if (c_dtype == TPC_BF16) {
+    TPC_CUDA(set_smem(tpc::gemm_bf16_tc<1>, tpc::GemmSmem::total));
+    TPC_LAUNCH("gemm_bf16_tc", st, (tpc::gemm_bf16_tc<1><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, g)));
+  } else {
+    TPC_CUDA(set_smem(tpc::gemm_bf16_tc<0>, tpc::GemmSmem::total));
+    TPC_LAUNCH("gemm_bf16_tc", st, (tpc::gemm_bf16_tc<0><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, g)));
+  }
+  return TPC_OK;
+}
+
+size_t tpc_logprob_scratch_bytes(int64_t V, int32_t chunk_rows) {
+  if (V < 1 || chunk_rows < 1) return 0;
+  return a256((size_t)chunk_rows * V * 4) + 2 * a256((size_t)chunk_rows * V * 2);
+}
+
+namespace {
+int logprob_check(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh, const int32_t* targets,
+                  void* scratch, size_t scratch_bytes, int32_t chunk_rows) {
+  if (!plan || !h || !W || !targets || !scratch) return fail(TPC_ERR_NULL, "logprob: NULL argument");
+  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
+  if (V < 8 || Dh < 8 || (V % 8) || (Dh % 8)) return fail(TPC_ERR_BAD_SHAPE, "logprob: V and Dh multiples of 8");
+  if (chunk_rows < 1) return fail(TPC_ERR_BAD_SHAPE, "logprob: chunk_rows >= 1");
+  if (scratch_bytes < tpc_logprob_scratch_bytes(V, chunk_rows)) return fail(TPC_ERR_WORKSPACE, "logprob: scratch too small");
+  if (reinterpret_cast<uintptr_t>(scratch) % 256) return fail(TPC_ERR_WORKSPACE, "logprob: scratch must be 256-byte aligned");
+  return TPC_OK;
+}
+}  // namespace
+
+int tpc_logprob_forward(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh,
+                        const int32_t* targets, float* logp, float* lse, void* scratch, size_t scratch_bytes,
+                        int32_t chunk_rows, int32_t* status, tpc_stream_t stream) {
+  if (int rc = logprob_check(plan, h, W, V, Dh, targets, scratch, scratch_bytes, chunk_rows)) return rc;
+  if (!logp || !lse) return fail(TPC_ERR_NULL, "logprob: logp and lse are required");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const tpc::Plan& p = plan->p;
+  float* Z = static_cast<float*>(scratch);
+  const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(h);
+  for (int64_t r0 = 0; r0 < p.n_unique; r0 += chunk_rows) {
+    const int R = (int)std::min<int64_t>(chunk_rows, p.n_unique - r0);
+    if (int rc = tpc_gemm_bf16(hb + r0 * Dh, W, Z, R, V, Dh, Dh, Dh, V, 0, 0, TPC_F32, 1.f, 0.f, status, stream)) return rc;
+    TPC_LAUNCH("lse_rows", st, (tpc::lse_rows_kernel<<<R, tpc::kLseThreads, 0, st>>>(Z, V, lse, (int)r0)));
+    TPC_LAUNCH("logprob_gather", st,
+               (tpc::logprob_gather_kernel<<<(R + 127) / 128, 128, 0, st>>>(p.dt, Z, V, (int)r0, R, lse, targets, logp,
+                                                                             status)));
+  }
+  return TPC_OK;
+}
+
+int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh,
+                         const int32_t* targets, const float* dlogp, const float* lse, float* dh, float* dW,
+                         void* scratch, size_t scratch_bytes, int32_t chunk_rows, int32_t* status,
+                         tpc_stream_t stream) {
+  if (int rc = logprob_check(plan, h, W, V, Dh, targets, scratch, scratch_bytes, chunk_rows)) return rc;
+  if (!dlogp || !lse || !dh || !dW) return fail(TPC_ERR_NULL, "logprob backward: dlogp, lse, dh and dW are required");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const tpc::Plan& p = plan->p;
+  char* sc = static_cast<char*>(scratch);
+  float* Z = reinterpret_cast<float*>(sc);
+  __nv_bfloat16* zh = reinterpret_cast<__nv_bfloat16*>(sc + a256((size_t)chunk_rows * V * 4));
+  __nv_bfloat16* zl = reinterpret_cast<__nv_bfloat16*>(sc + a256((size_t)chunk_rows * V * 4) + a256((size_t)chunk_rows * V * 2));
+  const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(h);
+  TPC_CUDA(cudaMemsetAsync(dW, 0, (size_t)V * Dh * 4, st));
+  for (int64_t r0 = 0; r0 < p.n_unique; r0 += chunk_rows) {
+    const int R = (int)std::min<int64_t>(chunk_rows, p.n_unique - r0);
+    if (int rc = tpc_gemm_bf16(hb + r0 * Dh, W, Z, R, V, Dh, Dh, Dh, V, 0, 0, TPC_F32, 1.f, 0.f, status, stream)) return rc;
+    TPC_LAUNCH("dz_rows", st,
+               (tpc::dz_rows_kernel<<<R, tpc::kLseThreads, 0, st>>>(p.dt, Z, V, (int)r0, lse, targets, dlogp, zh, zl,
+                                                                    status)));
+    // dH = dZ W  (W as an MN-major B: [V][Dh], N = Dh contiguous)
+    float* dhc = dh + r0 * Dh;
+    if (int rc = tpc_gemm_bf16(zh, W, dhc, R, Dh, V, V, Dh, Dh, 0, 1, TPC_F32, 1.f, 0.f, status, stream)) return rc;
+    if (int rc = tpc_gemm_bf16(zl, W, dhc, R, Dh, V, V, Dh, Dh, 0, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
+    // dW += dZ^T H  (dZ as an MN-major A: [R][V]; H as an MN-major B: [R][Dh])
+    if (int rc = tpc_gemm_bf16(zh, hb + r0 * Dh, dW, V, Dh, R, V, Dh, Dh, 1, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
+    if (int rc = tpc_gemm_bf16(zl, hb + r0 * Dh, dW, V, Dh, R, V, Dh, Dh, 1, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
+  }
   return TPC_OK;
 }
 
