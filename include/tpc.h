@@ -230,6 +230,31 @@ int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, i
                   int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype, float alpha, float beta, int32_t* status,
                   tpc_stream_t stream);
 
+/* ------------------------------------------------------------------ tree-masked attention */
+/*
+ * Softmax attention in which each token reads only its ancestors' keys and values and the earlier
+ * tokens of its own segment (HARTS Figure 1(b); Figure C.1(c): diagonal blocks causal, outputs
+ * return to compact rows).  Along any trajectory this is causal attention over the trajectory's
+ * prefix.  Compact-row tensors, bf16 inputs:
+ *   q, k: [N][H][d_qk], v: [N][H][d_v]; o: [N][H][d_v] and (backward) dq, dk, dv in io_dtype;
+ *   lse: fp32 [N][H] (natural log of the softmax normaliser of scale * q.k).
+ *   delta: caller scratch fp32 [N][H] (backward).  Built for d_qk = 192, d_v = 128.
+ * Deterministic: the backward sums every gradient in a fixed order without atomics.
+ */
+typedef struct tpc_attn_shape {
+  int32_t H;
+  int32_t d_qk, d_v;
+  float scale;
+  int32_t io_dtype; /* dtype of o (forward) and of o, dq, dk, dv (backward) */
+} tpc_attn_shape;
+int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* shape, const void* q, const void* k,
+                          const void* v, void* o, float* lse, int32_t* status, tpc_stream_t stream);
+int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* shape, const void* q, const void* k,
+                           const void* v, const void* o, const float* lse, const void* d_o, void* dq, void* dk,
+                           void* dv, float* delta, int32_t* status, tpc_stream_t stream);
+/* Trajectory position (depth from the root) of every compact row, int32 [N] (rotary positions). */
+int tpc_rope_positions(const tpc_plan* plan, int32_t* pos, tpc_stream_t stream);
+
 /* ------------------------------------------------------------------ log-probability recovery */
 /*
  * Log-probabilities of every original trajectory position from one logit row per unique row

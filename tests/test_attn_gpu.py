@@ -1,0 +1,55 @@
+"""Tree-masked attention on the GPU against the per-trajectory causal softmax oracle."""
+import numpy as np
+import pytest
+
+import synth
+from kda_case import TOL, err_ratio
+from oracle import attention as oat
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tpc():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    import tree_packed_chunkwise_b200 as t
+    t.lib()
+    return t
+
+
+@pytest.mark.parametrize("cfg,H", [("fig1", 2), ("agentic_small", 2)])
+def test_tree_attention_matches_oracle(tpc, cfg, H):
+    import torch
+    tree = synth.workload(cfg).tree
+    N = tree.n_rows
+    seed = 31
+    q = synth.normal_tensor(seed, 40, (N, H, 192), "bf16")
+    k = synth.normal_tensor(seed, 41, (N, H, 192), "bf16")
+    v = synth.normal_tensor(seed, 42, (N, H, 128), "bf16")
+    d_o = synth.normal_tensor(seed, 43, (N, H, 128), "bf16")
+    scale = 1.0 / np.sqrt(192.0)
+    o_ref, lse_ref = oat.tree_forward(tree, q, k, v, scale)
+    dq_ref, dk_ref, dv_ref = oat.tree_backward(tree, q, k, v, scale, d_o)
+    plan = tpc.Plan(tree.parent, tree.length, 64).upload()
+    st = tree.node_start()
+    dev = lambda a: torch.tensor(plan.to_compact(a, st, tree.length), dtype=torch.float32).to(torch.bfloat16).cuda()
+    comp = lambda a: plan.to_compact(a, st, tree.length)
+    qd, kd, vd, gd = dev(q), dev(k), dev(v), dev(d_o)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = tpc.tpc_tree_attn_forward(plan, qd, kd, vd, scale, out_dtype=torch.float32, status=status)
+    dq, dk, dv = tpc.tpc_tree_attn_backward(plan, qd, kd, vd, o, lse, gd, scale, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    errs = {"o": err_ratio(o.cpu().numpy(), comp(o_ref)), "lse": err_ratio(lse.cpu().numpy(), comp(lse_ref)),
+            "dq": err_ratio(dq.cpu().numpy(), comp(dq_ref)), "dk": err_ratio(dk.cpu().numpy(), comp(dk_ref)),
+            "dv": err_ratio(dv.cpu().numpy(), comp(dv_ref))}
+    print(cfg, errs)
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
+    # rotary positions: the depth of every row on its trajectories
+    pos = tpc.tpc_rope_positions(plan).cpu().numpy()
+    depth = np.concatenate([np.arange(int(sum(tree.length[u] for u in tree.path(v)[:-1])),
+                                      int(sum(tree.length[u] for u in tree.path(v))))
+                            for v in range(tree.n)])
+    assert np.array_equal(pos, comp(depth))

@@ -49,6 +49,11 @@ class KdaShape(ctypes.Structure):
                 ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
 
 
+class AttnShape(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("io_dtype", ctypes.c_int32)]
+
+
 class KdaFwdIO(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("g", ctypes.c_void_p),
                 ("beta", ctypes.c_void_p), ("init_state", ctypes.c_void_p), ("o", ctypes.c_void_p),
@@ -90,6 +95,9 @@ SIGNATURES = {
                                            ctypes.c_int32, _V, _V]),
     "tpc_logprob_backward": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V, _V, _V, _V, _V, _V,
                                             ctypes.c_size_t, ctypes.c_int32, _V, _V]),
+    "tpc_tree_attn_forward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V]),
+    "tpc_tree_attn_backward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V]),
+    "tpc_rope_positions": (ctypes.c_int, [_V, _V, _V]),
     "tpc_profile_enable": (None, [ctypes.c_int]),
     "tpc_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t]),
     "tpc_launch_count": (ctypes.c_longlong, []),
@@ -375,3 +383,45 @@ def tpc_logprob_backward(plan: Plan, h, W, targets, dlogp, lse, chunk_rows=2048,
                                       _ptr(dh), _ptr(dW), _ptr(scratch), scratch.numel(), chunk_rows, _ptr(status),
                                       _stream_ptr(stream)))
     return dh, dW
+
+
+# ------------------------------------------------------------------------------------ tree attention
+def _attn_shape(q, v, scale, io_dtype):
+    import torch
+    return AttnShape(q.shape[1], q.shape[2], v.shape[2], float(scale),
+                     TPC_BF16 if io_dtype == torch.bfloat16 else TPC_F32)
+
+
+def tpc_tree_attn_forward(plan: Plan, q, k, v, scale, out_dtype=None, status=None, stream=None):
+    """Tree-masked attention forward; returns (o, lse)."""
+    import torch
+    out_dtype = out_dtype or torch.float32
+    N, H, _ = q.shape
+    o = torch.empty(N, H, v.shape[2], dtype=out_dtype, device=q.device)
+    lse = torch.empty(N, H, dtype=torch.float32, device=q.device)
+    sh = _attn_shape(q, v, scale, out_dtype)
+    _check(lib().tpc_tree_attn_forward(plan.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                       _ptr(status), _stream_ptr(stream)))
+    return o, lse
+
+
+def tpc_tree_attn_backward(plan: Plan, q, k, v, o, lse, d_o, scale, status=None, stream=None):
+    """Gradients (dq, dk, dv) in o's dtype."""
+    import torch
+    N, H, _ = q.shape
+    dq = torch.empty(q.shape, dtype=o.dtype, device=q.device)
+    dk = torch.empty(k.shape, dtype=o.dtype, device=q.device)
+    dv = torch.empty(v.shape, dtype=o.dtype, device=q.device)
+    delta = torch.empty(N, H, dtype=torch.float32, device=q.device)
+    sh = _attn_shape(q, v, scale, o.dtype)
+    _check(lib().tpc_tree_attn_backward(plan.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                        _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(delta), _ptr(status),
+                                        _stream_ptr(stream)))
+    return dq, dk, dv
+
+
+def tpc_rope_positions(plan: Plan, device="cuda", stream=None):
+    import torch
+    pos = torch.empty(plan.info["n_unique"], dtype=torch.int32, device=device)
+    _check(lib().tpc_rope_positions(plan.handle, _ptr(pos), _stream_ptr(stream)))
+    return pos

@@ -1,0 +1,397 @@
+// Tree-masked softmax attention on tcgen05 (HARTS Figure 1(b): full attention reads ancestor keys
+// and values; Figure C.1(c): within a segment the diagonal blocks are causal, a later segment reads
+// its ancestors and never the reverse; outputs return to compact rows).
+//
+// A query tile (<= 128 rows of one node) visits the node's ancestor row ranges (a few contiguous
+// ranges in the compact layout, one per chain on its path) and then its own node's rows up to the
+// tile's end with the causal mask.  Forward: S = Q K^T (bf16 inputs, exact products), online
+// softmax in fp32 (one query row per thread), O += P V with P a bf16 hi/lo pair.  Backward,
+// deterministic: dQ per query tile (S and dP = dO V^T recomputed, dQ += dS K accumulated in TMEM);
+// dK, dV per key tile (<= 64 rows of one node), looping over the query rows that can see it: the
+// node's subtree rows from the tile on, one contiguous range in the compact layout.
+#pragma once
+#include "kda_tc.cuh"
+
+namespace tpc {
+
+constexpr int kAttnQK = 192, kAttnDV = 128, kAttnThreads = 128;
+
+namespace tck {
+
+// key tiles of a query tile: f(row start, rows, own-node flag) in a fixed order; stops on false
+template <class F>
+__device__ __forceinline__ bool for_key_tiles(const DevTables& t, const AttnTile& qt, F f) {
+  const AttnNode nd = t.attn_nodes[qt.node];
+  const int r1 = t.attn_nodes[qt.node + 1].range_begin;
+  for (int r = nd.range_begin; r < r1; ++r) {
+    const RowRange rr = t.attn_ranges[r];
+    for (int k0 = rr.start; k0 < rr.end; k0 += 64)
+      if (!f(k0, min(64, rr.end - k0), false)) return false;
+  }
+  const int end = qt.row + qt.n;
+  for (int k0 = nd.row_offset; k0 < end; k0 += 64)
+    if (!f(k0, min(64, end - k0), true)) return false;
+  return true;
+}
+
+template <typename T>
+__device__ __forceinline__ void st_out16(T* p, const float* v) {
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4)
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p) + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  } else {
+    __align__(16) __nv_bfloat16 b[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) b[j] = __float2bfloat16_rn(v[j]);
+    reinterpret_cast<uint4*>(p)[0] = reinterpret_cast<const uint4*>(b)[0];
+    reinterpret_cast<uint4*>(p)[1] = reinterpret_cast<const uint4*>(b)[1];
+  }
+}
+
+}  // namespace tck
+
+// ------------------------------------------------------------------------------------------ forward
+struct AttnFwdSmem {
+  static constexpr size_t Qb = size_t(128) * kAttnQK * 2, Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
+  static constexpr size_t Pb = size_t(128) * 64 * 2;
+  static constexpr size_t Q = 0, K = Q + Qb, V = K + Kb, P = V + Vb;
+  static constexpr size_t total = P + 2 * Pb;
+};
+
+template <typename Tout>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
+                const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, Tout* __restrict__ o,
+                float* __restrict__ lse, int* status) {
+  using namespace tck;
+  using S = AttnFwdSmem;
+  using bf = __nv_bfloat16;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
+  const AttnTile qt = t.attn_qtiles[blockIdx.x];
+  const int h = blockIdx.y, tid = threadIdx.x;
+  extern __shared__ __align__(1024) uint8_t asmem[];
+  uint8_t *sQ = asmem + S::Q, *sK = asmem + S::K, *sV = asmem + S::V, *sPh = asmem + S::P, *sPl = sPh + S::Pb;
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 256);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  auto ident = [](int, int, float x) { return x; };
+  build_tile_ld<128, DQ, false, bf, NT>(
+      sQ, nullptr, [&](int a) -> const bf* { return a < qt.n ? q + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; },
+      ident);
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  const uint32_t la = tb + ((uint32_t)(32 * (tid >> 5)) << 16);
+  Sync sy{&bar, 0u, status};
+  const int qrow = qt.row + tid;
+  float acc[DV];
+#pragma unroll
+  for (int j = 0; j < DV; ++j) acc[j] = 0.f;
+  float m = -INFINITY, l = 0.f;
+  const bool ok = for_key_tiles(t, qt, [&](int k0, int nk, bool own) -> bool {
+    build_tile_ld<64, DQ, false, bf, NT>(
+        sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
+    build_tile_ld<64, DV, false, bf, NT>(
+        sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+    if (!run(sy, [&] {
+          mma_chain(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sK), 64, false}, DQ,
+                    tc::idesc_bf16(128, 64, false, false), false);
+        }))
+      return false;
+    float s[64];
+    tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
+    tc::tmem_ld32(la + 32, *reinterpret_cast<float(*)[32]>(s + 32));
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+      const bool valid = j < nk && (!own || k0 + j <= qrow);
+      s[j] = valid ? s[j] * scale : -INFINITY;
+      mx = fmaxf(mx, s[j]);
+    }
+    const float m_new = fmaxf(m, mx);
+    const float corr = (m == -INFINITY) ? 0.f : expf(m - m_new);
+    float psum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+      s[j] = (s[j] == -INFINITY) ? 0.f : expf(s[j] - m_new);
+      psum += s[j];
+    }
+    l = l * corr + psum;
+    m = m_new;
+#pragma unroll
+    for (int j = 0; j < 64; j += 16) put16<128, true>(sPh, sPl, tid, j, s + j);
+    if (!run(sy, [&] {
+          mma4(tb + 64, tc::Op{tc::smem_u32(sPh), 128, false}, tc::Op{tc::smem_u32(sPl), 128, false},
+               tc::Op{tc::smem_u32(sV), 64, true}, tc::Op{tc::smem_u32(sV), 64, true}, 64,
+               tc::idesc_bf16(128, DV, false, true), false, false, true);
+        }))
+      return false;
+#pragma unroll
+    for (int c = 0; c < DV; c += 32) {
+      float pv[32];
+      tc::tmem_ld32(la + 64 + c, pv);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc[c + j] = acc[c + j] * corr + pv[j];
+    }
+    tc::fence_before_sync();
+    __syncthreads();  // tiles are rewritten by the next key tile
+    return true;
+  });
+  if (ok && tid < qt.n) {
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int j = 0; j < DV; ++j) acc[j] *= inv;
+    Tout* dst = o + ((size_t)qrow * H + h) * DV;
+#pragma unroll
+    for (int c = 0; c < DV; c += 16) st_out16(dst + c, acc + c);
+    lse[(size_t)qrow * H + h] = m + logf(l);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 256);
+}
+
+// ------------------------------------------------------------------------------------------ backward dQ
+// per query tile: delta = rowsum(dO * O) (also written for the dK/dV kernel), then over the key
+// tiles P = exp(scale S - lse), dP = dO V^T, dS = P (dP - delta), dQ += dS K; dq = scale dQ.
+struct AttnDqSmem {
+  static constexpr size_t Qb = size_t(128) * kAttnQK * 2, Ob = size_t(128) * kAttnDV * 2;
+  static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2, Pb = size_t(128) * 64 * 2;
+  static constexpr size_t Q = 0, dO = Q + Qb, K = dO + Ob, V = K + Kb, dS = V + Vb;
+  static constexpr size_t total = dS + 2 * Pb;
+};
+
+template <typename Tio>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_bwd_dq_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
+                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                   const Tio* __restrict__ o, const float* __restrict__ lse, const __nv_bfloat16* __restrict__ d_o,
+                   Tio* __restrict__ dq, float* __restrict__ delta, int* status) {
+  using namespace tck;
+  using S = AttnDqSmem;
+  using bf = __nv_bfloat16;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
+  const AttnTile qt = t.attn_qtiles[blockIdx.x];
+  const int h = blockIdx.y, tid = threadIdx.x;
+  extern __shared__ __align__(1024) uint8_t asmem[];
+  uint8_t *sQ = asmem + S::Q, *sO = asmem + S::dO, *sK = asmem + S::K, *sV = asmem + S::V, *sDh = asmem + S::dS,
+          *sDl = sDh + S::Pb;
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  auto ident = [](int, int, float x) { return x; };
+  build_tile_ld<128, DQ, false, bf, NT>(
+      sQ, nullptr, [&](int a) -> const bf* { return a < qt.n ? q + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; },
+      ident);
+  build_tile_ld<128, DV, false, bf, NT>(
+      sO, nullptr, [&](int a) -> const bf* { return a < qt.n ? d_o + ((size_t)(qt.row + a) * H + h) * DV : nullptr; },
+      ident);
+  const int qrow = qt.row + tid;
+  float dl = 0.f, ls = 0.f;
+  if (tid < qt.n) {
+    const Tio* orow = o + ((size_t)qrow * H + h) * DV;
+    const bf* grow = d_o + ((size_t)qrow * H + h) * DV;
+    for (int j = 0; j < DV; ++j) dl = fmaf(to_f(orow[j]), __bfloat162float(grow[j]), dl);
+    delta[(size_t)qrow * H + h] = dl;
+    ls = lse[(size_t)qrow * H + h];
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  const uint32_t la = tb + ((uint32_t)(32 * (tid >> 5)) << 16);
+  Sync sy{&bar, 0u, status};
+  bool first = true;
+  const bool ok = for_key_tiles(t, qt, [&](int k0, int nk, bool own) -> bool {
+    build_tile_ld<64, DQ, false, bf, NT>(
+        sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
+    build_tile_ld<64, DV, false, bf, NT>(
+        sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+    if (!run(sy, [&] {
+          mma_chain(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sK), 64, false}, DQ,
+                    tc::idesc_bf16(128, 64, false, false), false);
+          mma_chain(tb + 64, tc::Op{tc::smem_u32(sO), 128, false}, tc::Op{tc::smem_u32(sV), 64, false}, DV,
+                    tc::idesc_bf16(128, 64, false, false), false);
+        }))
+      return false;
+    float s[64], dp[64];
+    tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
+    tc::tmem_ld32(la + 32, *reinterpret_cast<float(*)[32]>(s + 32));
+    tc::tmem_ld32(la + 64, *reinterpret_cast<float(*)[32]>(dp));
+    tc::tmem_ld32(la + 96, *reinterpret_cast<float(*)[32]>(dp + 32));
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+      const bool valid = tid < qt.n && j < nk && (!own || k0 + j <= qrow);
+      const float p = valid ? expf(s[j] * scale - ls) : 0.f;
+      s[j] = p * (dp[j] - dl);
+    }
+#pragma unroll
+    for (int j = 0; j < 64; j += 16) put16<128, true>(sDh, sDl, tid, j, s + j);
+    const bool acc_on = !first;
+    first = false;
+    if (!run(sy, [&] {
+          mma4(tb + 128, tc::Op{tc::smem_u32(sDh), 128, false}, tc::Op{tc::smem_u32(sDl), 128, false},
+               tc::Op{tc::smem_u32(sK), 64, true}, tc::Op{tc::smem_u32(sK), 64, true}, 64,
+               tc::idesc_bf16(128, DQ, false, true), acc_on, false, true);
+        }))
+      return false;
+    tc::fence_before_sync();
+    __syncthreads();
+    return true;
+  });
+  if (ok) {
+    for (int c = 0; c < DQ; c += 32) {
+      float g[32];
+      tc::tmem_ld32(la + 128 + c, g);
+      if (tid < qt.n) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) g[j] *= scale;
+        Tio* dst = dq + ((size_t)qrow * H + h) * DQ + c;
+        st_out16(dst, g);
+        st_out16(dst + 16, g + 16);
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
+}
+
+// ------------------------------------------------------------------------------------------ backward dK, dV
+// per key tile of node u: query rows [row of the tile, subtree end of u) in tiles of 64 (queries of u
+// itself only from the key row on), S^T = K Q^T, dP^T = V dO^T, P^T = exp(scale S^T - lse),
+// dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 64 accumulators.
+struct AttnDkvSmem {
+  static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2, Pb = size_t(64) * 64 * 2;
+  static constexpr size_t K = 0, V = K + Kb, Q = V + Vb, dO = Q + Kb, P = dO + Vb, dS = P + 2 * Pb;
+  static constexpr size_t vec = dS + 2 * Pb;  // lse[64], delta[64]
+  static constexpr size_t total = vec + 2 * 64 * 4;
+};
+
+template <typename Tio>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_bwd_dkv_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
+                    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                    const float* __restrict__ lse, const __nv_bfloat16* __restrict__ d_o,
+                    const float* __restrict__ delta, Tio* __restrict__ dk, Tio* __restrict__ dv, int* status) {
+  using namespace tck;
+  using S = AttnDkvSmem;
+  using bf = __nv_bfloat16;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
+  const AttnTile kt = t.attn_ktiles[blockIdx.x];
+  const AttnNode nd = t.attn_nodes[kt.node];
+  const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  extern __shared__ __align__(1024) uint8_t asmem[];
+  uint8_t *sK = asmem + S::K, *sV = asmem + S::V, *sQ = asmem + S::Q, *sO = asmem + S::dO;
+  uint8_t *sPh = asmem + S::P, *sPl = sPh + S::Pb, *sDh = asmem + S::dS, *sDl = sDh + S::Pb;
+  float* sl = reinterpret_cast<float*>(asmem + S::vec);
+  float* sd = sl + 64;
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tslot;
+  if (w == 0) tc::tmem_alloc(&tslot, 512);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  auto ident = [](int, int, float x) { return x; };
+  const int k0 = kt.row, nk = kt.n;
+  build_tile_ld<64, DQ, false, bf, NT>(
+      sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
+  build_tile_ld<64, DV, false, bf, NT>(
+      sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
+  const int r = lane < 16 ? 16 * (w & 3) + lane : -1;  // key row of this thread (M = 64 layout)
+  const int own_end = nd.row_offset + nd.length, q_end = nd.subtree_end;
+  Sync sy{&bar, 0u, status};
+  bool ok = true, first = true;
+  for (int q0 = k0; q0 < q_end && ok; q0 += 64) {
+    const int nq = min(64, q_end - q0);
+    build_tile_ld<64, DQ, false, bf, NT>(
+        sQ, nullptr, [&](int a) -> const bf* { return a < nq ? q + ((size_t)(q0 + a) * H + h) * DQ : nullptr; },
+        ident);
+    build_tile_ld<64, DV, false, bf, NT>(
+        sO, nullptr, [&](int a) -> const bf* { return a < nq ? d_o + ((size_t)(q0 + a) * H + h) * DV : nullptr; },
+        ident);
+    if (tid < 64) {
+      sl[tid] = tid < nq ? lse[(size_t)(q0 + tid) * H + h] : 0.f;
+      sd[tid] = tid < nq ? delta[(size_t)(q0 + tid) * H + h] : 0.f;
+    }
+    ok = run(sy, [&] {
+      mma_chain(tb, tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sQ), 64, false}, DQ,
+                tc::idesc_bf16(64, 64, false, false), false);
+      mma_chain(tb + 64, tc::Op{tc::smem_u32(sV), 64, false}, tc::Op{tc::smem_u32(sO), 64, false}, DV,
+                tc::idesc_bf16(64, 64, false, false), false);
+    });
+    if (!ok) break;
+    float s[64], dp[64];
+    tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
+    tc::tmem_ld32(la + 32, *reinterpret_cast<float(*)[32]>(s + 32));
+    tc::tmem_ld32(la + 64, *reinterpret_cast<float(*)[32]>(dp));
+    tc::tmem_ld32(la + 96, *reinterpret_cast<float(*)[32]>(dp + 32));
+    if (r >= 0) {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const int qrow = q0 + j;
+        const bool valid = r < nk && j < nq && !(qrow < own_end && qrow < k0 + r);
+        const float p = valid ? expf(s[j] * scale - sl[j]) : 0.f;
+        s[j] = p;
+        dp[j] = p * (dp[j] - sd[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 64; j += 16) {
+        put16<64, true>(sPh, sPl, r, j, s + j);
+        put16<64, true>(sDh, sDl, r, j, dp + j);
+      }
+    }
+    const bool acc_on = !first;
+    first = false;
+    ok = run(sy, [&] {
+      mma4(tb + 128, tc::Op{tc::smem_u32(sPh), 64, false}, tc::Op{tc::smem_u32(sPl), 64, false},
+           tc::Op{tc::smem_u32(sO), 64, true}, tc::Op{tc::smem_u32(sO), 64, true}, 64,
+           tc::idesc_bf16(64, DV, false, true), acc_on, false, true);
+      mma4(tb + 256, tc::Op{tc::smem_u32(sDh), 64, false}, tc::Op{tc::smem_u32(sDl), 64, false},
+           tc::Op{tc::smem_u32(sQ), 64, true}, tc::Op{tc::smem_u32(sQ), 64, true}, 64,
+           tc::idesc_bf16(64, DQ, false, true), acc_on, false, true);
+    });
+    tc::fence_before_sync();
+    __syncthreads();
+  }
+  if (ok) {
+    for (int c = 0; c < DV; c += 32) {
+      float g[32];
+      tc::tmem_ld32(la + 128 + c, g);
+      if (r >= 0 && r < nk) {
+        Tio* dst = dv + ((size_t)(k0 + r) * H + h) * DV + c;
+        st_out16(dst, g);
+        st_out16(dst + 16, g + 16);
+      }
+    }
+    for (int c = 0; c < DQ; c += 32) {
+      float g[32];
+      tc::tmem_ld32(la + 256 + c, g);
+      if (r >= 0 && r < nk) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) g[j] *= scale;
+        Tio* dst = dk + ((size_t)(k0 + r) * H + h) * DQ + c;
+        st_out16(dst, g);
+        st_out16(dst + 16, g + 16);
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (w == 0) tc::tmem_dealloc(tb, 512);
+}
+
+}  // namespace tpc

@@ -71,15 +71,15 @@ __device__ __forceinline__ void ld8(const T* p, float (&x)[8]) {
   }
 }
 
-template <int A, int B, bool SPLIT, typename T, class RP, class F>
+template <int A, int B, bool SPLIT, typename T, int NT = kThreads, class RP, class F>
 __device__ __forceinline__ void build_tile_ld(uint8_t* hi, uint8_t* lo, RP rowp, F f) {
   constexpr int NCH = A * (B / 8);
-  static_assert(NCH % kThreads == 0, "tile chunks must be a multiple of the CTA size");
-  constexpr int IT = NCH / kThreads;
+  static_assert(NCH % NT == 0, "tile chunks must be a multiple of the CTA size");
+  constexpr int IT = NCH / NT;
   float x[IT][8];
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * kThreads, a = e % A, b0 = (e / A) * 8;
+    const int e = threadIdx.x + it * NT, a = e % A, b0 = (e / A) * 8;
     const T* p = rowp(a);
     if (p) ld8(p + b0, x[it]);
     else {
@@ -89,7 +89,7 @@ __device__ __forceinline__ void build_tile_ld(uint8_t* hi, uint8_t* lo, RP rowp,
   }
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * kThreads, a = e % A, b0 = (e / A) * 8;
+    const int e = threadIdx.x + it * NT, a = e % A, b0 = (e / A) * 8;
     __align__(16) __nv_bfloat16 hh[8];
     __align__(16) __nv_bfloat16 ll[8];
 #pragma unroll

@@ -38,6 +38,21 @@ struct SlotRec {
   int32_t n_cons;
 };
 
+// Tree-masked attention: a query in node v reads the rows of v's proper ancestors (a few
+// contiguous ranges: one per chain on the path) and the earlier rows of v itself.
+struct AttnNode {
+  int32_t row_offset, length, subtree_end;  // subtree rows = [row_offset, subtree_end)
+  int32_t range_begin;                      // ancestor ranges [range_begin, next node's range_begin)
+  int32_t pos0;                             // trajectory position of the node's first token
+  int32_t pad[3];
+};
+struct RowRange {
+  int32_t start, end;
+};
+struct AttnTile {
+  int32_t node, row, n, pad;  // n <= 128 query rows or <= 64 key rows of one node
+};
+
 // Device view of the uploaded tables (all pointers into the caller's buffer).
 struct DevTables {
   const SeqRec* seqs;
@@ -55,6 +70,10 @@ struct DevTables {
   const int32_t* occ_begin;        // [N + 1] occurrence CSR (trajectory order)
   const int32_t* occ_list;         // [n_expanded] expanded positions
   const int32_t* occ_count;        // [N]
+  const AttnNode* attn_nodes;      // [n_nodes + 1] (last entry: range_begin sentinel)
+  const RowRange* attn_ranges;     // ancestor row ranges [start, end)
+  const AttnTile* attn_qtiles;
+  const AttnTile* attn_ktiles;
 };
 
 struct Plan {
@@ -76,6 +95,9 @@ struct Plan {
   std::vector<int32_t> exp_rows, occ_begin, occ_list;
   std::vector<int64_t> exp_rows64, traj_offset;
   std::vector<int32_t> round_seq_begin, round_chunk_begin;  // [n_rounds + 1], host only
+  std::vector<AttnNode> attn_nodes;
+  std::vector<int32_t> attn_ranges;  // pairs
+  std::vector<AttnTile> attn_qtiles, attn_ktiles;
 
   // device upload
   void* dev = nullptr;

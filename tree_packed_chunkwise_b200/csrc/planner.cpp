@@ -288,6 +288,41 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
     if (!rp.empty()) P.tgt_begin.push_back((int32_t)P.tgt_parts.size());
   }
 
+  // attention tables: subtree ends, ancestor row ranges (merged when contiguous), query / key tiles
+  {
+    std::vector<int64_t> sub(n, 0);
+    for (int32_t v = n - 1; v >= 0; --v) {
+      sub[v] += length[v];
+      if (parent[v] >= 0) sub[parent[v]] += sub[v];
+    }
+    std::vector<std::vector<std::pair<int32_t, int32_t>>> rg(n);
+    for (int32_t v = 0; v < n; ++v) {
+      const int32_t p = parent[v];
+      if (p >= 0) {
+        rg[v] = rg[p];
+        const int32_t a = (int32_t)P.row_offset[p], b = a + length[p];
+        if (!rg[v].empty() && rg[v].back().second == a) rg[v].back().second = b;
+        else rg[v].push_back({a, b});
+      }
+    }
+    P.attn_nodes.resize(n + 1);
+    for (int32_t v = 0; v < n; ++v) {
+      AttnNode an{};
+      an.row_offset = (int32_t)P.row_offset[v];
+      an.length = length[v];
+      an.subtree_end = (int32_t)(P.row_offset[v] + sub[v]);
+      an.range_begin = (int32_t)(P.attn_ranges.size() / 2);
+      an.pos0 = (int32_t)P.s[v];
+      for (auto& r : rg[v]) { P.attn_ranges.push_back(r.first); P.attn_ranges.push_back(r.second); }
+      P.attn_nodes[v] = an;
+      for (int32_t r = 0; r < length[v]; r += 128)
+        P.attn_qtiles.push_back({v, (int32_t)P.row_offset[v] + r, std::min(128, length[v] - r), 0});
+      for (int32_t r = 0; r < length[v]; r += 64)
+        P.attn_ktiles.push_back({v, (int32_t)P.row_offset[v] + r, std::min(64, length[v] - r), 0});
+    }
+    P.attn_nodes[n] = AttnNode{0, 0, 0, (int32_t)(P.attn_ranges.size() / 2), 0, {0, 0, 0}};
+  }
+
   // expanded maps
   P.traj_offset.push_back(0);
   for (int32_t leaf : P.leaves) {
@@ -323,7 +358,9 @@ size_t device_layout(const Plan& p, std::vector<size_t>& off) {
       p.seqs.size() * sizeof(SeqRec), p.chunks.size() * sizeof(ChunkRec), p.slots.size() * sizeof(SlotRec),
       p.slot_cons.size() * 4, p.root_cons_begin.size() * 4, p.root_cons.size() * 4, p.replay_rows.size() * 4,
       p.tgt_row.size() * 4, p.tgt_begin.size() * 4, p.tgt_parts.size() * 4, p.row_tgt.size() * 4,
-      p.exp_rows.size() * 4, p.occ_begin.size() * 4, p.occ_list.size() * 4, p.occurrence.size() * 0 + (size_t)p.n_unique * 4};
+      p.exp_rows.size() * 4, p.occ_begin.size() * 4, p.occ_list.size() * 4, p.occurrence.size() * 0 + (size_t)p.n_unique * 4,
+      p.attn_nodes.size() * sizeof(AttnNode), p.attn_ranges.size() * 4, p.attn_qtiles.size() * sizeof(AttnTile),
+      p.attn_ktiles.size() * sizeof(AttnTile)};
   off.clear();
   size_t o = 0;
   for (size_t s : sizes) { off.push_back(o); o += align256(s); }
@@ -352,6 +389,10 @@ void pack_device_blob(const Plan& p, const std::vector<size_t>& off, std::vector
   std::vector<int32_t> cnt((size_t)p.n_unique);
   for (int64_t r = 0; r < p.n_unique; ++r) cnt[r] = p.occ_begin[r + 1] - p.occ_begin[r];
   put(14, cnt.data(), cnt.size() * 4);
+  put(15, p.attn_nodes.data(), p.attn_nodes.size() * sizeof(AttnNode));
+  put(16, p.attn_ranges.data(), p.attn_ranges.size() * 4);
+  put(17, p.attn_qtiles.data(), p.attn_qtiles.size() * sizeof(AttnTile));
+  put(18, p.attn_ktiles.data(), p.attn_ktiles.size() * sizeof(AttnTile));
 }
 
 DevTables device_view(const Plan& p, void* base, const std::vector<size_t>& off) {
@@ -373,6 +414,10 @@ DevTables device_view(const Plan& p, void* base, const std::vector<size_t>& off)
   d.occ_begin = (const int32_t*)at(12);
   d.occ_list = (const int32_t*)at(13);
   d.occ_count = (const int32_t*)at(14);
+  d.attn_nodes = (const AttnNode*)at(15);
+  d.attn_ranges = (const RowRange*)at(16);
+  d.attn_qtiles = (const AttnTile*)at(17);
+  d.attn_ktiles = (const AttnTile*)at(18);
   return d;
 }
 

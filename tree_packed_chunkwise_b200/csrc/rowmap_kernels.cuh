@@ -30,4 +30,10 @@ __global__ void occurrence_count_kernel(DevTables t, int32_t* __restrict__ count
   if (r < n) counts[r] = t.occ_count[r];
 }
 
+// absolute trajectory position (depth) of every compact row: one CTA per node
+__global__ void rope_positions_kernel(DevTables t, int32_t* __restrict__ pos) {
+  const AttnNode nd = t.attn_nodes[blockIdx.x];
+  for (int i = threadIdx.x; i < nd.length; i += blockDim.x) pos[nd.row_offset + i] = nd.pos0 + i;
+}
+
 }  // namespace tpc

@@ -14,6 +14,7 @@
 #include "kda_scan_tc.cuh"
 #include "gemm_tc.cuh"
 #include "logprob_kernels.cuh"
+#include "attn_tc.cuh"
 #include <cudaTypedefs.h>
 #include "plan.h"
 #include "rowmap_kernels.cuh"
@@ -643,6 +644,74 @@ int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int
     if (int rc = tpc_gemm_bf16(zh, hb + r0 * Dh, dW, V, Dh, R, V, Dh, Dh, 1, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
     if (int rc = tpc_gemm_bf16(zl, hb + r0 * Dh, dW, V, Dh, R, V, Dh, Dh, 1, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
   }
+  return TPC_OK;
+}
+
+namespace {
+int attn_check(const tpc_plan* plan, const tpc_attn_shape* s) {
+  if (!plan || !s) return fail(TPC_ERR_NULL, "attention: plan or shape is NULL");
+  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
+  if (s->d_qk != tpc::kAttnQK || s->d_v != tpc::kAttnDV || s->H < 1)
+    return fail(TPC_ERR_UNSUPPORTED, "attention: built for d_qk = 192, d_v = 128");
+  if (s->io_dtype != TPC_F32 && s->io_dtype != TPC_BF16) return fail(TPC_ERR_UNSUPPORTED, "attention: io dtype");
+  return TPC_OK;
+}
+}  // namespace
+
+int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const void* q, const void* k, const void* v,
+                          void* o, float* lse, int32_t* status, tpc_stream_t stream) {
+  if (int rc = attn_check(plan, s)) return rc;
+  if (!q || !k || !v || !o || !lse) return fail(TPC_ERR_NULL, "attention forward: NULL tensor");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const tpc::Plan& p = plan->p;
+  const dim3 grid((unsigned)p.attn_qtiles.size(), (unsigned)s->H);
+  using bf = __nv_bfloat16;
+  if (s->io_dtype == TPC_BF16) {
+    TPC_CUDA(set_smem(tpc::attn_fwd_tc<bf>, tpc::AttnFwdSmem::total));
+    TPC_LAUNCH("attn_fwd_tc", st,
+               (tpc::attn_fwd_tc<bf><<<grid, tpc::kAttnThreads, tpc::AttnFwdSmem::total, st>>>(
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, (bf*)o, lse, status)));
+  } else {
+    TPC_CUDA(set_smem(tpc::attn_fwd_tc<float>, tpc::AttnFwdSmem::total));
+    TPC_LAUNCH("attn_fwd_tc", st,
+               (tpc::attn_fwd_tc<float><<<grid, tpc::kAttnThreads, tpc::AttnFwdSmem::total, st>>>(
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, (float*)o, lse, status)));
+  }
+  return TPC_OK;
+}
+
+int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const void* q, const void* k,
+                           const void* v, const void* o, const float* lse, const void* d_o, void* dq, void* dk,
+                           void* dv, float* delta, int32_t* status, tpc_stream_t stream) {
+  if (int rc = attn_check(plan, s)) return rc;
+  if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv || !delta)
+    return fail(TPC_ERR_NULL, "attention backward: NULL tensor");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const tpc::Plan& p = plan->p;
+  using bf = __nv_bfloat16;
+  const dim3 gq((unsigned)p.attn_qtiles.size(), (unsigned)s->H), gk((unsigned)p.attn_ktiles.size(), (unsigned)s->H);
+  auto go = [&](auto tio) -> int {
+    using T = decltype(tio);
+    TPC_CUDA(set_smem(tpc::attn_bwd_dq_tc<T>, tpc::AttnDqSmem::total));
+    TPC_CUDA(set_smem(tpc::attn_bwd_dkv_tc<T>, tpc::AttnDkvSmem::total));
+    TPC_LAUNCH("attn_bwd_dq_tc", st,
+               (tpc::attn_bwd_dq_tc<T><<<gq, tpc::kAttnThreads, tpc::AttnDqSmem::total, st>>>(
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, (const T*)o, lse, (const bf*)d_o,
+                   (T*)dq, delta, status)));
+    TPC_LAUNCH("attn_bwd_dkv_tc", st,
+               (tpc::attn_bwd_dkv_tc<T><<<gk, tpc::kAttnThreads, tpc::AttnDkvSmem::total, st>>>(
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, lse, (const bf*)d_o, delta, (T*)dk,
+                   (T*)dv, status)));
+    return TPC_OK;
+  };
+  return s->io_dtype == TPC_BF16 ? go(bf{}) : go(float{});
+}
+
+int tpc_rope_positions(const tpc_plan* plan, int32_t* pos, tpc_stream_t stream) {
+  if (!plan || !pos) return fail(TPC_ERR_NULL, "plan or pos is NULL");
+  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TPC_LAUNCH("rope_positions", st, (tpc::rope_positions_kernel<<<plan->p.n, 128, 0, st>>>(plan->p.dt, pos)));
   return TPC_OK;
 }
 
