@@ -43,6 +43,15 @@ def kernel_flops(name, C, d):
             "kda_bwd_dkv": 10 * Cd + 2 * dd}.get(name, 0)
 
 
+# algorithmic HBM bytes per processed token-head of each kernel: the bytes of the layer's own
+# tensors (q, k, v, g, beta, dO in; o, dq, dk, dv, dg, dbeta out; bf16 except dg/dbeta fp32) that
+# the kernel must read or write; workspace traffic (chunk states, W, U, partials) is not counted
+def kernel_bytes(name, d):
+    name = name[:-3] if name.endswith("_tc") else name
+    return {"kda_fwd_prep": 6 * d + 2, "kda_fwd_out": 8 * d, "kda_bwd_prep": 8 * d, "kda_bwd_dq": 10 * d,
+            "kda_bwd_dkv": 14 * d + 6}.get(name, 0)
+
+
 # algorithmic HBM bytes per token-head of the whole step (bf16 I/O): forward reads q,k,v,g (8d)
 # + beta (2) and writes o (2d); backward reads those and dO and writes dq,dk,dv (6d), dg (4d), dbeta (4)
 def step_bytes_per_token_head(d):
@@ -159,6 +168,9 @@ def source_hash(names):
     return h.hexdigest()[:16]
 
 
+TRAFFIC_SOURCES = ["kda_tc.cuh", "tc.cuh", "common.cuh"]
+
+
 def committed_traffic(kernel):
     """dram bytes per launch from a committed ncu capture, if the kernel source is unchanged."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -167,7 +179,7 @@ def committed_traffic(kernel):
     with open(p) as f:
         j = json.load(f)
     e = j.get(kernel)
-    if not e or e.get("source_hash") != source_hash(["kda_kernels.cuh", "common.cuh"]):
+    if not e or e.get("source_hash") != source_hash(TRAFFIC_SOURCES):
         return None
     return e["bytes_per_launch"]
 
@@ -219,6 +231,104 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------------ hybrid layer group
+GROUP_WORKLOAD = "agentic"
+
+
+def group_flops_per_row(depth):
+    """Algorithmic FLOP of one unique row in the 3 KDA + 1 MLA group (forward + backward, the
+    recomputation not counted): projections 2 D (4 D + H) + 2 D^2 per KDA layer, 2 D (3648) +
+    2 (512)(2 D) + 2 D^2 for MLA, times 3 (backward = 2 x forward); attention 2 H (192 + 128)
+    (depth + 1) times 3.5 (backward = 2.5 x forward); KDA core 3 (10 C d + 6 d^2) per head."""
+    D, H, d, C = 2048, 16, 128, 64
+    kda_proj = 2 * D * (4 * D + H) + 2 * D * D
+    mla_proj = 2 * D * 3648 + 2 * 512 * 2 * D + 2 * D * D
+    gemm = 3 * (3 * kda_proj + mla_proj)
+    attn = 3.5 * 2 * H * (192 + 128) * (depth + 1)
+    core = 3 * H * 3 * (10 * C * d + 6 * d * d)
+    return gemm, attn, core
+
+
+def measure_group(args, world, rank, tpc, torch, peaks):
+    import synth.gpu as sgpu
+    w = synth.workload(GROUP_WORKLOAD)
+    t = w.tree
+    seed = 3 + 1000 * rank
+    plan = tpc.Plan(t.parent, t.length, 64).upload()
+    info = plan.info
+    N, NE = info["n_unique"], info["n_expanded"]
+    st = t.node_start()
+    src_rows = torch.tensor(plan.compact_source_rows(st, t.length), dtype=torch.int32, device="cuda")
+    D = 2048
+    x = sgpu.normal_rows(seed, synth.STREAM["group_x"], src_rows, D, "f32")
+    R = sgpu.normal_rows(seed, synth.STREAM["group_r"], None, D, "f32", shape=(NE,))
+    shapes = synth.group_weight_shapes(3)
+    W = {"kda": [tuple(sgpu.normal_rows(seed, synth.group_weight_stream(l, m), None, shp[1], "bf16", 0.02,
+                                        shape=(shp[0],)) for m, shp in enumerate(pair))
+                 for l, pair in enumerate(shapes["kda"])],
+         "mla": tuple(sgpu.normal_rows(seed, synth.group_weight_stream(15, m), None, shp[1], "bf16", 0.02,
+                                       shape=(shp[0],)) for m, shp in enumerate(shapes["mla"]))}
+    ws = tpc.group_workspace(plan, 3)
+    h = torch.empty(3, N, D, dtype=torch.float32, device="cuda")
+    y = torch.empty(N, D, dtype=torch.float32, device="cuda")
+    dx = torch.empty(N, D, dtype=torch.float32, device="cuda")
+    grads = {"kda": [tuple(torch.empty(m.shape, dtype=torch.float32, device="cuda") for m in pair) for pair in W["kda"]],
+             "mla": tuple(torch.empty(m.shape, dtype=torch.float32, device="cuda") for m in W["mla"])}
+    stream = torch.cuda.current_stream()
+
+    def step():
+        tpc.tpc_group_forward(plan, W, x, ws, h=h, y=y)
+        dy = tpc.tpc_reduce_expanded_to_unique(plan, R)
+        tpc.tpc_group_backward(plan, W, x, h, dy, ws, dx=dx, grads=grads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    code = tpc.tpc_group_status(plan, ws, 3)
+    K = max(1, args.group_steps)
+    n0 = tpc.tpc_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = (tpc.tpc_launch_count() - n0) / K
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / K
+    # per-kernel shares (separate pass, events around every launch)
+    tpc.tpc_profile_enable(True)
+    step()
+    torch.cuda.synchronize()
+    prof = tpc.tpc_profile_read()
+    tpc.tpc_profile_enable(False)
+    tot = sum(v[1] for v in prof.values())
+    kern = {k: {"launches": n, "ms": v, "share": v / tot} for k, (n, v) in prof.items()}
+    depth = np.concatenate([np.arange(a, a + l) for a, l in
+                            zip([sum(int(t.length[u]) for u in t.path(v)[:-1]) for v in range(t.n)], t.length)])
+    occ = depth  # rows in node order; the per-row count does not depend on the order
+    gemm_f, attn_f, core_f = group_flops_per_row(occ)
+    flops = float(N * gemm_f + attn_f.sum() + N * core_f)
+    tflops = flops / (ms / 1e3) / 1e12
+    peak = peaks["sustained"] or peaks["bf16_tflops"]
+    gemm_ms = sum(v["ms"] for k, v in kern.items() if k.startswith("gemm"))
+    attn_ms = sum(v["ms"] for k, v in kern.items() if k.startswith("attn"))
+    return {"workload": w.name + " (hybrid group: 3 KDA + 1 MLA, D=2048)", "n_unique": N, "n_expanded": NE,
+            "ms_per_step": ms, "unique_tokens_per_s": world * N / (ms / 1e3),
+            "expanded_tokens_per_s": world * NE / (ms / 1e3), "status": code, "launches_per_step": launches,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                         "algorithmic_tflop_per_step": flops / 1e12,
+                         "gemm_tflop_per_step": float(N * gemm_f) / 1e12,
+                         "attention_tflop_per_step": float(attn_f.sum()) / 1e12,
+                         "peak_source": "bf16 sustained, " + peaks["source"]},
+            "gemm_achieved_tflops": float(N * gemm_f) / 1e12 / (gemm_ms / 1e3) if gemm_ms else None,
+            "attention_achieved_tflops": float(attn_f.sum()) / 1e12 / (attn_ms / 1e3) if attn_ms else None,
+            "kernels": kern,
+            "precision": "bf16 weights; fp32 activations and gradients, tensor-core products from bf16 hi/lo pairs"}
+
+
 # ------------------------------------------------------------------------------------ GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -231,6 +341,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-expanded", action="store_true")
+    ap.add_argument("--no-group", action="store_true", help="skip the hybrid layer group (3 KDA + 1 MLA) measurement")
+    ap.add_argument("--group-steps", type=int, default=3)
     ap.add_argument("--workload", default=WORKLOAD, help="single_fork (default), agentic, agentic_small")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "tpc" else args.warmup
@@ -311,23 +423,26 @@ def main():
     kern = {}
     for name, (n, tot) in prof.items():
         per = tot / n
-        fl = kernel_flops(name, w.chunk, d)
-        units = tokens_proc * H if name not in ("kda_fwd_scan", "kda_bwd_scan") else tokens_proc * H / info["n_rounds"]
+        units = tokens_proc * H * args.steps / n  # token-heads one launch processes (averaged over launches)
         kern[name] = {"launches_per_step": n / args.steps, "ms_per_launch": per, "share": 0.0,
-                      "gflop_per_launch": fl * units / 1e9}
+                      "gflop_per_launch": kernel_flops(name, w.chunk, d) * units / 1e9,
+                      "gb_per_launch": kernel_bytes(name, d) * units / 1e9}
     total_ms = sum(v["ms_per_launch"] * v["launches_per_step"] for v in kern.values())
     for v in kern.values():
         v["share"] = v["ms_per_launch"] * v["launches_per_step"] / total_ms
     dom = max(kern, key=lambda k: kern[k]["share"])
     peaks = load_peaks()
     clocks = clk.summary()
-    sm_max = clocks.get("sm_max_mhz") or peaks["sm_max_mhz"]
-    alu_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12  # fp32 FMA lanes x 2 FLOP x max SM clock, TFLOP/s
     dk = kern[dom]
-    achieved = dk["gflop_per_launch"] / dk["ms_per_launch"]  # GFLOP/ms == TFLOP/s
-    roofline = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                "frac": achieved / alu_peak, "traffic": committed_traffic(dom),
-                "peak_source": "148 SMs x 128 fp32 lanes x 2 x max SM clock"}
+    # the KDA kernels sit below the B200 ridge point (tens of FLOP per algorithmic byte): HBM-bound
+    achieved = dk["gb_per_launch"] / dk["ms_per_launch"] * 1e3  # GB/s
+    tc_achieved = dk["gflop_per_launch"] / dk["ms_per_launch"]  # TFLOP/s
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(dom),
+                "algorithmic_gb_per_launch": dk["gb_per_launch"],
+                "tensor_frac": tc_achieved / peaks["bf16_tflops"], "tensor_achieved_tflops": tc_achieved,
+                "peak_source": "measured HBM copy bandwidth (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
+                else "fallback 6650 GB/s"}
     step_bytes = step_bytes_per_token_head(d) * tokens_proc * H
     step_flops = step_flops_per_token_head(w.chunk, d) * tokens_proc * H
     step_roof = {"hbm_frac": (step_bytes / (ms_step / 1e3)) / (peaks["hbm_gbs"] * 1e9),
@@ -403,6 +518,13 @@ def main():
         e2e = {"value": world * N / (ams / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ams}
 
+    # ---- hybrid layer group on the agentic tree (KDA buffers released first)
+    group = None
+    if not args.no_group:
+        del wsb, outs, grads, dev
+        torch.cuda.empty_cache()
+        group = measure_group(args, world, rank, tpc, torch, peaks)
+
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -420,7 +542,7 @@ def main():
                            "l2": "inputs+workspace > 1 GB per step, larger than L2"},
                 "value_expanded": value_exp, "roofline": roofline, "step_roofline": step_roof,
                 "kernels": kern, "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
-                "expanded_path": expanded}
+                "expanded_path": expanded, "hybrid_group": group}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

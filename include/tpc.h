@@ -230,6 +230,19 @@ int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, i
                   int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype, float alpha, float beta, int32_t* status,
                   tpc_stream_t stream);
 
+/*
+ * Split-precision form of tpc_gemm_bf16 for fp32 operands held as two bf16 matrices, X_hi = bf16(X)
+ * and X_lo = bf16(X - X_hi) (X = X_hi + X_lo to 2^-17 relative):
+ *   C = alpha * (A B + A_lo B + A B_lo) + beta * C,
+ * where A_lo and B_lo are optional (NULL: term left out; B_lo requires A_lo) and share A's and B's
+ * layout and leading dimensions.  With A_lo only (fp32 activations times bf16 weights) the result
+ * is the fp32 product to about 2^-16 relative; with both (two fp32 operands) the dropped
+ * A_lo B_lo term is below 2^-16 of the product.  Costs one tensor-core pass per term.
+ */
+int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B_lo, void* C, int64_t M, int64_t N,
+                   int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype,
+                   float alpha, float beta, int32_t* status, tpc_stream_t stream);
+
 /* ------------------------------------------------------------------ tree-masked attention */
 /*
  * Softmax attention in which each token reads only its ancestors' keys and values and the earlier
@@ -247,11 +260,22 @@ typedef struct tpc_attn_shape {
   float scale;
   int32_t io_dtype; /* dtype of o (forward) and of o, dq, dk, dv (backward) */
 } tpc_attn_shape;
+/*
+ * Optional bf16 low parts (NULL = zero) of inputs given as hi/lo pairs: an fp32 tensor x is passed
+ * as hi = bf16(x) in the main argument and lo = bf16(x - hi) here (x = hi + lo to 2^-17 relative).
+ * With any low part present, every product takes the three partial products hi hi + lo hi + hi lo,
+ * so fp32 inputs and upstream gradients enter without a bf16 rounding of their own.  lo may be NULL.
+ */
+typedef struct tpc_attn_lo {
+  const void* q; const void* k; const void* v; /* layouts of q, k, v */
+  const void* d_o;                             /* backward only, layout of d_o */
+} tpc_attn_lo;
 int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* shape, const void* q, const void* k,
-                          const void* v, void* o, float* lse, int32_t* status, tpc_stream_t stream);
+                          const void* v, const tpc_attn_lo* lo, void* o, float* lse, int32_t* status,
+                          tpc_stream_t stream);
 int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* shape, const void* q, const void* k,
-                           const void* v, const void* o, const float* lse, const void* d_o, void* dq, void* dk,
-                           void* dv, float* delta, int32_t* status, tpc_stream_t stream);
+                           const void* v, const tpc_attn_lo* lo, const void* o, const float* lse, const void* d_o,
+                           void* dq, void* dk, void* dv, float* delta, int32_t* status, tpc_stream_t stream);
 /* Trajectory position (depth from the root) of every compact row, int32 [N] (rotary positions). */
 int tpc_rope_positions(const tpc_plan* plan, int32_t* pos, tpc_stream_t stream);
 
@@ -279,6 +303,67 @@ int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int
                          const int32_t* targets, const float* dlogp, const float* lse, float* dh, float* dW,
                          void* scratch, size_t scratch_bytes, int32_t chunk_rows, int32_t* status,
                          tpc_stream_t stream);
+
+/* ------------------------------------------------------------------ hybrid layer group */
+/*
+ * A group of n_kda KDA layers followed by one latent-attention (MLA) layer on the compact rows of
+ * the plan's tree (HARTS Table 1: KDA and MLA layers in a 3:1 group; Figure C.1: each layer runs
+ * once per unique row; Table 7 and Section 4: activations recomputed in the backward pass).  The
+ * pages give no layer formulas; this library fixes the plainest pre-norm residual layers:
+ *   KDA layer: xn = RMSNorm(x) (unit weight, eps 1e-6); [q | k | v | g | beta] = xn W_in^T with
+ *     W_in [4 D + H][D] (rows: q, k, v, g blocks of D = H d_head, then H beta rows);
+ *     k L2-normalised per head (eps 1e-6), g = -0.1 softplus(.), beta = sigmoid(.);
+ *     y = x + KDA(q, k, v, g, beta) W_o^T, W_o [D][D].
+ *   MLA layer: xn = RMSNorm(x); [q | c | kr] = xn W_a^T, W_a [H (d_head + d_rope) + d_latent + d_rope][D]
+ *     (per head d_head no-position dims then d_rope rotary dims; c the latent; kr the rotary key
+ *     shared by every head); [k_nope | v] = c W_b^T, W_b [2 D][d_latent]; rotary half-split rotation
+ *     (base 10000) of q's and kr's rotary dims at the row's trajectory depth; k = [k_nope | kr];
+ *     tree-masked softmax attention with scale 1/sqrt(d_head + d_rope); y = x + o W_o^T, W_o [D][D].
+ * Precision: weights bf16; activations and gradients fp32.  Tensor-core products take fp32
+ * operands as bf16 hi/lo pairs (tpc_gemm_split, tpc_attn_lo), so no activation or gradient is
+ * rounded to bf16; the KDA recurrence runs on fp32 inputs.
+ * Built for D = 2048, H = 16, d_head = 128, d_rope = 64, d_latent = 512, chunk-64 plans.
+ */
+#define TPC_GROUP_MAX_KDA 8
+typedef struct tpc_group_shape {
+  int32_t D, H, d_head, d_rope, d_latent;
+  int32_t n_kda; /* KDA layers before the MLA layer, 0..TPC_GROUP_MAX_KDA */
+} tpc_group_shape;
+typedef struct tpc_group_kda_weights { const void* w_in; const void* w_o; } tpc_group_kda_weights;
+typedef struct tpc_group_mla_weights { const void* w_a; const void* w_b; const void* w_o; } tpc_group_mla_weights;
+typedef struct tpc_group_weights {
+  tpc_group_kda_weights kda[TPC_GROUP_MAX_KDA]; /* bf16, first n_kda used */
+  tpc_group_mla_weights mla;
+} tpc_group_weights;
+/* weight gradients, fp32, same shapes as the weights; overwritten by the backward */
+typedef struct tpc_group_kda_grads { float* w_in; float* w_o; } tpc_group_kda_grads;
+typedef struct tpc_group_mla_grads { float* w_a; float* w_b; float* w_o; } tpc_group_mla_grads;
+typedef struct tpc_group_grads {
+  tpc_group_kda_grads kda[TPC_GROUP_MAX_KDA];
+  tpc_group_mla_grads mla;
+} tpc_group_grads;
+
+/* Workspace bytes for tpc_group_forward / tpc_group_backward on this plan (0 if unsupported). */
+size_t tpc_group_workspace_bytes(const tpc_plan* plan, const tpc_group_shape* shape);
+/*
+ * Forward.  x: fp32 [N][D] (compact rows); h: fp32 [n_kda][N][D] receives each KDA layer's output
+ * (= the next layer's input, the only activations kept for the backward); y: fp32 [N][D].
+ * Errors: TPC_ERR_NULL, TPC_ERR_STATE, TPC_ERR_UNSUPPORTED, TPC_ERR_WORKSPACE, TPC_ERR_CUDA;
+ * device-side failures (GEMM or attention wait timeouts, KDA gate range) are read by
+ * tpc_group_status.
+ */
+int tpc_group_forward(const tpc_plan* plan, const tpc_group_shape* shape, const tpc_group_weights* w,
+                      const float* x, float* h, float* y, void* ws, size_t ws_bytes, tpc_stream_t stream);
+/*
+ * Backward of sum <dy, y>: recomputes every layer from its kept input (x, h), then runs its adjoint
+ * in reverse layer order.  dy fp32 [N][D] (occurrence-summed upstream gradient per compact row);
+ * dx fp32 [N][D] (may equal dy); weight gradients into g.  The workspace need not hold a forward.
+ */
+int tpc_group_backward(const tpc_plan* plan, const tpc_group_shape* shape, const tpc_group_weights* w,
+                       const float* x, const float* h, const float* dy, float* dx, const tpc_group_grads* g,
+                       void* ws, size_t ws_bytes, tpc_stream_t stream);
+/* Synchronises `stream`, returns and clears the first device-side error of the group's kernels. */
+int tpc_group_status(const tpc_plan* plan, const tpc_group_shape* shape, void* ws, tpc_stream_t stream);
 
 /* ------------------------------------------------------------------ allocation-free forward */
 /* Bytes of device scratch built into the library for tpc_kda_forward_static (64 MiB). */

@@ -16,11 +16,9 @@ MLA layer (y = x + o W_o^T):
     o = tree-masked softmax attention of q = [q_nope | q_rot], k = [k_nope | kr], v, with scale
         1/sqrt(d_head + d_rope)  (oracle.attention: causal along every trajectory)
 
-Precision mirror: with ``rounding`` on, the values that the device computes in bf16 are rounded
-to bf16 here at the same places (GEMM operands: RMSNorm outputs, layer outputs before W_o, the
-latent c, the upstream gradients entering each GEMM; the KDA and attention inputs and their
-upstream gradients).  Everything else is fp64.  With ``rounding`` off the group is the exact
-fp64 function, which the pins differentiate numerically.
+Precision: the device keeps activations and gradients in fp32 and forms its tensor-core products
+from bf16 hi/lo pairs (x = hi + lo to 2^-17 relative), so no activation is rounded to bf16 there;
+the oracle is the exact fp64 function of the bf16-valued weights.
 
 The backward is reverse-mode differentiation of this forward (torch autograd over fp64 CPU
 tensors), except for KDA and attention, whose adjoints are the hand-written ones of
@@ -57,47 +55,12 @@ class Dims:
         return self.H * (self.d_head + self.d_rope) + self.d_latent + self.d_rope
 
 
-def to_bf16(x: torch.Tensor) -> torch.Tensor:
-    """Round to the nearest bf16 value (ties to even), kept in fp64."""
-    return x.to(torch.float32).to(torch.bfloat16).to(torch.float64)
-
-
-class _Round(torch.autograd.Function):
-    """Forward rounds to bf16; the gradient passes unchanged (the rounded value is the input)."""
-
-    @staticmethod
-    def forward(ctx, x, on):
-        return to_bf16(x) if on else x.clone()
-
-    @staticmethod
-    def backward(ctx, g):
-        return g, None
-
-
-class _Gemm(torch.autograd.Function):
-    """y = r(a) w^T for a weight w [out][in] held in bf16; the backward rounds the upstream
-    gradient once, as the device does before its two gradient products."""
-
-    @staticmethod
-    def forward(ctx, a, w, on):
-        ar = to_bf16(a) if on else a
-        ctx.save_for_backward(ar, w)
-        ctx.on = on
-        return ar @ w.T
-
-    @staticmethod
-    def backward(ctx, gy):
-        ar, w = ctx.saved_tensors
-        g = to_bf16(gy) if ctx.on else gy
-        return g @ w, g.T @ ar, None
-
-
 class _Kda(torch.autograd.Function):
     """KDA over the tree (oracle.kda token-by-token recurrence along every trajectory)."""
 
     @staticmethod
-    def forward(ctx, q, k, v, g, beta, tree, on):
-        ctx.tree, ctx.on = tree, on
+    def forward(ctx, q, k, v, g, beta, tree):
+        ctx.tree = tree
         ctx.save_for_backward(q, k, v, g, beta)
         inputs = tuple(t.detach().numpy() for t in (q, k, v, g, beta))
         o, _ = okda.tree_forward(tree, inputs)
@@ -106,18 +69,17 @@ class _Kda(torch.autograd.Function):
     @staticmethod
     def backward(ctx, do):
         q, k, v, g, beta = ctx.saved_tensors
-        d = to_bf16(do) if ctx.on else do
         inputs = tuple(t.detach().numpy() for t in (q, k, v, g, beta))
-        grads = okda.tree_backward(ctx.tree, inputs, d.detach().numpy())
-        return tuple(torch.from_numpy(x) for x in grads[:5]) + (None, None)
+        grads = okda.tree_backward(ctx.tree, inputs, do.detach().numpy())
+        return tuple(torch.from_numpy(x) for x in grads[:5]) + (None,)
 
 
 class _Attn(torch.autograd.Function):
     """Tree-masked softmax attention (oracle.attention: causal along every trajectory)."""
 
     @staticmethod
-    def forward(ctx, q, k, v, tree, scale, on):
-        ctx.tree, ctx.scale, ctx.on = tree, scale, on
+    def forward(ctx, q, k, v, tree, scale):
+        ctx.tree, ctx.scale = tree, scale
         ctx.save_for_backward(q, k, v)
         o, _ = oatt.tree_forward(tree, q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), scale)
         return torch.from_numpy(o)
@@ -125,10 +87,9 @@ class _Attn(torch.autograd.Function):
     @staticmethod
     def backward(ctx, do):
         q, k, v = ctx.saved_tensors
-        d = to_bf16(do) if ctx.on else do
         qn, kn, vn = (t.detach().numpy() for t in (q, k, v))
-        dq, dk, dv = oatt.tree_backward(ctx.tree, qn, kn, vn, ctx.scale, d.detach().numpy())
-        return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv), None, None, None
+        dq, dk, dv = oatt.tree_backward(ctx.tree, qn, kn, vn, ctx.scale, do.detach().numpy())
+        return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv), None, None
 
 
 def rmsnorm(x: torch.Tensor, eps: float) -> torch.Tensor:
@@ -147,39 +108,37 @@ def rope(x: torch.Tensor, pos: torch.Tensor, base: float) -> torch.Tensor:
     return torch.cat([x1 * c - x2 * s, x1 * s + x2 * c], dim=-1)
 
 
-def kda_layer(tree, x, w_in, w_o, dims: Dims, rounding: bool, parts: dict | None = None):
+def kda_layer(tree, x, w_in, w_o, dims: Dims, parts: dict | None = None):
     N, D, H, dh = x.shape[0], dims.D, dims.H, dims.d_head
     xn = rmsnorm(x, dims.eps)
-    P = _Gemm.apply(xn, w_in, rounding)
+    P = xn @ w_in.T
     q = P[:, :D].reshape(N, H, dh)
     kt = P[:, D:2 * D].reshape(N, H, dh)
     k = kt / torch.sqrt((kt * kt).sum(dim=-1, keepdim=True) + dims.eps)
     v = P[:, 2 * D:3 * D].reshape(N, H, dh)
     g = -0.1 * torch.nn.functional.softplus(P[:, 3 * D:4 * D]).reshape(N, H, dh)
     beta = torch.sigmoid(P[:, 4 * D:4 * D + H])
-    ins = [_Round.apply(t, rounding) for t in (q, k, v, g, beta)]
-    o = _Kda.apply(*ins, tree, rounding).reshape(N, D)
+    o = _Kda.apply(q, k, v, g, beta, tree).reshape(N, D)
     if parts is not None:
-        parts.update(xn=xn, q=ins[0], k=ins[1], v=ins[2], g=ins[3], beta=ins[4], o=o)
-    return x + _Gemm.apply(o, w_o, rounding)
+        parts.update(xn=xn, q=q, k=k, v=v, g=g, beta=beta, o=o)
+    return x + o @ w_o.T
 
 
-def mla_layer(tree, pos, x, w_a, w_b, w_o, dims: Dims, rounding: bool, parts: dict | None = None):
+def mla_layer(tree, pos, x, w_a, w_b, w_o, dims: Dims, parts: dict | None = None):
     N, D, H, dh, dr, dl = x.shape[0], dims.D, dims.H, dims.d_head, dims.d_rope, dims.d_latent
     xn = rmsnorm(x, dims.eps)
-    P = _Gemm.apply(xn, w_a, rounding)
+    P = xn @ w_a.T
     qh = P[:, :H * (dh + dr)].reshape(N, H, dh + dr)
     c = P[:, H * (dh + dr):H * (dh + dr) + dl]
     kr = rope(P[:, H * (dh + dr) + dl:], pos, dims.base)
     q = torch.cat([qh[..., :dh], rope(qh[..., dh:], pos, dims.base)], dim=-1)
-    KV = _Gemm.apply(c, w_b, rounding)
+    KV = c @ w_b.T
     k = torch.cat([KV[:, :D].reshape(N, H, dh), kr[:, None, :].expand(N, H, dr)], dim=-1)
     v = KV[:, D:].reshape(N, H, dh)
-    q, k, v = (_Round.apply(t, rounding) for t in (q, k, v))
-    o = _Attn.apply(q, k, v, tree, 1.0 / np.sqrt(dh + dr), rounding).reshape(N, D)
+    o = _Attn.apply(q, k, v, tree, 1.0 / np.sqrt(dh + dr)).reshape(N, D)
     if parts is not None:
         parts.update(xn=xn, q=q, k=k, v=v, c=c, kr=kr, o=o)
-    return x + _Gemm.apply(o, w_o, rounding)
+    return x + o @ w_o.T
 
 
 def depth_positions(tree) -> np.ndarray:
@@ -192,7 +151,7 @@ def depth_positions(tree) -> np.ndarray:
     return pos
 
 
-def group_forward(tree, x, weights, dims: Dims = Dims(), rounding: bool = True):
+def group_forward(tree, x, weights, dims: Dims = Dims()):
     """y and every layer output for node-order rows x [N, D] (fp64 numpy).
 
     weights: {"kda": [(w_in, w_o), ...], "mla": (w_a, w_b, w_o)} as float64 arrays.
@@ -203,30 +162,33 @@ def group_forward(tree, x, weights, dims: Dims = Dims(), rounding: bool = True):
         h = torch.from_numpy(np.asarray(x, np.float64))
         outs = []
         for w_in, w_o in weights["kda"]:
-            h = kda_layer(tree, h, torch.from_numpy(w_in), torch.from_numpy(w_o), dims, rounding)
+            h = kda_layer(tree, h, torch.from_numpy(w_in), torch.from_numpy(w_o), dims)
             outs.append(h.numpy())
         w_a, w_b, w_o = (torch.from_numpy(w) for w in weights["mla"])
-        y = mla_layer(tree, pos, h, w_a, w_b, w_o, dims, rounding)
+        y = mla_layer(tree, pos, h, w_a, w_b, w_o, dims)
     return y.numpy(), outs
 
 
-def group_backward(tree, x, weights, dy, dims: Dims = Dims(), rounding: bool = True):
+def group_backward(tree, x, weights, dy, dims: Dims = Dims()):
     """Gradients of sum <dy, y> (dy per node-order row, occurrence-summed) w.r.t. x and every
-    weight: returns (y, dx, {"kda": [(dw_in, dw_o), ...], "mla": (dw_a, dw_b, dw_o)})."""
+    weight: returns (y, dx, {"kda": [(dw_in, dw_o), ...], "mla": (dw_a, dw_b, dw_o)}, [outputs of
+    the KDA layers])."""
     pos = torch.from_numpy(depth_positions(tree))
     xt = torch.tensor(np.asarray(x, np.float64), requires_grad=True)
     kw = [tuple(torch.tensor(w, requires_grad=True) for w in pair) for pair in weights["kda"]]
     mw = tuple(torch.tensor(w, requires_grad=True) for w in weights["mla"])
     h = xt
+    outs = []
     for w_in, w_o in kw:
-        h = kda_layer(tree, h, w_in, w_o, dims, rounding)
-    y = mla_layer(tree, pos, h, *mw, dims, rounding)
+        h = kda_layer(tree, h, w_in, w_o, dims)
+        outs.append(h.detach().numpy())
+    y = mla_layer(tree, pos, h, *mw, dims)
     loss = (y * torch.from_numpy(np.asarray(dy, np.float64))).sum()
     flat = [xt] + [w for pair in kw for w in pair] + list(mw)
     grads = torch.autograd.grad(loss, flat)
     dk = [(grads[1 + 2 * i].numpy(), grads[2 + 2 * i].numpy()) for i in range(len(kw))]
     dm = tuple(g.numpy() for g in grads[1 + 2 * len(kw):])
-    return y.detach().numpy(), grads[0].numpy(), {"kda": dk, "mla": dm}
+    return y.detach().numpy(), grads[0].numpy(), {"kda": dk, "mla": dm}, outs
 
 
 def occurrence_sum(tree, r_expanded) -> np.ndarray:

@@ -43,8 +43,13 @@ STREAM = {
     "d_o_exp": 8, "init": 9,
     "x": 10, "d_y": 11,
     "h": 30, "w_vocab": 31, "targets": 32, "d_logp": 33,
+    "group_x": 50, "group_r": 51,
     # layer weights of the hybrid group: 100 + 16 * layer + matrix id
 }
+
+
+def group_weight_stream(layer: int, matrix: int) -> int:
+    return 100 + 16 * layer + matrix
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1):
@@ -305,3 +310,37 @@ def rows_normal(seed: int, stream: int, rows, width: int, dtype: str, scale: flo
     if scale != 1.0:
         z = z * scale
     return round_to(z, dtype).astype(np.float64)
+
+
+# ---------------------------------------------------------------- hybrid layer group inputs
+def group_small_tree() -> Tree:
+    """Six segments (150, 70, 95, 40, 66, 33 rows): every trajectory spans several 64-row chunks
+    and no fork point is chunk-aligned, so replay, ragged chunks and ragged tiles all occur."""
+    return Tree(parent=np.array([-1, 0, 0, 1, 1, 2], np.int32),
+                length=np.array([150, 70, 95, 40, 66, 33], np.int32))
+
+
+GROUP_DIMS = {"D": 2048, "H": 16, "d_head": 128, "d_rope": 64, "d_latent": 512}
+
+
+def group_weight_shapes(n_kda: int, dims=None):
+    d = dims or GROUP_DIMS
+    D, H = d["D"], d["H"]
+    kda = [((4 * D + H, D), (D, D))] * n_kda
+    mla = ((H * (d["d_head"] + d["d_rope"]) + d["d_latent"] + d["d_rope"], D), (2 * D, d["d_latent"]), (D, D))
+    return {"kda": kda, "mla": mla}
+
+
+def group_inputs(seed: int, tree: Tree, n_kda: int = 3, dims=None, with_r: bool = True):
+    """Layer-group inputs: x [N, D] fp32 normals (node order), weights N(0, 0.02) rounded to bf16
+    ({"kda": [(w_in, w_o)] * n_kda, "mla": (w_a, w_b, w_o)}, [out][in]) and the upstream
+    gradient R [n_expanded, D] fp32 normals per trajectory position (trajectories in leaf order)."""
+    d = dims or GROUP_DIMS
+    x = rows_normal(seed, STREAM["group_x"], np.arange(tree.n_rows), d["D"], "f32")
+    shapes = group_weight_shapes(n_kda, d)
+    kda = [tuple(normal_tensor(seed, group_weight_stream(l, m), shp, "bf16", 0.02) for m, shp in enumerate(pair))
+           for l, pair in enumerate(shapes["kda"])]
+    mla = tuple(normal_tensor(seed, group_weight_stream(15, m), shp, "bf16", 0.02)
+                for m, shp in enumerate(shapes["mla"]))
+    R = rows_normal(seed, STREAM["group_r"], np.arange(tree.n_expanded()), d["D"], "f32") if with_r else None
+    return x, {"kda": kda, "mla": mla}, R

@@ -53,3 +53,39 @@ def test_tree_attention_matches_oracle(tpc, cfg, H):
                                       int(sum(tree.length[u] for u in tree.path(v))))
                             for v in range(tree.n)])
     assert np.array_equal(pos, comp(depth))
+
+
+def test_tree_attention_split_inputs(tpc):
+    """q, k, v and dO given as fp32 values in bf16 hi/lo pairs: results match the oracle on the fp32
+    values (no bf16 rounding of any input)."""
+    import torch
+    tree = synth.workload("agentic_small").tree
+    N, H = tree.n_rows, 2
+    seed = 32
+    q = synth.normal_tensor(seed, 40, (N, H, 192), "f32")
+    k = synth.normal_tensor(seed, 41, (N, H, 192), "f32")
+    v = synth.normal_tensor(seed, 42, (N, H, 128), "f32")
+    d_o = synth.normal_tensor(seed, 43, (N, H, 128), "f32")
+    scale = 1.0 / np.sqrt(192.0)
+    o_ref, lse_ref = oat.tree_forward(tree, q, k, v, scale)
+    dq_ref, dk_ref, dv_ref = oat.tree_backward(tree, q, k, v, scale, d_o)
+    plan = tpc.Plan(tree.parent, tree.length, 64).upload()
+    st = tree.node_start()
+    comp = lambda a: plan.to_compact(a, st, tree.length)
+    f32 = lambda a: torch.tensor(comp(a), dtype=torch.float32).cuda()
+    qh, ql = tpc.split_bf16(f32(q))
+    kh, kl = tpc.split_bf16(f32(k))
+    vh, vl = tpc.split_bf16(f32(v))
+    gh, gl = tpc.split_bf16(f32(d_o))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = tpc.tpc_tree_attn_forward(plan, qh, kh, vh, scale, out_dtype=torch.float32, status=status, q_lo=ql,
+                                       k_lo=kl, v_lo=vl)
+    dq, dk, dv = tpc.tpc_tree_attn_backward(plan, qh, kh, vh, o, lse, gh, scale, status=status, q_lo=ql, k_lo=kl,
+                                            v_lo=vl, d_o_lo=gl)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    errs = {"o": err_ratio(o.cpu().numpy(), comp(o_ref)), "lse": err_ratio(lse.cpu().numpy(), comp(lse_ref)),
+            "dq": err_ratio(dq.cpu().numpy(), comp(dq_ref)), "dk": err_ratio(dk.cpu().numpy(), comp(dk_ref)),
+            "dv": err_ratio(dv.cpu().numpy(), comp(dv_ref))}
+    print("split", errs)
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs

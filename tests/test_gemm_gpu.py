@@ -54,3 +54,27 @@ def test_gemm_rejects_bad_arguments(tpc):
     with pytest.raises(tpc.TpcError) as e:
         tpc.tpc_gemm_bf16(a, b)
     assert e.value.code == 2
+
+
+@pytest.mark.parametrize("M,N,K,passes", [(300, 500, 200, 2), (700, 1030, 2048, 2), (2048, 512, 454, 3)])
+def test_split_gemm_is_fp32_accurate(tpc, M, N, K, passes):
+    """fp32 operands as bf16 hi/lo pairs: the product matches fp64 to fp32 accumulation accuracy
+    (a bf16 operand rounding alone would leave errors near 2^-9 relative)."""
+    import torch
+    g = torch.Generator(device="cuda").manual_seed(M + N + K)
+    A = torch.randn(M, K, device="cuda", generator=g)
+    if passes == 2:
+        W = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+        ah, al = tpc.split_bf16(A)
+        C = tpc.tpc_gemm_split(ah, al, W, None)
+        ref = A.double() @ W.double().t()
+    else:  # weight-gradient form: both operands fp32 and stored MN-major ([K][M], [K][N])
+        Bt = torch.randn(K, N, device="cuda", generator=g)
+        At = A.t().contiguous()
+        ah, al = tpc.split_bf16(At)
+        bh, bl = tpc.split_bf16(Bt)
+        C = tpc.tpc_gemm_split(ah, al, bh, bl, a_mn=True, b_mn=True)
+        ref = A.double() @ Bt.double()
+    torch.cuda.synchronize()
+    err = ((C.double() - ref).abs().max() / ref.pow(2).mean().sqrt()).item()
+    assert err < 1e-4, err

@@ -96,6 +96,14 @@ def test_agentic_small_bf16(tpc):
     print("agentic_small errors", errs)
 
 
+def test_agentic_small_fp32_inputs_on_tensor_cores(tpc):
+    """fp32 inputs at d = 128, chunk 64 take the tensor-core kernels with split (hi/lo) operands."""
+    w = synth.workload("agentic_small")
+    case = Case(w.tree, 4, 128, 64, "f32", w.seed + 7)
+    errs = check(case, run_case(tpc, case)[1], TOL["bf16"])
+    print("agentic_small fp32-input errors", errs)
+
+
 def test_tree_forward_bitwise_equals_expanded(tpc):
     """Same chunk grid -> same arithmetic: every trajectory's outputs and final state are
     bitwise equal between the tree-packed call and the trajectory-expanded call."""

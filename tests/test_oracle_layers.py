@@ -1,7 +1,6 @@
 """Pins of the hybrid layer-group oracle (oracle.layers) against facts that do not come from it:
 numerical derivatives, per-trajectory runs of the same group, closed forms of its pieces."""
 import numpy as np
-import pytest
 import torch
 
 import synth
@@ -18,19 +17,19 @@ def tiny_weights(seed, dims, n_kda, scale=0.3):
 
 
 def loss(tree, x, weights, dy, dims):
-    y, _ = ol.group_forward(tree, x, weights, dims, rounding=False)
+    y, _ = ol.group_forward(tree, x, weights, dims)
     return float((y * dy).sum())
 
 
 def test_group_gradients_match_central_differences():
-    """Directional derivatives of the exact fp64 group (rounding off) on the worked-example tree."""
+    """Directional derivatives of the fp64 group on the worked-example tree."""
     tree = synth.fig1_tree()
     rng = np.random.default_rng(1)
     N = tree.n_rows
     x = rng.normal(size=(N, TINY.D))
     dy = rng.normal(size=(N, TINY.D))
     weights = tiny_weights(2, TINY, n_kda=2)
-    _, dx, dw = ol.group_backward(tree, x, weights, dy, TINY, rounding=False)
+    _, dx, dw, _ = ol.group_backward(tree, x, weights, dy, TINY)
     eps = 1e-5
 
     def check(analytic, perturb):
@@ -55,32 +54,28 @@ def test_group_gradients_match_central_differences():
         check(dw["mla"][wi], pert)
 
 
-@pytest.mark.parametrize("rounding", [False, True])
-def test_tree_group_equals_each_trajectory_alone(rounding):
+def test_tree_group_equals_each_trajectory_alone():
     """Running the group once on the tree gives every trajectory what it gets when run alone as a
     chain (HARTS Figure 1), and the tree's gradients are the sums of the trajectories' gradients
-    under the expanded loss sum_j <y_j, R_j>.  With bf16 rounding the forward still agrees exactly;
-    the gradients do not, since the tree rounds the occurrence-summed upstream gradient once."""
+    under the expanded loss sum_j <y_j, R_j>."""
     tree = synth.fig1_tree()
     rng = np.random.default_rng(3)
     x = rng.normal(size=(tree.n_rows, TINY.D))
     weights = tiny_weights(4, TINY, n_kda=1)
     R = rng.normal(size=(tree.n_expanded(), TINY.D))
-    y, dx, dw = ol.group_backward(tree, x, weights, ol.occurrence_sum(tree, R), TINY, rounding)
+    y, dx, dw, _ = ol.group_backward(tree, x, weights, ol.occurrence_sum(tree, R), TINY)
     dx_sum = np.zeros_like(dx)
     dw_sum = None
     j = 0
     for leaf in tree.leaves():
         rows = tree.trajectory_rows(leaf)
         chain = synth.Tree(parent=np.array([-1], np.int32), length=np.array([len(rows)], np.int32))
-        yt, dxt, dwt = ol.group_backward(chain, x[rows], weights, R[j:j + len(rows)], TINY, rounding)
+        yt, dxt, dwt, _ = ol.group_backward(chain, x[rows], weights, R[j:j + len(rows)], TINY)
         j += len(rows)
         assert np.allclose(yt, y[rows], rtol=0, atol=1e-12)
         np.add.at(dx_sum, rows, dxt)
         flat = [w for p in dwt["kda"] for w in p] + list(dwt["mla"])
         dw_sum = flat if dw_sum is None else [a + b for a, b in zip(dw_sum, flat)]
-    if rounding:
-        return
     assert np.allclose(dx_sum, dx, rtol=0, atol=1e-10)
     for a, b in zip(dw_sum, [w for p in dw["kda"] for w in p] + list(dw["mla"])):
         assert np.allclose(a, b, rtol=0, atol=1e-9 * max(1.0, np.abs(b).max()))
@@ -142,7 +137,7 @@ def test_kda_layer_gate_and_norm_values():
     w_in[d.D:2 * d.D, 0] = np.arange(1, d.D + 1)    # key projections (any scale)
     parts = {}
     ol.kda_layer(tree, torch.tensor(x), torch.tensor(w_in), torch.zeros(d.D, d.D, dtype=torch.float64), d,
-                 rounding=False, parts=parts)
+                 parts=parts)
     g = parts["g"][0, 0, :4].numpy()
     assert np.allclose(g, [-0.1 * np.log(2.0), -3.0, 0.0, -0.1 * np.log(1 + np.exp(2.0))], atol=1e-12)
     assert np.allclose(parts["beta"][0].numpy(), [0.5, 1 / (1 + np.exp(-3.0))], atol=1e-15)
@@ -159,7 +154,7 @@ def test_mla_scores_equal_the_absorbed_latent_form():
     w = tiny_weights(7, d, 0)["mla"]
     parts = {}
     pos = torch.from_numpy(ol.depth_positions(tree))
-    ol.mla_layer(tree, pos, x, *(torch.tensor(a) for a in w), d, rounding=False, parts=parts)
+    ol.mla_layer(tree, pos, x, *(torch.tensor(a) for a in w), d, parts=parts)
     c = parts["c"]
     for h in range(d.H):
         qn = parts["q"][:, h, :d.d_head]
@@ -168,10 +163,3 @@ def test_mla_scores_equal_the_absorbed_latent_form():
         assert torch.allclose(qn @ kn.T, (qn @ w_uk) @ c.T, rtol=1e-10, atol=1e-10)
         # every head sees the same rotary key
         assert torch.equal(parts["k"][:, h, d.d_head:], parts["kr"])
-
-
-def test_bf16_rounding_points():
-    v = torch.tensor([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 3.14159], dtype=torch.float64)
-    r = ol.to_bf16(v)
-    # ties go to even; 3.14159 -> 3.140625 (8 significant bits)
-    assert r.tolist() == [1.0, 1.0, 1.0 + 2 ** -6, 3.140625]

@@ -70,6 +70,25 @@ class KdaBwdIO(ctypes.Structure):
 
 # exported symbols of include/tpc.h: name -> (restype, argtypes)
 _V, _P = ctypes.c_void_p, ctypes.POINTER
+GROUP_MAX_KDA = 8
+
+
+class AttnLo(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("d_o", ctypes.c_void_p)]
+
+
+class GroupShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("D", "H", "d_head", "d_rope", "d_latent", "n_kda")]
+
+
+class GroupWeights(ctypes.Structure):
+    _fields_ = [("kda", (ctypes.c_void_p * 2) * GROUP_MAX_KDA), ("mla", ctypes.c_void_p * 3)]
+
+
+class GroupGrads(ctypes.Structure):
+    _fields_ = [("kda", (ctypes.c_void_p * 2) * GROUP_MAX_KDA), ("mla", ctypes.c_void_p * 3)]
+
+
 SIGNATURES = {
     "tpc_last_error": (ctypes.c_char_p, []),
     "tpc_version": (ctypes.c_char_p, []),
@@ -90,14 +109,22 @@ SIGNATURES = {
     "tpc_gemm_bf16": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_float, ctypes.c_float, _V, _V]),
+    "tpc_gemm_split": (ctypes.c_int, [_V, _V, _V, _V, _V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, ctypes.c_float, ctypes.c_float, _V, _V]),
     "tpc_logprob_scratch_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int32]),
     "tpc_logprob_forward": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V, _V, _V, _V, ctypes.c_size_t,
                                            ctypes.c_int32, _V, _V]),
     "tpc_logprob_backward": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V, _V, _V, _V, _V, _V,
                                             ctypes.c_size_t, ctypes.c_int32, _V, _V]),
-    "tpc_tree_attn_forward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V]),
-    "tpc_tree_attn_backward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V]),
+    "tpc_tree_attn_forward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V]),
+    "tpc_tree_attn_backward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V]),
     "tpc_rope_positions": (ctypes.c_int, [_V, _V, _V]),
+    "tpc_group_workspace_bytes": (ctypes.c_size_t, [_V, _P(GroupShape)]),
+    "tpc_group_forward": (ctypes.c_int, [_V, _P(GroupShape), _P(GroupWeights), _V, _V, _V, _V, ctypes.c_size_t, _V]),
+    "tpc_group_backward": (ctypes.c_int, [_V, _P(GroupShape), _P(GroupWeights), _V, _V, _V, _V, _P(GroupGrads), _V,
+                                          ctypes.c_size_t, _V]),
+    "tpc_group_status": (ctypes.c_int, [_V, _P(GroupShape), _V, _V]),
     "tpc_profile_enable": (None, [ctypes.c_int]),
     "tpc_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t]),
     "tpc_launch_count": (ctypes.c_longlong, []),
@@ -350,6 +377,29 @@ def tpc_gemm_bf16(a, b, c=None, a_mn=False, b_mn=False, out_dtype=None, alpha=1.
     return c
 
 
+def split_bf16(x):
+    """(hi, lo) bf16 pair of an fp32 tensor: hi = bf16(x), lo = bf16(x - hi) (host-side helper for tests)."""
+    import torch
+    hi = x.to(torch.bfloat16)
+    lo = (x - hi.float()).to(torch.bfloat16)
+    return hi, lo
+
+
+def tpc_gemm_split(a, a_lo, b, b_lo, c=None, a_mn=False, b_mn=False, alpha=1.0, beta=0.0, status=None, stream=None):
+    """C = alpha (A B + A_lo B + A B_lo) + beta C; a_lo / b_lo may be None.  fp32 C."""
+    import torch
+    M = a.shape[1] if a_mn else a.shape[0]
+    K = a.shape[0] if a_mn else a.shape[1]
+    N = b.shape[1] if b_mn else b.shape[0]
+    if c is None:
+        c = torch.empty(M, N, dtype=torch.float32, device=a.device)
+    _check(lib().tpc_gemm_split(a.data_ptr(), None if a_lo is None else a_lo.data_ptr(), b.data_ptr(),
+                                None if b_lo is None else b_lo.data_ptr(), c.data_ptr(), M, N, K, a.stride(0),
+                                b.stride(0), c.stride(0), int(a_mn), int(b_mn), TPC_F32, float(alpha), float(beta),
+                                None if status is None else status.data_ptr(), _stream_ptr(stream)))
+    return c
+
+
 # ------------------------------------------------------------------------------------ log-probabilities
 def logprob_scratch(V, chunk_rows, device="cuda"):
     import torch
@@ -392,21 +442,31 @@ def _attn_shape(q, v, scale, io_dtype):
                      TPC_BF16 if io_dtype == torch.bfloat16 else TPC_F32)
 
 
-def tpc_tree_attn_forward(plan: Plan, q, k, v, scale, out_dtype=None, status=None, stream=None):
-    """Tree-masked attention forward; returns (o, lse)."""
+def _attn_lo(q_lo=None, k_lo=None, v_lo=None, d_o_lo=None):
+    if q_lo is None and k_lo is None and v_lo is None and d_o_lo is None:
+        return None
+    dp = lambda t: None if t is None else t.data_ptr()
+    return ctypes.byref(AttnLo(dp(q_lo), dp(k_lo), dp(v_lo), dp(d_o_lo)))
+
+
+def tpc_tree_attn_forward(plan: Plan, q, k, v, scale, out_dtype=None, status=None, stream=None, q_lo=None, k_lo=None,
+                          v_lo=None, o=None, lse=None):
+    """Tree-masked attention forward; returns (o, lse).  *_lo: optional bf16 low parts (hi/lo pairs)."""
     import torch
     out_dtype = out_dtype or torch.float32
     N, H, _ = q.shape
-    o = torch.empty(N, H, v.shape[2], dtype=out_dtype, device=q.device)
-    lse = torch.empty(N, H, dtype=torch.float32, device=q.device)
-    sh = _attn_shape(q, v, scale, out_dtype)
-    _check(lib().tpc_tree_attn_forward(plan.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                       _ptr(status), _stream_ptr(stream)))
+    o = o if o is not None else torch.empty(N, H, v.shape[2], dtype=out_dtype, device=q.device)
+    lse = lse if lse is not None else torch.empty(N, H, dtype=torch.float32, device=q.device)
+    sh = _attn_shape(q, v, scale, o.dtype)
+    _check(lib().tpc_tree_attn_forward(plan.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v),
+                                       _attn_lo(q_lo, k_lo, v_lo), _ptr(o), _ptr(lse), _ptr(status),
+                                       _stream_ptr(stream)))
     return o, lse
 
 
-def tpc_tree_attn_backward(plan: Plan, q, k, v, o, lse, d_o, scale, status=None, stream=None):
-    """Gradients (dq, dk, dv) in o's dtype."""
+def tpc_tree_attn_backward(plan: Plan, q, k, v, o, lse, d_o, scale, status=None, stream=None, q_lo=None, k_lo=None,
+                           v_lo=None, d_o_lo=None):
+    """Gradients (dq, dk, dv) in o's dtype.  *_lo: optional bf16 low parts (hi/lo pairs)."""
     import torch
     N, H, _ = q.shape
     dq = torch.empty(q.shape, dtype=o.dtype, device=q.device)
@@ -414,9 +474,9 @@ def tpc_tree_attn_backward(plan: Plan, q, k, v, o, lse, d_o, scale, status=None,
     dv = torch.empty(v.shape, dtype=o.dtype, device=q.device)
     delta = torch.empty(N, H, dtype=torch.float32, device=q.device)
     sh = _attn_shape(q, v, scale, o.dtype)
-    _check(lib().tpc_tree_attn_backward(plan.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                        _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(delta), _ptr(status),
-                                        _stream_ptr(stream)))
+    _check(lib().tpc_tree_attn_backward(plan.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v),
+                                        _attn_lo(q_lo, k_lo, v_lo, d_o_lo), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq),
+                                        _ptr(dk), _ptr(dv), _ptr(delta), _ptr(status), _stream_ptr(stream)))
     return dq, dk, dv
 
 
@@ -425,3 +485,77 @@ def tpc_rope_positions(plan: Plan, device="cuda", stream=None):
     pos = torch.empty(plan.info["n_unique"], dtype=torch.int32, device=device)
     _check(lib().tpc_rope_positions(plan.handle, _ptr(pos), _stream_ptr(stream)))
     return pos
+
+
+# ------------------------------------------------------------------------------------ hybrid layer group
+GROUP_DIMS = {"D": 2048, "H": 16, "d_head": 128, "d_rope": 64, "d_latent": 512}
+
+
+def group_shape(n_kda: int = 3) -> GroupShape:
+    d = GROUP_DIMS
+    return GroupShape(d["D"], d["H"], d["d_head"], d["d_rope"], d["d_latent"], n_kda)
+
+
+def group_weight_shapes(n_kda: int = 3):
+    """{"kda": [(w_in, w_o) shapes] * n_kda, "mla": (w_a, w_b, w_o) shapes}, [out][in] row-major."""
+    d = GROUP_DIMS
+    D, H = d["D"], d["H"]
+    kda = (4 * D + H, D), (D, D)
+    mla = (H * (d["d_head"] + d["d_rope"]) + d["d_latent"] + d["d_rope"], D), (2 * D, d["d_latent"]), (D, D)
+    return {"kda": [kda] * n_kda, "mla": mla}
+
+
+def _group_ptrs(struct_cls, tensors):
+    s = struct_cls()
+    for i, pair in enumerate(tensors["kda"]):
+        for j, t in enumerate(pair):
+            s.kda[i][j] = t.data_ptr()
+    for j, t in enumerate(tensors["mla"]):
+        s.mla[j] = t.data_ptr()
+    return s
+
+
+def tpc_group_workspace_bytes(plan: Plan, n_kda: int = 3) -> int:
+    sh = group_shape(n_kda)
+    return int(lib().tpc_group_workspace_bytes(plan.handle, ctypes.byref(sh)))
+
+
+def group_workspace(plan: Plan, n_kda: int = 3, device="cuda"):
+    import torch
+    return torch.empty(tpc_group_workspace_bytes(plan, n_kda), dtype=torch.uint8, device=device)
+
+
+def tpc_group_forward(plan: Plan, weights, x, ws, h=None, y=None, stream=None):
+    """Forward of the layer group on compact rows x (fp32 [N][2048]); returns (y, h)."""
+    import torch
+    n_kda = len(weights["kda"])
+    N, D = x.shape
+    h = h if h is not None else torch.empty(max(n_kda, 1), N, D, dtype=torch.float32, device=x.device)
+    y = y if y is not None else torch.empty_like(x)
+    sh = group_shape(n_kda)
+    w = _group_ptrs(GroupWeights, weights)
+    _check(lib().tpc_group_forward(plan.handle, ctypes.byref(sh), ctypes.byref(w), _ptr(x), _ptr(h), _ptr(y),
+                                   _ptr(ws), ws.numel(), _stream_ptr(stream)))
+    return y, h
+
+
+def tpc_group_backward(plan: Plan, weights, x, h, dy, ws, dx=None, grads=None, stream=None):
+    """Backward (with recomputation) of sum <dy, y>; returns (dx, grads) with fp32 weight gradients."""
+    import torch
+    n_kda = len(weights["kda"])
+    dx = dx if dx is not None else torch.empty_like(dy)
+    if grads is None:
+        grads = {"kda": [tuple(torch.empty(w.shape, dtype=torch.float32, device=x.device) for w in pair)
+                         for pair in weights["kda"]],
+                 "mla": tuple(torch.empty(w.shape, dtype=torch.float32, device=x.device) for w in weights["mla"])}
+    sh = group_shape(n_kda)
+    w = _group_ptrs(GroupWeights, weights)
+    g = _group_ptrs(GroupGrads, grads)
+    _check(lib().tpc_group_backward(plan.handle, ctypes.byref(sh), ctypes.byref(w), _ptr(x), _ptr(h), _ptr(dy),
+                                    _ptr(dx), ctypes.byref(g), _ptr(ws), ws.numel(), _stream_ptr(stream)))
+    return dx, grads
+
+
+def tpc_group_status(plan: Plan, ws, n_kda: int = 3, stream=None) -> int:
+    sh = group_shape(n_kda)
+    return int(lib().tpc_group_status(plan.handle, ctypes.byref(sh), _ptr(ws), _stream_ptr(stream)))

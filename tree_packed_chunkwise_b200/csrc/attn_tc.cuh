@@ -9,6 +9,11 @@
 // deterministic: dQ per query tile (S and dP = dO V^T recomputed, dQ += dS K accumulated in TMEM);
 // dK, dV per key tile (<= 64 rows of one node), looping over the query rows that can see it: the
 // node's subtree rows from the tile on, one contiguous range in the compact layout.
+//
+// SPLIT kernels take q, k, v and dO as bf16 hi/lo pairs (fp32 values x = hi + lo to 2^-17
+// relative) and form every product from three partial products (hi hi + lo hi + hi lo), so that
+// fp32 inputs and upstream gradients enter without a bf16 rounding of their own.  The dQ kernel
+// then walks the keys in tiles of 32 (the split tiles take twice the shared memory).
 #pragma once
 #include "kda_tc.cuh"
 
@@ -19,18 +24,18 @@ constexpr int kAttnQK = 192, kAttnDV = 128, kAttnThreads = 128;
 namespace tck {
 
 // key tiles of a query tile: f(row start, rows, own-node flag) in a fixed order; stops on false
-template <class F>
+template <int KT = 64, class F>
 __device__ __forceinline__ bool for_key_tiles(const DevTables& t, const AttnTile& qt, F f) {
   const AttnNode nd = t.attn_nodes[qt.node];
   const int r1 = t.attn_nodes[qt.node + 1].range_begin;
   for (int r = nd.range_begin; r < r1; ++r) {
     const RowRange rr = t.attn_ranges[r];
-    for (int k0 = rr.start; k0 < rr.end; k0 += 64)
-      if (!f(k0, min(64, rr.end - k0), false)) return false;
+    for (int k0 = rr.start; k0 < rr.end; k0 += KT)
+      if (!f(k0, min(KT, rr.end - k0), false)) return false;
   }
   const int end = qt.row + qt.n;
-  for (int k0 = nd.row_offset; k0 < end; k0 += 64)
-    if (!f(k0, min(64, end - k0), true)) return false;
+  for (int k0 = nd.row_offset; k0 < end; k0 += KT)
+    if (!f(k0, min(KT, end - k0), true)) return false;
   return true;
 }
 
@@ -52,26 +57,32 @@ __device__ __forceinline__ void st_out16(T* p, const float* v) {
 }  // namespace tck
 
 // ------------------------------------------------------------------------------------------ forward
+template <bool SPLIT>
 struct AttnFwdSmem {
   static constexpr size_t Qb = size_t(128) * kAttnQK * 2, Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
-  static constexpr size_t Pb = size_t(128) * 64 * 2;
-  static constexpr size_t Q = 0, K = Q + Qb, V = K + Kb, P = V + Vb;
+  static constexpr size_t Pb = size_t(128) * 64 * 2, X = SPLIT ? 1 : 0;
+  static constexpr size_t Q = 0, Ql = Q + Qb, K = Ql + X * Qb, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb;
+  static constexpr size_t P = Vl + X * Vb;
   static constexpr size_t total = P + 2 * Pb;
+  static_assert(total <= 227 * 1024, "shared memory");
 };
 
-template <typename Tout>
+template <typename Tout, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
-                const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, Tout* __restrict__ o,
-                float* __restrict__ lse, int* status) {
+                const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
+                const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
+                const __nv_bfloat16* __restrict__ v_lo, Tout* __restrict__ o, float* __restrict__ lse,
+                int* status) {
   using namespace tck;
-  using S = AttnFwdSmem;
+  using S = AttnFwdSmem<SPLIT>;
   using bf = __nv_bfloat16;
   constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
   const AttnTile qt = t.attn_qtiles[blockIdx.x];
   const int h = blockIdx.y, tid = threadIdx.x;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  uint8_t *sQ = asmem + S::Q, *sK = asmem + S::K, *sV = asmem + S::V, *sPh = asmem + S::P, *sPl = sPh + S::Pb;
+  uint8_t *sQ = asmem + S::Q, *sQl = asmem + S::Ql, *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V,
+          *sVl = asmem + S::Vl, *sPh = asmem + S::P, *sPl = sPh + S::Pb;
   __shared__ __align__(8) uint64_t bar;
   __shared__ uint32_t tslot;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 256);
@@ -83,6 +94,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   build_tile_ld<128, DQ, false, bf, NT>(
       sQ, nullptr, [&](int a) -> const bf* { return a < qt.n ? q + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; },
       ident);
+  if constexpr (SPLIT)
+    build_tile_ld<128, DQ, false, bf, NT>(
+        sQl, nullptr,
+        [&](int a) -> const bf* { return a < qt.n && q_lo ? q_lo + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; },
+        ident);
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
@@ -98,9 +114,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
     build_tile_ld<64, DV, false, bf, NT>(
         sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+    if constexpr (SPLIT) {
+      build_tile_ld<64, DQ, false, bf, NT>(
+          sKl, nullptr,
+          [&](int a) -> const bf* { return a < nk && k_lo ? k_lo + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
+      build_tile_ld<64, DV, false, bf, NT>(
+          sVl, nullptr,
+          [&](int a) -> const bf* { return a < nk && v_lo ? v_lo + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+    }
     if (!run(sy, [&] {
-          mma_chain(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sK), 64, false}, DQ,
-                    tc::idesc_bf16(128, 64, false, false), false);
+          mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
+               tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sKl), 64, false}, DQ,
+               tc::idesc_bf16(128, 64, false, false), false, !SPLIT, !SPLIT);
         }))
       return false;
     float s[64];
@@ -127,8 +152,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int j = 0; j < 64; j += 16) put16<128, true>(sPh, sPl, tid, j, s + j);
     if (!run(sy, [&] {
           mma4(tb + 64, tc::Op{tc::smem_u32(sPh), 128, false}, tc::Op{tc::smem_u32(sPl), 128, false},
-               tc::Op{tc::smem_u32(sV), 64, true}, tc::Op{tc::smem_u32(sV), 64, true}, 64,
-               tc::idesc_bf16(128, DV, false, true), false, false, true);
+               tc::Op{tc::smem_u32(sV), 64, true}, tc::Op{tc::smem_u32(sVl), 64, true}, 64,
+               tc::idesc_bf16(128, DV, false, true), false, false, !SPLIT);
         }))
       return false;
 #pragma unroll
@@ -159,28 +184,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // ------------------------------------------------------------------------------------------ backward dQ
 // per query tile: delta = rowsum(dO * O) (also written for the dK/dV kernel), then over the key
 // tiles P = exp(scale S - lse), dP = dO V^T, dS = P (dP - delta), dQ += dS K; dq = scale dQ.
+template <bool SPLIT>
 struct AttnDqSmem {
+  static constexpr int KT = SPLIT ? 32 : 64;  // key rows per tile
+  static constexpr size_t X = SPLIT ? 1 : 0;
   static constexpr size_t Qb = size_t(128) * kAttnQK * 2, Ob = size_t(128) * kAttnDV * 2;
-  static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2, Pb = size_t(128) * 64 * 2;
-  static constexpr size_t Q = 0, dO = Q + Qb, K = dO + Ob, V = K + Kb, dS = V + Vb;
+  static constexpr size_t Kb = size_t(KT) * kAttnQK * 2, Vb = size_t(KT) * kAttnDV * 2, Pb = size_t(128) * KT * 2;
+  static constexpr size_t Q = 0, Ql = Q + Qb, dO = Ql + X * Qb, dOl = dO + Ob, K = dOl + X * Ob, Kl = K + Kb;
+  static constexpr size_t V = Kl + X * Kb, Vl = V + Vb, dS = Vl + X * Vb;
   static constexpr size_t total = dS + 2 * Pb;
+  static_assert(total <= 227 * 1024, "shared memory");
 };
 
-template <typename Tio>
+template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_bwd_dq_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
-                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-                   const Tio* __restrict__ o, const float* __restrict__ lse, const __nv_bfloat16* __restrict__ d_o,
+                   const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
+                   const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
+                   const __nv_bfloat16* __restrict__ v_lo, const Tio* __restrict__ o, const float* __restrict__ lse,
+                   const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ d_o_lo,
                    Tio* __restrict__ dq, float* __restrict__ delta, int* status) {
   using namespace tck;
-  using S = AttnDqSmem;
+  using S = AttnDqSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads, KT = S::KT;
   const AttnTile qt = t.attn_qtiles[blockIdx.x];
   const int h = blockIdx.y, tid = threadIdx.x;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  uint8_t *sQ = asmem + S::Q, *sO = asmem + S::dO, *sK = asmem + S::K, *sV = asmem + S::V, *sDh = asmem + S::dS,
-          *sDl = sDh + S::Pb;
+  uint8_t *sQ = asmem + S::Q, *sQl = asmem + S::Ql, *sO = asmem + S::dO, *sOl = asmem + S::dOl, *sK = asmem + S::K,
+          *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl, *sDh = asmem + S::dS, *sDl = sDh + S::Pb;
   __shared__ __align__(8) uint64_t bar;
   __shared__ uint32_t tslot;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
@@ -189,18 +221,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   auto ident = [](int, int, float x) { return x; };
-  build_tile_ld<128, DQ, false, bf, NT>(
-      sQ, nullptr, [&](int a) -> const bf* { return a < qt.n ? q + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; },
-      ident);
-  build_tile_ld<128, DV, false, bf, NT>(
-      sO, nullptr, [&](int a) -> const bf* { return a < qt.n ? d_o + ((size_t)(qt.row + a) * H + h) * DV : nullptr; },
-      ident);
+  auto qrows = [&](const bf* base) {
+    return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; };
+  };
+  auto orows = [&](const bf* base) {
+    return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DV : nullptr; };
+  };
+  build_tile_ld<128, DQ, false, bf, NT>(sQ, nullptr, qrows(q), ident);
+  build_tile_ld<128, DV, false, bf, NT>(sO, nullptr, orows(d_o), ident);
+  if constexpr (SPLIT) {
+    build_tile_ld<128, DQ, false, bf, NT>(sQl, nullptr, qrows(q_lo), ident);
+    build_tile_ld<128, DV, false, bf, NT>(sOl, nullptr, orows(d_o_lo), ident);
+  }
   const int qrow = qt.row + tid;
   float dl = 0.f, ls = 0.f;
   if (tid < qt.n) {
     const Tio* orow = o + ((size_t)qrow * H + h) * DV;
     const bf* grow = d_o + ((size_t)qrow * H + h) * DV;
-    for (int j = 0; j < DV; ++j) dl = fmaf(to_f(orow[j]), __bfloat162float(grow[j]), dl);
+    const bf* glow = SPLIT && d_o_lo ? d_o_lo + ((size_t)qrow * H + h) * DV : nullptr;
+    for (int j = 0; j < DV; ++j)
+      dl = fmaf(to_f(orow[j]), __bfloat162float(grow[j]) + (glow ? __bfloat162float(glow[j]) : 0.f), dl);
     delta[(size_t)qrow * H + h] = dl;
     ls = lse[(size_t)qrow * H + h];
   }
@@ -210,37 +250,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t la = tb + ((uint32_t)(32 * (tid >> 5)) << 16);
   Sync sy{&bar, 0u, status};
   bool first = true;
-  const bool ok = for_key_tiles(t, qt, [&](int k0, int nk, bool own) -> bool {
-    build_tile_ld<64, DQ, false, bf, NT>(
-        sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
-    build_tile_ld<64, DV, false, bf, NT>(
-        sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+  const bool ok = for_key_tiles<KT>(t, qt, [&](int k0, int nk, bool own) -> bool {
+    auto krows = [&](const bf* base, int w) {
+      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * w : nullptr; };
+    };
+    build_tile_ld<KT, DQ, false, bf, NT>(sK, nullptr, krows(k, DQ), ident);
+    build_tile_ld<KT, DV, false, bf, NT>(sV, nullptr, krows(v, DV), ident);
+    if constexpr (SPLIT) {
+      build_tile_ld<KT, DQ, false, bf, NT>(sKl, nullptr, krows(k_lo, DQ), ident);
+      build_tile_ld<KT, DV, false, bf, NT>(sVl, nullptr, krows(v_lo, DV), ident);
+    }
     if (!run(sy, [&] {
-          mma_chain(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sK), 64, false}, DQ,
-                    tc::idesc_bf16(128, 64, false, false), false);
-          mma_chain(tb + 64, tc::Op{tc::smem_u32(sO), 128, false}, tc::Op{tc::smem_u32(sV), 64, false}, DV,
-                    tc::idesc_bf16(128, 64, false, false), false);
+          mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
+               tc::Op{tc::smem_u32(sK), KT, false}, tc::Op{tc::smem_u32(sKl), KT, false}, DQ,
+               tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
+          mma4(tb + 64, tc::Op{tc::smem_u32(sO), 128, false}, tc::Op{tc::smem_u32(sOl), 128, false},
+               tc::Op{tc::smem_u32(sV), KT, false}, tc::Op{tc::smem_u32(sVl), KT, false}, DV,
+               tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
         }))
       return false;
-    float s[64], dp[64];
-    tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
-    tc::tmem_ld32(la + 32, *reinterpret_cast<float(*)[32]>(s + 32));
-    tc::tmem_ld32(la + 64, *reinterpret_cast<float(*)[32]>(dp));
-    tc::tmem_ld32(la + 96, *reinterpret_cast<float(*)[32]>(dp + 32));
+    float s[KT], dp[KT];
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
+    for (int c = 0; c < KT; c += 32) {
+      tc::tmem_ld32(la + c, *reinterpret_cast<float(*)[32]>(s + c));
+      tc::tmem_ld32(la + 64 + c, *reinterpret_cast<float(*)[32]>(dp + c));
+    }
+#pragma unroll
+    for (int j = 0; j < KT; ++j) {
       const bool valid = tid < qt.n && j < nk && (!own || k0 + j <= qrow);
       const float p = valid ? expf(s[j] * scale - ls) : 0.f;
       s[j] = p * (dp[j] - dl);
     }
 #pragma unroll
-    for (int j = 0; j < 64; j += 16) put16<128, true>(sDh, sDl, tid, j, s + j);
+    for (int j = 0; j < KT; j += 16) put16<128, true>(sDh, sDl, tid, j, s + j);
     const bool acc_on = !first;
     first = false;
     if (!run(sy, [&] {
           mma4(tb + 128, tc::Op{tc::smem_u32(sDh), 128, false}, tc::Op{tc::smem_u32(sDl), 128, false},
-               tc::Op{tc::smem_u32(sK), 64, true}, tc::Op{tc::smem_u32(sK), 64, true}, 64,
-               tc::idesc_bf16(128, DQ, false, true), acc_on, false, true);
+               tc::Op{tc::smem_u32(sK), KT, true}, tc::Op{tc::smem_u32(sKl), KT, true}, KT,
+               tc::idesc_bf16(128, DQ, false, true), acc_on, false, !SPLIT);
         }))
       return false;
     tc::fence_before_sync();
@@ -269,28 +317,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // per key tile of node u: query rows [row of the tile, subtree end of u) in tiles of 64 (queries of u
 // itself only from the key row on), S^T = K Q^T, dP^T = V dO^T, P^T = exp(scale S^T - lse),
 // dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 64 accumulators.
+template <bool SPLIT>
 struct AttnDkvSmem {
   static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2, Pb = size_t(64) * 64 * 2;
-  static constexpr size_t K = 0, V = K + Kb, Q = V + Vb, dO = Q + Kb, P = dO + Vb, dS = P + 2 * Pb;
+  static constexpr size_t X = SPLIT ? 1 : 0;
+  static constexpr size_t K = 0, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb, Q = Vl + X * Vb, Ql = Q + Kb;
+  static constexpr size_t dO = Ql + X * Kb, dOl = dO + Vb, P = dOl + X * Vb, dS = P + 2 * Pb;
   static constexpr size_t vec = dS + 2 * Pb;  // lse[64], delta[64]
   static constexpr size_t total = vec + 2 * 64 * 4;
+  static_assert(total <= 227 * 1024, "shared memory");
 };
 
-template <typename Tio>
+template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_bwd_dkv_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
-                    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-                    const float* __restrict__ lse, const __nv_bfloat16* __restrict__ d_o,
+                    const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
+                    const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
+                    const __nv_bfloat16* __restrict__ v_lo, const float* __restrict__ lse,
+                    const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ d_o_lo,
                     const float* __restrict__ delta, Tio* __restrict__ dk, Tio* __restrict__ dv, int* status) {
   using namespace tck;
-  using S = AttnDkvSmem;
+  using S = AttnDkvSmem<SPLIT>;
   using bf = __nv_bfloat16;
   constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
   const AttnTile kt = t.attn_ktiles[blockIdx.x];
   const AttnNode nd = t.attn_nodes[kt.node];
   const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  uint8_t *sK = asmem + S::K, *sV = asmem + S::V, *sQ = asmem + S::Q, *sO = asmem + S::dO;
+  uint8_t *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl, *sQ = asmem + S::Q,
+          *sQl = asmem + S::Ql, *sO = asmem + S::dO, *sOl = asmem + S::dOl;
   uint8_t *sPh = asmem + S::P, *sPl = sPh + S::Pb, *sDh = asmem + S::dS, *sDl = sDh + S::Pb;
   float* sl = reinterpret_cast<float*>(asmem + S::vec);
   float* sd = sl + 64;
@@ -307,6 +362,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
   build_tile_ld<64, DV, false, bf, NT>(
       sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+  if constexpr (SPLIT) {
+    build_tile_ld<64, DQ, false, bf, NT>(
+        sKl, nullptr,
+        [&](int a) -> const bf* { return a < nk && k_lo ? k_lo + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
+    build_tile_ld<64, DV, false, bf, NT>(
+        sVl, nullptr,
+        [&](int a) -> const bf* { return a < nk && v_lo ? v_lo + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+  }
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
@@ -323,15 +386,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     build_tile_ld<64, DV, false, bf, NT>(
         sO, nullptr, [&](int a) -> const bf* { return a < nq ? d_o + ((size_t)(q0 + a) * H + h) * DV : nullptr; },
         ident);
+    if constexpr (SPLIT) {
+      build_tile_ld<64, DQ, false, bf, NT>(
+          sQl, nullptr,
+          [&](int a) -> const bf* { return a < nq && q_lo ? q_lo + ((size_t)(q0 + a) * H + h) * DQ : nullptr; },
+          ident);
+      build_tile_ld<64, DV, false, bf, NT>(
+          sOl, nullptr,
+          [&](int a) -> const bf* { return a < nq && d_o_lo ? d_o_lo + ((size_t)(q0 + a) * H + h) * DV : nullptr; },
+          ident);
+    }
     if (tid < 64) {
       sl[tid] = tid < nq ? lse[(size_t)(q0 + tid) * H + h] : 0.f;
       sd[tid] = tid < nq ? delta[(size_t)(q0 + tid) * H + h] : 0.f;
     }
     ok = run(sy, [&] {
-      mma_chain(tb, tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sQ), 64, false}, DQ,
-                tc::idesc_bf16(64, 64, false, false), false);
-      mma_chain(tb + 64, tc::Op{tc::smem_u32(sV), 64, false}, tc::Op{tc::smem_u32(sO), 64, false}, DV,
-                tc::idesc_bf16(64, 64, false, false), false);
+      mma4(tb, tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sKl), 64, false},
+           tc::Op{tc::smem_u32(sQ), 64, false}, tc::Op{tc::smem_u32(sQl), 64, false}, DQ,
+           tc::idesc_bf16(64, 64, false, false), false, !SPLIT, !SPLIT);
+      mma4(tb + 64, tc::Op{tc::smem_u32(sV), 64, false}, tc::Op{tc::smem_u32(sVl), 64, false},
+           tc::Op{tc::smem_u32(sO), 64, false}, tc::Op{tc::smem_u32(sOl), 64, false}, DV,
+           tc::idesc_bf16(64, 64, false, false), false, !SPLIT, !SPLIT);
     });
     if (!ok) break;
     float s[64], dp[64];
@@ -358,11 +433,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     first = false;
     ok = run(sy, [&] {
       mma4(tb + 128, tc::Op{tc::smem_u32(sPh), 64, false}, tc::Op{tc::smem_u32(sPl), 64, false},
-           tc::Op{tc::smem_u32(sO), 64, true}, tc::Op{tc::smem_u32(sO), 64, true}, 64,
-           tc::idesc_bf16(64, DV, false, true), acc_on, false, true);
+           tc::Op{tc::smem_u32(sO), 64, true}, tc::Op{tc::smem_u32(sOl), 64, true}, 64,
+           tc::idesc_bf16(64, DV, false, true), acc_on, false, !SPLIT);
       mma4(tb + 256, tc::Op{tc::smem_u32(sDh), 64, false}, tc::Op{tc::smem_u32(sDl), 64, false},
-           tc::Op{tc::smem_u32(sQ), 64, true}, tc::Op{tc::smem_u32(sQ), 64, true}, 64,
-           tc::idesc_bf16(64, DQ, false, true), acc_on, false, true);
+           tc::Op{tc::smem_u32(sQ), 64, true}, tc::Op{tc::smem_u32(sQl), 64, true}, 64,
+           tc::idesc_bf16(64, DQ, false, true), acc_on, false, !SPLIT);
     });
     tc::fence_before_sync();
     __syncthreads();

@@ -2,6 +2,11 @@
 // in TMEM.  A is M x K and B is K x N; each is given either K-major (K contiguous: A as [M][K], B
 // as [N][K]) or MN-major (M resp. N contiguous: A as [K][M], B as [K][N]).
 //
+// Split precision: an fp32 operand X is passed as two bf16 matrices, X_hi = bf16(X) and
+// X_lo = bf16(X - X_hi), so that X = X_hi + X_lo to 2^-17 relative.  The kernel accumulates up to
+// three products in one TMEM accumulator: A_hi B_hi (+ A_lo B_hi) (+ A_hi B_lo); the dropped
+// A_lo B_lo term is below 2^-16 of the product.  The K loop simply runs once per product.
+//
 // One CTA per 128 x 256 output tile, K in steps of 64 through a 4-stage shared-memory pipeline:
 // a producer thread issues TMA loads (one 16-byte-wide box per 8-element core-matrix column of the
 // no-swizzle canonical layout), an MMA thread issues tcgen05.mma and frees stages by tcgen05.commit,
@@ -30,11 +35,13 @@ struct GemmArgs {
   float alpha, beta;  // beta != 0 reads C (fp32 only)
   void* C;
   int* status;
+  int passes;         // 1: A B;  2: + A_lo B;  3: + A B_lo
 };
 
 template <int C_BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_bf16_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, GemmArgs g) {
+    gemm_bf16_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                 const __grid_constant__ CUtensorMap tma_alo, const __grid_constant__ CUtensorMap tma_blo, GemmArgs g) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t gsm[];
   __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], accb;
@@ -42,6 +49,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * kGemmBN;
   const int KT = (g.K + kGemmBK - 1) / kGemmBK;
+  const int IT = KT * g.passes;  // pass p = it / KT uses (A, B), (A_lo, B), (A, B_lo)
   if (w == 0) tmem_alloc(&tslot, 256);
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
@@ -57,34 +65,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   bool ok = true;
   if (w == 0 && lane == 0) {
     // producer
-    for (int kt = 0; kt < KT && ok; ++kt) {
-      const int s = kt % kGemmStages;
-      if (kt >= kGemmStages && !mbar_wait(&empty[s], ((kt / kGemmStages) - 1) & 1)) {
+    for (int it = 0; it < IT && ok; ++it) {
+      const int s = it % kGemmStages, pass = it / KT, kt = it - pass * KT;
+      if (it >= kGemmStages && !mbar_wait(&empty[s], ((it / kGemmStages) - 1) & 1)) {
         set_status(g.status, 8);
         ok = false;
         break;
       }
+      const CUtensorMap* ma = pass == 1 ? &tma_alo : &tma_a;
+      const CUtensorMap* mb = pass == 2 ? &tma_blo : &tma_b;
       uint8_t* sa = gsm + s * GemmSmem::stage;
       uint8_t* sb = sa + GemmSmem::Ab;
       mbar_arrive_expect_tx(&full[s], (uint32_t)GemmSmem::stage);
       const int k0 = kt * kGemmBK;
       if (!g.a_mn) {
-        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sa + j * (kGemmBM / 8) * 128, &tma_a, k0 + 8 * j, m0, &full[s]);
+        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sa + j * (kGemmBM / 8) * 128, ma, k0 + 8 * j, m0, &full[s]);
       } else {
-        for (int j = 0; j < kGemmBM / 8; ++j) tma_load_2d(sa + j * (kGemmBK / 8) * 128, &tma_a, m0 + 8 * j, k0, &full[s]);
+        for (int j = 0; j < kGemmBM / 8; ++j) tma_load_2d(sa + j * (kGemmBK / 8) * 128, ma, m0 + 8 * j, k0, &full[s]);
       }
       if (!g.b_mn) {
-        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sb + j * (kGemmBN / 8) * 128, &tma_b, k0 + 8 * j, n0, &full[s]);
+        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sb + j * (kGemmBN / 8) * 128, mb, k0 + 8 * j, n0, &full[s]);
       } else {
-        for (int j = 0; j < kGemmBN / 8; ++j) tma_load_2d(sb + j * (kGemmBK / 8) * 128, &tma_b, n0 + 8 * j, k0, &full[s]);
+        for (int j = 0; j < kGemmBN / 8; ++j) tma_load_2d(sb + j * (kGemmBK / 8) * 128, mb, n0 + 8 * j, k0, &full[s]);
       }
     }
   } else if (w == 1 && lane == 0) {
     // MMA issuer
     const uint32_t id = idesc_bf16(kGemmBM, kGemmBN, g.a_mn != 0, g.b_mn != 0);
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % kGemmStages;
-      if (!mbar_wait(&full[s], (kt / kGemmStages) & 1)) {
+    for (int it = 0; it < IT; ++it) {
+      const int s = it % kGemmStages;
+      if (!mbar_wait(&full[s], (it / kGemmStages) & 1)) {
         set_status(g.status, 8);
         ok = false;
         break;
@@ -93,7 +103,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint8_t* sa = gsm + s * GemmSmem::stage;
       const Op a{smem_u32(sa), g.a_mn ? kGemmBK : kGemmBM, g.a_mn != 0};
       const Op b{smem_u32(sa + GemmSmem::Ab), g.b_mn ? kGemmBK : kGemmBN, g.b_mn != 0};
-      mma_chain(tb, a, b, kGemmBK, id, kt > 0);
+      mma_chain(tb, a, b, kGemmBK, id, it > 0);
       commit(&empty[s]);
     }
     commit(&accb);

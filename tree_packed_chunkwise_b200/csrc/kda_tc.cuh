@@ -915,13 +915,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   dG  = pdG + Kbar beta dB_k + k (e^{G-G_0} (dAt bf) - e^{G_0-G} (dAt^T af)),  dg = reverse cumsum of dG
 //   dv  = beta dB_v,  dbeta = rowsum(dB_k Kbar + dB_v v + dA Atilde)
 // Replayed rows go to the replay partials, rows replayed elsewhere to the target staging.
-struct BdkvTcSmem {
+// bf16 inputs stage the chunk's k rows in shared memory; fp32 inputs (twice the bytes, which do not
+// fit beside the other tiles) read them from global memory instead.
+template <typename Tin>
+struct BdkvTcSmemT {
+  static constexpr bool kStageK = sizeof(Tin) == 2;
   static constexpr int C = kTcC, D = kTcD, LD = D + 1, LC = C + 1;
   static constexpr size_t G = 0;
   static constexpr size_t At = G + sizeof(float) * C * LD;        // Atilde fp32 [C][LC]
   static constexpr size_t vec = At + sizeof(float) * C * LC;      // beta[C], ref[D], dbeta parts[6][C]
   static constexpr size_t Ks = (vec + sizeof(float) * (C + D + 6 * C) + 15) & ~size_t(15);      // staged k rows
-  static constexpr size_t Tt = (Ks + sizeof(__nv_bfloat16) * C * tck::kStagePitch + 1023) & ~size_t(1023);  // T tile
+  static constexpr size_t Tt = (Ks + (kStageK ? sizeof(Tin) * C * tck::kStagePitch : 0) + 1023) & ~size_t(1023);  // T tile
   static constexpr size_t CCb = size_t(C) * C * 2, CDb = size_t(C) * D * 2, DDb = size_t(D) * D * 2;
   static constexpr size_t R = Tt + 2 * CCb;
   static constexpr size_t Rbytes = 128 * 1024;
@@ -937,6 +941,7 @@ struct BdkvTcSmem {
   static constexpr size_t p5_dA = 0, p5_bf = 2 * CCb, p5_af = p5_bf + 2 * CDb;         // dAt, bf (MN), af (MN)
   static_assert(p2_V + 2 * CDb <= Rbytes && p2_S0 + 2 * DDb <= Rbytes && p3_dX + 4 * CDb <= Rbytes, "R");
   static_assert(inv_W2 + sizeof(float) * 4 * 16 * 17 <= p2_Tp, "inverse scratch overlaps T'");
+  static_assert(total <= 227 * 1024, "shared memory");
 };
 
 template <typename Tin, typename Tout>
@@ -945,7 +950,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, Tout* __restrict__ dk_,
                    Tout* __restrict__ dv_, float* __restrict__ dg_, float* __restrict__ dbeta_, KdaWs ws) {
   using namespace tck;
-  using S = BdkvTcSmem;
+  using S = BdkvTcSmemT<Tin>;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
   const int ci = blockIdx.x, h = blockIdx.y;
@@ -974,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
   for (int e = tid; e < 6 * C; e += blockDim.x) sdb[e] = 0.f;
   Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
-  stage_rows(sk, k_, srow, H, h, n);
+  if constexpr (S::kStageK) stage_rows(sk, k_, srow, H, h, n);
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
@@ -984,6 +989,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   Sync sy{&bar, 0u, ws.status};
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  // 16 values of k row r from column c0 on (zero for r >= n)
+  auto k16 = [&](int r, int c0, float(&kv)[16]) {
+    if constexpr (S::kStageK) {
+      staged16(sk, r, c0, kv);
+    } else if (r < n) {
+      const Tin* p = k_ + ((size_t)srow[r] * H + h) * D + c0;
+      float a[8], b[8];
+      ld8(p, a);
+      ld8(p + 8, b);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        kv[j] = a[j];
+        kv[j + 8] = b[j];
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) kv[j] = 0.f;
+    }
+  };
   const size_t base = (size_t)ci * H + h;
   const float* S0g = ws.S0 + base * D * D;
   const float* dUg = ws.dU + base * C * D;
@@ -1075,7 +1099,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float part = 0.f;
       if (c0 < D) {
         float kv[16], a[16], b[16];
-        staged16(sk, i, c0, kv);
+        k16(i, c0, kv);
         ld16g(pdk + i * D + c0, a);
         ld16g(pdG + i * D + c0, b);
 #pragma unroll
@@ -1167,7 +1191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (myrow < 0) continue;
       const int r = myrow;
       float kv[16], dkv[16], pg[16];
-      staged16(sk, r, c0, kv);
+      k16(r, c0, kv);
       ld16g(pdk + r * D + c0, dkv);
       ld16g(pdG + r * D + c0, pg);
 #pragma unroll

@@ -6,6 +6,7 @@
 #include <mutex>
 #include <new>
 #include <string>
+#include <type_traits>
 #include <vector>
 
 #include "../../include/tpc.h"
@@ -16,55 +17,27 @@
 #include "logprob_kernels.cuh"
 #include "attn_tc.cuh"
 #include <cudaTypedefs.h>
+#include "abi_internal.h"
 #include "plan.h"
 #include "rowmap_kernels.cuh"
 
-struct tpc_plan {
-  tpc::Plan p;
-};
-
-namespace {
+namespace tpc_abi {
 
 thread_local std::string g_err;
+Profiler g_prof;
 
 int fail(int code, const std::string& msg) {
   g_err = msg;
   return code;
 }
 
-#define TPC_CUDA(call)                                                                  \
-  do {                                                                                  \
-    cudaError_t e_ = (call);                                                            \
-    if (e_ != cudaSuccess) return fail(TPC_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
-  } while (0)
+}  // namespace tpc_abi
 
-size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+namespace {
 
-// Optional per-kernel timing: CUDA events around every launch (on the launching stream).
-struct Profiler {
-  bool on = false;
-  long long launches = 0;
-  struct Rec { const char* name; cudaEvent_t a, b; };
-  std::vector<Rec> recs;
-};
-Profiler g_prof;
-
-#define TPC_LAUNCH(NAME, STREAM, ...)                                     \
-  do {                                                                    \
-    cudaEvent_t a_ = nullptr, b_ = nullptr;                               \
-    if (g_prof.on) {                                                      \
-      TPC_CUDA(cudaEventCreate(&a_));                                     \
-      TPC_CUDA(cudaEventCreate(&b_));                                     \
-      TPC_CUDA(cudaEventRecord(a_, STREAM));                              \
-    }                                                                     \
-    __VA_ARGS__;                                                          \
-    TPC_CUDA(cudaGetLastError());                                         \
-    ++g_prof.launches;                                                    \
-    if (g_prof.on) {                                                      \
-      TPC_CUDA(cudaEventRecord(b_, STREAM));                              \
-      g_prof.recs.push_back({NAME, a_, b_});                              \
-    }                                                                     \
-  } while (0)
+using tpc_abi::a256;
+using tpc_abi::fail;
+using tpc_abi::g_prof;
 
 // workspace layout (bytes) for a plan + shape
 struct WsLayout {
@@ -155,7 +128,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
   const Tin* g = static_cast<const Tin*>(io->g);
   const Tin* b = static_cast<const Tin*>(io->beta);
   // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
-  constexpr bool kTensorCores = (C == kTcC && D == kTcD && std::is_same<Tin, __nv_bfloat16>::value);
+  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
   if constexpr (kTensorCores) {
     TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmem::total));
     TPC_LAUNCH("kda_fwd_prep_tc", st,
@@ -209,7 +182,7 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   const Tin* b = static_cast<const Tin*>(io->beta);
   const Tin* dO = static_cast<const Tin*>(io->d_o);
   // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
-  constexpr bool kTensorCores = (C == kTcC && D == kTcD && std::is_same<Tin, __nv_bfloat16>::value);
+  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
   if constexpr (kTensorCores) {
     TPC_CUDA(set_smem(kda_bwd_prep_tc<Tin>, BprepTcSmem::total));
     TPC_LAUNCH("kda_bwd_prep_tc", st,
@@ -234,12 +207,12 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   }
   if constexpr (kTensorCores) {
     TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
-    TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmem::total));
+    TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmemT<Tin>::total));
     TPC_LAUNCH("kda_bwd_dq_tc", st,
                (kda_bwd_dq_tc<Tin, Tout><<<dim3(nc, H), kThreads, BdqTcSmem::total, st>>>(
                    p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w)));
     TPC_LAUNCH("kda_bwd_dkv_tc", st,
-               (kda_bwd_dkv_tc<Tin, Tout><<<dim3(nc, H), kThreads, BdkvTcSmem::total, st>>>(
+               (kda_bwd_dkv_tc<Tin, Tout><<<dim3(nc, H), kThreads, BdkvTcSmemT<Tin>::total, st>>>(
                    p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg, io->dbeta,
                    w)));
   } else {
@@ -375,7 +348,7 @@ bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, u
 
 extern "C" {
 
-const char* tpc_last_error(void) { return g_err.c_str(); }
+const char* tpc_last_error(void) { return tpc_abi::g_err.c_str(); }
 const char* tpc_version(void) { return "tpc 0.1 (sm_100a)"; }
 
 int tpc_plan_create(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, tpc_plan** out) {
@@ -548,34 +521,50 @@ int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t st
   return TPC_OK;
 }
 
-int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
-                  int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype, float alpha, float beta, int32_t* status,
-                  tpc_stream_t stream) {
+int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B_lo, void* C, int64_t M, int64_t N,
+                   int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype,
+                   float alpha, float beta, int32_t* status, tpc_stream_t stream) {
   if (!A || !B || !C) return fail(TPC_ERR_NULL, "gemm: A, B and C are required");
   if (M < 1 || N < 1 || K < 1 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30))
     return fail(TPC_ERR_BAD_SHAPE, "gemm: sizes must be in [1, 2^30]");
-  if ((lda % 8) || (ldb % 8) || (reinterpret_cast<uintptr_t>(A) % 16) || (reinterpret_cast<uintptr_t>(B) % 16))
+  auto misaligned = [](const void* p) { return p && (reinterpret_cast<uintptr_t>(p) % 16) != 0; };
+  if ((lda % 8) || (ldb % 8) || misaligned(A) || misaligned(B) || misaligned(A_lo) || misaligned(B_lo))
     return fail(TPC_ERR_BAD_SHAPE, "gemm: A and B need 16-byte aligned bases and leading dimensions multiple of 8");
   if (c_dtype != TPC_F32 && c_dtype != TPC_BF16) return fail(TPC_ERR_UNSUPPORTED, "gemm: C is fp32 or bf16");
   if (c_dtype == TPC_BF16 && beta != 0.f) return fail(TPC_ERR_UNSUPPORTED, "gemm: beta needs an fp32 C");
   if (a_mn ? (lda < M) : (lda < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: lda too small");
   if (b_mn ? (ldb < N) : (ldb < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldb too small");
   if (ldc < N) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldc too small");
-  CUtensorMap ta, tb;
-  const bool ok_a = a_mn ? tensor_map(&ta, A, M, K, lda, tpc::kGemmBK) : tensor_map(&ta, A, K, M, lda, tpc::kGemmBM);
-  const bool ok_b = b_mn ? tensor_map(&tb, B, N, K, ldb, tpc::kGemmBK) : tensor_map(&tb, B, K, N, ldb, tpc::kGemmBN);
-  if (!ok_a || !ok_b) return fail(TPC_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
-  tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status};
+  if (B_lo && !A_lo) return fail(TPC_ERR_UNSUPPORTED, "gemm: B_lo needs A_lo (three-product form)");
+  auto encode = [&](CUtensorMap* m, const void* X, bool mn_major, int64_t mn, int64_t ld, int box) {
+    return mn_major ? tensor_map(m, X, mn, K, ld, tpc::kGemmBK) : tensor_map(m, X, K, mn, ld, box);
+  };
+  CUtensorMap ta, tb, talo, tblo;
+  bool ok = encode(&ta, A, a_mn, M, lda, tpc::kGemmBM) && encode(&tb, B, b_mn, N, ldb, tpc::kGemmBN);
+  ok = ok && encode(&talo, A_lo ? A_lo : A, a_mn, M, lda, tpc::kGemmBM);
+  ok = ok && encode(&tblo, B_lo ? B_lo : B, b_mn, N, ldb, tpc::kGemmBN);
+  if (!ok) return fail(TPC_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
+  const int passes = B_lo ? 3 : (A_lo ? 2 : 1);
+  tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status, passes};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid((unsigned)((N + tpc::kGemmBN - 1) / tpc::kGemmBN), (unsigned)((M + tpc::kGemmBM - 1) / tpc::kGemmBM));
   if (c_dtype == TPC_BF16) {
     TPC_CUDA(set_smem(tpc::gemm_bf16_tc<1>, tpc::GemmSmem::total));
-    TPC_LAUNCH("gemm_bf16_tc", st, (tpc::gemm_bf16_tc<1><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, g)));
+    TPC_LAUNCH("gemm_bf16_tc", st,
+               (tpc::gemm_bf16_tc<1><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
   } else {
     TPC_CUDA(set_smem(tpc::gemm_bf16_tc<0>, tpc::GemmSmem::total));
-    TPC_LAUNCH("gemm_bf16_tc", st, (tpc::gemm_bf16_tc<0><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, g)));
+    TPC_LAUNCH("gemm_bf16_tc", st,
+               (tpc::gemm_bf16_tc<0><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
   }
   return TPC_OK;
+}
+
+int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                  int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype, float alpha, float beta, int32_t* status,
+                  tpc_stream_t stream) {
+  return tpc_gemm_split(A, nullptr, B, nullptr, C, M, N, K, lda, ldb, ldc, a_mn, b_mn, c_dtype, alpha, beta, status,
+                        stream);
 }
 
 size_t tpc_logprob_scratch_bytes(int64_t V, int32_t chunk_rows) {
@@ -659,52 +648,64 @@ int attn_check(const tpc_plan* plan, const tpc_attn_shape* s) {
 }  // namespace
 
 int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const void* q, const void* k, const void* v,
-                          void* o, float* lse, int32_t* status, tpc_stream_t stream) {
+                          const tpc_attn_lo* lo, void* o, float* lse, int32_t* status, tpc_stream_t stream) {
   if (int rc = attn_check(plan, s)) return rc;
   if (!q || !k || !v || !o || !lse) return fail(TPC_ERR_NULL, "attention forward: NULL tensor");
+  const tpc_attn_lo L = lo ? *lo : tpc_attn_lo{};
+  const bool split = L.q || L.k || L.v;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const tpc::Plan& p = plan->p;
   const dim3 grid((unsigned)p.attn_qtiles.size(), (unsigned)s->H);
   using bf = __nv_bfloat16;
-  if (s->io_dtype == TPC_BF16) {
-    TPC_CUDA(set_smem(tpc::attn_fwd_tc<bf>, tpc::AttnFwdSmem::total));
+  auto go = [&](auto tout, auto split) -> int {
+    using T = decltype(tout);
+    constexpr bool SP = decltype(split)::value;
+    constexpr size_t smem = tpc::AttnFwdSmem<SP>::total;
+    TPC_CUDA(set_smem(tpc::attn_fwd_tc<T, SP>, smem));
     TPC_LAUNCH("attn_fwd_tc", st,
-               (tpc::attn_fwd_tc<bf><<<grid, tpc::kAttnThreads, tpc::AttnFwdSmem::total, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, (bf*)o, lse, status)));
-  } else {
-    TPC_CUDA(set_smem(tpc::attn_fwd_tc<float>, tpc::AttnFwdSmem::total));
-    TPC_LAUNCH("attn_fwd_tc", st,
-               (tpc::attn_fwd_tc<float><<<grid, tpc::kAttnThreads, tpc::AttnFwdSmem::total, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, (float*)o, lse, status)));
-  }
-  return TPC_OK;
+               (tpc::attn_fwd_tc<T, SP><<<grid, tpc::kAttnThreads, smem, st>>>(
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
+                   (const bf*)L.v, (T*)o, lse, status)));
+    return TPC_OK;
+  };
+  using Y = std::true_type;
+  using N = std::false_type;
+  if (s->io_dtype == TPC_BF16) return split ? go(bf{}, Y{}) : go(bf{}, N{});
+  return split ? go(float{}, Y{}) : go(float{}, N{});
 }
 
 int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const void* q, const void* k,
-                           const void* v, const void* o, const float* lse, const void* d_o, void* dq, void* dk,
-                           void* dv, float* delta, int32_t* status, tpc_stream_t stream) {
+                           const void* v, const tpc_attn_lo* lo, const void* o, const float* lse, const void* d_o,
+                           void* dq, void* dk, void* dv, float* delta, int32_t* status, tpc_stream_t stream) {
   if (int rc = attn_check(plan, s)) return rc;
   if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv || !delta)
     return fail(TPC_ERR_NULL, "attention backward: NULL tensor");
+  const tpc_attn_lo L = lo ? *lo : tpc_attn_lo{};
+  const bool split = L.q || L.k || L.v || L.d_o;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const tpc::Plan& p = plan->p;
   using bf = __nv_bfloat16;
   const dim3 gq((unsigned)p.attn_qtiles.size(), (unsigned)s->H), gk((unsigned)p.attn_ktiles.size(), (unsigned)s->H);
-  auto go = [&](auto tio) -> int {
+  auto go = [&](auto tio, auto split) -> int {
     using T = decltype(tio);
-    TPC_CUDA(set_smem(tpc::attn_bwd_dq_tc<T>, tpc::AttnDqSmem::total));
-    TPC_CUDA(set_smem(tpc::attn_bwd_dkv_tc<T>, tpc::AttnDkvSmem::total));
+    constexpr bool SP = decltype(split)::value;
+    constexpr size_t sq = tpc::AttnDqSmem<SP>::total, sk = tpc::AttnDkvSmem<SP>::total;
+    TPC_CUDA(set_smem(tpc::attn_bwd_dq_tc<T, SP>, sq));
+    TPC_CUDA(set_smem(tpc::attn_bwd_dkv_tc<T, SP>, sk));
     TPC_LAUNCH("attn_bwd_dq_tc", st,
-               (tpc::attn_bwd_dq_tc<T><<<gq, tpc::kAttnThreads, tpc::AttnDqSmem::total, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, (const T*)o, lse, (const bf*)d_o,
-                   (T*)dq, delta, status)));
+               (tpc::attn_bwd_dq_tc<T, SP><<<gq, tpc::kAttnThreads, sq, st>>>(
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
+                   (const bf*)L.v, (const T*)o, lse, (const bf*)d_o, (const bf*)L.d_o, (T*)dq, delta, status)));
     TPC_LAUNCH("attn_bwd_dkv_tc", st,
-               (tpc::attn_bwd_dkv_tc<T><<<gk, tpc::kAttnThreads, tpc::AttnDkvSmem::total, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)k, (const bf*)v, lse, (const bf*)d_o, delta, (T*)dk,
-                   (T*)dv, status)));
+               (tpc::attn_bwd_dkv_tc<T, SP><<<gk, tpc::kAttnThreads, sk, st>>>(
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
+                   (const bf*)L.v, lse, (const bf*)d_o, (const bf*)L.d_o, delta, (T*)dk, (T*)dv, status)));
     return TPC_OK;
   };
-  return s->io_dtype == TPC_BF16 ? go(bf{}) : go(float{});
+  using Y = std::true_type;
+  using N = std::false_type;
+  if (s->io_dtype == TPC_BF16) return split ? go(bf{}, Y{}) : go(bf{}, N{});
+  return split ? go(float{}, Y{}) : go(float{}, N{});
 }
 
 int tpc_rope_positions(const tpc_plan* plan, int32_t* pos, tpc_stream_t stream) {
