@@ -329,6 +329,102 @@ def measure_group(args, world, rank, tpc, torch, peaks):
             "precision": "bf16 weights; fp32 activations and gradients, tensor-core products from bf16 hi/lo pairs"}
 
 
+# ------------------------------------------------------------------------------------ wide tree + log-probs
+def measure_wide(args, world, rank, tpc, torch, peaks):
+    """The wide tree (512 trajectories on a 32,768-token prefix, two fork levels of 8): one KDA layer
+    with H = 32 run as four independent groups of 8 heads (the heads of a KDA layer do not interact;
+    one group's workspace fits the GPU, all 32 heads' would not), then per-position log-probability
+    recovery with hidden 2048 and vocabulary 65,536, forward and backward."""
+    import synth.gpu as sgpu
+    w = synth.workload("wide")
+    t = w.tree
+    seed = w.seed + 1000 * rank
+    plan = tpc.Plan(t.parent, t.length, 64).upload()
+    info = plan.info
+    N, NE, d, HG = info["n_unique"], info["n_expanded"], w.dk, 8
+    groups = w.H // HG
+    st = t.node_start()
+    src_rows = torch.tensor(plan.compact_source_rows(st, t.length), dtype=torch.int32, device="cuda")
+    bf = torch.bfloat16
+    ins = []
+    for gi in range(groups):
+        sg = seed + 17 * (gi + 1)
+        x = dict(zip(("q", "k", "v", "g", "beta"), sgpu.kda_inputs(sg, src_rows, HG, d, d, "bf16")))
+        x["d_o"] = sgpu.normal_rows(sg, synth.STREAM["d_o"], src_rows, HG * d, "bf16").view(N, HG, d)
+        x["d_final"] = sgpu.normal_rows(sg, synth.STREAM["d_final"], None, HG * d * d, "f32",
+                                        shape=(info["n_leaves"],)).view(info["n_leaves"], HG, d, d)
+        ins.append(x)
+    shape = tpc.kda_shape(HG, d, tpc.TPC_BF16, tpc.TPC_BF16)
+    wsb = tpc.alloc_workspace(plan, shape)
+    outs = [dict(o=torch.empty(N, HG, d, dtype=bf, device="cuda"),
+                 final=torch.empty(info["n_leaves"], HG, d, d, dtype=torch.float32, device="cuda"))
+            for _ in range(groups)]
+    grads = dict(dq=torch.empty(N, HG, d, dtype=bf, device="cuda"), dk=torch.empty(N, HG, d, dtype=bf, device="cuda"),
+                 dv=torch.empty(N, HG, d, dtype=bf, device="cuda"),
+                 dg=torch.empty(N, HG, d, dtype=torch.float32, device="cuda"),
+                 dbeta=torch.empty(N, HG, dtype=torch.float32, device="cuda"), d_init=None)
+    V, Dh, CR = 65536, 2048, 16384
+    hid = sgpu.normal_rows(seed, synth.STREAM["h"], src_rows, Dh, "bf16")
+    Wv = sgpu.normal_rows(seed, synth.STREAM["w_vocab"], None, Dh, "bf16", 0.02, shape=(V,))
+    targets = torch.randint(0, V, (NE,), dtype=torch.int32, device="cuda",
+                            generator=torch.Generator(device="cuda").manual_seed(seed))
+    dlogp = sgpu.normal_rows(seed, synth.STREAM["d_logp"], None, 1, "f32", shape=(NE,)).view(NE)
+    scratch = tpc.logprob_scratch(V, CR)
+    stream = torch.cuda.current_stream()
+
+    def kda_part():
+        for gi in range(groups):
+            x, o = ins[gi], outs[gi]
+            tpc.tpc_kda_forward(plan, x["q"], x["k"], x["v"], x["g"], x["beta"], ws=wsb, o=o["o"],
+                                final_state=o["final"], out_dtype=bf)
+            tpc.tpc_kda_backward(plan, wsb, x["q"], x["k"], x["v"], x["g"], x["beta"], x["d_o"], x["d_final"],
+                                 out_dtype=bf, grads=grads)
+
+    def logprob_part():
+        logp, lse = tpc.tpc_logprob_forward(plan, hid, Wv, targets, chunk_rows=CR, scratch=scratch)
+        tpc.tpc_logprob_backward(plan, hid, Wv, targets, dlogp, lse, chunk_rows=CR, scratch=scratch)
+
+    def timed(fn, k):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(e0.elapsed_time(e1), world) / k
+
+    for _ in range(args.warmup):
+        kda_part()
+        logprob_part()
+    torch.cuda.synchronize()
+    K = max(1, args.wide_steps)
+    kda_ms = timed(kda_part, K)
+    lp_ms = timed(logprob_part, K)
+    tpc.tpc_profile_enable(True)
+    logprob_part()
+    torch.cuda.synchronize()
+    prof = tpc.tpc_profile_read()
+    tpc.tpc_profile_enable(False)
+    gemm_ms = prof.get("gemm_bf16_tc", (0, 0.0))[1]
+    lp_flops = 3 * 2.0 * Dh * V * N  # logits, dh, dW (the backward's recomputed logits not counted)
+    kda_flops = 3.0 * w.H * (10 * 64 * d + 6 * d * d) * info["n_seq_tokens"]
+    step_ms = kda_ms + lp_ms
+    tflops = (lp_flops + kda_flops) / (step_ms / 1e3) / 1e12
+    peak = peaks["sustained"] or peaks["bf16_tflops"]
+    return {"workload": w.name + " + log-prob recovery (Dh 2048, V 65536)", "n_unique": N, "n_expanded": NE,
+            "heads": w.H, "head_groups": groups, "ms_per_step": step_ms, "kda_ms": kda_ms, "logprob_ms": lp_ms,
+            "unique_tokens_per_s": world * N / (step_ms / 1e3), "expanded_tokens_per_s": world * NE / (step_ms / 1e3),
+            "logprob_kernels": {k: {"launches": n, "ms": v} for k, (n, v) in prof.items()},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                         "algorithmic_tflop_per_step": (lp_flops + kda_flops) / 1e12,
+                         "logprob_gemm_achieved_tflops": (lp_flops + 2.0 * Dh * V * N) / 1e12 / (gemm_ms / 1e3)
+                         if gemm_ms else None,
+                         "peak_source": "bf16 sustained, " + peaks["source"]}}
+
+
 # ------------------------------------------------------------------------------------ GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -343,6 +439,8 @@ def main():
     ap.add_argument("--no-expanded", action="store_true")
     ap.add_argument("--no-group", action="store_true", help="skip the hybrid layer group (3 KDA + 1 MLA) measurement")
     ap.add_argument("--group-steps", type=int, default=3)
+    ap.add_argument("--no-wide", action="store_true", help="skip the wide tree with log-prob recovery")
+    ap.add_argument("--wide-steps", type=int, default=2)
     ap.add_argument("--workload", default=WORKLOAD, help="single_fork (default), agentic, agentic_small")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "tpc" else args.warmup
@@ -524,6 +622,16 @@ def main():
         del wsb, outs, grads, dev
         torch.cuda.empty_cache()
         group = measure_group(args, world, rank, tpc, torch, peaks)
+        torch.cuda.empty_cache()
+
+    # ---- wide tree: KDA (H = 32) and log-probability recovery
+    wide = None
+    if not args.no_wide:
+        if args.no_group:
+            del wsb, outs, grads, dev
+        torch.cuda.empty_cache()
+        wide = measure_wide(args, world, rank, tpc, torch, peaks)
+        torch.cuda.empty_cache()
 
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -542,7 +650,7 @@ def main():
                            "l2": "inputs+workspace > 1 GB per step, larger than L2"},
                 "value_expanded": value_exp, "roofline": roofline, "step_roofline": step_roof,
                 "kernels": kern, "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
-                "expanded_path": expanded, "hybrid_group": group}
+                "expanded_path": expanded, "hybrid_group": group, "wide_logprob": wide}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

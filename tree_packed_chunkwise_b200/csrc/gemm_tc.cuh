@@ -8,9 +8,10 @@
 // A_lo B_lo term is below 2^-16 of the product.  The K loop simply runs once per product.
 //
 // One CTA per 128 x 256 output tile, K in steps of 64 through a 4-stage shared-memory pipeline:
-// a producer thread issues TMA loads (one 16-byte-wide box per 8-element core-matrix column of the
-// no-swizzle canonical layout), an MMA thread issues tcgen05.mma and frees stages by tcgen05.commit,
-// all 128 threads run the epilogue (thread = row).  All waits are bounded.
+// a producer thread issues TMA loads into the 128-byte-swizzled canonical layout (K-major operand:
+// one box of 64 K x tile rows, each row one 128-byte line; MN-major operand: boxes of 64 M/N x 64 K,
+// each K row one 128-byte line), an MMA thread issues tcgen05.mma and frees stages by
+// tcgen05.commit, all 128 threads run the epilogue (thread = row).  All waits are bounded.
 #pragma once
 #include <cuda.h>
 
@@ -20,11 +21,25 @@
 namespace tpc {
 
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4, kGemmThreads = 128;
+// one MN-major 128-byte-swizzle block: 64 K rows of one 128-byte line
+constexpr uint32_t kSw128Atom = kGemmBK * 128;
+
+// Shared-memory descriptor of the 16-wide K step ks of a 128-byte-swizzled operand tile (descriptor
+// version 1, layout type 2 = 128-byte swizzle).  Groups of 8 rows of 128-byte lines are 1024 bytes
+// apart (SBO).  K-major: a line holds 64 K of one M/N row, the K step moves 32 bytes along it.
+// MN-major: a line holds 64 M/N of one K row, the K step moves 16 lines (2048 bytes), and the
+// 64-wide M/N blocks are kSw128Atom apart (LBO).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t base, bool mn, int ks) {
+  const uint32_t addr = mn ? base + (uint32_t)ks * 2048u : base + (uint32_t)ks * 32u;
+  const uint32_t lbo = mn ? kSw128Atom : 16u;
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((1024u >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
 
 struct GemmSmem {
   static constexpr size_t Ab = size_t(kGemmBM) * kGemmBK * 2, Bb = size_t(kGemmBN) * kGemmBK * 2;
   static constexpr size_t stage = Ab + Bb;
-  static constexpr size_t total = kGemmStages * stage;
+  static constexpr size_t total = kGemmStages * stage + 1024;  // + slack to align the stages to 1024 bytes
 };
 
 struct GemmArgs {
@@ -43,7 +58,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                  const __grid_constant__ CUtensorMap tma_alo, const __grid_constant__ CUtensorMap tma_blo, GemmArgs g) {
   using namespace tc;
-  extern __shared__ __align__(1024) uint8_t gsm[];
+  extern __shared__ __align__(1024) uint8_t gsm_raw[];
+  // the swizzle pattern is a function of the shared address: stages start on 1024-byte boundaries
+  uint8_t* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
   __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], accb;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -79,14 +96,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_arrive_expect_tx(&full[s], (uint32_t)GemmSmem::stage);
       const int k0 = kt * kGemmBK;
       if (!g.a_mn) {
-        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sa + j * (kGemmBM / 8) * 128, ma, k0 + 8 * j, m0, &full[s]);
+        tma_load_2d(sa, ma, k0, m0, &full[s]);
       } else {
-        for (int j = 0; j < kGemmBM / 8; ++j) tma_load_2d(sa + j * (kGemmBK / 8) * 128, ma, m0 + 8 * j, k0, &full[s]);
+        for (int j = 0; j < kGemmBM / 64; ++j) tma_load_2d(sa + j * kSw128Atom, ma, m0 + 64 * j, k0, &full[s]);
       }
       if (!g.b_mn) {
-        for (int j = 0; j < kGemmBK / 8; ++j) tma_load_2d(sb + j * (kGemmBN / 8) * 128, mb, k0 + 8 * j, n0, &full[s]);
+        tma_load_2d(sb, mb, k0, n0, &full[s]);
       } else {
-        for (int j = 0; j < kGemmBN / 8; ++j) tma_load_2d(sb + j * (kGemmBK / 8) * 128, mb, n0 + 8 * j, k0, &full[s]);
+        for (int j = 0; j < kGemmBN / 64; ++j) tma_load_2d(sb + j * kSw128Atom, mb, n0 + 64 * j, k0, &full[s]);
       }
     }
   } else if (w == 1 && lane == 0) {
@@ -100,10 +117,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       fence_after_sync();
-      const uint8_t* sa = gsm + s * GemmSmem::stage;
-      const Op a{smem_u32(sa), g.a_mn ? kGemmBK : kGemmBM, g.a_mn != 0};
-      const Op b{smem_u32(sa + GemmSmem::Ab), g.b_mn ? kGemmBK : kGemmBN, g.b_mn != 0};
-      mma_chain(tb, a, b, kGemmBK, id, it > 0);
+      const uint32_t sa = smem_u32(gsm + s * GemmSmem::stage), sb = sa + (uint32_t)GemmSmem::Ab;
+#pragma unroll
+      for (int ks = 0; ks < kGemmBK / 16; ++ks)
+        mma_bf16(tb, sw128_desc(sa, g.a_mn != 0, ks), sw128_desc(sb, g.b_mn != 0, ks), id, (it > 0 || ks) ? 1u : 0u);
       commit(&empty[s]);
     }
     commit(&accb);

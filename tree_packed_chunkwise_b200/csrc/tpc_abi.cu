@@ -325,8 +325,10 @@ int forward_static_impl(const tpc::Plan& p, const tpc::DevTables& dt, tpc::KdaWs
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
+// 2-D bf16 tensor map over [rows][cols] (leading dimension ld_elems): boxes of box_cols x box_rows
+// elements, 128-byte swizzle when box_cols is 64 (one 128-byte row per box row), none otherwise.
 bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems,
-                uint32_t box_rows) {
+                uint32_t box_rows, uint32_t box_cols = 8) {
   std::call_once(g_encode_once, [] {
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void**>(&g_encode), cudaEnableDefault,
@@ -337,10 +339,11 @@ bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, u
   if (!g_encode) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld_elems * 2};
-  cuuint32_t box[2] = {8, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -536,8 +539,10 @@ int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B
   if (b_mn ? (ldb < N) : (ldb < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldb too small");
   if (ldc < N) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldc too small");
   if (B_lo && !A_lo) return fail(TPC_ERR_UNSUPPORTED, "gemm: B_lo needs A_lo (three-product form)");
+  // 128-byte-swizzled boxes 64 elements wide: K-major [mn][K] boxes of 64 (K) x tile rows,
+  // MN-major [K][mn] boxes of 64 (mn) x 64 (K)
   auto encode = [&](CUtensorMap* m, const void* X, bool mn_major, int64_t mn, int64_t ld, int box) {
-    return mn_major ? tensor_map(m, X, mn, K, ld, tpc::kGemmBK) : tensor_map(m, X, K, mn, ld, box);
+    return mn_major ? tensor_map(m, X, mn, K, ld, tpc::kGemmBK, 64) : tensor_map(m, X, K, mn, ld, box, 64);
   };
   CUtensorMap ta, tb, talo, tblo;
   bool ok = encode(&ta, A, a_mn, M, lda, tpc::kGemmBM) && encode(&tb, B, b_mn, N, ldb, tpc::kGemmBN);
