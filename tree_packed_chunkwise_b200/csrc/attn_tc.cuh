@@ -57,6 +57,51 @@ __device__ __forceinline__ void st_out16(T* p, const float* v) {
 }  // namespace tck
 
 // ------------------------------------------------------------------------------------------ forward
+// Key tiles of a query tile, one at a time in the fixed order of for_key_tiles (for look-ahead).
+template <int KT>
+struct KeyTileIter {
+  const RowRange* ranges;
+  int r, r1, k, own_start, own_end;
+  __device__ void init(const DevTables& t, const AttnTile& qt) {
+    const AttnNode nd = t.attn_nodes[qt.node];
+    ranges = t.attn_ranges;
+    r = nd.range_begin;
+    r1 = t.attn_nodes[qt.node + 1].range_begin;
+    own_start = nd.row_offset;
+    own_end = qt.row + qt.n;
+    k = r < r1 ? ranges[r].start : own_start;
+  }
+  __device__ bool next(int& k0, int& nk, bool& own) {
+    while (r < r1) {
+      const RowRange rr = ranges[r];
+      if (k < rr.end) {
+        k0 = k; nk = min(KT, rr.end - k); own = false; k += KT;
+        return true;
+      }
+      ++r;
+      k = r < r1 ? ranges[r].start : own_start;
+    }
+    if (k < own_end) {
+      k0 = k; nk = min(KT, own_end - k); own = true; k += KT;
+      return true;
+    }
+    return false;
+  }
+};
+
+// Asynchronous load of an A x B bf16 tile (rows from rowp(a), nullptr = zeros) into the
+// core-matrix layout; `any` is a valid global address used for the zero-filled rows.
+template <int A, int B, int NT, class RP>
+__device__ __forceinline__ void tile_async(uint8_t* dst, RP rowp, const void* any) {
+  constexpr int NCH = A * (B / 8);
+#pragma unroll 4
+  for (int e = threadIdx.x; e < NCH; e += NT) {
+    const int a = e % A, b0 = (e / A) * 8;
+    const __nv_bfloat16* p = rowp(a);
+    tc::cp_async16(dst + tc::cm_off(a, b0, A), p ? (const void*)(p + b0) : any, p ? 16u : 0u);
+  }
+}
+
 template <bool SPLIT>
 struct AttnFwdSmem {
   static constexpr size_t Qb = size_t(128) * kAttnQK * 2, Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
@@ -67,6 +112,10 @@ struct AttnFwdSmem {
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
+// Per query tile: O accumulates in TMEM across the key tiles (P V products with accumulate), the
+// online softmax keeps a per-row reference maximum that is raised (and O, l rescaled) only when a
+// tile's maximum exceeds it by more than 8, so every p = exp(s - m) stays below e^8.  The next key
+// tile's K and V are fetched with cp.async while the current tile's softmax and P V run.
 template <typename Tout, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
@@ -78,6 +127,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using S = AttnFwdSmem<SPLIT>;
   using bf = __nv_bfloat16;
   constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
+  constexpr float kRaise = 8.f;
   const AttnTile qt = t.attn_qtiles[blockIdx.x];
   const int h = blockIdx.y, tid = threadIdx.x;
   extern __shared__ __align__(1024) uint8_t asmem[];
@@ -90,91 +140,118 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc::mbar_init(&bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  auto ident = [](int, int, float x) { return x; };
-  build_tile_ld<128, DQ, false, bf, NT>(
-      sQ, nullptr, [&](int a) -> const bf* { return a < qt.n ? q + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; },
-      ident);
-  if constexpr (SPLIT)
-    build_tile_ld<128, DQ, false, bf, NT>(
-        sQl, nullptr,
-        [&](int a) -> const bf* { return a < qt.n && q_lo ? q_lo + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; },
-        ident);
+  auto qrows = [&](const bf* base) {
+    return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; };
+  };
+  auto load_kv = [&](bool is_k, int k0, int nk) {
+    if (is_k) {
+      tile_async<64, DQ, NT>(sK, [=](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, k);
+      if constexpr (SPLIT)
+        tile_async<64, DQ, NT>(
+            sKl, [=](int a) -> const bf* { return a < nk && k_lo ? k_lo + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, k);
+    } else {
+      tile_async<64, DV, NT>(sV, [=](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, v);
+      if constexpr (SPLIT)
+        tile_async<64, DV, NT>(
+            sVl, [=](int a) -> const bf* { return a < nk && v_lo ? v_lo + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, v);
+    }
+  };
+  KeyTileIter<64> it;
+  it.init(t, qt);
+  int k0 = 0, nk = 0;
+  bool own = false;
+  bool have = it.next(k0, nk, own);
+  tile_async<128, DQ, NT>(sQ, qrows(q), q);
+  if constexpr (SPLIT) tile_async<128, DQ, NT>(sQl, qrows(q_lo), q);
+  if (have) load_kv(true, k0, nk);
+  tc::cp_async_commit();  // group: Q, K_0
+  if (have) load_kv(false, k0, nk);
+  tc::cp_async_commit();  // group: V_0
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   const uint32_t la = tb + ((uint32_t)(32 * (tid >> 5)) << 16);
   Sync sy{&bar, 0u, status};
   const int qrow = qt.row + tid;
-  float acc[DV];
-#pragma unroll
-  for (int j = 0; j < DV; ++j) acc[j] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  const bool ok = for_key_tiles(t, qt, [&](int k0, int nk, bool own) -> bool {
-    build_tile_ld<64, DQ, false, bf, NT>(
-        sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
-    build_tile_ld<64, DV, false, bf, NT>(
-        sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
-    if constexpr (SPLIT) {
-      build_tile_ld<64, DQ, false, bf, NT>(
-          sKl, nullptr,
-          [&](int a) -> const bf* { return a < nk && k_lo ? k_lo + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
-      build_tile_ld<64, DV, false, bf, NT>(
-          sVl, nullptr,
-          [&](int a) -> const bf* { return a < nk && v_lo ? v_lo + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
-    }
-    if (!run(sy, [&] {
-          mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
-               tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sKl), 64, false}, DQ,
-               tc::idesc_bf16(128, 64, false, false), false, !SPLIT, !SPLIT);
-        }))
-      return false;
+  float m_ref = -INFINITY, l = 0.f;
+  bool first = true, ok = true;
+  while (have) {
+    int k1 = 0, n1 = 0;
+    bool own1 = false;
+    const bool more = it.next(k1, n1, own1);
+    tc::cp_async_wait<1>();  // Q and this tile's K have arrived
+    ok = run(sy, [&] {
+      mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
+           tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sKl), 64, false}, DQ,
+           tc::idesc_bf16(128, 64, false, false), false, !SPLIT, !SPLIT);
+    });
+    if (!ok) break;
+    if (more) load_kv(true, k1, n1);  // K is free once S is in TMEM
+    tc::cp_async_commit();
     float s[64];
     tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
     tc::tmem_ld32(la + 32, *reinterpret_cast<float(*)[32]>(s + 32));
     float mx = -INFINITY;
 #pragma unroll
     for (int j = 0; j < 64; ++j) {
-      const bool valid = j < nk && (!own || k0 + j <= qrow);
+      const bool valid = tid < qt.n && j < nk && (!own || k0 + j <= qrow);
       s[j] = valid ? s[j] * scale : -INFINITY;
       mx = fmaxf(mx, s[j]);
     }
-    const float m_new = fmaxf(m, mx);
-    const float corr = (m == -INFINITY) ? 0.f : expf(m - m_new);
+    // raise the reference where a tile's maximum exceeds it by more than kRaise; O (accumulated so
+    // far) and l follow.  TMEM loads and stores are warp-collective: a warp rescales its 32 rows
+    // together when any of them raised (the others with factor 1).
+    const bool raise = mx > m_ref + kRaise;
+    const float corr = !raise ? 1.f : (m_ref == -INFINITY ? 0.f : expf(m_ref - mx));
+    if (raise) {
+      l *= corr;
+      m_ref = mx;
+    }
+    if (!first && __any_sync(0xffffffffu, raise)) {
+      for (int c = 0; c < DV; c += 16) {
+        float ov[16];
+        tc::tmem_ld16(la + 64 + c, ov);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ov[j] *= corr;
+        tc::tmem_st16(la + 64 + c, ov);
+      }
+    }
     float psum = 0.f;
 #pragma unroll
     for (int j = 0; j < 64; ++j) {
-      s[j] = (s[j] == -INFINITY) ? 0.f : expf(s[j] - m_new);
+      s[j] = s[j] == -INFINITY ? 0.f : expf(s[j] - m_ref);
       psum += s[j];
     }
-    l = l * corr + psum;
-    m = m_new;
+    l += psum;
 #pragma unroll
     for (int j = 0; j < 64; j += 16) put16<128, true>(sPh, sPl, tid, j, s + j);
-    if (!run(sy, [&] {
-          mma4(tb + 64, tc::Op{tc::smem_u32(sPh), 128, false}, tc::Op{tc::smem_u32(sPl), 128, false},
-               tc::Op{tc::smem_u32(sV), 64, true}, tc::Op{tc::smem_u32(sVl), 64, true}, 64,
-               tc::idesc_bf16(128, DV, false, true), false, false, !SPLIT);
-        }))
-      return false;
-#pragma unroll
-    for (int c = 0; c < DV; c += 32) {
-      float pv[32];
-      tc::tmem_ld32(la + 64 + c, pv);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) acc[c + j] = acc[c + j] * corr + pv[j];
-    }
-    tc::fence_before_sync();
-    __syncthreads();  // tiles are rewritten by the next key tile
-    return true;
-  });
-  if (ok && tid < qt.n) {
+    tc::cp_async_wait<1>();  // this tile's V has arrived
+    const bool acc_on = !first;
+    ok = run(sy, [&] {
+      mma4(tb + 64, tc::Op{tc::smem_u32(sPh), 128, false}, tc::Op{tc::smem_u32(sPl), 128, false},
+           tc::Op{tc::smem_u32(sV), 64, true}, tc::Op{tc::smem_u32(sVl), 64, true}, 64,
+           tc::idesc_bf16(128, DV, false, true), acc_on, false, !SPLIT);
+    });
+    if (!ok) break;
+    if (more) load_kv(false, k1, n1);  // V is free once P V is done
+    tc::cp_async_commit();
+    first = false;
+    k0 = k1; nk = n1; own = own1; have = more;
+  }
+  tc::cp_async_wait<0>();
+  if (ok) {
     const float inv = 1.f / l;
-#pragma unroll
-    for (int j = 0; j < DV; ++j) acc[j] *= inv;
     Tout* dst = o + ((size_t)qrow * H + h) * DV;
+    for (int c = 0; c < DV; c += 16) {
+      float ov[16];
+      tc::tmem_ld16(la + 64 + c, ov);  // warp-collective: every row takes part
+      if (tid < qt.n) {
 #pragma unroll
-    for (int c = 0; c < DV; c += 16) st_out16(dst + c, acc + c);
-    lse[(size_t)qrow * H + h] = m + logf(l);
+        for (int j = 0; j < 16; ++j) ov[j] *= inv;
+        st_out16(dst + c, ov);
+      }
+    }
+    if (tid < qt.n) lse[(size_t)qrow * H + h] = m_ref + logf(l);
   }
   tc::fence_before_sync();
   __syncthreads();

@@ -53,108 +53,169 @@ struct GemmArgs {
   int passes;         // 1: A B;  2: + A_lo B;  3: + A B_lo
 };
 
+// Persistent, warp-specialised: grid = min(tiles, SMs); each CTA walks tiles blockIdx.x,
+// blockIdx.x + gridDim.x, ... (N blocks fastest, so concurrent CTAs share A rows and all of B stays
+// in L2).  Warp 0 lane 0 issues TMA loads into a 4-stage ring; warp 1 lane 0 issues the MMAs into one
+// of two TMEM accumulators (256 columns each); warps 2-5 drain the other accumulator to global
+// memory (thread = row), so a tile's epilogue overlaps the next tile's main loop.  Every wait is
+// bounded; a timeout records TPC_ERR_TIMEOUT and every role stops.
+constexpr int kGemmThreadsP = 192;
+
 template <int C_BF16>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreadsP, 1)
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                  const __grid_constant__ CUtensorMap tma_alo, const __grid_constant__ CUtensorMap tma_blo, GemmArgs g) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t gsm_raw[];
   // the swizzle pattern is a function of the shared address: stages start on 1024-byte boundaries
   uint8_t* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
-  __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], accb;
+  __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], acc_full[2], acc_empty[2], done_bar;
   __shared__ uint32_t tslot;
+  __shared__ int abort_flag;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * kGemmBN;
   const int KT = (g.K + kGemmBK - 1) / kGemmBK;
   const int IT = KT * g.passes;  // pass p = it / KT uses (A, B), (A_lo, B), (A, B_lo)
-  if (w == 0) tmem_alloc(&tslot, 256);
+  const int n_tiles = (g.N + kGemmBN - 1) / kGemmBN, m_tiles = (g.M + kGemmBM - 1) / kGemmBM;
+  const int tiles = n_tiles * m_tiles;
+  if (w == 1) tmem_alloc(&tslot, 512);
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&accb, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
   fence_after_sync();
   const uint32_t tb = tslot;
-  bool ok = true;
-  if (w == 0 && lane == 0) {
-    // producer
-    for (int it = 0; it < IT && ok; ++it) {
-      const int s = it % kGemmStages, pass = it / KT, kt = it - pass * KT;
-      if (it >= kGemmStages && !mbar_wait(&empty[s], ((it / kGemmStages) - 1) & 1)) {
-        set_status(g.status, 8);
-        ok = false;
-        break;
-      }
-      const CUtensorMap* ma = pass == 1 ? &tma_alo : &tma_a;
-      const CUtensorMap* mb = pass == 2 ? &tma_blo : &tma_b;
-      uint8_t* sa = gsm + s * GemmSmem::stage;
-      uint8_t* sb = sa + GemmSmem::Ab;
-      mbar_arrive_expect_tx(&full[s], (uint32_t)GemmSmem::stage);
-      const int k0 = kt * kGemmBK;
-      if (!g.a_mn) {
-        tma_load_2d(sa, ma, k0, m0, &full[s]);
-      } else {
-        for (int j = 0; j < kGemmBM / 64; ++j) tma_load_2d(sa + j * kSw128Atom, ma, m0 + 64 * j, k0, &full[s]);
-      }
-      if (!g.b_mn) {
-        tma_load_2d(sb, mb, k0, n0, &full[s]);
-      } else {
-        for (int j = 0; j < kGemmBN / 64; ++j) tma_load_2d(sb + j * kSw128Atom, mb, n0 + 64 * j, k0, &full[s]);
-      }
-    }
-  } else if (w == 1 && lane == 0) {
-    // MMA issuer
-    const uint32_t id = idesc_bf16(kGemmBM, kGemmBN, g.a_mn != 0, g.b_mn != 0);
-    for (int it = 0; it < IT; ++it) {
-      const int s = it % kGemmStages;
-      if (!mbar_wait(&full[s], (it / kGemmStages) & 1)) {
-        set_status(g.status, 8);
-        ok = false;
-        break;
-      }
-      fence_after_sync();
-      const uint32_t sa = smem_u32(gsm + s * GemmSmem::stage), sb = sa + (uint32_t)GemmSmem::Ab;
-#pragma unroll
-      for (int ks = 0; ks < kGemmBK / 16; ++ks)
-        mma_bf16(tb, sw128_desc(sa, g.a_mn != 0, ks), sw128_desc(sb, g.b_mn != 0, ks), id, (it > 0 || ks) ? 1u : 0u);
-      commit(&empty[s]);
-    }
-    commit(&accb);
-  }
-  // epilogue: every thread waits for the accumulator (bounded)
-  const bool done = mbar_wait(&accb, 0, 4000000000ull);
-  const int failed = __syncthreads_or(done ? 0 : 1);
-  __syncwarp();
-  if (!failed) {
-    fence_after_sync();
-    const int m = m0 + 32 * w + lane;
-    const uint32_t la = tb + ((uint32_t)(32 * w) << 16);
-    for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
-      float v[16];
-      tmem_ld16(la + c0, v);
-      if (m >= g.M || n0 + c0 >= g.N) continue;
-      const int nn = min(16, g.N - (n0 + c0));
-      if (C_BF16) {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.C) + (size_t)m * g.ldc + n0 + c0;
-        for (int j = 0; j < nn; ++j) dst[j] = __float2bfloat16_rn(g.alpha * v[j]);
-      } else {
-        float* dst = static_cast<float*>(g.C) + (size_t)m * g.ldc + n0 + c0;
-        if (g.beta != 0.f)
-          for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j] + g.beta * dst[j];
-        else
-          for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j];
-      }
-    }
-  } else if (tid == 0) {
+  auto give_up = [&] {
     set_status(g.status, 8);
+    atomicExch(&abort_flag, 1);
+  };
+  auto aborted = [&] { return *((volatile int*)&abort_flag) != 0; };
+  if (w == 0) {
+    if (lane == 0) {  // producer
+      int it_all = 0;
+      for (int t = blockIdx.x; t < tiles && !aborted(); t += gridDim.x) {
+        const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * kGemmBN;
+        for (int it = 0; it < IT; ++it, ++it_all) {
+          const int s = it_all % kGemmStages, pass = it / KT, kt = it - pass * KT;
+          if (it_all >= kGemmStages && !mbar_wait(&empty[s], ((it_all / kGemmStages) - 1) & 1)) {
+            give_up();
+            break;
+          }
+          const CUtensorMap* ma = pass == 1 ? &tma_alo : &tma_a;
+          const CUtensorMap* mb = pass == 2 ? &tma_blo : &tma_b;
+          uint8_t* sa = gsm + s * GemmSmem::stage;
+          uint8_t* sb = sa + GemmSmem::Ab;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)GemmSmem::stage);
+          const int k0 = kt * kGemmBK;
+          if (!g.a_mn) {
+            tma_load_2d(sa, ma, k0, m0, &full[s]);
+          } else {
+            for (int j = 0; j < kGemmBM / 64; ++j) tma_load_2d(sa + j * kSw128Atom, ma, m0 + 64 * j, k0, &full[s]);
+          }
+          if (!g.b_mn) {
+            tma_load_2d(sb, mb, k0, n0, &full[s]);
+          } else {
+            for (int j = 0; j < kGemmBN / 64; ++j) tma_load_2d(sb + j * kSw128Atom, mb, n0 + 64 * j, k0, &full[s]);
+          }
+        }
+      }
+    }
+  } else if (w == 1) {
+    if (lane == 0) {  // MMA issuer
+      const uint32_t id = idesc_bf16(kGemmBM, kGemmBN, g.a_mn != 0, g.b_mn != 0);
+      int it_all = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok && !aborted(); t += gridDim.x, ++local) {
+        const int b = local & 1;
+        // the epilogue has drained this accumulator (its previous use was tile local - 2)
+        if (local >= 2 && !mbar_wait(&acc_empty[b], ((local >> 1) - 1) & 1, 4000000000ull)) {
+          give_up();
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        const uint32_t acc = tb + (uint32_t)(b * kGemmBN);
+        for (int it = 0; it < IT; ++it, ++it_all) {
+          const int s = it_all % kGemmStages;
+          if (!mbar_wait(&full[s], (it_all / kGemmStages) & 1)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          fence_after_sync();
+          const uint32_t sa = smem_u32(gsm + s * GemmSmem::stage), sb = sa + (uint32_t)GemmSmem::Ab;
+#pragma unroll
+          for (int ks = 0; ks < kGemmBK / 16; ++ks)
+            mma_bf16(acc, sw128_desc(sa, g.a_mn != 0, ks), sw128_desc(sb, g.b_mn != 0, ks), id,
+                     (it > 0 || ks) ? 1u : 0u);
+          commit(&empty[s]);
+        }
+        if (ok) commit(&acc_full[b]);
+      }
+      commit(&done_bar);  // arrives once every MMA issued above has completed
+      if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
+    }
+  } else {  // epilogue warps 2..5: TMEM lanes of sub-partition w % 4
+    const int sp = w & 3, row = 32 * sp + lane;
+    int local = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+      const int b = local & 1;
+      // decisions are warp-uniform: the TMEM loads below are warp-collective
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (local >> 1) & 1, 4000000000ull));
+      if (!got) {
+        if (lane == 0) give_up();
+        break;
+      }
+      if (__any_sync(0xffffffffu, aborted())) break;
+      fence_after_sync();
+      const int m = (t / n_tiles) * kGemmBM + row, n0 = (t % n_tiles) * kGemmBN;
+      const uint32_t la = tb + ((uint32_t)(32 * sp) << 16) + (uint32_t)(b * kGemmBN);
+      for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+        float v[16];
+        tmem_ld16(la + c0, v);
+        if (m >= g.M || n0 + c0 >= g.N) continue;
+        const int nn = min(16, g.N - (n0 + c0));
+        if (C_BF16) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.C) + (size_t)m * g.ldc + n0 + c0;
+          for (int j = 0; j < nn; ++j) dst[j] = __float2bfloat16_rn(g.alpha * v[j]);
+        } else {
+          float* dst = static_cast<float*>(g.C) + (size_t)m * g.ldc + n0 + c0;
+          if (nn == 16 && (g.ldc & 3) == 0) {
+            float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float4 x = make_float4(g.alpha * v[4 * j], g.alpha * v[4 * j + 1], g.alpha * v[4 * j + 2],
+                                     g.alpha * v[4 * j + 3]);
+              if (g.beta != 0.f) {
+                const float4 c = d4[j];
+                x.x += g.beta * c.x; x.y += g.beta * c.y; x.z += g.beta * c.z; x.w += g.beta * c.w;
+              }
+              d4[j] = x;
+            }
+          } else if (g.beta != 0.f) {
+            for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j] + g.beta * dst[j];
+          } else {
+            for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j];
+          }
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+    }
   }
   fence_before_sync();
   __syncthreads();
-  if (w == 0) tmem_dealloc(tb, 256);
+  if (w == 1) tmem_dealloc(tb, 512);
 }
 
 }  // namespace tpc

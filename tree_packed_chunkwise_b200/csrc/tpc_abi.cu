@@ -325,6 +325,15 @@ int forward_static_impl(const tpc::Plan& p, const tpc::DevTables& dt, tpc::KdaWs
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
+// multiprocessors of the current device (persistent grids)
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n < 1)
+    return 148;
+  return n;
+}
+
 // 2-D bf16 tensor map over [rows][cols] (leading dimension ld_elems): boxes of box_cols x box_rows
 // elements, 128-byte swizzle when box_cols is 64 (one 128-byte row per box row), none otherwise.
 bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems,
@@ -552,15 +561,17 @@ int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B
   const int passes = B_lo ? 3 : (A_lo ? 2 : 1);
   tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status, passes};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const dim3 grid((unsigned)((N + tpc::kGemmBN - 1) / tpc::kGemmBN), (unsigned)((M + tpc::kGemmBM - 1) / tpc::kGemmBM));
+  const int64_t tiles = ((N + tpc::kGemmBN - 1) / tpc::kGemmBN) * ((M + tpc::kGemmBM - 1) / tpc::kGemmBM);
+  if (tiles > (int64_t)1 << 31) return fail(TPC_ERR_BAD_SHAPE, "gemm: too many tiles");
+  const dim3 grid((unsigned)std::min<int64_t>(tiles, sm_count()));
   if (c_dtype == TPC_BF16) {
     TPC_CUDA(set_smem(tpc::gemm_bf16_tc<1>, tpc::GemmSmem::total));
     TPC_LAUNCH("gemm_bf16_tc", st,
-               (tpc::gemm_bf16_tc<1><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
+               (tpc::gemm_bf16_tc<1><<<grid, tpc::kGemmThreadsP, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
   } else {
     TPC_CUDA(set_smem(tpc::gemm_bf16_tc<0>, tpc::GemmSmem::total));
     TPC_LAUNCH("gemm_bf16_tc", st,
-               (tpc::gemm_bf16_tc<0><<<grid, tpc::kGemmThreads, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
+               (tpc::gemm_bf16_tc<0><<<grid, tpc::kGemmThreadsP, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
   }
   return TPC_OK;
 }
