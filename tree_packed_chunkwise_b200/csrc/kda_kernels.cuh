@@ -22,6 +22,7 @@ struct KdaWs {
   float *rdk, *rdv, *rdg, *rdb;                            // replay partials [R][H][D] / [R][H]
   float *tdk, *tdv, *tdg, *tdb;                            // own part of replay-target rows
   float *Mt, *Bc;  // tensor-core path: per-chunk state transition M (bf16 hi/lo operand tile) and B (fp32)
+  float *At, *Tm;  // tensor-core path: per-chunk gated key products Atilde and T = (I + diag(beta) Atilde)^{-1}
 };
 
 template <int C, int D>

@@ -445,17 +445,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
     ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
     if (ok) {
+      float* Ag = ws.At + ((size_t)ci * H + h) * C * C;  // kept for the backward
       acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
+        float a[16];
         for (int j = 0; j < 16; ++j) {
           const int i = i0 + j;
-          sA[r * LC + i] = (i < r) ? sb[r] * v[j] : 0.f;  // L = diag(beta) Atilde, strict lower
+          a[j] = (i < r) ? v[j] : 0.f;
+          sA[r * LC + i] = sb[r] * a[j];  // L = diag(beta) Atilde, strict lower
         }
+        st16g(Ag + r * C + i0, a);
       });
     }
   }
   if (ok) {
     __syncthreads();
     block_inverse<LC>(sT, sA, sW1, sW2);
+    {
+      float* Tg = ws.Tm + ((size_t)ci * H + h) * C * C;  // kept for the backward
+      for (int e = tid; e < C * C; e += blockDim.x) Tg[e] = sT[(e / C) * LC + (e % C)];
+    }
     // phase 2: W = T' Kbar and U' = T' V with T' = T diag(beta)
     uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
             *vl = vh + S::CDb;
@@ -1017,32 +1025,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int myrow = lane < 16 ? 16 * sp + lane : -1;  // M = 64 accumulator row of this thread
   const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
   // TMEM columns
-  constexpr int cA = 0, cW = 64, cU = 192, cdW = 320, cdB = 0, cdA = 256, cRS = 320, cCS = 0;
+  constexpr int cW = 64, cU = 192, cdW = 320, cdB = 0, cdA = 256, cRS = 320, cCS = 0;
 
-  // ---- phase 1: Atilde
+  // ---- phase 1: Atilde and T as the forward left them
+  bool ok = true;
+  float* sT = reinterpret_cast<float*>(R + S::inv_T);
   {
-    uint8_t *afh = R + S::p1_af, *afl = afh + S::CDb, *bfh = R + S::p1_bf, *bfl = bfh + S::CDb;
-    build_tile_ld<C, D, true, Tin>(afh, afl, row_k, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
-    build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
-  }
-  bool ok = run(sy, [&] {
-    const tc::Op ah{tc::smem_u32(R + S::p1_af), C, false}, al{tc::smem_u32(R + S::p1_af + S::CDb), C, false};
-    const tc::Op bh{tc::smem_u32(R + S::p1_bf), C, false}, bl{tc::smem_u32(R + S::p1_bf + S::CDb), C, false};
-    mma4(tb + cA, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false, false);
-  });
-  if (ok) {
-    float* sL = reinterpret_cast<float*>(R + S::inv_L);
-    float* sT = reinterpret_cast<float*>(R + S::inv_T);
-    acc_read<C, C>(tb, cA, [&](int r, int i0, const float* v) {
-      for (int j = 0; j < 16; ++j) {
-        const int i = i0 + j;
-        const float a = (i < r) ? v[j] : 0.f;
-        sAt[r * LC + i] = a;
-        sL[r * LC + i] = sb[r] * a;
-      }
-    });
+    const float* Ag = ws.At + base * C * C;
+    const float* Tg = ws.Tm + base * C * C;
+    for (int e = 4 * tid; e < C * C; e += 4 * blockDim.x) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(Ag + e));
+      const float4 tt = __ldg(reinterpret_cast<const float4*>(Tg + e));
+      const int r = e / C, i = e % C;
+      float* da = sAt + r * LC + i;
+      float* dt = sT + r * LC + i;
+      da[0] = a.x; da[1] = a.y; da[2] = a.z; da[3] = a.w;
+      dt[0] = tt.x; dt[1] = tt.y; dt[2] = tt.z; dt[3] = tt.w;
+    }
     __syncthreads();
-    block_inverse<LC>(sT, sL, reinterpret_cast<float*>(R + S::inv_W1), reinterpret_cast<float*>(R + S::inv_W2));
+  }
+  {
     // ---- phase 2a: W = T' Kbar, U' = T' V (T' = T diag(beta)); the T tile for T^T dX
     uint8_t *tph = R + S::p2_Tp, *tpl = tph + S::CCb, *kbh = R + S::p2_Kb, *kbl = kbh + S::CDb, *vh = R + S::p2_V,
             *vl = vh + S::CDb;

@@ -42,7 +42,7 @@ using tpc_abi::g_prof;
 // workspace layout (bytes) for a plan + shape
 struct WsLayout {
   size_t status, W, U, Khat, decay, S0, slot, dU, dS, dS0seq, pdk, pdG, rdk, rdv, rdg, rdb, tdk, tdv, tdg, tdb, Mt, Bc,
-      total;
+      At, Tm, total;
 };
 
 WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
@@ -74,6 +74,8 @@ WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
   const bool tensor_cores = (C == tpc::kTcC && D == tpc::kTcD);  // (bf16 inputs; sized for either)
   L.Mt = take(tensor_cores ? nc * H * (size_t)tpc::kMtileBytes : 0);
   L.Bc = take(tensor_cores ? nc * H * dd * 4 : 0);
+  L.At = take(tensor_cores ? nc * H * (size_t)C * C * 4 : 0);
+  L.Tm = take(tensor_cores ? nc * H * (size_t)C * C * 4 : 0);
   L.total = o;
   return L;
 }
@@ -87,7 +89,7 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
   w.dU = f(L.dU); w.dS = f(L.dS); w.dS0seq = f(L.dS0seq); w.pdk = f(L.pdk); w.pdG = f(L.pdG);
   w.rdk = f(L.rdk); w.rdv = f(L.rdv); w.rdg = f(L.rdg); w.rdb = f(L.rdb);
   w.tdk = f(L.tdk); w.tdv = f(L.tdv); w.tdg = f(L.tdg); w.tdb = f(L.tdb);
-  w.Mt = f(L.Mt); w.Bc = f(L.Bc);
+  w.Mt = f(L.Mt); w.Bc = f(L.Bc); w.At = f(L.At); w.Tm = f(L.Tm);
   return w;
 }
 
