@@ -391,17 +391,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------ backward dK, dV
-// per key tile of node u: query rows [row of the tile, subtree end of u) in tiles of 64 (queries of u
+// per key tile of node u: query rows [row of the tile, subtree end of u) in tiles of 32 (queries of u
 // itself only from the key row on), S^T = K Q^T, dP^T = V dO^T, P^T = exp(scale S^T - lse),
 // dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 64 accumulators.
+// Q and dO tiles are double-buffered: the next query tile is fetched with cp.async while the current
+// one's P, dS and the dV / dK products run.
 template <bool SPLIT>
 struct AttnDkvSmem {
-  static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2, Pb = size_t(64) * 64 * 2;
+  static constexpr int QT = 32;  // query rows per tile
   static constexpr size_t X = SPLIT ? 1 : 0;
-  static constexpr size_t K = 0, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb, Q = Vl + X * Vb, Ql = Q + Kb;
-  static constexpr size_t dO = Ql + X * Kb, dOl = dO + Vb, P = dOl + X * Vb, dS = P + 2 * Pb;
-  static constexpr size_t vec = dS + 2 * Pb;  // lse[64], delta[64]
-  static constexpr size_t total = vec + 2 * 64 * 4;
+  static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
+  static constexpr size_t Qb = size_t(QT) * kAttnQK * 2, Ob = size_t(QT) * kAttnDV * 2, Pb = size_t(64) * QT * 2;
+  static constexpr size_t QO = (1 + X) * (Qb + Ob);  // one query buffer: Q (+lo), dO (+lo)
+  static constexpr size_t K = 0, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb, Qbuf = Vl + X * Vb;
+  static constexpr size_t P = Qbuf + 2 * QO, dS = P + 2 * Pb;
+  static constexpr size_t vec = dS + 2 * Pb;  // lse[QT], delta[QT] per buffer
+  static constexpr size_t total = vec + 2 * 2 * QT * 4;
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
@@ -416,16 +421,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using namespace tck;
   using S = AttnDkvSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads, QT = S::QT;
   const AttnTile kt = t.attn_ktiles[blockIdx.x];
   const AttnNode nd = t.attn_nodes[kt.node];
   const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  uint8_t *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl, *sQ = asmem + S::Q,
-          *sQl = asmem + S::Ql, *sO = asmem + S::dO, *sOl = asmem + S::dOl;
+  uint8_t *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl;
   uint8_t *sPh = asmem + S::P, *sPl = sPh + S::Pb, *sDh = asmem + S::dS, *sDl = sDh + S::Pb;
-  float* sl = reinterpret_cast<float*>(asmem + S::vec);
-  float* sd = sl + 64;
+  float* svec = reinterpret_cast<float*>(asmem + S::vec);  // [buffer][lse QT | delta QT]
+  // query buffer b: Q, Q_lo, dO, dO_lo
+  auto qbuf = [&](int b, int part) -> uint8_t* {
+    uint8_t* base = asmem + S::Qbuf + (size_t)b * S::QO;
+    return part == 0 ? base : part == 1 ? base + S::Qb : part == 2 ? base + (1 + S::X) * S::Qb
+                                                                   : base + (1 + S::X) * S::Qb + S::Ob;
+  };
   __shared__ __align__(8) uint64_t bar;
   __shared__ uint32_t tslot;
   if (w == 0) tc::tmem_alloc(&tslot, 512);
@@ -433,67 +442,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc::mbar_init(&bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  auto ident = [](int, int, float x) { return x; };
   const int k0 = kt.row, nk = kt.n;
-  build_tile_ld<64, DQ, false, bf, NT>(
-      sK, nullptr, [&](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
-  build_tile_ld<64, DV, false, bf, NT>(
-      sV, nullptr, [&](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+  auto krows = [&](const bf* base, int width) {
+    return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
+  };
+  tile_async<64, DQ, NT>(sK, krows(k, DQ), k);
+  tile_async<64, DV, NT>(sV, krows(v, DV), v);
   if constexpr (SPLIT) {
-    build_tile_ld<64, DQ, false, bf, NT>(
-        sKl, nullptr,
-        [&](int a) -> const bf* { return a < nk && k_lo ? k_lo + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, ident);
-    build_tile_ld<64, DV, false, bf, NT>(
-        sVl, nullptr,
-        [&](int a) -> const bf* { return a < nk && v_lo ? v_lo + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, ident);
+    tile_async<64, DQ, NT>(sKl, krows(k_lo, DQ), k);
+    tile_async<64, DV, NT>(sVl, krows(v_lo, DV), v);
   }
+  const int own_end = nd.row_offset + nd.length, q_end = nd.subtree_end;
+  // query tile at row q0 into buffer b (rows past q_end are zero)
+  auto load_q = [&](int b, int q0) {
+    const int nq = min(QT, q_end - q0);
+    auto rows = [=](const bf* base, int width) {
+      return [=](int a) -> const bf* { return a < nq && base ? base + ((size_t)(q0 + a) * H + h) * width : nullptr; };
+    };
+    tile_async<QT, DQ, NT>(qbuf(b, 0), rows(q, DQ), q);
+    tile_async<QT, DV, NT>(qbuf(b, 2), rows(d_o, DV), d_o);
+    if constexpr (SPLIT) {
+      tile_async<QT, DQ, NT>(qbuf(b, 1), rows(q_lo, DQ), q);
+      tile_async<QT, DV, NT>(qbuf(b, 3), rows(d_o_lo, DV), d_o);
+    }
+  };
+  if (k0 < q_end) load_q(0, k0);
+  tc::cp_async_commit();  // group: K, V, query tile 0
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
   const int r = lane < 16 ? 16 * (w & 3) + lane : -1;  // key row of this thread (M = 64 layout)
-  const int own_end = nd.row_offset + nd.length, q_end = nd.subtree_end;
   Sync sy{&bar, 0u, status};
   bool ok = true, first = true;
-  for (int q0 = k0; q0 < q_end && ok; q0 += 64) {
-    const int nq = min(64, q_end - q0);
-    build_tile_ld<64, DQ, false, bf, NT>(
-        sQ, nullptr, [&](int a) -> const bf* { return a < nq ? q + ((size_t)(q0 + a) * H + h) * DQ : nullptr; },
-        ident);
-    build_tile_ld<64, DV, false, bf, NT>(
-        sO, nullptr, [&](int a) -> const bf* { return a < nq ? d_o + ((size_t)(q0 + a) * H + h) * DV : nullptr; },
-        ident);
-    if constexpr (SPLIT) {
-      build_tile_ld<64, DQ, false, bf, NT>(
-          sQl, nullptr,
-          [&](int a) -> const bf* { return a < nq && q_lo ? q_lo + ((size_t)(q0 + a) * H + h) * DQ : nullptr; },
-          ident);
-      build_tile_ld<64, DV, false, bf, NT>(
-          sOl, nullptr,
-          [&](int a) -> const bf* { return a < nq && d_o_lo ? d_o_lo + ((size_t)(q0 + a) * H + h) * DV : nullptr; },
-          ident);
-    }
-    if (tid < 64) {
+  int b = 0;
+  for (int q0 = k0; q0 < q_end && ok; q0 += QT, b ^= 1) {
+    const int nq = min(QT, q_end - q0);
+    const bool more = q0 + QT < q_end;
+    tc::cp_async_wait<0>();  // this query tile (and, the first time, K and V) have arrived
+    float* sl = svec + b * 2 * QT;
+    float* sd = sl + QT;
+    if (tid < QT) {
       sl[tid] = tid < nq ? lse[(size_t)(q0 + tid) * H + h] : 0.f;
       sd[tid] = tid < nq ? delta[(size_t)(q0 + tid) * H + h] : 0.f;
     }
+    uint8_t *sQ = qbuf(b, 0), *sQl = qbuf(b, 1), *sO = qbuf(b, 2), *sOl = qbuf(b, 3);
     ok = run(sy, [&] {
       mma4(tb, tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sKl), 64, false},
-           tc::Op{tc::smem_u32(sQ), 64, false}, tc::Op{tc::smem_u32(sQl), 64, false}, DQ,
-           tc::idesc_bf16(64, 64, false, false), false, !SPLIT, !SPLIT);
+           tc::Op{tc::smem_u32(sQ), QT, false}, tc::Op{tc::smem_u32(sQl), QT, false}, DQ,
+           tc::idesc_bf16(64, QT, false, false), false, !SPLIT, !SPLIT);
       mma4(tb + 64, tc::Op{tc::smem_u32(sV), 64, false}, tc::Op{tc::smem_u32(sVl), 64, false},
-           tc::Op{tc::smem_u32(sO), 64, false}, tc::Op{tc::smem_u32(sOl), 64, false}, DV,
-           tc::idesc_bf16(64, 64, false, false), false, !SPLIT, !SPLIT);
+           tc::Op{tc::smem_u32(sO), QT, false}, tc::Op{tc::smem_u32(sOl), QT, false}, DV,
+           tc::idesc_bf16(64, QT, false, false), false, !SPLIT, !SPLIT);
     });
     if (!ok) break;
-    float s[64], dp[64];
+    // the other buffer was last read by the previous tile's dV / dK products, which have completed
+    if (more) load_q(b ^ 1, q0 + QT);
+    tc::cp_async_commit();
+    float s[QT], dp[QT];
     tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
-    tc::tmem_ld32(la + 32, *reinterpret_cast<float(*)[32]>(s + 32));
     tc::tmem_ld32(la + 64, *reinterpret_cast<float(*)[32]>(dp));
-    tc::tmem_ld32(la + 96, *reinterpret_cast<float(*)[32]>(dp + 32));
     if (r >= 0) {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
+      for (int j = 0; j < QT; ++j) {
         const int qrow = q0 + j;
         const bool valid = r < nk && j < nq && !(qrow < own_end && qrow < k0 + r);
         const float p = valid ? expf(s[j] * scale - sl[j]) : 0.f;
@@ -501,7 +512,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         dp[j] = p * (dp[j] - sd[j]);
       }
 #pragma unroll
-      for (int j = 0; j < 64; j += 16) {
+      for (int j = 0; j < QT; j += 16) {
         put16<64, true>(sPh, sPl, r, j, s + j);
         put16<64, true>(sDh, sDl, r, j, dp + j);
       }
@@ -510,21 +521,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     first = false;
     ok = run(sy, [&] {
       mma4(tb + 128, tc::Op{tc::smem_u32(sPh), 64, false}, tc::Op{tc::smem_u32(sPl), 64, false},
-           tc::Op{tc::smem_u32(sO), 64, true}, tc::Op{tc::smem_u32(sOl), 64, true}, 64,
+           tc::Op{tc::smem_u32(sO), QT, true}, tc::Op{tc::smem_u32(sOl), QT, true}, QT,
            tc::idesc_bf16(64, DV, false, true), acc_on, false, !SPLIT);
       mma4(tb + 256, tc::Op{tc::smem_u32(sDh), 64, false}, tc::Op{tc::smem_u32(sDl), 64, false},
-           tc::Op{tc::smem_u32(sQ), 64, true}, tc::Op{tc::smem_u32(sQl), 64, true}, 64,
+           tc::Op{tc::smem_u32(sQ), QT, true}, tc::Op{tc::smem_u32(sQl), QT, true}, QT,
            tc::idesc_bf16(64, DQ, false, true), acc_on, false, !SPLIT);
     });
-    tc::fence_before_sync();
-    __syncthreads();
   }
+  tc::cp_async_wait<0>();
   if (ok) {
     for (int c = 0; c < DV; c += 32) {
       float g[32];
       tc::tmem_ld32(la + 128 + c, g);
       if (r >= 0 && r < nk) {
         Tio* dst = dv + ((size_t)(k0 + r) * H + h) * DV + c;
+        if (first) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) g[j] = 0.f;
+        }
         st_out16(dst, g);
         st_out16(dst + 16, g + 16);
       }
@@ -534,7 +548,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc::tmem_ld32(la + 256 + c, g);
       if (r >= 0 && r < nk) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) g[j] *= scale;
+        for (int j = 0; j < 32; ++j) g[j] = first ? 0.f : g[j] * scale;
         Tio* dst = dk + ((size_t)(k0 + r) * H + h) * DQ + c;
         st_out16(dst, g);
         st_out16(dst + 16, g + 16);
