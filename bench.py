@@ -251,7 +251,7 @@ def group_flops_per_row(depth):
 
 def measure_group(args, world, rank, tpc, torch, peaks):
     import synth.gpu as sgpu
-    w = synth.workload(GROUP_WORKLOAD)
+    w = synth.workload(args.group_workload)
     t = w.tree
     seed = 3 + 1000 * rank
     plan = tpc.Plan(t.parent, t.length, 64).upload()
@@ -439,6 +439,7 @@ def main():
     ap.add_argument("--no-expanded", action="store_true")
     ap.add_argument("--no-group", action="store_true", help="skip the hybrid layer group (3 KDA + 1 MLA) measurement")
     ap.add_argument("--group-steps", type=int, default=3)
+    ap.add_argument("--group-workload", default=GROUP_WORKLOAD, help="tree of the hybrid group (agentic by default)")
     ap.add_argument("--no-wide", action="store_true", help="skip the wide tree with log-prob recovery")
     ap.add_argument("--wide-steps", type=int, default=2)
     ap.add_argument("--workload", default=WORKLOAD, help="single_fork (default), agentic, agentic_small")
