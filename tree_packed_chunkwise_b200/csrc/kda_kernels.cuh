@@ -23,6 +23,7 @@ struct KdaWs {
   float *tdk, *tdv, *tdg, *tdb;                            // own part of replay-target rows
   float *Mt, *Bc;  // tensor-core path: per-chunk state transition M (bf16 hi/lo operand tile) and B (fp32)
   float *At, *Tm;  // tensor-core path: per-chunk gated key products Atilde and T = (I + diag(beta) Atilde)^{-1}
+  float *Pm;       // tensor-core path: per-chunk masked gated products P = lower_incl(gated(q, k))
 };
 
 template <int C, int D>

@@ -546,11 +546,11 @@ struct OutTcSmem {
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_out_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
-                   const Tin* __restrict__ g_, Tout* __restrict__ o_, KdaWs ws) {
+                   const Tin* __restrict__ g_, Tout* __restrict__ o_, KdaWs ws, int chunk0 = 0) {
   using namespace tck;
   using S = OutTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD;
-  const int ci = blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -598,10 +598,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
   uint8_t *qbh = wh, *qbl = wl;
   if (ok) {
+    float* Pg = ws.Pm + base * C * C;  // kept for the backward
     acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
       float m[16];
       for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
       put16<C, true>(ph, pl, r, i0, m);
+      st16g(Pg + r * C + i0, m);
     });
     acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
       float u[16];
@@ -689,27 +691,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
   };
   const size_t base = (size_t)ci * H + h;
-  uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
   uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *doh = tsm + S::dO, *dol = doh + S::CDb;
   uint8_t *wh = tsm + S::Wt, *wl = wh + S::CDb;
-  build_tile_ld<C, D, true, Tin>(qfh, qfl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
-  build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
   build_tile_ld<C, D, true, Tin>(qbh, qbl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c]); });
   build_tile_ld<C, D, !EX, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
   const float* Wg = ws.W + base * C * D;
   build_tile_ld<C, D, true, float>(wh, wl, [&](int r) { return Wg + r * D; }, [&](int, int, float x) { return -x; });
-  bool ok = run(sy, [&] {
-    const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
-    const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
-    mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false);
-  });
+  // P (masked gated q k products) as the forward left it
   uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *duh = pl + S::CCb, *dul = duh + S::CDb;
-  if (ok) {
-    acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
+  {
+    const float* Pg = ws.Pm + base * C * C;
+    for (int e = tid; e < C * (C / 16); e += blockDim.x) {
+      const int r = e / (C / 16), i0 = (e % (C / 16)) * 16;
       float m[16];
-      for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+      ld16g(Pg + r * C + i0, m);
       put16<C, true>(ph, pl, r, i0, m);  // element (r, i): MN-major operand P^T (k = r, m = i)
-    });
+    }
+  }
+  bool ok = true;
+  {
     ok = run(sy, [&] {
       const tc::Op pH{tc::smem_u32(ph), C, true}, pL{tc::smem_u32(pl), C, true};
       const tc::Op oH{tc::smem_u32(doh), C, true}, oL{tc::smem_u32(dol), C, true};
@@ -767,12 +767,13 @@ struct BdqTcSmem {
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_bwd_dq_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
-                  const Tin* __restrict__ g_, const Tin* __restrict__ do_, Tout* __restrict__ dq_, KdaWs ws) {
+                  const Tin* __restrict__ g_, const Tin* __restrict__ do_, Tout* __restrict__ dq_, KdaWs ws,
+                  int chunk0 = 0) {
   using namespace tck;
   using S = BdqTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -956,12 +957,13 @@ template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_bwd_dkv_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, Tout* __restrict__ dk_,
-                   Tout* __restrict__ dv_, float* __restrict__ dg_, float* __restrict__ dbeta_, KdaWs ws) {
+                   Tout* __restrict__ dv_, float* __restrict__ dg_, float* __restrict__ dbeta_, KdaWs ws,
+                   int chunk0 = 0) {
   using namespace tck;
   using S = BdkvTcSmemT<Tin>;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];

@@ -39,10 +39,16 @@ using tpc_abi::a256;
 using tpc_abi::fail;
 using tpc_abi::g_prof;
 
+#define TPC_TRY_ABI(call)        \
+  do {                           \
+    const int r_ = (call);       \
+    if (r_ != TPC_OK) return r_; \
+  } while (0)
+
 // workspace layout (bytes) for a plan + shape
 struct WsLayout {
   size_t status, W, U, Khat, decay, S0, slot, dU, dS, dS0seq, pdk, pdG, rdk, rdv, rdg, rdb, tdk, tdv, tdg, tdb, Mt, Bc,
-      At, Tm, total;
+      At, Tm, Pm, total;
 };
 
 WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
@@ -76,6 +82,7 @@ WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
   L.Bc = take(tensor_cores ? nc * H * dd * 4 : 0);
   L.At = take(tensor_cores ? nc * H * (size_t)C * C * 4 : 0);
   L.Tm = take(tensor_cores ? nc * H * (size_t)C * C * 4 : 0);
+  L.Pm = take(tensor_cores ? nc * H * (size_t)C * C * 4 : 0);
   L.total = o;
   return L;
 }
@@ -89,7 +96,7 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
   w.dU = f(L.dU); w.dS = f(L.dS); w.dS0seq = f(L.dS0seq); w.pdk = f(L.pdk); w.pdG = f(L.pdG);
   w.rdk = f(L.rdk); w.rdv = f(L.rdv); w.rdg = f(L.rdg); w.rdb = f(L.rdb);
   w.tdk = f(L.tdk); w.tdv = f(L.tdv); w.tdg = f(L.tdg); w.tdb = f(L.tdb);
-  w.Mt = f(L.Mt); w.Bc = f(L.Bc); w.At = f(L.At); w.Tm = f(L.Tm);
+  w.Mt = f(L.Mt); w.Bc = f(L.Bc); w.At = f(L.At); w.Tm = f(L.Tm); w.Pm = f(L.Pm);
   return w;
 }
 
@@ -110,6 +117,30 @@ int check_shape(const tpc_plan* plan, const tpc_kda_shape* s) {
 template <class KernelT>
 cudaError_t set_smem(KernelT k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// A second stream per device for per-round work that may overlap the next round's sequential scan
+// (created once, non-blocking; ordered against the caller's stream by events).
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static std::vector<cudaStream_t> streams;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)streams.size() <= dev) streams.resize(dev + 1, nullptr);
+  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
+
+// work queued on `to` from now on runs after everything already queued on `from`
+int stream_after(cudaStream_t to, cudaStream_t from) {
+  cudaEvent_t e;
+  TPC_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  TPC_CUDA(cudaEventRecord(e, from));
+  TPC_CUDA(cudaStreamWaitEvent(to, e, 0));
+  TPC_CUDA(cudaEventDestroy(e));
+  return TPC_OK;
 }
 
 template <int C, int D, typename Tin, typename Tout>
@@ -139,25 +170,34 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     TPC_LAUNCH("kda_fwd_prep", st,
                (kda_fwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, fwd_prep_smem<C, D>(), st>>>(p.dt, H, k, v, g, b, w)));
   }
-  if constexpr (kTensorCores) TPC_CUDA(set_smem(kda_scan_tc<false>, ScanTcSmem::total));
-  for (int r = 1; r <= p.n_rounds; ++r) {
-    const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-    if constexpr (kTensorCores) {
-      TPC_LAUNCH("kda_fwd_scan_tc", st,
-                 (kda_scan_tc<false><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
-                     p.dt, s0, H, io->init_state, io->final_state, nullptr, w)));
-    } else {
+  if constexpr (kTensorCores) {
+    // round r's output kernel (its chunks only) runs on a second stream while round r + 1 scans
+    TPC_CUDA(set_smem(kda_scan_tc<false>, ScanTcSmem::total));
+    TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
+    cudaStream_t side = side_stream();
+    if (!side) return fail(TPC_ERR_CUDA, "could not create the library's second stream");
+    for (int r = 1; r <= p.n_rounds; ++r) {
+      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+      const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
+      if (s1 > s0)
+        TPC_LAUNCH("kda_fwd_scan_tc", st,
+                   (kda_scan_tc<false><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
+                       p.dt, s0, H, io->init_state, io->final_state, nullptr, w)));
+      if (c1 > c0) {
+        TPC_TRY_ABI(stream_after(side, st));
+        TPC_LAUNCH("kda_fwd_out_tc", side,
+                   (kda_fwd_out_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, OutTcSmem::total, side>>>(
+                       p.dt, H, q, k, g, static_cast<Tout*>(io->o), w, c0)));
+      }
+    }
+    TPC_TRY_ABI(stream_after(st, side));
+  } else {
+    for (int r = 1; r <= p.n_rounds; ++r) {
+      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       TPC_LAUNCH("kda_fwd_scan", st,
                  (kda_fwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads, scan_smem<C, D, DVT>(), st>>>(
                      p.dt, s0, H, io->init_state, io->final_state, w)));
     }
-  }
-  if constexpr (kTensorCores) {
-    TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
-    TPC_LAUNCH("kda_fwd_out_tc", st,
-               (kda_fwd_out_tc<Tin, Tout><<<dim3(nc, H), kThreads, OutTcSmem::total, st>>>(
-                   p.dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
-  } else {
     TPC_LAUNCH("kda_fwd_out", st,
                (kda_fwd_out<C, D, Tin, Tout><<<dim3(nc, H), kThreads, out_smem<C, D>(), st>>>(
                    p.dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
@@ -193,31 +233,40 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
     TPC_LAUNCH("kda_bwd_prep", st,
                (kda_bwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, bprep_smem<C, D>(), st>>>(p.dt, H, q, k, g, dO, w)));
   }
-  if constexpr (kTensorCores) TPC_CUDA(set_smem(kda_scan_tc<true>, ScanTcSmem::total));
-  for (int r = p.n_rounds; r >= 1; --r) {
-    const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-    if constexpr (kTensorCores) {
-      TPC_LAUNCH("kda_bwd_scan_tc", st,
-                 (kda_scan_tc<true><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
-                     p.dt, s0, H, nullptr, nullptr, io->d_final, w)));
-    } else {
+  if constexpr (kTensorCores) {
+    // round r's chunk kernels (its chunks only) run on a second stream while round r - 1 scans
+    TPC_CUDA(set_smem(kda_scan_tc<true>, ScanTcSmem::total));
+    TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
+    TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmemT<Tin>::total));
+    cudaStream_t side = side_stream();
+    if (!side) return fail(TPC_ERR_CUDA, "could not create the library's second stream");
+    for (int r = p.n_rounds; r >= 1; --r) {
+      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+      const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
+      if (s1 > s0)
+        TPC_LAUNCH("kda_bwd_scan_tc", st,
+                   (kda_scan_tc<true><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
+                       p.dt, s0, H, nullptr, nullptr, io->d_final, w)));
+      if (c1 > c0) {
+        TPC_TRY_ABI(stream_after(side, st));
+        TPC_LAUNCH("kda_bwd_dq_tc", side,
+                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdqTcSmem::total, side>>>(
+                       p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w, c0)));
+        TPC_LAUNCH("kda_bwd_dkv_tc", side,
+                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdkvTcSmemT<Tin>::total, side>>>(
+                       p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg,
+                       io->dbeta, w, c0)));
+      }
+    }
+    TPC_TRY_ABI(stream_after(st, side));
+  } else {
+    for (int r = p.n_rounds; r >= 1; --r) {
+      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       TPC_LAUNCH("kda_bwd_scan", st,
                  (kda_bwd_scan<C, D, DVT><<<dim3(s1 - s0, H, D / DVT), kThreads,
                                             scan_smem<C, D, DVT>() + sizeof(float) * D * (DVT + 1), st>>>(
                      p.dt, s0, H, io->d_final, w)));
     }
-  }
-  if constexpr (kTensorCores) {
-    TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
-    TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmemT<Tin>::total));
-    TPC_LAUNCH("kda_bwd_dq_tc", st,
-               (kda_bwd_dq_tc<Tin, Tout><<<dim3(nc, H), kThreads, BdqTcSmem::total, st>>>(
-                   p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w)));
-    TPC_LAUNCH("kda_bwd_dkv_tc", st,
-               (kda_bwd_dkv_tc<Tin, Tout><<<dim3(nc, H), kThreads, BdkvTcSmemT<Tin>::total, st>>>(
-                   p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg, io->dbeta,
-                   w)));
-  } else {
     TPC_LAUNCH("kda_bwd_dq", st,
                (kda_bwd_dq<C, D, Tin, Tout><<<dim3(nc, H), kThreads, bdq_smem<C, D>(), st>>>(
                    p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w)));
