@@ -51,11 +51,12 @@ struct GemmArgs {
   void* C;
   int* status;
   int passes;         // 1: A B;  2: + A_lo B;  3: + A B_lo
+  int m_fast;         // tile order: 1 = M blocks fastest (concurrent CTAs share B), 0 = N blocks fastest
 };
 
 // Persistent, warp-specialised: grid = min(tiles, SMs); each CTA walks tiles blockIdx.x,
-// blockIdx.x + gridDim.x, ... (N blocks fastest, so concurrent CTAs share A rows and all of B stays
-// in L2).  Warp 0 lane 0 issues TMA loads into a 4-stage ring; warp 1 lane 0 issues the MMAs into one
+// blockIdx.x + gridDim.x, ...  The tile order runs along the smaller of M and N fastest, so the
+// CTAs in flight share the tiles of the larger operand and the smaller one stays in L2.  Warp 0 lane 0 issues TMA loads into a 4-stage ring; warp 1 lane 0 issues the MMAs into one
 // of two TMEM accumulators (256 columns each); warps 2-5 drain the other accumulator to global
 // memory (thread = row), so a tile's epilogue overlaps the next tile's main loop.  Every wait is
 // bounded; a timeout records TPC_ERR_TIMEOUT and every role stops.
@@ -77,6 +78,8 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
   const int IT = KT * g.passes;  // pass p = it / KT uses (A, B), (A_lo, B), (A, B_lo)
   const int n_tiles = (g.N + kGemmBN - 1) / kGemmBN, m_tiles = (g.M + kGemmBM - 1) / kGemmBM;
   const int tiles = n_tiles * m_tiles;
+  auto tile_m = [&](int t) { return g.m_fast ? t % m_tiles : t / n_tiles; };
+  auto tile_n = [&](int t) { return g.m_fast ? t / m_tiles : t % n_tiles; };
   if (w == 1) tmem_alloc(&tslot, 512);
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
     if (lane == 0) {  // producer
       int it_all = 0;
       for (int t = blockIdx.x; t < tiles && !aborted(); t += gridDim.x) {
-        const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * kGemmBN;
+        const int m0 = tile_m(t) * kGemmBM, n0 = tile_n(t) * kGemmBN;
         for (int it = 0; it < IT; ++it, ++it_all) {
           const int s = it_all % kGemmStages, pass = it / KT, kt = it - pass * KT;
           if (it_all >= kGemmStages && !mbar_wait(&empty[s], ((it_all / kGemmStages) - 1) & 1)) {
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       }
       if (__any_sync(0xffffffffu, aborted())) break;
       fence_after_sync();
-      const int m = (t / n_tiles) * kGemmBM + row, n0 = (t % n_tiles) * kGemmBN;
+      const int m = tile_m(t) * kGemmBM + row, n0 = tile_n(t) * kGemmBN;
       const uint32_t la = tb + ((uint32_t)(32 * sp) << 16) + (uint32_t)(b * kGemmBN);
       for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
         float v[16];

@@ -610,7 +610,8 @@ int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B
   ok = ok && encode(&tblo, B_lo ? B_lo : B, b_mn, N, ldb, tpc::kGemmBN);
   if (!ok) return fail(TPC_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   const int passes = B_lo ? 3 : (A_lo ? 2 : 1);
-  tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status, passes};
+  tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status, passes,
+                  M < N ? 1 : 0};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t tiles = ((N + tpc::kGemmBN - 1) / tpc::kGemmBN) * ((M + tpc::kGemmBM - 1) / tpc::kGemmBM);
   if (tiles > (int64_t)1 << 31) return fail(TPC_ERR_BAD_SHAPE, "gemm: too many tiles");
