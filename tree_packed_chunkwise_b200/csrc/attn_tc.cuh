@@ -115,9 +115,14 @@ struct AttnFwdSmem {
 // Per query tile: O accumulates in TMEM across the key tiles (P V products with accumulate), the
 // online softmax keeps a per-row reference maximum that is raised (and O, l rescaled) only when a
 // tile's maximum exceeds it by more than 8, so every p = exp(s - m) stays below e^8.  The next key
-// tile's K and V are fetched with cp.async while the current tile's softmax and P V run.
+// tile's K and V are fetched with cp.async while the current tile's softmax and P V run.  Eight
+// warps: warp w holds the TMEM lanes (query rows) of sub-partition w % 4 and the column half
+// w / 4 (S columns 32 h .. 32 h + 31, O columns 64 h .. 64 h + 63); the two threads of a row combine
+// their partial maxima and sums through shared memory, in a fixed order.
+constexpr int kAttnFwdThreads = 256;
+
 template <typename Tout, bool SPLIT>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnFwdThreads, 1)
     attn_fwd_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
                 const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
                 const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
@@ -126,16 +131,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using namespace tck;
   using S = AttnFwdSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnFwdThreads;
   constexpr float kRaise = 8.f;
   const AttnTile qt = t.attn_qtiles[blockIdx.x];
-  const int h = blockIdx.y, tid = threadIdx.x;
+  const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int row = 32 * (w & 3) + lane, half = w >> 2;
   extern __shared__ __align__(1024) uint8_t asmem[];
   uint8_t *sQ = asmem + S::Q, *sQl = asmem + S::Ql, *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V,
           *sVl = asmem + S::Vl, *sPh = asmem + S::P, *sPl = sPh + S::Pb;
+  __shared__ float red_max[2][128], red_sum[2][128];
   __shared__ __align__(8) uint64_t bar;
   __shared__ uint32_t tslot;
-  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 256);
+  if (w == 0) tc::tmem_alloc(&tslot, 256);
   if (tid == 0) {
     tc::mbar_init(&bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -170,9 +177,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
-  const uint32_t la = tb + ((uint32_t)(32 * (tid >> 5)) << 16);
+  const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
   Sync sy{&bar, 0u, status};
-  const int qrow = qt.row + tid;
+  const int qrow = qt.row + row;
   float m_ref = -INFINITY, l = 0.f;
   bool first = true, ok = true;
   while (have) {
@@ -188,19 +195,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (!ok) break;
     if (more) load_kv(true, k1, n1);  // K is free once S is in TMEM
     tc::cp_async_commit();
-    float s[64];
-    tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
-    tc::tmem_ld32(la + 32, *reinterpret_cast<float(*)[32]>(s + 32));
+    float s[32];
+    tc::tmem_ld32(la + 32 * half, s);
     float mx = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      const bool valid = tid < qt.n && j < nk && (!own || k0 + j <= qrow);
+    for (int j = 0; j < 32; ++j) {
+      const int c = 32 * half + j;
+      const bool valid = row < qt.n && c < nk && (!own || k0 + c <= qrow);
       s[j] = valid ? s[j] * scale : -INFINITY;
       mx = fmaxf(mx, s[j]);
     }
-    // raise the reference where a tile's maximum exceeds it by more than kRaise; O (accumulated so
-    // far) and l follow.  TMEM loads and stores are warp-collective: a warp rescales its 32 rows
-    // together when any of them raised (the others with factor 1).
+    red_max[half][row] = mx;
+    __syncthreads();
+    mx = fmaxf(red_max[0][row], red_max[1][row]);
+    // raise the reference where the tile's maximum exceeds it by more than kRaise; O (accumulated so
+    // far) and l follow.  Both threads of a row take the same decision; TMEM loads and stores are
+    // warp-collective, so a warp rescales its 32 rows together when any of them raised.
     const bool raise = mx > m_ref + kRaise;
     const float corr = !raise ? 1.f : (m_ref == -INFINITY ? 0.f : expf(m_ref - mx));
     if (raise) {
@@ -208,23 +218,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       m_ref = mx;
     }
     if (!first && __any_sync(0xffffffffu, raise)) {
-      for (int c = 0; c < DV; c += 16) {
+      for (int c = 0; c < DV / 2; c += 16) {
         float ov[16];
-        tc::tmem_ld16(la + 64 + c, ov);
+        tc::tmem_ld16(la + 64 + DV / 2 * half + c, ov);
 #pragma unroll
         for (int j = 0; j < 16; ++j) ov[j] *= corr;
-        tc::tmem_st16(la + 64 + c, ov);
+        tc::tmem_st16(la + 64 + DV / 2 * half + c, ov);
       }
     }
     float psum = 0.f;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
+    for (int j = 0; j < 32; ++j) {
       s[j] = s[j] == -INFINITY ? 0.f : expf(s[j] - m_ref);
       psum += s[j];
     }
-    l += psum;
+    red_sum[half][row] = psum;
 #pragma unroll
-    for (int j = 0; j < 64; j += 16) put16<128, true>(sPh, sPl, tid, j, s + j);
+    for (int j = 0; j < 32; j += 16) put16<128, true>(sPh, sPl, row, 32 * half + j, s + j);
+    __syncthreads();
+    l += red_sum[0][row] + red_sum[1][row];
     tc::cp_async_wait<1>();  // this tile's V has arrived
     const bool acc_on = !first;
     ok = run(sy, [&] {
@@ -241,21 +253,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc::cp_async_wait<0>();
   if (ok) {
     const float inv = 1.f / l;
-    Tout* dst = o + ((size_t)qrow * H + h) * DV;
-    for (int c = 0; c < DV; c += 16) {
+    Tout* dst = o + ((size_t)qrow * H + h) * DV + DV / 2 * half;
+    for (int c = 0; c < DV / 2; c += 16) {
       float ov[16];
-      tc::tmem_ld16(la + 64 + c, ov);  // warp-collective: every row takes part
-      if (tid < qt.n) {
+      tc::tmem_ld16(la + 64 + DV / 2 * half + c, ov);  // warp-collective: every row takes part
+      if (row < qt.n) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) ov[j] *= inv;
         st_out16(dst + c, ov);
       }
     }
-    if (tid < qt.n) lse[(size_t)qrow * H + h] = m_ref + logf(l);
+    if (row < qt.n && half == 0) lse[(size_t)qrow * H + h] = m_ref + logf(l);
   }
   tc::fence_before_sync();
   __syncthreads();
-  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 256);
+  if (w == 0) tc::tmem_dealloc(tb, 256);
 }
 
 // ------------------------------------------------------------------------------------------ backward dQ
@@ -273,8 +285,12 @@ struct AttnDqSmem {
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
+// Eight warps: warp w holds the query rows of TMEM sub-partition w % 4 and the column half w / 4 of
+// each key tile (and of dQ at the end).
+constexpr int kAttnDqThreads = 256;
+
 template <typename Tio, bool SPLIT>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnDqThreads, 1)
     attn_bwd_dq_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
                    const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
                    const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
@@ -284,15 +300,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using namespace tck;
   using S = AttnDqSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads, KT = S::KT;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnDqThreads, KT = S::KT, KH = KT / 2;
   const AttnTile qt = t.attn_qtiles[blockIdx.x];
-  const int h = blockIdx.y, tid = threadIdx.x;
+  const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int row = 32 * (w & 3) + lane, half = w >> 2;
   extern __shared__ __align__(1024) uint8_t asmem[];
   uint8_t *sQ = asmem + S::Q, *sQl = asmem + S::Ql, *sO = asmem + S::dO, *sOl = asmem + S::dOl, *sK = asmem + S::K,
           *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl, *sDh = asmem + S::dS, *sDl = sDh + S::Pb;
+  __shared__ float s_dl[128], s_ls[128];
   __shared__ __align__(8) uint64_t bar;
   __shared__ uint32_t tslot;
-  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  if (w == 0) tc::tmem_alloc(&tslot, 512);
   if (tid == 0) {
     tc::mbar_init(&bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -310,26 +328,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     build_tile_ld<128, DQ, false, bf, NT>(sQl, nullptr, qrows(q_lo), ident);
     build_tile_ld<128, DV, false, bf, NT>(sOl, nullptr, orows(d_o_lo), ident);
   }
-  const int qrow = qt.row + tid;
-  float dl = 0.f, ls = 0.f;
-  if (tid < qt.n) {
-    const Tio* orow = o + ((size_t)qrow * H + h) * DV;
-    const bf* grow = d_o + ((size_t)qrow * H + h) * DV;
-    const bf* glow = SPLIT && d_o_lo ? d_o_lo + ((size_t)qrow * H + h) * DV : nullptr;
-    for (int j = 0; j < DV; ++j)
-      dl = fmaf(to_f(orow[j]), __bfloat162float(grow[j]) + (glow ? __bfloat162float(glow[j]) : 0.f), dl);
-    delta[(size_t)qrow * H + h] = dl;
-    ls = lse[(size_t)qrow * H + h];
+  const int qrow = qt.row + row;
+  if (half == 0) {
+    float dl = 0.f, ls = 0.f;
+    if (row < qt.n) {
+      const Tio* orow = o + ((size_t)qrow * H + h) * DV;
+      const bf* grow = d_o + ((size_t)qrow * H + h) * DV;
+      const bf* glow = SPLIT && d_o_lo ? d_o_lo + ((size_t)qrow * H + h) * DV : nullptr;
+      for (int j = 0; j < DV; ++j)
+        dl = fmaf(to_f(orow[j]), __bfloat162float(grow[j]) + (glow ? __bfloat162float(glow[j]) : 0.f), dl);
+      delta[(size_t)qrow * H + h] = dl;
+      ls = lse[(size_t)qrow * H + h];
+    }
+    s_dl[row] = dl;
+    s_ls[row] = ls;
   }
   __syncthreads();
+  const float dl = s_dl[row], ls = s_ls[row];
   tc::fence_after_sync();
   const uint32_t tb = tslot;
-  const uint32_t la = tb + ((uint32_t)(32 * (tid >> 5)) << 16);
+  const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
   Sync sy{&bar, 0u, status};
   bool first = true;
   const bool ok = for_key_tiles<KT>(t, qt, [&](int k0, int nk, bool own) -> bool {
-    auto krows = [&](const bf* base, int w) {
-      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * w : nullptr; };
+    auto krows = [&](const bf* base, int width) {
+      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
     };
     build_tile_ld<KT, DQ, false, bf, NT>(sK, nullptr, krows(k, DQ), ident);
     build_tile_ld<KT, DV, false, bf, NT>(sV, nullptr, krows(v, DV), ident);
@@ -346,20 +369,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
         }))
       return false;
-    float s[KT], dp[KT];
+    float s[KH], dp[KH];
 #pragma unroll
-    for (int c = 0; c < KT; c += 32) {
-      tc::tmem_ld32(la + c, *reinterpret_cast<float(*)[32]>(s + c));
-      tc::tmem_ld32(la + 64 + c, *reinterpret_cast<float(*)[32]>(dp + c));
+    for (int c = 0; c < KH; c += 16) {
+      tc::tmem_ld16(la + KH * half + c, *reinterpret_cast<float(*)[16]>(s + c));
+      tc::tmem_ld16(la + 64 + KH * half + c, *reinterpret_cast<float(*)[16]>(dp + c));
     }
 #pragma unroll
-    for (int j = 0; j < KT; ++j) {
-      const bool valid = tid < qt.n && j < nk && (!own || k0 + j <= qrow);
+    for (int j = 0; j < KH; ++j) {
+      const int c = KH * half + j;
+      const bool valid = row < qt.n && c < nk && (!own || k0 + c <= qrow);
       const float p = valid ? expf(s[j] * scale - ls) : 0.f;
       s[j] = p * (dp[j] - dl);
     }
 #pragma unroll
-    for (int j = 0; j < KT; j += 16) put16<128, true>(sDh, sDl, tid, j, s + j);
+    for (int j = 0; j < KH; j += 16) put16<128, true>(sDh, sDl, row, KH * half + j, s + j);
     const bool acc_on = !first;
     first = false;
     if (!run(sy, [&] {
@@ -373,13 +397,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     return true;
   });
   if (ok) {
-    for (int c = 0; c < DQ; c += 32) {
+    for (int c = 0; c < DQ / 2; c += 32) {
       float g[32];
-      tc::tmem_ld32(la + 128 + c, g);
-      if (tid < qt.n) {
+      tc::tmem_ld32(la + 128 + DQ / 2 * half + c, g);
+      if (row < qt.n) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) g[j] *= scale;
-        Tio* dst = dq + ((size_t)qrow * H + h) * DQ + c;
+        Tio* dst = dq + ((size_t)qrow * H + h) * DQ + DQ / 2 * half + c;
         st_out16(dst, g);
         st_out16(dst + 16, g + 16);
       }
@@ -387,7 +411,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
+  if (w == 0) tc::tmem_dealloc(tb, 512);
 }
 
 // ------------------------------------------------------------------------------------------ backward dK, dV
@@ -410,8 +434,12 @@ struct AttnDkvSmem {
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
+// Eight warps: warps w and w + 4 share the key rows of TMEM sub-partition w % 4 (M = 64 layout:
+// lanes 0..15) and split the columns of every query tile and of dV / dK at the end.
+constexpr int kAttnDkvThreads = 256;
+
 template <typename Tio, bool SPLIT>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnDkvThreads, 1)
     attn_bwd_dkv_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
                     const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
                     const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
@@ -421,7 +449,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using namespace tck;
   using S = AttnDkvSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnThreads, QT = S::QT;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnDkvThreads, QT = S::QT, QH = QT / 2;
   const AttnTile kt = t.attn_ktiles[blockIdx.x];
   const AttnNode nd = t.attn_nodes[kt.node];
   const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -473,6 +501,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tb = tslot;
   const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
   const int r = lane < 16 ? 16 * (w & 3) + lane : -1;  // key row of this thread (M = 64 layout)
+  const int half = w >> 2;                                // column half of this warp
   Sync sy{&bar, 0u, status};
   bool ok = true, first = true;
   int b = 0;
@@ -499,23 +528,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // the other buffer was last read by the previous tile's dV / dK products, which have completed
     if (more) load_q(b ^ 1, q0 + QT);
     tc::cp_async_commit();
-    float s[QT], dp[QT];
-    tc::tmem_ld32(la, *reinterpret_cast<float(*)[32]>(s));
-    tc::tmem_ld32(la + 64, *reinterpret_cast<float(*)[32]>(dp));
+    float s[QH], dp[QH];
+    tc::tmem_ld16(la + QH * half, *reinterpret_cast<float(*)[16]>(s));
+    tc::tmem_ld16(la + 64 + QH * half, *reinterpret_cast<float(*)[16]>(dp));
     if (r >= 0) {
 #pragma unroll
-      for (int j = 0; j < QT; ++j) {
-        const int qrow = q0 + j;
-        const bool valid = r < nk && j < nq && !(qrow < own_end && qrow < k0 + r);
-        const float p = valid ? expf(s[j] * scale - sl[j]) : 0.f;
+      for (int j = 0; j < QH; ++j) {
+        const int c = QH * half + j, qrow = q0 + c;
+        const bool valid = r < nk && c < nq && !(qrow < own_end && qrow < k0 + r);
+        const float p = valid ? expf(s[j] * scale - sl[c]) : 0.f;
         s[j] = p;
-        dp[j] = p * (dp[j] - sd[j]);
+        dp[j] = p * (dp[j] - sd[c]);
       }
-#pragma unroll
-      for (int j = 0; j < QT; j += 16) {
-        put16<64, true>(sPh, sPl, r, j, s + j);
-        put16<64, true>(sDh, sDl, r, j, dp + j);
-      }
+      put16<64, true>(sPh, sPl, r, QH * half, s);
+      put16<64, true>(sDh, sDl, r, QH * half, dp);
     }
     const bool acc_on = !first;
     first = false;
@@ -530,7 +556,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   tc::cp_async_wait<0>();
   if (ok) {
-    for (int c = 0; c < DV; c += 32) {
+    for (int c = DV / 2 * half; c < DV / 2 * (half + 1); c += 32) {
       float g[32];
       tc::tmem_ld32(la + 128 + c, g);
       if (r >= 0 && r < nk) {
@@ -543,7 +569,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         st_out16(dst + 16, g + 16);
       }
     }
-    for (int c = 0; c < DQ; c += 32) {
+    for (int c = DQ / 2 * half; c < DQ / 2 * (half + 1); c += 32) {
       float g[32];
       tc::tmem_ld32(la + 256 + c, g);
       if (r >= 0 && r < nk) {

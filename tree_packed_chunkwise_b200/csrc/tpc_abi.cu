@@ -731,7 +731,7 @@ int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const v
     constexpr size_t smem = tpc::AttnFwdSmem<SP>::total;
     TPC_CUDA(set_smem(tpc::attn_fwd_tc<T, SP>, smem));
     TPC_LAUNCH("attn_fwd_tc", st,
-               (tpc::attn_fwd_tc<T, SP><<<grid, tpc::kAttnThreads, smem, st>>>(
+               (tpc::attn_fwd_tc<T, SP><<<grid, tpc::kAttnFwdThreads, smem, st>>>(
                    p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
                    (const bf*)L.v, (T*)o, lse, status)));
     return TPC_OK;
@@ -761,11 +761,11 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
     TPC_CUDA(set_smem(tpc::attn_bwd_dq_tc<T, SP>, sq));
     TPC_CUDA(set_smem(tpc::attn_bwd_dkv_tc<T, SP>, sk));
     TPC_LAUNCH("attn_bwd_dq_tc", st,
-               (tpc::attn_bwd_dq_tc<T, SP><<<gq, tpc::kAttnThreads, sq, st>>>(
+               (tpc::attn_bwd_dq_tc<T, SP><<<gq, tpc::kAttnDqThreads, sq, st>>>(
                    p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
                    (const bf*)L.v, (const T*)o, lse, (const bf*)d_o, (const bf*)L.d_o, (T*)dq, delta, status)));
     TPC_LAUNCH("attn_bwd_dkv_tc", st,
-               (tpc::attn_bwd_dkv_tc<T, SP><<<gk, tpc::kAttnThreads, sk, st>>>(
+               (tpc::attn_bwd_dkv_tc<T, SP><<<gk, tpc::kAttnDkvThreads, sk, st>>>(
                    p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
                    (const bf*)L.v, lse, (const bf*)d_o, (const bf*)L.d_o, delta, (T*)dk, (T*)dv, status)));
     return TPC_OK;
