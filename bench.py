@@ -600,7 +600,7 @@ def main():
         hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in res[0].items()}
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = sum(v.numel() * v.element_size() for v in hout.values())
-        copy = torch.cuda.Stream()
+        copy, down = torch.cuda.Stream(), torch.cuda.Stream()  # uploads and downloads (PCIe is duplex)
         ev = lambda: torch.cuda.Event()
 
         def run_one(x, r):
@@ -626,16 +626,22 @@ def main():
                 run_one(sets[b], res[b])
                 done[b] = ev()
                 done[b].record(stream)
-                with torch.cuda.stream(copy):
-                    copy.wait_event(done[b])
+                with torch.cuda.stream(down):
+                    down.wait_event(done[b])
                     for k in hout:
                         hout[k].copy_(res[b][k], non_blocking=True)
-                    if i + 2 < n:  # next use of set b: step i + 2
+                    drained = ev()
+                    drained.record(down)
+                if i + 2 < n:  # next use of set b: step i + 2, after its inputs are consumed and results read
+                    with torch.cuda.stream(copy):
+                        copy.wait_event(done[b])
+                        copy.wait_event(drained)
                         for k in host:
                             sets[b][k].copy_(host[k], non_blocking=True)
                         up[b] = ev()
                         up[b].record(copy)
             stream.wait_stream(copy)
+            stream.wait_stream(down)
 
         stream_steps(3)
         torch.cuda.synchronize()
@@ -649,8 +655,9 @@ def main():
         e2e = {"value": world * N / (ams / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ams,
                "how": "per step: H2D of all inputs from pinned host memory, forward + backward through the C ABI, "
-                      "D2H of all results; uploads and downloads run on a copy stream overlapping the "
-                      "neighbouring steps' compute (two device buffer sets); the timed region spans all copies"}
+                      "D2H of all results; uploads and downloads run on two copy streams overlapping each "
+                      "other and the neighbouring steps' compute (two device buffer sets); the timed region "
+                      "spans all copies"}
         del sets, res
 
     # ---- hybrid layer group on the agentic tree (KDA buffers released first)

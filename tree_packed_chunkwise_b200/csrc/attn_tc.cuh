@@ -349,26 +349,49 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
   const uint32_t tb = tslot;
   const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
   Sync sy{&bar, 0u, status};
-  bool first = true;
-  const bool ok = for_key_tiles<KT>(t, qt, [&](int k0, int nk, bool own) -> bool {
-    auto krows = [&](const bf* base, int width) {
-      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
+  // key tiles with one tile of look-ahead: V of the next tile is fetched by cp.async while this tile's
+  // dS and dQ products run, K of the next tile once this tile's dQ product has read K
+  auto load_k = [&](int k0, int nk) {
+    auto rows = [=](const bf* base) {
+      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * DQ : nullptr; };
     };
-    build_tile_ld<KT, DQ, false, bf, NT>(sK, nullptr, krows(k, DQ), ident);
-    build_tile_ld<KT, DV, false, bf, NT>(sV, nullptr, krows(v, DV), ident);
-    if constexpr (SPLIT) {
-      build_tile_ld<KT, DQ, false, bf, NT>(sKl, nullptr, krows(k_lo, DQ), ident);
-      build_tile_ld<KT, DV, false, bf, NT>(sVl, nullptr, krows(v_lo, DV), ident);
-    }
-    if (!run(sy, [&] {
-          mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
-               tc::Op{tc::smem_u32(sK), KT, false}, tc::Op{tc::smem_u32(sKl), KT, false}, DQ,
-               tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
-          mma4(tb + 64, tc::Op{tc::smem_u32(sO), 128, false}, tc::Op{tc::smem_u32(sOl), 128, false},
-               tc::Op{tc::smem_u32(sV), KT, false}, tc::Op{tc::smem_u32(sVl), KT, false}, DV,
-               tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
-        }))
-      return false;
+    tile_async<KT, DQ, NT>(sK, rows(k), k);
+    if constexpr (SPLIT) tile_async<KT, DQ, NT>(sKl, rows(k_lo), k);
+  };
+  auto load_v = [&](int k0, int nk) {
+    auto rows = [=](const bf* base) {
+      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * DV : nullptr; };
+    };
+    tile_async<KT, DV, NT>(sV, rows(v), v);
+    if constexpr (SPLIT) tile_async<KT, DV, NT>(sVl, rows(v_lo), v);
+  };
+  KeyTileIter<KT> it;
+  it.init(t, qt);
+  int k0 = 0, nk = 0;
+  bool own = false;
+  bool have = it.next(k0, nk, own);
+  if (have) {
+    load_k(k0, nk);
+    load_v(k0, nk);
+  }
+  tc::cp_async_commit();
+  bool first = true, ok = true;
+  while (have) {
+    int k1 = 0, n1 = 0;
+    bool own1 = false;
+    const bool more = it.next(k1, n1, own1);
+    tc::cp_async_wait<0>();  // this tile's K and V have arrived
+    ok = run(sy, [&] {
+      mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
+           tc::Op{tc::smem_u32(sK), KT, false}, tc::Op{tc::smem_u32(sKl), KT, false}, DQ,
+           tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
+      mma4(tb + 64, tc::Op{tc::smem_u32(sO), 128, false}, tc::Op{tc::smem_u32(sOl), 128, false},
+           tc::Op{tc::smem_u32(sV), KT, false}, tc::Op{tc::smem_u32(sVl), KT, false}, DV,
+           tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
+    });
+    if (!ok) break;
+    if (more) load_v(k1, n1);  // V is free once dP is in TMEM
+    tc::cp_async_commit();
     float s[KH], dp[KH];
 #pragma unroll
     for (int c = 0; c < KH; c += 16) {
@@ -386,16 +409,17 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
     for (int j = 0; j < KH; j += 16) put16<128, true>(sDh, sDl, row, KH * half + j, s + j);
     const bool acc_on = !first;
     first = false;
-    if (!run(sy, [&] {
-          mma4(tb + 128, tc::Op{tc::smem_u32(sDh), 128, false}, tc::Op{tc::smem_u32(sDl), 128, false},
-               tc::Op{tc::smem_u32(sK), KT, true}, tc::Op{tc::smem_u32(sKl), KT, true}, KT,
-               tc::idesc_bf16(128, DQ, false, true), acc_on, false, !SPLIT);
-        }))
-      return false;
-    tc::fence_before_sync();
-    __syncthreads();
-    return true;
-  });
+    ok = run(sy, [&] {
+      mma4(tb + 128, tc::Op{tc::smem_u32(sDh), 128, false}, tc::Op{tc::smem_u32(sDl), 128, false},
+           tc::Op{tc::smem_u32(sK), KT, true}, tc::Op{tc::smem_u32(sKl), KT, true}, KT,
+           tc::idesc_bf16(128, DQ, false, true), acc_on, false, !SPLIT);
+    });
+    if (!ok) break;
+    if (more) load_k(k1, n1);  // K is free once dQ has read it
+    tc::cp_async_commit();
+    k0 = k1; nk = n1; own = own1; have = more;
+  }
+  tc::cp_async_wait<0>();
   if (ok) {
     for (int c = 0; c < DQ / 2; c += 32) {
       float g[32];
