@@ -165,11 +165,11 @@ typedef struct tpc_kda_fwd_io {
  * recurrence (the chunk grid is aligned to trajectory positions).
  * Errors: TPC_ERR_NULL, TPC_ERR_STATE (plan not uploaded),
  * TPC_ERR_UNSUPPORTED, TPC_ERR_WORKSPACE, TPC_ERR_CUDA.
- * Streams: on the tensor-core path (chunk 64, d 128) each round's per-chunk output work runs on a
- * second, library-owned stream so that it overlaps the next round's sequential scan; that stream
- * is ordered after `stream` by an event and `stream` waits for it before the call's last work, so
- * everything is complete when work queued on `stream` after the call runs (stream capture sees
- * the fork and the join).  tpc_kda_backward does the same with its per-round gradient kernels.
+ * Streams: on the tensor-core path (chunk 64, d 128) the sequential state scans run on a
+ * library-owned high-priority stream, ordered against `stream` by events (one per round), so that
+ * the per-chunk kernels of neighbouring rounds on `stream` overlap them; `stream` waits for every
+ * scan before the call's last work, so everything is complete when work queued on `stream` after
+ * the call runs (stream capture sees the fork and the join).  tpc_kda_backward does the same.
  */
 int tpc_kda_forward(const tpc_plan* plan, const tpc_kda_shape* shape, const tpc_kda_fwd_io* io,
                     void* ws, size_t ws_bytes, tpc_stream_t stream);

@@ -395,12 +395,12 @@ struct PrepTcSmem {
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_prep_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
-                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, KdaWs ws) {
+                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, KdaWs ws, int chunk0 = 0) {
   using namespace tck;
   using S = PrepTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -656,12 +656,12 @@ struct BprepTcSmem {
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_bwd_prep_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
-                    const Tin* __restrict__ g_, const Tin* __restrict__ do_, KdaWs ws) {
+                    const Tin* __restrict__ g_, const Tin* __restrict__ do_, KdaWs ws, int chunk0 = 0) {
   using namespace tck;
   using S = BprepTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];

@@ -119,17 +119,22 @@ cudaError_t set_smem(KernelT k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-// A second stream per device for per-round work that may overlap the next round's sequential scan
-// (created once, non-blocking; ordered against the caller's stream by events).
-cudaStream_t side_stream() {
+// A high-priority stream per device for the sequential state scans (created once, non-blocking,
+// ordered against the caller's stream by events): the scans are the critical path of a step, so
+// when an SM frees up their CTAs go before the caller-stream chunk kernels that overlap them.
+cudaStream_t scan_stream() {
   static std::mutex mu;
   static std::vector<cudaStream_t> streams;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
   if ((int)streams.size() <= dev) streams.resize(dev + 1, nullptr);
-  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-    streams[dev] = nullptr;
+  if (!streams[dev]) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&streams[dev], cudaStreamNonBlocking, greatest) != cudaSuccess)
+      streams[dev] = nullptr;
+  }
   return streams[dev];
 }
 
@@ -162,36 +167,44 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
   const Tin* b = static_cast<const Tin*>(io->beta);
   // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
   constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  std::vector<cudaEvent_t> scans;
   if constexpr (kTensorCores) {
+    // Per round r: prep(r) and then out(r) on the caller's stream, scan(r) on the high-priority scan
+    // stream after prep(r) and scan(r - 1).  The caller's stream runs prep(1..R), out(1..R) in that
+    // order, so the later rounds' prep overlaps scan(1) and out(r) overlaps scan(r + 1).
     TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmem::total));
-    TPC_LAUNCH("kda_fwd_prep_tc", st,
-               (kda_fwd_prep_tc<Tin><<<dim3(nc, H), kThreads, PrepTcSmem::total, st>>>(p.dt, H, k, v, g, b, w)));
+    TPC_CUDA(set_smem(kda_scan_tc<false>, ScanTcSmem::total));
+    TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
+    cudaStream_t hs = scan_stream();
+    if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
+    for (int r = 1; r <= p.n_rounds; ++r) {
+      const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
+      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+      if (c1 > c0)
+        TPC_LAUNCH("kda_fwd_prep_tc", st,
+                   (kda_fwd_prep_tc<Tin><<<dim3(c1 - c0, H), kThreads, PrepTcSmem::total, st>>>(p.dt, H, k, v, g, b,
+                                                                                                  w, c0)));
+      TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
+      if (s1 > s0)
+        TPC_LAUNCH("kda_fwd_scan_tc", hs,
+                   (kda_scan_tc<false><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, hs>>>(
+                       p.dt, s0, H, io->init_state, io->final_state, nullptr, w)));
+      scans.emplace_back();
+      TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
+      TPC_CUDA(cudaEventRecord(scans.back(), hs));
+    }
+    for (int r = 1; r <= p.n_rounds; ++r) {
+      const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
+      TPC_CUDA(cudaStreamWaitEvent(st, scans[r - 1], 0));
+      TPC_CUDA(cudaEventDestroy(scans[r - 1]));
+      if (c1 > c0)
+        TPC_LAUNCH("kda_fwd_out_tc", st,
+                   (kda_fwd_out_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, OutTcSmem::total, st>>>(
+                       p.dt, H, q, k, g, static_cast<Tout*>(io->o), w, c0)));
+    }
   } else {
     TPC_LAUNCH("kda_fwd_prep", st,
                (kda_fwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, fwd_prep_smem<C, D>(), st>>>(p.dt, H, k, v, g, b, w)));
-  }
-  if constexpr (kTensorCores) {
-    // round r's output kernel (its chunks only) runs on a second stream while round r + 1 scans
-    TPC_CUDA(set_smem(kda_scan_tc<false>, ScanTcSmem::total));
-    TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
-    cudaStream_t side = side_stream();
-    if (!side) return fail(TPC_ERR_CUDA, "could not create the library's second stream");
-    for (int r = 1; r <= p.n_rounds; ++r) {
-      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-      const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
-      if (s1 > s0)
-        TPC_LAUNCH("kda_fwd_scan_tc", st,
-                   (kda_scan_tc<false><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
-                       p.dt, s0, H, io->init_state, io->final_state, nullptr, w)));
-      if (c1 > c0) {
-        TPC_TRY_ABI(stream_after(side, st));
-        TPC_LAUNCH("kda_fwd_out_tc", side,
-                   (kda_fwd_out_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, OutTcSmem::total, side>>>(
-                       p.dt, H, q, k, g, static_cast<Tout*>(io->o), w, c0)));
-      }
-    }
-    TPC_TRY_ABI(stream_after(st, side));
-  } else {
     for (int r = 1; r <= p.n_rounds; ++r) {
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       TPC_LAUNCH("kda_fwd_scan", st,
@@ -225,41 +238,51 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   const Tin* dO = static_cast<const Tin*>(io->d_o);
   // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
   constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  std::vector<cudaEvent_t> scans;
   if constexpr (kTensorCores) {
+    // Rounds in reverse: prep(r) on the caller's stream; the reverse scan(r) on the high-priority
+    // scan stream after prep(r) and scan(r + 1); then dq(r), dk/dv(r) on the caller's stream after
+    // scan(r).  The caller's stream runs prep(R..1), then dq / dk-dv(R..1), so the earlier rounds'
+    // prep overlaps scan(R) and dq / dk-dv(r) overlap scan(r - 1).
     TPC_CUDA(set_smem(kda_bwd_prep_tc<Tin>, BprepTcSmem::total));
-    TPC_LAUNCH("kda_bwd_prep_tc", st,
-               (kda_bwd_prep_tc<Tin><<<dim3(nc, H), kThreads, BprepTcSmem::total, st>>>(p.dt, H, q, k, g, dO, w)));
-  } else {
-    TPC_LAUNCH("kda_bwd_prep", st,
-               (kda_bwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, bprep_smem<C, D>(), st>>>(p.dt, H, q, k, g, dO, w)));
-  }
-  if constexpr (kTensorCores) {
-    // round r's chunk kernels (its chunks only) run on a second stream while round r - 1 scans
     TPC_CUDA(set_smem(kda_scan_tc<true>, ScanTcSmem::total));
     TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
     TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmemT<Tin>::total));
-    cudaStream_t side = side_stream();
-    if (!side) return fail(TPC_ERR_CUDA, "could not create the library's second stream");
+    cudaStream_t hs = scan_stream();
+    if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
     for (int r = p.n_rounds; r >= 1; --r) {
-      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
+      const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+      if (c1 > c0)
+        TPC_LAUNCH("kda_bwd_prep_tc", st,
+                   (kda_bwd_prep_tc<Tin><<<dim3(c1 - c0, H), kThreads, BprepTcSmem::total, st>>>(p.dt, H, q, k, g, dO,
+                                                                                                   w, c0)));
+      TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
       if (s1 > s0)
-        TPC_LAUNCH("kda_bwd_scan_tc", st,
-                   (kda_scan_tc<true><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, st>>>(
+        TPC_LAUNCH("kda_bwd_scan_tc", hs,
+                   (kda_scan_tc<true><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, hs>>>(
                        p.dt, s0, H, nullptr, nullptr, io->d_final, w)));
+      scans.emplace_back();
+      TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
+      TPC_CUDA(cudaEventRecord(scans.back(), hs));
+    }
+    for (int r = p.n_rounds, i = 0; r >= 1; --r, ++i) {
+      const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
+      TPC_CUDA(cudaStreamWaitEvent(st, scans[i], 0));
+      TPC_CUDA(cudaEventDestroy(scans[i]));
       if (c1 > c0) {
-        TPC_TRY_ABI(stream_after(side, st));
-        TPC_LAUNCH("kda_bwd_dq_tc", side,
-                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdqTcSmem::total, side>>>(
+        TPC_LAUNCH("kda_bwd_dq_tc", st,
+                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdqTcSmem::total, st>>>(
                        p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w, c0)));
-        TPC_LAUNCH("kda_bwd_dkv_tc", side,
-                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdkvTcSmemT<Tin>::total, side>>>(
+        TPC_LAUNCH("kda_bwd_dkv_tc", st,
+                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdkvTcSmemT<Tin>::total, st>>>(
                        p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg,
                        io->dbeta, w, c0)));
       }
     }
-    TPC_TRY_ABI(stream_after(st, side));
   } else {
+    TPC_LAUNCH("kda_bwd_prep", st,
+               (kda_bwd_prep<C, D, Tin><<<dim3(nc, H), kThreads, bprep_smem<C, D>(), st>>>(p.dt, H, q, k, g, dO, w)));
     for (int r = p.n_rounds; r >= 1; --r) {
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       TPC_LAUNCH("kda_bwd_scan", st,
