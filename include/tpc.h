@@ -332,7 +332,11 @@ int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int
 #define TPC_GROUP_MAX_KDA 8
 typedef struct tpc_group_shape {
   int32_t D, H, d_head, d_rope, d_latent;
-  int32_t n_kda; /* KDA layers before the MLA layer, 0..TPC_GROUP_MAX_KDA */
+  int32_t n_kda;         /* KDA layers before the MLA layer, 0..TPC_GROUP_MAX_KDA */
+  int32_t reuse_forward; /* backward only: 1 = the workspace still holds this group's forward on the
+                            same inputs (tpc_group_forward was the last call to use it); the last
+                            (MLA) layer, whose activations are then still resident, is not recomputed.
+                            0 = recompute every layer.  Results are bitwise the same either way. */
 } tpc_group_shape;
 typedef struct tpc_group_kda_weights { const void* w_in; const void* w_o; } tpc_group_kda_weights;
 typedef struct tpc_group_mla_weights { const void* w_a; const void* w_b; const void* w_o; } tpc_group_mla_weights;
@@ -362,7 +366,8 @@ int tpc_group_forward(const tpc_plan* plan, const tpc_group_shape* shape, const 
 /*
  * Backward of sum <dy, y>: recomputes every layer from its kept input (x, h), then runs its adjoint
  * in reverse layer order.  dy fp32 [N][D] (occurrence-summed upstream gradient per compact row);
- * dx fp32 [N][D] (may equal dy); weight gradients into g.  The workspace need not hold a forward.
+ * dx fp32 [N][D] (may equal dy); weight gradients into g.  The workspace need not hold a forward,
+ * unless shape->reuse_forward is set (see tpc_group_shape).
  */
 int tpc_group_backward(const tpc_plan* plan, const tpc_group_shape* shape, const tpc_group_weights* w,
                        const float* x, const float* h, const float* dy, float* dx, const tpc_group_grads* g,

@@ -51,3 +51,9 @@ def test_group_matches_oracle(tpc, tree_name, n_kda):
     # the backward is deterministic: a second run gives the same bits
     dx2, g2 = tpc.tpc_group_backward(plan, Wd, xd, h, dyd, ws)
     assert torch.equal(dx, dx2) and all(torch.equal(a, b) for a, b in zip(g["mla"], g2["mla"]))
+    # right after a forward the last layer need not be recomputed: the same bits
+    tpc.tpc_group_forward(plan, Wd, xd, ws)
+    dx3, g3 = tpc.tpc_group_backward(plan, Wd, xd, h, dyd, ws, reuse_forward=True)
+    assert torch.equal(dx, dx3)
+    assert all(torch.equal(a, b) for a, b in zip(g["mla"], g3["mla"]))
+    assert all(torch.equal(a, b) for p1, p2 in zip(g["kda"], g3["kda"]) for a, b in zip(p1, p2))

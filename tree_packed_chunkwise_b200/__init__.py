@@ -78,7 +78,7 @@ class AttnLo(ctypes.Structure):
 
 
 class GroupShape(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("D", "H", "d_head", "d_rope", "d_latent", "n_kda")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("D", "H", "d_head", "d_rope", "d_latent", "n_kda", "reuse_forward")]
 
 
 class GroupWeights(ctypes.Structure):
@@ -491,9 +491,9 @@ def tpc_rope_positions(plan: Plan, device="cuda", stream=None):
 GROUP_DIMS = {"D": 2048, "H": 16, "d_head": 128, "d_rope": 64, "d_latent": 512}
 
 
-def group_shape(n_kda: int = 3) -> GroupShape:
+def group_shape(n_kda: int = 3, reuse_forward: bool = False) -> GroupShape:
     d = GROUP_DIMS
-    return GroupShape(d["D"], d["H"], d["d_head"], d["d_rope"], d["d_latent"], n_kda)
+    return GroupShape(d["D"], d["H"], d["d_head"], d["d_rope"], d["d_latent"], n_kda, int(reuse_forward))
 
 
 def group_weight_shapes(n_kda: int = 3):
@@ -539,8 +539,10 @@ def tpc_group_forward(plan: Plan, weights, x, ws, h=None, y=None, stream=None):
     return y, h
 
 
-def tpc_group_backward(plan: Plan, weights, x, h, dy, ws, dx=None, grads=None, stream=None):
-    """Backward (with recomputation) of sum <dy, y>; returns (dx, grads) with fp32 weight gradients."""
+def tpc_group_backward(plan: Plan, weights, x, h, dy, ws, dx=None, grads=None, stream=None, reuse_forward=False):
+    """Backward (with recomputation) of sum <dy, y>; returns (dx, grads) with fp32 weight gradients.
+    reuse_forward: ws still holds tpc_group_forward's result on the same inputs (the last layer is then
+    not recomputed)."""
     import torch
     n_kda = len(weights["kda"])
     dx = dx if dx is not None else torch.empty_like(dy)
@@ -548,7 +550,7 @@ def tpc_group_backward(plan: Plan, weights, x, h, dy, ws, dx=None, grads=None, s
         grads = {"kda": [tuple(torch.empty(w.shape, dtype=torch.float32, device=x.device) for w in pair)
                          for pair in weights["kda"]],
                  "mla": tuple(torch.empty(w.shape, dtype=torch.float32, device=x.device) for w in weights["mla"])}
-    sh = group_shape(n_kda)
+    sh = group_shape(n_kda, reuse_forward)
     w = _group_ptrs(GroupWeights, weights)
     g = _group_ptrs(GroupGrads, grads)
     _check(lib().tpc_group_backward(plan.handle, ctypes.byref(sh), ctypes.byref(w), _ptr(x), _ptr(h), _ptr(dy),

@@ -211,11 +211,12 @@ int mla_layer_forward(const tpc_plan* plan, const tpc_group_mla_weights& w, cons
   return TPC_OK;
 }
 
+// resident: the workspace still holds this layer's forward (it was the last layer of the forward)
 int mla_layer_backward(const tpc_plan* plan, const tpc_group_mla_weights& w, const tpc_group_mla_grads& gr,
-                       const float* x, float* dx, Bufs& b, cudaStream_t st) {
+                       const float* x, float* dx, Bufs& b, bool resident, cudaStream_t st) {
   const int64_t N = plan->p.n_unique;
   const int rows = grid_rows(plan);
-  TPC_TRY(mla_layer_forward(plan, w, x, nullptr, b, st));  // recompute
+  if (!resident) TPC_TRY(mla_layer_forward(plan, w, x, nullptr, b, st));  // recompute
   TPC_TRY(split(dx, b.dy, N * kGrpD, st));
   TPC_TRY(gemm_aw(b.dy, w.w_o, b.dob, N, kGrpD, kGrpD, kGrpD, kGrpD, kGrpD, 1, 0.f, b.status, st));
   TPC_TRY(gemm_aa(b.dy, b.ob, gr.w_o, kGrpD, kGrpD, N, kGrpD, kGrpD, kGrpD, b.status, st));
@@ -299,7 +300,7 @@ int tpc_group_backward(const tpc_plan* plan, const tpc_group_shape* s, const tpc
   TPC_TRY(tpc_rope_positions(plan, b.pos, st));
   if (dx != dy) TPC_CUDA(cudaMemcpyAsync(dx, dy, ND * 4, cudaMemcpyDeviceToDevice, st));
   const float* mla_in = s->n_kda > 0 ? h + (s->n_kda - 1) * ND : x;
-  TPC_TRY(mla_layer_backward(plan, w->mla, g->mla, mla_in, dx, b, st));
+  TPC_TRY(mla_layer_backward(plan, w->mla, g->mla, mla_in, dx, b, s->reuse_forward != 0, st));
   for (int l = s->n_kda - 1; l >= 0; --l) {
     const float* in = l > 0 ? h + (l - 1) * ND : x;
     TPC_TRY(kda_layer_backward(plan, w->kda[l], g->kda[l], in, dx, b, st));
