@@ -439,28 +439,49 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------ backward dK, dV
-// per key tile of node u: query rows [row of the tile, subtree end of u) in tiles of 32 (queries of u
-// itself only from the key row on), S^T = K Q^T, dP^T = V dO^T, P^T = exp(scale S^T - lse),
-// dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 64 accumulators.
-// Q and dO tiles are double-buffered: the next query tile is fetched with cp.async while the current
-// one's P, dS and the dV / dK products run.
+// per key tile of node u (<= 64 rows): query rows [row of the tile, subtree end of u) in tiles of 32
+// (queries of u itself only from the key row on), S^T = K Q^T, dP^T = V dO^T, P^T = exp(scale S^T -
+// lse), dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 64 accumulators.
+//
+// Warp-specialised: warp 0 issues the MMAs, warps 1-3 stream the query tiles (Q, dO, their lo
+// parts, lse and delta) through a three-stage ring with cp.async, warps 4-11 turn S^T and dP^T into
+// P^T and dS^T.  S^T / dP^T have two TMEM buffers, so the products of query tile j + 1 run on the
+// tensor core while the P / dS math of tile j runs on the SIMT cores; the dV / dK products of tile j
+// follow once its P^T and dS^T are in shared memory.  Every wait is bounded; a timeout records
+// TPC_ERR_TIMEOUT and every role stops.
 template <bool SPLIT>
 struct AttnDkvSmem {
-  static constexpr int QT = 32;  // query rows per tile
+  static constexpr int QT = 32, NS = 3;  // query rows per tile, ring stages
   static constexpr size_t X = SPLIT ? 1 : 0;
   static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
   static constexpr size_t Qb = size_t(QT) * kAttnQK * 2, Ob = size_t(QT) * kAttnDV * 2, Pb = size_t(64) * QT * 2;
-  static constexpr size_t QO = (1 + X) * (Qb + Ob);  // one query buffer: Q (+lo), dO (+lo)
-  static constexpr size_t K = 0, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb, Qbuf = Vl + X * Vb;
-  static constexpr size_t P = Qbuf + 2 * QO, dS = P + 2 * Pb;
-  static constexpr size_t vec = dS + 2 * Pb;  // lse[QT], delta[QT] per buffer
-  static constexpr size_t total = vec + 2 * 2 * QT * 4;
+  // one ring stage: Q, Q_lo, dO, dO_lo, lse[QT], delta[QT]
+  static constexpr size_t sQ = 0, sQl = sQ + Qb, sO = sQl + X * Qb, sOl = sO + Ob, sL = sOl + X * Ob, sD = sL + QT * 4;
+  static constexpr size_t stage = sD + QT * 4;
+  static constexpr size_t K = 0, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb, ring = Vl + X * Vb;
+  static constexpr size_t P = ring + NS * stage, Pl = P + Pb, dS = Pl + Pb, dSl = dS + Pb;
+  static constexpr size_t total = dSl + Pb;
   static_assert(total <= 227 * 1024, "shared memory");
+  static_assert(stage % 128 == 0, "stage alignment");
 };
 
-// Eight warps: warps w and w + 4 share the key rows of TMEM sub-partition w % 4 (M = 64 layout:
-// lanes 0..15) and split the columns of every query tile and of dV / dK at the end.
-constexpr int kAttnDkvThreads = 256;
+constexpr int kAttnDkvThreads = 384;
+
+// Asynchronous load of an A x B bf16 tile (rows from rowp(a), nullptr = zeros) into the core-matrix
+// layout by NT threads (this one: t).  A warp moves 16 rows x 32 bytes (whole 32-byte sectors) and
+// writes four 128-byte lines of shared memory.  A, B multiples of 16.
+template <int A, int B, int NT, class RP>
+__device__ __forceinline__ void tile_async_t(uint8_t* dst, RP rowp, const void* any, int t) {
+  static_assert(A % 16 == 0 && B % 16 == 0, "tile shape");
+  constexpr int NCH = A * (B / 8), RB = A / 16;
+#pragma unroll 4
+  for (int e = t; e < NCH; e += NT) {
+    const int sub = e & 31, g = e >> 5;
+    const int a = 16 * (g % RB) + (sub >> 1), b0 = 8 * (2 * (g / RB) + (sub & 1));
+    const __nv_bfloat16* p = rowp(a);
+    tc::cp_async16(dst + tc::cm_off(a, b0, A), p ? (const void*)(p + b0) : any, p ? 16u : 0u);
+  }
+}
 
 template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnDkvThreads, 1)
@@ -471,143 +492,215 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
                     const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ d_o_lo,
                     const float* __restrict__ delta, Tio* __restrict__ dk, Tio* __restrict__ dv, int* status) {
   using namespace tck;
+  using namespace tc;
   using S = AttnDkvSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnDkvThreads, QT = S::QT, QH = QT / 2;
-  const AttnTile kt = t.attn_ktiles[blockIdx.x];
+  constexpr int DQ = kAttnQK, DV = kAttnDV, QT = S::QT, NS = S::NS, NP = 96;
+  // TMEM columns: dV (128), dK (192), then two buffers of S^T (32) and dP^T (32)
+  constexpr uint32_t cDV = 0, cDK = 128, cS = 320, cP = 352, cBuf = 64;
+  // grid: one block per (key tile, head), heads fastest; the planner lists the key tiles by
+  // decreasing work, so the longest blocks start first
+  const AttnTile kt = t.attn_ktiles[blockIdx.x / H];
+  const int h = blockIdx.x % H;
   const AttnNode nd = t.attn_nodes[kt.node];
-  const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int k0 = kt.row, nk = kt.n, own_end = nd.row_offset + nd.length, q_end = nd.subtree_end;
+  const int n_tiles = (q_end - k0 + QT - 1) / QT;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  uint8_t *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl;
-  uint8_t *sPh = asmem + S::P, *sPl = sPh + S::Pb, *sDh = asmem + S::dS, *sDl = sDh + S::Pb;
-  float* svec = reinterpret_cast<float*>(asmem + S::vec);  // [buffer][lse QT | delta QT]
-  // query buffer b: Q, Q_lo, dO, dO_lo
-  auto qbuf = [&](int b, int part) -> uint8_t* {
-    uint8_t* base = asmem + S::Qbuf + (size_t)b * S::QO;
-    return part == 0 ? base : part == 1 ? base + S::Qb : part == 2 ? base + (1 + S::X) * S::Qb
-                                                                   : base + (1 + S::X) * S::Qb + S::Ob;
-  };
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t full[NS], empty[NS], s_full[2], s_empty[2], p_full, p_empty, done_bar;
   __shared__ uint32_t tslot;
-  if (w == 0) tc::tmem_alloc(&tslot, 512);
+  __shared__ int abort_flag;
+  uint8_t *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl;
+  uint8_t *sPh = asmem + S::P, *sPl = asmem + S::Pl, *sDh = asmem + S::dS, *sDl = asmem + S::dSl;
+  auto stage = [&](int s) { return asmem + S::ring + (size_t)s * S::stage; };
+  if (w == 0) tmem_alloc(&tslot, 512);
   if (tid == 0) {
-    tc::mbar_init(&bar, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], NP);  // one arrival per loading thread once its copies have landed
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 8);  // one arrival per P / dS warp
+    }
+    mbar_init(&p_full, 8);
+    mbar_init(&p_empty, 1);
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const int k0 = kt.row, nk = kt.n;
-  auto krows = [&](const bf* base, int width) {
-    return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
-  };
-  tile_async<64, DQ, NT>(sK, krows(k, DQ), k);
-  tile_async<64, DV, NT>(sV, krows(v, DV), v);
-  if constexpr (SPLIT) {
-    tile_async<64, DQ, NT>(sKl, krows(k_lo, DQ), k);
-    tile_async<64, DV, NT>(sVl, krows(v_lo, DV), v);
-  }
-  const int own_end = nd.row_offset + nd.length, q_end = nd.subtree_end;
-  // query tile at row q0 into buffer b (rows past q_end are zero)
-  auto load_q = [&](int b, int q0) {
-    const int nq = min(QT, q_end - q0);
-    auto rows = [=](const bf* base, int width) {
-      return [=](int a) -> const bf* { return a < nq && base ? base + ((size_t)(q0 + a) * H + h) * width : nullptr; };
-    };
-    tile_async<QT, DQ, NT>(qbuf(b, 0), rows(q, DQ), q);
-    tile_async<QT, DV, NT>(qbuf(b, 2), rows(d_o, DV), d_o);
-    if constexpr (SPLIT) {
-      tile_async<QT, DQ, NT>(qbuf(b, 1), rows(q_lo, DQ), q);
-      tile_async<QT, DV, NT>(qbuf(b, 3), rows(d_o_lo, DV), d_o);
-    }
-  };
-  if (k0 < q_end) load_q(0, k0);
-  tc::cp_async_commit();  // group: K, V, query tile 0
   __syncthreads();
-  tc::fence_after_sync();
+  fence_after_sync();
   const uint32_t tb = tslot;
-  const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
-  const int r = lane < 16 ? 16 * (w & 3) + lane : -1;  // key row of this thread (M = 64 layout)
-  const int half = w >> 2;                                // column half of this warp
-  Sync sy{&bar, 0u, status};
-  bool ok = true, first = true;
-  int b = 0;
-  for (int q0 = k0; q0 < q_end && ok; q0 += QT, b ^= 1) {
-    const int nq = min(QT, q_end - q0);
-    const bool more = q0 + QT < q_end;
-    tc::cp_async_wait<0>();  // this query tile (and, the first time, K and V) have arrived
-    float* sl = svec + b * 2 * QT;
-    float* sd = sl + QT;
-    if (tid < QT) {
-      sl[tid] = tid < nq ? lse[(size_t)(q0 + tid) * H + h] : 0.f;
-      sd[tid] = tid < nq ? delta[(size_t)(q0 + tid) * H + h] : 0.f;
-    }
-    uint8_t *sQ = qbuf(b, 0), *sQl = qbuf(b, 1), *sO = qbuf(b, 2), *sOl = qbuf(b, 3);
-    ok = run(sy, [&] {
-      mma4(tb, tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sKl), 64, false},
-           tc::Op{tc::smem_u32(sQ), QT, false}, tc::Op{tc::smem_u32(sQl), QT, false}, DQ,
-           tc::idesc_bf16(64, QT, false, false), false, !SPLIT, !SPLIT);
-      mma4(tb + 64, tc::Op{tc::smem_u32(sV), 64, false}, tc::Op{tc::smem_u32(sVl), 64, false},
-           tc::Op{tc::smem_u32(sO), QT, false}, tc::Op{tc::smem_u32(sOl), QT, false}, DV,
-           tc::idesc_bf16(64, QT, false, false), false, !SPLIT, !SPLIT);
-    });
-    if (!ok) break;
-    // the other buffer was last read by the previous tile's dV / dK products, which have completed
-    if (more) load_q(b ^ 1, q0 + QT);
-    tc::cp_async_commit();
-    float s[QH], dp[QH];
-    tc::tmem_ld16(la + QH * half, *reinterpret_cast<float(*)[16]>(s));
-    tc::tmem_ld16(la + 64 + QH * half, *reinterpret_cast<float(*)[16]>(dp));
-    if (r >= 0) {
-#pragma unroll
-      for (int j = 0; j < QH; ++j) {
-        const int c = QH * half + j, qrow = q0 + c;
-        const bool valid = r < nk && c < nq && !(qrow < own_end && qrow < k0 + r);
-        const float p = valid ? expf(s[j] * scale - sl[c]) : 0.f;
-        s[j] = p;
-        dp[j] = p * (dp[j] - sd[c]);
-      }
-      put16<64, true>(sPh, sPl, r, QH * half, s);
-      put16<64, true>(sDh, sDl, r, QH * half, dp);
-    }
-    const bool acc_on = !first;
-    first = false;
-    ok = run(sy, [&] {
-      mma4(tb + 128, tc::Op{tc::smem_u32(sPh), 64, false}, tc::Op{tc::smem_u32(sPl), 64, false},
-           tc::Op{tc::smem_u32(sO), QT, true}, tc::Op{tc::smem_u32(sOl), QT, true}, QT,
-           tc::idesc_bf16(64, DV, false, true), acc_on, false, !SPLIT);
-      mma4(tb + 256, tc::Op{tc::smem_u32(sDh), 64, false}, tc::Op{tc::smem_u32(sDl), 64, false},
-           tc::Op{tc::smem_u32(sQ), QT, true}, tc::Op{tc::smem_u32(sQl), QT, true}, QT,
-           tc::idesc_bf16(64, DQ, false, true), acc_on, false, !SPLIT);
-    });
-  }
-  tc::cp_async_wait<0>();
-  if (ok) {
-    for (int c = DV / 2 * half; c < DV / 2 * (half + 1); c += 32) {
-      float g[32];
-      tc::tmem_ld32(la + 128 + c, g);
-      if (r >= 0 && r < nk) {
-        Tio* dst = dv + ((size_t)(k0 + r) * H + h) * DV + c;
-        if (first) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) g[j] = 0.f;
+  auto give_up = [&] {
+    set_status(status, kStatusTimeout);
+    atomicExch(&abort_flag, 1);
+  };
+  auto aborted = [&] { return *((volatile int*)&abort_flag) != 0; };
+
+  if (w == 0) {
+    if (lane == 0) {  // ------------------------------------------------ MMA issuer
+      const uint32_t id_s = idesc_bf16(64, QT, false, false);
+      const uint32_t id_dv = idesc_bf16(64, DV, false, true), id_dk = idesc_bf16(64, DQ, false, true);
+      for (int j = 0; j <= n_tiles && !aborted(); ++j) {
+        if (j < n_tiles) {  // S^T, dP^T of query tile j (stage j % NS also holds K, V before tile 0)
+          const int s = j % NS, b = j & 1;
+          if (!mbar_wait(&full[s], (j / NS) & 1) || (j >= 2 && !mbar_wait(&s_empty[b], ((j >> 1) - 1) & 1))) {
+            give_up();
+            break;
+          }
+          fence_after_sync();
+          uint8_t* st = stage(s);
+          mma4(tb + cS + cBuf * b, Op{smem_u32(sK), 64, false}, Op{smem_u32(sKl), 64, false},
+               Op{smem_u32(st + S::sQ), QT, false}, Op{smem_u32(st + S::sQl), QT, false}, DQ, id_s, false, !SPLIT,
+               !SPLIT);
+          mma4(tb + cP + cBuf * b, Op{smem_u32(sV), 64, false}, Op{smem_u32(sVl), 64, false},
+               Op{smem_u32(st + S::sO), QT, false}, Op{smem_u32(st + S::sOl), QT, false}, DV, id_s, false, !SPLIT,
+               !SPLIT);
+          commit(&s_full[b]);
         }
-        st_out16(dst, g);
-        st_out16(dst + 16, g + 16);
+        if (j >= 1) {  // dV, dK of query tile j - 1
+          const int jp = j - 1, s = jp % NS;
+          if (!mbar_wait(&p_full, jp & 1)) {
+            give_up();
+            break;
+          }
+          fence_after_sync();
+          uint8_t* st = stage(s);
+          mma4(tb + cDV, Op{smem_u32(sPh), 64, false}, Op{smem_u32(sPl), 64, false},
+               Op{smem_u32(st + S::sO), QT, true}, Op{smem_u32(st + S::sOl), QT, true}, QT, id_dv, jp > 0, false,
+               !SPLIT);
+          mma4(tb + cDK, Op{smem_u32(sDh), 64, false}, Op{smem_u32(sDl), 64, false},
+               Op{smem_u32(st + S::sQ), QT, true}, Op{smem_u32(st + S::sQl), QT, true}, QT, id_dk, jp > 0, false,
+               !SPLIT);
+          commit(&p_empty);   // P^T, dS^T may be overwritten
+          commit(&empty[s]);  // the stage may be refilled
+        }
+      }
+      commit(&done_bar);  // arrives once every MMA issued above has completed
+      if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
+    }
+  } else if (w < 4) {  // ------------------------------------------------ loads (96 threads)
+    const int p = tid - 32;
+    auto krows = [&](const bf* base, int width) {
+      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
+    };
+    int j = 0;
+    for (; j < n_tiles; ++j) {
+      const int s = j % NS;
+      if (j >= NS && !mbar_wait(&empty[s], ((j / NS) - 1) & 1)) {
+        give_up();
+        break;
+      }
+      if (aborted()) break;
+      if (j == 0) {  // K, V travel with the first query tile
+        tile_async_t<64, DQ, NP>(sK, krows(k, DQ), k, p);
+        tile_async_t<64, DV, NP>(sV, krows(v, DV), v, p);
+        if constexpr (SPLIT) {
+          tile_async_t<64, DQ, NP>(sKl, krows(k_lo, DQ), k, p);
+          tile_async_t<64, DV, NP>(sVl, krows(v_lo, DV), v, p);
+        }
+      }
+      const int q0 = k0 + j * QT, nq = min(QT, q_end - q0);
+      auto rows = [=](const bf* base, int width) {
+        return [=](int a) -> const bf* { return a < nq && base ? base + ((size_t)(q0 + a) * H + h) * width : nullptr; };
+      };
+      uint8_t* st = stage(s);
+      tile_async_t<QT, DQ, NP>(st + S::sQ, rows(q, DQ), q, p);
+      tile_async_t<QT, DV, NP>(st + S::sO, rows(d_o, DV), d_o, p);
+      if constexpr (SPLIT) {
+        tile_async_t<QT, DQ, NP>(st + S::sQl, rows(q_lo, DQ), q, p);
+        tile_async_t<QT, DV, NP>(st + S::sOl, rows(d_o_lo, DV), d_o, p);
+      }
+      if (p < 2 * QT) {
+        const int c = p % QT;
+        const float* src = (p < QT ? lse : delta) + (size_t)(q0 + min(c, nq - 1)) * H + h;
+        cp_async4(st + (p < QT ? S::sL : S::sD) + 4 * c, src, c < nq ? 4u : 0u);
+      }
+      cp_async_commit();
+      if (j >= 1) {  // the previous stage has landed: publish it to the tensor core and the P / dS warps
+        cp_async_wait<1>();
+        fence_async_smem();
+        mbar_arrive(&full[(j - 1) % NS]);
       }
     }
-    for (int c = DQ / 2 * half; c < DQ / 2 * (half + 1); c += 32) {
-      float g[32];
-      tc::tmem_ld32(la + 256 + c, g);
-      if (r >= 0 && r < nk) {
+    cp_async_wait<0>();
+    fence_async_smem();
+    if (j == n_tiles && n_tiles > 0) mbar_arrive(&full[(n_tiles - 1) % NS]);
+  } else {  // ------------------------------------------------ P^T, dS^T (warps 4-11)
+    const int sp = w & 3, half = (w - 4) >> 2;
+    const int r = lane < 16 ? 16 * sp + lane : -1;  // key row of this thread (M = 64 layout)
+    const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
+    bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar, parity));
+      if (!got && lane == 0) give_up();
+      return got && !__any_sync(0xffffffffu, aborted());
+    };
+    for (int j = 0; j < n_tiles; ++j) {
+      const int s = j % NS, b = j & 1;
+      if (!(ok = wait_all(&s_full[b], (j >> 1) & 1))) break;
+      fence_after_sync();
+      float sv[16], dp[16];
+      tmem_ld16(la + cS + cBuf * b + 16 * half, sv);
+      tmem_ld16(la + cP + cBuf * b + 16 * half, dp);
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[b]);
+      if (!(ok = wait_all(&full[s], (j / NS) & 1))) break;  // lse and delta of the tile
+      const uint8_t* st = stage(s);
+      const float* sl = reinterpret_cast<const float*>(st + S::sL);
+      const float* sd = reinterpret_cast<const float*>(st + S::sD);
+      const int q0 = k0 + j * QT, nq = min(QT, q_end - q0);
+      if (r >= 0) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) g[j] = first ? 0.f : g[j] * scale;
-        Tio* dst = dk + ((size_t)(k0 + r) * H + h) * DQ + c;
-        st_out16(dst, g);
-        st_out16(dst + 16, g + 16);
+        for (int jj = 0; jj < 16; ++jj) {
+          const int c = 16 * half + jj, qrow = q0 + c;
+          const bool valid = r < nk && c < nq && !(qrow < own_end && qrow < k0 + r);
+          const float pv = valid ? expf(sv[jj] * scale - sl[c]) : 0.f;
+          sv[jj] = pv;
+          dp[jj] = pv * (dp[jj] - sd[c]);
+        }
+      }
+      if (j >= 1 && !(ok = wait_all(&p_empty, (j - 1) & 1))) break;  // dV, dK of tile j - 1 are done
+      if (r >= 0) {
+        put16<64, true>(sPh, sPl, r, 16 * half, sv);
+        put16<64, true>(sDh, sDl, r, 16 * half, dp);
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full);
+    }
+    if (ok && n_tiles > 0) ok = wait_all(&p_empty, (n_tiles - 1) & 1);
+    if (ok) {
+      const bool none = n_tiles == 0;
+      for (int c = DV / 2 * half; c < DV / 2 * (half + 1); c += 32) {
+        float g[32];
+        tmem_ld32(la + cDV + c, g);
+        if (r >= 0 && r < nk) {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) g[jj] = none ? 0.f : g[jj];
+          Tio* dst = dv + ((size_t)(k0 + r) * H + h) * DV + c;
+          st_out16(dst, g);
+          st_out16(dst + 16, g + 16);
+        }
+      }
+      for (int c = DQ / 2 * half; c < DQ / 2 * (half + 1); c += 32) {
+        float g[32];
+        tmem_ld32(la + cDK + c, g);
+        if (r >= 0 && r < nk) {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) g[jj] = none ? 0.f : g[jj] * scale;
+          Tio* dst = dk + ((size_t)(k0 + r) * H + h) * DQ + c;
+          st_out16(dst, g);
+          st_out16(dst + 16, g + 16);
+        }
       }
     }
   }
-  tc::fence_before_sync();
+  fence_before_sync();
   __syncthreads();
-  if (w == 0) tc::tmem_dealloc(tb, 512);
+  if (w == 0) tmem_dealloc(tb, 512);
 }
 
 }  // namespace tpc
