@@ -102,24 +102,44 @@ __device__ __forceinline__ void tile_async(uint8_t* dst, RP rowp, const void* an
   }
 }
 
+// Asynchronous load of an A x B bf16 tile (rows from rowp(a), nullptr = zeros) into the core-matrix
+// layout by NT threads (this one: t).  A warp moves 16 rows x 32 bytes (whole 32-byte sectors) and
+// writes four 128-byte lines of shared memory.  A, B multiples of 16.
+template <int A, int B, int NT, class RP>
+__device__ __forceinline__ void tile_async_t(uint8_t* dst, RP rowp, const void* any, int t) {
+  static_assert(A % 16 == 0 && B % 16 == 0, "tile shape");
+  constexpr int NCH = A * (B / 8), RB = A / 16;
+#pragma unroll 4
+  for (int e = t; e < NCH; e += NT) {
+    const int sub = e & 31, g = e >> 5;
+    const int a = 16 * (g % RB) + (sub >> 1), b0 = 8 * (2 * (g / RB) + (sub & 1));
+    const __nv_bfloat16* p = rowp(a);
+    tc::cp_async16(dst + tc::cm_off(a, b0, A), p ? (const void*)(p + b0) : any, p ? 16u : 0u);
+  }
+}
+
+// Forward, per query tile (<= 128 rows of one node) and head, warp-specialised:
+//   warp 0      issues the MMAs: S_j = Q K_j^T into one of three TMEM buffers, then O += P_j V_j;
+//   warps 1-2   stream the key tiles K_j (and their lo parts) through a three-stage ring,
+//   warps 3-4   stream V_j through a two-stage ring (cp.async; a stage is published once landed);
+//   warps 5-12  two threads per query row (key columns split in halves): Q is loaded once into TMEM
+//               (the A operand of S), then per key tile the online softmax (base-2 exponentials of
+//               log2-scaled scores) reads S_j, writes P_j as a bf16 hi/lo pair back into the same
+//               TMEM columns (the A operand of P V), and keeps a reference maximum that is raised
+//               (O and l rescaled) only when a tile's maximum exceeds it by more than a factor e^8.
+// The products of tiles j + 1 and j + 2 run on the tensor core while the softmax of tile j runs.
 template <bool SPLIT>
 struct AttnFwdSmem {
-  static constexpr size_t Qb = size_t(128) * kAttnQK * 2, Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
-  static constexpr size_t Pb = size_t(128) * 64 * 2, X = SPLIT ? 1 : 0;
-  static constexpr size_t Q = 0, Ql = Q + Qb, K = Ql + X * Qb, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb;
-  static constexpr size_t P = Vl + X * Vb;
-  static constexpr size_t total = P + 2 * Pb;
+  static constexpr int NK = 3, NV = 2;
+  static constexpr size_t X = SPLIT ? 2 : 1;  // hi (and lo) parts
+  static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
+  static constexpr size_t Kst = X * Kb, Vst = X * Vb;  // one ring stage
+  static constexpr size_t K = 0, V = K + NK * Kst;
+  static constexpr size_t total = V + NV * Vst;
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
-// Per query tile: O accumulates in TMEM across the key tiles (P V products with accumulate), the
-// online softmax keeps a per-row reference maximum that is raised (and O, l rescaled) only when a
-// tile's maximum exceeds it by more than 8, so every p = exp(s - m) stays below e^8.  The next key
-// tile's K and V are fetched with cp.async while the current tile's softmax and P V run.  Eight
-// warps: warp w holds the TMEM lanes (query rows) of sub-partition w % 4 and the column half
-// w / 4 (S columns 32 h .. 32 h + 31, O columns 64 h .. 64 h + 63); the two threads of a row combine
-// their partial maxima and sums through shared memory, in a fixed order.
-constexpr int kAttnFwdThreads = 256;
+constexpr int kAttnFwdThreads = 416;
 
 template <typename Tout, bool SPLIT>
 __global__ void __launch_bounds__(kAttnFwdThreads, 1)
@@ -129,146 +149,281 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
                 const __nv_bfloat16* __restrict__ v_lo, Tout* __restrict__ o, float* __restrict__ lse,
                 int* status) {
   using namespace tck;
+  using namespace tc;
   using S = AttnFwdSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnFwdThreads;
-  constexpr float kRaise = 8.f;
-  const AttnTile qt = t.attn_qtiles[blockIdx.x];
-  const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int row = 32 * (w & 3) + lane, half = w >> 2;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NK = S::NK, NV = S::NV, NL = 64;  // NL threads per loader team
+  constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+  constexpr float kRaise2 = 8.f * kLog2e;  // raise threshold (e^8) in log2 units
+  // TMEM columns: Q hi (96), Q lo (96), O (128), three S / P buffers (64 each)
+  constexpr uint32_t cQh = 0, cQl = 96, cO = 192, cS = 320, cBuf = 64;
+  // grid: one block per (query tile, head), query tiles fastest, so that the blocks resident at one
+  // time read the same head's keys and values (shared in L2); the planner lists the query tiles of
+  // a head by decreasing work, so the longest blocks start first
+  const int n_qt = gridDim.x / H;
+  const AttnTile qt = t.attn_qtiles[blockIdx.x % n_qt];
+  const int h = blockIdx.x / n_qt;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  uint8_t *sQ = asmem + S::Q, *sQl = asmem + S::Ql, *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V,
-          *sVl = asmem + S::Vl, *sPh = asmem + S::P, *sPl = sPh + S::Pb;
-  __shared__ float red_max[2][128], red_sum[2][128];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], s_full[3], p_full[3], pv_done[3],
+      q_ready, done_bar;
   __shared__ uint32_t tslot;
-  if (w == 0) tc::tmem_alloc(&tslot, 256);
+  __shared__ int abort_flag;
+  __shared__ float red_sum[2][128];
+  auto kst = [&](int s) { return asmem + S::K + (size_t)s * S::Kst; };
+  auto vst = [&](int s) { return asmem + S::V + (size_t)s * S::Vst; };
+  if (w == 0) tmem_alloc(&tslot, 512);
   if (tid == 0) {
-    tc::mbar_init(&bar, 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(&kfull[s], NL);
+      mbar_init(&kempty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(&vfull[s], NL);
+      mbar_init(&vempty[s], 1);
+    }
+    for (int b = 0; b < 3; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 8);  // one arrival per softmax warp
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(&q_ready, 8);
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  auto qrows = [&](const bf* base) {
-    return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; };
-  };
-  auto load_kv = [&](bool is_k, int k0, int nk) {
-    if (is_k) {
-      tile_async<64, DQ, NT>(sK, [=](int a) -> const bf* { return a < nk ? k + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, k);
-      if constexpr (SPLIT)
-        tile_async<64, DQ, NT>(
-            sKl, [=](int a) -> const bf* { return a < nk && k_lo ? k_lo + ((size_t)(k0 + a) * H + h) * DQ : nullptr; }, k);
-    } else {
-      tile_async<64, DV, NT>(sV, [=](int a) -> const bf* { return a < nk ? v + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, v);
-      if constexpr (SPLIT)
-        tile_async<64, DV, NT>(
-            sVl, [=](int a) -> const bf* { return a < nk && v_lo ? v_lo + ((size_t)(k0 + a) * H + h) * DV : nullptr; }, v);
-    }
-  };
-  KeyTileIter<64> it;
-  it.init(t, qt);
-  int k0 = 0, nk = 0;
-  bool own = false;
-  bool have = it.next(k0, nk, own);
-  tile_async<128, DQ, NT>(sQ, qrows(q), q);
-  if constexpr (SPLIT) tile_async<128, DQ, NT>(sQl, qrows(q_lo), q);
-  if (have) load_kv(true, k0, nk);
-  tc::cp_async_commit();  // group: Q, K_0
-  if (have) load_kv(false, k0, nk);
-  tc::cp_async_commit();  // group: V_0
   __syncthreads();
-  tc::fence_after_sync();
+  fence_after_sync();
   const uint32_t tb = tslot;
-  const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
-  Sync sy{&bar, 0u, status};
-  const int qrow = qt.row + row;
-  float m_ref = -INFINITY, l = 0.f;
-  bool first = true, ok = true;
-  while (have) {
-    int k1 = 0, n1 = 0;
-    bool own1 = false;
-    const bool more = it.next(k1, n1, own1);
-    tc::cp_async_wait<1>();  // Q and this tile's K have arrived
-    ok = run(sy, [&] {
-      mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
-           tc::Op{tc::smem_u32(sK), 64, false}, tc::Op{tc::smem_u32(sKl), 64, false}, DQ,
-           tc::idesc_bf16(128, 64, false, false), false, !SPLIT, !SPLIT);
-    });
-    if (!ok) break;
-    if (more) load_kv(true, k1, n1);  // K is free once S is in TMEM
-    tc::cp_async_commit();
-    float s[32];
-    tc::tmem_ld32(la + 32 * half, s);
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int c = 32 * half + j;
-      const bool valid = row < qt.n && c < nk && (!own || k0 + c <= qrow);
-      s[j] = valid ? s[j] * scale : -INFINITY;
-      mx = fmaxf(mx, s[j]);
+  auto give_up = [&] {
+    set_status(status, kStatusTimeout);
+    atomicExch(&abort_flag, 1);
+  };
+  auto aborted = [&] { return *((volatile int*)&abort_flag) != 0; };
+  // number of key tiles of this query tile
+  int n_tiles = 0;
+  {
+    KeyTileIter<64> it;
+    it.init(t, qt);
+    int a, b;
+    bool c;
+    while (it.next(a, b, c)) ++n_tiles;
+  }
+
+  if (w == 0) {
+    if (lane == 0) {  // ------------------------------------------------ MMA issuer
+      const uint32_t id_s = idesc_bf16(128, 64, false, false), id_o = idesc_bf16(128, DV, false, true);
+      bool ok = mbar_wait(&q_ready, 0);
+      if (!ok) give_up();
+      for (int j = 0; ok && j <= n_tiles && !aborted(); ++j) {
+        if (j < n_tiles) {  // S_j = Q K_j^T
+          const int ks = j % NK, b = j % 3;
+          if (!mbar_wait(&kfull[ks], (j / NK) & 1) || (j >= 3 && !mbar_wait(&pv_done[b], ((j - 3) / 3) & 1))) {
+            give_up();
+            break;
+          }
+          fence_after_sync();
+          const uint32_t d = tb + cS + cBuf * b;
+          const Op kh{smem_u32(kst(ks)), 64, false}, kl{smem_u32(kst(ks) + S::Kb), 64, false};
+          for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQh + 8 * s, op_desc(kh, s), id_s, s ? 1u : 0u);
+          if constexpr (SPLIT) {
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQl + 8 * s, op_desc(kh, s), id_s, 1u);
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQh + 8 * s, op_desc(kl, s), id_s, 1u);
+          }
+          commit(&kempty[ks]);
+          commit(&s_full[b]);
+        }
+        if (j >= 1) {  // O += P_{j-1} V_{j-1}
+          const int jp = j - 1, b = jp % 3, vs = jp % NV;
+          if (!mbar_wait(&p_full[b], (jp / 3) & 1) || !mbar_wait(&vfull[vs], (jp / NV) & 1)) {
+            give_up();
+            break;
+          }
+          fence_after_sync();
+          const uint32_t ph = tb + cS + cBuf * b, pl = ph + 32;
+          const Op vh{smem_u32(vst(vs)), 64, true}, vl{smem_u32(vst(vs) + S::Vb), 64, true};
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, op_desc(vh, s), id_o, (jp > 0 || s) ? 1u : 0u);
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, pl + 8 * s, op_desc(vh, s), id_o, 1u);
+          if constexpr (SPLIT)
+            for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, op_desc(vl, s), id_o, 1u);
+          commit(&vempty[vs]);
+          commit(&pv_done[b]);
+        }
+      }
+      commit(&done_bar);  // arrives once every MMA issued above has completed
+      if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
     }
-    red_max[half][row] = mx;
-    __syncthreads();
-    mx = fmaxf(red_max[0][row], red_max[1][row]);
-    // raise the reference where the tile's maximum exceeds it by more than kRaise; O (accumulated so
-    // far) and l follow.  Both threads of a row take the same decision; TMEM loads and stores are
-    // warp-collective, so a warp rescales its 32 rows together when any of them raised.
-    const bool raise = mx > m_ref + kRaise;
-    const float corr = !raise ? 1.f : (m_ref == -INFINITY ? 0.f : expf(m_ref - mx));
-    if (raise) {
-      l *= corr;
-      m_ref = mx;
-    }
-    if (!first && __any_sync(0xffffffffu, raise)) {
-      for (int c = 0; c < DV / 2; c += 16) {
-        float ov[16];
-        tc::tmem_ld16(la + 64 + DV / 2 * half + c, ov);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ov[j] *= corr;
-        tc::tmem_st16(la + 64 + DV / 2 * half + c, ov);
+  } else if (w <= 4) {  // ------------------------------------------------ loader teams
+    const bool team_k = w <= 2;
+    const int p = tid - (team_k ? 32 : 96);
+    KeyTileIter<64> it;
+    it.init(t, qt);
+    int k0 = 0, nk = 0, j = 0;
+    bool own = false;
+    for (; it.next(k0, nk, own); ++j) {
+      const int NS = team_k ? NK : NV, s = j % NS;
+      if (j >= NS && !mbar_wait(team_k ? &kempty[s] : &vempty[s], ((j / NS) - 1) & 1)) {
+        give_up();
+        break;
+      }
+      if (aborted()) break;
+      auto rows = [=](const bf* base, int width) {
+        return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
+      };
+      if (team_k) {
+        tile_async_t<64, DQ, NL>(kst(s), rows(k, DQ), k, p);
+        if constexpr (SPLIT) tile_async_t<64, DQ, NL>(kst(s) + S::Kb, rows(k_lo, DQ), k, p);
+      } else {
+        tile_async_t<64, DV, NL>(vst(s), rows(v, DV), v, p);
+        if constexpr (SPLIT) tile_async_t<64, DV, NL>(vst(s) + S::Vb, rows(v_lo, DV), v, p);
+      }
+      cp_async_commit();
+      if (j >= 1) {  // the previous tile has landed: publish it
+        cp_async_wait<1>();
+        fence_async_smem();
+        mbar_arrive(team_k ? &kfull[(j - 1) % NK] : &vfull[(j - 1) % NV]);
       }
     }
-    float psum = 0.f;
+    cp_async_wait<0>();
+    fence_async_smem();
+    if (j == n_tiles && n_tiles > 0) mbar_arrive(team_k ? &kfull[(n_tiles - 1) % NK] : &vfull[(n_tiles - 1) % NV]);
+  } else {  // ------------------------------------------------ softmax (warps 5-12)
+    // warp w holds the TMEM lanes (query rows) of sub-partition w % 4 and the key columns of half
+    // (w - 5) / 4 for the exponentials; each thread reads the whole row of S for the row maximum, so
+    // the two threads of a row take the same decisions without exchanging data per key tile
+    const int sp = w & 3, half = (w - 5) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
+    const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
+    const float sl2 = scale * kLog2e;  // scores in log2 units: t = s scale log2(e)
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar, parity));
+      if (!got && lane == 0) give_up();
+      return got && !__any_sync(0xffffffffu, aborted());
+    };
+    // the two warps of a row pair meet once, after the last key tile (named barrier, 64 threads)
+    auto pair_sync = [&] { asm volatile("bar.sync %0, 64;" ::"r"(1 + sp) : "memory"); };
+    {  // this half of Q (and its lo part) into TMEM: a bf16 pair per 32-bit column, as in memory
+      const bool in = row < qt.n;
+      constexpr int HC = DQ / 4;  // 48 columns per half
+      for (int part = 0; part < (SPLIT ? 2 : 1); ++part) {
+        const bf* src = part ? q_lo : q;
+        const uint4* g4 = (in && src) ? reinterpret_cast<const uint4*>(src + ((size_t)qrow * H + h) * DQ) + HC / 4 * half
+                                      : nullptr;
+        for (int c0 = 0; c0 < HC; c0 += 16) {
+          float r[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      s[j] = s[j] == -INFINITY ? 0.f : expf(s[j] - m_ref);
-      psum += s[j];
-    }
-    red_sum[half][row] = psum;
-#pragma unroll
-    for (int j = 0; j < 32; j += 16) put16<128, true>(sPh, sPl, row, 32 * half + j, s + j);
-    __syncthreads();
-    l += red_sum[0][row] + red_sum[1][row];
-    tc::cp_async_wait<1>();  // this tile's V has arrived
-    const bool acc_on = !first;
-    ok = run(sy, [&] {
-      mma4(tb + 64, tc::Op{tc::smem_u32(sPh), 128, false}, tc::Op{tc::smem_u32(sPl), 128, false},
-           tc::Op{tc::smem_u32(sV), 64, true}, tc::Op{tc::smem_u32(sVl), 64, true}, 64,
-           tc::idesc_bf16(128, DV, false, true), acc_on, false, !SPLIT);
-    });
-    if (!ok) break;
-    if (more) load_kv(false, k1, n1);  // V is free once P V is done
-    tc::cp_async_commit();
-    first = false;
-    k0 = k1; nk = n1; own = own1; have = more;
-  }
-  tc::cp_async_wait<0>();
-  if (ok) {
-    const float inv = 1.f / l;
-    Tout* dst = o + ((size_t)qrow * H + h) * DV + DV / 2 * half;
-    for (int c = 0; c < DV / 2; c += 16) {
-      float ov[16];
-      tc::tmem_ld16(la + 64 + DV / 2 * half + c, ov);  // warp-collective: every row takes part
-      if (row < qt.n) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ov[j] *= inv;
-        st_out16(dst + c, ov);
+          for (int i = 0; i < 4; ++i) {
+            const uint4 x = g4 ? g4[c0 / 4 + i] : make_uint4(0u, 0u, 0u, 0u);
+            r[4 * i] = __uint_as_float(x.x); r[4 * i + 1] = __uint_as_float(x.y);
+            r[4 * i + 2] = __uint_as_float(x.z); r[4 * i + 3] = __uint_as_float(x.w);
+          }
+          tmem_st16(la + (part ? cQl : cQh) + HC * half + c0, r);
+        }
       }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_ready);
     }
-    if (row < qt.n && half == 0) lse[(size_t)qrow * H + h] = m_ref + logf(l);
+    KeyTileIter<64> it;
+    it.init(t, qt);
+    int k0 = 0, nk = 0;
+    bool own = false, ok = true;
+    float m_ref = -INFINITY, l = 0.f;  // m_ref in log2 units; l: this half's share of the row sum
+    for (int j = 0; j < n_tiles; ++j) {
+      it.next(k0, nk, own);
+      const int b = j % 3;
+      if (!(ok = wait_all(&s_full[b], (j / 3) & 1))) break;
+      fence_after_sync();
+      const uint32_t sb = la + cS + cBuf * b;
+      float tv[32], mx = -INFINITY;  // tv: this half's scores
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32_nowait(sb, r0);
+        tmem_ld32_nowait(sb + 32, r1);
+        tmem_wait_ld();
+        const bool masked = own || nk < 64;  // ragged key tile or the node's own (causal) rows
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float x0 = __uint_as_float(r0[c]) * sl2, x1 = __uint_as_float(r1[c]) * sl2;
+          if (masked) {
+            if (c >= nk || (own && k0 + c > qrow)) x0 = -INFINITY;
+            if (32 + c >= nk || (own && k0 + 32 + c > qrow)) x1 = -INFINITY;
+          }
+          mx = fmaxf(mx, fmaxf(x0, x1));
+          tv[c] = half ? x1 : x0;
+        }
+      }
+      // raise the reference where the tile's maximum exceeds it by more than kRaise; O (all tiles so
+      // far, so the previous P V must have completed) and l follow.  Both threads of a row take the
+      // same decision; TMEM loads and stores are warp-collective, so a warp rescales its 32 rows
+      // together when any of them raised.
+      const bool raise = mx > m_ref + kRaise2;
+      const float corr = !raise ? 1.f : (m_ref == -INFINITY ? 0.f : exp2f(m_ref - mx));
+      if (raise) {
+        l *= corr;
+        m_ref = mx;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        if (!(ok = wait_all(&pv_done[(j - 1) % 3], ((j - 1) / 3) & 1))) break;
+        fence_after_sync();
+        for (int c0 = 0; c0 < DV / 2; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32_nowait(la + cO + DV / 2 * half + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * corr);
+          tmem_st32_nowait(la + cO + DV / 2 * half + c0, r);
+        }
+        tmem_wait_st();
+      }
+      const float mb = m_ref == -INFINITY ? 0.f : m_ref;
+      float psum = 0.f;
+      float ph[16], pl[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        const float p0 = exp2f(tv[c] - mb), p1 = exp2f(tv[c + 1] - mb);
+        psum += p0 + p1;
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+        const float2 hf = __bfloat1622float2(hi);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+        ph[c / 2] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&hi));
+        pl[c / 2] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&lo));
+      }
+      l += psum;
+      // P hi in columns 0..31 of the buffer, lo in 32..63; this half's keys are 16 columns of each
+      tmem_st16(sb + 16 * half, ph);
+      tmem_st16(sb + 32 + 16 * half, pl);
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
+    }
+    if (ok && n_tiles > 0) ok = wait_all(&pv_done[(n_tiles - 1) % 3], ((n_tiles - 1) / 3) & 1);
+    red_sum[half][row] = l;
+    pair_sync();
+    if (ok) {
+      fence_after_sync();
+      const float lt = l + red_sum[half ^ 1][row];
+      const float inv = n_tiles > 0 ? 1.f / lt : 0.f;
+      Tout* dst = o + ((size_t)qrow * H + h) * DV + DV / 2 * half;
+      for (int c0 = 0; c0 < DV / 2; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32_nowait(la + cO + DV / 2 * half + c0, r);  // warp-collective: every row takes part
+        tmem_wait_ld();
+        if (row < qt.n) {
+          float ov[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = __uint_as_float(r[c]) * inv;
+          st_out16(dst + c0, ov);
+          st_out16(dst + c0 + 16, ov + 16);
+        }
+      }
+      if (row < qt.n && half == 0) lse[(size_t)qrow * H + h] = (m_ref + log2f(lt)) * kLn2;
+    }
   }
-  tc::fence_before_sync();
+  fence_before_sync();
   __syncthreads();
-  if (w == 0) tc::tmem_dealloc(tb, 256);
+  if (w == 0) tmem_dealloc(tb, 512);
 }
+
 
 // ------------------------------------------------------------------------------------------ backward dQ
 // per query tile: delta = rowsum(dO * O) (also written for the dK/dV kernel), then over the key
@@ -467,22 +622,6 @@ struct AttnDkvSmem {
 
 constexpr int kAttnDkvThreads = 384;
 
-// Asynchronous load of an A x B bf16 tile (rows from rowp(a), nullptr = zeros) into the core-matrix
-// layout by NT threads (this one: t).  A warp moves 16 rows x 32 bytes (whole 32-byte sectors) and
-// writes four 128-byte lines of shared memory.  A, B multiples of 16.
-template <int A, int B, int NT, class RP>
-__device__ __forceinline__ void tile_async_t(uint8_t* dst, RP rowp, const void* any, int t) {
-  static_assert(A % 16 == 0 && B % 16 == 0, "tile shape");
-  constexpr int NCH = A * (B / 8), RB = A / 16;
-#pragma unroll 4
-  for (int e = t; e < NCH; e += NT) {
-    const int sub = e & 31, g = e >> 5;
-    const int a = 16 * (g % RB) + (sub >> 1), b0 = 8 * (2 * (g / RB) + (sub & 1));
-    const __nv_bfloat16* p = rowp(a);
-    tc::cp_async16(dst + tc::cm_off(a, b0, A), p ? (const void*)(p + b0) : any, p ? 16u : 0u);
-  }
-}
-
 template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnDkvThreads, 1)
     attn_bwd_dkv_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
@@ -498,10 +637,12 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
   constexpr int DQ = kAttnQK, DV = kAttnDV, QT = S::QT, NS = S::NS, NP = 96;
   // TMEM columns: dV (128), dK (192), then two buffers of S^T (32) and dP^T (32)
   constexpr uint32_t cDV = 0, cDK = 128, cS = 320, cP = 352, cBuf = 64;
-  // grid: one block per (key tile, head), heads fastest; the planner lists the key tiles by
-  // decreasing work, so the longest blocks start first
-  const AttnTile kt = t.attn_ktiles[blockIdx.x / H];
-  const int h = blockIdx.x % H;
+  // grid: one block per (key tile, head), key tiles fastest, so that the blocks resident at one
+  // time read the same head's query rows (shared in L2); the planner lists the key tiles of a head
+  // by decreasing work, so the longest blocks start first
+  const int n_kt = gridDim.x / H;
+  const AttnTile kt = t.attn_ktiles[blockIdx.x % n_kt];
+  const int h = blockIdx.x / n_kt;
   const AttnNode nd = t.attn_nodes[kt.node];
   const int k0 = kt.row, nk = kt.n, own_end = nd.row_offset + nd.length, q_end = nd.subtree_end;
   const int n_tiles = (q_end - k0 + QT - 1) / QT;

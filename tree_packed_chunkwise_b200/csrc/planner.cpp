@@ -321,6 +321,12 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
         P.attn_ktiles.push_back({v, (int32_t)P.row_offset[v] + r, std::min(64, length[v] - r), 0});
     }
     P.attn_nodes[n] = AttnNode{0, 0, 0, (int32_t)(P.attn_ranges.size() / 2), 0, {0, 0, 0}};
+    // query tiles by decreasing work (the keys they read: the node's ancestor rows and its own rows up
+    // to the tile's end), so that the longest forward and dQ blocks start first; ties keep node order
+    std::stable_sort(P.attn_qtiles.begin(), P.attn_qtiles.end(), [&](const AttnTile& a, const AttnTile& b) {
+      const AttnNode &na = P.attn_nodes[a.node], &nb = P.attn_nodes[b.node];
+      return na.pos0 + (a.row - na.row_offset) + a.n > nb.pos0 + (b.row - nb.row_offset) + b.n;
+    });
     // key tiles by decreasing work (the query rows that read them: the subtree from the tile on), so
     // that the dK / dV blocks with the longest query ranges start first; ties keep node order
     std::stable_sort(P.attn_ktiles.begin(), P.attn_ktiles.end(), [&](const AttnTile& a, const AttnTile& b) {

@@ -746,7 +746,7 @@ int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const v
   const bool split = L.q || L.k || L.v;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const tpc::Plan& p = plan->p;
-  const dim3 grid((unsigned)p.attn_qtiles.size(), (unsigned)s->H);
+  const dim3 grid((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest
   using bf = __nv_bfloat16;
   auto go = [&](auto tout, auto split) -> int {
     using T = decltype(tout);
@@ -777,7 +777,7 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
   const tpc::Plan& p = plan->p;
   using bf = __nv_bfloat16;
   const dim3 gq((unsigned)p.attn_qtiles.size(), (unsigned)s->H);
-  const dim3 gk((unsigned)(p.attn_ktiles.size() * (size_t)s->H));  // (key tile, head), heads fastest
+  const dim3 gk((unsigned)(p.attn_ktiles.size() * (size_t)s->H));  // (key tile, head), key tiles fastest
   auto go = [&](auto tio, auto split) -> int {
     using T = decltype(tio);
     constexpr bool SP = decltype(split)::value;
