@@ -119,15 +119,16 @@ __device__ __forceinline__ void tile_async_t(uint8_t* dst, RP rowp, const void* 
 }
 
 // Forward, per query tile (<= 128 rows of one node) and head, warp-specialised:
-//   warp 0      issues the MMAs: S_j = Q K_j^T into one of three TMEM buffers, then O += P_j V_j;
+//   warp 0      issues the MMAs: S_j = Q K_j^T into one of two TMEM buffers, then O += P_j V_j;
 //   warps 1-2   stream the key tiles K_j (and their lo parts) through a three-stage ring,
 //   warps 3-4   stream V_j through a two-stage ring (cp.async; a stage is published once landed);
 //   warps 5-12  two threads per query row (key columns split in halves): Q is loaded once into TMEM
 //               (the A operand of S), then per key tile the online softmax (base-2 exponentials of
-//               log2-scaled scores) reads S_j, writes P_j as a bf16 hi/lo pair back into the same
-//               TMEM columns (the A operand of P V), and keeps a reference maximum that is raised
-//               (O and l rescaled) only when a tile's maximum exceeds it by more than a factor e^8.
-// The products of tiles j + 1 and j + 2 run on the tensor core while the softmax of tile j runs.
+//               log2-scaled scores) reads S_j (releasing its buffer), writes P_j as a bf16 hi/lo
+//               pair into a TMEM buffer of its own (the A operand of P V) once P_{j-1} V_{j-1} has
+//               completed, and keeps a reference maximum that is raised (O and l rescaled) only when
+//               a tile's maximum exceeds it by more than a factor e^8.
+// S_{j+1} and P_{j-1} V_{j-1} run on the tensor core while the softmax of tile j runs.
 template <bool SPLIT>
 struct AttnFwdSmem {
   static constexpr int NK = 3, NV = 2;
@@ -155,8 +156,8 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   constexpr int DQ = kAttnQK, DV = kAttnDV, NK = S::NK, NV = S::NV, NL = 64;  // NL threads per loader team
   constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
   constexpr float kRaise2 = 8.f * kLog2e;  // raise threshold (e^8) in log2 units
-  // TMEM columns: Q hi (96), Q lo (96), O (128), three S / P buffers (64 each)
-  constexpr uint32_t cQh = 0, cQl = 96, cO = 192, cS = 320, cBuf = 64;
+  // TMEM columns: Q hi (96), Q lo (96), O (128), two S buffers (64 each), P hi (32) and lo (32)
+  constexpr uint32_t cQh = 0, cQl = 96, cO = 192, cS = 320, cBuf = 64, cP = 448;
   // grid: one block per (query tile, head), query tiles fastest, so that the blocks resident at one
   // time read the same head's keys and values (shared in L2); the planner lists the query tiles of
   // a head by decreasing work, so the longest blocks start first
@@ -165,8 +166,8 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   const int h = blockIdx.x / n_qt;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  __shared__ __align__(8) uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], s_full[3], p_full[3], pv_done[3],
-      q_ready, done_bar;
+  __shared__ __align__(8) uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], s_full[2], s_read[2], p_full,
+      pv_done, q_ready, done_bar;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
   __shared__ float red_sum[2][128];
@@ -182,11 +183,12 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       mbar_init(&vfull[s], NL);
       mbar_init(&vempty[s], 1);
     }
-    for (int b = 0; b < 3; ++b) {
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 8);  // one arrival per softmax warp
-      mbar_init(&pv_done[b], 1);
+      mbar_init(&s_read[b], 8);  // one arrival per softmax warp
     }
+    mbar_init(&p_full, 8);
+    mbar_init(&pv_done, 1);
     mbar_init(&q_ready, 8);
     mbar_init(&done_bar, 1);
     abort_flag = 0;
@@ -217,8 +219,8 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       if (!ok) give_up();
       for (int j = 0; ok && j <= n_tiles && !aborted(); ++j) {
         if (j < n_tiles) {  // S_j = Q K_j^T
-          const int ks = j % NK, b = j % 3;
-          if (!mbar_wait(&kfull[ks], (j / NK) & 1) || (j >= 3 && !mbar_wait(&pv_done[b], ((j - 3) / 3) & 1))) {
+          const int ks = j % NK, b = j & 1;
+          if (!mbar_wait(&kfull[ks], (j / NK) & 1) || (j >= 2 && !mbar_wait(&s_read[b], ((j >> 1) - 1) & 1))) {
             give_up();
             break;
           }
@@ -234,20 +236,20 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
           commit(&s_full[b]);
         }
         if (j >= 1) {  // O += P_{j-1} V_{j-1}
-          const int jp = j - 1, b = jp % 3, vs = jp % NV;
-          if (!mbar_wait(&p_full[b], (jp / 3) & 1) || !mbar_wait(&vfull[vs], (jp / NV) & 1)) {
+          const int jp = j - 1, vs = jp % NV;
+          if (!mbar_wait(&p_full, jp & 1) || !mbar_wait(&vfull[vs], (jp / NV) & 1)) {
             give_up();
             break;
           }
           fence_after_sync();
-          const uint32_t ph = tb + cS + cBuf * b, pl = ph + 32;
+          const uint32_t ph = tb + cP, pl = ph + 32;
           const Op vh{smem_u32(vst(vs)), 64, true}, vl{smem_u32(vst(vs) + S::Vb), 64, true};
           for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, op_desc(vh, s), id_o, (jp > 0 || s) ? 1u : 0u);
           for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, pl + 8 * s, op_desc(vh, s), id_o, 1u);
           if constexpr (SPLIT)
             for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, op_desc(vl, s), id_o, 1u);
           commit(&vempty[vs]);
-          commit(&pv_done[b]);
+          commit(&pv_done);
         }
       }
       commit(&done_bar);  // arrives once every MMA issued above has completed
@@ -277,16 +279,13 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
         tile_async_t<64, DV, NL>(vst(s), rows(v, DV), v, p);
         if constexpr (SPLIT) tile_async_t<64, DV, NL>(vst(s) + S::Vb, rows(v_lo, DV), v, p);
       }
+      // publish the tile as soon as it has landed (the writes are made visible to the tensor core)
       cp_async_commit();
-      if (j >= 1) {  // the previous tile has landed: publish it
-        cp_async_wait<1>();
-        fence_async_smem();
-        mbar_arrive(team_k ? &kfull[(j - 1) % NK] : &vfull[(j - 1) % NV]);
-      }
+      cp_async_wait<0>();
+      fence_async_smem();
+      mbar_arrive(team_k ? &kfull[s] : &vfull[s]);
     }
     cp_async_wait<0>();
-    fence_async_smem();
-    if (j == n_tiles && n_tiles > 0) mbar_arrive(team_k ? &kfull[(n_tiles - 1) % NK] : &vfull[(n_tiles - 1) % NV]);
   } else {  // ------------------------------------------------ softmax (warps 5-12)
     // warp w holds the TMEM lanes (query rows) of sub-partition w % 4 and the key columns of half
     // (w - 5) / 4 for the exponentials; each thread reads the whole row of S for the row maximum, so
@@ -330,8 +329,8 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
     float m_ref = -INFINITY, l = 0.f;  // m_ref in log2 units; l: this half's share of the row sum
     for (int j = 0; j < n_tiles; ++j) {
       it.next(k0, nk, own);
-      const int b = j % 3;
-      if (!(ok = wait_all(&s_full[b], (j / 3) & 1))) break;
+      const int b = j & 1;
+      if (!(ok = wait_all(&s_full[b], (j >> 1) & 1))) break;
       fence_after_sync();
       const uint32_t sb = la + cS + cBuf * b;
       float tv[32], mx = -INFINITY;  // tv: this half's scores
@@ -340,6 +339,9 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
         tmem_ld32_nowait(sb, r0);
         tmem_ld32_nowait(sb + 32, r1);
         tmem_wait_ld();
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_read[b]);  // the buffer may take S_{j+2}
         const bool masked = own || nk < 64;  // ragged key tile or the node's own (causal) rows
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -362,9 +364,12 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
         l *= corr;
         m_ref = mx;
       }
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {
-        if (!(ok = wait_all(&pv_done[(j - 1) % 3], ((j - 1) / 3) & 1))) break;
+      // P_{j-1} V_{j-1} has completed: O is final up to tile j - 1 and the P buffer is free
+      if (j > 0) {
+        if (!(ok = wait_all(&pv_done, (j - 1) & 1))) break;
         fence_after_sync();
+      }
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
         for (int c0 = 0; c0 < DV / 2; c0 += 32) {
           uint32_t r[32];
           tmem_ld32_nowait(la + cO + DV / 2 * half + c0, r);
@@ -389,14 +394,14 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
         pl[c / 2] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&lo));
       }
       l += psum;
-      // P hi in columns 0..31 of the buffer, lo in 32..63; this half's keys are 16 columns of each
-      tmem_st16(sb + 16 * half, ph);
-      tmem_st16(sb + 32 + 16 * half, pl);
+      // P hi in columns 0..31 of its buffer, lo in 32..63; this half's keys are 16 columns of each
+      tmem_st16(la + cP + 16 * half, ph);
+      tmem_st16(la + cP + 32 + 16 * half, pl);
       fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[b]);
+      if (lane == 0) mbar_arrive(&p_full);
     }
-    if (ok && n_tiles > 0) ok = wait_all(&pv_done[(n_tiles - 1) % 3], ((n_tiles - 1) / 3) & 1);
+    if (ok && n_tiles > 0) ok = wait_all(&pv_done, (n_tiles - 1) & 1);
     red_sum[half][row] = l;
     pair_sync();
     if (ok) {
@@ -426,23 +431,25 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
 
 
 // ------------------------------------------------------------------------------------------ backward dQ
-// per query tile: delta = rowsum(dO * O) (also written for the dK/dV kernel), then over the key
-// tiles P = exp(scale S - lse), dP = dO V^T, dS = P (dP - delta), dQ += dS K; dq = scale dQ.
+// per query tile (<= 128 rows of one node) and head: delta = rowsum(dO * O) (also written for the
+// dK/dV kernel), then over the key tiles P = exp(scale S - lse), dP = dO V^T, dS = P (dP - delta),
+// dQ += dS K; dq = scale dQ.  Warp-specialised like the forward:
+//   warp 0      issues S_j = Q K_j^T, then dQ += dS_{j-1} K_{j-1}, then dP_j = dO V_j^T;
+//   warps 1-2   stream K_j through a two-stage ring; warps 3-4 load dO once, then stream V_j;
+//   warps 5-12  two threads per query row (key columns in halves): Q into TMEM once, delta; per key
+//               tile they read S_j (releasing it for S_{j+1}) and dP_j, and write dS_j as a bf16
+//               hi/lo pair over their own dP_j columns (the A operand of the dQ product).
 template <bool SPLIT>
 struct AttnDqSmem {
-  static constexpr int KT = SPLIT ? 32 : 64;  // key rows per tile
-  static constexpr size_t X = SPLIT ? 1 : 0;
-  static constexpr size_t Qb = size_t(128) * kAttnQK * 2, Ob = size_t(128) * kAttnDV * 2;
-  static constexpr size_t Kb = size_t(KT) * kAttnQK * 2, Vb = size_t(KT) * kAttnDV * 2, Pb = size_t(128) * KT * 2;
-  static constexpr size_t Q = 0, Ql = Q + Qb, dO = Ql + X * Qb, dOl = dO + Ob, K = dOl + X * Ob, Kl = K + Kb;
-  static constexpr size_t V = Kl + X * Kb, Vl = V + Vb, dS = Vl + X * Vb;
-  static constexpr size_t total = dS + 2 * Pb;
+  static constexpr int NK = 2, NV = 2;
+  static constexpr size_t X = SPLIT ? 2 : 1;
+  static constexpr size_t Ob = size_t(128) * kAttnDV * 2, Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
+  static constexpr size_t dO = 0, K = dO + X * Ob, V = K + NK * X * Kb;
+  static constexpr size_t total = V + NV * X * Vb;
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
-// Eight warps: warp w holds the query rows of TMEM sub-partition w % 4 and the column half w / 4 of
-// each key tile (and of dQ at the end).
-constexpr int kAttnDqThreads = 256;
+constexpr int kAttnDqThreads = 416;
 
 template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnDqThreads, 1)
@@ -453,144 +460,262 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
                    const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ d_o_lo,
                    Tio* __restrict__ dq, float* __restrict__ delta, int* status) {
   using namespace tck;
+  using namespace tc;
   using S = AttnDqSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NT = kAttnDqThreads, KT = S::KT, KH = KT / 2;
-  const AttnTile qt = t.attn_qtiles[blockIdx.x];
-  const int h = blockIdx.y, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int row = 32 * (w & 3) + lane, half = w >> 2;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NK = S::NK, NV = S::NV, NL = 64;
+  constexpr float kLog2e = 1.4426950408889634f;
+  // TMEM columns: Q hi (96), Q lo (96), dQ (192), S (64), dP / dS (64)
+  constexpr uint32_t cQh = 0, cQl = 96, cG = 192, cS = 384, cP = 448;
+  // grid: one block per (query tile, head), query tiles fastest (see the forward)
+  const int n_qt = gridDim.x / H;
+  const AttnTile qt = t.attn_qtiles[blockIdx.x % n_qt];
+  const int h = blockIdx.x / n_qt;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(1024) uint8_t asmem[];
-  uint8_t *sQ = asmem + S::Q, *sQl = asmem + S::Ql, *sO = asmem + S::dO, *sOl = asmem + S::dOl, *sK = asmem + S::K,
-          *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl, *sDh = asmem + S::dS, *sDl = sDh + S::Pb;
-  __shared__ float s_dl[128], s_ls[128];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], do_full, q_ready, s_full, s_read,
+      dp_full, ds_full, dq_done, done_bar;
   __shared__ uint32_t tslot;
-  if (w == 0) tc::tmem_alloc(&tslot, 512);
+  __shared__ int abort_flag;
+  uint8_t* sO = asmem + S::dO;
+  auto kst = [&](int s) { return asmem + S::K + (size_t)s * S::X * S::Kb; };
+  auto vst = [&](int s) { return asmem + S::V + (size_t)s * S::X * S::Vb; };
+  if (w == 0) tmem_alloc(&tslot, 512);
   if (tid == 0) {
-    tc::mbar_init(&bar, 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(&kfull[s], NL);
+      mbar_init(&kempty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(&vfull[s], NL);
+      mbar_init(&vempty[s], 1);
+    }
+    mbar_init(&do_full, NL);
+    mbar_init(&q_ready, 8);  // one arrival per softmax warp
+    mbar_init(&s_full, 1);
+    mbar_init(&s_read, 8);
+    mbar_init(&dp_full, 1);
+    mbar_init(&ds_full, 8);
+    mbar_init(&dq_done, 1);
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  auto ident = [](int, int, float x) { return x; };
-  auto qrows = [&](const bf* base) {
-    return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DQ : nullptr; };
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = tslot;
+  auto give_up = [&] {
+    set_status(status, kStatusTimeout);
+    atomicExch(&abort_flag, 1);
   };
-  auto orows = [&](const bf* base) {
-    return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DV : nullptr; };
-  };
-  build_tile_ld<128, DQ, false, bf, NT>(sQ, nullptr, qrows(q), ident);
-  build_tile_ld<128, DV, false, bf, NT>(sO, nullptr, orows(d_o), ident);
-  if constexpr (SPLIT) {
-    build_tile_ld<128, DQ, false, bf, NT>(sQl, nullptr, qrows(q_lo), ident);
-    build_tile_ld<128, DV, false, bf, NT>(sOl, nullptr, orows(d_o_lo), ident);
+  auto aborted = [&] { return *((volatile int*)&abort_flag) != 0; };
+  int n_tiles = 0;
+  {
+    KeyTileIter<64> it;
+    it.init(t, qt);
+    int a, b;
+    bool c;
+    while (it.next(a, b, c)) ++n_tiles;
   }
-  const int qrow = qt.row + row;
-  if (half == 0) {
-    float dl = 0.f, ls = 0.f;
-    if (row < qt.n) {
+
+  if (w == 0) {
+    if (lane == 0) {  // ------------------------------------------------ MMA issuer
+      const uint32_t id_s = idesc_bf16(128, 64, false, false), id_g = idesc_bf16(128, DQ, false, true);
+      bool ok = mbar_wait(&q_ready, 0) && mbar_wait(&do_full, 0);
+      if (!ok) give_up();
+      const Op oh{smem_u32(sO), 128, false}, ol{smem_u32(sO + S::Ob), 128, false};
+      for (int j = 0; ok && j <= n_tiles && !aborted(); ++j) {
+        if (j < n_tiles) {  // S_j = Q K_j^T, once the softmax warps have read S_{j-1}
+          const int ks = j % NK;
+          if (!mbar_wait(&kfull[ks], (j / NK) & 1) || (j >= 1 && !mbar_wait(&s_read, (j - 1) & 1))) {
+            give_up();
+            break;
+          }
+          fence_after_sync();
+          const Op kh{smem_u32(kst(ks)), 64, false}, kl{smem_u32(kst(ks) + S::Kb), 64, false};
+          for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQh + 8 * s, op_desc(kh, s), id_s, s ? 1u : 0u);
+          if constexpr (SPLIT) {
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQl + 8 * s, op_desc(kh, s), id_s, 1u);
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQh + 8 * s, op_desc(kl, s), id_s, 1u);
+          }
+          commit(&s_full);
+        }
+        if (j >= 1) {  // dQ += dS_{j-1} K_{j-1}: dS in the dP columns, hi / lo in each half's 32 columns
+          const int jp = j - 1, ks = jp % NK;
+          if (!mbar_wait(&ds_full, jp & 1)) {
+            give_up();
+            break;
+          }
+          fence_after_sync();
+          const Op kh{smem_u32(kst(ks)), 64, true}, kl{smem_u32(kst(ks) + S::Kb), 64, true};
+          auto a_hi = [&](int s) { return tb + cP + 32 * (s >> 1) + 8 * (s & 1); };
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), op_desc(kh, s), id_g, (jp > 0 || s) ? 1u : 0u);
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s) + 16, op_desc(kh, s), id_g, 1u);
+          if constexpr (SPLIT)
+            for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), op_desc(kl, s), id_g, 1u);
+          commit(&kempty[ks]);
+          commit(&dq_done);
+        }
+        if (j < n_tiles) {  // dP_j = dO V_j^T, once dQ has read dS_{j-1} from the same columns
+          const int vs = j % NV;
+          if (!mbar_wait(&vfull[vs], (j / NV) & 1) || (j >= 1 && !mbar_wait(&dq_done, (j - 1) & 1))) {
+            give_up();
+            break;
+          }
+          fence_after_sync();
+          const Op vh{smem_u32(vst(vs)), 64, false}, vl{smem_u32(vst(vs) + S::Vb), 64, false};
+          mma4(tb + cP, oh, ol, vh, vl, DV, id_s, false, !SPLIT, !SPLIT);
+          commit(&vempty[vs]);
+          commit(&dp_full);
+        }
+      }
+      commit(&done_bar);  // arrives once every MMA issued above has completed
+      if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
+    }
+  } else if (w <= 4) {  // ------------------------------------------------ loader teams
+    const bool team_k = w <= 2;
+    const int p = tid - (team_k ? 32 : 96);
+    if (!team_k) {  // dO of the query tile (and its lo part)
+      auto rows = [&](const bf* base) {
+        return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DV : nullptr; };
+      };
+      tile_async_t<128, DV, NL>(sO, rows(d_o), d_o, p);
+      if constexpr (SPLIT) tile_async_t<128, DV, NL>(sO + S::Ob, rows(d_o_lo), d_o, p);
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_async_smem();
+      mbar_arrive(&do_full);
+    }
+    KeyTileIter<64> it;
+    it.init(t, qt);
+    int k0 = 0, nk = 0, j = 0;
+    bool own = false;
+    for (; it.next(k0, nk, own); ++j) {
+      const int NS = team_k ? NK : NV, s = j % NS;
+      if (j >= NS && !mbar_wait(team_k ? &kempty[s] : &vempty[s], ((j / NS) - 1) & 1)) {
+        give_up();
+        break;
+      }
+      if (aborted()) break;
+      auto rows = [=](const bf* base, int width) {
+        return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
+      };
+      if (team_k) {
+        tile_async_t<64, DQ, NL>(kst(s), rows(k, DQ), k, p);
+        if constexpr (SPLIT) tile_async_t<64, DQ, NL>(kst(s) + S::Kb, rows(k_lo, DQ), k, p);
+      } else {
+        tile_async_t<64, DV, NL>(vst(s), rows(v, DV), v, p);
+        if constexpr (SPLIT) tile_async_t<64, DV, NL>(vst(s) + S::Vb, rows(v_lo, DV), v, p);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_async_smem();
+      mbar_arrive(team_k ? &kfull[s] : &vfull[s]);
+    }
+    cp_async_wait<0>();
+  } else {  // ------------------------------------------------ P, dS (warps 5-12)
+    const int sp = w & 3, half = (w - 5) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
+    const bool in = row < qt.n;
+    const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
+    const float sl2 = scale * kLog2e;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar, parity));
+      if (!got && lane == 0) give_up();
+      return got && !__any_sync(0xffffffffu, aborted());
+    };
+    {  // this half of Q (and its lo part) into TMEM
+      constexpr int HC = DQ / 4;
+      for (int part = 0; part < (SPLIT ? 2 : 1); ++part) {
+        const bf* src = part ? q_lo : q;
+        const uint4* g4 = (in && src) ? reinterpret_cast<const uint4*>(src + ((size_t)qrow * H + h) * DQ) + HC / 4 * half
+                                      : nullptr;
+        for (int c0 = 0; c0 < HC; c0 += 16) {
+          float r[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 x = g4 ? g4[c0 / 4 + i] : make_uint4(0u, 0u, 0u, 0u);
+            r[4 * i] = __uint_as_float(x.x); r[4 * i + 1] = __uint_as_float(x.y);
+            r[4 * i + 2] = __uint_as_float(x.z); r[4 * i + 3] = __uint_as_float(x.w);
+          }
+          tmem_st16(la + (part ? cQl : cQh) + HC * half + c0, r);
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_ready);
+    }
+    // delta = rowsum(dO O) over the whole row (both threads of a row), lse of the row
+    float dl = 0.f, ls2 = 0.f;
+    if (in) {
       const Tio* orow = o + ((size_t)qrow * H + h) * DV;
       const bf* grow = d_o + ((size_t)qrow * H + h) * DV;
       const bf* glow = SPLIT && d_o_lo ? d_o_lo + ((size_t)qrow * H + h) * DV : nullptr;
-      for (int j = 0; j < DV; ++j)
-        dl = fmaf(to_f(orow[j]), __bfloat162float(grow[j]) + (glow ? __bfloat162float(glow[j]) : 0.f), dl);
-      delta[(size_t)qrow * H + h] = dl;
-      ls = lse[(size_t)qrow * H + h];
+      for (int c = 0; c < DV; ++c)
+        dl = fmaf(to_f(orow[c]), __bfloat162float(grow[c]) + (glow ? __bfloat162float(glow[c]) : 0.f), dl);
+      if (half == 0) delta[(size_t)qrow * H + h] = dl;
+      ls2 = lse[(size_t)qrow * H + h] * kLog2e;
     }
-    s_dl[row] = dl;
-    s_ls[row] = ls;
-  }
-  __syncthreads();
-  const float dl = s_dl[row], ls = s_ls[row];
-  tc::fence_after_sync();
-  const uint32_t tb = tslot;
-  const uint32_t la = tb + ((uint32_t)(32 * (w & 3)) << 16);
-  Sync sy{&bar, 0u, status};
-  // key tiles with one tile of look-ahead: V of the next tile is fetched by cp.async while this tile's
-  // dS and dQ products run, K of the next tile once this tile's dQ product has read K
-  auto load_k = [&](int k0, int nk) {
-    auto rows = [=](const bf* base) {
-      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * DQ : nullptr; };
-    };
-    tile_async<KT, DQ, NT>(sK, rows(k), k);
-    if constexpr (SPLIT) tile_async<KT, DQ, NT>(sKl, rows(k_lo), k);
-  };
-  auto load_v = [&](int k0, int nk) {
-    auto rows = [=](const bf* base) {
-      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * DV : nullptr; };
-    };
-    tile_async<KT, DV, NT>(sV, rows(v), v);
-    if constexpr (SPLIT) tile_async<KT, DV, NT>(sVl, rows(v_lo), v);
-  };
-  KeyTileIter<KT> it;
-  it.init(t, qt);
-  int k0 = 0, nk = 0;
-  bool own = false;
-  bool have = it.next(k0, nk, own);
-  if (have) {
-    load_k(k0, nk);
-    load_v(k0, nk);
-  }
-  tc::cp_async_commit();
-  bool first = true, ok = true;
-  while (have) {
-    int k1 = 0, n1 = 0;
-    bool own1 = false;
-    const bool more = it.next(k1, n1, own1);
-    tc::cp_async_wait<0>();  // this tile's K and V have arrived
-    ok = run(sy, [&] {
-      mma4(tb, tc::Op{tc::smem_u32(sQ), 128, false}, tc::Op{tc::smem_u32(sQl), 128, false},
-           tc::Op{tc::smem_u32(sK), KT, false}, tc::Op{tc::smem_u32(sKl), KT, false}, DQ,
-           tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
-      mma4(tb + 64, tc::Op{tc::smem_u32(sO), 128, false}, tc::Op{tc::smem_u32(sOl), 128, false},
-           tc::Op{tc::smem_u32(sV), KT, false}, tc::Op{tc::smem_u32(sVl), KT, false}, DV,
-           tc::idesc_bf16(128, KT, false, false), false, !SPLIT, !SPLIT);
-    });
-    if (!ok) break;
-    if (more) load_v(k1, n1);  // V is free once dP is in TMEM
-    tc::cp_async_commit();
-    float s[KH], dp[KH];
+    KeyTileIter<64> it;
+    it.init(t, qt);
+    int k0 = 0, nk = 0;
+    bool own = false, ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      it.next(k0, nk, own);
+      if (!(ok = wait_all(&s_full, j & 1)) || !(ok = wait_all(&dp_full, j & 1))) break;
+      fence_after_sync();
+      uint32_t rs[32], rp[32];
+      tmem_ld32_nowait(la + cS + 32 * half, rs);
+      tmem_ld32_nowait(la + cP + 32 * half, rp);
+      tmem_wait_ld();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_read);  // S may take S_{j+1}
+      const bool masked = !in || own || nk < 64;
+      float gh[16], gl[16];
 #pragma unroll
-    for (int c = 0; c < KH; c += 16) {
-      tc::tmem_ld16(la + KH * half + c, *reinterpret_cast<float(*)[16]>(s + c));
-      tc::tmem_ld16(la + 64 + KH * half + c, *reinterpret_cast<float(*)[16]>(dp + c));
+      for (int c = 0; c < 32; c += 2) {
+        float ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int kc = 32 * half + c + e;
+          const bool valid = !masked || (in && kc < nk && !(own && k0 + kc > qrow));
+          const float pv = valid ? exp2f(__uint_as_float(rs[c + e]) * sl2 - ls2) : 0.f;
+          ds[e] = pv * (__uint_as_float(rp[c + e]) - dl);
+        }
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(ds[0], ds[1]);
+        const float2 hf = __bfloat1622float2(hi);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(ds[0] - hf.x, ds[1] - hf.y);
+        gh[c / 2] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&hi));
+        gl[c / 2] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&lo));
+      }
+      // dS over this half's own dP columns: hi in the first 16, lo in the last 16
+      tmem_st16(la + cP + 32 * half, gh);
+      tmem_st16(la + cP + 32 * half + 16, gl);
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_full);
     }
+    if (ok && n_tiles > 0) ok = wait_all(&dq_done, (n_tiles - 1) & 1);
+    if (ok) {
+      fence_after_sync();
+      for (int c0 = 0; c0 < DQ / 2; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32_nowait(la + cG + DQ / 2 * half + c0, r);  // warp-collective: every row takes part
+        tmem_wait_ld();
+        if (in) {
+          float g[32];
 #pragma unroll
-    for (int j = 0; j < KH; ++j) {
-      const int c = KH * half + j;
-      const bool valid = row < qt.n && c < nk && (!own || k0 + c <= qrow);
-      const float p = valid ? expf(s[j] * scale - ls) : 0.f;
-      s[j] = p * (dp[j] - dl);
-    }
-#pragma unroll
-    for (int j = 0; j < KH; j += 16) put16<128, true>(sDh, sDl, row, KH * half + j, s + j);
-    const bool acc_on = !first;
-    first = false;
-    ok = run(sy, [&] {
-      mma4(tb + 128, tc::Op{tc::smem_u32(sDh), 128, false}, tc::Op{tc::smem_u32(sDl), 128, false},
-           tc::Op{tc::smem_u32(sK), KT, true}, tc::Op{tc::smem_u32(sKl), KT, true}, KT,
-           tc::idesc_bf16(128, DQ, false, true), acc_on, false, !SPLIT);
-    });
-    if (!ok) break;
-    if (more) load_k(k1, n1);  // K is free once dQ has read it
-    tc::cp_async_commit();
-    k0 = k1; nk = n1; own = own1; have = more;
-  }
-  tc::cp_async_wait<0>();
-  if (ok) {
-    for (int c = 0; c < DQ / 2; c += 32) {
-      float g[32];
-      tc::tmem_ld32(la + 128 + DQ / 2 * half + c, g);
-      if (row < qt.n) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) g[j] *= scale;
-        Tio* dst = dq + ((size_t)qrow * H + h) * DQ + DQ / 2 * half + c;
-        st_out16(dst, g);
-        st_out16(dst + 16, g + 16);
+          for (int c = 0; c < 32; ++c) g[c] = n_tiles > 0 ? __uint_as_float(r[c]) * scale : 0.f;
+          Tio* dst = dq + ((size_t)qrow * H + h) * DQ + DQ / 2 * half + c0;
+          st_out16(dst, g);
+          st_out16(dst + 16, g + 16);
+        }
       }
     }
   }
-  tc::fence_before_sync();
+  fence_before_sync();
   __syncthreads();
-  if (w == 0) tc::tmem_dealloc(tb, 512);
+  if (w == 0) tmem_dealloc(tb, 512);
 }
 
 // ------------------------------------------------------------------------------------------ backward dK, dV
@@ -758,16 +883,13 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
         const float* src = (p < QT ? lse : delta) + (size_t)(q0 + min(c, nq - 1)) * H + h;
         cp_async4(st + (p < QT ? S::sL : S::sD) + 4 * c, src, c < nq ? 4u : 0u);
       }
+      // publish the stage to the tensor core and the P / dS warps as soon as it has landed
       cp_async_commit();
-      if (j >= 1) {  // the previous stage has landed: publish it to the tensor core and the P / dS warps
-        cp_async_wait<1>();
-        fence_async_smem();
-        mbar_arrive(&full[(j - 1) % NS]);
-      }
+      cp_async_wait<0>();
+      fence_async_smem();
+      mbar_arrive(&full[s]);
     }
     cp_async_wait<0>();
-    fence_async_smem();
-    if (j == n_tiles && n_tiles > 0) mbar_arrive(&full[(n_tiles - 1) % NS]);
   } else {  // ------------------------------------------------ P^T, dS^T (warps 4-11)
     const int sp = w & 3, half = (w - 4) >> 2;
     const int r = lane < 16 ? 16 * sp + lane : -1;  // key row of this thread (M = 64 layout)

@@ -776,7 +776,7 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const tpc::Plan& p = plan->p;
   using bf = __nv_bfloat16;
-  const dim3 gq((unsigned)p.attn_qtiles.size(), (unsigned)s->H);
+  const dim3 gq((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest
   const dim3 gk((unsigned)(p.attn_ktiles.size() * (size_t)s->H));  // (key tile, head), key tiles fastest
   auto go = [&](auto tio, auto split) -> int {
     using T = decltype(tio);
