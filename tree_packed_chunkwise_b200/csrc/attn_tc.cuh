@@ -54,6 +54,29 @@ __device__ __forceinline__ void st_out16(T* p, const float* v) {
   }
 }
 
+// x0, x1 as packed bf16 hi / lo pairs (element 0 in the low half): x = hi + lo to ~2^-17
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// 16 packed values (8 pairs along the contiguous index) of row a at (a, b0..b0+15) of K-major
+// core-matrix tiles with A rows, hi and lo parts
+template <int A>
+__device__ __forceinline__ void put16_packed(uint8_t* hi, uint8_t* lo, int a, int b0, const uint32_t* ph,
+                                             const uint32_t* pl) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    *reinterpret_cast<uint4*>(hi + tc::cm_off(a, b0 + 8 * half, A)) =
+        make_uint4(ph[4 * half], ph[4 * half + 1], ph[4 * half + 2], ph[4 * half + 3]);
+    *reinterpret_cast<uint4*>(lo + tc::cm_off(a, b0 + 8 * half, A)) =
+        make_uint4(pl[4 * half], pl[4 * half + 1], pl[4 * half + 2], pl[4 * half + 3]);
+  }
+}
+
 }  // namespace tck
 
 // ------------------------------------------------------------------------------------------ forward
@@ -760,6 +783,8 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
   using S = AttnDkvSmem<SPLIT>;
   using bf = __nv_bfloat16;
   constexpr int DQ = kAttnQK, DV = kAttnDV, QT = S::QT, NS = S::NS, NP = 96;
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float sl2 = scale * kLog2e;
   // TMEM columns: dV (128), dK (192), then two buffers of S^T (32) and dP^T (32)
   constexpr uint32_t cDV = 0, cDK = 128, cS = 320, cP = 352, cBuf = 64;
   // grid: one block per (key tile, head), key tiles fastest, so that the blocks resident at one
@@ -915,20 +940,27 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       const float* sl = reinterpret_cast<const float*>(st + S::sL);
       const float* sd = reinterpret_cast<const float*>(st + S::sD);
       const int q0 = k0 + j * QT, nq = min(QT, q_end - q0);
+      // P^T and dS^T of this thread's 16 entries as packed bf16 hi / lo pairs (base-2 exponentials)
+      uint32_t ph[8], pl[8], gh[8], gl[8];
       if (r >= 0) {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int c = 16 * half + jj, qrow = q0 + c;
-          const bool valid = r < nk && c < nq && !(qrow < own_end && qrow < k0 + r);
-          const float pv = valid ? expf(sv[jj] * scale - sl[c]) : 0.f;
-          sv[jj] = pv;
-          dp[jj] = pv * (dp[jj] - sd[c]);
+        for (int jj = 0; jj < 16; jj += 2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 16 * half + jj + e, qrow = q0 + c;
+            const bool valid = r < nk && c < nq && !(qrow < own_end && qrow < k0 + r);
+            pv[e] = valid ? exp2f(fmaf(sv[jj + e], sl2, -sl[c] * kLog2e)) : 0.f;
+            dsv[e] = pv[e] * (dp[jj + e] - sd[c]);
+          }
+          split2(pv[0], pv[1], ph[jj / 2], pl[jj / 2]);
+          split2(dsv[0], dsv[1], gh[jj / 2], gl[jj / 2]);
         }
       }
       if (j >= 1 && !(ok = wait_all(&p_empty, (j - 1) & 1))) break;  // dV, dK of tile j - 1 are done
       if (r >= 0) {
-        put16<64, true>(sPh, sPl, r, 16 * half, sv);
-        put16<64, true>(sDh, sDl, r, 16 * half, dp);
+        put16_packed<64>(sPh, sPl, r, 16 * half, ph, pl);
+        put16_packed<64>(sDh, sDl, r, 16 * half, gh, gl);
       }
       fence_async_smem();
       __syncwarp();
