@@ -143,9 +143,9 @@ __device__ __forceinline__ void tile_async_t(uint8_t* dst, RP rowp, const void* 
 
 // Forward, per query tile (<= 128 rows of one node) and head, warp-specialised:
 //   warp 0      issues the MMAs: S_j = Q K_j^T into one of two TMEM buffers, then O += P_j V_j;
-//   warps 1-2   stream the key tiles K_j (and their lo parts) through a three-stage ring,
-//   warps 3-4   stream V_j through a two-stage ring (cp.async; a stage is published once landed);
-//   warps 5-12  two threads per query row (key columns split in halves): Q is loaded once into TMEM
+//   warp 1      streams the key tiles K_j (and their lo parts) through a three-stage ring and
+//   warp 2      V_j through a two-stage ring, by TMA (128-byte-swizzled boxes of 64 features);
+//   warps 3-10  two threads per query row (key columns split in halves): Q is loaded once into TMEM
 //               (the A operand of S), then per key tile the online softmax (base-2 exponentials of
 //               log2-scaled scores) reads S_j (releasing its buffer), writes P_j as a bf16 hi/lo
 //               pair into a TMEM buffer of its own (the A operand of P V) once P_{j-1} V_{j-1} has
@@ -159,24 +159,24 @@ struct AttnFwdSmem {
   static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
   static constexpr size_t Kst = X * Kb, Vst = X * Vb;  // one ring stage
   static constexpr size_t K = 0, V = K + NK * Kst;
-  static constexpr size_t total = V + NV * Vst;
+  static constexpr size_t total = V + NV * Vst + 1024;  // + slack to align the boxes to 1024 bytes
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
-constexpr int kAttnFwdThreads = 416;
+constexpr int kAttnFwdThreads = 352;
 
 template <typename Tout, bool SPLIT>
 __global__ void __launch_bounds__(kAttnFwdThreads, 1)
     attn_fwd_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
-                const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
-                const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
-                const __nv_bfloat16* __restrict__ v_lo, Tout* __restrict__ o, float* __restrict__ lse,
+                const __nv_bfloat16* __restrict__ q_lo, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_v,
+                const __grid_constant__ CUtensorMap tm_vl, Tout* __restrict__ o, float* __restrict__ lse,
                 int* status) {
   using namespace tck;
   using namespace tc;
   using S = AttnFwdSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NK = S::NK, NV = S::NV, NL = 64;  // NL threads per loader team
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NK = S::NK, NV = S::NV;
   constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
   constexpr float kRaise2 = 8.f * kLog2e;  // raise threshold (e^8) in log2 units
   // TMEM columns: Q hi (96), Q lo (96), O (128), two S buffers (64 each), P hi (32) and lo (32)
@@ -188,7 +188,9 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   const AttnTile qt = t.attn_qtiles[blockIdx.x % n_qt];
   const int h = blockIdx.x / n_qt;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  extern __shared__ __align__(1024) uint8_t asmem[];
+  extern __shared__ __align__(1024) uint8_t asmem_raw[];
+  // the swizzle pattern is a function of the shared address: boxes start on 1024-byte boundaries
+  uint8_t* asmem = asmem_raw + ((1024u - (smem_u32(asmem_raw) & 1023u)) & 1023u);
   __shared__ __align__(8) uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], s_full[2], s_read[2], p_full,
       pv_done, q_ready, done_bar;
   __shared__ uint32_t tslot;
@@ -199,11 +201,11 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   if (w == 0) tmem_alloc(&tslot, 512);
   if (tid == 0) {
     for (int s = 0; s < NK; ++s) {
-      mbar_init(&kfull[s], NL);
+      mbar_init(&kfull[s], 1);  // the loader's arrival with the expected bytes
       mbar_init(&kempty[s], 1);
     }
     for (int s = 0; s < NV; ++s) {
-      mbar_init(&vfull[s], NL);
+      mbar_init(&vfull[s], 1);
       mbar_init(&vempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -249,11 +251,11 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
           }
           fence_after_sync();
           const uint32_t d = tb + cS + cBuf * b;
-          const Op kh{smem_u32(kst(ks)), 64, false}, kl{smem_u32(kst(ks) + S::Kb), 64, false};
-          for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQh + 8 * s, op_desc(kh, s), id_s, s ? 1u : 0u);
+          const uint32_t kh = smem_u32(kst(ks)), kl = kh + (uint32_t)S::Kb;
+          for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQh + 8 * s, sw_desc_k(kh, 64, s), id_s, s ? 1u : 0u);
           if constexpr (SPLIT) {
-            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQl + 8 * s, op_desc(kh, s), id_s, 1u);
-            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQh + 8 * s, op_desc(kl, s), id_s, 1u);
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQl + 8 * s, sw_desc_k(kh, 64, s), id_s, 1u);
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(d, tb + cQh + 8 * s, sw_desc_k(kl, 64, s), id_s, 1u);
           }
           commit(&kempty[ks]);
           commit(&s_full[b]);
@@ -266,11 +268,11 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
           }
           fence_after_sync();
           const uint32_t ph = tb + cP, pl = ph + 32;
-          const Op vh{smem_u32(vst(vs)), 64, true}, vl{smem_u32(vst(vs) + S::Vb), 64, true};
-          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, op_desc(vh, s), id_o, (jp > 0 || s) ? 1u : 0u);
-          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, pl + 8 * s, op_desc(vh, s), id_o, 1u);
+          const uint32_t vh = smem_u32(vst(vs)), vl = vh + (uint32_t)S::Vb;
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, sw_desc_mn(vh, 64, s), id_o, (jp > 0 || s) ? 1u : 0u);
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, pl + 8 * s, sw_desc_mn(vh, 64, s), id_o, 1u);
           if constexpr (SPLIT)
-            for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, op_desc(vl, s), id_o, 1u);
+            for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cO, ph + 8 * s, sw_desc_mn(vl, 64, s), id_o, 1u);
           commit(&vempty[vs]);
           commit(&pv_done);
         }
@@ -278,42 +280,39 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       commit(&done_bar);  // arrives once every MMA issued above has completed
       if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
     }
-  } else if (w <= 4) {  // ------------------------------------------------ loader teams
-    const bool team_k = w <= 2;
-    const int p = tid - (team_k ? 32 : 96);
-    KeyTileIter<64> it;
-    it.init(t, qt);
-    int k0 = 0, nk = 0, j = 0;
-    bool own = false;
-    for (; it.next(k0, nk, own); ++j) {
-      const int NS = team_k ? NK : NV, s = j % NS;
-      if (j >= NS && !mbar_wait(team_k ? &kempty[s] : &vempty[s], ((j / NS) - 1) & 1)) {
-        give_up();
-        break;
+  } else if (w <= 2) {  // ------------------------------------------------ loaders (one thread each)
+    if (lane == 0) {
+      const bool is_k = w == 1;
+      const int NS = is_k ? NK : NV, F = is_k ? DQ : DV;
+      const uint32_t part = (uint32_t)(is_k ? S::Kb : S::Vb), bytes = (uint32_t)(SPLIT ? 2 : 1) * part;
+      KeyTileIter<64> it;
+      it.init(t, qt);
+      int k0 = 0, nk = 0, j = 0;
+      bool own = false;
+      for (; it.next(k0, nk, own); ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(is_k ? &kempty[s] : &vempty[s], ((j / NS) - 1) & 1)) {
+          give_up();
+          break;
+        }
+        if (aborted()) break;
+        uint64_t* bar = is_k ? &kfull[s] : &vfull[s];
+        uint8_t* dst = is_k ? kst(s) : vst(s);
+        // rows k0 .. k0 + 63 of head h (rows past the tile's end are masked by the softmax; rows past
+        // the tensor's end are filled with zeros)
+        mbar_arrive_expect_tx(bar, bytes);
+        for (int c = 0; c < F / 64; ++c) {
+          tma_load_3d(dst + c * 64 * 128, is_k ? (const void*)&tm_k : (const void*)&tm_v, 64 * c, h, k0, bar);
+          if constexpr (SPLIT)
+            tma_load_3d(dst + part + c * 64 * 128, is_k ? (const void*)&tm_kl : (const void*)&tm_vl, 64 * c, h, k0, bar);
+        }
       }
-      if (aborted()) break;
-      auto rows = [=](const bf* base, int width) {
-        return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
-      };
-      if (team_k) {
-        tile_async_t<64, DQ, NL>(kst(s), rows(k, DQ), k, p);
-        if constexpr (SPLIT) tile_async_t<64, DQ, NL>(kst(s) + S::Kb, rows(k_lo, DQ), k, p);
-      } else {
-        tile_async_t<64, DV, NL>(vst(s), rows(v, DV), v, p);
-        if constexpr (SPLIT) tile_async_t<64, DV, NL>(vst(s) + S::Vb, rows(v_lo, DV), v, p);
-      }
-      // publish the tile as soon as it has landed (the writes are made visible to the tensor core)
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_async_smem();
-      mbar_arrive(team_k ? &kfull[s] : &vfull[s]);
     }
-    cp_async_wait<0>();
-  } else {  // ------------------------------------------------ softmax (warps 5-12)
+  } else if (w >= 3) {  // ------------------------------------------------ softmax (warps 3-10)
     // warp w holds the TMEM lanes (query rows) of sub-partition w % 4 and the key columns of half
-    // (w - 5) / 4 for the exponentials; each thread reads the whole row of S for the row maximum, so
+    // (w - 3) / 4 for the exponentials; each thread reads the whole row of S for the row maximum, so
     // the two threads of a row take the same decisions without exchanging data per key tile
-    const int sp = w & 3, half = (w - 5) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
+    const int sp = w & 3, half = (w - 3) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
     const float sl2 = scale * kLog2e;  // scores in log2 units: t = s scale log2(e)
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {

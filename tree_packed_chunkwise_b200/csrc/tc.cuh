@@ -136,6 +136,31 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// Tiled TMA load (3-D tensor map, no multicast); the innermost coordinate x must be a multiple of
+// 16 bytes' worth of elements.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Descriptors of 128-byte-swizzled bf16 operand tiles stored as 64-column TMA boxes of `rows` rows
+// (each box row one 128-byte line, 8-row groups 1024 bytes apart).  K-major (a line holds 64 K of one
+// M/N row; 16-wide K step s in box s / 4 at byte 32 (s % 4)); MN-major (a line holds 64 M/N of one
+// K row; the K step moves 16 lines, the 64-wide M/N blocks are one box apart).
+__device__ __forceinline__ uint64_t sw128_desc_raw(uint32_t addr, uint32_t lbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((1024u >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ uint64_t sw_desc_k(uint32_t base, int rows, int s) {
+  return sw128_desc_raw(base + (uint32_t)(s >> 2) * (uint32_t)rows * 128u + (uint32_t)(s & 3) * 32u, 16u);
+}
+__device__ __forceinline__ uint64_t sw_desc_mn(uint32_t base, int rows, int s) {
+  return sw128_desc_raw(base + (uint32_t)s * 2048u, (uint32_t)rows * 128u);
+}
+
 // writes by threads to shared memory become visible to the tensor core (async proxy)
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }

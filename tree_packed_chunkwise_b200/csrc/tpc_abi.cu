@@ -430,6 +430,22 @@ bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, u
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over a [rows][heads][features] tensor (feature dimension contiguous): boxes
+// of 64 features x 1 head x box_rows rows, each box row one 128-byte swizzled line; rows past the
+// end read as zeros.
+bool tensor_map_rows(CUtensorMap* m, const void* ptr, uint64_t features, uint64_t heads, uint64_t rows,
+                     uint32_t box_rows) {
+  CUtensorMap probe;
+  if (!tensor_map(&probe, ptr, 64, 1, 64, 8, 64)) return false;  // looks up the encoder
+  cuuint64_t dims[3] = {features, heads, rows};
+  cuuint64_t strides[2] = {features * 2, heads * features * 2};
+  cuuint32_t box[3] = {64, 1, box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -748,6 +764,12 @@ int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const v
   const tpc::Plan& p = plan->p;
   const dim3 grid((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest
   using bf = __nv_bfloat16;
+  const uint64_t NR = (uint64_t)p.n_unique;
+  CUtensorMap tk, tkl, tv, tvl;
+  bool ok = tensor_map_rows(&tk, k, tpc::kAttnQK, s->H, NR, 64) && tensor_map_rows(&tv, v, tpc::kAttnDV, s->H, NR, 64);
+  ok = ok && tensor_map_rows(&tkl, L.k ? L.k : k, tpc::kAttnQK, s->H, NR, 64) &&
+       tensor_map_rows(&tvl, L.v ? L.v : v, tpc::kAttnDV, s->H, NR, 64);
+  if (!ok) return fail(TPC_ERR_CUDA, "attention forward: cuTensorMapEncodeTiled failed");
   auto go = [&](auto tout, auto split) -> int {
     using T = decltype(tout);
     constexpr bool SP = decltype(split)::value;
@@ -755,8 +777,7 @@ int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const v
     TPC_CUDA(set_smem(tpc::attn_fwd_tc<T, SP>, smem));
     TPC_LAUNCH("attn_fwd_tc", st,
                (tpc::attn_fwd_tc<T, SP><<<grid, tpc::kAttnFwdThreads, smem, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
-                   (const bf*)L.v, (T*)o, lse, status)));
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, tk, tkl, tv, tvl, (T*)o, lse, status)));
     return TPC_OK;
   };
   using Y = std::true_type;
