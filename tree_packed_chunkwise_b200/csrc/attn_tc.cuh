@@ -457,8 +457,9 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
 // dK/dV kernel), then over the key tiles P = exp(scale S - lse), dP = dO V^T, dS = P (dP - delta),
 // dQ += dS K; dq = scale dQ.  Warp-specialised like the forward:
 //   warp 0      issues S_j = Q K_j^T, then dQ += dS_{j-1} K_{j-1}, then dP_j = dO V_j^T;
-//   warps 1-2   stream K_j through a two-stage ring; warps 3-4 load dO once, then stream V_j;
-//   warps 5-12  two threads per query row (key columns in halves): Q into TMEM once, delta; per key
+//   warp 1      streams K_j through a two-stage ring; warp 2 loads dO once, then streams V_j (TMA,
+//               128-byte-swizzled boxes of 64 features);
+//   warps 3-10  two threads per query row (key columns in halves): Q into TMEM once, delta; per key
 //               tile they read S_j (releasing it for S_{j+1}) and dP_j, and write dS_j as a bf16
 //               hi/lo pair over their own dP_j columns (the A operand of the dQ product).
 template <bool SPLIT>
@@ -467,25 +468,26 @@ struct AttnDqSmem {
   static constexpr size_t X = SPLIT ? 2 : 1;
   static constexpr size_t Ob = size_t(128) * kAttnDV * 2, Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
   static constexpr size_t dO = 0, K = dO + X * Ob, V = K + NK * X * Kb;
-  static constexpr size_t total = V + NV * X * Vb;
+  static constexpr size_t total = V + NV * X * Vb + 1024;  // + slack to align the boxes to 1024 bytes
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
-constexpr int kAttnDqThreads = 416;
+constexpr int kAttnDqThreads = 352;
 
 template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnDqThreads, 1)
     attn_bwd_dq_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
-                   const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
-                   const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
-                   const __nv_bfloat16* __restrict__ v_lo, const Tio* __restrict__ o, const float* __restrict__ lse,
+                   const __nv_bfloat16* __restrict__ q_lo, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_vl, const __grid_constant__ CUtensorMap tm_o,
+                   const __grid_constant__ CUtensorMap tm_ol, const Tio* __restrict__ o, const float* __restrict__ lse,
                    const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ d_o_lo,
                    Tio* __restrict__ dq, float* __restrict__ delta, int* status) {
   using namespace tck;
   using namespace tc;
   using S = AttnDqSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, NK = S::NK, NV = S::NV, NL = 64;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, NK = S::NK, NV = S::NV;
   constexpr float kLog2e = 1.4426950408889634f;
   // TMEM columns: Q hi (96), Q lo (96), dQ (192), S (64), dP / dS (64)
   constexpr uint32_t cQh = 0, cQl = 96, cG = 192, cS = 384, cP = 448;
@@ -494,7 +496,8 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
   const AttnTile qt = t.attn_qtiles[blockIdx.x % n_qt];
   const int h = blockIdx.x / n_qt;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  extern __shared__ __align__(1024) uint8_t asmem[];
+  extern __shared__ __align__(1024) uint8_t asmem_raw[];
+  uint8_t* asmem = asmem_raw + ((1024u - (smem_u32(asmem_raw) & 1023u)) & 1023u);  // 1024-byte aligned boxes
   __shared__ __align__(8) uint64_t kfull[NK], kempty[NK], vfull[NV], vempty[NV], do_full, q_ready, s_full, s_read,
       dp_full, ds_full, dq_done, done_bar;
   __shared__ uint32_t tslot;
@@ -505,14 +508,14 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
   if (w == 0) tmem_alloc(&tslot, 512);
   if (tid == 0) {
     for (int s = 0; s < NK; ++s) {
-      mbar_init(&kfull[s], NL);
+      mbar_init(&kfull[s], 1);  // the loader's arrival with the expected bytes
       mbar_init(&kempty[s], 1);
     }
     for (int s = 0; s < NV; ++s) {
-      mbar_init(&vfull[s], NL);
+      mbar_init(&vfull[s], 1);
       mbar_init(&vempty[s], 1);
     }
-    mbar_init(&do_full, NL);
+    mbar_init(&do_full, 1);
     mbar_init(&q_ready, 8);  // one arrival per softmax warp
     mbar_init(&s_full, 1);
     mbar_init(&s_read, 8);
@@ -545,7 +548,7 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
       const uint32_t id_s = idesc_bf16(128, 64, false, false), id_g = idesc_bf16(128, DQ, false, true);
       bool ok = mbar_wait(&q_ready, 0) && mbar_wait(&do_full, 0);
       if (!ok) give_up();
-      const Op oh{smem_u32(sO), 128, false}, ol{smem_u32(sO + S::Ob), 128, false};
+      const uint32_t oh = smem_u32(sO), ol = oh + (uint32_t)S::Ob;
       for (int j = 0; ok && j <= n_tiles && !aborted(); ++j) {
         if (j < n_tiles) {  // S_j = Q K_j^T, once the softmax warps have read S_{j-1}
           const int ks = j % NK;
@@ -554,11 +557,11 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
             break;
           }
           fence_after_sync();
-          const Op kh{smem_u32(kst(ks)), 64, false}, kl{smem_u32(kst(ks) + S::Kb), 64, false};
-          for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQh + 8 * s, op_desc(kh, s), id_s, s ? 1u : 0u);
+          const uint32_t kh = smem_u32(kst(ks)), kl = kh + (uint32_t)S::Kb;
+          for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQh + 8 * s, sw_desc_k(kh, 64, s), id_s, s ? 1u : 0u);
           if constexpr (SPLIT) {
-            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQl + 8 * s, op_desc(kh, s), id_s, 1u);
-            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQh + 8 * s, op_desc(kl, s), id_s, 1u);
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQl + 8 * s, sw_desc_k(kh, 64, s), id_s, 1u);
+            for (int s = 0; s < DQ / 16; ++s) mma_bf16_ts(tb + cS, tb + cQh + 8 * s, sw_desc_k(kl, 64, s), id_s, 1u);
           }
           commit(&s_full);
         }
@@ -569,12 +572,12 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
             break;
           }
           fence_after_sync();
-          const Op kh{smem_u32(kst(ks)), 64, true}, kl{smem_u32(kst(ks) + S::Kb), 64, true};
+          const uint32_t kh = smem_u32(kst(ks)), kl = kh + (uint32_t)S::Kb;
           auto a_hi = [&](int s) { return tb + cP + 32 * (s >> 1) + 8 * (s & 1); };
-          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), op_desc(kh, s), id_g, (jp > 0 || s) ? 1u : 0u);
-          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s) + 16, op_desc(kh, s), id_g, 1u);
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), sw_desc_mn(kh, 64, s), id_g, (jp > 0 || s) ? 1u : 0u);
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s) + 16, sw_desc_mn(kh, 64, s), id_g, 1u);
           if constexpr (SPLIT)
-            for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), op_desc(kl, s), id_g, 1u);
+            for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), sw_desc_mn(kl, 64, s), id_g, 1u);
           commit(&kempty[ks]);
           commit(&dq_done);
         }
@@ -585,8 +588,12 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
             break;
           }
           fence_after_sync();
-          const Op vh{smem_u32(vst(vs)), 64, false}, vl{smem_u32(vst(vs) + S::Vb), 64, false};
-          mma4(tb + cP, oh, ol, vh, vl, DV, id_s, false, !SPLIT, !SPLIT);
+          const uint32_t vh = smem_u32(vst(vs)), vl = vh + (uint32_t)S::Vb;
+          for (int s = 0; s < DV / 16; ++s) mma_bf16(tb + cP, sw_desc_k(oh, 128, s), sw_desc_k(vh, 64, s), id_s, s ? 1u : 0u);
+          if constexpr (SPLIT) {
+            for (int s = 0; s < DV / 16; ++s) mma_bf16(tb + cP, sw_desc_k(ol, 128, s), sw_desc_k(vh, 64, s), id_s, 1u);
+            for (int s = 0; s < DV / 16; ++s) mma_bf16(tb + cP, sw_desc_k(oh, 128, s), sw_desc_k(vl, 64, s), id_s, 1u);
+          }
           commit(&vempty[vs]);
           commit(&dp_full);
         }
@@ -594,49 +601,41 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
       commit(&done_bar);  // arrives once every MMA issued above has completed
       if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
     }
-  } else if (w <= 4) {  // ------------------------------------------------ loader teams
-    const bool team_k = w <= 2;
-    const int p = tid - (team_k ? 32 : 96);
-    if (!team_k) {  // dO of the query tile (and its lo part)
-      auto rows = [&](const bf* base) {
-        return [=](int a) -> const bf* { return a < qt.n && base ? base + ((size_t)(qt.row + a) * H + h) * DV : nullptr; };
-      };
-      tile_async_t<128, DV, NL>(sO, rows(d_o), d_o, p);
-      if constexpr (SPLIT) tile_async_t<128, DV, NL>(sO + S::Ob, rows(d_o_lo), d_o, p);
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_async_smem();
-      mbar_arrive(&do_full);
-    }
-    KeyTileIter<64> it;
-    it.init(t, qt);
-    int k0 = 0, nk = 0, j = 0;
-    bool own = false;
-    for (; it.next(k0, nk, own); ++j) {
-      const int NS = team_k ? NK : NV, s = j % NS;
-      if (j >= NS && !mbar_wait(team_k ? &kempty[s] : &vempty[s], ((j / NS) - 1) & 1)) {
-        give_up();
-        break;
+  } else if (w <= 2) {  // ------------------------------------------------ loaders (one thread each)
+    if (lane == 0) {
+      const bool is_k = w == 1;
+      if (!is_k) {  // dO rows of the query tile (rows past the tile are masked, past the tensor zero)
+        mbar_arrive_expect_tx(&do_full, (uint32_t)(SPLIT ? 2 : 1) * (uint32_t)S::Ob);
+        for (int c = 0; c < DV / 64; ++c) {
+          tma_load_3d(sO + c * 128 * 128, &tm_o, 64 * c, h, qt.row, &do_full);
+          if constexpr (SPLIT) tma_load_3d(sO + S::Ob + c * 128 * 128, &tm_ol, 64 * c, h, qt.row, &do_full);
+        }
       }
-      if (aborted()) break;
-      auto rows = [=](const bf* base, int width) {
-        return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
-      };
-      if (team_k) {
-        tile_async_t<64, DQ, NL>(kst(s), rows(k, DQ), k, p);
-        if constexpr (SPLIT) tile_async_t<64, DQ, NL>(kst(s) + S::Kb, rows(k_lo, DQ), k, p);
-      } else {
-        tile_async_t<64, DV, NL>(vst(s), rows(v, DV), v, p);
-        if constexpr (SPLIT) tile_async_t<64, DV, NL>(vst(s) + S::Vb, rows(v_lo, DV), v, p);
+      const int NS = is_k ? NK : NV, F = is_k ? DQ : DV;
+      const uint32_t part = (uint32_t)(is_k ? S::Kb : S::Vb), bytes = (uint32_t)(SPLIT ? 2 : 1) * part;
+      KeyTileIter<64> it;
+      it.init(t, qt);
+      int k0 = 0, nk = 0, j = 0;
+      bool own = false;
+      for (; it.next(k0, nk, own); ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(is_k ? &kempty[s] : &vempty[s], ((j / NS) - 1) & 1)) {
+          give_up();
+          break;
+        }
+        if (aborted()) break;
+        uint64_t* bar = is_k ? &kfull[s] : &vfull[s];
+        uint8_t* dst = is_k ? kst(s) : vst(s);
+        mbar_arrive_expect_tx(bar, bytes);
+        for (int c = 0; c < F / 64; ++c) {
+          tma_load_3d(dst + c * 64 * 128, is_k ? (const void*)&tm_k : (const void*)&tm_v, 64 * c, h, k0, bar);
+          if constexpr (SPLIT)
+            tma_load_3d(dst + part + c * 64 * 128, is_k ? (const void*)&tm_kl : (const void*)&tm_vl, 64 * c, h, k0, bar);
+        }
       }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_async_smem();
-      mbar_arrive(team_k ? &kfull[s] : &vfull[s]);
     }
-    cp_async_wait<0>();
-  } else {  // ------------------------------------------------ P, dS (warps 5-12)
-    const int sp = w & 3, half = (w - 5) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
+  } else if (w >= 3) {  // ------------------------------------------------ P, dS (warps 3-10)
+    const int sp = w & 3, half = (w - 3) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
     const bool in = row < qt.n;
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
     const float sl2 = scale * kLog2e;
@@ -745,9 +744,9 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
 // (queries of u itself only from the key row on), S^T = K Q^T, dP^T = V dO^T, P^T = exp(scale S^T -
 // lse), dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 64 accumulators.
 //
-// Warp-specialised: warp 0 issues the MMAs, warps 1-3 stream the query tiles (Q, dO, their lo
-// parts, lse and delta) through a three-stage ring with cp.async, warps 4-11 turn S^T and dP^T into
-// P^T and dS^T.  S^T / dP^T have two TMEM buffers, so the products of query tile j + 1 run on the
+// Warp-specialised: warp 0 issues the MMAs, warp 1 streams K, V and then the query tiles (Q, dO and
+// their lo parts) through a three-stage ring by TMA (128-byte-swizzled boxes of 64 features), warp 2
+// adds lse and delta of each query tile by cp.async, warps 3-10 turn S^T and dP^T into P^T and dS^T.  S^T / dP^T have two TMEM buffers, so the products of query tile j + 1 run on the
 // tensor core while the P / dS math of tile j runs on the SIMT cores; the dV / dK products of tile j
 // follow once its P^T and dS^T are in shared memory.  Every wait is bounded; a timeout records
 // TPC_ERR_TIMEOUT and every role stops.
@@ -757,31 +756,32 @@ struct AttnDkvSmem {
   static constexpr size_t X = SPLIT ? 1 : 0;
   static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
   static constexpr size_t Qb = size_t(QT) * kAttnQK * 2, Ob = size_t(QT) * kAttnDV * 2, Pb = size_t(64) * QT * 2;
-  // one ring stage: Q, Q_lo, dO, dO_lo, lse[QT], delta[QT]
+  // one ring stage: Q, Q_lo, dO, dO_lo (swizzled boxes), lse[QT], delta[QT]; stages 1024-byte aligned
   static constexpr size_t sQ = 0, sQl = sQ + Qb, sO = sQl + X * Qb, sOl = sO + Ob, sL = sOl + X * Ob, sD = sL + QT * 4;
-  static constexpr size_t stage = sD + QT * 4;
+  static constexpr size_t stage = (sD + QT * 4 + 1023) & ~size_t(1023);
   static constexpr size_t K = 0, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb, ring = Vl + X * Vb;
   static constexpr size_t P = ring + NS * stage, Pl = P + Pb, dS = Pl + Pb, dSl = dS + Pb;
-  static constexpr size_t total = dSl + Pb;
+  static constexpr size_t total = dSl + Pb + 1024;  // + slack to align the boxes to 1024 bytes
   static_assert(total <= 227 * 1024, "shared memory");
-  static_assert(stage % 128 == 0, "stage alignment");
+  static_assert(stage % 1024 == 0, "stage alignment");
 };
 
-constexpr int kAttnDkvThreads = 384;
+constexpr int kAttnDkvThreads = 352;
 
 template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnDkvThreads, 1)
-    attn_bwd_dkv_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ q,
-                    const __nv_bfloat16* __restrict__ q_lo, const __nv_bfloat16* __restrict__ k,
-                    const __nv_bfloat16* __restrict__ k_lo, const __nv_bfloat16* __restrict__ v,
-                    const __nv_bfloat16* __restrict__ v_lo, const float* __restrict__ lse,
-                    const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ d_o_lo,
-                    const float* __restrict__ delta, Tio* __restrict__ dk, Tio* __restrict__ dv, int* status) {
+    attn_bwd_dkv_tc(DevTables t, int H, float scale,
+                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ql,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kl,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_vl,
+                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_ol,
+                    const float* __restrict__ lse, const float* __restrict__ delta, Tio* __restrict__ dk,
+                    Tio* __restrict__ dv, int* status) {
   using namespace tck;
   using namespace tc;
   using S = AttnDkvSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, QT = S::QT, NS = S::NS, NP = 96;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, QT = S::QT, NS = S::NS;
   constexpr float kLog2e = 1.4426950408889634f;
   const float sl2 = scale * kLog2e;
   // TMEM columns: dV (128), dK (192), then two buffers of S^T (32) and dP^T (32)
@@ -796,7 +796,8 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
   const int k0 = kt.row, nk = kt.n, own_end = nd.row_offset + nd.length, q_end = nd.subtree_end;
   const int n_tiles = (q_end - k0 + QT - 1) / QT;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  extern __shared__ __align__(1024) uint8_t asmem[];
+  extern __shared__ __align__(1024) uint8_t asmem_raw[];
+  uint8_t* asmem = asmem_raw + ((1024u - (smem_u32(asmem_raw) & 1023u)) & 1023u);  // 1024-byte aligned boxes
   __shared__ __align__(8) uint64_t full[NS], empty[NS], s_full[2], s_empty[2], p_full, p_empty, done_bar;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
@@ -806,7 +807,7 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
   if (w == 0) tmem_alloc(&tslot, 512);
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], NP);  // one arrival per loading thread once its copies have landed
+      mbar_init(&full[s], 33);  // the TMA thread's arrival with the expected bytes, the lse / delta warp
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -840,13 +841,23 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
             break;
           }
           fence_after_sync();
-          uint8_t* st = stage(s);
-          mma4(tb + cS + cBuf * b, Op{smem_u32(sK), 64, false}, Op{smem_u32(sKl), 64, false},
-               Op{smem_u32(st + S::sQ), QT, false}, Op{smem_u32(st + S::sQl), QT, false}, DQ, id_s, false, !SPLIT,
-               !SPLIT);
-          mma4(tb + cP + cBuf * b, Op{smem_u32(sV), 64, false}, Op{smem_u32(sVl), 64, false},
-               Op{smem_u32(st + S::sO), QT, false}, Op{smem_u32(st + S::sOl), QT, false}, DV, id_s, false, !SPLIT,
-               !SPLIT);
+          const uint32_t st = smem_u32(stage(s));
+          const uint32_t kh = smem_u32(sK), kl = smem_u32(sKl), vh = smem_u32(sV), vl = smem_u32(sVl);
+          const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
+                         ol = st + (uint32_t)S::sOl;
+          const uint32_t dS_ = tb + cS + cBuf * b, dP_ = tb + cP + cBuf * b;
+          for (int s2 = 0; s2 < DQ / 16; ++s2) mma_bf16(dS_, sw_desc_k(kh, 64, s2), sw_desc_k(qh, QT, s2), id_s, s2 ? 1u : 0u);
+          for (int s2 = 0; s2 < DV / 16; ++s2) mma_bf16(dP_, sw_desc_k(vh, 64, s2), sw_desc_k(oh, QT, s2), id_s, s2 ? 1u : 0u);
+          if constexpr (SPLIT) {
+            for (int s2 = 0; s2 < DQ / 16; ++s2) {
+              mma_bf16(dS_, sw_desc_k(kl, 64, s2), sw_desc_k(qh, QT, s2), id_s, 1u);
+              mma_bf16(dS_, sw_desc_k(kh, 64, s2), sw_desc_k(ql, QT, s2), id_s, 1u);
+            }
+            for (int s2 = 0; s2 < DV / 16; ++s2) {
+              mma_bf16(dP_, sw_desc_k(vl, 64, s2), sw_desc_k(oh, QT, s2), id_s, 1u);
+              mma_bf16(dP_, sw_desc_k(vh, 64, s2), sw_desc_k(ol, QT, s2), id_s, 1u);
+            }
+          }
           commit(&s_full[b]);
         }
         if (j >= 1) {  // dV, dK of query tile j - 1
@@ -856,13 +867,20 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
             break;
           }
           fence_after_sync();
-          uint8_t* st = stage(s);
-          mma4(tb + cDV, Op{smem_u32(sPh), 64, false}, Op{smem_u32(sPl), 64, false},
-               Op{smem_u32(st + S::sO), QT, true}, Op{smem_u32(st + S::sOl), QT, true}, QT, id_dv, jp > 0, false,
-               !SPLIT);
-          mma4(tb + cDK, Op{smem_u32(sDh), 64, false}, Op{smem_u32(sDl), 64, false},
-               Op{smem_u32(st + S::sQ), QT, true}, Op{smem_u32(st + S::sQl), QT, true}, QT, id_dk, jp > 0, false,
-               !SPLIT);
+          const uint32_t st = smem_u32(stage(s));
+          const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
+                         ol = st + (uint32_t)S::sOl;
+          const Op ph{smem_u32(sPh), 64, false}, pl{smem_u32(sPl), 64, false};
+          const Op gh{smem_u32(sDh), 64, false}, gl{smem_u32(sDl), 64, false};
+          for (int s2 = 0; s2 < QT / 16; ++s2) {
+            const uint32_t acc = (jp > 0 || s2) ? 1u : 0u;
+            mma_bf16(tb + cDV, op_desc(ph, s2), sw_desc_mn(oh, QT, s2), id_dv, acc);
+            mma_bf16(tb + cDV, op_desc(pl, s2), sw_desc_mn(oh, QT, s2), id_dv, 1u);
+            if constexpr (SPLIT) mma_bf16(tb + cDV, op_desc(ph, s2), sw_desc_mn(ol, QT, s2), id_dv, 1u);
+            mma_bf16(tb + cDK, op_desc(gh, s2), sw_desc_mn(qh, QT, s2), id_dk, acc);
+            mma_bf16(tb + cDK, op_desc(gl, s2), sw_desc_mn(qh, QT, s2), id_dk, 1u);
+            if constexpr (SPLIT) mma_bf16(tb + cDK, op_desc(gh, s2), sw_desc_mn(ql, QT, s2), id_dk, 1u);
+          }
           commit(&p_empty);   // P^T, dS^T may be overwritten
           commit(&empty[s]);  // the stage may be refilled
         }
@@ -870,52 +888,54 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       commit(&done_bar);  // arrives once every MMA issued above has completed
       if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
     }
-  } else if (w < 4) {  // ------------------------------------------------ loads (96 threads)
-    const int p = tid - 32;
-    auto krows = [&](const bf* base, int width) {
-      return [=](int a) -> const bf* { return a < nk && base ? base + ((size_t)(k0 + a) * H + h) * width : nullptr; };
-    };
-    int j = 0;
-    for (; j < n_tiles; ++j) {
-      const int s = j % NS;
-      if (j >= NS && !mbar_wait(&empty[s], ((j / NS) - 1) & 1)) {
-        give_up();
-        break;
-      }
-      if (aborted()) break;
-      if (j == 0) {  // K, V travel with the first query tile
-        tile_async_t<64, DQ, NP>(sK, krows(k, DQ), k, p);
-        tile_async_t<64, DV, NP>(sV, krows(v, DV), v, p);
-        if constexpr (SPLIT) {
-          tile_async_t<64, DQ, NP>(sKl, krows(k_lo, DQ), k, p);
-          tile_async_t<64, DV, NP>(sVl, krows(v_lo, DV), v, p);
+  } else if (w <= 2) {  // ------------------------------------------------ loads
+    // warp 1 (one thread): TMA of K, V (with the first query tile) and of each query tile's Q, dO;
+    // warp 2: lse and delta of the tile (rows past the subtree are masked, past the tensor zero)
+    const bool tma = w == 1;
+    if (!tma || lane == 0) {
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(&empty[s], ((j / NS) - 1) & 1)) {
+          give_up();
+          break;
+        }
+        if (aborted()) break;
+        const int q0 = k0 + j * QT, nq = min(QT, q_end - q0);
+        uint8_t* st = stage(s);
+        if (tma) {
+          const uint32_t kv = j == 0 ? (uint32_t)(SPLIT ? 2 : 1) * (uint32_t)(S::Kb + S::Vb) : 0u;
+          mbar_arrive_expect_tx(&full[s], kv + (uint32_t)(SPLIT ? 2 : 1) * (uint32_t)(S::Qb + S::Ob));
+          if (j == 0) {
+            for (int c = 0; c < DQ / 64; ++c) {
+              tma_load_3d(sK + c * 64 * 128, &tm_k, 64 * c, h, k0, &full[s]);
+              if constexpr (SPLIT) tma_load_3d(sKl + c * 64 * 128, &tm_kl, 64 * c, h, k0, &full[s]);
+            }
+            for (int c = 0; c < DV / 64; ++c) {
+              tma_load_3d(sV + c * 64 * 128, &tm_v, 64 * c, h, k0, &full[s]);
+              if constexpr (SPLIT) tma_load_3d(sVl + c * 64 * 128, &tm_vl, 64 * c, h, k0, &full[s]);
+            }
+          }
+          for (int c = 0; c < DQ / 64; ++c) {
+            tma_load_3d(st + S::sQ + c * QT * 128, &tm_q, 64 * c, h, q0, &full[s]);
+            if constexpr (SPLIT) tma_load_3d(st + S::sQl + c * QT * 128, &tm_ql, 64 * c, h, q0, &full[s]);
+          }
+          for (int c = 0; c < DV / 64; ++c) {
+            tma_load_3d(st + S::sO + c * QT * 128, &tm_o, 64 * c, h, q0, &full[s]);
+            if constexpr (SPLIT) tma_load_3d(st + S::sOl + c * QT * 128, &tm_ol, 64 * c, h, q0, &full[s]);
+          }
+        } else {
+          const size_t src = (size_t)(q0 + min(lane, nq - 1)) * H + h;
+          cp_async4(st + S::sL + 4 * lane, lse + src, lane < nq ? 4u : 0u);
+          cp_async4(st + S::sD + 4 * lane, delta + src, lane < nq ? 4u : 0u);
+          cp_async_commit();
+          cp_async_wait<0>();
+          mbar_arrive(&full[s]);
         }
       }
-      const int q0 = k0 + j * QT, nq = min(QT, q_end - q0);
-      auto rows = [=](const bf* base, int width) {
-        return [=](int a) -> const bf* { return a < nq && base ? base + ((size_t)(q0 + a) * H + h) * width : nullptr; };
-      };
-      uint8_t* st = stage(s);
-      tile_async_t<QT, DQ, NP>(st + S::sQ, rows(q, DQ), q, p);
-      tile_async_t<QT, DV, NP>(st + S::sO, rows(d_o, DV), d_o, p);
-      if constexpr (SPLIT) {
-        tile_async_t<QT, DQ, NP>(st + S::sQl, rows(q_lo, DQ), q, p);
-        tile_async_t<QT, DV, NP>(st + S::sOl, rows(d_o_lo, DV), d_o, p);
-      }
-      if (p < 2 * QT) {
-        const int c = p % QT;
-        const float* src = (p < QT ? lse : delta) + (size_t)(q0 + min(c, nq - 1)) * H + h;
-        cp_async4(st + (p < QT ? S::sL : S::sD) + 4 * c, src, c < nq ? 4u : 0u);
-      }
-      // publish the stage to the tensor core and the P / dS warps as soon as it has landed
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_async_smem();
-      mbar_arrive(&full[s]);
+      if (!tma) cp_async_wait<0>();
     }
-    cp_async_wait<0>();
-  } else {  // ------------------------------------------------ P^T, dS^T (warps 4-11)
-    const int sp = w & 3, half = (w - 4) >> 2;
+  } else if (w >= 3) {  // ------------------------------------------------ P^T, dS^T (warps 3-10)
+    const int sp = w & 3, half = (w - 3) >> 2;
     const int r = lane < 16 ? 16 * sp + lane : -1;  // key row of this thread (M = 64 layout)
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
     bool ok = true;

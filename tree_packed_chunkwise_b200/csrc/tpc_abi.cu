@@ -799,6 +799,20 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
   using bf = __nv_bfloat16;
   const dim3 gq((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest
   const dim3 gk((unsigned)(p.attn_ktiles.size() * (size_t)s->H));  // (key tile, head), key tiles fastest
+  const uint64_t NR = (uint64_t)p.n_unique;
+  const unsigned Hh = (unsigned)s->H;
+  CUtensorMap tk, tkl, tv, tvl, to, tol, tq32, tql32, to32, tol32;
+  bool ok = tensor_map_rows(&tk, k, tpc::kAttnQK, Hh, NR, 64) && tensor_map_rows(&tv, v, tpc::kAttnDV, Hh, NR, 64) &&
+            tensor_map_rows(&tkl, L.k ? L.k : k, tpc::kAttnQK, Hh, NR, 64) &&
+            tensor_map_rows(&tvl, L.v ? L.v : v, tpc::kAttnDV, Hh, NR, 64) &&
+            tensor_map_rows(&to, d_o, tpc::kAttnDV, Hh, NR, 128) &&
+            tensor_map_rows(&tol, L.d_o ? L.d_o : d_o, tpc::kAttnDV, Hh, NR, 128);
+  constexpr uint32_t QT = tpc::AttnDkvSmem<true>::QT;
+  ok = ok && tensor_map_rows(&tq32, q, tpc::kAttnQK, Hh, NR, QT) &&
+       tensor_map_rows(&tql32, L.q ? L.q : q, tpc::kAttnQK, Hh, NR, QT) &&
+       tensor_map_rows(&to32, d_o, tpc::kAttnDV, Hh, NR, QT) &&
+       tensor_map_rows(&tol32, L.d_o ? L.d_o : d_o, tpc::kAttnDV, Hh, NR, QT);
+  if (!ok) return fail(TPC_ERR_CUDA, "attention backward: cuTensorMapEncodeTiled failed");
   auto go = [&](auto tio, auto split) -> int {
     using T = decltype(tio);
     constexpr bool SP = decltype(split)::value;
@@ -807,12 +821,12 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
     TPC_CUDA(set_smem(tpc::attn_bwd_dkv_tc<T, SP>, sk));
     TPC_LAUNCH("attn_bwd_dq_tc", st,
                (tpc::attn_bwd_dq_tc<T, SP><<<gq, tpc::kAttnDqThreads, sq, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
-                   (const bf*)L.v, (const T*)o, lse, (const bf*)d_o, (const bf*)L.d_o, (T*)dq, delta, status)));
+                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, tk, tkl, tv, tvl, to, tol, (const T*)o, lse,
+                   (const bf*)d_o, (const bf*)L.d_o, (T*)dq, delta, status)));
     TPC_LAUNCH("attn_bwd_dkv_tc", st,
                (tpc::attn_bwd_dkv_tc<T, SP><<<gk, tpc::kAttnDkvThreads, sk, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, (const bf*)k, (const bf*)L.k, (const bf*)v,
-                   (const bf*)L.v, lse, (const bf*)d_o, (const bf*)L.d_o, delta, (T*)dk, (T*)dv, status)));
+                   p.dt, s->H, s->scale, tq32, tql32, tk, tkl, tv, tvl, to32, tol32, lse, delta, (T*)dk, (T*)dv,
+                   status)));
     return TPC_OK;
   };
   using Y = std::true_type;
