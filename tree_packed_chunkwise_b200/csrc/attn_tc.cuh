@@ -740,26 +740,26 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------ backward dK, dV
-// per key tile of node u (<= 64 rows): query rows [row of the tile, subtree end of u) in tiles of 32
+// per key tile of node u (<= 128 rows): query rows [row of the tile, subtree end of u) in tiles of 32
 // (queries of u itself only from the key row on), S^T = K Q^T, dP^T = V dO^T, P^T = exp(scale S^T -
-// lse), dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 64 accumulators.
+// lse), dS^T = P^T (dP^T - delta); dV += P^T dO, dK += dS^T Q; dk = scale dK.  M = 128 accumulators.
 //
-// Warp-specialised: warp 0 issues the MMAs, warp 1 streams K, V and then the query tiles (Q, dO and
-// their lo parts) through a three-stage ring by TMA (128-byte-swizzled boxes of 64 features), warp 2
-// adds lse and delta of each query tile by cp.async, warps 3-10 turn S^T and dP^T into P^T and dS^T.  S^T / dP^T have two TMEM buffers, so the products of query tile j + 1 run on the
-// tensor core while the P / dS math of tile j runs on the SIMT cores; the dV / dK products of tile j
-// follow once its P^T and dS^T are in shared memory.  Every wait is bounded; a timeout records
+// Warp-specialised: warp 0 issues the MMAs, warp 1 loads K and then streams the query tiles (Q, dO
+// and their lo parts) through a two-stage ring by TMA (128-byte-swizzled boxes of 64 features),
+// warp 2 adds lse and delta of each query tile by cp.async, warps 3-10 load V into TMEM (the A
+// operand of dP^T) and turn S^T, dP^T into P^T, dS^T.  The products of query tile j + 1 run on the
+// tensor core while the P / dS math of tile j runs.  Every wait is bounded; a timeout records
 // TPC_ERR_TIMEOUT and every role stops.
 template <bool SPLIT>
 struct AttnDkvSmem {
-  static constexpr int QT = 32, NS = 3;  // query rows per tile, ring stages
-  static constexpr size_t X = SPLIT ? 1 : 0;
-  static constexpr size_t Kb = size_t(64) * kAttnQK * 2, Vb = size_t(64) * kAttnDV * 2;
-  static constexpr size_t Qb = size_t(QT) * kAttnQK * 2, Ob = size_t(QT) * kAttnDV * 2, Pb = size_t(64) * QT * 2;
+  static constexpr int KT = 128, QT = 32, NS = 2;  // key rows, query rows per tile, ring stages
+  static constexpr size_t X = SPLIT ? 2 : 1;
+  static constexpr size_t Kb = size_t(KT) * kAttnQK * 2;
+  static constexpr size_t Qb = size_t(QT) * kAttnQK * 2, Ob = size_t(QT) * kAttnDV * 2, Pb = size_t(KT) * QT * 2;
   // one ring stage: Q, Q_lo, dO, dO_lo (swizzled boxes), lse[QT], delta[QT]; stages 1024-byte aligned
-  static constexpr size_t sQ = 0, sQl = sQ + Qb, sO = sQl + X * Qb, sOl = sO + Ob, sL = sOl + X * Ob, sD = sL + QT * 4;
+  static constexpr size_t sQ = 0, sQl = sQ + Qb, sO = sQ + X * Qb, sOl = sO + Ob, sL = sO + X * Ob, sD = sL + QT * 4;
   static constexpr size_t stage = (sD + QT * 4 + 1023) & ~size_t(1023);
-  static constexpr size_t K = 0, Kl = K + Kb, V = Kl + X * Kb, Vl = V + Vb, ring = Vl + X * Vb;
+  static constexpr size_t K = 0, ring = K + X * Kb;
   static constexpr size_t P = ring + NS * stage, Pl = P + Pb, dS = Pl + Pb, dSl = dS + Pb;
   static constexpr size_t total = dSl + Pb + 1024;  // + slack to align the boxes to 1024 bytes
   static_assert(total <= 227 * 1024, "shared memory");
@@ -770,22 +770,21 @@ constexpr int kAttnDkvThreads = 352;
 
 template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnDkvThreads, 1)
-    attn_bwd_dkv_tc(DevTables t, int H, float scale,
-                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ql,
-                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kl,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_vl,
-                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_ol,
-                    const float* __restrict__ lse, const float* __restrict__ delta, Tio* __restrict__ dk,
-                    Tio* __restrict__ dv, int* status) {
+    attn_bwd_dkv_tc(DevTables t, int H, float scale, const __nv_bfloat16* __restrict__ v,
+                    const __nv_bfloat16* __restrict__ v_lo, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_ql, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_o,
+                    const __grid_constant__ CUtensorMap tm_ol, const float* __restrict__ lse,
+                    const float* __restrict__ delta, Tio* __restrict__ dk, Tio* __restrict__ dv, int* status) {
   using namespace tck;
   using namespace tc;
   using S = AttnDkvSmem<SPLIT>;
   using bf = __nv_bfloat16;
-  constexpr int DQ = kAttnQK, DV = kAttnDV, QT = S::QT, NS = S::NS;
+  constexpr int DQ = kAttnQK, DV = kAttnDV, KT = S::KT, QT = S::QT, NS = S::NS;
   constexpr float kLog2e = 1.4426950408889634f;
   const float sl2 = scale * kLog2e;
-  // TMEM columns: dV (128), dK (192), then two buffers of S^T (32) and dP^T (32)
-  constexpr uint32_t cDV = 0, cDK = 128, cS = 320, cP = 352, cBuf = 64;
+  // TMEM columns: dV (128), dK (192), V hi (64) and lo (64) as bf16 pairs, S^T (32), dP^T (32)
+  constexpr uint32_t cDV = 0, cDK = 128, cVh = 320, cVl = 384, cS = 448, cP = 480;
   // grid: one block per (key tile, head), key tiles fastest, so that the blocks resident at one
   // time read the same head's query rows (shared in L2); the planner lists the key tiles of a head
   // by decreasing work, so the longest blocks start first
@@ -798,10 +797,10 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(1024) uint8_t asmem_raw[];
   uint8_t* asmem = asmem_raw + ((1024u - (smem_u32(asmem_raw) & 1023u)) & 1023u);  // 1024-byte aligned boxes
-  __shared__ __align__(8) uint64_t full[NS], empty[NS], s_full[2], s_empty[2], p_full, p_empty, done_bar;
+  __shared__ __align__(8) uint64_t full[NS], empty[NS], v_ready, s_full, s_read, p_full, p_empty, done_bar;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
-  uint8_t *sK = asmem + S::K, *sKl = asmem + S::Kl, *sV = asmem + S::V, *sVl = asmem + S::Vl;
+  uint8_t *sK = asmem + S::K, *sKl = sK + S::Kb;
   uint8_t *sPh = asmem + S::P, *sPl = asmem + S::Pl, *sDh = asmem + S::dS, *sDl = asmem + S::dSl;
   auto stage = [&](int s) { return asmem + S::ring + (size_t)s * S::stage; };
   if (w == 0) tmem_alloc(&tslot, 512);
@@ -810,10 +809,9 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       mbar_init(&full[s], 33);  // the TMA thread's arrival with the expected bytes, the lse / delta warp
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 8);  // one arrival per P / dS warp
-    }
+    mbar_init(&v_ready, 8);  // one arrival per P / dS warp
+    mbar_init(&s_full, 1);
+    mbar_init(&s_read, 8);
     mbar_init(&p_full, 8);
     mbar_init(&p_empty, 1);
     mbar_init(&done_bar, 1);
@@ -831,34 +829,35 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
 
   if (w == 0) {
     if (lane == 0) {  // ------------------------------------------------ MMA issuer
-      const uint32_t id_s = idesc_bf16(64, QT, false, false);
-      const uint32_t id_dv = idesc_bf16(64, DV, false, true), id_dk = idesc_bf16(64, DQ, false, true);
-      for (int j = 0; j <= n_tiles && !aborted(); ++j) {
-        if (j < n_tiles) {  // S^T, dP^T of query tile j (stage j % NS also holds K, V before tile 0)
-          const int s = j % NS, b = j & 1;
-          if (!mbar_wait(&full[s], (j / NS) & 1) || (j >= 2 && !mbar_wait(&s_empty[b], ((j >> 1) - 1) & 1))) {
+      const uint32_t id_s = idesc_bf16(128, QT, false, false);
+      const uint32_t id_dv = idesc_bf16(128, DV, false, true), id_dk = idesc_bf16(128, DQ, false, true);
+      bool ok = mbar_wait(&v_ready, 0);
+      if (!ok) give_up();
+      for (int j = 0; ok && j <= n_tiles && !aborted(); ++j) {
+        if (j < n_tiles) {  // S^T, dP^T of query tile j (stage 0 also brings K before tile 0)
+          const int s = j % NS;
+          if (!mbar_wait(&full[s], (j / NS) & 1) || (j >= 1 && !mbar_wait(&s_read, (j - 1) & 1))) {
             give_up();
             break;
           }
           fence_after_sync();
           const uint32_t st = smem_u32(stage(s));
-          const uint32_t kh = smem_u32(sK), kl = smem_u32(sKl), vh = smem_u32(sV), vl = smem_u32(sVl);
+          const uint32_t kh = smem_u32(sK), kl = smem_u32(sKl);
           const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
                          ol = st + (uint32_t)S::sOl;
-          const uint32_t dS_ = tb + cS + cBuf * b, dP_ = tb + cP + cBuf * b;
-          for (int s2 = 0; s2 < DQ / 16; ++s2) mma_bf16(dS_, sw_desc_k(kh, 64, s2), sw_desc_k(qh, QT, s2), id_s, s2 ? 1u : 0u);
-          for (int s2 = 0; s2 < DV / 16; ++s2) mma_bf16(dP_, sw_desc_k(vh, 64, s2), sw_desc_k(oh, QT, s2), id_s, s2 ? 1u : 0u);
+          for (int s2 = 0; s2 < DQ / 16; ++s2) mma_bf16(tb + cS, sw_desc_k(kh, KT, s2), sw_desc_k(qh, QT, s2), id_s, s2 ? 1u : 0u);
+          for (int s2 = 0; s2 < DV / 16; ++s2) mma_bf16_ts(tb + cP, tb + cVh + 8 * s2, sw_desc_k(oh, QT, s2), id_s, s2 ? 1u : 0u);
           if constexpr (SPLIT) {
             for (int s2 = 0; s2 < DQ / 16; ++s2) {
-              mma_bf16(dS_, sw_desc_k(kl, 64, s2), sw_desc_k(qh, QT, s2), id_s, 1u);
-              mma_bf16(dS_, sw_desc_k(kh, 64, s2), sw_desc_k(ql, QT, s2), id_s, 1u);
+              mma_bf16(tb + cS, sw_desc_k(kl, KT, s2), sw_desc_k(qh, QT, s2), id_s, 1u);
+              mma_bf16(tb + cS, sw_desc_k(kh, KT, s2), sw_desc_k(ql, QT, s2), id_s, 1u);
             }
             for (int s2 = 0; s2 < DV / 16; ++s2) {
-              mma_bf16(dP_, sw_desc_k(vl, 64, s2), sw_desc_k(oh, QT, s2), id_s, 1u);
-              mma_bf16(dP_, sw_desc_k(vh, 64, s2), sw_desc_k(ol, QT, s2), id_s, 1u);
+              mma_bf16_ts(tb + cP, tb + cVl + 8 * s2, sw_desc_k(oh, QT, s2), id_s, 1u);
+              mma_bf16_ts(tb + cP, tb + cVh + 8 * s2, sw_desc_k(ol, QT, s2), id_s, 1u);
             }
           }
-          commit(&s_full[b]);
+          commit(&s_full);
         }
         if (j >= 1) {  // dV, dK of query tile j - 1
           const int jp = j - 1, s = jp % NS;
@@ -870,8 +869,8 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
           const uint32_t st = smem_u32(stage(s));
           const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
                          ol = st + (uint32_t)S::sOl;
-          const Op ph{smem_u32(sPh), 64, false}, pl{smem_u32(sPl), 64, false};
-          const Op gh{smem_u32(sDh), 64, false}, gl{smem_u32(sDl), 64, false};
+          const Op ph{smem_u32(sPh), KT, false}, pl{smem_u32(sPl), KT, false};
+          const Op gh{smem_u32(sDh), KT, false}, gl{smem_u32(sDl), KT, false};
           for (int s2 = 0; s2 < QT / 16; ++s2) {
             const uint32_t acc = (jp > 0 || s2) ? 1u : 0u;
             mma_bf16(tb + cDV, op_desc(ph, s2), sw_desc_mn(oh, QT, s2), id_dv, acc);
@@ -889,7 +888,7 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
     }
   } else if (w <= 2) {  // ------------------------------------------------ loads
-    // warp 1 (one thread): TMA of K, V (with the first query tile) and of each query tile's Q, dO;
+    // warp 1 (one thread): TMA of K (with the first query tile) and of each query tile's Q, dO;
     // warp 2: lse and delta of the tile (rows past the subtree are masked, past the tensor zero)
     const bool tma = w == 1;
     if (!tma || lane == 0) {
@@ -903,16 +902,12 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
         const int q0 = k0 + j * QT, nq = min(QT, q_end - q0);
         uint8_t* st = stage(s);
         if (tma) {
-          const uint32_t kv = j == 0 ? (uint32_t)(SPLIT ? 2 : 1) * (uint32_t)(S::Kb + S::Vb) : 0u;
-          mbar_arrive_expect_tx(&full[s], kv + (uint32_t)(SPLIT ? 2 : 1) * (uint32_t)(S::Qb + S::Ob));
+          const uint32_t kb = j == 0 ? (uint32_t)(SPLIT ? 2 : 1) * (uint32_t)S::Kb : 0u;
+          mbar_arrive_expect_tx(&full[s], kb + (uint32_t)(SPLIT ? 2 : 1) * (uint32_t)(S::Qb + S::Ob));
           if (j == 0) {
             for (int c = 0; c < DQ / 64; ++c) {
-              tma_load_3d(sK + c * 64 * 128, &tm_k, 64 * c, h, k0, &full[s]);
-              if constexpr (SPLIT) tma_load_3d(sKl + c * 64 * 128, &tm_kl, 64 * c, h, k0, &full[s]);
-            }
-            for (int c = 0; c < DV / 64; ++c) {
-              tma_load_3d(sV + c * 64 * 128, &tm_v, 64 * c, h, k0, &full[s]);
-              if constexpr (SPLIT) tma_load_3d(sVl + c * 64 * 128, &tm_vl, 64 * c, h, k0, &full[s]);
+              tma_load_3d(sK + c * KT * 128, &tm_k, 64 * c, h, k0, &full[s]);
+              if constexpr (SPLIT) tma_load_3d(sKl + c * KT * 128, &tm_kl, 64 * c, h, k0, &full[s]);
             }
           }
           for (int c = 0; c < DQ / 64; ++c) {
@@ -935,8 +930,10 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       if (!tma) cp_async_wait<0>();
     }
   } else if (w >= 3) {  // ------------------------------------------------ P^T, dS^T (warps 3-10)
-    const int sp = w & 3, half = (w - 3) >> 2;
-    const int r = lane < 16 ? 16 * sp + lane : -1;  // key row of this thread (M = 64 layout)
+    // warp w holds the TMEM lanes (key rows) of sub-partition w % 4 and the query columns of half
+    // (w - 3) / 4 of each tile (and of dV / dK at the end)
+    const int sp = w & 3, half = (w - 3) >> 2, r = 32 * sp + lane;
+    const bool in = r < nk;
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
     bool ok = true;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
@@ -944,16 +941,42 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       if (!got && lane == 0) give_up();
       return got && !__any_sync(0xffffffffu, aborted());
     };
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j % NS, b = j & 1;
-      if (!(ok = wait_all(&s_full[b], (j >> 1) & 1))) break;
-      fence_after_sync();
-      float sv[16], dp[16];
-      tmem_ld16(la + cS + cBuf * b + 16 * half, sv);
-      tmem_ld16(la + cP + cBuf * b + 16 * half, dp);
+    {  // this half of the key row's V (and its lo part) into TMEM: a bf16 pair per 32-bit column
+      for (int part = 0; part < (SPLIT ? 2 : 1); ++part) {
+        const bf* src = part ? v_lo : v;
+        const uint4* g4 =
+            (in && src) ? reinterpret_cast<const uint4*>(src + ((size_t)(k0 + r) * H + h) * DV) + 8 * half : nullptr;
+        uint32_t rr[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 x = g4 ? g4[i] : make_uint4(0u, 0u, 0u, 0u);
+          rr[4 * i] = x.x; rr[4 * i + 1] = x.y; rr[4 * i + 2] = x.z; rr[4 * i + 3] = x.w;
+        }
+        tmem_st32_nowait(la + (part ? cVl : cVh) + 32 * half, rr);
+      }
+      tmem_wait_st();
       fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[b]);
+      if (lane == 0) mbar_arrive(&v_ready);
+    }
+    for (int j = 0; j < n_tiles; ++j) {
+      const int s = j % NS;
+      if (!(ok = wait_all(&s_full, j & 1))) break;
+      fence_after_sync();
+      uint32_t rs[16], rp[16];
+      {
+        float a[16], b[16];
+        tmem_ld16(la + cS + 16 * half, a);
+        tmem_ld16(la + cP + 16 * half, b);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          rs[c] = __float_as_uint(a[c]);
+          rp[c] = __float_as_uint(b[c]);
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_read);  // S^T, dP^T may take the next tile
       if (!(ok = wait_all(&full[s], (j / NS) & 1))) break;  // lse and delta of the tile
       const uint8_t* st = stage(s);
       const float* sl = reinterpret_cast<const float*>(st + S::sL);
@@ -961,37 +984,34 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       const int q0 = k0 + j * QT, nq = min(QT, q_end - q0);
       // P^T and dS^T of this thread's 16 entries as packed bf16 hi / lo pairs (base-2 exponentials)
       uint32_t ph[8], pl[8], gh[8], gl[8];
-      if (r >= 0) {
 #pragma unroll
-        for (int jj = 0; jj < 16; jj += 2) {
-          float pv[2], dsv[2];
+      for (int jj = 0; jj < 16; jj += 2) {
+        float pv[2], dsv[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 16 * half + jj + e, qrow = q0 + c;
-            const bool valid = r < nk && c < nq && !(qrow < own_end && qrow < k0 + r);
-            pv[e] = valid ? exp2f(fmaf(sv[jj + e], sl2, -sl[c] * kLog2e)) : 0.f;
-            dsv[e] = pv[e] * (dp[jj + e] - sd[c]);
-          }
-          split2(pv[0], pv[1], ph[jj / 2], pl[jj / 2]);
-          split2(dsv[0], dsv[1], gh[jj / 2], gl[jj / 2]);
+        for (int e = 0; e < 2; ++e) {
+          const int c = 16 * half + jj + e, qrow = q0 + c;
+          const bool valid = in && c < nq && !(qrow < own_end && qrow < k0 + r);
+          pv[e] = valid ? exp2f(fmaf(__uint_as_float(rs[jj + e]), sl2, -sl[c] * kLog2e)) : 0.f;
+          dsv[e] = pv[e] * (__uint_as_float(rp[jj + e]) - sd[c]);
         }
+        split2(pv[0], pv[1], ph[jj / 2], pl[jj / 2]);
+        split2(dsv[0], dsv[1], gh[jj / 2], gl[jj / 2]);
       }
       if (j >= 1 && !(ok = wait_all(&p_empty, (j - 1) & 1))) break;  // dV, dK of tile j - 1 are done
-      if (r >= 0) {
-        put16_packed<64>(sPh, sPl, r, 16 * half, ph, pl);
-        put16_packed<64>(sDh, sDl, r, 16 * half, gh, gl);
-      }
+      put16_packed<KT>(sPh, sPl, r, 16 * half, ph, pl);
+      put16_packed<KT>(sDh, sDl, r, 16 * half, gh, gl);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full);
     }
     if (ok && n_tiles > 0) ok = wait_all(&p_empty, (n_tiles - 1) & 1);
     if (ok) {
+      fence_after_sync();
       const bool none = n_tiles == 0;
       for (int c = DV / 2 * half; c < DV / 2 * (half + 1); c += 32) {
         float g[32];
         tmem_ld32(la + cDV + c, g);
-        if (r >= 0 && r < nk) {
+        if (in) {
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) g[jj] = none ? 0.f : g[jj];
           Tio* dst = dv + ((size_t)(k0 + r) * H + h) * DV + c;
@@ -1002,7 +1022,7 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       for (int c = DQ / 2 * half; c < DQ / 2 * (half + 1); c += 32) {
         float g[32];
         tmem_ld32(la + cDK + c, g);
-        if (r >= 0 && r < nk) {
+        if (in) {
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) g[jj] = none ? 0.f : g[jj] * scale;
           Tio* dst = dk + ((size_t)(k0 + r) * H + h) * DQ + c;

@@ -50,7 +50,7 @@ struct RowRange {
   int32_t start, end;
 };
 struct AttnTile {
-  int32_t node, row, n, pad;  // n <= 128 query rows or <= 64 key rows of one node
+  int32_t node, row, n, pad;  // n <= 128 query or key rows of one node
 };
 
 // Device view of the uploaded tables (all pointers into the caller's buffer).

@@ -317,8 +317,8 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
       P.attn_nodes[v] = an;
       for (int32_t r = 0; r < length[v]; r += 128)
         P.attn_qtiles.push_back({v, (int32_t)P.row_offset[v] + r, std::min(128, length[v] - r), 0});
-      for (int32_t r = 0; r < length[v]; r += 64)
-        P.attn_ktiles.push_back({v, (int32_t)P.row_offset[v] + r, std::min(64, length[v] - r), 0});
+      for (int32_t r = 0; r < length[v]; r += 128)
+        P.attn_ktiles.push_back({v, (int32_t)P.row_offset[v] + r, std::min(128, length[v] - r), 0});
     }
     P.attn_nodes[n] = AttnNode{0, 0, 0, (int32_t)(P.attn_ranges.size() / 2), 0, {0, 0, 0}};
     // query tiles by decreasing work (the keys they read: the node's ancestor rows and its own rows up

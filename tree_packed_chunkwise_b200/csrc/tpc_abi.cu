@@ -812,6 +812,10 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
        tensor_map_rows(&tql32, L.q ? L.q : q, tpc::kAttnQK, Hh, NR, QT) &&
        tensor_map_rows(&to32, d_o, tpc::kAttnDV, Hh, NR, QT) &&
        tensor_map_rows(&tol32, L.d_o ? L.d_o : d_o, tpc::kAttnDV, Hh, NR, QT);
+  CUtensorMap tk128, tkl128;  // key tiles of the dK / dV kernel
+  constexpr uint32_t KT = tpc::AttnDkvSmem<true>::KT;
+  ok = ok && tensor_map_rows(&tk128, k, tpc::kAttnQK, Hh, NR, KT) &&
+       tensor_map_rows(&tkl128, L.k ? L.k : k, tpc::kAttnQK, Hh, NR, KT);
   if (!ok) return fail(TPC_ERR_CUDA, "attention backward: cuTensorMapEncodeTiled failed");
   auto go = [&](auto tio, auto split) -> int {
     using T = decltype(tio);
@@ -825,8 +829,8 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
                    (const bf*)d_o, (const bf*)L.d_o, (T*)dq, delta, status)));
     TPC_LAUNCH("attn_bwd_dkv_tc", st,
                (tpc::attn_bwd_dkv_tc<T, SP><<<gk, tpc::kAttnDkvThreads, sk, st>>>(
-                   p.dt, s->H, s->scale, tq32, tql32, tk, tkl, tv, tvl, to32, tol32, lse, delta, (T*)dk, (T*)dv,
-                   status)));
+                   p.dt, s->H, s->scale, (const bf*)v, (const bf*)L.v, tq32, tql32, tk128, tkl128, to32, tol32, lse,
+                   delta, (T*)dk, (T*)dv, status)));
     return TPC_OK;
   };
   using Y = std::true_type;
