@@ -459,9 +459,10 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
 //   warp 0      issues S_j = Q K_j^T, then dQ += dS_{j-1} K_{j-1}, then dP_j = dO V_j^T;
 //   warp 1      streams K_j through a two-stage ring; warp 2 loads dO once, then streams V_j (TMA,
 //               128-byte-swizzled boxes of 64 features);
-//   warps 3-10  two threads per query row (key columns in halves): Q into TMEM once, delta; per key
-//               tile they read S_j (releasing it for S_{j+1}) and dP_j, and write dS_j as a bf16
-//               hi/lo pair over their own dP_j columns (the A operand of the dQ product).
+//   warps 3-18  four threads per query row (key columns in quarters of 16): Q into TMEM once, delta;
+//               per key tile they read S_j (releasing it for S_{j+1}) and dP_j, and write dS_j as
+//               bf16 hi/lo pairs over their own 16 dP_j columns (hi in the first 8, lo in the last 8:
+//               the A operand of the dQ product, one K step per quarter).
 template <bool SPLIT>
 struct AttnDqSmem {
   static constexpr int NK = 2, NV = 2;
@@ -472,7 +473,7 @@ struct AttnDqSmem {
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
-constexpr int kAttnDqThreads = 352;
+constexpr int kAttnDqThreads = 608;
 
 template <typename Tio, bool SPLIT>
 __global__ void __launch_bounds__(kAttnDqThreads, 1)
@@ -516,11 +517,11 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
       mbar_init(&vempty[s], 1);
     }
     mbar_init(&do_full, 1);
-    mbar_init(&q_ready, 8);  // one arrival per softmax warp
+    mbar_init(&q_ready, 8);  // one arrival per warp of the first two column quarters
     mbar_init(&s_full, 1);
-    mbar_init(&s_read, 8);
+    mbar_init(&s_read, 16);  // one arrival per P / dS warp
     mbar_init(&dp_full, 1);
-    mbar_init(&ds_full, 8);
+    mbar_init(&ds_full, 16);
     mbar_init(&dq_done, 1);
     mbar_init(&done_bar, 1);
     abort_flag = 0;
@@ -573,9 +574,9 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
           }
           fence_after_sync();
           const uint32_t kh = smem_u32(kst(ks)), kl = kh + (uint32_t)S::Kb;
-          auto a_hi = [&](int s) { return tb + cP + 32 * (s >> 1) + 8 * (s & 1); };
+          auto a_hi = [&](int s) { return tb + cP + 16 * s; };  // K step s: keys 16 s .. 16 s + 15
           for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), sw_desc_mn(kh, 64, s), id_g, (jp > 0 || s) ? 1u : 0u);
-          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s) + 16, sw_desc_mn(kh, 64, s), id_g, 1u);
+          for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s) + 8, sw_desc_mn(kh, 64, s), id_g, 1u);
           if constexpr (SPLIT)
             for (int s = 0; s < 4; ++s) mma_bf16_ts(tb + cG, a_hi(s), sw_desc_mn(kl, 64, s), id_g, 1u);
           commit(&kempty[ks]);
@@ -634,8 +635,8 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
         }
       }
     }
-  } else if (w >= 3) {  // ------------------------------------------------ P, dS (warps 3-10)
-    const int sp = w & 3, half = (w - 3) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
+  } else if (w >= 3) {  // ------------------------------------------------ P, dS (warps 3-18)
+    const int sp = w & 3, quarter = (w - 3) >> 2, row = 32 * sp + lane, qrow = qt.row + row;
     const bool in = row < qt.n;
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
     const float sl2 = scale * kLog2e;
@@ -644,7 +645,8 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
       if (!got && lane == 0) give_up();
       return got && !__any_sync(0xffffffffu, aborted());
     };
-    {  // this half of Q (and its lo part) into TMEM
+    if (quarter < 2) {  // half `quarter` of Q (and its lo part) into TMEM
+      const int half = quarter;
       constexpr int HC = DQ / 4;
       for (int part = 0; part < (SPLIT ? 2 : 1); ++part) {
         const bf* src = part ? q_lo : q;
@@ -673,7 +675,7 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
       const bf* glow = SPLIT && d_o_lo ? d_o_lo + ((size_t)qrow * H + h) * DV : nullptr;
       for (int c = 0; c < DV; ++c)
         dl = fmaf(to_f(orow[c]), __bfloat162float(grow[c]) + (glow ? __bfloat162float(glow[c]) : 0.f), dl);
-      if (half == 0) delta[(size_t)qrow * H + h] = dl;
+      if (quarter == 0) delta[(size_t)qrow * H + h] = dl;
       ls2 = lse[(size_t)qrow * H + h] * kLog2e;
     }
     KeyTileIter<64> it;
@@ -684,34 +686,30 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
       it.next(k0, nk, own);
       if (!(ok = wait_all(&s_full, j & 1)) || !(ok = wait_all(&dp_full, j & 1))) break;
       fence_after_sync();
-      uint32_t rs[32], rp[32];
-      tmem_ld32_nowait(la + cS + 32 * half, rs);
-      tmem_ld32_nowait(la + cP + 32 * half, rp);
-      tmem_wait_ld();
+      float rs[16], rp[16];
+      tmem_ld16(la + cS + 16 * quarter, rs);
+      tmem_ld16(la + cP + 16 * quarter, rp);
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_read);  // S may take S_{j+1}
       const bool masked = !in || own || nk < 64;
-      float gh[16], gl[16];
+      float g[16];  // dS of the quarter's 16 keys: 8 hi pairs, then 8 lo pairs
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
+      for (int c = 0; c < 16; c += 2) {
         float ds[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int kc = 32 * half + c + e;
+          const int kc = 16 * quarter + c + e;
           const bool valid = !masked || (in && kc < nk && !(own && k0 + kc > qrow));
-          const float pv = valid ? exp2f(__uint_as_float(rs[c + e]) * sl2 - ls2) : 0.f;
-          ds[e] = pv * (__uint_as_float(rp[c + e]) - dl);
+          const float pv = valid ? exp2f(rs[c + e] * sl2 - ls2) : 0.f;
+          ds[e] = pv * (rp[c + e] - dl);
         }
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(ds[0], ds[1]);
-        const float2 hf = __bfloat1622float2(hi);
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(ds[0] - hf.x, ds[1] - hf.y);
-        gh[c / 2] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&hi));
-        gl[c / 2] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&lo));
+        uint32_t hi, lo;
+        split2(ds[0], ds[1], hi, lo);
+        g[c / 2] = __uint_as_float(hi);
+        g[8 + c / 2] = __uint_as_float(lo);
       }
-      // dS over this half's own dP columns: hi in the first 16, lo in the last 16
-      tmem_st16(la + cP + 32 * half, gh);
-      tmem_st16(la + cP + 32 * half + 16, gl);
+      tmem_st16(la + cP + 16 * quarter, g);  // over this quarter's own dP columns
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full);
@@ -719,17 +717,13 @@ __global__ void __launch_bounds__(kAttnDqThreads, 1)
     if (ok && n_tiles > 0) ok = wait_all(&dq_done, (n_tiles - 1) & 1);
     if (ok) {
       fence_after_sync();
-      for (int c0 = 0; c0 < DQ / 2; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32_nowait(la + cG + DQ / 2 * half + c0, r);  // warp-collective: every row takes part
-        tmem_wait_ld();
+      for (int c0 = 0; c0 < DQ / 4; c0 += 16) {
+        float g[16];
+        tmem_ld16(la + cG + DQ / 4 * quarter + c0, g);  // warp-collective: every row takes part
         if (in) {
-          float g[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) g[c] = n_tiles > 0 ? __uint_as_float(r[c]) * scale : 0.f;
-          Tio* dst = dq + ((size_t)qrow * H + h) * DQ + DQ / 2 * half + c0;
-          st_out16(dst, g);
-          st_out16(dst + 16, g + 16);
+          for (int c = 0; c < 16; ++c) g[c] = n_tiles > 0 ? g[c] * scale : 0.f;
+          st_out16(dq + ((size_t)qrow * H + h) * DQ + DQ / 4 * quarter + c0, g);
         }
       }
     }
