@@ -4,40 +4,29 @@
 //
 // A query tile (<= 128 rows of one node) visits the node's ancestor row ranges (a few contiguous
 // ranges in the compact layout, one per chain on its path) and then its own node's rows up to the
-// tile's end with the causal mask.  Forward: S = Q K^T (bf16 inputs, exact products), online
-// softmax in fp32 (one query row per thread), O += P V with P a bf16 hi/lo pair.  Backward,
-// deterministic: dQ per query tile (S and dP = dO V^T recomputed, dQ += dS K accumulated in TMEM);
-// dK, dV per key tile (<= 64 rows of one node), looping over the query rows that can see it: the
-// node's subtree rows from the tile on, one contiguous range in the compact layout.
+// tile's end with the causal mask, in key tiles of 64.  Forward: S = Q K^T, online softmax in fp32,
+// O += P V with P a bf16 hi/lo pair.  Backward, deterministic (no atomics): dQ per query tile (S and
+// dP = dO V^T recomputed, dQ += dS K accumulated in TMEM); dK, dV per key tile (<= 128 rows of one
+// node), looping over the query rows that can see it: the node's subtree rows from the tile on, one
+// contiguous range in the compact layout.
+//
+// All three kernels are warp-specialised (one MMA-issuing thread, TMA loader threads, softmax
+// warps) with mbarrier-ordered pipelines and bounded waits.  Row tiles arrive by TMA from 3-D tensor
+// maps (rows x heads x features) as 128-byte-swizzled boxes of 64 features; the operand that stays
+// put for a whole block (Q in the forward and dQ, V in dK/dV) and the softmax outputs that feed a
+// product as its M side (P, dS) live in TMEM as A operands.
 //
 // SPLIT kernels take q, k, v and dO as bf16 hi/lo pairs (fp32 values x = hi + lo to 2^-17
 // relative) and form every product from three partial products (hi hi + lo hi + hi lo), so that
-// fp32 inputs and upstream gradients enter without a bf16 rounding of their own.  The dQ kernel
-// then walks the keys in tiles of 32 (the split tiles take twice the shared memory).
+// fp32 inputs and upstream gradients enter without a bf16 rounding of their own.
 #pragma once
 #include "kda_tc.cuh"
 
 namespace tpc {
 
-constexpr int kAttnQK = 192, kAttnDV = 128, kAttnThreads = 128;
+constexpr int kAttnQK = 192, kAttnDV = 128;
 
 namespace tck {
-
-// key tiles of a query tile: f(row start, rows, own-node flag) in a fixed order; stops on false
-template <int KT = 64, class F>
-__device__ __forceinline__ bool for_key_tiles(const DevTables& t, const AttnTile& qt, F f) {
-  const AttnNode nd = t.attn_nodes[qt.node];
-  const int r1 = t.attn_nodes[qt.node + 1].range_begin;
-  for (int r = nd.range_begin; r < r1; ++r) {
-    const RowRange rr = t.attn_ranges[r];
-    for (int k0 = rr.start; k0 < rr.end; k0 += KT)
-      if (!f(k0, min(KT, rr.end - k0), false)) return false;
-  }
-  const int end = qt.row + qt.n;
-  for (int k0 = nd.row_offset; k0 < end; k0 += KT)
-    if (!f(k0, min(KT, end - k0), true)) return false;
-  return true;
-}
 
 template <typename T>
 __device__ __forceinline__ void st_out16(T* p, const float* v) {
@@ -80,7 +69,8 @@ __device__ __forceinline__ void put16_packed(uint8_t* hi, uint8_t* lo, int a, in
 }  // namespace tck
 
 // ------------------------------------------------------------------------------------------ forward
-// Key tiles of a query tile, one at a time in the fixed order of for_key_tiles (for look-ahead).
+// Key tiles of a query tile, one at a time: the node's ancestor ranges in order, then its own rows up
+// to the tile's end.
 template <int KT>
 struct KeyTileIter {
   const RowRange* ranges;
@@ -112,34 +102,7 @@ struct KeyTileIter {
   }
 };
 
-// Asynchronous load of an A x B bf16 tile (rows from rowp(a), nullptr = zeros) into the
-// core-matrix layout; `any` is a valid global address used for the zero-filled rows.
-template <int A, int B, int NT, class RP>
-__device__ __forceinline__ void tile_async(uint8_t* dst, RP rowp, const void* any) {
-  constexpr int NCH = A * (B / 8);
-#pragma unroll 4
-  for (int e = threadIdx.x; e < NCH; e += NT) {
-    const int a = e % A, b0 = (e / A) * 8;
-    const __nv_bfloat16* p = rowp(a);
-    tc::cp_async16(dst + tc::cm_off(a, b0, A), p ? (const void*)(p + b0) : any, p ? 16u : 0u);
-  }
-}
 
-// Asynchronous load of an A x B bf16 tile (rows from rowp(a), nullptr = zeros) into the core-matrix
-// layout by NT threads (this one: t).  A warp moves 16 rows x 32 bytes (whole 32-byte sectors) and
-// writes four 128-byte lines of shared memory.  A, B multiples of 16.
-template <int A, int B, int NT, class RP>
-__device__ __forceinline__ void tile_async_t(uint8_t* dst, RP rowp, const void* any, int t) {
-  static_assert(A % 16 == 0 && B % 16 == 0, "tile shape");
-  constexpr int NCH = A * (B / 8), RB = A / 16;
-#pragma unroll 4
-  for (int e = t; e < NCH; e += NT) {
-    const int sub = e & 31, g = e >> 5;
-    const int a = 16 * (g % RB) + (sub >> 1), b0 = 8 * (2 * (g / RB) + (sub & 1));
-    const __nv_bfloat16* p = rowp(a);
-    tc::cp_async16(dst + tc::cm_off(a, b0, A), p ? (const void*)(p + b0) : any, p ? 16u : 0u);
-  }
-}
 
 // Forward, per query tile (<= 128 rows of one node) and head, warp-specialised:
 //   warp 0      issues the MMAs: S_j = Q K_j^T into one of two TMEM buffers, then O += P_j V_j;
