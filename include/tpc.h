@@ -257,6 +257,8 @@ int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B
  *   q, k: [N][H][d_qk], v: [N][H][d_v]; o: [N][H][d_v] and (backward) dq, dk, dv in io_dtype;
  *   lse: fp32 [N][H] (natural log of the softmax normaliser of scale * q.k).
  *   delta: caller scratch fp32 [N][H] (backward).  Built for d_qk = 192, d_v = 128.
+ *   q, k, v, d_o and their low parts are read by TMA: base pointers 16-byte aligned (a tensor map
+ *   that cannot be encoded returns TPC_ERR_CUDA before any launch).
  * Deterministic: the backward sums every gradient in a fixed order without atomics.
  */
 typedef struct tpc_attn_shape {
