@@ -7,7 +7,8 @@
 // three products in one TMEM accumulator: A_hi B_hi (+ A_lo B_hi) (+ A_hi B_lo); the dropped
 // A_lo B_lo term is below 2^-16 of the product.  The K loop simply runs once per product.
 //
-// One CTA per 128 x 256 output tile, K in steps of 64 through a 4-stage shared-memory pipeline:
+// Output tiles of 128 x 256 (K < 4096) or 256 x 256 (two 128-row halves, each an M = 128 MMA into
+// its own TMEM accumulator), K in steps of 64 through a 4- resp. 3-stage shared-memory pipeline:
 // a producer thread issues TMA loads into the 128-byte-swizzled canonical layout (K-major operand:
 // one box of 64 K x tile rows, each row one 128-byte line; MN-major operand: boxes of 64 M/N x 64 K,
 // each K row one 128-byte line), an MMA thread issues tcgen05.mma and frees stages by
@@ -20,7 +21,9 @@
 
 namespace tpc {
 
-constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4, kGemmThreads = 128;
+constexpr int kGemmBN = 256, kGemmBK = 64, kGemmThreads = 128;
+constexpr int kGemmHalf = 128;      // rows per MMA and per TMEM accumulator
+constexpr int kGemmLongK = 4096;    // K from which the 256-row tile is used
 // one MN-major 128-byte-swizzle block: 64 K rows of one 128-byte line
 constexpr uint32_t kSw128Atom = kGemmBK * 128;
 
@@ -36,10 +39,14 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t base, bool mn, int ks) {
          ((uint64_t)((1024u >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-struct GemmSmem {
-  static constexpr size_t Ab = size_t(kGemmBM) * kGemmBK * 2, Bb = size_t(kGemmBN) * kGemmBK * 2;
+// HV = 128-row halves per tile: 1 (two TMEM accumulators, the epilogue of a tile overlaps the next
+// tile's main loop) or 2 (both accumulators hold one tile; more K in flight per stage)
+template <int HV>
+struct GemmCfg {
+  static constexpr int BM = kGemmHalf * HV, stages = HV == 2 ? 3 : 4, nacc = HV == 2 ? 1 : 2;
+  static constexpr size_t Ab = size_t(BM) * kGemmBK * 2, Bb = size_t(kGemmBN) * kGemmBK * 2;
   static constexpr size_t stage = Ab + Bb;
-  static constexpr size_t total = kGemmStages * stage + 1024;  // + slack to align the stages to 1024 bytes
+  static constexpr size_t total = stages * stage + 1024;  // + slack to align the stages to 1024 bytes
 };
 
 struct GemmArgs {
@@ -56,21 +63,28 @@ struct GemmArgs {
 
 // Persistent, warp-specialised: grid = min(tiles, SMs); each CTA walks tiles blockIdx.x,
 // blockIdx.x + gridDim.x, ...  The tile order runs along the smaller of M and N fastest, so the
-// CTAs in flight share the tiles of the larger operand and the smaller one stays in L2.  Warp 0 lane 0 issues TMA loads into a 4-stage ring; warp 1 lane 0 issues the MMAs into one
-// of two TMEM accumulators (256 columns each); warps 2-5 drain the other accumulator to global
-// memory (thread = row), so a tile's epilogue overlaps the next tile's main loop.  Every wait is
-// bounded; a timeout records TPC_ERR_TIMEOUT and every role stops.
+// CTAs in flight share the tiles of the larger operand and the smaller one stays in L2.  Warp 0
+// lane 0 issues TMA loads into the stage ring; warp 1 lane 0 issues per 16-wide K step one MMA per
+// 128-row half.  HV = 1: two TMEM accumulators of 256 columns alternate between tiles, so warps
+// 2-5 drain one tile (thread = row) while the next one's main loop runs.  HV = 2: the two
+// accumulators hold the two halves of one tile and are drained (thread = one row of each half)
+// before the next tile starts; per MMA cycle this moves a third less operand data and keeps 1.5x
+// the MMA time in flight per stage, which pays once K is long.  Every wait is bounded; a timeout
+// records TPC_ERR_TIMEOUT and every role stops.
 constexpr int kGemmThreadsP = 192;
 
-template <int C_BF16>
+template <int C_BF16, int HV>
 __global__ void __launch_bounds__(kGemmThreadsP, 1)
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                  const __grid_constant__ CUtensorMap tma_alo, const __grid_constant__ CUtensorMap tma_blo, GemmArgs g) {
   using namespace tc;
+  using Cfg = GemmCfg<HV>;
+  constexpr int kGemmBM = Cfg::BM, kGemmStages = Cfg::stages, NACC = Cfg::nacc;
+  using GemmSmem = Cfg;
   extern __shared__ __align__(1024) uint8_t gsm_raw[];
   // the swizzle pattern is a function of the shared address: stages start on 1024-byte boundaries
   uint8_t* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
-  __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], acc_full[2], acc_empty[2], done_bar;
+  __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], acc_full[NACC], acc_empty[NACC], done_bar;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -86,7 +100,7 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
     }
@@ -134,13 +148,15 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
     }
   } else if (w == 1) {
     if (lane == 0) {  // MMA issuer
-      const uint32_t id = idesc_bf16(kGemmBM, kGemmBN, g.a_mn != 0, g.b_mn != 0);
+      const uint32_t id = idesc_bf16(kGemmHalf, kGemmBN, g.a_mn != 0, g.b_mn != 0);
+      // second 128-row half of the A stage: 128 lines on (K-major) or two 64-row blocks on (MN-major)
+      const uint32_t a_half = g.a_mn ? 2u * kSw128Atom : (uint32_t)kGemmHalf * 128u;
       int it_all = 0, local = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok && !aborted(); t += gridDim.x, ++local) {
-        const int b = local & 1;
-        // the epilogue has drained this accumulator (its previous use was tile local - 2)
-        if (local >= 2 && !mbar_wait(&acc_empty[b], ((local >> 1) - 1) & 1, 4000000000ull)) {
+        // the epilogue has drained this tile's accumulator(s) (their previous use: tile local - NACC)
+        const int b = local % NACC;
+        if (local >= NACC && !mbar_wait(&acc_empty[b], ((local / NACC) - 1) & 1, 4000000000ull)) {
           give_up();
           ok = false;
           break;
@@ -157,9 +173,13 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
           fence_after_sync();
           const uint32_t sa = smem_u32(gsm + s * GemmSmem::stage), sb = sa + (uint32_t)GemmSmem::Ab;
 #pragma unroll
-          for (int ks = 0; ks < kGemmBK / 16; ++ks)
-            mma_bf16(acc, sw128_desc(sa, g.a_mn != 0, ks), sw128_desc(sb, g.b_mn != 0, ks), id,
-                     (it > 0 || ks) ? 1u : 0u);
+          for (int ks = 0; ks < kGemmBK / 16; ++ks) {
+            const uint64_t db = sw128_desc(sb, g.b_mn != 0, ks);
+            const uint32_t accum = (it > 0 || ks) ? 1u : 0u;
+            mma_bf16(acc, sw128_desc(sa, g.a_mn != 0, ks), db, id, accum);
+            if constexpr (HV == 2)
+              mma_bf16(acc + (uint32_t)kGemmBN, sw128_desc(sa + a_half, g.a_mn != 0, ks), db, id, accum);
+          }
           commit(&empty[s]);
         }
         if (ok) commit(&acc_full[b]);
@@ -167,47 +187,50 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       commit(&done_bar);  // arrives once every MMA issued above has completed
       if (!mbar_wait(&done_bar, 0, 2000000000ull)) give_up();
     }
-  } else {  // epilogue warps 2..5: TMEM lanes of sub-partition w % 4
+  } else {  // epilogue warps 2..5: TMEM lanes of sub-partition w % 4, one row of each half
     const int sp = w & 3, row = 32 * sp + lane;
     int local = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
-      const int b = local & 1;
       // decisions are warp-uniform: the TMEM loads below are warp-collective
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (local >> 1) & 1, 4000000000ull));
+      const int b = local % NACC;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (local / NACC) & 1, 4000000000ull));
       if (!got) {
         if (lane == 0) give_up();
         break;
       }
       if (__any_sync(0xffffffffu, aborted())) break;
       fence_after_sync();
-      const int m = tile_m(t) * kGemmBM + row, n0 = tile_n(t) * kGemmBN;
-      const uint32_t la = tb + ((uint32_t)(32 * sp) << 16) + (uint32_t)(b * kGemmBN);
-      for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
-        float v[16];
-        tmem_ld16(la + c0, v);
-        if (m >= g.M || n0 + c0 >= g.N) continue;
-        const int nn = min(16, g.N - (n0 + c0));
-        if (C_BF16) {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.C) + (size_t)m * g.ldc + n0 + c0;
-          for (int j = 0; j < nn; ++j) dst[j] = __float2bfloat16_rn(g.alpha * v[j]);
-        } else {
-          float* dst = static_cast<float*>(g.C) + (size_t)m * g.ldc + n0 + c0;
-          if (nn == 16 && (g.ldc & 3) == 0) {
-            float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float4 x = make_float4(g.alpha * v[4 * j], g.alpha * v[4 * j + 1], g.alpha * v[4 * j + 2],
-                                     g.alpha * v[4 * j + 3]);
-              if (g.beta != 0.f) {
-                const float4 c = d4[j];
-                x.x += g.beta * c.x; x.y += g.beta * c.y; x.z += g.beta * c.z; x.w += g.beta * c.w;
-              }
-              d4[j] = x;
-            }
-          } else if (g.beta != 0.f) {
-            for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j] + g.beta * dst[j];
+      const int n0 = tile_n(t) * kGemmBN;
+      for (int half = 0; half < HV; ++half) {
+        const int m = tile_m(t) * kGemmBM + kGemmHalf * half + row;
+        const uint32_t la = tb + ((uint32_t)(32 * sp) << 16) + (uint32_t)((b + half) * kGemmBN);
+        for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+          float v[16];
+          tmem_ld16(la + c0, v);
+          if (m >= g.M || n0 + c0 >= g.N) continue;
+          const int nn = min(16, g.N - (n0 + c0));
+          if (C_BF16) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.C) + (size_t)m * g.ldc + n0 + c0;
+            for (int j = 0; j < nn; ++j) dst[j] = __float2bfloat16_rn(g.alpha * v[j]);
           } else {
-            for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j];
+            float* dst = static_cast<float*>(g.C) + (size_t)m * g.ldc + n0 + c0;
+            if (nn == 16 && (g.ldc & 3) == 0) {
+              float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                float4 x = make_float4(g.alpha * v[4 * j], g.alpha * v[4 * j + 1], g.alpha * v[4 * j + 2],
+                                       g.alpha * v[4 * j + 3]);
+                if (g.beta != 0.f) {
+                  const float4 c = d4[j];
+                  x.x += g.beta * c.x; x.y += g.beta * c.y; x.z += g.beta * c.z; x.w += g.beta * c.w;
+                }
+                d4[j] = x;
+              }
+            } else if (g.beta != 0.f) {
+              for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j] + g.beta * dst[j];
+            } else {
+              for (int j = 0; j < nn; ++j) dst[j] = g.alpha * v[j];
+            }
           }
         }
       }

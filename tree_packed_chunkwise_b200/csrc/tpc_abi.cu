@@ -643,28 +643,34 @@ int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B
   auto encode = [&](CUtensorMap* m, const void* X, bool mn_major, int64_t mn, int64_t ld, int box) {
     return mn_major ? tensor_map(m, X, mn, K, ld, tpc::kGemmBK, 64) : tensor_map(m, X, K, mn, ld, box, 64);
   };
+  // tile height: 256 rows (two halves) once K is long enough to hide the non-overlapped epilogue
+  const int HV = K >= tpc::kGemmLongK ? 2 : 1;
+  const int BM = tpc::kGemmHalf * HV;
   CUtensorMap ta, tb, talo, tblo;
-  bool ok = encode(&ta, A, a_mn, M, lda, tpc::kGemmBM) && encode(&tb, B, b_mn, N, ldb, tpc::kGemmBN);
-  ok = ok && encode(&talo, A_lo ? A_lo : A, a_mn, M, lda, tpc::kGemmBM);
+  bool ok = encode(&ta, A, a_mn, M, lda, BM) && encode(&tb, B, b_mn, N, ldb, tpc::kGemmBN);
+  ok = ok && encode(&talo, A_lo ? A_lo : A, a_mn, M, lda, BM);
   ok = ok && encode(&tblo, B_lo ? B_lo : B, b_mn, N, ldb, tpc::kGemmBN);
   if (!ok) return fail(TPC_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   const int passes = B_lo ? 3 : (A_lo ? 2 : 1);
   tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status, passes,
                   M < N ? 1 : 0};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t tiles = ((N + tpc::kGemmBN - 1) / tpc::kGemmBN) * ((M + tpc::kGemmBM - 1) / tpc::kGemmBM);
+  const int64_t tiles = ((N + tpc::kGemmBN - 1) / tpc::kGemmBN) * ((M + BM - 1) / BM);
   if (tiles > (int64_t)1 << 31) return fail(TPC_ERR_BAD_SHAPE, "gemm: too many tiles");
   const dim3 grid((unsigned)std::min<int64_t>(tiles, sm_count()));
-  if (c_dtype == TPC_BF16) {
-    TPC_CUDA(set_smem(tpc::gemm_bf16_tc<1>, tpc::GemmSmem::total));
+  auto go = [&](auto cb, auto hv) -> int {
+    constexpr int CB = decltype(cb)::value, H2 = decltype(hv)::value;
+    constexpr size_t smem = tpc::GemmCfg<H2>::total;
+    TPC_CUDA(set_smem(tpc::gemm_bf16_tc<CB, H2>, smem));
     TPC_LAUNCH("gemm_bf16_tc", st,
-               (tpc::gemm_bf16_tc<1><<<grid, tpc::kGemmThreadsP, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
-  } else {
-    TPC_CUDA(set_smem(tpc::gemm_bf16_tc<0>, tpc::GemmSmem::total));
-    TPC_LAUNCH("gemm_bf16_tc", st,
-               (tpc::gemm_bf16_tc<0><<<grid, tpc::kGemmThreadsP, tpc::GemmSmem::total, st>>>(ta, tb, talo, tblo, g)));
-  }
-  return TPC_OK;
+               (tpc::gemm_bf16_tc<CB, H2><<<grid, tpc::kGemmThreadsP, smem, st>>>(ta, tb, talo, tblo, g)));
+    return TPC_OK;
+  };
+  using I0 = std::integral_constant<int, 0>;
+  using I1 = std::integral_constant<int, 1>;
+  using I2 = std::integral_constant<int, 2>;
+  if (c_dtype == TPC_BF16) return HV == 2 ? go(I1{}, I2{}) : go(I1{}, I1{});
+  return HV == 2 ? go(I0{}, I2{}) : go(I0{}, I1{});
 }
 
 int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
