@@ -408,10 +408,8 @@ int sm_count() {
   return n;
 }
 
-// 2-D bf16 tensor map over [rows][cols] (leading dimension ld_elems): boxes of box_cols x box_rows
-// elements, 128-byte swizzle when box_cols is 64 (one 128-byte row per box row), none otherwise.
-bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems,
-                uint32_t box_rows, uint32_t box_cols = 8) {
+// the driver's tensor-map encoder (looked up once)
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   std::call_once(g_encode_once, [] {
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void**>(&g_encode), cudaEnableDefault,
@@ -419,15 +417,22 @@ bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, u
         q != cudaDriverEntryPointSuccess)
       g_encode = nullptr;
   });
-  if (!g_encode) return false;
+  return g_encode;
+}
+
+// 2-D bf16 tensor map over [rows][cols] (leading dimension ld_elems): boxes of 64 columns x box_rows
+// rows, each box row one 128-byte swizzled line.
+bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems,
+                uint32_t box_rows) {
+  const auto enc = encoder();
+  if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld_elems * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
-  const CUtensorMapSwizzle sw = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 3-D bf16 tensor map over a [rows][heads][features] tensor (feature dimension contiguous): boxes
@@ -435,15 +440,15 @@ bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, u
 // end read as zeros.
 bool tensor_map_rows(CUtensorMap* m, const void* ptr, uint64_t features, uint64_t heads, uint64_t rows,
                      uint32_t box_rows) {
-  CUtensorMap probe;
-  if (!tensor_map(&probe, ptr, 64, 1, 64, 8, 64)) return false;  // looks up the encoder
+  const auto enc = encoder();
+  if (!enc) return false;
   cuuint64_t dims[3] = {features, heads, rows};
   cuuint64_t strides[2] = {features * 2, heads * features * 2};
   cuuint32_t box[3] = {64, 1, box_rows};
   cuuint32_t es[3] = {1, 1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -641,7 +646,7 @@ int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B
   // 128-byte-swizzled boxes 64 elements wide: K-major [mn][K] boxes of 64 (K) x tile rows,
   // MN-major [K][mn] boxes of 64 (mn) x 64 (K)
   auto encode = [&](CUtensorMap* m, const void* X, bool mn_major, int64_t mn, int64_t ld, int box) {
-    return mn_major ? tensor_map(m, X, mn, K, ld, tpc::kGemmBK, 64) : tensor_map(m, X, K, mn, ld, box, 64);
+    return mn_major ? tensor_map(m, X, mn, K, ld, tpc::kGemmBK) : tensor_map(m, X, K, mn, ld, box);
   };
   // tile height: 256 rows (two halves) once K is long enough to hide the non-overlapped epilogue
   const int HV = K >= tpc::kGemmLongK ? 2 : 1;
