@@ -790,55 +790,67 @@ __global__ void __launch_bounds__(kAttnDkvThreads, 1)
       const uint32_t id_dv = idesc_bf16(128, DV, false, true), id_dk = idesc_bf16(128, DQ, false, true);
       bool ok = mbar_wait(&v_ready, 0);
       if (!ok) give_up();
-      for (int j = 0; ok && j <= n_tiles && !aborted(); ++j) {
-        if (j < n_tiles) {  // S^T, dP^T of query tile j (stage 0 also brings K before tile 0)
-          const int s = j % NS;
-          if (!mbar_wait(&full[s], (j / NS) & 1) || (j >= 1 && !mbar_wait(&s_read, (j - 1) & 1))) {
-            give_up();
-            break;
+      // S^T, dP^T of tile jS (needs its stage loaded and the previous S^T read) and dV, dK of tile jD
+      // (needs P^T, dS^T of tile jD in shared memory) are independent: issue whichever is ready,
+      // dV / dK first, since they release the stage that the load of tile jD + 2 waits for.
+      auto issue_s = [&](int j) {
+        const uint32_t st = smem_u32(stage(j % NS));
+        const uint32_t kh = smem_u32(sK), kl = smem_u32(sKl);
+        const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
+                       ol = st + (uint32_t)S::sOl;
+        for (int s2 = 0; s2 < DQ / 16; ++s2) mma_bf16(tb + cS, sw_desc_k(kh, KT, s2), sw_desc_k(qh, QT, s2), id_s, s2 ? 1u : 0u);
+        for (int s2 = 0; s2 < DV / 16; ++s2) mma_bf16_ts(tb + cP, tb + cVh + 8 * s2, sw_desc_k(oh, QT, s2), id_s, s2 ? 1u : 0u);
+        if constexpr (SPLIT) {
+          for (int s2 = 0; s2 < DQ / 16; ++s2) {
+            mma_bf16(tb + cS, sw_desc_k(kl, KT, s2), sw_desc_k(qh, QT, s2), id_s, 1u);
+            mma_bf16(tb + cS, sw_desc_k(kh, KT, s2), sw_desc_k(ql, QT, s2), id_s, 1u);
           }
-          fence_after_sync();
-          const uint32_t st = smem_u32(stage(s));
-          const uint32_t kh = smem_u32(sK), kl = smem_u32(sKl);
-          const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
-                         ol = st + (uint32_t)S::sOl;
-          for (int s2 = 0; s2 < DQ / 16; ++s2) mma_bf16(tb + cS, sw_desc_k(kh, KT, s2), sw_desc_k(qh, QT, s2), id_s, s2 ? 1u : 0u);
-          for (int s2 = 0; s2 < DV / 16; ++s2) mma_bf16_ts(tb + cP, tb + cVh + 8 * s2, sw_desc_k(oh, QT, s2), id_s, s2 ? 1u : 0u);
-          if constexpr (SPLIT) {
-            for (int s2 = 0; s2 < DQ / 16; ++s2) {
-              mma_bf16(tb + cS, sw_desc_k(kl, KT, s2), sw_desc_k(qh, QT, s2), id_s, 1u);
-              mma_bf16(tb + cS, sw_desc_k(kh, KT, s2), sw_desc_k(ql, QT, s2), id_s, 1u);
-            }
-            for (int s2 = 0; s2 < DV / 16; ++s2) {
-              mma_bf16_ts(tb + cP, tb + cVl + 8 * s2, sw_desc_k(oh, QT, s2), id_s, 1u);
-              mma_bf16_ts(tb + cP, tb + cVh + 8 * s2, sw_desc_k(ol, QT, s2), id_s, 1u);
-            }
+          for (int s2 = 0; s2 < DV / 16; ++s2) {
+            mma_bf16_ts(tb + cP, tb + cVl + 8 * s2, sw_desc_k(oh, QT, s2), id_s, 1u);
+            mma_bf16_ts(tb + cP, tb + cVh + 8 * s2, sw_desc_k(ol, QT, s2), id_s, 1u);
           }
-          commit(&s_full);
         }
-        if (j >= 1) {  // dV, dK of query tile j - 1
-          const int jp = j - 1, s = jp % NS;
-          if (!mbar_wait(&p_full, jp & 1)) {
-            give_up();
-            break;
-          }
+        commit(&s_full);
+      };
+      auto issue_d = [&](int jp) {
+        const int s = jp % NS;
+        const uint32_t st = smem_u32(stage(s));
+        const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
+                       ol = st + (uint32_t)S::sOl;
+        const Op ph{smem_u32(sPh), KT, false}, pl{smem_u32(sPl), KT, false};
+        const Op gh{smem_u32(sDh), KT, false}, gl{smem_u32(sDl), KT, false};
+        for (int s2 = 0; s2 < QT / 16; ++s2) {
+          const uint32_t acc = (jp > 0 || s2) ? 1u : 0u;
+          mma_bf16(tb + cDV, op_desc(ph, s2), sw_desc_mn(oh, QT, s2), id_dv, acc);
+          mma_bf16(tb + cDV, op_desc(pl, s2), sw_desc_mn(oh, QT, s2), id_dv, 1u);
+          if constexpr (SPLIT) mma_bf16(tb + cDV, op_desc(ph, s2), sw_desc_mn(ol, QT, s2), id_dv, 1u);
+          mma_bf16(tb + cDK, op_desc(gh, s2), sw_desc_mn(qh, QT, s2), id_dk, acc);
+          mma_bf16(tb + cDK, op_desc(gl, s2), sw_desc_mn(qh, QT, s2), id_dk, 1u);
+          if constexpr (SPLIT) mma_bf16(tb + cDK, op_desc(gh, s2), sw_desc_mn(ql, QT, s2), id_dk, 1u);
+        }
+        commit(&p_empty);   // P^T, dS^T may be overwritten
+        commit(&empty[s]);  // the stage may be refilled
+      };
+      int jS = 0, jD = 0;
+      uint64_t t_last = globaltimer();
+      while (ok && jD < n_tiles) {
+        if (aborted()) break;
+        bool issued = false;
+        if (jD < jS && mbar_try_wait(&p_full, jD & 1)) {
           fence_after_sync();
-          const uint32_t st = smem_u32(stage(s));
-          const uint32_t qh = st + (uint32_t)S::sQ, ql = st + (uint32_t)S::sQl, oh = st + (uint32_t)S::sO,
-                         ol = st + (uint32_t)S::sOl;
-          const Op ph{smem_u32(sPh), KT, false}, pl{smem_u32(sPl), KT, false};
-          const Op gh{smem_u32(sDh), KT, false}, gl{smem_u32(sDl), KT, false};
-          for (int s2 = 0; s2 < QT / 16; ++s2) {
-            const uint32_t acc = (jp > 0 || s2) ? 1u : 0u;
-            mma_bf16(tb + cDV, op_desc(ph, s2), sw_desc_mn(oh, QT, s2), id_dv, acc);
-            mma_bf16(tb + cDV, op_desc(pl, s2), sw_desc_mn(oh, QT, s2), id_dv, 1u);
-            if constexpr (SPLIT) mma_bf16(tb + cDV, op_desc(ph, s2), sw_desc_mn(ol, QT, s2), id_dv, 1u);
-            mma_bf16(tb + cDK, op_desc(gh, s2), sw_desc_mn(qh, QT, s2), id_dk, acc);
-            mma_bf16(tb + cDK, op_desc(gl, s2), sw_desc_mn(qh, QT, s2), id_dk, 1u);
-            if constexpr (SPLIT) mma_bf16(tb + cDK, op_desc(gh, s2), sw_desc_mn(ql, QT, s2), id_dk, 1u);
-          }
-          commit(&p_empty);   // P^T, dS^T may be overwritten
-          commit(&empty[s]);  // the stage may be refilled
+          issue_d(jD++);
+          issued = true;
+        } else if (jS < n_tiles && mbar_try_wait(&full[jS % NS], (jS / NS) & 1) &&
+                   (jS == 0 || mbar_try_wait(&s_read, (jS - 1) & 1))) {
+          fence_after_sync();
+          issue_s(jS++);
+          issued = true;
+        }
+        if (issued) {
+          t_last = globaltimer();
+        } else if (globaltimer() - t_last > 1000000000ull) {  // nothing became ready for a second
+          give_up();
+          ok = false;
         }
       }
       commit(&done_bar);  // arrives once every MMA issued above has completed
