@@ -23,7 +23,8 @@ def padded(x):
     return buf[:, :c]
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 500, 200), (1, 8, 8), (700, 1030, 2048)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 500, 200), (1, 8, 8), (700, 1030, 2048),
+                                   (300, 520, 4100), (520, 300, 4620)])
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 0), (0, 1), (1, 1)])
 def test_gemm_matches_torch(tpc, M, N, K, a_mn, b_mn):
     import torch
