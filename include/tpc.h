@@ -55,7 +55,13 @@ enum tpc_status_code {
   TPC_ERR_STATE = 10        /* plan not uploaded / wrong call order */
 };
 
-enum tpc_dtype { TPC_F32 = 0, TPC_BF16 = 1 };
+/*
+ * Element types.  TPC_F32_SPLIT is an input type of the KDA calls only: fp32 tensors that the
+ * tensor-core kernels (chunk 64, d 128) take as bf16 pairs hi + lo, each product formed as
+ * hi*hi + lo*hi + hi*lo in fp32 (about 1e-4 of the output RMS in max error).  TPC_F32 inputs run
+ * the fp32 CUDA-core kernels, whose results match the fp64 recurrence to about 1e-6.
+ */
+enum tpc_dtype { TPC_F32 = 0, TPC_BF16 = 1, TPC_F32_SPLIT = 2 };
 
 /* Returns the message of the last failed call on this thread ("" if none). */
 const char* tpc_last_error(void);
@@ -133,7 +139,7 @@ int tpc_plan_upload(tpc_plan* plan, void* dev, size_t bytes, tpc_stream_t stream
 typedef struct tpc_kda_shape {
   int32_t H;          /* heads */
   int32_t dk, dv;     /* head dims; dk == dv in {32, 64, 128} */
-  int32_t in_dtype;   /* tpc_dtype of q, k, v, g, beta, d_o */
+  int32_t in_dtype;   /* tpc_dtype of q, k, v, g, beta, d_o (TPC_F32_SPLIT: fp32 data) */
   int32_t out_dtype;  /* tpc_dtype of o, dq, dk, dv */
 } tpc_kda_shape;
 
@@ -396,12 +402,19 @@ int tpc_group_status(const tpc_plan* plan, const tpc_group_shape* shape, void* w
  *   Set-up: the first call on a device looks up the array's device address (with that device
  *       current); make that first call before any stream capture.
  *   Sharing: every call uses the same array and it keeps the previous call's contents; the call
- *       clears its status word itself.  Calls that overlap on the GPU (other streams, other host
+ *       clears its status word itself (tpc_kda_static_status reads it).  Calls that overlap on the GPU (other streams, other host
  *       threads) race on the array: serialise them.  tpc_kda_backward cannot follow this call (the
  *       workspace it needs is not kept).
  */
 int tpc_kda_forward_static(const tpc_plan* plan, const tpc_kda_shape* shape, const tpc_kda_fwd_io* io,
                            tpc_stream_t stream);
+/*
+ * Reads (after synchronising `stream`) and clears the status word of the allocation-free forward
+ * on the current device: kernel-side checks of tpc_kda_forward_static (the gate range) record
+ * their code there, since that call has no caller workspace.  Returns TPC_OK, TPC_ERR_RANGE or
+ * TPC_ERR_DEVICE_CHECK.  Allocates nothing.
+ */
+int tpc_kda_static_status(tpc_stream_t stream);
 
 /* ------------------------------------------------------------------ diagnostics */
 /* Per-kernel timing: when enabled, every launch is bracketed by CUDA events recorded on
@@ -412,6 +425,13 @@ void tpc_profile_enable(int on);
 int tpc_profile_read(char* buf, size_t len);
 /* Number of kernels this library has launched in the process. */
 long long tpc_launch_count(void);
+/*
+ * Check of the device-side timeout path: one CTA runs the bounded mbarrier wait that every
+ * tensor-core kernel of this library uses, on a barrier that nothing arrives on (no copy or MMA in
+ * flight), with a limit of timeout_ns (1e3 .. 1e8).  The wait runs out, the kernel writes
+ * TPC_ERR_TIMEOUT into *status (a caller-owned device int) and returns; the context stays usable.
+ */
+int tpc_debug_wait_timeout(int32_t* status, int64_t timeout_ns, tpc_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -266,28 +266,30 @@ def workload(cfg: str) -> Workload:
 
 
 # ---------------------------------------------------------------- KDA inputs (node order)
-def kda_inputs(seed: int, rows, H: int, dk: int, dv: int, dtype: str):
+def kda_inputs(seed: int, rows, H: int, dk: int, dv: int, dtype: str, heads=None):
     """q, k, v, g [len(rows), H, d] and beta [len(rows), H] for the given node-order rows.
 
     Values are returned as float64 arrays holding exactly the rounded
-    (fp32 or bf16) values that the device generator writes.
+    (fp32 or bf16) values that the device generator writes.  ``heads``
+    (a list of head indices of the H-head tensors) returns only those heads.
     """
     rows = np.asarray(rows, np.int64)
     n = rows.shape[0]
+    hs = np.arange(H) if heads is None else np.asarray(heads, np.int64)
 
     def flat(width):
-        return (rows[:, None, None] * H + np.arange(H)[None, :, None]) * width + np.arange(width)[None, None, :]
+        return (rows[:, None, None] * H + hs[None, :, None]) * width + np.arange(width)[None, None, :]
 
     q = round_to(normal_f64(seed, STREAM["q"], flat(dk)), dtype)
     zk = normal_f64(seed, STREAM["k"], flat(dk))
-    ss = np.zeros((n, H), np.float64)
+    ss = np.zeros((n, len(hs)), np.float64)
     for c in range(dk):  # fixed summation order, mirrored on the device
         ss = ss + zk[:, :, c] * zk[:, :, c]
     k = round_to(zk / np.sqrt(ss)[:, :, None], dtype)
     v = round_to(normal_f64(seed, STREAM["v"], flat(dv)), dtype)
     zg = normal_f64(seed, STREAM["g"], flat(dk))
     g = round_to(-0.1 * np.log1p(np.exp(zg)), dtype)
-    zb = normal_f64(seed, STREAM["beta"], rows[:, None] * H + np.arange(H)[None, :])
+    zb = normal_f64(seed, STREAM["beta"], rows[:, None] * H + hs[None, :])
     beta = round_to(1.0 / (1.0 + np.exp(-zb)), dtype)
     f = np.float64
     return q.astype(f), k.astype(f), v.astype(f), g.astype(f), beta.astype(f)

@@ -37,6 +37,160 @@ def single_fork_case(tpc):
     return w, t, plan, st, src, x
 
 
+# ------------------------------------------------------------------------------------ windowed parity
+def windowed_parity(tpc, tree, H, d, seed, heads, specs, label):
+    """Full-size tree-packed forward + backward against the token-by-token oracle on windows.
+
+    specs: list of dicts {leaf, windows: [(first, last + 1) node-order rows], d_final: bool}.  The
+    upstream output gradient is non-zero (N(0, 1), bf16) only on the windows' rows and the final-state
+    gradient only on the flagged leaves, so every input gradient equals the sum, over the specs'
+    trajectories, of the oracle's backward of that trajectory (HARTS abstract: gradients of dependent
+    work accumulate into the shared prefix), and rows on no such trajectory get exactly zero.  Heads
+    are independent: the oracle runs on ``heads`` only.  Outputs and the flagged leaves' final states
+    are compared over the whole trajectories."""
+    import torch
+    import synth.gpu as sgpu
+    plan = tpc.Plan(tree.parent, tree.length, 64).upload()
+    info = plan.info
+    N = info["n_unique"]
+    st = tree.node_start()
+    src_np = plan.compact_source_rows(st, tree.length)
+    inv = np.empty(N, np.int64)
+    inv[src_np] = np.arange(N)
+    src = torch.tensor(src_np, dtype=torch.int32, device="cuda")
+    x = dict(zip(("q", "k", "v", "g", "beta"), sgpu.kda_inputs(seed, src, H, d, d, "bf16")))
+    leaves = list(tree.leaves())
+    d_o = torch.zeros(N, H, d, dtype=torch.bfloat16, device="cuda")
+    d_fin = torch.zeros(len(leaves), H, d, d, dtype=torch.float32, device="cuda")
+    win_rows = {}
+    for sp in specs:
+        rows = np.concatenate([np.arange(a, b) for a, b in sp["windows"]]) if sp["windows"] else np.zeros(0, np.int64)
+        win_rows[sp["leaf"]] = rows
+        if len(rows):
+            vals = synth.rows_normal(seed, synth.STREAM["d_o"], rows, H * d, "bf16").reshape(len(rows), H, d)
+            d_o[torch.tensor(inv[rows], device="cuda")] = torch.tensor(vals, dtype=torch.float32).to(
+                torch.bfloat16).cuda()
+        if sp["d_final"]:
+            li = leaves.index(sp["leaf"])
+            d_fin[li] = torch.tensor(synth.normal_tensor(seed, synth.STREAM["d_final"], (H, d, d), "f32",
+                                                         first=li * H * d * d), dtype=torch.float32)
+    o, fin, ws = tpc.tpc_kda_forward(plan, x["q"], x["k"], x["v"], x["g"], x["beta"], out_dtype=torch.float32)
+    gr = tpc.tpc_kda_backward(plan, ws, x["q"], x["k"], x["v"], x["g"], x["beta"], d_o, d_fin,
+                              out_dtype=torch.float32, want_d_init=False)
+    torch.cuda.synchronize()
+    tpc.tpc_status(plan, ws, H, d)
+    # the oracle, trajectory by trajectory, gradients summed per node-order row
+    union = np.unique(np.concatenate([tree.trajectory_rows(sp["leaf"]) for sp in specs]))
+    pos = {r: i for i, r in enumerate(union)}
+    nh = len(heads)
+    acc = {k: np.zeros((len(union), nh, d)) for k in ("dq", "dk", "dv", "dg")}
+    acc["dbeta"] = np.zeros((len(union), nh))
+    o_ref = np.zeros((len(union), nh, d))
+    fin_ref = {}
+    for sp in specs:
+        rows = tree.trajectory_rows(sp["leaf"])
+        inp = synth.kda_inputs(seed, rows, H, d, d, "bf16", heads=heads)
+        dO = np.zeros((len(rows), nh, d))
+        wr = win_rows[sp["leaf"]]
+        if len(wr):
+            vals = synth.rows_normal(seed, synth.STREAM["d_o"], wr, H * d, "bf16").reshape(len(wr), H, d)[:, heads]
+            where = {r: i for i, r in enumerate(rows)}
+            dO[[where[r] for r in wr]] = vals
+        li = leaves.index(sp["leaf"])
+        dF = None
+        if sp["d_final"]:
+            dF = synth.normal_tensor(seed, synth.STREAM["d_final"], (H, d, d), "f32", first=li * H * d * d)[heads]
+        o_t, S_t = okda.forward(*inp)
+        g_t = okda.backward(*inp, dO, dF)
+        ix = np.array([pos[r] for r in rows])
+        o_ref[ix] = o_t
+        fin_ref[li] = S_t
+        for key, val in zip(("dq", "dk", "dv", "dg", "dbeta"), g_t[:5]):
+            np.add.at(acc[key], ix, val)
+    cix = torch.tensor(inv[union], device="cuda")
+    hix = torch.tensor(heads, device="cuda")
+    pick = lambda t: t[cix][:, hix].float().cpu().numpy()
+    errs = {"o": err_ratio(pick(o), o_ref)}
+    for li, S in fin_ref.items():
+        errs[f"final[{li}]"] = err_ratio(fin[li][hix].cpu().numpy(), S)
+    for key in ("dq", "dk", "dv", "dg", "dbeta"):
+        errs[key] = err_ratio(pick(gr[key]), acc[key])
+    # rows on no checked trajectory: exactly zero gradient (all heads)
+    off = torch.ones(N, dtype=torch.bool, device="cuda")
+    off[cix] = False
+    zero_off = {key: float(gr[key][off].abs().max().item()) if off.any() else 0.0
+                for key in ("dq", "dk", "dv", "dg", "dbeta")}
+    print(label, {k: f"{v:.2e}" for k, v in errs.items()}, "off-trajectory max |grad|", zero_off,
+          "trajectory rows", len(union), "of", N)
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
+    assert all(z == 0.0 for z in zero_off.values()), zero_off
+    return plan
+
+
+def test_single_fork_windowed_backward_vs_oracle(tpc):
+    """Full single-fork tree (N = 29,073, H = 16): the upstream gradient on the last 64 rows of the
+    longest branch (the reverse scan crosses the fork and the 128 prefix chunks) and the final-state
+    gradient of a second leaf; outputs, both final states and all gradients of heads 0 and 9
+    against the oracle."""
+    w = synth.workload("single_fork")
+    t = w.tree
+    leaves = list(t.leaves())
+    lens = [len(t.trajectory_rows(l)) for l in leaves]
+    longest = leaves[int(np.argmax(lens))]
+    other = leaves[0] if leaves[0] != longest else leaves[1]
+    st = t.node_start()
+    end = st[longest] + t.length[longest]
+    specs = [dict(leaf=longest, windows=[(end - 64, end)], d_final=False),
+             dict(leaf=other, windows=[], d_final=True)]
+    windowed_parity(tpc, t, w.H, w.dk, w.seed, [0, 9], specs, "single-fork windowed")
+
+
+def test_agentic_full_windowed_with_replay_vs_oracle(tpc):
+    """Full agentic tree (64 leaves, 5 fork levels, H = 16, with replay rows): a trajectory whose path
+    holds replay-started sequences, upstream gradient on the last 64 rows of its leaf and on 64 rows
+    inside a replay-started node, plus its final-state gradient; outputs, final state and every
+    gradient of heads 3 and 12 against the oracle."""
+    w = synth.workload("agentic")
+    t = w.tree
+    plan = tpc.Plan(t.parent, t.length, 64)
+    tb = plan.tables()
+    assert plan.info["replay_total"] > 0
+    best, best_n = None, -1
+    for leaf in t.leaves():
+        path = t.path(leaf)
+        n_rep = sum(1 for v in path if tb["replay_len"][v] > 0)
+        if n_rep > best_n or (n_rep == best_n and tb["round"][leaf] > tb["round"][best]):
+            best, best_n = leaf, n_rep
+    assert best_n >= 2
+    st = t.node_start()
+    path = t.path(best)
+    rep = [v for v in path if tb["replay_len"][v] > 0][0]
+    end = st[best] + t.length[best]
+    windows = [(st[rep], st[rep] + min(64, int(t.length[rep])))] if rep != best else []
+    windows.append((max(end - 64, st[best]), end))
+    specs = [dict(leaf=best, windows=windows, d_final=True)]
+    print("agentic leaf", best, "replay-started nodes on the path", best_n, "rounds", plan.info["n_rounds"])
+    windowed_parity(tpc, t, w.H, w.dk, w.seed, [3, 12], specs, "agentic windowed")
+
+
+def test_wide_tree_windowed_vs_oracle(tpc):
+    """Full wide tree (32,768-token prefix = 512 sequential chunks, 512 leaves) as bench.py runs its
+    KDA layer (one group of 8 of the 32 heads per call): upstream gradient on the last 64 rows of the
+    prefix and of a depth-3 leaf, final-state gradient of that leaf; outputs, final state and all
+    gradients of heads 1 and 6 against the oracle."""
+    w = synth.workload("wide")
+    t = w.tree
+    leaves = list(t.leaves())
+    lens = [len(t.trajectory_rows(l)) for l in leaves]
+    leaf = leaves[int(np.argmax(lens))]
+    st = t.node_start()
+    pend = int(t.length[0])
+    end = st[leaf] + t.length[leaf]
+    windows = [(pend - 64, pend), (max(end - 64, st[leaf]), end)]
+    specs = [dict(leaf=leaf, windows=windows, d_final=True)]
+    windowed_parity(tpc, t, 8, w.dk, w.seed + 17, [1, 6], specs, "wide windowed (8-head group)")
+
+
 def test_single_fork_full_forward(tpc):
     """Full single-fork tree (N = 29,073, H = 16, d = 128, chunk 64, bf16 inputs): outputs of the
     first 256 tokens and of the first 64 tokens after one fork against the token-by-token oracle;

@@ -65,3 +65,25 @@ def test_static_forward_rejects_oversized_problem(tpc):
     with pytest.raises(tpc.TpcError) as e:
         tpc.tpc_kda_forward_static(plan, z, z, z, z, zb)
     assert e.value.code == 5 and "bytes" in str(e.value)
+
+
+def test_static_forward_status_word_is_readable(tpc):
+    """The allocation-free forward keeps its status word in the built-in array; its kernel-side gate
+    check is read (and cleared) by tpc_kda_static_status."""
+    import torch
+    tree = synth.Tree(np.array([-1], np.int32), np.array([40], np.int32))
+    case = Case(tree, 1, 32, 16, "f32", 3)
+    case.inputs = list(case.inputs)
+    case.inputs[3] = case.inputs[3] * 0 - 20.0  # decay 300 inside a 16-row sub-block: out of range
+    plan = tpc.Plan(tree.parent, tree.length, 16)
+    x = to_torch_compact(case, tpc.Plan(tree.parent, tree.length, 16).upload())
+    tpc.tpc_kda_forward_static(plan, x["q"], x["k"], x["v"], x["g"], x["beta"])
+    with pytest.raises(tpc.TpcError) as e:
+        tpc.tpc_kda_static_status()
+    assert e.value.code == 9
+    tpc.tpc_kda_static_status()  # cleared
+    ok = Case(tree, 1, 32, 16, "f32", 4)
+    y = to_torch_compact(ok, tpc.Plan(tree.parent, tree.length, 16).upload())
+    tpc.tpc_kda_forward_static(plan, y["q"], y["k"], y["v"], y["g"], y["beta"])
+    tpc.tpc_kda_static_status()
+

@@ -15,7 +15,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtpc.so")
 
-TPC_F32, TPC_BF16 = 0, 1
+TPC_F32, TPC_BF16, TPC_F32_SPLIT = 0, 1, 2
 _STATUS = {0: "TPC_OK", 1: "TPC_ERR_INVALID_TREE", 2: "TPC_ERR_BAD_SHAPE", 3: "TPC_ERR_UNSUPPORTED",
            4: "TPC_ERR_NULL", 5: "TPC_ERR_WORKSPACE", 6: "TPC_ERR_CUDA", 7: "TPC_ERR_DEVICE_CHECK",
            8: "TPC_ERR_TIMEOUT", 9: "TPC_ERR_RANGE", 10: "TPC_ERR_STATE"}
@@ -106,6 +106,7 @@ SIGNATURES = {
     "tpc_gather_expanded": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int32, _V]),
     "tpc_occurrence_counts": (ctypes.c_int, [_V, _V, _V]),
     "tpc_kda_forward_static": (ctypes.c_int, [_V, _P(KdaShape), _P(KdaFwdIO), _V]),
+    "tpc_kda_static_status": (ctypes.c_int, [_V]),
     "tpc_gemm_bf16": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_float, ctypes.c_float, _V, _V]),
@@ -128,6 +129,7 @@ SIGNATURES = {
     "tpc_profile_enable": (None, [ctypes.c_int]),
     "tpc_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t]),
     "tpc_launch_count": (ctypes.c_longlong, []),
+    "tpc_debug_wait_timeout": (ctypes.c_int, [_V, ctypes.c_int64, _V]),
 }
 
 _lib = None
@@ -223,9 +225,39 @@ class Plan:
 
 
 # ------------------------------------------------------------------------------------ KDA
-def _dtype_code(t):
+def _dtype_code(t, split=False):
     import torch
-    return TPC_BF16 if t.dtype == torch.bfloat16 else TPC_F32
+    if t.dtype == torch.bfloat16:
+        return TPC_BF16
+    return TPC_F32_SPLIT if split else TPC_F32
+
+
+def _check_kda_tensors(plan: Plan, named: dict, d_final=None, init_state=None):
+    """Raises TpcError (TPC_ERR_BAD_SHAPE) before any launch unless every per-row tensor has the
+    plan's n_unique rows, shape [N, H, d] ([N, H] for beta), one dtype (bf16 or fp32), is
+    contiguous and lives on the current CUDA device; the state tensors must be fp32 [n, H, d, d]."""
+    import torch
+    N = plan.info["n_unique"]
+    q = named["q"]
+    if q.dim() != 3:
+        raise TpcError(2, f"q must be [N, H, d], got {tuple(q.shape)}")
+    _, H, d = q.shape
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else None
+    for name, t in named.items():
+        want = (N, H) if name == "beta" else (N, H, d)
+        if tuple(t.shape) != want:
+            raise TpcError(2, f"{name} has shape {tuple(t.shape)}, expected {want} (n_unique = {N})")
+        if t.dtype != q.dtype or t.dtype not in (torch.bfloat16, torch.float32):
+            raise TpcError(2, f"{name} has dtype {t.dtype}; all inputs must share one dtype, bf16 or fp32")
+        if not t.is_contiguous():
+            raise TpcError(2, f"{name} is not contiguous")
+        if t.device != dev:
+            raise TpcError(2, f"{name} is on {t.device}, not the current device {dev}")
+    for name, t, n in (("d_final", d_final, plan.info["n_leaves"]), ("init_state", init_state, plan.info["n_roots"])):
+        if t is None:
+            continue
+        if tuple(t.shape) != (n, H, d, d) or t.dtype != torch.float32 or not t.is_contiguous() or t.device != dev:
+            raise TpcError(2, f"{name} must be a contiguous fp32 [{n}, {H}, {d}, {d}] tensor on {dev}")
 
 
 def kda_shape(H, d, in_dtype, out_dtype) -> KdaShape:
@@ -245,12 +277,15 @@ def alloc_workspace(plan: Plan, shape: KdaShape, device="cuda"):
 
 
 def tpc_kda_forward(plan: Plan, q, k, v, g, beta, init_state=None, out_dtype=None, ws=None, o=None,
-                    final_state=None, want_final=True, stream=None):
-    """Tree-packed forward.  Tensors in compact row order; returns (o, final_state, ws)."""
+                    final_state=None, want_final=True, stream=None, split=False):
+    """Tree-packed forward.  Tensors in compact row order; returns (o, final_state, ws).
+    split: fp32 inputs on the tensor-core kernels as bf16 hi/lo pairs (TPC_F32_SPLIT) instead of
+    the exact fp32 CUDA-core kernels."""
     import torch
+    _check_kda_tensors(plan, dict(q=q, k=k, v=v, g=g, beta=beta), init_state=init_state)
     N, H, d = q.shape
     out_dtype = out_dtype or q.dtype
-    shape = kda_shape(H, d, _dtype_code(q), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
+    shape = kda_shape(H, d, _dtype_code(q, split), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
     if ws is None:
         ws = alloc_workspace(plan, shape, q.device)
     if o is None:
@@ -270,6 +305,7 @@ def tpc_kda_forward_static(plan: Plan, q, k, v, g, beta, init_state=None, out_dt
     """Forward that allocates nothing on the device: tables and workspace live in the library's
     built-in scratch array (see include/tpc.h).  Returns (o, final_state)."""
     import torch
+    _check_kda_tensors(plan, dict(q=q, k=k, v=v, g=g, beta=beta), init_state=init_state)
     N, H, d = q.shape
     out_dtype = out_dtype or q.dtype
     shape = kda_shape(H, d, _dtype_code(q), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
@@ -284,13 +320,20 @@ def tpc_kda_forward_static(plan: Plan, q, k, v, g, beta, init_state=None, out_dt
     return o, final_state
 
 
+def tpc_kda_static_status(stream=None):
+    """Raises TpcError if a kernel-side check of the allocation-free forward failed (then clears it)."""
+    _check(lib().tpc_kda_static_status(_stream_ptr(stream)))
+
+
 def tpc_kda_backward(plan: Plan, ws, q, k, v, g, beta, d_o, d_final=None, init_state=None, out_dtype=None,
-                     want_d_init=True, grads=None, stream=None):
-    """Backward; returns dict(dq, dk, dv, dg, dbeta, d_init)."""
+                     want_d_init=True, grads=None, stream=None, split=False):
+    """Backward; returns dict(dq, dk, dv, dg, dbeta, d_init).  split: as tpc_kda_forward (must match
+    the forward that filled ws)."""
     import torch
+    _check_kda_tensors(plan, dict(q=q, k=k, v=v, g=g, beta=beta, d_o=d_o), d_final=d_final, init_state=init_state)
     N, H, d = q.shape
     out_dtype = out_dtype or q.dtype
-    shape = kda_shape(H, d, _dtype_code(q), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
+    shape = kda_shape(H, d, _dtype_code(q, split), TPC_BF16 if out_dtype == torch.bfloat16 else TPC_F32)
     if grads is None:
         dev = q.device
         grads = dict(dq=torch.empty(N, H, d, dtype=out_dtype, device=dev),
@@ -358,6 +401,12 @@ def tpc_profile_read() -> dict:
 
 def tpc_launch_count() -> int:
     return int(lib().tpc_launch_count())
+
+
+def tpc_debug_wait_timeout(status, timeout_ns=1_000_000, stream=None):
+    """Runs the library's bounded device wait on a barrier nothing arrives on; status (int32 device
+    tensor) receives TPC_ERR_TIMEOUT."""
+    _check(lib().tpc_debug_wait_timeout(_ptr(status), int(timeout_ns), _stream_ptr(stream)))
 
 
 # ------------------------------------------------------------------------------------ dense products

@@ -28,7 +28,8 @@ bool group_supported(const tpc_group_shape* s) {
 }
 
 // the KDA layer runs the recurrence on fp32 inputs and outputs (tensor-core path, split products)
-tpc_kda_shape kda_shape() { return tpc_kda_shape{kGrpH, kGrpDH, kGrpDH, TPC_F32, TPC_F32}; }
+// fp32 activations on the tensor-core KDA kernels (bf16 hi/lo operands)
+tpc_kda_shape kda_shape() { return tpc_kda_shape{kGrpH, kGrpDH, kGrpDH, TPC_F32_SPLIT, TPC_F32}; }
 
 tpc_attn_shape attn_shape() {
   return tpc_attn_shape{kGrpH, kGrpQK, kGrpDH, 1.0f / sqrtf((float)kGrpQK), TPC_F32};

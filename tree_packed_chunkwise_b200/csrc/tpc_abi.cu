@@ -109,8 +109,11 @@ int check_shape(const tpc_plan* plan, const tpc_kda_shape* s) {
   if (s->dk != s->dv) return fail(TPC_ERR_UNSUPPORTED, "dk != dv is not built");
   if (!shape_supported(plan->p.C, s->dk))
     return fail(TPC_ERR_UNSUPPORTED, "built (chunk, d) pairs: (16,32), (32,64), (64,128)");
-  if ((s->in_dtype != TPC_F32 && s->in_dtype != TPC_BF16) || (s->out_dtype != TPC_F32 && s->out_dtype != TPC_BF16))
-    return fail(TPC_ERR_UNSUPPORTED, "dtype must be TPC_F32 or TPC_BF16");
+  if ((s->in_dtype != TPC_F32 && s->in_dtype != TPC_BF16 && s->in_dtype != TPC_F32_SPLIT) ||
+      (s->out_dtype != TPC_F32 && s->out_dtype != TPC_BF16))
+    return fail(TPC_ERR_UNSUPPORTED, "in_dtype TPC_F32, TPC_BF16 or TPC_F32_SPLIT; out_dtype TPC_F32 or TPC_BF16");
+  if (s->in_dtype == TPC_F32_SPLIT && !(plan->p.C == tpc::kTcC && s->dk == tpc::kTcD))
+    return fail(TPC_ERR_UNSUPPORTED, "TPC_F32_SPLIT is built for chunk 64, d 128 (the tensor-core path)");
   return TPC_OK;
 }
 
@@ -148,7 +151,7 @@ int stream_after(cudaStream_t to, cudaStream_t from) {
   return TPC_OK;
 }
 
-template <int C, int D, typename Tin, typename Tout>
+template <int C, int D, typename Tin, typename Tout, bool TC>
 int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_io* io, void* ws, cudaStream_t st) {
   using namespace tpc;
   constexpr int DVT = D < 32 ? D : 32;
@@ -165,10 +168,10 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
   const Tin* v = static_cast<const Tin*>(io->v);
   const Tin* g = static_cast<const Tin*>(io->g);
   const Tin* b = static_cast<const Tin*>(io->beta);
-  // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
-  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  // tensor cores at chunk 64 / d 128 for bf16 inputs and for fp32 inputs given as TPC_F32_SPLIT;
+  // TPC_F32 inputs take the exact CUDA-core path
   std::vector<cudaEvent_t> scans;
-  if constexpr (kTensorCores) {
+  if constexpr (TC) {
     // Per round r: prep(r) and then out(r) on the caller's stream, scan(r) on the high-priority scan
     // stream after prep(r) and scan(r - 1).  The caller's stream runs prep(1..R), out(1..R) in that
     // order, so the later rounds' prep overlaps scan(1) and out(r) overlaps scan(r + 1).
@@ -218,7 +221,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
   return TPC_OK;
 }
 
-template <int C, int D, typename Tin, typename Tout>
+template <int C, int D, typename Tin, typename Tout, bool TC>
 int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_io* io, void* ws, cudaStream_t st) {
   using namespace tpc;
   constexpr int DVT = D < 32 ? D : 32;
@@ -236,10 +239,9 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   const Tin* g = static_cast<const Tin*>(io->g);
   const Tin* b = static_cast<const Tin*>(io->beta);
   const Tin* dO = static_cast<const Tin*>(io->d_o);
-  // tensor cores for bf16 inputs at chunk 64 / d 128; fp32 inputs keep the exact CUDA-core path
-  constexpr bool kTensorCores = (C == kTcC && D == kTcD);
+  // tensor-core or exact CUDA-core path, as in forward_impl
   std::vector<cudaEvent_t> scans;
-  if constexpr (kTensorCores) {
+  if constexpr (TC) {
     // Rounds in reverse: prep(r) on the caller's stream; the reverse scan(r) on the high-priority
     // scan stream after prep(r) and scan(r + 1); then dq(r), dk/dv(r) on the caller's stream after
     // scan(r).  The caller's stream runs prep(R..1), then dq / dk-dv(R..1), so the earlier rounds'
@@ -310,23 +312,26 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   return TPC_OK;
 }
 
+// Calls f(C, D, Tin{}, Tout{}, TC) with the shape's compile-time parameters.  TC (tensor cores):
+// chunk 64 / d 128 with bf16 inputs or with fp32 inputs given as TPC_F32_SPLIT.
 template <class F>
 int dispatch(const tpc_plan* plan, const tpc_kda_shape* s, F&& f) {
   const int C = plan->p.C, D = s->dk;
-  const bool ib = s->in_dtype == TPC_BF16, ob = s->out_dtype == TPC_BF16;
-#define TPC_CASE(CC, DD)                                                                         \
-  if (C == CC && D == DD) {                                                                      \
-    if (ib && ob) return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{}, \
-                           __nv_bfloat16{}, __nv_bfloat16{});                                    \
-    if (ib) return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{},       \
-                     __nv_bfloat16{}, float{});                                                  \
-    if (ob) return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{},       \
-                     float{}, __nv_bfloat16{});                                                  \
-    return f(std::integral_constant<int, CC>{}, std::integral_constant<int, DD>{}, float{}, float{}); \
+  const bool ib = s->in_dtype == TPC_BF16, ob = s->out_dtype == TPC_BF16, split = s->in_dtype == TPC_F32_SPLIT;
+  using Y = std::true_type;
+  using N = std::false_type;
+#define TPC_CASE(CC, DD, TCB, TCF)                                                                          \
+  if (C == CC && D == DD) {                                                                                 \
+    using IC = std::integral_constant<int, CC>;                                                             \
+    using ID = std::integral_constant<int, DD>;                                                             \
+    if (ib && ob) return f(IC{}, ID{}, __nv_bfloat16{}, __nv_bfloat16{}, TCB{});                            \
+    if (ib) return f(IC{}, ID{}, __nv_bfloat16{}, float{}, TCB{});                                          \
+    if (ob) return split ? f(IC{}, ID{}, float{}, __nv_bfloat16{}, TCF{}) : f(IC{}, ID{}, float{}, __nv_bfloat16{}, N{}); \
+    return split ? f(IC{}, ID{}, float{}, float{}, TCF{}) : f(IC{}, ID{}, float{}, float{}, N{});          \
   }
-  TPC_CASE(16, 32)
-  TPC_CASE(32, 64)
-  TPC_CASE(64, 128)
+  TPC_CASE(16, 32, N, N)
+  TPC_CASE(32, 64, N, N)
+  TPC_CASE(64, 128, Y, Y)
 #undef TPC_CASE
   return fail(TPC_ERR_UNSUPPORTED, "unsupported (chunk, d)");
 }
@@ -344,16 +349,19 @@ void* g_static_ptr[kMaxDevices] = {};
 cudaError_t g_static_rc[kMaxDevices] = {};
 std::once_flag g_static_once[kMaxDevices];
 
-// forward-only workspace: status word, W, U, Khat, decay, S0 and slot states
+// The array starts with the status word (a fixed place, read by tpc_kda_static_status), then the
+// plan tables, then the forward-only workspace: W, U, Khat, decay, S0 and slot states.
+constexpr size_t kStaticStatusBytes = 256;
+
 size_t static_ws_layout(const tpc::Plan& p, int H, int C, int D, size_t base, tpc::KdaWs* w, char* dev) {
   size_t o = base;
   auto take = [&](size_t bytes) { size_t r = o; o += a256(bytes); return r; };
   const size_t nc = p.chunks.size(), cd = (size_t)C * D, dd = (size_t)D * D;
-  const size_t st = take(256), W = take(nc * H * cd * 4), U = take(nc * H * cd * 4), K = take(nc * H * cd * 4);
+  const size_t W = take(nc * H * cd * 4), U = take(nc * H * cd * 4), K = take(nc * H * cd * 4);
   const size_t dec = take(nc * H * D * 4), S0 = take(nc * H * dd * 4), sl = take(p.slots.size() * H * dd * 4);
   if (w && dev) {
     *w = tpc::KdaWs{};
-    w->status = reinterpret_cast<int*>(dev + st);
+    w->status = reinterpret_cast<int*>(dev);
     w->W = reinterpret_cast<float*>(dev + W);
     w->U = reinterpret_cast<float*>(dev + U);
     w->Khat = reinterpret_cast<float*>(dev + K);
@@ -362,6 +370,21 @@ size_t static_ws_layout(const tpc::Plan& p, int H, int C, int D, size_t base, tp
     w->slot = reinterpret_cast<float*>(dev + sl);
   }
   return o;
+}
+
+// Device address of the scratch array on the current device: looked up once per device, with that
+// device current (cudaGetSymbolAddress), and cached.
+int static_base(char** out) {
+  int dev = 0;
+  TPC_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(TPC_ERR_UNSUPPORTED, "device ordinal out of range");
+  std::call_once(g_static_once[dev], [dev] {
+    g_static_rc[dev] = cudaGetSymbolAddress(&g_static_ptr[dev], g_static_scratch);
+  });
+  if (g_static_rc[dev] != cudaSuccess || !g_static_ptr[dev])
+    return fail(TPC_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(g_static_rc[dev]));
+  *out = static_cast<char*>(g_static_ptr[dev]);
+  return TPC_OK;
 }
 
 template <int C, int D, typename Tin, typename Tout>
@@ -392,6 +415,22 @@ int forward_static_impl(const tpc::Plan& p, const tpc::DevTables& dt, tpc::KdaWs
              (kda_fwd_out<C, D, Tin, Tout><<<dim3(nc, H), kThreads, out_smem<C, D>(), st>>>(
                  dt, H, q, k, g, static_cast<Tout*>(io->o), w)));
   return TPC_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Diagnostics: the bounded mbarrier wait every tensor-core kernel uses, on a barrier that nothing
+// arrives on and with no copy or MMA in flight, so that the wait runs out and the timeout path
+// (status word set, kernel returns, context intact) can be checked from the host.
+__global__ void wait_timeout_probe(int* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    tpc::tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const bool ok = tpc::tc::mbar_wait(&bar, 0, timeout_ns);
+  const int failed = __syncthreads_or(ok ? 0 : 1);
+  if (failed && threadIdx.x == 0) tpc::set_status(status, tpc::kStatusTimeout);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -558,8 +597,9 @@ int tpc_kda_forward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_
   if (ws_bytes < tpc_kda_workspace_bytes(plan, s)) return fail(TPC_ERR_WORKSPACE, "workspace too small");
   if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(TPC_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout) {
-    return forward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout)>(plan->p, s, io, ws, st);
+  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout, auto tc) {
+    return forward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout), decltype(tc)::value>(
+        plan->p, s, io, ws, st);
   });
 }
 
@@ -571,8 +611,9 @@ int tpc_kda_backward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda
     return fail(TPC_ERR_NULL, "backward: inputs, d_o, gradient outputs and ws are required");
   if (ws_bytes < tpc_kda_workspace_bytes(plan, s)) return fail(TPC_ERR_WORKSPACE, "workspace too small");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout) {
-    return backward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout)>(plan->p, s, io, ws, st);
+  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout, auto tc) {
+    return backward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout), decltype(tc)::value>(
+        plan->p, s, io, ws, st);
   });
 }
 
@@ -895,32 +936,46 @@ int tpc_kda_forward_static(const tpc_plan* plan, const tpc_kda_shape* s, const t
   const tpc::Plan& p = plan->p;
   std::vector<size_t> off;
   const size_t table_bytes = tpc::device_layout(p, off);
-  const size_t need = static_ws_layout(p, s->H, p.C, s->dk, a256(table_bytes), nullptr, nullptr);
+  const size_t need = static_ws_layout(p, s->H, p.C, s->dk, kStaticStatusBytes + a256(table_bytes), nullptr, nullptr);
   if (need > (size_t)TPC_STATIC_SCRATCH_BYTES)
     return fail(TPC_ERR_WORKSPACE, "problem needs " + std::to_string(need) + " bytes of device scratch; the "
                 "allocation-free forward holds at most " + std::to_string((size_t)TPC_STATIC_SCRATCH_BYTES));
-  int dev = 0;
-  TPC_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return fail(TPC_ERR_UNSUPPORTED, "device ordinal out of range");
-  // once per device, with that device current: the device address of the scratch array
-  std::call_once(g_static_once[dev], [dev] {
-    g_static_rc[dev] = cudaGetSymbolAddress(&g_static_ptr[dev], g_static_scratch);
-  });
-  if (g_static_rc[dev] != cudaSuccess || !g_static_ptr[dev])
-    return fail(TPC_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(g_static_rc[dev]));
-  char* base = static_cast<char*>(g_static_ptr[dev]);
+  char* base = nullptr;
+  if (int rc = static_base(&base)) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // plan tables at the start of the array (pageable source: staged before cudaMemcpyAsync returns)
+  // plan tables after the status word (pageable source: staged before cudaMemcpyAsync returns)
   std::vector<uint8_t> blob;
   tpc::pack_device_blob(p, off, blob);
-  TPC_CUDA(cudaMemcpyAsync(base, blob.data(), table_bytes, cudaMemcpyHostToDevice, st));
-  const tpc::DevTables dt = tpc::device_view(p, base, off);
+  char* tables = base + kStaticStatusBytes;
+  TPC_CUDA(cudaMemcpyAsync(tables, blob.data(), table_bytes, cudaMemcpyHostToDevice, st));
+  const tpc::DevTables dt = tpc::device_view(p, tables, off);
   tpc::KdaWs w;
-  static_ws_layout(p, s->H, p.C, s->dk, a256(table_bytes), &w, base);
-  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout) {
+  static_ws_layout(p, s->H, p.C, s->dk, kStaticStatusBytes + a256(table_bytes), &w, base);
+  return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout, auto) {
     return forward_static_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout)>(p, dt, w, s, io,
                                                                                                         st);
   });
+}
+
+int tpc_debug_wait_timeout(int32_t* status, int64_t timeout_ns, tpc_stream_t stream) {
+  if (!status) return fail(TPC_ERR_NULL, "status is NULL");
+  if (timeout_ns < 1000 || timeout_ns > 100000000) return fail(TPC_ERR_BAD_SHAPE, "timeout_ns in [1e3, 1e8]");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TPC_LAUNCH("wait_timeout_probe", st, (wait_timeout_probe<<<1, 32, 0, st>>>(status, (unsigned long long)timeout_ns)));
+  return TPC_OK;
+}
+
+int tpc_kda_static_status(tpc_stream_t stream) {
+  char* base = nullptr;
+  if (int rc = static_base(&base)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int code = 0;
+  TPC_CUDA(cudaStreamSynchronize(st));
+  TPC_CUDA(cudaMemcpy(&code, base, 4, cudaMemcpyDeviceToHost));
+  TPC_CUDA(cudaMemset(base, 0, 4));
+  if (code == TPC_ERR_RANGE) return fail(TPC_ERR_RANGE, "gate decay inside a 16-row sub-block exceeds 80 (log units)");
+  if (code) return fail(TPC_ERR_DEVICE_CHECK, "kernel-side check failed with code " + std::to_string(code));
+  return TPC_OK;
 }
 
 }  // extern "C"
