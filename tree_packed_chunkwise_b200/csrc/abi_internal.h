@@ -1,5 +1,6 @@
 // Internals shared by the translation units of the C ABI: error reporting, launch accounting.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <string>
@@ -18,6 +19,21 @@ namespace tpc_abi {
 int fail(int code, const std::string& msg);
 
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <class KernelT>
+cudaError_t set_smem(KernelT k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// multiprocessors of the current device (persistent grids)
+int sm_count();
+// 2-D bf16 TMA tensor map over [rows][cols] (leading dimension ld_elems): boxes of 64 columns x
+// box_rows rows, each box row one 128-byte swizzled line.
+bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems, uint32_t box_rows);
+// 3-D bf16 TMA tensor map over a [rows][heads][features] tensor: boxes of 64 features x 1 head x
+// box_rows rows in the 128-byte-swizzled layout; rows past the end read as zeros.
+bool tensor_map_rows(CUtensorMap* m, const void* ptr, uint64_t features, uint64_t heads, uint64_t rows,
+                     uint32_t box_rows);
 
 // Optional per-kernel timing: CUDA events around every launch (on the launching stream).
 struct Profiler {

@@ -24,6 +24,9 @@ struct KdaWs {
   float *Mt, *Bc;  // tensor-core path: per-chunk state transition M (bf16 hi/lo operand tile) and B (fp32)
   float *At, *Tm;  // tensor-core path: per-chunk gated key products Atilde and T = (I + diag(beta) Atilde)^{-1}
   float *Pm;       // tensor-core path: per-chunk masked gated products P = lower_incl(gated(q, k))
+  // The tensor-core path keeps W, U (U' then U), Pm, S0 and dS as hi/lo bf16 operand tiles (same
+  // bytes as fp32), and dU additionally as the tile dUt.
+  float *dUt;
 };
 
 template <int C, int D>

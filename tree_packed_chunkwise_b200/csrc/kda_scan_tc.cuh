@@ -4,7 +4,8 @@
 // B = Khat^T U' (both formed in parallel by the prep kernel; M is stored as a bf16 hi/lo tile in the
 // tensor-core operand layout).  The forward scan computes S <- M S + B per chunk, the backward scan
 // dS <- M^T dS + X (X = Qbar^T dO - W^T dU0), each as one M = 128 tcgen05 product per chunk (three
-// hi/lo chains) with the next chunk's M tile arriving by a bulk asynchronous copy meanwhile.
+// hi/lo chains) with the next chunk's M tile and additive term (B, resp. X, stored slice by slice:
+// [chunk][head][slice][row][32] fp32) arriving by bulk asynchronous copies meanwhile.
 // One CTA of 128 threads per (sequence of the round, head, 32-column slice of d_v); thread c owns
 // row c of the state slice.
 #pragma once
@@ -12,14 +13,17 @@
 
 namespace tpc {
 
-constexpr int kScanThreads = 128, kScanDVT = 32;
+// bytes of one chunk-head's additive-term slice (128 rows x 32 fp32)
+constexpr uint32_t kScanAddBytes = kTcD * kScanDVT * 4;
 
 struct ScanTcSmem {
   static constexpr size_t M0 = 0, M1 = kMtileBytes;              // double-buffered M tiles
   static constexpr size_t St = 2 * size_t(kMtileBytes);          // state slice hi/lo (MN-major, K = 128)
   static constexpr size_t StB = size_t(kTcD) * kScanDVT * 2;
-  static constexpr size_t total = St + 2 * StB;
+  static constexpr size_t Add = St + 2 * StB;                    // double-buffered additive-term slices
+  static constexpr size_t total = Add + 2 * size_t(kScanAddBytes);
 };
+
 
 namespace tck {
 
@@ -31,10 +35,13 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* st
   return !failed;
 }
 
-__device__ __forceinline__ void load_mtile(uint8_t* dst, const uint8_t* src, uint64_t* bar) {
-  tc::mbar_arrive_expect_tx(bar, kMtileBytes);
+// the chunk's M tile and this CTA's slice of its additive term, on one mbarrier
+__device__ __forceinline__ void load_mtile(uint8_t* dst, const uint8_t* src, float* add_dst, const float* add_src,
+                                           uint64_t* bar) {
+  tc::mbar_arrive_expect_tx(bar, kMtileBytes + kScanAddBytes);
 #pragma unroll
   for (int p = 0; p < 4; ++p) tc::bulk_g2s(dst + p * (kMtileBytes / 4), src + p * (kMtileBytes / 4), kMtileBytes / 4, bar);
+  tc::bulk_g2s(add_dst, add_src, kScanAddBytes, bar);
 }
 
 // state slice (row c = this thread, 32 columns) -> MN-major hi/lo operand tile (k = c, n = j)
@@ -69,6 +76,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   const SeqRec sq = t.seqs[si];
   extern __shared__ __align__(1024) uint8_t tsm[];
   uint8_t* mbuf[2] = {tsm + S::M0, tsm + S::M1};
+  float* abuf[2] = {reinterpret_cast<float*>(tsm + S::Add), reinterpret_cast<float*>(tsm + S::Add + kScanAddBytes)};
   uint8_t *sth = tsm + S::St, *stl = sth + S::StB;
   __shared__ __align__(8) uint64_t bar_m[2];
   __shared__ __align__(8) uint64_t bar_mma;
@@ -91,6 +99,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   auto mtile = [&](int ci) {
     return reinterpret_cast<const uint8_t*>(ws.Mt) + ((size_t)ci * H + h) * kMtileBytes;
   };
+  // this CTA's slice of the chunk's additive term: B (forward) or X (reverse), both kept in ws.Bc
+  auto addslice = [&](int ci) { return ws.Bc + ((size_t)ci * H + h) * D * D + (size_t)blockIdx.z * D * DVT; };
+  auto prefetch = [&](int q) {
+    const int ci = chunk_at(q);
+    load_mtile(mbuf[q & 1], mtile(ci), abuf[q & 1], addslice(ci), &bar_m[q & 1]);
+  };
   // initial value: forward -> initial / imported state; reverse -> gradient of the final state
   {
     const float* src = nullptr;
@@ -104,17 +118,13 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     else
       for (int j = 0; j < 32; ++j) s[j] = 0.f;
   }
-  if (c == 0) load_mtile(mbuf[0], mtile(chunk_at(0)), &bar_m[0]);
+  if (c == 0) prefetch(0);
   uint32_t mma_phase = 0;
   bool ok = true;
   for (int q = 0; q < nch && ok; ++q) {
     const int ci = chunk_at(q);
     const size_t base = (size_t)ci * H + h;
-    float add[32];
-    if (!REVERSE) {
-      st32g(ws.S0 + base * D * D + c * D + j0, s);               // chunk-start state
-      ld32g(ws.Bc + base * D * D + c * D + j0, add);             // B of this chunk
-    } else {
+    if (REVERSE) {
       const int slot = t.chunks[ci].export_slot;
       if (slot >= 0) {  // gradients of the exported boundary state, consumers in a fixed order
         const SlotRec sr = t.slots[slot];
@@ -124,19 +134,29 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           for (int j = 0; j < 32; ++j) s[j] += g2[j];
         }
       }
-      float* dSg = ws.dS + base * D * D + c * D + j0;
-      ld32g(dSg, add);   // X of this chunk
-      st32g(dSg, s);     // gradient of the chunk-end state, for the chunk kernels
     }
     put_state(sth, stl, c, s);
-    if (c == 0 && q + 1 < nch) load_mtile(mbuf[(q + 1) & 1], mtile(chunk_at(q + 1)), &bar_m[(q + 1) & 1]);
+    if (c == 0 && q + 1 < nch) prefetch(q + 1);
     ok = wait_all(&bar_m[q & 1], (q >> 1) & 1, ws.status);
     if (!ok) break;
+    float add[32];  // B (forward) or X (reverse) of this chunk, row c of the slice
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 u = reinterpret_cast<const float4*>(abuf[q & 1] + c * DVT)[i];
+      add[4 * i] = u.x; add[4 * i + 1] = u.y; add[4 * i + 2] = u.z; add[4 * i + 3] = u.w;
+    }
     tc::fence_async_smem();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     if (c == 0) {
+      // the state slice tile goes to the chunk kernels as it is: forward the chunk-start state S0,
+      // reverse the gradient of the chunk-end state (hi/lo operand tiles, this slice's 8 KB of each)
+      uint8_t* dst = reinterpret_cast<uint8_t*>(REVERSE ? ws.dS : ws.S0) + base * kStateTileBytes +
+                     (size_t)blockIdx.z * S::StB;
+      tc::bulk_s2g(dst, sth, (uint32_t)S::StB);
+      tc::bulk_s2g(dst + kStateTileBytes / 2, stl, (uint32_t)S::StB);
+      tc::bulk_commit();
       const tc::Op mH{tc::smem_u32(mbuf[q & 1]), D, REVERSE}, mL{tc::smem_u32(mbuf[q & 1] + kMtileBytes / 2), D, REVERSE};
       const tc::Op sH{tc::smem_u32(sth), D, true}, sL{tc::smem_u32(stl), D, true};
       mma4(tb, mH, mL, sH, sL, D, tc::idesc_bf16(D, DVT, REVERSE, true), false, false, false);
@@ -153,6 +173,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       const int slot = t.chunks[ci].export_slot;
       if (slot >= 0) st32g(ws.slot + ((size_t)slot * H + h) * D * D + c * D + j0, s);
     }
+    if (c == 0) tc::bulk_wait_read();
     tc::fence_before_sync();
     __syncthreads();  // the state tile and this M buffer are free again
   }
@@ -166,6 +187,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     // give copies still in flight a last bounded chance before the shared memory is released
     tc::mbar_wait(&bar_m[0], 0, 200000000ull);
   }
+  if (c == 0) tc::bulk_wait_all();
   tc::fence_before_sync();
   __syncthreads();
   if ((c >> 5) == 0) tc::tmem_dealloc(tb, 32);

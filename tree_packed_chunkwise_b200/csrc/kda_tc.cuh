@@ -24,8 +24,19 @@ namespace tpc {
 
 constexpr int kTcC = 64, kTcD = 128;
 constexpr uint32_t kMtileBytes = 2u * kTcD * kTcD * 2u;  // state transition tile: hi + lo bf16, 128 x 128
+// chunk-start state S0 and chunk-end state gradient dS as hi/lo bf16 operand tiles (element (c, j) at
+// cm_off(c, j, 128) in the hi half, the same in the lo half): one 128 x 128 tile per chunk and head
+constexpr uint32_t kStateTileBytes = 2u * kTcD * kTcD * 2u;
 constexpr float kMaxChunkDecay = 80.f;  // G_first - G_last per channel over one chunk
 enum : int { kStatusTimeout = 8 };
+// state scans: CTA size and width of the d_v slice one CTA owns
+constexpr int kScanThreads = 128, kScanDVT = 32;
+
+// offset (floats) of element (c, j) of a chunk-head's d x d additive term (B or X) in the
+// slice-major layout [slice][row][32] that the scans read by bulk copies
+__host__ __device__ __forceinline__ size_t slice_major(int c, int j) {
+  return ((size_t)(j / kScanDVT) * kTcD + c) * kScanDVT + (j % kScanDVT);
+}
 
 namespace tck {
 
@@ -252,6 +263,109 @@ __device__ __forceinline__ bool run(Sync& s, F issue) {
   s.phase ^= 1u;
   fence_after_sync();
   return true;
+}
+
+// Bulk asynchronous loads into shared memory, completion on their own mbarrier (issued by one
+// thread; every thread waits with ld_wait).
+struct Ld {
+  uint64_t* bar;
+  uint32_t phase;
+  int* status;
+};
+
+// one chunk-head's state tile (S0 or dS: hi half then lo half, kStateTileBytes) into hi and lo
+__device__ __forceinline__ void ld_state_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kStateTileBytes;
+  tc::mbar_arrive_expect_tx(l.bar, kStateTileBytes);
+  tc::bulk_g2s(hi, src, kStateTileBytes / 2, l.bar);
+  tc::bulk_g2s(lo, src + kStateTileBytes / 2, kStateTileBytes / 2, l.bar);
+}
+
+// one chunk-head's C x D hi/lo tile (hi half, then lo half: kCDTileBytes in all), and C x C tile
+constexpr uint32_t kCDTileBytes = 2u * kTcC * kTcD * 2u, kCCTileBytes = 2u * kTcC * kTcC * 2u;
+__device__ __forceinline__ void ld_cd_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kCDTileBytes;
+  tc::mbar_arrive_expect_tx(l.bar, kCDTileBytes);
+  tc::bulk_g2s(hi, src, kCDTileBytes / 2, l.bar);
+  tc::bulk_g2s(lo, src + kCDTileBytes / 2, kCDTileBytes / 2, l.bar);
+}
+__device__ __forceinline__ void ld_cc_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kCCTileBytes;
+  tc::mbar_arrive_expect_tx(l.bar, kCCTileBytes);
+  tc::bulk_g2s(hi, src, kCCTileBytes / 2, l.bar);
+  tc::bulk_g2s(lo, src + kCCTileBytes / 2, kCCTileBytes / 2, l.bar);
+}
+// bulk stores (issuing thread, after the tile writes were fenced and synchronised; the caller waits
+// with bulk_wait_read / bulk_wait_all before the shared buffers are reused or the CTA exits)
+__device__ __forceinline__ void store_cd_tile(float* tiles, size_t base, const uint8_t* hi, const uint8_t* lo) {
+  uint8_t* dst = reinterpret_cast<uint8_t*>(tiles) + base * kCDTileBytes;
+  tc::bulk_s2g(dst, hi, kCDTileBytes / 2);
+  tc::bulk_s2g(dst + kCDTileBytes / 2, lo, kCDTileBytes / 2);
+  tc::bulk_commit();
+}
+__device__ __forceinline__ void store_cc_tile(float* tiles, size_t base, const uint8_t* hi, const uint8_t* lo) {
+  uint8_t* dst = reinterpret_cast<uint8_t*>(tiles) + base * kCCTileBytes;
+  tc::bulk_s2g(dst, hi, kCCTileBytes / 2);
+  tc::bulk_s2g(dst + kCCTileBytes / 2, lo, kCCTileBytes / 2);
+  tc::bulk_commit();
+}
+// element (i, c) of a C x D hi/lo tile in global memory, 16 consecutive c from c0, as fp32 (hi + lo)
+__device__ __forceinline__ void cd_tile16(const float* tiles, size_t base, int i, int c0, float (&v)[16]) {
+  const uint8_t* t = reinterpret_cast<const uint8_t*>(tiles) + base * kCDTileBytes;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t off = cm_off(i, c0 + 8 * half, kTcC);
+    const uint4 h = __ldg(reinterpret_cast<const uint4*>(t + off));
+    const uint4 l = __ldg(reinterpret_cast<const uint4*>(t + kCDTileBytes / 2 + off));
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&h);
+    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&l);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 a = __bfloat1622float2(h2[k]), b = __bfloat1622float2(l2[k]);
+      v[8 * half + 2 * k] = a.x + b.x;
+      v[8 * half + 2 * k + 1] = a.y + b.y;
+    }
+  }
+}
+
+// bounded wait for the loads issued on l (CTA-wide vote); false on every thread after recording
+// TPC_ERR_TIMEOUT
+__device__ __forceinline__ bool ld_wait(Ld& l) {
+  const bool ok = tc::mbar_wait(l.bar, l.phase);
+  const int failed = __syncthreads_or(ok ? 0 : 1);
+  if (failed) {
+    if (threadIdx.x == 0) set_status(l.status, kStatusTimeout);
+    tc::mbar_wait(l.bar, l.phase, 200000000ull);  // copies still in flight get a last bounded chance
+    return false;
+  }
+  l.phase ^= 1u;
+  return true;
+}
+
+// sum over j of a(c, j) b(c, j) for two state tiles in global memory (hi + lo of each), row c
+__device__ __forceinline__ float state_row_dot(const float* ta, const float* tb, size_t base, int c) {
+  const uint8_t* a = reinterpret_cast<const uint8_t*>(ta) + base * kStateTileBytes;
+  const uint8_t* b = reinterpret_cast<const uint8_t*>(tb) + base * kStateTileBytes;
+  float acc = 0.f;
+  for (int j0 = 0; j0 < kTcD; j0 += 8) {
+    const uint32_t off = cm_off(c, j0, kTcD);
+    const uint4 ah = __ldg(reinterpret_cast<const uint4*>(a + off));
+    const uint4 al = __ldg(reinterpret_cast<const uint4*>(a + kStateTileBytes / 2 + off));
+    const uint4 bh = __ldg(reinterpret_cast<const uint4*>(b + off));
+    const uint4 bl = __ldg(reinterpret_cast<const uint4*>(b + kStateTileBytes / 2 + off));
+    const __nv_bfloat162* ah2 = reinterpret_cast<const __nv_bfloat162*>(&ah);
+    const __nv_bfloat162* al2 = reinterpret_cast<const __nv_bfloat162*>(&al);
+    const __nv_bfloat162* bh2 = reinterpret_cast<const __nv_bfloat162*>(&bh);
+    const __nv_bfloat162* bl2 = reinterpret_cast<const __nv_bfloat162*>(&bl);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 x1 = __bfloat1622float2(ah2[k]), x2 = __bfloat1622float2(al2[k]);
+      const float2 y1 = __bfloat1622float2(bh2[k]), y2 = __bfloat1622float2(bl2[k]);
+      acc = fmaf(x1.x + x2.x, y1.x + y2.x, acc);
+      acc = fmaf(x1.y + x2.y, y1.y + y2.y, acc);
+    }
+  }
+  return acc;
 }
 
 // three chains: hi*hi + lo*hi + hi*lo (both operands split) or two (b exact: lo of b absent)
@@ -482,23 +596,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // phase 3: the chunk's state transition S_end = M S_0 + B with M = Diag(e^{G_C}) - Khat^T W and
       // B = Khat^T U' (Khat = k e^{G_C - G})
       const size_t base = (size_t)ci * H + h;
-      float* Wg = ws.W + base * C * D;
-      float* Ug = ws.U + base * C * D;
       uint8_t *wth = tl, *wtl = tl + S::CDb, *uth = tl + 2 * S::CDb, *utl = tl + 3 * S::CDb, *khh = tl + 4 * S::CDb,
               *khl = tl + 5 * S::CDb;
-      acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) {
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(Wg + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        put16<C, true>(wth, wtl, r, c0, v);  // element (i, c): MN-major (k = i)
-      });
-      acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) {
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(Ug + r * D + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        put16<C, true>(uth, utl, r, c0, v);
-      });
+      // W and U' as hi/lo tiles, element (i, c) at cm_off(i, c, C): the operands of this phase and,
+      // stored as they are, of the output and backward kernels
+      acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) { put16<C, true>(wth, wtl, r, c0, v); });
+      acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) { put16<C, true>(uth, utl, r, c0, v); });
       const float* gC = sG + (n - 1) * LD;
       build_tile_ld<C, D, true, Tin>(khh, khl, row_k, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
       ok = run(sy, [&] {
+        store_cd_tile(ws.W, base, wth, wtl);
+        store_cd_tile(ws.U, base, uth, utl);
         const uint32_t id = tc::idesc_bf16(D, D, true, true);
         const tc::Op kH{tc::smem_u32(khh), C, true}, kL{tc::smem_u32(khl), C, true};
         const tc::Op wH{tc::smem_u32(wth), C, true}, wL{tc::smem_u32(wtl), C, true};
@@ -515,13 +623,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 16; ++j) m[j] = (c0 + j == c ? gam : 0.f) - v[j];
           put16<D, true>(Mt, Mt + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
         });
-        acc_read<D, D>(tb, 128, [&](int c, int j0, const float* v) {
+        acc_read<D, D>(tb, 128, [&](int c, int j0, const float* v) {  // slice-major for the scan's bulk loads
           for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(Bg + c * D + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            *reinterpret_cast<float4*>(Bg + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         });
       }
     }
   }
+  if (tid == 0) tc::bulk_wait_all();
   tc::fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
@@ -557,14 +666,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sG = reinterpret_cast<float*>(tsm + S::G);
   float* sref = reinterpret_cast<float*>(tsm + S::vec);
   __shared__ int srow[C];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
+  const size_t base = (size_t)ci * H + h;
+  uint8_t *s0h = tsm + S::S0, *s0l = s0h + S::DDb;
   for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  Ld ld{&bar_ld, 0u, ws.status};
   if (tid == 0) {
     tc::mbar_init(&bar, 1);
+    tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    ld_state_tile(ld, s0h, s0l, ws.S0, base);  // the chunk-start state, as the scan left it
+    ld_cd_tile(ld, tsm + S::Wq, tsm + S::Wq + S::CDb, ws.W, base);  // W, as the prep kernel left it
   }
   __syncthreads();
   load_gate(sG, LD, g_, srow, H, h, n);
@@ -576,19 +691,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   Sync sy{&bar, 0u, ws.status};
   auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  const size_t base = (size_t)ci * H + h;
-  const float* S0g = ws.S0 + base * D * D;
-  const float* Wg = ws.W + base * C * D;
-  float* Ug = ws.U + base * C * D;
   // TMEM: P [0,64), W S0 [64,192), O [192,320)
   uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
-  uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb, *s0h = tsm + S::S0, *s0l = s0h + S::DDb;
+  uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb;
   build_tile_ld<C, D, true, Tin>(qfh, qfl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
   build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
-  build_tile_ld<C, D, true, float>(wh, wl, [&](int r) { return Wg + r * D; }, [&](int, int, float x) { return x; });
-  build_tile_ld<D, D, true, float>(s0h, s0l, [&](int c) { return S0g + c * D; }, [&](int, int, float x) { return x; });
   const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
-  bool ok = run(sy, [&] {
+  bool ok = ld_wait(ld);
+  ok = ok && run(sy, [&] {
     const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
     const tc::Op wH{tc::smem_u32(wh), C, false}, wL{tc::smem_u32(wl), C, false};
@@ -598,24 +708,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
   uint8_t *qbh = wh, *qbl = wl;
   if (ok) {
-    float* Pg = ws.Pm + base * C * C;  // kept for the backward
     acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
       float m[16];
       for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
-      put16<C, true>(ph, pl, r, i0, m);
-      st16g(Pg + r * C + i0, m);
+      put16<C, true>(ph, pl, r, i0, m);  // kept (as this tile) for the backward
     });
     acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
       float u[16];
-      for (int j = 0; j < 16; j += 4) {
-        const float4 up = *reinterpret_cast<const float4*>(Ug + i * D + j0 + j);
-        u[j] = up.x - v[j]; u[j + 1] = up.y - v[j + 1]; u[j + 2] = up.z - v[j + 2]; u[j + 3] = up.w - v[j + 3];
-        *reinterpret_cast<float4*>(Ug + i * D + j0 + j) = make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
-      }
-      put16<C, true>(uh, ul, i, j0, u);  // element (i, j): MN-major (k = i)
+      cd_tile16(ws.U, base, i, j0, u);  // U'
+      for (int j = 0; j < 16; ++j) u[j] -= v[j];
+      put16<C, true>(uh, ul, i, j0, u);  // element (i, j): MN-major (k = i); kept for the backward
     });
     build_tile_ld<C, D, true, Tin>(qbh, qbl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c]); });
     ok = run(sy, [&] {
+      store_cc_tile(ws.Pm, base, ph, pl);
+      store_cd_tile(ws.U, base, uh, ul);  // U replaces U'
+
       const uint32_t id = tc::idesc_bf16(C, D, false, true);
       const tc::Op qH{tc::smem_u32(qbh), C, false}, qL{tc::smem_u32(qbl), C, false};
       const tc::Op pH{tc::smem_u32(ph), C, false}, pL{tc::smem_u32(pl), C, false};
@@ -632,6 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       });
     }
   }
+  if (tid == 0) tc::bulk_wait_all();
   tc::fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
@@ -649,7 +758,7 @@ struct BprepTcSmem {
   static constexpr size_t R = tiles;             // qf, bf (4 CDb) -> P (2 CCb) + dU0 (2 CDb)
   static constexpr size_t Qb = R + 4 * CDb;      // Qbar, MN-major
   static constexpr size_t dO = Qb + 2 * CDb;     // dO, MN-major
-  static constexpr size_t Wt = dO + 2 * CDb;     // -W, MN-major
+  static constexpr size_t Wt = dO + 2 * CDb;     // W (as the prep kernel stored it), used MN-major
   static constexpr size_t total = Wt + 2 * CDb;
 };
 
@@ -668,14 +777,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sG = reinterpret_cast<float*>(tsm + S::G);
   float* sref = reinterpret_cast<float*>(tsm + S::vec);
   __shared__ int srow[C];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
+  const size_t base = (size_t)ci * H + h;
+  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *doh = tsm + S::dO, *dol = doh + S::CDb;
+  uint8_t *wh = tsm + S::Wt, *wl = wh + S::CDb;
+  // P (masked gated q k products; element (r, i), the MN-major operand P^T) as the forward left it
+  uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *duh = pl + S::CCb, *dul = duh + S::CDb;
   for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  Ld ld{&bar_ld, 0u, ws.status};
   if (tid == 0) {
     tc::mbar_init(&bar, 1);
+    tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    ld_cd_tile(ld, wh, wl, ws.W, base);
+    ld_cc_tile(ld, ph, pl, ws.Pm, base);
   }
   __syncthreads();
   load_gate(sG, LD, g_, srow, H, h, n);
@@ -690,26 +808,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto row_do = [&](int a) -> const Tin* {
     return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
   };
-  const size_t base = (size_t)ci * H + h;
-  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *doh = tsm + S::dO, *dol = doh + S::CDb;
-  uint8_t *wh = tsm + S::Wt, *wl = wh + S::CDb;
   build_tile_ld<C, D, true, Tin>(qbh, qbl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c]); });
   build_tile_ld<C, D, !EX, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
-  const float* Wg = ws.W + base * C * D;
-  build_tile_ld<C, D, true, float>(wh, wl, [&](int r) { return Wg + r * D; }, [&](int, int, float x) { return -x; });
-  // P (masked gated q k products) as the forward left it
-  uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *duh = pl + S::CCb, *dul = duh + S::CDb;
-  {
-    const float* Pg = ws.Pm + base * C * C;
-    for (int e = tid; e < C * (C / 16); e += blockDim.x) {
-      const int r = e / (C / 16), i0 = (e % (C / 16)) * 16;
-      float m[16];
-      ld16g(Pg + r * C + i0, m);
-      put16<C, true>(ph, pl, r, i0, m);  // element (r, i): MN-major operand P^T (k = r, m = i)
-    }
-  }
-  bool ok = true;
-  {
+  bool ok = ld_wait(ld);
+  if (ok) {
     ok = run(sy, [&] {
       const tc::Op pH{tc::smem_u32(ph), C, true}, pL{tc::smem_u32(pl), C, true};
       const tc::Op oH{tc::smem_u32(doh), C, true}, oL{tc::smem_u32(dol), C, true};
@@ -719,9 +821,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     float* dU = ws.dU + base * C * D;
     acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
+      float m[16];
       for (int j = 0; j < 16; j += 4)
         *reinterpret_cast<float4*>(dU + i * D + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-      put16<C, true>(duh, dul, i, j0, v);  // element (i, j): MN-major operand (k = i, n = j)
+      for (int j = 0; j < 16; ++j) m[j] = -v[j];
+      put16<C, true>(duh, dul, i, j0, m);  // -dU0, element (i, j): MN-major operand (k = i, n = j)
     });
     ok = run(sy, [&] {
       const uint32_t id = tc::idesc_bf16(D, D, true, true);
@@ -734,10 +838,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
   }
   if (ok) {
-    float* X = ws.dS + base * D * D;
+    // X goes where the forward kept B (dead once the forward scans are done), slice-major for the
+    // reverse scan's bulk loads
+    float* X = ws.Bc + base * D * D;
     acc_read<D, D>(tb, 192, [&](int c, int j0, const float* v) {
       for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(X + c * D + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        *reinterpret_cast<float4*>(X + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     });
   }
   tc::fence_before_sync();
@@ -780,14 +886,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sG = reinterpret_cast<float*>(tsm + S::G);
   float* sref = reinterpret_cast<float*>(tsm + S::vec);
   __shared__ int srow[C];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
+  const size_t base = (size_t)ci * H + h;
+  uint8_t *doh = tsm + S::R, *dol = doh + S::CDb, *uh = dol + S::CDb, *ul = uh + S::CDb;
+  uint8_t *sh = ul + S::CDb, *sl = sh + S::DDb;
   for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  Ld ld{&bar_ld, 0u, ws.status};
   if (tid == 0) {
     tc::mbar_init(&bar, 1);
+    tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
+    ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
   }
   __syncthreads();
   load_gate(sG, LD, g_, srow, H, h, n);
@@ -802,44 +915,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto row_do = [&](int a) -> const Tin* {
     return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
   };
-  const size_t base = (size_t)ci * H + h;
-  const float* S0g = ws.S0 + base * D * D;
-  const float* dSg = ws.dS + base * D * D;
-  const float* Ug = ws.U + base * C * D;
   // TMEM columns: Tq [0,128), T1 [128,256), RS [256,384), dP [384,448) then CS [384,512)
   constexpr int cTq = 0, cT1 = 128, cRS = 256, cCS = 384;
-  uint8_t *doh = tsm + S::R, *dol = doh + S::CDb, *uh = dol + S::CDb, *ul = uh + S::CDb;
-  uint8_t *sh = ul + S::CDb, *sl = sh + S::DDb;
   build_tile_ld<C, D, !EX, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
-  build_tile_ld<C, D, true, float>(uh, ul, [&](int i) { return Ug + i * D; }, [&](int, int, float x) { return x; });
-  build_tile_ld<D, D, true, float>(sh, sl, [&](int c) { return S0g + c * D; }, [&](int, int, float x) { return x; });
   const tc::Op oH{tc::smem_u32(doh), C, false}, oL{tc::smem_u32(dol), C, false};
   const tc::Op uH{tc::smem_u32(uh), C, false}, uL{tc::smem_u32(ul), C, false};
   const tc::Op sH{tc::smem_u32(sh), D, false}, sL{tc::smem_u32(sl), D, false};
-  bool ok = run(sy, [&] {
+  bool ok = ld_wait(ld);
+  ok = ok && run(sy, [&] {
     mma4(tb + cCS, oH, oL, uH, uL, D, tc::idesc_bf16(C, C, false, false), false, EX, false);   // dP (raw)
     mma4(tb + cTq, oH, oL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, EX, false);  // Tq
   });
   if (ok) {
-    // phase 2: T1 = U dS^T and dU = dU0 + Khat dS (Khat = k e^{G_C - G}, K-major in the dO slot)
-    build_tile_ld<D, D, true, float>(sh, sl, [&](int c) { return dSg + c * D; }, [&](int, int, float x) { return x; });
+    // phase 2: T1 = U dS^T and dU = dU0 + Khat dS (Khat = k e^{G_C - G}, K-major in the dO slot);
+    // the gradient of the chunk-end state replaces S0 in its buffer
+    if (tid == 0) ld_state_tile(ld, sh, sl, ws.dS, base);
     const float* gC = sG + (n - 1) * LD;
     build_tile_ld<C, D, true, Tin>(doh, dol, row_k, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
-    ok = run(sy, [&] {
+    ok = ld_wait(ld);
+    ok = ok && run(sy, [&] {
       mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
       const tc::Op kH{tc::smem_u32(doh), C, false}, kL{tc::smem_u32(dol), C, false};
       const tc::Op dH{tc::smem_u32(sh), D, true}, dL{tc::smem_u32(sl), D, true};
       mma4(tb + cRS, kH, kL, dH, dL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
     });
     if (ok) {
-      float* dUg = ws.dU + base * C * D;
+      // dU = dU0 + Khat dS as a hi/lo tile (element (i, j) at cm_off(i, j, C), in the consumed Khat
+      // slot) for the dk / dv kernel
+      const float* dUg = ws.dU + base * C * D;
       acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) {
+        float u[16];
         for (int j = 0; j < 16; j += 4) {
-          float4 u = *reinterpret_cast<const float4*>(dUg + i * D + j0 + j);
-          u.x += v[j]; u.y += v[j + 1]; u.z += v[j + 2]; u.w += v[j + 3];
-          *reinterpret_cast<float4*>(dUg + i * D + j0 + j) = u;
+          const float4 a = *reinterpret_cast<const float4*>(dUg + i * D + j0 + j);
+          u[j] = a.x + v[j]; u[j + 1] = a.y + v[j + 1]; u[j + 2] = a.z + v[j + 2]; u[j + 3] = a.w + v[j + 3];
         }
+        put16<C, true>(doh, dol, i, j0, u);
       });
+      tc::fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        store_cd_tile(ws.dUt, base, doh, dol);
+        tc::bulk_wait_read();
+      }
+      __syncthreads();
     }
   }
   uint8_t *pH8 = tsm + S::R, *pL8 = pH8 + S::CCb, *bh = pL8 + S::CCb, *bl = bh + S::CDb, *qh = bl + S::CDb,
@@ -902,15 +1020,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = tid; c < D; c += blockDim.x) {
       float acc = 0.f;
       for (int i = 0; i < n; ++i) acc += sbuf[i * LD + c];
-      float acc2 = 0.f;
-      for (int j = 0; j < D; j += 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(dSg + c * D + j));
-        const float4 b = __ldg(reinterpret_cast<const float4*>(S0g + c * D + j));
-        acc2 = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc2))));
-      }
+      const float acc2 = state_row_dot(ws.dS, ws.S0, base, c);  // sum_j dS_cj S0_cj
       pdG[(n - 1) * D + c] += acc + expf(sG[(n - 1) * LD + c]) * acc2;
     }
   }
+  if (tid == 0) tc::bulk_wait_all();
   tc::fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
@@ -976,13 +1090,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* tTl = tTh + S::CCb;
   uint8_t* R = tsm + S::R;
   __shared__ int srow[C];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
   for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
+  Ld ld{&bar_ld, 0u, ws.status};
   if (tid == 0) {
     tc::mbar_init(&bar, 1);
+    tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -1019,8 +1135,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
   const size_t base = (size_t)ci * H + h;
-  const float* S0g = ws.S0 + base * D * D;
-  const float* dUg = ws.dU + base * C * D;
   float* pdk = ws.pdk + base * C * D;
   float* pdG = ws.pdG + base * C * D;
   const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
@@ -1066,9 +1180,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // ---- phase 2b: dW' = dU S0^T
     uint8_t *duh = R + S::p2_dU, *dul = duh + S::CDb, *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
-    build_tile_ld<C, D, true, float>(duh, dul, [&](int r) { return dUg + r * D; }, [&](int, int, float x) { return x; });
-    build_tile_ld<D, D, true, float>(s0h, s0l, [&](int c) { return S0g + c * D; }, [&](int, int, float x) { return x; });
-    ok = run(sy, [&] {
+    if (tid == 0) {  // the phase 2a operands are consumed
+      ld_state_tile(ld, s0h, s0l, ws.S0, base);
+      ld_cd_tile(ld, duh, dul, ws.dUt, base);
+    }
+    ok = ld_wait(ld);
+    ok = ok && run(sy, [&] {
       const tc::Op aH{tc::smem_u32(duh), C, false}, aL{tc::smem_u32(dul), C, false};
       const tc::Op bH{tc::smem_u32(s0h), D, false}, bL{tc::smem_u32(s0l), D, false};
       mma4(tb + cdW, aH, aL, bH, bL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
@@ -1084,8 +1201,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) m[j] = -v[j];
       put16<C, true>(dxh, dxl, r, c0, m);
     });
-    build_tile_ld<C, D, true, float>(dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), [&](int r) { return dUg + r * D; }, [&](int, int, float x) { return x; });
-    ok = run(sy, [&] {
+    if (tid == 0) ld_cd_tile(ld, dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), ws.dUt, base);
+    ok = ld_wait(ld);
+    ok = ok && run(sy, [&] {
       const tc::Op aH{tc::smem_u32(tTh), C, true}, aL{tc::smem_u32(tTl), C, true};
       const tc::Op bH{tc::smem_u32(dxh), C, true}, bL{tc::smem_u32(dxl), C, true};
       mma4(tb + cdB, aH, aL, bH, bL, C, tc::idesc_bf16(C, 2 * D, true, true), false, false, false);

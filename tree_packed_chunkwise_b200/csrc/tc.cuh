@@ -126,6 +126,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                : "memory");
 }
 
+// Bulk asynchronous copy this CTA's shared memory -> global (bulk async-group of the issuing thread).
+// Addresses 16-byte aligned, bytes a multiple of 16.  The writing threads make the shared data
+// visible first (fence_async_smem + barrier); the issuing thread commits the group and waits for it.
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// waits until this thread's committed bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// waits until this thread's committed bulk stores are complete (visible in global memory)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Tiled TMA load (2-D tensor map, no multicast) into this CTA's shared memory; the innermost
 // coordinate x must be a multiple of 8 elements for bf16 (16 bytes).
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {

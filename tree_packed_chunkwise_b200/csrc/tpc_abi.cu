@@ -13,9 +13,6 @@
 #include "kda_kernels.cuh"
 #include "kda_tc.cuh"
 #include "kda_scan_tc.cuh"
-#include "gemm_tc.cuh"
-#include "logprob_kernels.cuh"
-#include "attn_tc.cuh"
 #include <cudaTypedefs.h>
 #include "abi_internal.h"
 #include "plan.h"
@@ -31,6 +28,65 @@ int fail(int code, const std::string& msg) {
   return code;
 }
 
+// ------------------------------------------------------------------------------------------------
+// TMA tensor maps (driver entry point looked up through the runtime; no link against libcuda)
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+}  // namespace
+
+// multiprocessors of the current device (persistent grids)
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n < 1)
+    return 148;
+  return n;
+}
+
+// the driver's tensor-map encoder (looked up once)
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void**>(&g_encode), cudaEnableDefault,
+                                &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      g_encode = nullptr;
+  });
+  return g_encode;
+}
+
+// 2-D bf16 tensor map over [rows][cols] (leading dimension ld_elems): boxes of 64 columns x box_rows
+// rows, each box row one 128-byte swizzled line.
+bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems,
+                uint32_t box_rows) {
+  const auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 tensor map over a [rows][heads][features] tensor (feature dimension contiguous): boxes
+// of 64 features x 1 head x box_rows rows, each box row one 128-byte swizzled line; rows past the
+// end read as zeros.
+bool tensor_map_rows(CUtensorMap* m, const void* ptr, uint64_t features, uint64_t heads, uint64_t rows,
+                     uint32_t box_rows) {
+  const auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {features, heads, rows};
+  cuuint64_t strides[2] = {features * 2, heads * features * 2};
+  cuuint32_t box[3] = {64, 1, box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tpc_abi
 
 namespace {
@@ -38,6 +94,7 @@ namespace {
 using tpc_abi::a256;
 using tpc_abi::fail;
 using tpc_abi::g_prof;
+using tpc_abi::set_smem;
 
 #define TPC_TRY_ABI(call)        \
   do {                           \
@@ -97,6 +154,7 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
   w.rdk = f(L.rdk); w.rdv = f(L.rdv); w.rdg = f(L.rdg); w.rdb = f(L.rdb);
   w.tdk = f(L.tdk); w.tdv = f(L.tdv); w.tdg = f(L.tdg); w.tdb = f(L.tdb);
   w.Mt = f(L.Mt); w.Bc = f(L.Bc); w.At = f(L.At); w.Tm = f(L.Tm); w.Pm = f(L.Pm);
+  w.dUt = f(L.Khat);  // the tensor-core path keeps its dU tile where the CUDA-core path keeps Khat
   return w;
 }
 
@@ -115,11 +173,6 @@ int check_shape(const tpc_plan* plan, const tpc_kda_shape* s) {
   if (s->in_dtype == TPC_F32_SPLIT && !(plan->p.C == tpc::kTcC && s->dk == tpc::kTcD))
     return fail(TPC_ERR_UNSUPPORTED, "TPC_F32_SPLIT is built for chunk 64, d 128 (the tensor-core path)");
   return TPC_OK;
-}
-
-template <class KernelT>
-cudaError_t set_smem(KernelT k, size_t bytes) {
-  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 // A high-priority stream per device for the sequential state scans (created once, non-blocking,
@@ -433,62 +486,6 @@ __global__ void wait_timeout_probe(int* status, unsigned long long timeout_ns) {
   if (failed && threadIdx.x == 0) tpc::set_status(status, tpc::kStatusTimeout);
 }
 
-// ------------------------------------------------------------------------------------------------
-// TMA tensor maps (driver entry point looked up through the runtime; no link against libcuda)
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-// multiprocessors of the current device (persistent grids)
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      n < 1)
-    return 148;
-  return n;
-}
-
-// the driver's tensor-map encoder (looked up once)
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-  std::call_once(g_encode_once, [] {
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void**>(&g_encode), cudaEnableDefault,
-                                &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      g_encode = nullptr;
-  });
-  return g_encode;
-}
-
-// 2-D bf16 tensor map over [rows][cols] (leading dimension ld_elems): boxes of 64 columns x box_rows
-// rows, each box row one 128-byte swizzled line.
-bool tensor_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld_elems,
-                uint32_t box_rows) {
-  const auto enc = encoder();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {ld_elems * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 3-D bf16 tensor map over a [rows][heads][features] tensor (feature dimension contiguous): boxes
-// of 64 features x 1 head x box_rows rows, each box row one 128-byte swizzled line; rows past the
-// end read as zeros.
-bool tensor_map_rows(CUtensorMap* m, const void* ptr, uint64_t features, uint64_t heads, uint64_t rows,
-                     uint32_t box_rows) {
-  const auto enc = encoder();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {features, heads, rows};
-  cuuint64_t strides[2] = {features * 2, heads * features * 2};
-  cuuint32_t box[3] = {64, 1, box_rows};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 }  // namespace
 
@@ -667,228 +664,6 @@ int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t st
   TPC_LAUNCH("occurrence_count", st,
              (tpc::occurrence_count_kernel<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(plan->p.dt, counts, N)));
   return TPC_OK;
-}
-
-int tpc_gemm_split(const void* A, const void* A_lo, const void* B, const void* B_lo, void* C, int64_t M, int64_t N,
-                   int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype,
-                   float alpha, float beta, int32_t* status, tpc_stream_t stream) {
-  if (!A || !B || !C) return fail(TPC_ERR_NULL, "gemm: A, B and C are required");
-  if (M < 1 || N < 1 || K < 1 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30))
-    return fail(TPC_ERR_BAD_SHAPE, "gemm: sizes must be in [1, 2^30]");
-  auto misaligned = [](const void* p) { return p && (reinterpret_cast<uintptr_t>(p) % 16) != 0; };
-  if ((lda % 8) || (ldb % 8) || misaligned(A) || misaligned(B) || misaligned(A_lo) || misaligned(B_lo))
-    return fail(TPC_ERR_BAD_SHAPE, "gemm: A and B need 16-byte aligned bases and leading dimensions multiple of 8");
-  if (c_dtype != TPC_F32 && c_dtype != TPC_BF16) return fail(TPC_ERR_UNSUPPORTED, "gemm: C is fp32 or bf16");
-  if (c_dtype == TPC_BF16 && beta != 0.f) return fail(TPC_ERR_UNSUPPORTED, "gemm: beta needs an fp32 C");
-  if (a_mn ? (lda < M) : (lda < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: lda too small");
-  if (b_mn ? (ldb < N) : (ldb < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldb too small");
-  if (ldc < N) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldc too small");
-  if (B_lo && !A_lo) return fail(TPC_ERR_UNSUPPORTED, "gemm: B_lo needs A_lo (three-product form)");
-  // 128-byte-swizzled boxes 64 elements wide: K-major [mn][K] boxes of 64 (K) x tile rows,
-  // MN-major [K][mn] boxes of 64 (mn) x 64 (K)
-  auto encode = [&](CUtensorMap* m, const void* X, bool mn_major, int64_t mn, int64_t ld, int box) {
-    return mn_major ? tensor_map(m, X, mn, K, ld, tpc::kGemmBK) : tensor_map(m, X, K, mn, ld, box);
-  };
-  // tile height: 256 rows (two halves) once K is long enough to hide the non-overlapped epilogue
-  const int HV = K >= tpc::kGemmLongK ? 2 : 1;
-  const int BM = tpc::kGemmHalf * HV;
-  CUtensorMap ta, tb, talo, tblo;
-  bool ok = encode(&ta, A, a_mn, M, lda, BM) && encode(&tb, B, b_mn, N, ldb, tpc::kGemmBN);
-  ok = ok && encode(&talo, A_lo ? A_lo : A, a_mn, M, lda, BM);
-  ok = ok && encode(&tblo, B_lo ? B_lo : B, b_mn, N, ldb, tpc::kGemmBN);
-  if (!ok) return fail(TPC_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
-  const int passes = B_lo ? 3 : (A_lo ? 2 : 1);
-  tpc::GemmArgs g{(int)M, (int)N, (int)K, a_mn, b_mn, c_dtype, (long long)ldc, alpha, beta, C, status, passes,
-                  M < N ? 1 : 0};
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t tiles = ((N + tpc::kGemmBN - 1) / tpc::kGemmBN) * ((M + BM - 1) / BM);
-  if (tiles > (int64_t)1 << 31) return fail(TPC_ERR_BAD_SHAPE, "gemm: too many tiles");
-  const dim3 grid((unsigned)std::min<int64_t>(tiles, sm_count()));
-  auto go = [&](auto cb, auto hv) -> int {
-    constexpr int CB = decltype(cb)::value, H2 = decltype(hv)::value;
-    constexpr size_t smem = tpc::GemmCfg<H2>::total;
-    TPC_CUDA(set_smem(tpc::gemm_bf16_tc<CB, H2>, smem));
-    TPC_LAUNCH("gemm_bf16_tc", st,
-               (tpc::gemm_bf16_tc<CB, H2><<<grid, tpc::kGemmThreadsP, smem, st>>>(ta, tb, talo, tblo, g)));
-    return TPC_OK;
-  };
-  using I0 = std::integral_constant<int, 0>;
-  using I1 = std::integral_constant<int, 1>;
-  using I2 = std::integral_constant<int, 2>;
-  if (c_dtype == TPC_BF16) return HV == 2 ? go(I1{}, I2{}) : go(I1{}, I1{});
-  return HV == 2 ? go(I0{}, I2{}) : go(I0{}, I1{});
-}
-
-int tpc_gemm_bf16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
-                  int64_t ldc, int32_t a_mn, int32_t b_mn, int32_t c_dtype, float alpha, float beta, int32_t* status,
-                  tpc_stream_t stream) {
-  return tpc_gemm_split(A, nullptr, B, nullptr, C, M, N, K, lda, ldb, ldc, a_mn, b_mn, c_dtype, alpha, beta, status,
-                        stream);
-}
-
-size_t tpc_logprob_scratch_bytes(int64_t V, int32_t chunk_rows) {
-  if (V < 1 || chunk_rows < 1) return 0;
-  return a256((size_t)chunk_rows * V * 4) + 2 * a256((size_t)chunk_rows * V * 2);
-}
-
-namespace {
-int logprob_check(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh, const int32_t* targets,
-                  void* scratch, size_t scratch_bytes, int32_t chunk_rows) {
-  if (!plan || !h || !W || !targets || !scratch) return fail(TPC_ERR_NULL, "logprob: NULL argument");
-  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
-  if (V < 8 || Dh < 8 || (V % 8) || (Dh % 8)) return fail(TPC_ERR_BAD_SHAPE, "logprob: V and Dh multiples of 8");
-  if (chunk_rows < 1) return fail(TPC_ERR_BAD_SHAPE, "logprob: chunk_rows >= 1");
-  if (scratch_bytes < tpc_logprob_scratch_bytes(V, chunk_rows)) return fail(TPC_ERR_WORKSPACE, "logprob: scratch too small");
-  if (reinterpret_cast<uintptr_t>(scratch) % 256) return fail(TPC_ERR_WORKSPACE, "logprob: scratch must be 256-byte aligned");
-  return TPC_OK;
-}
-}  // namespace
-
-int tpc_logprob_forward(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh,
-                        const int32_t* targets, float* logp, float* lse, void* scratch, size_t scratch_bytes,
-                        int32_t chunk_rows, int32_t* status, tpc_stream_t stream) {
-  if (int rc = logprob_check(plan, h, W, V, Dh, targets, scratch, scratch_bytes, chunk_rows)) return rc;
-  if (!logp || !lse) return fail(TPC_ERR_NULL, "logprob: logp and lse are required");
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const tpc::Plan& p = plan->p;
-  float* Z = static_cast<float*>(scratch);
-  const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(h);
-  for (int64_t r0 = 0; r0 < p.n_unique; r0 += chunk_rows) {
-    const int R = (int)std::min<int64_t>(chunk_rows, p.n_unique - r0);
-    if (int rc = tpc_gemm_bf16(hb + r0 * Dh, W, Z, R, V, Dh, Dh, Dh, V, 0, 0, TPC_F32, 1.f, 0.f, status, stream)) return rc;
-    TPC_LAUNCH("lse_rows", st, (tpc::lse_rows_kernel<<<R, tpc::kLseThreads, 0, st>>>(Z, V, lse, (int)r0)));
-    TPC_LAUNCH("logprob_gather", st,
-               (tpc::logprob_gather_kernel<<<(R + 127) / 128, 128, 0, st>>>(p.dt, Z, V, (int)r0, R, lse, targets, logp,
-                                                                             status)));
-  }
-  return TPC_OK;
-}
-
-int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh,
-                         const int32_t* targets, const float* dlogp, const float* lse, float* dh, float* dW,
-                         void* scratch, size_t scratch_bytes, int32_t chunk_rows, int32_t* status,
-                         tpc_stream_t stream) {
-  if (int rc = logprob_check(plan, h, W, V, Dh, targets, scratch, scratch_bytes, chunk_rows)) return rc;
-  if (!dlogp || !lse || !dh || !dW) return fail(TPC_ERR_NULL, "logprob backward: dlogp, lse, dh and dW are required");
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const tpc::Plan& p = plan->p;
-  char* sc = static_cast<char*>(scratch);
-  float* Z = reinterpret_cast<float*>(sc);
-  __nv_bfloat16* zh = reinterpret_cast<__nv_bfloat16*>(sc + a256((size_t)chunk_rows * V * 4));
-  __nv_bfloat16* zl = reinterpret_cast<__nv_bfloat16*>(sc + a256((size_t)chunk_rows * V * 4) + a256((size_t)chunk_rows * V * 2));
-  const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(h);
-  TPC_CUDA(cudaMemsetAsync(dW, 0, (size_t)V * Dh * 4, st));
-  for (int64_t r0 = 0; r0 < p.n_unique; r0 += chunk_rows) {
-    const int R = (int)std::min<int64_t>(chunk_rows, p.n_unique - r0);
-    if (int rc = tpc_gemm_bf16(hb + r0 * Dh, W, Z, R, V, Dh, Dh, Dh, V, 0, 0, TPC_F32, 1.f, 0.f, status, stream)) return rc;
-    TPC_LAUNCH("dz_rows", st,
-               (tpc::dz_rows_kernel<<<R, tpc::kLseThreads, 0, st>>>(p.dt, Z, V, (int)r0, lse, targets, dlogp, zh, zl,
-                                                                    status)));
-    // dH = dZ W  (W as an MN-major B: [V][Dh], N = Dh contiguous)
-    float* dhc = dh + r0 * Dh;
-    if (int rc = tpc_gemm_bf16(zh, W, dhc, R, Dh, V, V, Dh, Dh, 0, 1, TPC_F32, 1.f, 0.f, status, stream)) return rc;
-    if (int rc = tpc_gemm_bf16(zl, W, dhc, R, Dh, V, V, Dh, Dh, 0, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
-    // dW += dZ^T H  (dZ as an MN-major A: [R][V]; H as an MN-major B: [R][Dh])
-    if (int rc = tpc_gemm_bf16(zh, hb + r0 * Dh, dW, V, Dh, R, V, Dh, Dh, 1, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
-    if (int rc = tpc_gemm_bf16(zl, hb + r0 * Dh, dW, V, Dh, R, V, Dh, Dh, 1, 1, TPC_F32, 1.f, 1.f, status, stream)) return rc;
-  }
-  return TPC_OK;
-}
-
-namespace {
-int attn_check(const tpc_plan* plan, const tpc_attn_shape* s) {
-  if (!plan || !s) return fail(TPC_ERR_NULL, "attention: plan or shape is NULL");
-  if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
-  if (s->d_qk != tpc::kAttnQK || s->d_v != tpc::kAttnDV || s->H < 1)
-    return fail(TPC_ERR_UNSUPPORTED, "attention: built for d_qk = 192, d_v = 128");
-  if (s->io_dtype != TPC_F32 && s->io_dtype != TPC_BF16) return fail(TPC_ERR_UNSUPPORTED, "attention: io dtype");
-  return TPC_OK;
-}
-}  // namespace
-
-int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const void* q, const void* k, const void* v,
-                          const tpc_attn_lo* lo, void* o, float* lse, int32_t* status, tpc_stream_t stream) {
-  if (int rc = attn_check(plan, s)) return rc;
-  if (!q || !k || !v || !o || !lse) return fail(TPC_ERR_NULL, "attention forward: NULL tensor");
-  const tpc_attn_lo L = lo ? *lo : tpc_attn_lo{};
-  const bool split = L.q || L.k || L.v;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const tpc::Plan& p = plan->p;
-  const dim3 grid((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest
-  using bf = __nv_bfloat16;
-  const uint64_t NR = (uint64_t)p.n_unique;
-  CUtensorMap tk, tkl, tv, tvl;
-  bool ok = tensor_map_rows(&tk, k, tpc::kAttnQK, s->H, NR, 64) && tensor_map_rows(&tv, v, tpc::kAttnDV, s->H, NR, 64);
-  ok = ok && tensor_map_rows(&tkl, L.k ? L.k : k, tpc::kAttnQK, s->H, NR, 64) &&
-       tensor_map_rows(&tvl, L.v ? L.v : v, tpc::kAttnDV, s->H, NR, 64);
-  if (!ok) return fail(TPC_ERR_CUDA, "attention forward: cuTensorMapEncodeTiled failed");
-  auto go = [&](auto tout, auto split) -> int {
-    using T = decltype(tout);
-    constexpr bool SP = decltype(split)::value;
-    constexpr size_t smem = tpc::AttnFwdSmem<SP>::total;
-    TPC_CUDA(set_smem(tpc::attn_fwd_tc<T, SP>, smem));
-    TPC_LAUNCH("attn_fwd_tc", st,
-               (tpc::attn_fwd_tc<T, SP><<<grid, tpc::kAttnFwdThreads, smem, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, tk, tkl, tv, tvl, (T*)o, lse, status)));
-    return TPC_OK;
-  };
-  using Y = std::true_type;
-  using N = std::false_type;
-  if (s->io_dtype == TPC_BF16) return split ? go(bf{}, Y{}) : go(bf{}, N{});
-  return split ? go(float{}, Y{}) : go(float{}, N{});
-}
-
-int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const void* q, const void* k,
-                           const void* v, const tpc_attn_lo* lo, const void* o, const float* lse, const void* d_o,
-                           void* dq, void* dk, void* dv, float* delta, int32_t* status, tpc_stream_t stream) {
-  if (int rc = attn_check(plan, s)) return rc;
-  if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv || !delta)
-    return fail(TPC_ERR_NULL, "attention backward: NULL tensor");
-  const tpc_attn_lo L = lo ? *lo : tpc_attn_lo{};
-  const bool split = L.q || L.k || L.v || L.d_o;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const tpc::Plan& p = plan->p;
-  using bf = __nv_bfloat16;
-  const dim3 gq((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest
-  const dim3 gk((unsigned)(p.attn_ktiles.size() * (size_t)s->H));  // (key tile, head), key tiles fastest
-  const uint64_t NR = (uint64_t)p.n_unique;
-  const unsigned Hh = (unsigned)s->H;
-  CUtensorMap tk, tkl, tv, tvl, to, tol, tq32, tql32, to32, tol32;
-  bool ok = tensor_map_rows(&tk, k, tpc::kAttnQK, Hh, NR, 64) && tensor_map_rows(&tv, v, tpc::kAttnDV, Hh, NR, 64) &&
-            tensor_map_rows(&tkl, L.k ? L.k : k, tpc::kAttnQK, Hh, NR, 64) &&
-            tensor_map_rows(&tvl, L.v ? L.v : v, tpc::kAttnDV, Hh, NR, 64) &&
-            tensor_map_rows(&to, d_o, tpc::kAttnDV, Hh, NR, 128) &&
-            tensor_map_rows(&tol, L.d_o ? L.d_o : d_o, tpc::kAttnDV, Hh, NR, 128);
-  constexpr uint32_t QT = tpc::AttnDkvSmem<true>::QT;
-  ok = ok && tensor_map_rows(&tq32, q, tpc::kAttnQK, Hh, NR, QT) &&
-       tensor_map_rows(&tql32, L.q ? L.q : q, tpc::kAttnQK, Hh, NR, QT) &&
-       tensor_map_rows(&to32, d_o, tpc::kAttnDV, Hh, NR, QT) &&
-       tensor_map_rows(&tol32, L.d_o ? L.d_o : d_o, tpc::kAttnDV, Hh, NR, QT);
-  CUtensorMap tk128, tkl128;  // key tiles of the dK / dV kernel
-  constexpr uint32_t KT = tpc::AttnDkvSmem<true>::KT;
-  ok = ok && tensor_map_rows(&tk128, k, tpc::kAttnQK, Hh, NR, KT) &&
-       tensor_map_rows(&tkl128, L.k ? L.k : k, tpc::kAttnQK, Hh, NR, KT);
-  if (!ok) return fail(TPC_ERR_CUDA, "attention backward: cuTensorMapEncodeTiled failed");
-  auto go = [&](auto tio, auto split) -> int {
-    using T = decltype(tio);
-    constexpr bool SP = decltype(split)::value;
-    constexpr size_t sq = tpc::AttnDqSmem<SP>::total, sk = tpc::AttnDkvSmem<SP>::total;
-    TPC_CUDA(set_smem(tpc::attn_bwd_dq_tc<T, SP>, sq));
-    TPC_CUDA(set_smem(tpc::attn_bwd_dkv_tc<T, SP>, sk));
-    TPC_LAUNCH("attn_bwd_dq_tc", st,
-               (tpc::attn_bwd_dq_tc<T, SP><<<gq, tpc::kAttnDqThreads, sq, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)q, (const bf*)L.q, tk, tkl, tv, tvl, to, tol, (const T*)o, lse,
-                   (const bf*)d_o, (const bf*)L.d_o, (T*)dq, delta, status)));
-    TPC_LAUNCH("attn_bwd_dkv_tc", st,
-               (tpc::attn_bwd_dkv_tc<T, SP><<<gk, tpc::kAttnDkvThreads, sk, st>>>(
-                   p.dt, s->H, s->scale, (const bf*)v, (const bf*)L.v, tq32, tql32, tk128, tkl128, to32, tol32, lse,
-                   delta, (T*)dk, (T*)dv, status)));
-    return TPC_OK;
-  };
-  using Y = std::true_type;
-  using N = std::false_type;
-  if (s->io_dtype == TPC_BF16) return split ? go(bf{}, Y{}) : go(bf{}, N{});
-  return split ? go(float{}, Y{}) : go(float{}, N{});
 }
 
 int tpc_rope_positions(const tpc_plan* plan, int32_t* pos, tpc_stream_t stream) {
