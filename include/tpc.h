@@ -85,6 +85,26 @@ int tpc_plan_create(const int32_t* parent, const int32_t* length, int32_t n_node
                     int32_t chunk, tpc_plan** out);
 void tpc_plan_destroy(tpc_plan* plan);
 
+/*
+ * Planner modes.  TPC_PLAN_MIN_ROUNDS is tpc_plan_create's plan.  The other two are the ablations
+ * the HARTS pages compare against (Figure 4: node-wise linear attention; Figure 5: no replay):
+ *   TPC_PLAN_NODEWISE  every segment is a sequence of its own (no direct continuations); each starts
+ *                      at its aligned boundary b_v with the same bounded replay, one round after the
+ *                      segment holding token b_v - 1, so the call count is the depth of that chain
+ *                      and every trajectory keeps its chunkwise numerical path.
+ *   TPC_PLAN_NO_REPLAY side sequences start exactly at their fork point s_v from the state after
+ *                      token s_v - 1 (no replay): the producing sequence cuts a chunk at s_v to
+ *                      export that state, the side sequence's chunk grid starts at s_v.  Chunk
+ *                      boundaries then differ from the trajectory-expanded grid, so results differ
+ *                      from the per-trajectory chunkwise path in the last bits.
+ * Every other call accepts a plan of any mode.
+ */
+enum tpc_plan_mode { TPC_PLAN_MIN_ROUNDS = 0, TPC_PLAN_NODEWISE = 1, TPC_PLAN_NO_REPLAY = 2 };
+/* tpc_plan_create with a planner mode (above).  Errors as tpc_plan_create; an unknown mode is
+ * TPC_ERR_UNSUPPORTED. */
+int tpc_plan_create_mode(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, int32_t mode,
+                         tpc_plan** out);
+
 typedef struct tpc_plan_info {
   int64_t n_unique;     /* unique token rows N */
   int64_t n_expanded;   /* sum of trajectory lengths */

@@ -27,6 +27,14 @@ itself holds token b_c - 1, else e.  H(v, e) = extra rounds below v:
 0 for a leaf, else min over the continued child c* of
 max(H(c*, delta_c*(e)), max_{c != c*} delta_c(e) + H(c, 0)).
 Ties: smaller H, then larger replay saved (s_c - b_c), then smaller id.
+
+Ablation modes (HARTS Figure 4 compares node-wise linear attention, Figure 5 a variant without
+replay; the pages describe neither further, so these are the plainest readings):
+  * "nodewise": no node continues its parent; each node starts its own sequence at b_v from its
+    anchor's boundary state (same bounded replay), one round after the anchor (round 1 if b_v = 0);
+  * "noreplay": a side node starts exactly at s_v from the state after token s_v - 1 (its parent
+    holds it), so b_v = s_v and a(v) = parent(v); the same dynamic program picks the continuations.
+    Its producer must cut a chunk at s_v to export that state (chunk_count models the cuts).
 """
 from __future__ import annotations
 
@@ -114,14 +122,23 @@ def _children(parent):
     return ch
 
 
-def plan(parent, length, C) -> Plan:
+MODES = ("min_rounds", "nodewise", "noreplay")
+
+
+def plan(parent, length, C, mode="min_rounds") -> Plan:
     parent = np.asarray(parent, np.int64)
     length = np.asarray(length, np.int64)
     validate(parent, length)
+    if mode not in MODES:
+        raise ValueError(f"unknown mode {mode}")
     n = len(parent)
     ch = _children(parent)
     s = positions(parent, length)
-    b, a = anchors(parent, length, s, C)
+    if mode == "noreplay":
+        b = s.copy()                          # handoff exactly at the fork point
+        a = np.where(parent >= 0, parent, -1)  # the parent holds token s_v - 1
+    else:
+        b, a = anchors(parent, length, s, C)
 
     def delta(v, c, e):
         return 1 if s[v] < b[c] else e
@@ -130,7 +147,7 @@ def plan(parent, length, C) -> Plan:
     H = np.zeros((n, 2), np.int64)
     choice = np.full((n, 2), -1, np.int64)
     for v in range(n - 1, -1, -1):
-        if not ch[v]:
+        if not ch[v] or mode == "nodewise":
             continue
         for e in (0, 1):
             best = None
@@ -153,6 +170,10 @@ def plan(parent, length, C) -> Plan:
     for v in range(n):
         if parent[v] < 0:
             rnd[v], ee[v] = 1, 0
+        if mode == "nodewise":
+            if parent[v] >= 0:
+                rnd[v] = 1 if b[v] == 0 else rnd[a[v]] + 1
+            continue
         if ch[v]:
             cs = choice[v, ee[v]]
             cont_child[v] = cs
@@ -165,8 +186,9 @@ def plan(parent, length, C) -> Plan:
                     rnd[c] = rnd[v] + delta(v, c, ee[v])
                     ee[c] = 0
     roots = [v for v in range(n) if parent[v] < 0]
-    n_rounds = int(1 + max(H[r, 0] for r in roots))
-    assert n_rounds == int(rnd.max())
+    n_rounds = int(rnd.max())
+    if mode != "nodewise":
+        assert n_rounds == int(1 + max(H[r, 0] for r in roots))
 
     # compact layout: DFS preorder, continuation child first, then others by id; roots by id
     row_offset = np.zeros(n, np.int64)
@@ -237,6 +259,33 @@ def plan(parent, length, C) -> Plan:
                 cont_child=cont_child, replay_start=replay_start, replay_len=replay_len,
                 row_offset=row_offset, occurrence=occ, n_rounds=n_rounds, seqs=seqs, slots=slots,
                 leaves=leaves)
+
+
+def chunk_count(pl: Plan) -> int:
+    """Chunks of the packed calls: each sequence is cut at multiples of C from its start and, in
+    addition, wherever it exports a boundary state (only off the grid in no-replay plans)."""
+    total = 0
+    for si, sq in enumerate(pl.seqs):
+        cuts = {sl["b"] for sl in pl.slots if sl["producer_seq"] == si}
+        p0, start, end = sq["start"], sq["start"], sq["end"]
+        while p0 < end:
+            p1 = min(start + ((p0 - start) // pl.C + 1) * pl.C, end)
+            later = [c for c in cuts if c > p0]
+            if later:
+                p1 = min(p1, min(later))
+            total += 1
+            p0 = p1
+    return total
+
+
+def handoff_depth(parent) -> np.ndarray:
+    """Per node, the boundary-state handoffs on the way from the root to its first token: the
+    segment boundaries on its path (its depth in the tree; the root is 0)."""
+    parent = np.asarray(parent, np.int64)
+    dep = np.zeros(len(parent), np.int64)
+    for v in range(len(parent)):
+        dep[v] = 0 if parent[v] < 0 else dep[parent[v]] + 1
+    return dep
 
 
 # ------------------------------------------------------------------ brute force

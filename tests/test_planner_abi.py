@@ -39,9 +39,12 @@ def test_every_declared_symbol_is_exported(tpc):
     assert names <= set(tpc.SIGNATURES), names - set(tpc.SIGNATURES)
 
 
-def compare(tpc, parent, length, C):
-    ref = P.plan(parent, length, C)
-    pl = tpc.Plan(parent, length, C)
+MODE_CODE = {"min_rounds": 0, "nodewise": 1, "noreplay": 2}
+
+
+def compare(tpc, parent, length, C, mode="min_rounds"):
+    ref = P.plan(parent, length, C, mode)
+    pl = tpc.Plan(parent, length, C, MODE_CODE[mode])
     tb = pl.tables()
     assert pl.info["n_rounds"] == ref.n_rounds
     assert np.array_equal(tb["round"], ref.round)
@@ -58,6 +61,7 @@ def compare(tpc, parent, length, C):
     assert pl.info["replay_total"] == ref.replay_total
     assert pl.info["n_slots"] == len(ref.slots)
     assert pl.info["n_seqs"] == len(ref.seqs)
+    assert pl.info["n_chunks"] == P.chunk_count(ref)
     return pl
 
 
@@ -75,6 +79,49 @@ def test_planner_bit_exact_random(tpc, C):
         parent = [-1] + [(-1 if rng.random() < 0.05 else int(rng.integers(0, i))) for i in range(1, n)]
         length = rng.integers(1, 4 * C, size=n)
         compare(tpc, parent, length, C)
+
+
+@pytest.mark.parametrize("mode", ["nodewise", "noreplay"])
+@pytest.mark.parametrize("cfg", ["fig1", "single_fork", "agentic", "agentic_small", "wide"])
+def test_ablation_planners_bit_exact_on_workloads(tpc, cfg, mode):
+    w = synth.workload(cfg)
+    compare(tpc, w.tree.parent, w.tree.length, w.chunk, mode)
+
+
+@pytest.mark.parametrize("mode", ["nodewise", "noreplay"])
+@pytest.mark.parametrize("C", [16, 64])
+def test_ablation_planners_bit_exact_random(tpc, C, mode):
+    rng = np.random.default_rng(100 + C + MODE_CODE[mode])
+    for _ in range(300):
+        n = int(rng.integers(1, 40))
+        parent = [-1] + [(-1 if rng.random() < 0.05 else int(rng.integers(0, i))) for i in range(1, n)]
+        length = rng.integers(1, 4 * C, size=n)
+        compare(tpc, parent, length, C, mode)
+
+
+def test_ablation_planners_on_fig1(tpc):
+    """Fig. 1 tree (A 40 -> B 24, C 17; B -> D 9, E 31), chunk 16, worked by hand from the two
+    ablation rules.  Node-wise: A in call 1; B, C start at 32 from A's state (8 replayed rows each)
+    in call 2; D, E start at 64 from B's state in call 3; chunks 3 + 2 + 2 + 1 + 2 = 10.
+    No replay: the minimum-call structure of the main plan (call 1 = A, B, D; call 2 = C, E) with
+    C starting at 40 and no replayed row, so A-B-D is cut at 40 to export that state: chunks
+    [0,16) [16,32) [32,40) [40,48) [48,64) [64,73), C [40,56) [56,57), E [64,80) [80,95) = 10."""
+    w = synth.workload("fig1")
+    t = w.tree
+    nw = tpc.Plan(t.parent, t.length, 16, tpc.PLAN_NODEWISE)
+    tb = nw.tables()
+    assert nw.info["n_rounds"] == 3 and list(tb["round"]) == [1, 2, 2, 3, 3]
+    assert list(tb["is_cont"]) == [0, 0, 0, 0, 0] and list(tb["replay_len"]) == [0, 8, 8, 0, 0]
+    assert nw.info["n_chunks"] == 10 and nw.info["replay_total"] == 16 and nw.info["n_seqs"] == 5
+    nr = tpc.Plan(t.parent, t.length, 16, tpc.PLAN_NO_REPLAY)
+    tb = nr.tables()
+    assert nr.info["n_rounds"] == 2 and list(tb["round"]) == [1, 1, 2, 1, 2]
+    assert list(tb["replay_len"]) == [0, -1, 0, -1, 0] and list(tb["replay_start"]) == [0, -1, 40, -1, 64]
+    assert list(tb["anchor"]) == [-1, 0, 0, 1, 1]
+    assert nr.info["n_chunks"] == 10 and nr.info["replay_total"] == 0
+    with pytest.raises(tpc.TpcError) as e:
+        tpc.Plan(t.parent, t.length, 16, 7)
+    assert e.value.code == 3
 
 
 def test_fig1_chunk_table(tpc):

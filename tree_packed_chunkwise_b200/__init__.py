@@ -94,6 +94,7 @@ SIGNATURES = {
     "tpc_version": (ctypes.c_char_p, []),
     "tpc_plan_create": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int32, _P(_V)]),
     "tpc_plan_destroy": (None, [_V]),
+    "tpc_plan_create_mode": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P(_V)]),
     "tpc_plan_get_info": (ctypes.c_int, [_V, _P(PlanInfo)]),
     "tpc_plan_export": (ctypes.c_int, [_V, _P(PlanTables)]),
     "tpc_plan_device_bytes": (ctypes.c_size_t, [_V]),
@@ -166,15 +167,20 @@ def _stream_ptr(stream):
 
 
 # ------------------------------------------------------------------------------------ plan
-class Plan:
-    """Round plan of a rollout tree (host object; ``upload`` places its tables on the device)."""
+PLAN_MIN_ROUNDS, PLAN_NODEWISE, PLAN_NO_REPLAY = 0, 1, 2
 
-    def __init__(self, parent, length, chunk: int):
+
+class Plan:
+    """Round plan of a rollout tree (host object; ``upload`` places its tables on the device).
+    mode: PLAN_MIN_ROUNDS (default), or the ablations PLAN_NODEWISE / PLAN_NO_REPLAY."""
+
+    def __init__(self, parent, length, chunk: int, mode: int = PLAN_MIN_ROUNDS):
         parent = np.ascontiguousarray(parent, np.int32)
         length = np.ascontiguousarray(length, np.int32)
         h = ctypes.c_void_p()
-        _check(lib().tpc_plan_create(parent.ctypes.data_as(i32p), length.ctypes.data_as(i32p),
-                                     int(parent.shape[0]), int(chunk), ctypes.byref(h)))
+        _check(lib().tpc_plan_create_mode(parent.ctypes.data_as(i32p), length.ctypes.data_as(i32p),
+                                          int(parent.shape[0]), int(chunk), int(mode), ctypes.byref(h)))
+        self.mode = int(mode)
         self._h = h
         self.n_nodes = int(parent.shape[0])
         info = PlanInfo()

@@ -76,8 +76,11 @@ struct DevTables {
   const AttnTile* attn_ktiles;
 };
 
+// planner modes (tpc_plan_create_mode)
+enum : int { kPlanMinRounds = 0, kPlanNodewise = 1, kPlanNoReplay = 2 };
+
 struct Plan {
-  int32_t C = 0, n = 0;
+  int32_t C = 0, n = 0, mode = 0;
   std::vector<int32_t> parent, length;
   std::vector<int64_t> s, b;
   std::vector<int32_t> anchor, round, is_cont, cont_child, replay_start, replay_len, occurrence;
@@ -107,7 +110,8 @@ struct Plan {
 };
 
 // Builds the plan; returns an empty string or an error message.
-std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, int32_t C, Plan& out);
+std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, int32_t C, Plan& out,
+                       int mode = kPlanMinRounds);
 // Packs the device blob; returns the layout (offsets per table) and the total bytes.
 size_t device_layout(const Plan& p, std::vector<size_t>& offsets);
 void pack_device_blob(const Plan& p, const std::vector<size_t>& offsets, std::vector<uint8_t>& blob);

@@ -14,7 +14,17 @@
 //   delta_c(e) = 1 if the parent v holds token b_c - 1 (s_v < b_c), else e
 //   H(v, e)    = min_{c*} max(H(c*, delta_c*(e)), max_{c != c*} delta_c(e) + H(c, 0))
 // Ties: smaller H, then larger replay saved (s_c - b_c), then smaller id.
+//
+// Two ablation modes reuse everything else (HARTS Figure 4 "Node-wise LA", Figure 5 "No-replay"):
+//   node-wise: no node continues its parent; every node is a sequence of its own that starts at
+//     b_v from its anchor's boundary state (with the same bounded replay), one round after the
+//     anchor's round, so the rounds equal the anchor depth;
+//   no replay: a side sequence starts exactly at its fork point s_v from the state after token
+//     s_v - 1 (held by the parent), so b_v = s_v and nothing is replayed; the producing sequence
+//     cuts a chunk at s_v to export that state mid-grid, and the side sequence's own chunk grid
+//     starts at s_v.  The same dynamic program then yields the fewest rounds under that rule.
 #include <algorithm>
+#include <climits>
 #include <cstring>
 #include <map>
 #include <tuple>
@@ -23,11 +33,13 @@
 
 namespace tpc {
 
-std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, int32_t C, Plan& P) {
+std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, int32_t C, Plan& P, int mode) {
   if (n <= 0) return "tree has no nodes";
   if (C != 16 && C != 32 && C != 64) return "chunk size must be 16, 32 or 64";
+  if (mode != kPlanMinRounds && mode != kPlanNodewise && mode != kPlanNoReplay) return "unknown plan mode";
   P = Plan();
   P.C = C;
+  P.mode = mode;
   P.n = n;
   P.parent.assign(parent, parent + n);
   P.length.assign(length, length + n);
@@ -59,7 +71,7 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
   for (int32_t v = 0; v < n; ++v) {
     int32_t p = parent[v];
     P.s[v] = p < 0 ? 0 : P.s[p] + length[p];
-    P.b[v] = (P.s[v] / C) * C;
+    P.b[v] = mode == kPlanNoReplay ? P.s[v] : (P.s[v] / C) * C;
     if (P.b[v] > 0) {
       int32_t u = p;
       while (P.s[u] > P.b[v] - 1) u = parent[u];
@@ -70,11 +82,11 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
   for (int32_t v = 0; v < n; ++v)
     if (P.s[v] + length[v] >= (int64_t(1) << 31)) return "trajectory longer than 2^31 tokens";
 
-  // bottom-up DP
+  // bottom-up DP (node-wise plans continue nothing: choice stays -1)
   std::vector<int64_t> H(2 * n, 0);
   std::vector<int32_t> choice(2 * n, -1);
   for (int32_t v = n - 1; v >= 0; --v) {
-    if (nch[v] == 0) continue;
+    if (nch[v] == 0 || mode == kPlanNodewise) continue;
     for (int e = 0; e < 2; ++e) {
       // top-2 of the independent cost y_c = delta_c(e) + H(c, 0)
       int64_t m1 = -1, m2 = -1;
@@ -111,6 +123,10 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
   std::vector<int32_t> ee(n, 0);
   for (int32_t v = 0; v < n; ++v) {
     if (parent[v] < 0) { P.round[v] = 1; ee[v] = 0; P.roots.push_back(v); }
+    if (mode == kPlanNodewise) {  // one sequence per node, one round after its anchor's
+      if (parent[v] >= 0) P.round[v] = P.b[v] == 0 ? 1 : P.round[P.anchor[v]] + 1;
+      continue;
+    }
     if (nch[v] == 0) continue;
     int32_t cs = choice[2 * v + ee[v]];
     P.cont_child[v] = cs;
@@ -238,24 +254,35 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
       while (P.s[u] > pos) u = parent[u];
       P.replay_rows.push_back((int32_t)(P.row_offset[u] + (pos - P.s[u])));
     }
+    // chunk boundaries: the sequence's grid (multiples of C from its start) and every position at
+    // which it exports a boundary state (grid points, except in no-replay plans)
+    std::vector<int64_t> cuts;
+    for (auto it = slot_at.lower_bound({(int32_t)si, INT64_MIN}); it != slot_at.end() && it->first.first == (int32_t)si;
+         ++it)
+      cuts.push_back(it->first.second);
+    size_t next_cut = 0;
     int32_t idx = 0;
-    for (int64_t p0 = r.start_pos; p0 < end; p0 += C, ++idx) {
+    for (int64_t p0 = r.start_pos; p0 < end; ++idx) {
+      while (next_cut < cuts.size() && cuts[next_cut] <= p0) ++next_cut;
+      int64_t p1 = std::min<int64_t>(r.start_pos + ((p0 - r.start_pos) / C + 1) * C, end);
+      if (next_cut < cuts.size()) p1 = std::min<int64_t>(p1, cuts[next_cut]);
       ChunkRec c{};
       c.seq = (int32_t)si;
       c.pos0 = (int32_t)p0;
-      c.n_rows = (int32_t)std::min<int64_t>(C, end - p0);
-      c.n_replay = (int32_t)std::max<int64_t>(0, std::min<int64_t>(s_h, p0 + c.n_rows) - p0);
+      c.n_rows = (int32_t)(p1 - p0);
+      c.n_replay = (int32_t)std::max<int64_t>(0, std::min<int64_t>(s_h, p1) - p0);
       int64_t first_own = std::max<int64_t>(p0, s_h);
       c.row_start = (int32_t)(P.row_offset[h] + (first_own - s_h));
-      c.replay_base = replay_base;
-      auto it = slot_at.find({(int32_t)si, p0 + c.n_rows});
+      c.replay_base = replay_base;  // replayed rows (< C of them) all fall in the first chunk
+      auto it = slot_at.find({(int32_t)si, p1});
       c.export_slot = -1;
-      if (it != slot_at.end() && c.n_rows == C) {
+      if (it != slot_at.end()) {
         c.export_slot = it->second;
         P.slots[it->second].export_chunk = (int32_t)P.chunks.size();
       }
       c.idx_in_seq = idx;
       P.chunks.push_back(c);
+      p0 = p1;
     }
     r.n_chunks = idx;
     P.max_seq_chunks = std::max(P.max_seq_chunks, idx);

@@ -494,24 +494,29 @@ extern "C" {
 const char* tpc_last_error(void) { return tpc_abi::g_err.c_str(); }
 const char* tpc_version(void) { return "tpc 0.1 (sm_100a)"; }
 
-int tpc_plan_create(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, tpc_plan** out) {
+int tpc_plan_create_mode(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, int32_t mode,
+                         tpc_plan** out) {
   if (!parent || !length || !out) return fail(TPC_ERR_NULL, "parent, length and out must be non-NULL");
   *out = nullptr;
   tpc_plan* p = new (std::nothrow) tpc_plan();
   if (!p) return fail(TPC_ERR_CUDA, "out of host memory");
   std::string err;
   try {
-    err = tpc::build_plan(parent, length, n_nodes, chunk, p->p);
+    err = tpc::build_plan(parent, length, n_nodes, chunk, p->p, mode);
   } catch (const std::exception& e) {
     err = std::string("planner: ") + e.what();
   }
   if (!err.empty()) {
     delete p;
-    const bool unsup = err.find("chunk size") != std::string::npos;
+    const bool unsup = err.find("chunk size") != std::string::npos || err.find("plan mode") != std::string::npos;
     return fail(unsup ? TPC_ERR_UNSUPPORTED : TPC_ERR_INVALID_TREE, err);
   }
   *out = p;
   return TPC_OK;
+}
+
+int tpc_plan_create(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, tpc_plan** out) {
+  return tpc_plan_create_mode(parent, length, n_nodes, chunk, TPC_PLAN_MIN_ROUNDS, out);
 }
 
 void tpc_plan_destroy(tpc_plan* plan) { delete plan; }
