@@ -155,6 +155,34 @@ int tpc_plan_export(const tpc_plan* plan, tpc_plan_tables* tables);
 size_t tpc_plan_device_bytes(const tpc_plan* plan);
 int tpc_plan_upload(tpc_plan* plan, void* dev, size_t bytes, tpc_stream_t stream);
 
+/* ------------------------------------------------------------------ microbatches (L1) */
+/*
+ * First-level (L1) microbatch planner: compression-oriented packing of the trajectories of many
+ * rollout trees under a budget of unique token rows per microbatch (HARTS abstract: a two-level
+ * planner first constructs compression-oriented microbatches; Figure 1(c); Table 4).  The pages
+ * give no algorithm; this one keeps a tree whole when its unique tokens fit the budget, cuts a
+ * larger tree along its depth-first leaf order (so that trajectories sharing the longest prefixes
+ * stay together; a piece closes before the leaf whose new path tokens would exceed the budget, and
+ * a trajectory longer than the budget is a piece alone), and places pieces first-fit in decreasing
+ * cost order (ties: smaller first leaf id).  Host only, deterministic.
+ *   parent, length: the forest of all trees of the step (conventions above), n nodes.
+ *   budget: unique token rows per microbatch (>= 1).
+ *   leaf_mb: host [n_leaves] (leaves in id order) receives each trajectory's microbatch.
+ *   mb_unique, mb_expanded: host [max_mb] or NULL: per microbatch the tokens of the union of its
+ *   trajectories' paths, and the sum of their lengths.
+ *   stats: totals, compression = expanded / unique, balance = mean unique / max unique.
+ * Errors: TPC_ERR_NULL, TPC_ERR_INVALID_TREE, TPC_ERR_BAD_SHAPE (budget < 1, or more microbatches
+ * than max_mb while mb_unique or mb_expanded is given; stats->n_microbatches then holds the count).
+ */
+typedef struct tpc_microbatch_stats {
+  int32_t n_microbatches;
+  int64_t unique_tokens, expanded_tokens, max_unique;
+  double compression, balance;
+} tpc_microbatch_stats;
+int tpc_microbatch_plan(const int32_t* parent, const int32_t* length, int32_t n_nodes, int64_t budget,
+                        int32_t* leaf_mb, int64_t* mb_unique, int64_t* mb_expanded, int32_t max_mb,
+                        tpc_microbatch_stats* stats);
+
 /* ------------------------------------------------------------------ KDA */
 typedef struct tpc_kda_shape {
   int32_t H;          /* heads */

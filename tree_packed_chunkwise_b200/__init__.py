@@ -44,6 +44,12 @@ class PlanTables(ctypes.Structure):
                 ("expanded_rows", i64p), ("traj_offset", i64p)]
 
 
+class MicrobatchStats(ctypes.Structure):
+    _fields_ = [("n_microbatches", ctypes.c_int32), ("unique_tokens", ctypes.c_int64),
+                ("expanded_tokens", ctypes.c_int64), ("max_unique", ctypes.c_int64),
+                ("compression", ctypes.c_double), ("balance", ctypes.c_double)]
+
+
 class KdaShape(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
                 ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
@@ -94,6 +100,8 @@ SIGNATURES = {
     "tpc_version": (ctypes.c_char_p, []),
     "tpc_plan_create": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int32, _P(_V)]),
     "tpc_plan_destroy": (None, [_V]),
+    "tpc_microbatch_plan": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int64, i32p, i64p, i64p,
+                                           ctypes.c_int32, _P(MicrobatchStats)]),
     "tpc_plan_create_mode": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P(_V)]),
     "tpc_plan_get_info": (ctypes.c_int, [_V, _P(PlanInfo)]),
     "tpc_plan_export": (ctypes.c_int, [_V, _P(PlanTables)]),
@@ -228,6 +236,48 @@ class Plan:
     def to_compact(self, node_rows_array: np.ndarray, node_start: np.ndarray, length: np.ndarray) -> np.ndarray:
         """Reorders a node-order row array to the compact layout."""
         return node_rows_array[self.compact_source_rows(node_start, length)]
+
+
+# ------------------------------------------------------------------------------------ microbatches
+def tpc_microbatch_plan(parent, length, budget: int):
+    """L1 microbatches of a forest: (leaf_mb [n_leaves] int32 in leaf-id order, mb_unique, mb_expanded,
+    stats dict).  Host only."""
+    parent = np.ascontiguousarray(parent, np.int32)
+    length = np.ascontiguousarray(length, np.int32)
+    n = int(parent.shape[0])
+    has_child = np.zeros(n, bool)
+    has_child[parent[parent >= 0]] = True
+    n_leaves = int((~has_child).sum())
+    leaf_mb = np.zeros(max(n_leaves, 1), np.int32)
+    mu = np.zeros(max(n_leaves, 1), np.int64)
+    me = np.zeros(max(n_leaves, 1), np.int64)
+    st = MicrobatchStats()
+    _check(lib().tpc_microbatch_plan(parent.ctypes.data_as(i32p), length.ctypes.data_as(i32p), n, int(budget),
+                                     leaf_mb.ctypes.data_as(i32p), mu.ctypes.data_as(i64p), me.ctypes.data_as(i64p),
+                                     len(mu), ctypes.byref(st)))
+    m = st.n_microbatches
+    return leaf_mb[:n_leaves], mu[:m], me[:m], {f: getattr(st, f) for f, _ in MicrobatchStats._fields_}
+
+
+def microbatch_forest(parent, length, leaf_mb, m):
+    """(parent, length, node ids) of the sub-forest holding microbatch m's trajectories (the nodes on
+    their paths, renumbered in increasing original id)."""
+    parent = np.asarray(parent, np.int64)
+    n = len(parent)
+    has_child = np.zeros(n, bool)
+    has_child[parent[parent >= 0]] = True
+    leaves = np.nonzero(~has_child)[0]
+    keep = np.zeros(n, bool)
+    for l in leaves[np.asarray(leaf_mb) == m]:
+        v = int(l)
+        while v >= 0 and not keep[v]:
+            keep[v] = True
+            v = int(parent[v])
+    ids = np.nonzero(keep)[0]
+    new = -np.ones(n, np.int64)
+    new[ids] = np.arange(len(ids))
+    sub_parent = np.where(parent[ids] >= 0, new[np.maximum(parent[ids], 0)], -1).astype(np.int32)
+    return sub_parent, np.asarray(length)[ids].astype(np.int32), ids
 
 
 # ------------------------------------------------------------------------------------ KDA
