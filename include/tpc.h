@@ -105,6 +105,22 @@ enum tpc_plan_mode { TPC_PLAN_MIN_ROUNDS = 0, TPC_PLAN_NODEWISE = 1, TPC_PLAN_NO
 int tpc_plan_create_mode(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, int32_t mode,
                          tpc_plan** out);
 
+/*
+ * Plan with external boundary-state exports, for sharing windows across microbatches (HARTS
+ * abstract: within a sharing window, gradients from dependent microbatches accumulate before one
+ * backward pass through the shared prefix; Figure 3: the producer's backward runs after its
+ * consumers').  Export e asks for the state after token export_pos[e] - 1 on the path of node
+ * export_node[e], which must hold that token (s < pos <= s + length) at a position that is a
+ * multiple of the chunk, so that a consumer microbatch can start there and keep its trajectories'
+ * chunkwise numerical path (its replayed rows, pos .. fork - 1, are its own first segment).
+ * The forward writes each export's state into the workspace (tpc_kda_export_states copies it out);
+ * tpc_kda_backward_window adds the consumers' gradients of those states to the reverse scan where
+ * it crosses them, in export order after the in-tree consumers.
+ * Errors: as tpc_plan_create_mode; TPC_ERR_INVALID_TREE for an export that breaks the rule above.
+ */
+int tpc_plan_create_window(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, int32_t mode,
+                           int32_t n_exports, const int32_t* export_node, const int64_t* export_pos, tpc_plan** out);
+
 typedef struct tpc_plan_info {
   int64_t n_unique;     /* unique token rows N */
   int64_t n_expanded;   /* sum of trajectory lengths */
@@ -113,6 +129,7 @@ typedef struct tpc_plan_info {
   int32_t n_nodes, n_rounds, n_seqs, n_chunks, n_slots, n_leaves, n_roots, chunk;
   int32_t max_seq_chunks; /* longest sequence, in chunks */
   int32_t n_replay_targets;
+  int32_t n_exports;      /* external boundary-state exports (tpc_plan_create_window) */
 } tpc_plan_info;
 int tpc_plan_get_info(const tpc_plan* plan, tpc_plan_info* info);
 
@@ -253,6 +270,20 @@ int tpc_kda_backward(const tpc_plan* plan, const tpc_kda_shape* shape, const tpc
                      void* ws, size_t ws_bytes, tpc_stream_t stream);
 
 /*
+ * After tpc_kda_forward on a plan with exports: states [n_exports, H, dk, dv] fp32 receives each
+ * exported boundary state (device to device copies on `stream`).
+ */
+int tpc_kda_export_states(const tpc_plan* plan, const tpc_kda_shape* shape, const void* ws, float* states,
+                          tpc_stream_t stream);
+/*
+ * tpc_kda_backward with the gradients of the exported states (export_grads [n_exports, H, dk, dv]
+ * fp32, e.g. the d_init of the consumer microbatches, summed per export) added to the reverse scan;
+ * NULL means zero.  tpc_kda_backward is this call with NULL.
+ */
+int tpc_kda_backward_window(const tpc_plan* plan, const tpc_kda_shape* shape, const tpc_kda_bwd_io* io,
+                            const float* export_grads, void* ws, size_t ws_bytes, tpc_stream_t stream);
+
+/*
  * Reads (after synchronising `stream`) and clears the status word that
  * kernels write in `ws`.  Returns TPC_OK or the first recorded error.
  */
@@ -273,6 +304,13 @@ int tpc_gather_expanded(const tpc_plan* plan, const void* x_unique, void* x_exp,
                         int32_t elem_bytes, tpc_stream_t stream);
 /* Occurrence count per compact row (int32 [N]). */
 int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t stream);
+/* Row gather dst[i] = src[rows[i]] (rows of `width` elements of elem_bytes 2 or 4; n_rows rows). */
+int tpc_gather_rows(const void* src, const int32_t* rows, void* dst, int64_t n_rows, int64_t width, int32_t elem_bytes,
+                    tpc_stream_t stream);
+/* Row accumulation dst[rows[i]] += src[i] (fp32, `width` per row); the rows of one call must be
+ * distinct (one writer per row), so repeated calls in a fixed order sum deterministically.  Used to
+ * return a consumer microbatch's replayed-row gradients to the producer's rows. */
+int tpc_add_rows(const float* src, const int32_t* rows, float* dst, int64_t n_rows, int64_t width, tpc_stream_t stream);
 
 /* ------------------------------------------------------------------ dense products */
 /*

@@ -35,7 +35,8 @@ class PlanInfo(ctypes.Structure):
                 ("n_seq_tokens", ctypes.c_int64), ("n_nodes", ctypes.c_int32), ("n_rounds", ctypes.c_int32),
                 ("n_seqs", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("n_slots", ctypes.c_int32),
                 ("n_leaves", ctypes.c_int32), ("n_roots", ctypes.c_int32), ("chunk", ctypes.c_int32),
-                ("max_seq_chunks", ctypes.c_int32), ("n_replay_targets", ctypes.c_int32)]
+                ("max_seq_chunks", ctypes.c_int32), ("n_replay_targets", ctypes.c_int32),
+                ("n_exports", ctypes.c_int32)]
 
 
 class PlanTables(ctypes.Structure):
@@ -103,6 +104,12 @@ SIGNATURES = {
     "tpc_microbatch_plan": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int64, i32p, i64p, i64p,
                                            ctypes.c_int32, _P(MicrobatchStats)]),
     "tpc_plan_create_mode": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P(_V)]),
+    "tpc_plan_create_window": (ctypes.c_int, [i32p, i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.c_int32, i32p, i64p, _P(_V)]),
+    "tpc_kda_export_states": (ctypes.c_int, [_V, _P(KdaShape), _V, _V, _V]),
+    "tpc_kda_backward_window": (ctypes.c_int, [_V, _P(KdaShape), _P(KdaBwdIO), _V, _V, ctypes.c_size_t, _V]),
+    "tpc_gather_rows": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _V]),
+    "tpc_add_rows": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V]),
     "tpc_plan_get_info": (ctypes.c_int, [_V, _P(PlanInfo)]),
     "tpc_plan_export": (ctypes.c_int, [_V, _P(PlanTables)]),
     "tpc_plan_device_bytes": (ctypes.c_size_t, [_V]),
@@ -182,12 +189,17 @@ class Plan:
     """Round plan of a rollout tree (host object; ``upload`` places its tables on the device).
     mode: PLAN_MIN_ROUNDS (default), or the ablations PLAN_NODEWISE / PLAN_NO_REPLAY."""
 
-    def __init__(self, parent, length, chunk: int, mode: int = PLAN_MIN_ROUNDS):
+    def __init__(self, parent, length, chunk: int, mode: int = PLAN_MIN_ROUNDS, exports=None):
+        """exports: optional [(node, position)] boundary states to export (tpc_plan_create_window)."""
         parent = np.ascontiguousarray(parent, np.int32)
         length = np.ascontiguousarray(length, np.int32)
         h = ctypes.c_void_p()
-        _check(lib().tpc_plan_create_mode(parent.ctypes.data_as(i32p), length.ctypes.data_as(i32p),
-                                          int(parent.shape[0]), int(chunk), int(mode), ctypes.byref(h)))
+        ex = list(exports or [])
+        en = np.ascontiguousarray([e[0] for e in ex] or [0], np.int32)
+        ep = np.ascontiguousarray([e[1] for e in ex] or [0], np.int64)
+        _check(lib().tpc_plan_create_window(parent.ctypes.data_as(i32p), length.ctypes.data_as(i32p),
+                                            int(parent.shape[0]), int(chunk), int(mode), len(ex),
+                                            en.ctypes.data_as(i32p), ep.ctypes.data_as(i64p), ctypes.byref(h)))
         self.mode = int(mode)
         self._h = h
         self.n_nodes = int(parent.shape[0])
@@ -381,8 +393,33 @@ def tpc_kda_static_status(stream=None):
     _check(lib().tpc_kda_static_status(_stream_ptr(stream)))
 
 
+def tpc_kda_export_states(plan: Plan, ws, H, d, stream=None):
+    """The plan's exported boundary states after tpc_kda_forward: fp32 [n_exports, H, d, d]."""
+    import torch
+    out = torch.empty(plan.info["n_exports"], H, d, d, dtype=torch.float32, device=ws.device)
+    shape = kda_shape(H, d, 0, 0)
+    _check(lib().tpc_kda_export_states(plan.handle, ctypes.byref(shape), _ptr(ws), _ptr(out), _stream_ptr(stream)))
+    return out
+
+
+def tpc_gather_rows(src, rows, stream=None):
+    """dst[i] = src[rows[i]] for a [R, ...] tensor (2- or 4-byte elements) and int32 device rows."""
+    import torch
+    width = int(np.prod(src.shape[1:]))
+    out = torch.empty((rows.numel(),) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    _check(lib().tpc_gather_rows(_ptr(src), _ptr(rows), _ptr(out), rows.numel(), width, src.element_size(),
+                                 _stream_ptr(stream)))
+    return out
+
+
+def tpc_add_rows(src, rows, dst, stream=None):
+    """dst[rows[i]] += src[i] (fp32; distinct rows)."""
+    width = int(np.prod(src.shape[1:]))
+    _check(lib().tpc_add_rows(_ptr(src), _ptr(rows), _ptr(dst), rows.numel(), width, _stream_ptr(stream)))
+
+
 def tpc_kda_backward(plan: Plan, ws, q, k, v, g, beta, d_o, d_final=None, init_state=None, out_dtype=None,
-                     want_d_init=True, grads=None, stream=None, split=False):
+                     want_d_init=True, grads=None, stream=None, split=False, export_grads=None):
     """Backward; returns dict(dq, dk, dv, dg, dbeta, d_init).  split: as tpc_kda_forward (must match
     the forward that filled ws)."""
     import torch
@@ -404,8 +441,8 @@ def tpc_kda_backward(plan: Plan, ws, q, k, v, g, beta, d_o, d_final=None, init_s
                   None if d_final is None else d_final.data_ptr(),
                   grads["dq"].data_ptr(), grads["dk"].data_ptr(), grads["dv"].data_ptr(), grads["dg"].data_ptr(),
                   grads["dbeta"].data_ptr(), None if grads.get("d_init") is None else grads["d_init"].data_ptr())
-    _check(lib().tpc_kda_backward(plan.handle, ctypes.byref(shape), ctypes.byref(io), _ptr(ws), ws.numel(),
-                                  _stream_ptr(stream)))
+    _check(lib().tpc_kda_backward_window(plan.handle, ctypes.byref(shape), ctypes.byref(io), _ptr(export_grads),
+                                         _ptr(ws), ws.numel(), _stream_ptr(stream)))
     return grads
 
 

@@ -273,10 +273,13 @@ struct Ld {
   int* status;
 };
 
+// One phase of loads: the issuing thread first calls ld_expect with the phase's total bytes (the
+// barrier's single arrival), then issues the copies (ld_state_tile, ld_cd_tile, ld_cc_tile).
+__device__ __forceinline__ void ld_expect(Ld& l, uint32_t bytes) { tc::mbar_arrive_expect_tx(l.bar, bytes); }
+
 // one chunk-head's state tile (S0 or dS: hi half then lo half, kStateTileBytes) into hi and lo
 __device__ __forceinline__ void ld_state_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
   const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kStateTileBytes;
-  tc::mbar_arrive_expect_tx(l.bar, kStateTileBytes);
   tc::bulk_g2s(hi, src, kStateTileBytes / 2, l.bar);
   tc::bulk_g2s(lo, src + kStateTileBytes / 2, kStateTileBytes / 2, l.bar);
 }
@@ -285,13 +288,11 @@ __device__ __forceinline__ void ld_state_tile(Ld& l, uint8_t* hi, uint8_t* lo, c
 constexpr uint32_t kCDTileBytes = 2u * kTcC * kTcD * 2u, kCCTileBytes = 2u * kTcC * kTcC * 2u;
 __device__ __forceinline__ void ld_cd_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
   const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kCDTileBytes;
-  tc::mbar_arrive_expect_tx(l.bar, kCDTileBytes);
   tc::bulk_g2s(hi, src, kCDTileBytes / 2, l.bar);
   tc::bulk_g2s(lo, src + kCDTileBytes / 2, kCDTileBytes / 2, l.bar);
 }
 __device__ __forceinline__ void ld_cc_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
   const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kCCTileBytes;
-  tc::mbar_arrive_expect_tx(l.bar, kCCTileBytes);
   tc::bulk_g2s(hi, src, kCCTileBytes / 2, l.bar);
   tc::bulk_g2s(lo, src + kCCTileBytes / 2, kCCTileBytes / 2, l.bar);
 }
@@ -678,6 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bar, 1);
     tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    ld_expect(ld, kStateTileBytes + kCDTileBytes);
     ld_state_tile(ld, s0h, s0l, ws.S0, base);  // the chunk-start state, as the scan left it
     ld_cd_tile(ld, tsm + S::Wq, tsm + S::Wq + S::CDb, ws.W, base);  // W, as the prep kernel left it
   }
@@ -792,6 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bar, 1);
     tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    ld_expect(ld, kCDTileBytes + kCCTileBytes);
     ld_cd_tile(ld, wh, wl, ws.W, base);
     ld_cc_tile(ld, ph, pl, ws.Pm, base);
   }
@@ -899,6 +902,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bar, 1);
     tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    ld_expect(ld, kStateTileBytes + kCDTileBytes);
     ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
     ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
   }
@@ -929,7 +933,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // phase 2: T1 = U dS^T and dU = dU0 + Khat dS (Khat = k e^{G_C - G}, K-major in the dO slot);
     // the gradient of the chunk-end state replaces S0 in its buffer
-    if (tid == 0) ld_state_tile(ld, sh, sl, ws.dS, base);
+    if (tid == 0) {
+      ld_expect(ld, kStateTileBytes);
+      ld_state_tile(ld, sh, sl, ws.dS, base);
+    }
     const float* gC = sG + (n - 1) * LD;
     build_tile_ld<C, D, true, Tin>(doh, dol, row_k, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
     ok = ld_wait(ld);
@@ -1181,6 +1188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- phase 2b: dW' = dU S0^T
     uint8_t *duh = R + S::p2_dU, *dul = duh + S::CDb, *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
     if (tid == 0) {  // the phase 2a operands are consumed
+      ld_expect(ld, kStateTileBytes + kCDTileBytes);
       ld_state_tile(ld, s0h, s0l, ws.S0, base);
       ld_cd_tile(ld, duh, dul, ws.dUt, base);
     }
@@ -1201,7 +1209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) m[j] = -v[j];
       put16<C, true>(dxh, dxl, r, c0, m);
     });
-    if (tid == 0) ld_cd_tile(ld, dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), ws.dUt, base);
+    if (tid == 0) {
+      ld_expect(ld, kCDTileBytes);
+      ld_cd_tile(ld, dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), ws.dUt, base);
+    }
     ok = ld_wait(ld);
     ok = ok && run(sy, [&] {
       const tc::Op aH{tc::smem_u32(tTh), C, true}, aL{tc::smem_u32(tTl), C, true};

@@ -98,6 +98,7 @@ struct Plan {
   std::vector<int32_t> exp_rows, occ_begin, occ_list;
   std::vector<int64_t> exp_rows64, traj_offset;
   std::vector<int32_t> round_seq_begin, round_chunk_begin;  // [n_rounds + 1], host only
+  std::vector<int32_t> ext_slot;  // slot of each external export (its consumer id is n_seqs + e)
   std::vector<AttnNode> attn_nodes;
   std::vector<int32_t> attn_ranges;  // pairs
   std::vector<AttnTile> attn_qtiles, attn_ktiles;
@@ -110,8 +111,10 @@ struct Plan {
 };
 
 // Builds the plan; returns an empty string or an error message.
+// ext_node / ext_pos: external boundary-state exports (sharing windows), n_ext of them.
 std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, int32_t C, Plan& out,
-                       int mode = kPlanMinRounds);
+                       int mode = kPlanMinRounds, int32_t n_ext = 0, const int32_t* ext_node = nullptr,
+                       const int64_t* ext_pos = nullptr);
 // Packs the device blob; returns the layout (offsets per table) and the total bytes.
 size_t device_layout(const Plan& p, std::vector<size_t>& offsets);
 void pack_device_blob(const Plan& p, const std::vector<size_t>& offsets, std::vector<uint8_t>& blob);

@@ -33,7 +33,8 @@
 
 namespace tpc {
 
-std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, int32_t C, Plan& P, int mode) {
+std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, int32_t C, Plan& P, int mode,
+                       int32_t n_ext, const int32_t* ext_node, const int64_t* ext_pos) {
   if (n <= 0) return "tree has no nodes";
   if (C != 16 && C != 32 && C != 64) return "chunk size must be 16, 32 or 64";
   if (mode != kPlanMinRounds && mode != kPlanNodewise && mode != kPlanNoReplay) return "unknown plan mode";
@@ -79,6 +80,16 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
     }
   }
   if (P.s.empty()) return "internal";
+  // external exports (sharing windows): the state after token pos - 1 of node u's path, u holding it
+  if (n_ext < 0 || (n_ext > 0 && (!ext_node || !ext_pos))) return "exports: count or arrays invalid";
+  for (int32_t e = 0; e < n_ext; ++e) {
+    const int32_t u = ext_node[e];
+    const int64_t b = ext_pos[e];
+    if (u < 0 || u >= n) return "export " + std::to_string(e) + ": node out of range";
+    if (b % C != 0 || b <= P.s[u] || b > P.s[u] + length[u])
+      return "export " + std::to_string(e) + ": position must be a multiple of the chunk inside node " +
+             std::to_string(u) + " (s < pos <= s + length)";
+  }
   for (int32_t v = 0; v < n; ++v)
     if (P.s[v] + length[v] >= (int64_t(1) << 31)) return "trajectory longer than 2^31 tokens";
 
@@ -197,12 +208,13 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
     seq_leaf.push_back(u);
   }
 
-  // slots: distinct (anchor, b) over heads with b > 0
+  // slots: distinct (anchor, b) over heads with b > 0, and the external exports
   std::map<std::pair<int32_t, int64_t>, std::vector<int32_t>> keyset;
   for (size_t si = 0; si < P.seqs.size(); ++si) {
     int32_t h = P.seqs[si].head;
     if (parent[h] >= 0 && P.b[h] > 0) keyset[{P.anchor[h], P.b[h]}].push_back((int32_t)si);
   }
+  for (int32_t e = 0; e < n_ext; ++e) keyset[{ext_node[e], ext_pos[e]}];  // (no in-tree consumer needed)
   std::vector<std::tuple<int32_t, int32_t, int64_t, int32_t>> skeys;  // (round, producer seq, b, anchor)
   for (auto& kv : keyset)
     skeys.emplace_back(P.round[kv.first.first], seq_of[kv.first.first], kv.first.second, kv.first.first);
@@ -220,8 +232,22 @@ std::string build_plan(const int32_t* parent, const int32_t* length, int32_t n, 
     sr.n_cons = (int32_t)cons.size();
     int32_t sid = (int32_t)P.slots.size();
     for (int32_t c : cons) { P.slot_cons.push_back(c); P.seqs[c].import_id = sid; }
+    // external consumers after the in-tree ones: pseudo-sequence ids n_seqs + e, whose start-state
+    // gradients the caller provides (tpc_kda_backward_window)
+    for (int32_t e = 0; e < n_ext; ++e)
+      if (ext_node[e] == an && ext_pos[e] == bb) {
+        P.slot_cons.push_back((int32_t)P.seqs.size() + e);
+        sr.n_cons++;
+      }
     slot_at[{sr.producer_seq, bb}] = sid;
     P.slots.push_back(sr);
+  }
+  P.ext_slot.assign(n_ext, -1);
+  for (int32_t e = 0; e < n_ext; ++e) {
+    const int32_t pseudo = (int32_t)P.seqs.size() + e;
+    for (size_t sid = 0; sid < P.slots.size(); ++sid)
+      for (int32_t m = 0; m < P.slots[sid].n_cons; ++m)
+        if (P.slot_cons[P.slots[sid].cons_begin + m] == pseudo) P.ext_slot[e] = (int32_t)sid;
   }
 
   // root consumers (sequences reading an initial state), by head id

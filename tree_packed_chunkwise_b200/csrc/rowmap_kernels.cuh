@@ -31,6 +31,23 @@ __global__ void occurrence_count_kernel(DevTables t, int32_t* __restrict__ count
 }
 
 // absolute trajectory position (depth) of every compact row: one CTA per node
+// dst[i] = src[rows[i]] (rows of `width` elements)
+template <typename T>
+__global__ void gather_list_kernel(const T* __restrict__ src, const int32_t* __restrict__ rows, T* __restrict__ dst,
+                                   int64_t width) {
+  const int64_t i = blockIdx.x;
+  const T* s = src + (int64_t)rows[i] * width;
+  for (int64_t c = threadIdx.x; c < width; c += blockDim.x) dst[i * width + c] = s[c];
+}
+
+// dst[rows[i]] += src[i]; the rows of one call are distinct (one writer per row, no atomics)
+__global__ void add_list_kernel(const float* __restrict__ src, const int32_t* __restrict__ rows, float* __restrict__ dst,
+                                int64_t width) {
+  const int64_t i = blockIdx.x;
+  float* d = dst + (int64_t)rows[i] * width;
+  for (int64_t c = threadIdx.x; c < width; c += blockDim.x) d[c] += src[i * width + c];
+}
+
 __global__ void rope_positions_kernel(DevTables t, int32_t* __restrict__ pos) {
   const AttnNode nd = t.attn_nodes[blockIdx.x];
   for (int i = threadIdx.x; i < nd.length; i += blockDim.x) pos[nd.row_offset + i] = nd.pos0 + i;

@@ -123,7 +123,7 @@ WsLayout ws_layout(const tpc::Plan& p, int H, int C, int D) {
   L.slot = take(p.slots.size() * H * dd * 4);
   L.dU = take(nc * H * cd * 4);
   L.dS = take(nc * H * dd * 4);
-  L.dS0seq = take(p.seqs.size() * H * dd * 4);
+  L.dS0seq = take((p.seqs.size() + p.ext_slot.size()) * H * dd * 4);  // + external consumers' gradients
   L.pdk = take(nc * H * cd * 4);
   L.pdG = take(nc * H * cd * 4);
   L.rdk = take(R * H * D * 4);
@@ -494,15 +494,17 @@ extern "C" {
 const char* tpc_last_error(void) { return tpc_abi::g_err.c_str(); }
 const char* tpc_version(void) { return "tpc 0.1 (sm_100a)"; }
 
-int tpc_plan_create_mode(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, int32_t mode,
-                         tpc_plan** out) {
+int tpc_plan_create_window(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, int32_t mode,
+                           int32_t n_exports, const int32_t* export_node, const int64_t* export_pos, tpc_plan** out) {
   if (!parent || !length || !out) return fail(TPC_ERR_NULL, "parent, length and out must be non-NULL");
+  if (n_exports < 0 || (n_exports > 0 && (!export_node || !export_pos)))
+    return fail(TPC_ERR_NULL, "export_node and export_pos are required when n_exports > 0");
   *out = nullptr;
   tpc_plan* p = new (std::nothrow) tpc_plan();
   if (!p) return fail(TPC_ERR_CUDA, "out of host memory");
   std::string err;
   try {
-    err = tpc::build_plan(parent, length, n_nodes, chunk, p->p, mode);
+    err = tpc::build_plan(parent, length, n_nodes, chunk, p->p, mode, n_exports, export_node, export_pos);
   } catch (const std::exception& e) {
     err = std::string("planner: ") + e.what();
   }
@@ -513,6 +515,11 @@ int tpc_plan_create_mode(const int32_t* parent, const int32_t* length, int32_t n
   }
   *out = p;
   return TPC_OK;
+}
+
+int tpc_plan_create_mode(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, int32_t mode,
+                         tpc_plan** out) {
+  return tpc_plan_create_window(parent, length, n_nodes, chunk, mode, 0, nullptr, nullptr, out);
 }
 
 int tpc_plan_create(const int32_t* parent, const int32_t* length, int32_t n_nodes, int32_t chunk, tpc_plan** out) {
@@ -538,6 +545,7 @@ int tpc_plan_get_info(const tpc_plan* plan, tpc_plan_info* info) {
   info->chunk = p.C;
   info->max_seq_chunks = p.max_seq_chunks;
   info->n_replay_targets = (int32_t)p.tgt_row.size();
+  info->n_exports = (int32_t)p.ext_slot.size();
   return TPC_OK;
 }
 
@@ -605,18 +613,74 @@ int tpc_kda_forward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_
   });
 }
 
-int tpc_kda_backward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_bwd_io* io, void* ws, size_t ws_bytes,
-                     tpc_stream_t stream) {
+int tpc_kda_backward_window(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_bwd_io* io,
+                            const float* export_grads, void* ws, size_t ws_bytes, tpc_stream_t stream) {
   if (int rc = check_shape(plan, s)) return rc;
   if (!io || !io->q || !io->k || !io->v || !io->g || !io->beta || !io->d_o || !io->dq || !io->dk || !io->dv ||
       !io->dg || !io->dbeta || !ws)
     return fail(TPC_ERR_NULL, "backward: inputs, d_o, gradient outputs and ws are required");
   if (ws_bytes < tpc_kda_workspace_bytes(plan, s)) return fail(TPC_ERR_WORKSPACE, "workspace too small");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the external consumers' start-state gradients enter the reverse scans like in-tree consumers'
+  const tpc::Plan& pl = plan->p;
+  if (!pl.ext_slot.empty()) {
+    const WsLayout L = ws_layout(pl, s->H, pl.C, s->dk);
+    const size_t per = (size_t)s->H * s->dk * s->dv * 4;
+    char* dst = static_cast<char*>(ws) + L.dS0seq + pl.seqs.size() * per;
+    if (export_grads)
+      TPC_CUDA(cudaMemcpyAsync(dst, export_grads, pl.ext_slot.size() * per, cudaMemcpyDeviceToDevice, st));
+    else
+      TPC_CUDA(cudaMemsetAsync(dst, 0, pl.ext_slot.size() * per, st));
+  }
   return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout, auto tc) {
     return backward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout), decltype(tc)::value>(
         plan->p, s, io, ws, st);
   });
+}
+
+int tpc_kda_backward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_bwd_io* io, void* ws, size_t ws_bytes,
+                     tpc_stream_t stream) {
+  return tpc_kda_backward_window(plan, s, io, nullptr, ws, ws_bytes, stream);
+}
+
+int tpc_kda_export_states(const tpc_plan* plan, const tpc_kda_shape* s, const void* ws, float* states,
+                          tpc_stream_t stream) {
+  if (int rc = check_shape(plan, s)) return rc;
+  if (!ws || !states) return fail(TPC_ERR_NULL, "ws and states are required");
+  const tpc::Plan& pl = plan->p;
+  const WsLayout L = ws_layout(pl, s->H, pl.C, s->dk);
+  const size_t per = (size_t)s->H * s->dk * s->dv * 4;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (size_t e = 0; e < pl.ext_slot.size(); ++e)
+    TPC_CUDA(cudaMemcpyAsync(reinterpret_cast<char*>(states) + e * per,
+                             static_cast<const char*>(ws) + L.slot + (size_t)pl.ext_slot[e] * per, per,
+                             cudaMemcpyDeviceToDevice, st));
+  return TPC_OK;
+}
+
+int tpc_gather_rows(const void* src, const int32_t* rows, void* dst, int64_t n_rows, int64_t width, int32_t elem_bytes,
+                    tpc_stream_t stream) {
+  if (!src || !rows || !dst) return fail(TPC_ERR_NULL, "src, rows and dst are required");
+  if (n_rows < 0 || width < 1 || (elem_bytes != 2 && elem_bytes != 4))
+    return fail(TPC_ERR_BAD_SHAPE, "n_rows >= 0, width >= 1, elem_bytes 2 or 4");
+  if (n_rows == 0) return TPC_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (elem_bytes == 2)
+    TPC_LAUNCH("gather_rows", st, (tpc::gather_list_kernel<uint16_t><<<(unsigned)n_rows, 128, 0, st>>>(
+                                      (const uint16_t*)src, rows, (uint16_t*)dst, width)));
+  else
+    TPC_LAUNCH("gather_rows", st, (tpc::gather_list_kernel<uint32_t><<<(unsigned)n_rows, 128, 0, st>>>(
+                                      (const uint32_t*)src, rows, (uint32_t*)dst, width)));
+  return TPC_OK;
+}
+
+int tpc_add_rows(const float* src, const int32_t* rows, float* dst, int64_t n_rows, int64_t width, tpc_stream_t stream) {
+  if (!src || !rows || !dst) return fail(TPC_ERR_NULL, "src, rows and dst are required");
+  if (n_rows < 0 || width < 1) return fail(TPC_ERR_BAD_SHAPE, "n_rows >= 0, width >= 1");
+  if (n_rows == 0) return TPC_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TPC_LAUNCH("add_rows", st, (tpc::add_list_kernel<<<(unsigned)n_rows, 128, 0, st>>>(src, rows, dst, width)));
+  return TPC_OK;
 }
 
 int tpc_status(const tpc_plan* plan, const tpc_kda_shape* s, void* ws, tpc_stream_t stream) {
