@@ -169,6 +169,20 @@ int tpc_plan_export(const tpc_plan* plan, tpc_plan_tables* tables);
  * records the address in the plan, which every later device call uses.
  * The memory must stay valid while the plan is used.
  */
+/*
+ * Diagnostics: the device-facing tables as int32 rows (caller-owned host arrays, NULL skips one):
+ *   seqs   [n_seqs][8]   chunk_begin, n_chunks, import (slot >= 0, or -(root ordinal + 1)),
+ *                        leaf ordinal (-1: the chain ends at an internal node), head node, round,
+ *                        start position, replayed rows
+ *   chunks [n_chunks][8] sequence, rows, replayed rows, first own compact row, replay base, export
+ *                        slot (-1 none), first position, index in the sequence
+ *   slots  [n_slots][4]  producing sequence, exporting chunk, first consumer, consumers
+ *   slot_cons [sum of consumers] consumer sequences (n_seqs + e for external export e)
+ *   replay_rows [replay_total] compact row of every replayed row
+ */
+int tpc_plan_debug_tables(const tpc_plan* plan, int32_t* seqs, int32_t* chunks, int32_t* slots, int32_t* slot_cons,
+                          int32_t* replay_rows);
+
 size_t tpc_plan_device_bytes(const tpc_plan* plan);
 int tpc_plan_upload(tpc_plan* plan, void* dev, size_t bytes, tpc_stream_t stream);
 

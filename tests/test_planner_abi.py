@@ -142,3 +142,44 @@ def test_invalid_inputs_return_status(tpc):
         tpc.Plan([-1], [4], 48)
     assert e.value.code == 3
     assert tpc.lib().tpc_plan_device_bytes(None) == 0
+
+
+def check_device_tables(pl, n_leaves, n_roots, C):
+    """Bounds every kernel relies on: rows, replay indices, slots, consumers, leaves and imports."""
+    d = pl.debug_tables()
+    i = pl.info
+    N, R = i["n_unique"], i["replay_total"]
+    ns, nc, nsl = i["n_seqs"], i["n_chunks"], i["n_slots"]
+    for si, (cb, n_ch, imp, leaf, head, rnd, start, nrep) in enumerate(d["seqs"]):
+        assert 0 <= cb and cb + n_ch <= nc and n_ch >= 1
+        assert -1 <= leaf < n_leaves and 1 <= rnd <= i["n_rounds"] and 0 <= nrep < C
+        assert (0 <= imp < nsl) or (-n_roots <= imp <= -1)
+    for ci, (seq, n, nrep, row0, rbase, slot, pos0, idx) in enumerate(d["chunks"]):
+        assert 0 <= seq < ns and 1 <= n <= C and 0 <= nrep <= n
+        assert 0 <= row0 and row0 + (n - nrep) <= N
+        assert nrep == 0 or (0 <= rbase and rbase + nrep <= R)
+        assert -1 <= slot < nsl
+    for prod, ech, cb, ncons in d["slots"]:
+        assert 0 <= prod < ns and 0 <= ech < nc and d["chunks"][ech][5] >= 0
+        assert all(0 <= c < ns + i["n_exports"] for c in d["slot_cons"][cb:cb + ncons])
+    assert np.all((d["replay_rows"] >= 0) & (d["replay_rows"] < N))
+
+
+@pytest.mark.parametrize("mode", ["min_rounds", "nodewise", "noreplay"])
+def test_device_tables_within_bounds(tpc, mode):
+    for cfg in ("fig1", "agentic_small", "agentic", "single_fork"):
+        w = synth.workload(cfg)
+        t = w.tree
+        pl = tpc.Plan(t.parent, t.length, w.chunk, MODE_CODE[mode])
+        check_device_tables(pl, len(t.leaves()), int((t.parent < 0).sum()), w.chunk)
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        n = int(rng.integers(1, 30))
+        parent = np.array([-1] + [(-1 if rng.random() < 0.05 else int(rng.integers(0, i))) for i in range(1, n)],
+                          np.int32)
+        length = rng.integers(1, 150, size=n).astype(np.int32)
+        pl = tpc.Plan(parent, length, 64, MODE_CODE[mode])
+        has_child = np.zeros(n, bool)
+        has_child[parent[parent >= 0]] = True
+        check_device_tables(pl, int((~has_child).sum()), int((parent < 0).sum()), 64)
+

@@ -113,6 +113,7 @@ SIGNATURES = {
     "tpc_plan_get_info": (ctypes.c_int, [_V, _P(PlanInfo)]),
     "tpc_plan_export": (ctypes.c_int, [_V, _P(PlanTables)]),
     "tpc_plan_device_bytes": (ctypes.c_size_t, [_V]),
+    "tpc_plan_debug_tables": (ctypes.c_int, [_V, _V, _V, _V, _V, _V]),
     "tpc_plan_upload": (ctypes.c_int, [_V, _V, ctypes.c_size_t, _V]),
     "tpc_kda_workspace_bytes": (ctypes.c_size_t, [_V, _P(KdaShape)]),
     "tpc_kda_forward": (ctypes.c_int, [_V, _P(KdaShape), _P(KdaFwdIO), _V, ctypes.c_size_t, _V]),
@@ -228,6 +229,21 @@ class Plan:
         t = PlanTables(**{k: v.ctypes.data_as(i64p if v.dtype == np.int64 else i32p) for k, v in out.items()})
         _check(lib().tpc_plan_export(self._h, ctypes.byref(t)))
         return out
+
+    def debug_tables(self) -> dict:
+        """The device-facing sequence / chunk / slot tables (tpc_plan_debug_tables) as int32 arrays."""
+        i = self.info
+        seqs = np.zeros((i["n_seqs"], 8), np.int32)
+        chunks = np.zeros((i["n_chunks"], 8), np.int32)
+        slots = np.zeros((i["n_slots"], 4), np.int32)
+        ncons = 0
+        _check(lib().tpc_plan_debug_tables(self._h, None, None, slots.ctypes.data, None, None))
+        ncons = int(slots[:, 3].sum()) if len(slots) else 0
+        cons = np.zeros(max(ncons, 1), np.int32)
+        rep = np.zeros(max(i["replay_total"], 1), np.int32)
+        _check(lib().tpc_plan_debug_tables(self._h, seqs.ctypes.data, chunks.ctypes.data, slots.ctypes.data,
+                                           cons.ctypes.data, rep.ctypes.data))
+        return dict(seqs=seqs, chunks=chunks, slots=slots, slot_cons=cons[:ncons], replay_rows=rep[:i["replay_total"]])
 
     def upload(self, device="cuda", stream=None):
         import torch

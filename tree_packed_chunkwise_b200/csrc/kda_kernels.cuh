@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kThreads) kda_fwd_scan(DevTables t, int seq0, 
       }
     }
   }
-  if (final_state) {
+  if (final_state && s.leaf >= 0) {  // a sequence ending at an internal node has no final state
     float* dst = final_state + ((size_t)s.leaf * H + h) * K::DD;
     for (int e = threadIdx.x; e < D * DVT; e += blockDim.x) {
       const int c = e / DVT, j = e % DVT;
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(kThreads) kda_bwd_scan(DevTables t, int seq0, 
   float* sdec = sX + D * LT;
   for (int e = threadIdx.x; e < D * DVT; e += blockDim.x) {
     const int c = e / DVT, j = e % DVT;
-    sdS[c * LT + j] = d_final ? d_final[((size_t)s.leaf * H + h) * K::DD + c * D + j0 + j] : 0.f;
+    sdS[c * LT + j] = (d_final && s.leaf >= 0) ? d_final[((size_t)s.leaf * H + h) * K::DD + c * D + j0 + j] : 0.f;
   }
   __syncthreads();
   for (int q = s.n_chunks - 1; q >= 0; --q) {

@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     if (!REVERSE) {
       if (sq.import_id >= 0) src = ws.slot + ((size_t)sq.import_id * H + h) * D * D;
       else if (init) src = init + ((size_t)(-(sq.import_id + 1)) * H + h) * D * D;
-    } else if (d_final) {
+    } else if (d_final && sq.leaf >= 0) {  // a sequence ending at an internal node has no final state
       src = d_final + ((size_t)sq.leaf * H + h) * D * D;
     }
     if (src) ld32g(src + c * D + j0, s);
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   }
   if (ok) {
     if (!REVERSE) {
-      if (final_state) st32g(final_state + ((size_t)sq.leaf * H + h) * D * D + c * D + j0, s);
+      if (final_state && sq.leaf >= 0) st32g(final_state + ((size_t)sq.leaf * H + h) * D * D + c * D + j0, s);
     } else {
       st32g(ws.dS0seq + ((size_t)si * H + h) * D * D + c * D + j0, s);
     }

@@ -11,7 +11,8 @@ struct SeqRec {
   int32_t chunk_begin;  // first chunk (chunks of a sequence are consecutive)
   int32_t n_chunks;
   int32_t import_id;    // >= 0: boundary-state slot; < 0: initial state of root ordinal -(id+1)
-  int32_t leaf;         // leaf ordinal whose final state this sequence produces
+  int32_t leaf;         // leaf ordinal whose final state this sequence produces; -1 when the chain
+                        // ends at an internal node (node-wise plans), which has no final state
   int32_t head;         // head node id
   int32_t round;        // 1-based
   int32_t start_pos;    // absolute position of the first (possibly replayed) row

@@ -568,6 +568,20 @@ int tpc_plan_export(const tpc_plan* plan, tpc_plan_tables* t) {
   return TPC_OK;
 }
 
+int tpc_plan_debug_tables(const tpc_plan* plan, int32_t* seqs, int32_t* chunks, int32_t* slots, int32_t* slot_cons,
+                          int32_t* replay_rows) {
+  if (!plan) return fail(TPC_ERR_NULL, "plan is NULL");
+  const tpc::Plan& p = plan->p;
+  static_assert(sizeof(tpc::SeqRec) == 8 * 4 && sizeof(tpc::ChunkRec) == 8 * 4 && sizeof(tpc::SlotRec) == 4 * 4,
+                "table records are rows of int32");
+  if (seqs) std::memcpy(seqs, p.seqs.data(), p.seqs.size() * sizeof(tpc::SeqRec));
+  if (chunks) std::memcpy(chunks, p.chunks.data(), p.chunks.size() * sizeof(tpc::ChunkRec));
+  if (slots) std::memcpy(slots, p.slots.data(), p.slots.size() * sizeof(tpc::SlotRec));
+  if (slot_cons) std::memcpy(slot_cons, p.slot_cons.data(), p.slot_cons.size() * 4);
+  if (replay_rows) std::memcpy(replay_rows, p.replay_rows.data(), p.replay_rows.size() * 4);
+  return TPC_OK;
+}
+
 size_t tpc_plan_device_bytes(const tpc_plan* plan) {
   if (!plan) return 0;
   std::vector<size_t> off;
