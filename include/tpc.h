@@ -417,6 +417,37 @@ int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int
                          void* scratch, size_t scratch_bytes, int32_t chunk_rows, int32_t* status,
                          tpc_stream_t stream);
 
+/* ------------------------------------------------------------------ compact MoE routing */
+/*
+ * Deterministic top-k routing of the unique rows with occurrence counts (HARTS abstract: for
+ * deterministic top-k routing without token dropping, occurrence counts restore MoE objective
+ * weights and expert-load statistics; Figure 1: q_B = 2 restores them without repeating routing or
+ * expert computation; Figure C.1(d): multiplicity-weighted router losses and expert-load counts).
+ * Every unique row u is routed once; each of its q_u trajectory positions would route identically,
+ * so statistics over positions are q_u-weighted sums over unique rows.
+ *   tpc_moe_route: z_u = W_r h_u (fp32, a fixed-order sum over the hidden dimension of separately
+ *     rounded products, so the top-k decision is reproducible), lse_u, the top-k experts (larger
+ *     logit first, ties to the lower expert index) and their gates (softmax renormalised over the
+ *     top-k), expert_load_e = sum_u q_u [e in topk(u)] (exact integers) and
+ *     prob_sum_e = sum_u q_u softmax(z_u)_e.
+ *     h: bf16 [N_unique][Dh] (compact rows), w_router: bf16 [E][Dh], Dh a multiple of 64, E <= 256,
+ *     1 <= k <= min(E, 8).  logits fp32 [N][E], lse fp32 [N], topk_idx int32 [N][k], topk_gate fp32
+ *     [N][k], expert_load int64 [E], prob_sum fp32 [E].
+ *   tpc_moe_router_loss: with n = n_expanded positions, L_aux = E / (k n^2) sum_e load_e P_e and
+ *     L_z = (1/n) sum over positions of lse^2 (losses[0], losses[1], device fp32), and dlogits fp32
+ *     [N][E] = the gradient of a L_aux + b L_z with respect to each unique row's logits (the
+ *     occurrence-weighted sum of the per-position gradients; the routing is held fixed).
+ *   scratch: tpc_moe_scratch_bytes(plan, E) bytes of caller device memory.  All reductions run in a
+ *   fixed order.  The expert FFNs themselves are ordinary per-row products and are not part of this.
+ */
+size_t tpc_moe_scratch_bytes(const tpc_plan* plan, int32_t E);
+int tpc_moe_route(const tpc_plan* plan, const void* h, const void* w_router, int64_t Dh, int32_t E, int32_t k,
+                  float* logits, float* lse, int32_t* topk_idx, float* topk_gate, int64_t* expert_load,
+                  float* prob_sum, void* scratch, size_t scratch_bytes, tpc_stream_t stream);
+int tpc_moe_router_loss(const tpc_plan* plan, const float* logits, const float* lse, const int64_t* expert_load,
+                        const float* prob_sum, int32_t E, int32_t k, float a, float b, float* losses, float* dlogits,
+                        void* scratch, size_t scratch_bytes, tpc_stream_t stream);
+
 /* ------------------------------------------------------------------ hybrid layer group */
 /*
  * A group of n_kda KDA layers followed by one latent-attention (MLA) layer on the compact rows of

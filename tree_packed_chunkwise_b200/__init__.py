@@ -138,6 +138,11 @@ SIGNATURES = {
     "tpc_tree_attn_forward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V]),
     "tpc_tree_attn_backward": (ctypes.c_int, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V]),
     "tpc_rope_positions": (ctypes.c_int, [_V, _V, _V]),
+    "tpc_moe_scratch_bytes": (ctypes.c_size_t, [_V, ctypes.c_int32]),
+    "tpc_moe_route": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _V, _V, _V, _V, _V,
+                                     _V, _V, ctypes.c_size_t, _V]),
+    "tpc_moe_router_loss": (ctypes.c_int, [_V, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                                           ctypes.c_float, _V, _V, _V, ctypes.c_size_t, _V]),
     "tpc_group_workspace_bytes": (ctypes.c_size_t, [_V, _P(GroupShape)]),
     "tpc_group_forward": (ctypes.c_int, [_V, _P(GroupShape), _P(GroupWeights), _V, _V, _V, _V, ctypes.c_size_t, _V]),
     "tpc_group_backward": (ctypes.c_int, [_V, _P(GroupShape), _P(GroupWeights), _V, _V, _V, _V, _P(GroupGrads), _V,
@@ -643,6 +648,41 @@ def tpc_rope_positions(plan: Plan, device="cuda", stream=None):
     pos = torch.empty(plan.info["n_unique"], dtype=torch.int32, device=device)
     _check(lib().tpc_rope_positions(plan.handle, _ptr(pos), _stream_ptr(stream)))
     return pos
+
+
+# ------------------------------------------------------------------------------------ compact MoE routing
+def tpc_moe_route(plan: Plan, h, w_router, k, scratch=None, stream=None):
+    """Routes every unique row once (include/tpc.h).  Returns dict(logits, lse, topk_idx, topk_gate,
+    expert_load, prob_sum, scratch)."""
+    import torch
+    N, Dh = h.shape
+    E = w_router.shape[0]
+    dev = h.device
+    n = int(lib().tpc_moe_scratch_bytes(plan.handle, E))
+    scratch = scratch if scratch is not None else torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+    out = dict(logits=torch.empty(N, E, dtype=torch.float32, device=dev),
+               lse=torch.empty(N, dtype=torch.float32, device=dev),
+               topk_idx=torch.empty(N, k, dtype=torch.int32, device=dev),
+               topk_gate=torch.empty(N, k, dtype=torch.float32, device=dev),
+               expert_load=torch.empty(E, dtype=torch.int64, device=dev),
+               prob_sum=torch.empty(E, dtype=torch.float32, device=dev), scratch=scratch)
+    _check(lib().tpc_moe_route(plan.handle, _ptr(h), _ptr(w_router), Dh, E, k, _ptr(out["logits"]), _ptr(out["lse"]),
+                               _ptr(out["topk_idx"]), _ptr(out["topk_gate"]), _ptr(out["expert_load"]),
+                               _ptr(out["prob_sum"]), _ptr(scratch), scratch.numel(), _stream_ptr(stream)))
+    return out
+
+
+def tpc_moe_router_loss(plan: Plan, routed: dict, k, a=1.0, b=1.0, stream=None):
+    """(losses fp32 [2] = (L_aux, L_z), dlogits fp32 [N, E]) of the routing result."""
+    import torch
+    N, E = routed["logits"].shape
+    losses = torch.empty(2, dtype=torch.float32, device=routed["logits"].device)
+    dz = torch.empty_like(routed["logits"])
+    sc = routed["scratch"]
+    _check(lib().tpc_moe_router_loss(plan.handle, _ptr(routed["logits"]), _ptr(routed["lse"]),
+                                     _ptr(routed["expert_load"]), _ptr(routed["prob_sum"]), E, k, float(a), float(b),
+                                     _ptr(losses), _ptr(dz), _ptr(sc), sc.numel(), _stream_ptr(stream)))
+    return losses, dz
 
 
 # ------------------------------------------------------------------------------------ hybrid layer group

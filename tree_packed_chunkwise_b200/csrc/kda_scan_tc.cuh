@@ -2,10 +2,13 @@
 //
 // Per chunk the state update is affine: S_end = M S_0 + B with M = Diag(e^{G_C}) - Khat^T W and
 // B = Khat^T U' (both formed in parallel by the prep kernel; M is stored as a bf16 hi/lo tile in the
-// tensor-core operand layout).  The forward scan computes S <- M S + B per chunk, the backward scan
-// dS <- M^T dS + X (X = Qbar^T dO - W^T dU0), each as one M = 128 tcgen05 product per chunk (three
-// hi/lo chains) with the next chunk's M tile and additive term (B, resp. X, stored slice by slice:
-// [chunk][head][slice][row][32] fp32) arriving by bulk asynchronous copies meanwhile.
+// tensor-core operand layout).  The forward scan computes S <- M S + B per chunk; the backward scan
+// dS <- M^T dS + Qeff^T dO with Qeff = Qbar - P W (formed by the output kernel; O = Qeff S0 + P U',
+// so Qeff^T dO is the output's contribution to the chunk-start state gradient).  Each step is one
+// accumulator of M = 128 tcgen05 products (three hi/lo chains), with the next chunk's operands
+// arriving by asynchronous copies meanwhile: forward the M tile and this CTA's slice of B (stored
+// slice by slice, [chunk][head][slice][row][32] fp32); backward the M tile, the Qeff tile and the
+// chunk's rows of this CTA's 32 columns of dO.
 // One CTA of 128 threads per (sequence of the round, head, 32-column slice of d_v); thread c owns
 // row c of the state slice.
 #pragma once
@@ -16,12 +19,19 @@ namespace tpc {
 // bytes of one chunk-head's additive-term slice (128 rows x 32 fp32)
 constexpr uint32_t kScanAddBytes = kTcD * kScanDVT * 4;
 
-struct ScanTcSmem {
+template <bool REVERSE>
+struct ScanTcSmemT {
   static constexpr size_t M0 = 0, M1 = kMtileBytes;              // double-buffered M tiles
   static constexpr size_t St = 2 * size_t(kMtileBytes);          // state slice hi/lo (MN-major, K = 128)
   static constexpr size_t StB = size_t(kTcD) * kScanDVT * 2;
-  static constexpr size_t Add = St + 2 * StB;                    // double-buffered additive-term slices
-  static constexpr size_t total = Add + 2 * size_t(kScanAddBytes);
+  // double-buffered: forward the B slices, reverse the Qeff tiles (hi/lo, C x D)
+  static constexpr size_t X = St + 2 * StB;
+  static constexpr size_t XB = REVERSE ? size_t(2) * kTcC * kTcD * 2 : size_t(kScanAddBytes);
+  // reverse: double-buffered dO slices, hi/lo operand tiles of C rows x 32 columns (k = row, n = column)
+  static constexpr size_t dO = X + 2 * XB;
+  static constexpr size_t dOB = REVERSE ? size_t(kTcC) * kScanDVT * 2 : 0;
+  static constexpr size_t total = dO + 2 * 2 * dOB;
+  static_assert(total <= 227 * 1024, "shared memory");
 };
 
 
@@ -35,13 +45,46 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* st
   return !failed;
 }
 
-// the chunk's M tile and this CTA's slice of its additive term, on one mbarrier
-__device__ __forceinline__ void load_mtile(uint8_t* dst, const uint8_t* src, float* add_dst, const float* add_src,
-                                           uint64_t* bar) {
-  tc::mbar_arrive_expect_tx(bar, kMtileBytes + kScanAddBytes);
+// the chunk's M tile and a second operand (forward: this CTA's B slice; reverse: the Qeff tile), on one
+// mbarrier with one expected-bytes arrival
+__device__ __forceinline__ void load_mtile(uint8_t* dst, const uint8_t* src, uint8_t* x_dst, const uint8_t* x_src,
+                                           uint32_t x_bytes, uint64_t* bar) {
+  tc::mbar_arrive_expect_tx(bar, kMtileBytes + x_bytes);
 #pragma unroll
   for (int p = 0; p < 4; ++p) tc::bulk_g2s(dst + p * (kMtileBytes / 4), src + p * (kMtileBytes / 4), kMtileBytes / 4, bar);
-  tc::bulk_g2s(add_dst, add_src, kScanAddBytes, bar);
+  tc::bulk_g2s(x_dst, x_src, x_bytes / 2, bar);
+  tc::bulk_g2s(x_dst + x_bytes / 2, x_src + x_bytes / 2, x_bytes / 2, bar);
+}
+
+// This CTA's 32 columns (j0 ..) of the chunk's dO rows as an MN-major operand tile (k = chunk row,
+// n = column; element (r, j) at cm_off(r, j, C)), hi (and lo for fp32 data); rows that are replays
+// or past the chunk's end are zero.  bf16: asynchronous 16-byte copies (completed by the caller with
+// cp_async_wait); fp32: loaded, split and stored now.
+template <typename Tin>
+__device__ __forceinline__ void load_do_slice(uint8_t* hi, uint8_t* lo, const Tin* d_o, const ChunkRec& ch, int H,
+                                              int h, int j0) {
+  constexpr int C = kTcC;
+  for (int p = threadIdx.x; p < C * (kScanDVT / 8); p += blockDim.x) {
+    const int r = p >> 2, g = p & 3;
+    const bool own = r >= ch.n_replay && r < ch.n_rows;
+    const size_t row = own ? (size_t)(ch.row_start + (r - ch.n_replay)) : 0;
+    const Tin* src = d_o + (row * H + h) * kTcD + j0 + 8 * g;
+    const uint32_t off = cm_off(r, 8 * g, C);
+    if constexpr (sizeof(Tin) == 2) {
+      tc::cp_async16(hi + off, src, own ? 16u : 0u);
+    } else {
+      float x[8];
+      if (own) ld8(src, x);
+      else
+        for (int j = 0; j < 8; ++j) x[j] = 0.f;
+      __align__(16) __nv_bfloat16 a[8];
+      __align__(16) __nv_bfloat16 b[8];
+      for (int j = 0; j < 8; ++j) split_bf16(x[j], a[j], b[j]);
+      *reinterpret_cast<uint4*>(hi + off) = *reinterpret_cast<const uint4*>(a);
+      *reinterpret_cast<uint4*>(lo + off) = *reinterpret_cast<const uint4*>(b);
+    }
+  }
+  if constexpr (sizeof(Tin) == 2) tc::cp_async_commit();
 }
 
 // state slice (row c = this thread, 32 columns) -> MN-major hi/lo operand tile (k = c, n = j)
@@ -65,18 +108,21 @@ __device__ __forceinline__ void st32g(float* p, const float (&v)[32]) {
 
 }  // namespace tck
 
-template <bool REVERSE>
+// REVERSE: d_o [N, H, D] (Tin) is the output gradient; forward: unused
+template <bool REVERSE, typename Tin>
 __global__ void __launch_bounds__(kScanThreads, 1)
     kda_scan_tc(DevTables t, int seq0, int H, const float* __restrict__ init, float* __restrict__ final_state,
-                const float* __restrict__ d_final, KdaWs ws) {
+                const float* __restrict__ d_final, KdaWs ws, const Tin* __restrict__ d_o) {
   using namespace tck;
-  using S = ScanTcSmem;
-  constexpr int D = kTcD, DVT = kScanDVT;
+  using S = ScanTcSmemT<REVERSE>;
+  constexpr int D = kTcD, C = kTcC, DVT = kScanDVT;
+  constexpr bool EX = sizeof(Tin) == 2;  // bf16 dO: exact operand, no lo part
   const int si = seq0 + blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVT;
   const SeqRec sq = t.seqs[si];
   extern __shared__ __align__(1024) uint8_t tsm[];
   uint8_t* mbuf[2] = {tsm + S::M0, tsm + S::M1};
-  float* abuf[2] = {reinterpret_cast<float*>(tsm + S::Add), reinterpret_cast<float*>(tsm + S::Add + kScanAddBytes)};
+  uint8_t* xbuf[2] = {tsm + S::X, tsm + S::X + S::XB};
+  uint8_t* dobuf[2] = {tsm + S::dO, tsm + S::dO + 2 * S::dOB};  // hi, then lo at + dOB
   uint8_t *sth = tsm + S::St, *stl = sth + S::StB;
   __shared__ __align__(8) uint64_t bar_m[2];
   __shared__ __align__(8) uint64_t bar_mma;
@@ -99,11 +145,20 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   auto mtile = [&](int ci) {
     return reinterpret_cast<const uint8_t*>(ws.Mt) + ((size_t)ci * H + h) * kMtileBytes;
   };
-  // this CTA's slice of the chunk's additive term: B (forward) or X (reverse), both kept in ws.Bc
-  auto addslice = [&](int ci) { return ws.Bc + ((size_t)ci * H + h) * D * D + (size_t)blockIdx.z * D * DVT; };
-  auto prefetch = [&](int q) {
+  // forward: this CTA's slice of B; reverse: the chunk's Qeff tile (kept where the forward kept W)
+  auto xsrc = [&](int ci) -> const uint8_t* {
+    if (REVERSE) return reinterpret_cast<const uint8_t*>(ws.W) + ((size_t)ci * H + h) * S::XB;
+    return reinterpret_cast<const uint8_t*>(ws.Bc + ((size_t)ci * H + h) * D * D + (size_t)blockIdx.z * D * DVT);
+  };
+  auto prefetch = [&](int q) {  // thread 0: bulk copies
     const int ci = chunk_at(q);
-    load_mtile(mbuf[q & 1], mtile(ci), abuf[q & 1], addslice(ci), &bar_m[q & 1]);
+    load_mtile(mbuf[q & 1], mtile(ci), xbuf[q & 1], xsrc(ci), (uint32_t)S::XB, &bar_m[q & 1]);
+  };
+  auto prefetch_do = [&](int q) {  // every thread
+    if constexpr (REVERSE) {
+      const ChunkRec ch = t.chunks[chunk_at(q)];
+      load_do_slice<Tin>(dobuf[q & 1], dobuf[q & 1] + S::dOB, d_o, ch, H, h, j0);
+    }
   };
   // initial value: forward -> initial / imported state; reverse -> gradient of the final state
   {
@@ -119,6 +174,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       for (int j = 0; j < 32; ++j) s[j] = 0.f;
   }
   if (c == 0) prefetch(0);
+  prefetch_do(0);
   uint32_t mma_phase = 0;
   bool ok = true;
   for (int q = 0; q < nch && ok; ++q) {
@@ -136,14 +192,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       }
     }
     put_state(sth, stl, c, s);
+    if constexpr (REVERSE && EX) tc::cp_async_wait<0>();  // this chunk's dO slice (issued a step ago)
     if (c == 0 && q + 1 < nch) prefetch(q + 1);
+    if (q + 1 < nch) prefetch_do(q + 1);
     ok = wait_all(&bar_m[q & 1], (q >> 1) & 1, ws.status);
     if (!ok) break;
-    float add[32];  // B (forward) or X (reverse) of this chunk, row c of the slice
+    float add[32];  // forward: B of this chunk, row c of the slice
+    if constexpr (!REVERSE) {
+      const float* ab = reinterpret_cast<const float*>(xbuf[q & 1]);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 u = reinterpret_cast<const float4*>(abuf[q & 1] + c * DVT)[i];
-      add[4 * i] = u.x; add[4 * i + 1] = u.y; add[4 * i + 2] = u.z; add[4 * i + 3] = u.w;
+      for (int i = 0; i < 8; ++i) {
+        const float4 u = reinterpret_cast<const float4*>(ab + c * DVT)[i];
+        add[4 * i] = u.x; add[4 * i + 1] = u.y; add[4 * i + 2] = u.z; add[4 * i + 3] = u.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) add[j] = 0.f;
     }
     tc::fence_async_smem();
     tc::fence_before_sync();
@@ -160,6 +224,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       const tc::Op mH{tc::smem_u32(mbuf[q & 1]), D, REVERSE}, mL{tc::smem_u32(mbuf[q & 1] + kMtileBytes / 2), D, REVERSE};
       const tc::Op sH{tc::smem_u32(sth), D, true}, sL{tc::smem_u32(stl), D, true};
       mma4(tb, mH, mL, sH, sL, D, tc::idesc_bf16(D, DVT, REVERSE, true), false, false, false);
+      if constexpr (REVERSE) {  // + Qeff^T dO (A: the Qeff tile read MN-major, k = chunk row)
+        const tc::Op eH{tc::smem_u32(xbuf[q & 1]), C, true}, eL{tc::smem_u32(xbuf[q & 1] + S::XB / 2), C, true};
+        const tc::Op oH{tc::smem_u32(dobuf[q & 1]), C, true}, oL{tc::smem_u32(dobuf[q & 1] + S::dOB), C, true};
+        mma4(tb, eH, eL, oH, oL, C, tc::idesc_bf16(D, DVT, true, true), true, false, EX);
+      }
       tc::commit(&bar_mma);
     }
     ok = wait_all(&bar_mma, mma_phase, ws.status);
@@ -187,6 +256,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     // give copies still in flight a last bounded chance before the shared memory is released
     tc::mbar_wait(&bar_m[0], 0, 200000000ull);
   }
+  if constexpr (REVERSE && EX) tc::cp_async_wait<0>();
   if (c == 0) tc::bulk_wait_all();
   tc::fence_before_sync();
   __syncthreads();

@@ -639,17 +639,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // --------------------------------------------------------------------------------- forward output
 // per (chunk, head), with the chunk-start state S0 from the scan:
-//   U = U' - W S0 (written back for the backward),  P = lower_incl(gated(q, k)),  O = Qbar S0 + P U
+//   U = U' - W S0 (written back for the backward),  P = lower_incl(gated(q, k)),  O = Qbar S0 + P U,
+//   and for the reverse scan Qeff = Qbar - P W (so that O = Qeff S0 + P U' and the state-independent
+//   part of the reverse step is Qeff^T dO); Qeff is stored where W was (the backward recomputes W)
 struct OutTcSmem {
   static constexpr int C = kTcC, D = kTcD, LD = D + 1;
   static constexpr size_t G = 0;
   static constexpr size_t vec = G + sizeof(float) * C * LD;  // ref[D]
   static constexpr size_t tiles = (vec + sizeof(float) * D + 1023) & ~size_t(1023);
   static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2, DDb = size_t(D) * D * 2;
-  // R (4 CDb): run 1 qf + bf; run 2 P (2 CCb) + U (2 CDb).  Wq (2 CDb): run 1 W, run 2 Qbar.
+  // R (4 CDb): run 1 qf + bf; run 2 P (2 CCb) + U (2 CDb).  Wq (2 CDb): W.  Qb (2 CDb): Qbar.
   static constexpr size_t R = tiles;
   static constexpr size_t Wq = R + 4 * CDb;
-  static constexpr size_t S0 = Wq + 2 * CDb;    // S0 hi/lo (D x D, MN-major)
+  static constexpr size_t Qb = Wq + 2 * CDb;
+  static constexpr size_t S0 = Qb + 2 * CDb;    // S0 hi/lo (D x D, MN-major); then the Qeff tile
   static constexpr size_t total = S0 + 2 * DDb;
 };
 
@@ -693,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Sync sy{&bar, 0u, ws.status};
   auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  // TMEM: P [0,64), W S0 [64,192), O [192,320)
+  // TMEM: P [0,64), W S0 [64,192), O [192,320), P W [320,448)
   uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
   uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb;
   build_tile_ld<C, D, true, Tin>(qfh, qfl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
@@ -708,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma4(tb + 64, wH, wL, sH, sL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
   });
   uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
-  uint8_t *qbh = wh, *qbl = wl;
+  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb;
   if (ok) {
     acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
       float m[16];
@@ -730,8 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const tc::Op qH{tc::smem_u32(qbh), C, false}, qL{tc::smem_u32(qbl), C, false};
       const tc::Op pH{tc::smem_u32(ph), C, false}, pL{tc::smem_u32(pl), C, false};
       const tc::Op uH{tc::smem_u32(uh), C, true}, uL{tc::smem_u32(ul), C, true};
+      const tc::Op wH{tc::smem_u32(wh), C, true}, wL{tc::smem_u32(wl), C, true};  // W as B (k = i, n = c)
       mma4(tb + 192, qH, qL, sH, sL, D, id, false, false, false);
       mma4(tb + 192, pH, pL, uH, uL, C, id, true, false, false);
+      mma4(tb + 320, pH, pL, wH, wL, C, id, false, false, false);
     });
     if (ok) {
       acc_read<C, D>(tb, 192, [&](int r, int j0, const float* v) {
@@ -740,6 +745,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 16; ++j) dst[j] = from_f<Tout>(v[j]);
         }
       });
+      // Qeff = Qbar - P W (element (r, c)) into the S0 buffer, which the products above consumed
+      uint8_t *eh = s0h, *el = s0h + S::CDb;
+      acc_read<C, D>(tb, 320, [&](int r, int c0, const float* v) {
+        float e[16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t off = cm_off(r, c0 + 8 * half, C);
+          const uint4 hq = *reinterpret_cast<const uint4*>(qbh + off), lq = *reinterpret_cast<const uint4*>(qbl + off);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
+          const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lq);
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            const float2 a = __bfloat1622float2(h2[k2]), b = __bfloat1622float2(l2[k2]);
+            e[8 * half + 2 * k2] = (a.x + b.x) - v[8 * half + 2 * k2];
+            e[8 * half + 2 * k2 + 1] = (a.y + b.y) - v[8 * half + 2 * k2 + 1];
+          }
+        }
+        put16<C, true>(eh, el, r, c0, e);
+      });
+      tc::fence_async_smem();
+      __syncthreads();
+      if (tid == 0) store_cd_tile(ws.W, base, eh, el);
     }
   }
   if (tid == 0) tc::bulk_wait_all();
@@ -855,7 +882,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // --------------------------------------------------------------------------------- backward dq
-// per (chunk, head), with S0 (chunk start state), dS (gradient of the chunk end state) and U:
+// per (chunk, head), with S0 (chunk start state), dS (gradient of the chunk end state), U and P:
+//   dU = P^T dO + Khat dS                                   (for the dk / dv kernel)
 //   dP = lower_incl(dO U^T), Tq = dO S0^T, T1 = U dS^T,
 //   RS = dP bf (bf = k e^{G_0 - G}),  CS = dP^T qf (qf = q e^{G - G_0})
 //   dq  = e^G Tq + e^{G - G_0} RS                         (final)
@@ -869,8 +897,10 @@ struct BdqTcSmem {
   static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2, DDb = size_t(D) * D * 2;
   // phase 1: dO (K-major) | U (K-major) | S0 (K-major D x D); phase 2: dS in the S0 slot;
   // phase 3: dP | bf (MN) | qf (MN) over the dO/U/S0 space; epilogue row buffer (C x LD fp32) after.
+  // Pt: the forward's P tile (element (r, i)), read as P^T for dU = P^T dO + Khat dS.
   static constexpr size_t R = tiles;
-  static constexpr size_t total = R + 4 * CDb + 2 * DDb;
+  static constexpr size_t Pt = R + 4 * CDb + 2 * DDb;
+  static constexpr size_t total = Pt + 2 * CCb;
 };
 
 template <typename Tin, typename Tout>
@@ -902,9 +932,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bar, 1);
     tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    ld_expect(ld, kStateTileBytes + kCDTileBytes);
+    ld_expect(ld, kStateTileBytes + kCDTileBytes + kCCTileBytes);
     ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
     ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
+    ld_cc_tile(ld, tsm + S::Pt, tsm + S::Pt + S::CCb, ws.Pm, base);  // P, as the output kernel left it
   }
   __syncthreads();
   load_gate(sG, LD, g_, srow, H, h, n);
@@ -928,6 +959,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool ok = ld_wait(ld);
   ok = ok && run(sy, [&] {
     mma4(tb + cCS, oH, oL, uH, uL, D, tc::idesc_bf16(C, C, false, false), false, EX, false);   // dP (raw)
+    {  // dU = P^T dO, accumulated further in phase 2 (P^T: the P tile read MN-major; dO read MN-major)
+      const tc::Op pH{tc::smem_u32(tsm + S::Pt), C, true}, pL{tc::smem_u32(tsm + S::Pt + S::CCb), C, true};
+      const tc::Op dH{tc::smem_u32(doh), C, true}, dL{tc::smem_u32(dol), C, true};
+      mma4(tb + cRS, pH, pL, dH, dL, C, tc::idesc_bf16(C, D, true, true), false, false, EX);
+    }
     mma4(tb + cTq, oH, oL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, EX, false);  // Tq
   });
   if (ok) {
@@ -944,20 +980,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
       const tc::Op kH{tc::smem_u32(doh), C, false}, kL{tc::smem_u32(dol), C, false};
       const tc::Op dH{tc::smem_u32(sh), D, true}, dL{tc::smem_u32(sl), D, true};
-      mma4(tb + cRS, kH, kL, dH, dL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
+      mma4(tb + cRS, kH, kL, dH, dL, D, tc::idesc_bf16(C, D, false, true), true, false, false);
     });
     if (ok) {
       // dU = dU0 + Khat dS as a hi/lo tile (element (i, j) at cm_off(i, j, C), in the consumed Khat
       // slot) for the dk / dv kernel
-      const float* dUg = ws.dU + base * C * D;
-      acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) {
-        float u[16];
-        for (int j = 0; j < 16; j += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(dUg + i * D + j0 + j);
-          u[j] = a.x + v[j]; u[j + 1] = a.y + v[j + 1]; u[j + 2] = a.z + v[j + 2]; u[j + 3] = a.w + v[j + 3];
-        }
-        put16<C, true>(doh, dol, i, j0, u);
-      });
+      acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) { put16<C, true>(doh, dol, i, j0, v); });
       tc::fence_async_smem();
       __syncthreads();
       if (tid == 0) {

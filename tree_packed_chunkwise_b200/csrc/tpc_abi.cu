@@ -229,7 +229,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     // stream after prep(r) and scan(r - 1).  The caller's stream runs prep(1..R), out(1..R) in that
     // order, so the later rounds' prep overlaps scan(1) and out(r) overlaps scan(r + 1).
     TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmem::total));
-    TPC_CUDA(set_smem(kda_scan_tc<false>, ScanTcSmem::total));
+    TPC_CUDA(set_smem(kda_scan_tc<false, Tin>, ScanTcSmemT<false>::total));
     TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
     cudaStream_t hs = scan_stream();
     if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
@@ -243,8 +243,9 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
       if (s1 > s0)
         TPC_LAUNCH("kda_fwd_scan_tc", hs,
-                   (kda_scan_tc<false><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, hs>>>(
-                       p.dt, s0, H, io->init_state, io->final_state, nullptr, w)));
+                   (kda_scan_tc<false, Tin><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads,
+                                              ScanTcSmemT<false>::total, hs>>>(p.dt, s0, H, io->init_state,
+                                                                              io->final_state, nullptr, w, nullptr)));
       scans.emplace_back();
       TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
@@ -295,28 +296,21 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
   // tensor-core or exact CUDA-core path, as in forward_impl
   std::vector<cudaEvent_t> scans;
   if constexpr (TC) {
-    // Rounds in reverse: prep(r) on the caller's stream; the reverse scan(r) on the high-priority
-    // scan stream after prep(r) and scan(r + 1); then dq(r), dk/dv(r) on the caller's stream after
-    // scan(r).  The caller's stream runs prep(R..1), then dq / dk-dv(R..1), so the earlier rounds'
-    // prep overlaps scan(R) and dq / dk-dv(r) overlap scan(r - 1).
-    TPC_CUDA(set_smem(kda_bwd_prep_tc<Tin>, BprepTcSmem::total));
-    TPC_CUDA(set_smem(kda_scan_tc<true>, ScanTcSmem::total));
+    // Rounds in reverse: the reverse scan(r) (which also forms the output's contribution Qeff^T dO)
+    // on the high-priority scan stream after the caller's prior work and scan(r + 1); then dq(r),
+    // dk/dv(r) on the caller's stream after scan(r), so dq / dk-dv(r) overlap scan(r - 1).
+    TPC_CUDA(set_smem(kda_scan_tc<true, Tin>, ScanTcSmemT<true>::total));
     TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
     TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmemT<Tin>::total));
     cudaStream_t hs = scan_stream();
     if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
+    TPC_TRY_ABI(stream_after(hs, st));  // the scans after the caller's prior work (forward, d_o)
     for (int r = p.n_rounds; r >= 1; --r) {
-      const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-      if (c1 > c0)
-        TPC_LAUNCH("kda_bwd_prep_tc", st,
-                   (kda_bwd_prep_tc<Tin><<<dim3(c1 - c0, H), kThreads, BprepTcSmem::total, st>>>(p.dt, H, q, k, g, dO,
-                                                                                                   w, c0)));
-      TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
       if (s1 > s0)
         TPC_LAUNCH("kda_bwd_scan_tc", hs,
-                   (kda_scan_tc<true><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmem::total, hs>>>(
-                       p.dt, s0, H, nullptr, nullptr, io->d_final, w)));
+                   (kda_scan_tc<true, Tin><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmemT<true>::total,
+                                             hs>>>(p.dt, s0, H, nullptr, nullptr, io->d_final, w, dO)));
       scans.emplace_back();
       TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
