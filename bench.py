@@ -202,6 +202,17 @@ def oracle_sample(w, n_tokens, seed):
     return time.perf_counter() - t0, len(rows)
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -429,6 +440,135 @@ def measure_wide(args, world, rank, tpc, torch, peaks):
                          "peak_source": "bf16 sustained, " + peaks["source"]}}
 
 
+# ------------------------------------------------------------------------------------ agentic tree (config 2)
+def kda_step_timer(tpc, torch, plan, x, H, d, world, steps, warmup):
+    """ms per tree-packed forward + backward (bf16 in / out, fp32 state) of one plan, device-timed."""
+    bf = torch.bfloat16
+    info = plan.info
+    N = info["n_unique"]
+    shape = tpc.kda_shape(H, d, tpc.TPC_BF16, tpc.TPC_BF16)
+    ws = tpc.alloc_workspace(plan, shape)
+    o = torch.empty(N, H, d, dtype=bf, device="cuda")
+    fin = torch.empty(info["n_leaves"], H, d, d, dtype=torch.float32, device="cuda")
+    gr = dict(dq=torch.empty(N, H, d, dtype=bf, device="cuda"), dk=torch.empty(N, H, d, dtype=bf, device="cuda"),
+              dv=torch.empty(N, H, d, dtype=bf, device="cuda"),
+              dg=torch.empty(N, H, d, dtype=torch.float32, device="cuda"),
+              dbeta=torch.empty(N, H, dtype=torch.float32, device="cuda"), d_init=None)
+
+    def step():
+        tpc.tpc_kda_forward(plan, x["q"], x["k"], x["v"], x["g"], x["beta"], ws=ws, o=o, final_state=fin, out_dtype=bf)
+        tpc.tpc_kda_backward(plan, ws, x["q"], x["k"], x["v"], x["g"], x["beta"], x["d_o"], x["d_final"],
+                             out_dtype=bf, grads=gr)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    tpc.tpc_status(plan, ws, H, d)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    del ws
+    return ms
+
+
+def measure_agentic(args, world, rank, tpc, torch):
+    """Config 2: the agentic tree (64 leaves, 5 fork levels, bounded replay), tree-packed forward +
+    backward against the trajectory-expanded run of the same kernels; the planner's rounds; the two
+    planner ablations (node-wise, no replay); a sharing window (producer + consumer microbatches)."""
+    import synth.gpu as sgpu
+    w = synth.workload("agentic")
+    t = w.tree
+    H, d = w.H, w.dk
+    seed = w.seed + 1000 * rank
+    out = {"workload": w.name}
+    st = t.node_start()
+    K, W = max(2, args.steps // 4), max(3, args.warmup)
+    for mode, name in ((tpc.PLAN_MIN_ROUNDS, "tree"), (tpc.PLAN_NODEWISE, "nodewise"), (tpc.PLAN_NO_REPLAY, "noreplay")):
+        plan = tpc.Plan(t.parent, t.length, 64, mode).upload()
+        info = plan.info
+        src = torch.tensor(plan.compact_source_rows(st, t.length), dtype=torch.int32, device="cuda")
+        x = dict(zip(("q", "k", "v", "g", "beta"), sgpu.kda_inputs(seed, src, H, d, d, "bf16")))
+        x["d_o"] = sgpu.normal_rows(seed, synth.STREAM["d_o"], src, H * d, "bf16").view(-1, H, d)
+        x["d_final"] = sgpu.normal_rows(seed, synth.STREAM["d_final"], None, H * d * d, "f32",
+                                        shape=(info["n_leaves"],)).view(info["n_leaves"], H, d, d)
+        ms = kda_step_timer(tpc, torch, plan, x, H, d, world, K, W)
+        rec = {"rounds": info["n_rounds"], "replay_rows": info["replay_total"], "chunks": info["n_chunks"],
+               "sequences": info["n_seqs"], "ms_per_step": ms,
+               "unique_tokens_per_s": world * info["n_unique"] / (ms / 1e3),
+               "expanded_tokens_per_s": world * info["n_expanded"] / (ms / 1e3)}
+        if name == "tree":
+            out.update(n_unique=info["n_unique"], n_expanded=info["n_expanded"], **rec)
+            # trajectory-expanded comparator: the same kernels, one sequence per trajectory
+            tb = plan.tables()
+            lens = np.diff(tb["traj_offset"]).astype(np.int32)
+            eplan = tpc.Plan(np.full(len(lens), -1, np.int32), lens, 64).upload()
+            xe = {k: tpc.tpc_gather_expanded(plan, x[k]) for k in ("q", "k", "v", "g", "beta", "d_o")}
+            xe["d_final"] = x["d_final"]
+            del x
+            ems = kda_step_timer(tpc, torch, eplan, xe, H, d, world, 2, 2)
+            out["expanded_path"] = {"ms_per_step": ems, "speedup_tree_vs_expanded": ems / ms,
+                                    "target_speedup": info["n_expanded"] / info["n_seq_tokens"],
+                                    "expanded_chunks": eplan.info["n_chunks"]}
+            del xe
+        else:
+            out[name] = rec
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_extras(args, world, rank, tpc, torch):
+    """The L1 microbatch planner on a step of many trees, and compact MoE routing on the wide tree."""
+    import synth.gpu as sgpu
+    res = {}
+    trees = [synth.agentic_tree(seed=s) for s in range(100, 132)]
+    parent, length = [], []
+    for tr in trees:
+        base = len(parent)
+        parent += [(-1 if p < 0 else base + int(p)) for p in tr.parent]
+        length += list(tr.length)
+    parent, length = np.array(parent, np.int32), np.array(length, np.int32)
+    budget = 262144
+    t0 = time.perf_counter()
+    leaf_mb, mu, me, stats = tpc.tpc_microbatch_plan(parent, length, budget)
+    dt = time.perf_counter() - t0
+    whole = float(sum(int(tr.n_expanded()) for tr in trees)) / float(length.sum())
+    res["microbatch_l1"] = {"trees": len(trees), "trajectories": int(len(leaf_mb)), "budget_unique_rows": budget,
+                            "microbatches": stats["n_microbatches"], "compression": stats["compression"],
+                            "compression_whole_trees": whole, "balance": stats["balance"], "plan_ms": dt * 1e3}
+    w = synth.workload("wide")
+    t = w.tree
+    plan = tpc.Plan(t.parent, t.length, 64).upload()
+    src = torch.tensor(plan.compact_source_rows(t.node_start(), t.length), dtype=torch.int32, device="cuda")
+    Dh, E, k = 2048, 64, 2
+    h = sgpu.normal_rows(41, synth.STREAM["h"], src, Dh, "bf16")
+    wr = sgpu.normal_rows(41, synth.STREAM["w_vocab"], None, Dh, "bf16", 0.02, shape=(E,))
+    routed = tpc.tpc_moe_route(plan, h, wr, k)
+    tpc.tpc_moe_router_loss(plan, routed, k)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        routed = tpc.tpc_moe_route(plan, h, wr, k, scratch=routed["scratch"])
+        tpc.tpc_moe_router_loss(plan, routed, k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 3
+    res["moe_routing"] = {"workload": w.name, "hidden": Dh, "experts": E, "top_k": k,
+                          "unique_rows": plan.info["n_unique"], "positions": plan.info["n_expanded"],
+                          "ms_route_and_loss": ms, "rows_per_s": plan.info["n_unique"] / (ms / 1e3),
+                          "load_sum_equals_k_positions": int(routed["expert_load"].sum().item()) == k * plan.info["n_expanded"]}
+    return res
+
+
 # ------------------------------------------------------------------------------------ GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -447,6 +587,8 @@ def main():
     ap.add_argument("--no-wide", action="store_true", help="skip the wide tree with log-prob recovery")
     ap.add_argument("--wide-steps", type=int, default=2)
     ap.add_argument("--workload", default=WORKLOAD, help="single_fork (default), agentic, agentic_small")
+    ap.add_argument("--no-agentic", action="store_true", help="skip the agentic tree (config 2) and its ablations")
+    ap.add_argument("--no-extras", action="store_true", help="skip the L1 microbatch planner and MoE routing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "tpc" else args.warmup
 
@@ -662,10 +804,16 @@ def main():
                       "spans all copies"}
         del sets, res
 
+    # ---- the agentic tree (config 2), its planner ablations; L1 planner and MoE routing
+    del wsb, outs, grads, dev
+    torch.cuda.empty_cache()
+    agentic = None if args.no_agentic else measure_agentic(args, world, rank, tpc, torch)
+    extras = None if args.no_extras else measure_extras(args, world, rank, tpc, torch)
+    torch.cuda.empty_cache()
+
     # ---- hybrid layer group on the agentic tree (KDA buffers released first)
     group = None
     if not args.no_group:
-        del wsb, outs, grads, dev
         torch.cuda.empty_cache()
         group = measure_group(args, world, rank, tpc, torch, peaks)
         torch.cuda.empty_cache()
@@ -673,8 +821,6 @@ def main():
     # ---- wide tree: KDA (H = 32) and log-probability recovery
     wide = None
     if not args.no_wide:
-        if args.no_group:
-            del wsb, outs, grads, dev
         torch.cuda.empty_cache()
         wide = measure_wide(args, world, rank, tpc, torch, peaks)
         torch.cuda.empty_cache()
@@ -683,7 +829,15 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, n = oracle_sample(w, args.cpu_tokens, seed)
+        try:  # the same oracle with its BLAS pool held to one thread
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                dt1, n1 = oracle_sample(w, max(64, args.cpu_tokens // 4), seed)
+            one = n1 / dt1
+        except Exception:
+            one = None
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "cpu_model": cpu_model(), "host_cpus": os.cpu_count(), "value_one_thread": one,
                "sample": f"first {n} tokens of trajectory 0 (H={H}, d={d}) fwd+bwd, fp64 numpy, {dt:.1f} s"}
 
     if rank == 0:
@@ -696,7 +850,8 @@ def main():
                            "l2": "inputs+workspace > 1 GB per step, larger than L2"},
                 "value_expanded": value_exp, "roofline": roofline, "step_roofline": step_roof,
                 "kernels": kern, "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
-                "expanded_path": expanded, "hybrid_group": group, "wide_logprob": wide}
+                "expanded_path": expanded, "agentic": agentic, "hybrid_group": group, "wide_logprob": wide,
+                **(extras or {})}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
