@@ -155,6 +155,45 @@ __device__ __forceinline__ void stage_rows(T* dst, const T* src, const int* rows
   }
 }
 
+// Asynchronous copy of the chunk's rows of a bf16 input into shared memory (row pitch kStagePitch);
+// rows >= n are zero.  Completed by cp_async_wait + a barrier.
+__device__ __forceinline__ void stage_rows_async(__nv_bfloat16* dst, const __nv_bfloat16* src, const int* rows, int H,
+                                                 int h, int n) {
+  constexpr int VEC = 8, NCH = kTcC * (kTcD / VEC);
+  for (int e = threadIdx.x; e < NCH; e += blockDim.x) {
+    const int a = e / (kTcD / VEC), b0 = (e % (kTcD / VEC)) * VEC;
+    const bool in = a < n;
+    tc::cp_async16(dst + a * kStagePitch + b0, src + ((size_t)(in ? rows[a] : 0) * H + h) * kTcD + b0, in ? 16u : 0u);
+  }
+  tc::cp_async_commit();
+}
+
+// A x B tile from staged bf16 rows (row a at st + a * kStagePitch), value f(a, b, x)
+template <int A, int B, bool SPLIT, class F>
+__device__ __forceinline__ void build_tile_st(uint8_t* hi, uint8_t* lo, const __nv_bfloat16* st, F f) {
+  for (int e = threadIdx.x; e < A * (B / 8); e += blockDim.x) {
+    const int a = e % A, b0 = (e / A) * 8;
+    const uint4 u = *reinterpret_cast<const uint4*>(st + a * kStagePitch + b0);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    __align__(16) __nv_bfloat16 hh[8];
+    __align__(16) __nv_bfloat16 ll[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 x = __bfloat1622float2(b2[j]);
+      const float y0 = f(a, b0 + 2 * j, x.x), y1 = f(a, b0 + 2 * j + 1, x.y);
+      if (SPLIT) {
+        split_bf16(y0, hh[2 * j], ll[2 * j]);
+        split_bf16(y1, hh[2 * j + 1], ll[2 * j + 1]);
+      } else {
+        hh[2 * j] = __float2bfloat16_rn(y0);
+        hh[2 * j + 1] = __float2bfloat16_rn(y1);
+      }
+    }
+    *reinterpret_cast<uint4*>(hi + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(hh);
+    if (SPLIT) *reinterpret_cast<uint4*>(lo + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(ll);
+  }
+}
+
 // 16 consecutive values of a staged row as fp32
 template <typename T>
 __device__ __forceinline__ void staged16(const T* st, int r, int c0, float (&v)[16]) {
@@ -493,7 +532,8 @@ __device__ __forceinline__ float ld_in(const T* base, const int* rows, int H, in
 // --------------------------------------------------------------------------------- forward prep
 // per (chunk, head): Atilde = gated(k, k) (strict lower), T = (I + diag(beta) Atilde)^{-1},
 // W = T diag(beta) Kbar, U' = T diag(beta) V, Khat = k e^{G_C - G}, decay = e^{G_C}.
-struct PrepTcSmem {
+template <typename Tin>
+struct PrepTcSmemT {
   static constexpr int C = kTcC, D = kTcD, LD = D + 1, LC = C + 1;
   static constexpr size_t G = 0;
   static constexpr size_t A = G + sizeof(float) * C * LD;
@@ -504,7 +544,11 @@ struct PrepTcSmem {
   static constexpr size_t tiles = (vec + sizeof(float) * (C + 2 * D) + 1023) & ~size_t(1023);
   // phase 1: af hi/lo, bf hi/lo (C x D each); phase 2: T' hi/lo (C x C), Kbar hi/lo, V hi/lo (C x D)
   static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2;
-  static constexpr size_t total = tiles + 6 * CDb;  // phase 3: W, U' (MN) and Khat (MN) hi/lo
+  // bf16 inputs: the chunk's k and v rows staged once (pitch kStagePitch)
+  static constexpr size_t Stage = tiles + 6 * CDb;  // phase 3: W, U' (MN) and Khat (MN) hi/lo
+  static constexpr size_t StB = sizeof(Tin) == 2 ? size_t(C) * tck::kStagePitch * 2 : 0;
+  static constexpr size_t total = Stage + 2 * StB;
+  static_assert(total <= 227 * 1024, "shared memory");
 };
 
 template <typename Tin>
@@ -512,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     kda_fwd_prep_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
                     const Tin* __restrict__ g_, const Tin* __restrict__ beta_, KdaWs ws, int chunk0 = 0) {
   using namespace tck;
-  using S = PrepTcSmem;
+  using S = PrepTcSmemT<Tin>;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
   const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
@@ -540,22 +584,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // bf16: the chunk's k and v rows into shared memory while the gates load and accumulate
+  [[maybe_unused]] __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
+  [[maybe_unused]] __nv_bfloat16* sv = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
+  if constexpr (EX) {
+    stage_rows_async(sk, k_, srow, H, h, n);
+    stage_rows_async(sv, v_, srow, H, h, n);
+  }
   for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, ws.status);
+  if constexpr (EX) tc::cp_async_wait<0>();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  // a C x D tile of k (or v) transformed by f, from the staged rows (bf16) or from global memory
+  auto k_tile = [&](uint8_t* hi, uint8_t* lo, auto f) {
+    if constexpr (EX) build_tile_st<C, D, true>(hi, lo, sk, f);
+    else build_tile_ld<C, D, true, Tin>(hi, lo, row_k, f);
+  };
   bool ok = true;
   // phase 1: Atilde = af bf^T with af = k e^{G - ref}, bf = k e^{ref - G}
   {
     uint8_t *afh = tl, *afl = tl + S::CDb, *bfh = tl + 2 * S::CDb, *bfl = tl + 3 * S::CDb;
-    build_tile_ld<C, D, true, Tin>(afh, afl, row_k, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
-    build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
+    k_tile(afh, afl, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
+    k_tile(bfh, bfl, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
     const tc::Op ah{tc::smem_u32(afh), C, false}, al{tc::smem_u32(afl), C, false};
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
     ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
@@ -583,8 +640,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
             *vl = vh + S::CDb;
     build_tile<C, C, true>(th, tlo, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
-    build_tile_ld<C, D, true, Tin>(kh, kl, row_k, [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); });
-    build_tile_ld<C, D, !EX, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
+    k_tile(kh, kl, [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); });
+    if constexpr (EX) build_tile_st<C, D, false>(vh, vl, sv, [&](int, int, float x) { return x; });
+    else build_tile_ld<C, D, true, Tin>(vh, vl, row_v, [&](int, int, float x) { return x; });
     const tc::Op tH{tc::smem_u32(th), C, false}, tL{tc::smem_u32(tlo), C, false};
     const tc::Op kH{tc::smem_u32(kh), C, true}, kL{tc::smem_u32(kl), C, true};
     const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
@@ -604,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) { put16<C, true>(wth, wtl, r, c0, v); });
       acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) { put16<C, true>(uth, utl, r, c0, v); });
       const float* gC = sG + (n - 1) * LD;
-      build_tile_ld<C, D, true, Tin>(khh, khl, row_k, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
+      k_tile(khh, khl, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
       ok = run(sy, [&] {
         store_cd_tile(ws.W, base, wth, wtl);
         store_cd_tile(ws.U, base, uth, utl);
@@ -900,7 +958,10 @@ struct BdqTcSmem {
   // Pt: the forward's P tile (element (r, i)), read as P^T for dU = P^T dO + Khat dS.
   static constexpr size_t R = tiles;
   static constexpr size_t Pt = R + 4 * CDb + 2 * DDb;
-  static constexpr size_t total = Pt + 2 * CCb;
+  static constexpr size_t Stage = Pt + 2 * CCb;  // bf16 inputs: the chunk's q and k rows (pitch kStagePitch)
+  static constexpr size_t StB = size_t(C) * tck::kStagePitch * 2;
+  static constexpr size_t total = Stage + 2 * StB;
+  static_assert(total <= 227 * 1024, "shared memory");
 };
 
 template <typename Tin, typename Tout>
@@ -938,9 +999,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     ld_cc_tile(ld, tsm + S::Pt, tsm + S::Pt + S::CCb, ws.Pm, base);  // P, as the output kernel left it
   }
   __syncthreads();
+  // bf16: the chunk's q and k rows into shared memory while the gates load and accumulate
+  [[maybe_unused]] __nv_bfloat16* stq = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
+  [[maybe_unused]] __nv_bfloat16* stk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
+  if constexpr (EX) {
+    stage_rows_async(stq, q_, srow, H, h, n);
+    stage_rows_async(stk, k_, srow, H, h, n);
+  }
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
+  if constexpr (EX) tc::cp_async_wait<0>();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
@@ -974,7 +1043,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ld_state_tile(ld, sh, sl, ws.dS, base);
     }
     const float* gC = sG + (n - 1) * LD;
-    build_tile_ld<C, D, true, Tin>(doh, dol, row_k, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
+    auto khf = [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); };
+    if constexpr (EX) build_tile_st<C, D, true>(doh, dol, stk, khf);
+    else build_tile_ld<C, D, true, Tin>(doh, dol, row_k, khf);
     ok = ld_wait(ld);
     ok = ok && run(sy, [&] {
       mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
@@ -1003,8 +1074,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
       put16<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
     });
-    build_tile_ld<C, D, true, Tin>(bh, bl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
-    build_tile_ld<C, D, true, Tin>(qh, ql, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
+    auto bff = [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); };
+    auto qff = [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); };
+    if constexpr (EX) {
+      build_tile_st<C, D, true>(bh, bl, stk, bff);
+      build_tile_st<C, D, true>(qh, ql, stq, qff);
+    } else {
+      build_tile_ld<C, D, true, Tin>(bh, bl, row_k, bff);
+      build_tile_ld<C, D, true, Tin>(qh, ql, row_q, qff);
+    }
     ok = run(sy, [&] {
       const uint32_t id = tc::idesc_bf16(C, D, false, true), idT = tc::idesc_bf16(C, D, true, true);
       const tc::Op pK{tc::smem_u32(pH8), C, false}, pKl{tc::smem_u32(pL8), C, false};  // dP (r, i), K-major
@@ -1021,8 +1099,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* sbuf = reinterpret_cast<float*>(tsm + S::R);  // [C][LD]: k e^{G_C - G} T1 per row
     Tin* sq = reinterpret_cast<Tin*>(tsm + S::R + sizeof(float) * C * LD);
     Tin* sk = sq + C * kStagePitch;
-    stage_rows(sq, q_, srow, H, h, n);
-    stage_rows(sk, k_, srow, H, h, n);
+    if constexpr (EX) {  // staged at the start
+      sq = reinterpret_cast<Tin*>(stq);
+      sk = reinterpret_cast<Tin*>(stk);
+    } else {
+      stage_rows(sq, q_, srow, H, h, n);
+      stage_rows(sk, k_, srow, H, h, n);
+    }
     __syncthreads();
     const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
     const int r = lane < 16 ? 16 * sp + lane : -1;
@@ -1140,10 +1223,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
   for (int e = tid; e < 6 * C; e += blockDim.x) sdb[e] = 0.f;
   Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
-  if constexpr (S::kStageK) stage_rows(sk, k_, srow, H, h, n);
+  if constexpr (S::kStageK) stage_rows_async(reinterpret_cast<__nv_bfloat16*>(sk), reinterpret_cast<const __nv_bfloat16*>(k_), srow, H, h, n);
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
+  if constexpr (S::kStageK) tc::cp_async_wait<0>();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
@@ -1201,7 +1285,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             *vl = vh + S::CDb;
     build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
     build_tile<C, C, true>(tTh, tTl, [&](int r, int i) { return sT[r * LC + i]; });
-    build_tile_ld<C, D, true, Tin>(kbh, kbl, row_k, [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); });
+    auto kbf = [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); };
+    if constexpr (S::kStageK) build_tile_st<C, D, true>(kbh, kbl, reinterpret_cast<const __nv_bfloat16*>(sk), kbf);
+    else build_tile_ld<C, D, true, Tin>(kbh, kbl, row_k, kbf);
     build_tile_ld<C, D, !EX, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
     ok = run(sy, [&] {
       const uint32_t id = tc::idesc_bf16(C, D, false, true);
@@ -1331,8 +1417,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
     uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
-    build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
-    build_tile_ld<C, D, true, Tin>(afh, afl, row_k, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
+    auto bff = [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); };
+    auto aff = [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); };
+    if constexpr (S::kStageK) {
+      build_tile_st<C, D, true>(bfh, bfl, reinterpret_cast<const __nv_bfloat16*>(sk), bff);
+      build_tile_st<C, D, true>(afh, afl, reinterpret_cast<const __nv_bfloat16*>(sk), aff);
+    } else {
+      build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, bff);
+      build_tile_ld<C, D, true, Tin>(afh, afl, row_k, aff);
+    }
     ok = run(sy, [&] {
       const tc::Op pK{tc::smem_u32(dah), C, false}, pKl{tc::smem_u32(dal), C, false};
       const tc::Op pM{tc::smem_u32(dah), C, true}, pMl{tc::smem_u32(dal), C, true};

@@ -228,7 +228,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     // Per round r: prep(r) and then out(r) on the caller's stream, scan(r) on the high-priority scan
     // stream after prep(r) and scan(r - 1).  The caller's stream runs prep(1..R), out(1..R) in that
     // order, so the later rounds' prep overlaps scan(1) and out(r) overlaps scan(r + 1).
-    TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmem::total));
+    TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmemT<Tin>::total));
     TPC_CUDA(set_smem(kda_scan_tc<false, Tin>, ScanTcSmemT<false>::total));
     TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
     cudaStream_t hs = scan_stream();
@@ -238,7 +238,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       if (c1 > c0)
         TPC_LAUNCH("kda_fwd_prep_tc", st,
-                   (kda_fwd_prep_tc<Tin><<<dim3(c1 - c0, H), kThreads, PrepTcSmem::total, st>>>(p.dt, H, k, v, g, b,
+                   (kda_fwd_prep_tc<Tin><<<dim3(c1 - c0, H), kThreads, PrepTcSmemT<Tin>::total, st>>>(p.dt, H, k, v, g, b,
                                                                                                   w, c0)));
       TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
       if (s1 > s0)
