@@ -384,7 +384,7 @@ def measure_wide(args, world, rank, tpc, torch, peaks):
     targets = torch.randint(0, V, (NE,), dtype=torch.int32, device="cuda",
                             generator=torch.Generator(device="cuda").manual_seed(seed))
     dlogp = sgpu.normal_rows(seed, synth.STREAM["d_logp"], None, 1, "f32", shape=(NE,)).view(NE)
-    scratch = tpc.logprob_scratch(V, CR)
+    scratch = tpc.logprob_scratch(plan, V, CR)
     stream = torch.cuda.current_stream()
 
     def kda_part():

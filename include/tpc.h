@@ -400,15 +400,21 @@ int tpc_rope_positions(const tpc_plan* plan, int32_t* pos, tpc_stream_t stream);
  * expanded vocabulary-sized logits).  For compact row u with hidden state h_u and output matrix
  * W [V][Dh]: z_u = W h_u, lse_u = log sum exp z_u, and for each occurrence j of u (trajectory
  * order, tpc_plan_export's expanded_rows) with target y_j: logp_j = z_u[y_j] - lse_u.
+ * No logit matrix is stored: the tensor-core GEMM's epilogue reduces each 256-column tile of z to
+ * its (max, sum of exponentials) per row, lse combines those in a fixed order, and every target
+ * logit is its own fp32 dot product W_{y_j} . h_u.
  *   h: bf16 [N_unique][Dh] (compact order), W: bf16 [V][Dh], targets: int32 [n_expanded] in [0, V).
- *   logp: fp32 [n_expanded], lse: fp32 [N_unique].  V and Dh multiples of 8.
- *   scratch: caller device memory of tpc_logprob_scratch_bytes(V, chunk_rows) bytes (256-aligned);
- *   logits exist only for chunk_rows unique rows at a time.
+ *   logp: fp32 [n_expanded], lse: fp32 [N_unique].  V and Dh multiples of 8, V < 2^31.
+ *   scratch: caller device memory of tpc_logprob_scratch_bytes(plan, V, chunk_rows) bytes
+ *   (256-aligned); the GEMMs run chunk_rows unique rows at a time.
  *   status: optional device int; a target outside [0, V) records TPC_ERR_DEVICE_CHECK.
- * Backward of sum_j dlogp_j logp_j: dh fp32 [N_unique][Dh] and dW fp32 [V][Dh] (overwritten),
- * from the forward's lse.  Deterministic (fixed chunk and occurrence order).
+ * Backward of sum_j dlogp_j logp_j: dh fp32 [N_unique][Dh] and dW fp32 [V][Dh] (overwritten), from
+ * the forward's lse.  dz_u = sum_j dlogp_j onehot(y_j) - s_u softmax(z_u) (s_u: u's weight sum):
+ * the dense part comes out of the recomputed logit tile's epilogue as bf16 and enters one
+ * tensor-core pass each of dh = dz W and dW = dz^T h; the one-hot part is added exactly in fp32
+ * (occurrences grouped by target for dW).  Deterministic (fixed chunk and occurrence order).
  */
-size_t tpc_logprob_scratch_bytes(int64_t V, int32_t chunk_rows);
+size_t tpc_logprob_scratch_bytes(const tpc_plan* plan, int64_t V, int32_t chunk_rows);
 int tpc_logprob_forward(const tpc_plan* plan, const void* h, const void* W, int64_t V, int64_t Dh,
                         const int32_t* targets, float* logp, float* lse, void* scratch, size_t scratch_bytes,
                         int32_t chunk_rows, int32_t* status, tpc_stream_t stream);

@@ -285,7 +285,7 @@ def test_wide_tree_logprob_full_size_sampled_rows(tpc):
     targets = torch.tensor(targets_np, device="cuda")
     dlogp = torch.tensor(dlogp_np, dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    scratch = tpc.logprob_scratch(V, CR)
+    scratch = tpc.logprob_scratch(plan, V, CR)
     logp, lse = tpc.tpc_logprob_forward(plan, h, W, targets, chunk_rows=CR, scratch=scratch, status=status)
     dh, dW = tpc.tpc_logprob_backward(plan, h, W, targets, dlogp, lse, chunk_rows=CR, scratch=scratch, status=status)
     torch.cuda.synchronize()

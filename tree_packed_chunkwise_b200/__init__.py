@@ -130,7 +130,7 @@ SIGNATURES = {
     "tpc_gemm_split": (ctypes.c_int, [_V, _V, _V, _V, _V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                       ctypes.c_int32, ctypes.c_float, ctypes.c_float, _V, _V]),
-    "tpc_logprob_scratch_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int32]),
+    "tpc_logprob_scratch_bytes": (ctypes.c_size_t, [_V, ctypes.c_int64, ctypes.c_int32]),
     "tpc_logprob_forward": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V, _V, _V, _V, ctypes.c_size_t,
                                            ctypes.c_int32, _V, _V]),
     "tpc_logprob_backward": (ctypes.c_int, [_V, _V, _V, ctypes.c_int64, ctypes.c_int64, _V, _V, _V, _V, _V, _V,
@@ -564,9 +564,9 @@ def tpc_gemm_split(a, a_lo, b, b_lo, c=None, a_mn=False, b_mn=False, alpha=1.0, 
 
 
 # ------------------------------------------------------------------------------------ log-probabilities
-def logprob_scratch(V, chunk_rows, device="cuda"):
+def logprob_scratch(plan: Plan, V, chunk_rows, device="cuda"):
     import torch
-    n = int(lib().tpc_logprob_scratch_bytes(V, chunk_rows))
+    n = int(lib().tpc_logprob_scratch_bytes(plan.handle, V, chunk_rows))
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
@@ -575,7 +575,7 @@ def tpc_logprob_forward(plan: Plan, h, W, targets, chunk_rows=2048, scratch=None
     import torch
     V, Dh = W.shape
     chunk_rows = min(chunk_rows, plan.info["n_unique"])
-    scratch = scratch if scratch is not None else logprob_scratch(V, chunk_rows, h.device)
+    scratch = scratch if scratch is not None else logprob_scratch(plan, V, chunk_rows, h.device)
     logp = torch.empty(plan.info["n_expanded"], dtype=torch.float32, device=h.device)
     lse = torch.empty(plan.info["n_unique"], dtype=torch.float32, device=h.device)
     _check(lib().tpc_logprob_forward(plan.handle, _ptr(h), _ptr(W), V, Dh, _ptr(targets), _ptr(logp), _ptr(lse),
@@ -589,7 +589,7 @@ def tpc_logprob_backward(plan: Plan, h, W, targets, dlogp, lse, chunk_rows=2048,
     import torch
     V, Dh = W.shape
     chunk_rows = min(chunk_rows, plan.info["n_unique"])
-    scratch = scratch if scratch is not None else logprob_scratch(V, chunk_rows, h.device)
+    scratch = scratch if scratch is not None else logprob_scratch(plan, V, chunk_rows, h.device)
     dh = torch.empty(plan.info["n_unique"], Dh, dtype=torch.float32, device=h.device)
     dW = torch.empty(V, Dh, dtype=torch.float32, device=h.device)
     _check(lib().tpc_logprob_backward(plan.handle, _ptr(h), _ptr(W), V, Dh, _ptr(targets), _ptr(dlogp), _ptr(lse),

@@ -49,6 +49,13 @@ struct GemmCfg {
   static constexpr size_t total = stages * stage + 1024;  // + slack to align the stages to 1024 bytes
 };
 
+// Epilogues: kEpiStore writes alpha * acc (+ beta * C); kEpiLsePart writes, per row and 256-column
+// tile, (max, sum of exp(acc - max)) over the tile's columns into C = float2 [M][ldc] at column
+// tile_n (the rows' log-sum-exp is combined from these later, the accumulator is never stored);
+// kEpiSoftmaxGrad writes bf16 -row_b[m] * exp(acc - row_a[m]) (row_a = log-sum-exp, row_b = the row's
+// gradient weight) into C = bf16 [M][ldc].
+enum : int { kEpiStore = 0, kEpiLsePart = 1, kEpiSoftmaxGrad = 2 };
+
 struct GemmArgs {
   int M, N, K;
   int a_mn, b_mn;     // 1: MN-major
@@ -59,6 +66,9 @@ struct GemmArgs {
   int* status;
   int passes;         // 1: A B;  2: + A_lo B;  3: + A B_lo
   int m_fast;         // tile order: 1 = M blocks fastest (concurrent CTAs share B), 0 = N blocks fastest
+  int epi;            // kEpi*
+  const float* row_a; // per-row inputs of kEpiSoftmaxGrad (indexed by the GEMM row)
+  const float* row_b;
 };
 
 // Persistent, warp-specialised: grid = min(tiles, SMs); each CTA walks tiles blockIdx.x,
@@ -204,6 +214,42 @@ __global__ void __launch_bounds__(kGemmThreadsP, 1)
       for (int half = 0; half < HV; ++half) {
         const int m = tile_m(t) * kGemmBM + kGemmHalf * half + row;
         const uint32_t la = tb + ((uint32_t)(32 * sp) << 16) + (uint32_t)((b + half) * kGemmBN);
+        if (g.epi == kEpiLsePart) {  // running max and sum of exponentials over the tile's columns
+          float mx = -INFINITY, sm = 0.f;
+          for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+            float v[16];
+            tmem_ld16(la + c0, v);
+            const int nn = min(16, g.N - (n0 + c0));
+            float lm = mx;
+            for (int j = 0; j < nn; ++j) lm = fmaxf(lm, v[j]);
+            if (nn > 0 && lm > -INFINITY) {
+              sm *= expf(mx - lm);
+              for (int j = 0; j < nn; ++j) sm += expf(v[j] - lm);
+              mx = lm;
+            }
+          }
+          if (m < g.M) reinterpret_cast<float2*>(g.C)[(size_t)m * g.ldc + tile_n(t)] = make_float2(mx, sm);
+          continue;
+        }
+        if (g.epi == kEpiSoftmaxGrad) {  // dense part of the log-softmax gradient, as bf16
+          const float ra = m < g.M ? g.row_a[m] : 0.f, rb = m < g.M ? g.row_b[m] : 0.f;
+          for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+            float v[16];
+            tmem_ld16(la + c0, v);
+            if (m >= g.M || n0 + c0 >= g.N) continue;
+            const int nn = min(16, g.N - (n0 + c0));
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.C) + (size_t)m * g.ldc + n0 + c0;
+            if (nn == 16 && (g.ldc & 7) == 0) {
+              __align__(16) __nv_bfloat16 o[16];
+              for (int j = 0; j < 16; ++j) o[j] = __float2bfloat16_rn(-rb * expf(v[j] - ra));
+              reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(o)[0];
+              reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(o)[1];
+            } else {
+              for (int j = 0; j < nn; ++j) dst[j] = __float2bfloat16_rn(-rb * expf(v[j] - ra));
+            }
+          }
+          continue;
+        }
         for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
           float v[16];
           tmem_ld16(la + c0, v);
