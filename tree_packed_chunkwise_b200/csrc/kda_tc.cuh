@@ -632,10 +632,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     __syncthreads();
     block_inverse<LC>(sT, sA, sW1, sW2);
-    {
-      float* Tg = ws.Tm + ((size_t)ci * H + h) * C * C;  // kept for the backward
-      for (int e = tid; e < C * C; e += blockDim.x) Tg[e] = sT[(e / C) * LC + (e % C)];
-    }
+    // T as a hi/lo tile (element (r, i) at cm_off(r, i, C)) for the backward, built where L was
+    uint8_t *ttH = reinterpret_cast<uint8_t*>(sA), *ttL = ttH + S::CCb;
+    build_tile<C, C, true>(ttH, ttL, [&](int r, int i) { return sT[r * LC + i]; });
     // phase 2: W = T' Kbar and U' = T' V with T' = T diag(beta)
     uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
             *vl = vh + S::CDb;
@@ -648,6 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
     const uint32_t id = tc::idesc_bf16(C, D, false, true);
     ok = run(sy, [&] {
+      store_cc_tile(ws.Tm, ((size_t)ci * H + h), ttH, ttL);
       mma3(tb + 64, tH, tL, kH, kL, C, id, false, false);
       mma3(tb + 192, tH, tL, vH, vL, C, id, false, EX);
     });
@@ -1224,10 +1224,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int e = tid; e < 6 * C; e += blockDim.x) sdb[e] = 0.f;
   Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
   if constexpr (S::kStageK) stage_rows_async(reinterpret_cast<__nv_bfloat16*>(sk), reinterpret_cast<const __nv_bfloat16*>(k_), srow, H, h, n);
+  {  // Atilde (fp32, padded rows) by 4-byte asynchronous copies; T (hi/lo tile) by a bulk copy
+    const size_t cb = (size_t)ci * H + h;
+    const float* Ag = ws.At + cb * C * C;
+    for (int e = tid; e < C * C; e += blockDim.x) tc::cp_async4(sAt + (e / C) * LC + (e % C), Ag + e, 4u);
+    tc::cp_async_commit();
+    if (tid == 0) {
+      ld_expect(ld, kCCTileBytes);
+      ld_cc_tile(ld, tTh, tTl, ws.Tm, cb);
+    }
+  }
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr);
-  if constexpr (S::kStageK) tc::cp_async_wait<0>();
+  tc::cp_async_wait<0>();  // staged k and Atilde
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
@@ -1260,31 +1270,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int myrow = lane < 16 ? 16 * sp + lane : -1;  // M = 64 accumulator row of this thread
   const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
   // TMEM columns
-  constexpr int cW = 64, cU = 192, cdW = 320, cdB = 0, cdA = 256, cRS = 320, cCS = 0;
+  // dB_k [0, 128) stays in TMEM until the last phase; CS reuses the dB_v columns [128, 256)
+  constexpr int cW = 64, cU = 192, cdW = 320, cdB = 0, cdA = 256, cRS = 320, cCS = 128;
 
-  // ---- phase 1: Atilde and T as the forward left them
-  bool ok = true;
-  float* sT = reinterpret_cast<float*>(R + S::inv_T);
-  {
-    const float* Ag = ws.At + base * C * C;
-    const float* Tg = ws.Tm + base * C * C;
-    for (int e = 4 * tid; e < C * C; e += 4 * blockDim.x) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(Ag + e));
-      const float4 tt = __ldg(reinterpret_cast<const float4*>(Tg + e));
-      const int r = e / C, i = e % C;
-      float* da = sAt + r * LC + i;
-      float* dt = sT + r * LC + i;
-      da[0] = a.x; da[1] = a.y; da[2] = a.z; da[3] = a.w;
-      dt[0] = tt.x; dt[1] = tt.y; dt[2] = tt.z; dt[3] = tt.w;
-    }
-    __syncthreads();
-  }
-  {
+  // ---- phase 1: Atilde and T as the forward left them (loaded above)
+  bool ok = ld_wait(ld);
+  // element (r, i) of T from its hi/lo tile
+  auto tval = [&](int r, int i) {
+    const uint32_t o = cm_off(r, i, C);
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tTh + o)) +
+           __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tTl + o));
+  };
+  if (ok) {
     // ---- phase 2a: W = T' Kbar, U' = T' V (T' = T diag(beta)); the T tile for T^T dX
     uint8_t *tph = R + S::p2_Tp, *tpl = tph + S::CCb, *kbh = R + S::p2_Kb, *kbl = kbh + S::CDb, *vh = R + S::p2_V,
             *vl = vh + S::CDb;
-    build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
-    build_tile<C, C, true>(tTh, tTl, [&](int r, int i) { return sT[r * LC + i]; });
+    build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return tval(r, i) * sb[i]; });
     auto kbf = [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); };
     if constexpr (S::kStageK) build_tile_st<C, D, true>(kbh, kbl, reinterpret_cast<const __nv_bfloat16*>(sk), kbf);
     else build_tile_ld<C, D, true, Tin>(kbh, kbl, row_k, kbf);
@@ -1344,21 +1345,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = myrow;
       put16<C, true>(dbh, dbl, i, c0, v);
       float part = 0.f;
-      if (c0 < D) {
-        float kv[16], a[16], b[16];
+      if (c0 < D) {  // (the dk / dG terms of dB_k are added in the last phase, from TMEM)
+        float kv[16];
         k16(i, c0, kv);
-        ld16g(pdk + i * D + c0, a);
-        ld16g(pdG + i * D + c0, b);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float eg = expf(sG[i * LD + c0 + j]);
-          const float bdb = sb[i] * v[j];
-          a[j] += eg * bdb;
-          b[j] += kv[j] * eg * bdb;
-          part = fmaf(v[j], kv[j] * eg, part);
-        }
-        st16g(pdk + i * D + c0, a);
-        st16g(pdG + i * D + c0, b);
+        for (int j = 0; j < 16; ++j) part = fmaf(v[j], kv[j] * expf(sG[i * LD + c0 + j]), part);
       } else if (i < n) {
         const int c1 = c0 - D;
         float vv[16], val[16];
@@ -1436,12 +1427,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
   }
   if (ok) {
-    // ---- final: dk, dG = partials + gated terms; dG staged for the reverse cumulative sum
+    // ---- final: dk, dG = partials + dB_k terms + gated terms; dG staged for the reverse cumulative sum
     float* sdG = reinterpret_cast<float*>(R);  // [C][LD]
     for (int c0 = grp * 16; c0 < D; c0 += 32) {
-      float rs[16], cs[16];
+      float rs[16], cs[16], dbk[16];
       tc::tmem_ld16(la + cRS + c0, rs);
       tc::tmem_ld16(la + cCS + c0, cs);
+      tc::tmem_ld16(la + cdB + c0, dbk);
       if (myrow < 0) continue;
       const int r = myrow;
       float kv[16], dkv[16], pg[16];
@@ -1453,8 +1445,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c = c0 + j;
         const float Gr = sG[r * LD + c], G0 = sref[c];
         const float a = expf(Gr - G0) * rs[j], b = expf(G0 - Gr) * cs[j];
-        dkv[j] += a + b;
-        sdG[r * LD + c] = r < n ? pg[j] + kv[j] * (a - b) : 0.f;
+        const float wb = expf(Gr) * sb[r] * dbk[j];
+        dkv[j] += wb + (a + b);
+        sdG[r * LD + c] = r < n ? pg[j] + kv[j] * (wb + (a - b)) : 0.f;
       }
       if (r < n) {
         if (r < ch.n_replay) {
