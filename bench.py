@@ -351,7 +351,7 @@ def measure_wide(args, world, rank, tpc, torch, peaks):
     one group's workspace fits the GPU, all 32 heads' would not), then per-position log-probability
     recovery with hidden 2048 and vocabulary 65,536, forward and backward."""
     import synth.gpu as sgpu
-    w = synth.workload("wide")
+    w = synth.workload(args.wide_workload)
     t = w.tree
     seed = w.seed + 1000 * rank
     plan = tpc.Plan(t.parent, t.length, 64).upload()
@@ -586,6 +586,7 @@ def main():
     ap.add_argument("--group-workload", default=GROUP_WORKLOAD, help="tree of the hybrid group (agentic by default)")
     ap.add_argument("--no-wide", action="store_true", help="skip the wide tree with log-prob recovery")
     ap.add_argument("--wide-steps", type=int, default=2)
+    ap.add_argument("--wide-workload", default="wide", help="tree of the log-prob measurement (a smaller one for profiling)")
     ap.add_argument("--workload", default=WORKLOAD, help="single_fork (default), agentic, agentic_small")
     ap.add_argument("--no-agentic", action="store_true", help="skip the agentic tree (config 2) and its ablations")
     ap.add_argument("--no-extras", action="store_true", help="skip the L1 microbatch planner and MoE routing")

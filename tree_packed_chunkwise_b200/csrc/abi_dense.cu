@@ -39,7 +39,9 @@ int gemm_launch(const void* A, const void* A_lo, const void* B, const void* B_lo
   if (c_dtype == TPC_BF16 && beta != 0.f) return fail(TPC_ERR_UNSUPPORTED, "gemm: beta needs an fp32 C");
   if (a_mn ? (lda < M) : (lda < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: lda too small");
   if (b_mn ? (ldb < N) : (ldb < K)) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldb too small");
-  if (ldc < N) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldc too small");
+  // kEpiLsePart writes one (max, sum) pair per row and column tile, the other epilogues one value per column
+  const int64_t c_cols = epi == tpc::kEpiLsePart ? (N + tpc::kGemmBN - 1) / tpc::kGemmBN : N;
+  if (ldc < c_cols) return fail(TPC_ERR_BAD_SHAPE, "gemm: ldc too small");
   if (B_lo && !A_lo) return fail(TPC_ERR_UNSUPPORTED, "gemm: B_lo needs A_lo (three-product form)");
   // 128-byte-swizzled boxes 64 elements wide: K-major [mn][K] boxes of 64 (K) x tile rows,
   // MN-major [K][mn] boxes of 64 (mn) x 64 (K)
