@@ -36,12 +36,14 @@ WORKLOAD = "single_fork"
 
 # algorithmic FLOP per processed token-head of each kernel (chunk C, head dim d): the matrix
 # products of the chunkwise form, 2 C d per token for each product within a chunk and 2 d^2 for each
-# product with a d x d state; forward kernels 10 C d + 6 d^2 in all, backward 18 C d + 14 d^2
+# product with a d x d state; forward kernels 10 C d + 6 d^2 in all, backward 18 C d + 14 d^2.  The
+# reverse scan carries M^T dS and the output's state gradient Qbar^T dO - W^T (P^T dO) (one product
+# with Qeff = Qbar - P W); the dq kernel forms P^T dO.
 def kernel_flops(name, C, d):
     Cd, dd = C * d, d * d
     name = name[:-3] if name.endswith("_tc") else name
     return {"kda_fwd_prep": 6 * Cd, "kda_fwd_scan": 4 * dd, "kda_fwd_out": 4 * Cd + 2 * dd,
-            "kda_bwd_prep": 2 * Cd + 4 * dd, "kda_bwd_scan": 4 * dd, "kda_bwd_dq": 6 * Cd + 4 * dd,
+            "kda_bwd_scan": 8 * dd, "kda_bwd_dq": 8 * Cd + 4 * dd,
             "kda_bwd_dkv": 10 * Cd + 2 * dd}.get(name, 0)
 
 
@@ -50,7 +52,7 @@ def kernel_flops(name, C, d):
 # the kernel must read or write; workspace traffic (chunk states, W, U, partials) is not counted
 def kernel_bytes(name, d):
     name = name[:-3] if name.endswith("_tc") else name
-    return {"kda_fwd_prep": 6 * d + 2, "kda_fwd_out": 8 * d, "kda_bwd_prep": 8 * d, "kda_bwd_dq": 10 * d,
+    return {"kda_fwd_prep": 6 * d + 2, "kda_fwd_out": 8 * d, "kda_bwd_dq": 10 * d,
             "kda_bwd_dkv": 14 * d + 6}.get(name, 0)
 
 

@@ -8,7 +8,7 @@ def test_kernel_flops_sum_to_the_chunkwise_totals():
     for C, d in [(64, 128), (16, 32)]:
         Cd, dd = C * d, d * d
         fwd = sum(bench.kernel_flops(k, C, d) for k in ("kda_fwd_prep_tc", "kda_fwd_scan_tc", "kda_fwd_out_tc"))
-        bwd = sum(bench.kernel_flops(k, C, d) for k in ("kda_bwd_prep_tc", "kda_bwd_scan_tc", "kda_bwd_dq_tc",
+        bwd = sum(bench.kernel_flops(k, C, d) for k in ("kda_bwd_scan_tc", "kda_bwd_dq_tc",
                                                          "kda_bwd_dkv_tc"))
         assert fwd == 10 * Cd + 6 * dd
         assert bwd == 18 * Cd + 14 * dd

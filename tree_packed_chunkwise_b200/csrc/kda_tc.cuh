@@ -13,7 +13,8 @@
 // a later row of the chunk, so a row shared by several trajectories gets the same bits whether its
 // chunk continues into one branch or another (each trajectory keeps its chunkwise numerical path).
 // Factors stay within e^{+-80} while a channel decays by at most kMaxChunkDecay over one chunk
-// (checked; TPC_ERR_RANGE otherwise).
+// (checked; TPC_ERR_RANGE otherwise).  In shared memory the cumulative gates are kept in base-2
+// units (G log2 e), so every factor e^{G_a - G_b} is one hardware exp2 of a difference.
 #pragma once
 #include <type_traits>
 
@@ -23,11 +24,15 @@
 namespace tpc {
 
 constexpr int kTcC = 64, kTcD = 128;
+// CTA size of the per-chunk tensor-core kernels: 16 warps, i.e. four warps per TMEM sub-partition
+// (kTcGroups warp groups of 128 threads split the columns of every accumulator read)
+constexpr int kTcThreads = 512, kTcGroups = kTcThreads / 128;
 constexpr uint32_t kMtileBytes = 2u * kTcD * kTcD * 2u;  // state transition tile: hi + lo bf16, 128 x 128
 // chunk-start state S0 and chunk-end state gradient dS as hi/lo bf16 operand tiles (element (c, j) at
 // cm_off(c, j, 128) in the hi half, the same in the lo half): one 128 x 128 tile per chunk and head
 constexpr uint32_t kStateTileBytes = 2u * kTcD * kTcD * 2u;
 constexpr float kMaxChunkDecay = 80.f;  // G_first - G_last per channel over one chunk
+constexpr float kLog2e = 1.4426950408889634f;
 enum : int { kStatusTimeout = 8 };
 // state scans: CTA size and width of the d_v slice one CTA owns
 constexpr int kScanThreads = 128, kScanDVT = 32;
@@ -82,7 +87,7 @@ __device__ __forceinline__ void ld8(const T* p, float (&x)[8]) {
   }
 }
 
-template <int A, int B, bool SPLIT, typename T, int NT = kThreads, class RP, class F>
+template <int A, int B, bool SPLIT, typename T, int NT = kTcThreads, class RP, class F>
 __device__ __forceinline__ void build_tile_ld(uint8_t* hi, uint8_t* lo, RP rowp, F f) {
   constexpr int NCH = A * (B / 8);
   static_assert(NCH % NT == 0, "tile chunks must be a multiple of the CTA size");
@@ -114,15 +119,50 @@ __device__ __forceinline__ void build_tile_ld(uint8_t* hi, uint8_t* lo, RP rowp,
   }
 }
 
+// Two tiles (hi/lo) of the same rows, values f1(a, b, x) and f2(a, b, x), from one load of the rows
+template <int A, int B, typename T, class RP, class F1, class F2>
+__device__ __forceinline__ void build_tile2_ld(uint8_t* hi1, uint8_t* lo1, uint8_t* hi2, uint8_t* lo2, RP rowp, F1 f1,
+                                               F2 f2) {
+  constexpr int NCH = A * (B / 8), NT = kTcThreads;
+  static_assert(NCH % NT == 0, "tile chunks must be a multiple of the CTA size");
+  constexpr int IT = NCH / NT;
+  float x[IT][8];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * NT, a = e % A, b0 = (e / A) * 8;
+    const T* p = rowp(a);
+    if (p) ld8(p + b0, x[it]);
+    else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[it][j] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e = threadIdx.x + it * NT, a = e % A, b0 = (e / A) * 8;
+    __align__(16) __nv_bfloat16 h1[8], l1[8], h2[8], l2[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      split_bf16(f1(a, b0 + j, x[it][j]), h1[j], l1[j]);
+      split_bf16(f2(a, b0 + j, x[it][j]), h2[j], l2[j]);
+    }
+    const uint32_t off = cm_off(a, b0, A);
+    *reinterpret_cast<uint4*>(hi1 + off) = *reinterpret_cast<const uint4*>(h1);
+    *reinterpret_cast<uint4*>(lo1 + off) = *reinterpret_cast<const uint4*>(l1);
+    *reinterpret_cast<uint4*>(hi2 + off) = *reinterpret_cast<const uint4*>(h2);
+    *reinterpret_cast<uint4*>(lo2 + off) = *reinterpret_cast<const uint4*>(l2);
+  }
+}
+
 // Gate rows of the chunk into G (fp32, pitch LD): every thread issues its 16-byte loads first;
 // neighbouring threads take neighbouring rows (conflict-free stores).  Rows >= n are zero.
 template <typename T>
 __device__ __forceinline__ void load_gate(float* G, int LD, const T* g_, const int* rows, int H, int h, int n) {
-  constexpr int NCH = kTcC * (kTcD / 8), IT = NCH / kThreads;
+  constexpr int NCH = kTcC * (kTcD / 8), IT = NCH / kTcThreads;
   float x[IT][8];
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * kThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
+    const int e = threadIdx.x + it * kTcThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
     if (a < n) ld8(g_ + ((size_t)rows[a] * H + h) * kTcD + b0, x[it]);
     else
 #pragma unroll
@@ -130,7 +170,7 @@ __device__ __forceinline__ void load_gate(float* G, int LD, const T* g_, const i
   }
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * kThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
+    const int e = threadIdx.x + it * kTcThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
 #pragma unroll
     for (int j = 0; j < 8; ++j) G[a * LD + b0 + j] = x[it][j];
   }
@@ -140,17 +180,17 @@ __device__ __forceinline__ void load_gate(float* G, int LD, const T* g_, const i
 constexpr int kStagePitch = kTcD + 8;
 template <typename T>
 __device__ __forceinline__ void stage_rows(T* dst, const T* src, const int* rows, int H, int h, int n) {
-  constexpr int VEC = 16 / sizeof(T), NCH = kTcC * (kTcD / VEC), IT = NCH / kThreads;
+  constexpr int VEC = 16 / sizeof(T), NCH = kTcC * (kTcD / VEC), IT = NCH / kTcThreads;
   uint4 x[IT];
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * kThreads, a = e / (kTcD / VEC), b0 = (e % (kTcD / VEC)) * VEC;
+    const int e = threadIdx.x + it * kTcThreads, a = e / (kTcD / VEC), b0 = (e % (kTcD / VEC)) * VEC;
     x[it] = a < n ? __ldg(reinterpret_cast<const uint4*>(src + ((size_t)rows[a] * H + h) * kTcD + b0))
                   : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * kThreads, a = e / (kTcD / VEC), b0 = (e % (kTcD / VEC)) * VEC;
+    const int e = threadIdx.x + it * kTcThreads, a = e / (kTcD / VEC), b0 = (e % (kTcD / VEC)) * VEC;
     *reinterpret_cast<uint4*>(dst + a * kStagePitch + b0) = x[it];
   }
 }
@@ -194,6 +234,37 @@ __device__ __forceinline__ void build_tile_st(uint8_t* hi, uint8_t* lo, const __
   }
 }
 
+// C x D K-major tile (element (a, b) at cm_off(a, b, A)) of raw bf16 rows gathered by 16-byte
+// asynchronous copies (one per row and 8 columns); rows that rowp maps to nullptr are zero.
+// Completed by cp_async_wait + a barrier.
+template <int A, int B, class RP>
+__device__ __forceinline__ void tile_async_bf16(uint8_t* hi, RP rowp, const void* any_valid) {
+  for (int e = threadIdx.x; e < A * (B / 8); e += blockDim.x) {
+    const int a = e % A, b0 = (e / A) * 8;
+    const __nv_bfloat16* p = rowp(a);
+    tc::cp_async16(hi + cm_off(a, b0, A), p ? static_cast<const void*>(p + b0) : any_valid, p ? 16u : 0u);
+  }
+  tc::cp_async_commit();
+}
+
+// 16 values (a, b0 .. b0 + 15) of a K-major hi/lo tile in shared memory, as fp32 (hi + lo)
+template <int A>
+__device__ __forceinline__ void tile16(const uint8_t* hi, const uint8_t* lo, int a, int b0, float (&v)[16]) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t off = cm_off(a, b0 + 8 * half, A);
+    const uint4 hq = *reinterpret_cast<const uint4*>(hi + off), lq = *reinterpret_cast<const uint4*>(lo + off);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
+    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lq);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 x = __bfloat1622float2(h2[k]), y = __bfloat1622float2(l2[k]);
+      v[8 * half + 2 * k] = x.x + y.x;
+      v[8 * half + 2 * k + 1] = x.y + y.y;
+    }
+  }
+}
+
 // 16 consecutive values of a staged row as fp32
 template <typename T>
 __device__ __forceinline__ void staged16(const T* st, int r, int c0, float (&v)[16]) {
@@ -225,12 +296,12 @@ __device__ __forceinline__ void ld16g(const float* p, float (&v)[16]) {
     v[j] = u.x; v[j + 1] = u.y; v[j + 2] = u.z; v[j + 3] = u.w;
   }
 }
-__device__ __forceinline__ void st16g(float* p, const float (&v)[16]) {
+__device__ __forceinline__ void st16g(float* p, const float* v) {
 #pragma unroll
   for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(p + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
 }
 template <typename T>
-__device__ __forceinline__ void st16_out(T* p, const float (&v)[16]) {
+__device__ __forceinline__ void st16_out(T* p, const float* v) {
   if constexpr (sizeof(T) == 4) {
     st16g(reinterpret_cast<float*>(p), v);
   } else {
@@ -242,13 +313,13 @@ __device__ __forceinline__ void st16_out(T* p, const float (&v)[16]) {
   }
 }
 
-// Reads an M x N fp32 accumulator (N a multiple of 32) starting at TMEM column col0:
+// Reads an M x N fp32 accumulator (N a multiple of 16) starting at TMEM column col0:
 // f(m, n0, v) gets 16 consecutive columns n0 .. n0+15 of row m.  Warp w reads the lanes of
-// sub-partition w % 4; the two groups of four warps take alternating 16-column chunks.
+// sub-partition w % 4; the kTcGroups groups of four warps take interleaved 16-column chunks.
 template <int M, int N, class F>
 __device__ __forceinline__ void acc_read(uint32_t tbase, int col0, F f) {
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, sp = w & 3, grp = (w >> 2) & 1;
-  for (int c = grp * 16; c < N; c += 32) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, sp = w & 3, grp = w >> 2;
+  for (int c = grp * 16; c < N; c += 16 * kTcGroups) {
     float v[16];
     tmem_ld16(tbase + ((uint32_t)(32 * sp) << 16) + (uint32_t)(col0 + c), v);
     const int m = (M == 128) ? 32 * sp + lane : (lane < 16 ? 16 * sp + lane : -1);
@@ -382,12 +453,15 @@ __device__ __forceinline__ bool ld_wait(Ld& l) {
   return true;
 }
 
-// sum over j of a(c, j) b(c, j) for two state tiles in global memory (hi + lo of each), row c
-__device__ __forceinline__ float state_row_dot(const float* ta, const float* tb, size_t base, int c) {
+// sum over j in [j_begin, j_end) of a(c, j) b(c, j) for two state tiles in global memory (hi + lo of
+// each), row c
+__device__ __forceinline__ float state_row_dot(const float* ta, const float* tb, size_t base, int c, int j_begin,
+                                               int j_end) {
   const uint8_t* a = reinterpret_cast<const uint8_t*>(ta) + base * kStateTileBytes;
   const uint8_t* b = reinterpret_cast<const uint8_t*>(tb) + base * kStateTileBytes;
   float acc = 0.f;
-  for (int j0 = 0; j0 < kTcD; j0 += 8) {
+#pragma unroll 4
+  for (int j0 = j_begin; j0 < j_end; j0 += 8) {
     const uint32_t off = cm_off(c, j0, kTcD);
     const uint4 ah = __ldg(reinterpret_cast<const uint4*>(a + off));
     const uint4 al = __ldg(reinterpret_cast<const uint4*>(a + kStateTileBytes / 2 + off));
@@ -508,18 +582,30 @@ __device__ __forceinline__ void block_inverse(float* T, const float* L, float* W
   __syncthreads();
 }
 
-// G <- inclusive cumulative gate over the chunk's rows (rows >= n repeat row n - 1); the reference
-// (row 0) goes to ref[c].  Flags TPC_ERR_RANGE when a channel decays by more than kMaxChunkDecay.
-__device__ __forceinline__ void cumsum_ref(float* G, int LD, int n, float* ref, int* status) {
-  for (int c = threadIdx.x; c < kTcD; c += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < kTcC; ++i) {
-      if (i < n) acc += G[i * LD + c];
-      G[i * LD + c] = acc;
-    }
-    ref[c] = G[c];
-    if (status && !(G[c] - G[(n - 1) * LD + c] <= kMaxChunkDecay)) set_status(status, kStatusRange);
+// G <- inclusive cumulative gate over the chunk's rows (rows >= n repeat row n - 1), in base-2 units;
+// the reference (row 0) goes to ref[c].  Flags TPC_ERR_RANGE when a channel decays by more than
+// kMaxChunkDecay.  Four threads per channel, each a quarter of the rows: the quarters' totals, then
+// each quarter's running sum from the earlier quarters' totals.  Row i's value depends on rows <= i
+// only (the same bits whichever rows follow it in the chunk).  scratch: 4 x kTcD floats.
+__device__ __forceinline__ void cumsum_ref(float* G, int LD, int n, float* ref, int* status, float* scratch) {
+  static_assert(kTcThreads == 4 * kTcD && kTcC == 64, "four threads per channel, 16 rows each");
+  const int c = threadIdx.x % kTcD, q = threadIdx.x / kTcD, i0 = 16 * q;
+  float a = 0.f;
+#pragma unroll
+  for (int i = i0; i < i0 + 16; ++i)
+    if (i < n) a += G[i * LD + c];
+  scratch[q * kTcD + c] = a;
+  __syncthreads();
+  float acc = 0.f;
+  for (int p = 0; p < q; ++p) acc += scratch[p * kTcD + c];
+#pragma unroll
+  for (int i = i0; i < i0 + 16; ++i) {
+    if (i < n) acc += G[i * LD + c];
+    G[i * LD + c] = acc * kLog2e;
   }
+  if (q == 0) ref[c] = G[c];
+  __syncthreads();  // G and ref complete
+  if (q == 0 && status && !(G[c] - G[(kTcC - 1) * LD + c] <= kMaxChunkDecay * kLog2e)) set_status(status, kStatusRange);
 }
 
 template <typename T>
@@ -552,7 +638,7 @@ struct PrepTcSmemT {
 };
 
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     kda_fwd_prep_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
                     const Tin* __restrict__ g_, const Tin* __restrict__ beta_, KdaWs ws, int chunk0 = 0) {
   using namespace tck;
@@ -594,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
-  cumsum_ref(sG, LD, n, sref, ws.status);
+  cumsum_ref(sG, LD, n, sref, ws.status, reinterpret_cast<float*>(tl));  // (tiles not yet in use)
   if constexpr (EX) tc::cp_async_wait<0>();
   __syncthreads();
   tc::fence_after_sync();
@@ -611,8 +697,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // phase 1: Atilde = af bf^T with af = k e^{G - ref}, bf = k e^{ref - G}
   {
     uint8_t *afh = tl, *afl = tl + S::CDb, *bfh = tl + 2 * S::CDb, *bfl = tl + 3 * S::CDb;
-    k_tile(afh, afl, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
-    k_tile(bfh, bfl, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
+    k_tile(afh, afl, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); });
+    k_tile(bfh, bfl, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
     const tc::Op ah{tc::smem_u32(afh), C, false}, al{tc::smem_u32(afl), C, false};
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
     ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
@@ -639,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
             *vl = vh + S::CDb;
     build_tile<C, C, true>(th, tlo, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
-    k_tile(kh, kl, [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); });
+    k_tile(kh, kl, [&](int i, int c, float x) { return x * tc::ex2(sG[i * LD + c]); });
     if constexpr (EX) build_tile_st<C, D, false>(vh, vl, sv, [&](int, int, float x) { return x; });
     else build_tile_ld<C, D, true, Tin>(vh, vl, row_v, [&](int, int, float x) { return x; });
     const tc::Op tH{tc::smem_u32(th), C, false}, tL{tc::smem_u32(tlo), C, false};
@@ -662,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) { put16<C, true>(wth, wtl, r, c0, v); });
       acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) { put16<C, true>(uth, utl, r, c0, v); });
       const float* gC = sG + (n - 1) * LD;
-      k_tile(khh, khl, [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); });
+      k_tile(khh, khl, [&](int i, int c, float x) { return x * tc::ex2(gC[c] - sG[i * LD + c]); });
       ok = run(sy, [&] {
         store_cd_tile(ws.W, base, wth, wtl);
         store_cd_tile(ws.U, base, uth, utl);
@@ -678,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* Bg = ws.Bc + base * D * D;
         acc_read<D, D>(tb, 0, [&](int c, int c0, const float* v) {
           float m[16];
-          const float gam = expf(gC[c]);
+          const float gam = tc::ex2(gC[c]);
           for (int j = 0; j < 16; ++j) m[j] = (c0 + j == c ? gam : 0.f) - v[j];
           put16<D, true>(Mt, Mt + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
         });
@@ -715,7 +801,7 @@ struct OutTcSmem {
 };
 
 template <typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     kda_fwd_out_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
                    const Tin* __restrict__ g_, Tout* __restrict__ o_, KdaWs ws, int chunk0 = 0) {
   using namespace tck;
@@ -747,8 +833,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
-  cumsum_ref(sG, LD, n, sref, nullptr);
-  __syncthreads();
+  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb;
+  cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(qbh));  // (the Qbar tile comes later)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
@@ -757,8 +843,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // TMEM: P [0,64), W S0 [64,192), O [192,320), P W [320,448)
   uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
   uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb;
-  build_tile_ld<C, D, true, Tin>(qfh, qfl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); });
-  build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); });
+  // qf = q e^{G - ref} and Qbar = q e^G from one load of q; bf = k e^{ref - G}
+  build_tile2_ld<C, D, Tin>(
+      qfh, qfl, qbh, qbl, row_q, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); },
+      [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c]); });
+  build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
   const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
   bool ok = ld_wait(ld);
   ok = ok && run(sy, [&] {
@@ -769,20 +858,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma4(tb + 64, wH, wL, sH, sL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
   });
   uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
-  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb;
   if (ok) {
+    if (tid == 0) {  // U' (as the prep kernel left it) into the consumed qf / bf space
+      ld_expect(ld, kCDTileBytes);
+      ld_cd_tile(ld, uh, ul, ws.U, base);
+    }
     acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
       float m[16];
       for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
       put16<C, true>(ph, pl, r, i0, m);  // kept (as this tile) for the backward
     });
+    ok = ld_wait(ld);
+  }
+  if (ok) {
     acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
       float u[16];
-      cd_tile16(ws.U, base, i, j0, u);  // U'
+      tile16<C>(uh, ul, i, j0, u);  // U'
       for (int j = 0; j < 16; ++j) u[j] -= v[j];
-      put16<C, true>(uh, ul, i, j0, u);  // element (i, j): MN-major (k = i); kept for the backward
+      put16<C, true>(uh, ul, i, j0, u);  // U, element (i, j): MN-major (k = i); kept for the backward
     });
-    build_tile_ld<C, D, true, Tin>(qbh, qbl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c]); });
     ok = run(sy, [&] {
       store_cc_tile(ws.Pm, base, ph, pl);
       store_cd_tile(ws.U, base, uh, ul);  // U replaces U'
@@ -798,28 +892,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
     if (ok) {
       acc_read<C, D>(tb, 192, [&](int r, int j0, const float* v) {
-        if (r >= ch.n_replay && r < n) {
-          Tout* dst = o_ + ((size_t)srow[r] * H + h) * D + j0;
-          for (int j = 0; j < 16; ++j) dst[j] = from_f<Tout>(v[j]);
-        }
+        if (r >= ch.n_replay && r < n) st16_out(o_ + ((size_t)srow[r] * H + h) * D + j0, v);
       });
       // Qeff = Qbar - P W (element (r, c)) into the S0 buffer, which the products above consumed
       uint8_t *eh = s0h, *el = s0h + S::CDb;
       acc_read<C, D>(tb, 320, [&](int r, int c0, const float* v) {
         float e[16];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t off = cm_off(r, c0 + 8 * half, C);
-          const uint4 hq = *reinterpret_cast<const uint4*>(qbh + off), lq = *reinterpret_cast<const uint4*>(qbl + off);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
-          const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lq);
-#pragma unroll
-          for (int k2 = 0; k2 < 4; ++k2) {
-            const float2 a = __bfloat1622float2(h2[k2]), b = __bfloat1622float2(l2[k2]);
-            e[8 * half + 2 * k2] = (a.x + b.x) - v[8 * half + 2 * k2];
-            e[8 * half + 2 * k2 + 1] = (a.y + b.y) - v[8 * half + 2 * k2 + 1];
-          }
-        }
+        tile16<C>(qbh, qbl, r, c0, e);  // Qbar
+        for (int j = 0; j < 16; ++j) e[j] -= v[j];
         put16<C, true>(eh, el, r, c0, e);
       });
       tc::fence_async_smem();
@@ -828,112 +908,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (tid == 0) tc::bulk_wait_all();
-  tc::fence_before_sync();
-  __syncthreads();
-  if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
-}
-
-// --------------------------------------------------------------------------------- backward prep
-// per (chunk, head): dU0 = P^T dO and X = Qbar^T dO - W^T dU0 (the state-independent parts of the
-// reverse scan).  dO rows of replayed rows are zero.
-struct BprepTcSmem {
-  static constexpr int C = kTcC, D = kTcD, LD = D + 1;
-  static constexpr size_t G = 0;
-  static constexpr size_t vec = G + sizeof(float) * C * LD;
-  static constexpr size_t tiles = (vec + sizeof(float) * D + 1023) & ~size_t(1023);
-  static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2;
-  static constexpr size_t R = tiles;             // qf, bf (4 CDb) -> P (2 CCb) + dU0 (2 CDb)
-  static constexpr size_t Qb = R + 4 * CDb;      // Qbar, MN-major
-  static constexpr size_t dO = Qb + 2 * CDb;     // dO, MN-major
-  static constexpr size_t Wt = dO + 2 * CDb;     // W (as the prep kernel stored it), used MN-major
-  static constexpr size_t total = Wt + 2 * CDb;
-};
-
-template <typename Tin>
-__global__ void __launch_bounds__(kThreads, 1)
-    kda_bwd_prep_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
-                    const Tin* __restrict__ g_, const Tin* __restrict__ do_, KdaWs ws, int chunk0 = 0) {
-  using namespace tck;
-  using S = BprepTcSmem;
-  constexpr int C = S::C, D = S::D, LD = S::LD;
-  constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
-  const ChunkRec ch = t.chunks[ci];
-  const int n = ch.n_rows;
-  extern __shared__ __align__(1024) uint8_t tsm[];
-  float* sG = reinterpret_cast<float*>(tsm + S::G);
-  float* sref = reinterpret_cast<float*>(tsm + S::vec);
-  __shared__ int srow[C];
-  __shared__ __align__(8) uint64_t bar, bar_ld;
-  __shared__ uint32_t tslot;
-  const int tid = threadIdx.x;
-  const size_t base = (size_t)ci * H + h;
-  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb, *doh = tsm + S::dO, *dol = doh + S::CDb;
-  uint8_t *wh = tsm + S::Wt, *wl = wh + S::CDb;
-  // P (masked gated q k products; element (r, i), the MN-major operand P^T) as the forward left it
-  uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *duh = pl + S::CCb, *dul = duh + S::CDb;
-  for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
-  if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
-  Ld ld{&bar_ld, 0u, ws.status};
-  if (tid == 0) {
-    tc::mbar_init(&bar, 1);
-    tc::mbar_init(&bar_ld, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    ld_expect(ld, kCDTileBytes + kCCTileBytes);
-    ld_cd_tile(ld, wh, wl, ws.W, base);
-    ld_cc_tile(ld, ph, pl, ws.Pm, base);
-  }
-  __syncthreads();
-  load_gate(sG, LD, g_, srow, H, h, n);
-  __syncthreads();
-  cumsum_ref(sG, LD, n, sref, nullptr);
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tb = tslot;
-  Sync sy{&bar, 0u, ws.status};
-  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_do = [&](int a) -> const Tin* {
-    return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
-  };
-  build_tile_ld<C, D, true, Tin>(qbh, qbl, row_q, [&](int r, int c, float x) { return x * expf(sG[r * LD + c]); });
-  build_tile_ld<C, D, !EX, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
-  bool ok = ld_wait(ld);
-  if (ok) {
-    ok = run(sy, [&] {
-      const tc::Op pH{tc::smem_u32(ph), C, true}, pL{tc::smem_u32(pl), C, true};
-      const tc::Op oH{tc::smem_u32(doh), C, true}, oL{tc::smem_u32(dol), C, true};
-      mma3(tb + 64, pH, pL, oH, oL, C, tc::idesc_bf16(C, D, true, true), false, EX);
-    });
-  }
-  if (ok) {
-    float* dU = ws.dU + base * C * D;
-    acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
-      float m[16];
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(dU + i * D + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-      for (int j = 0; j < 16; ++j) m[j] = -v[j];
-      put16<C, true>(duh, dul, i, j0, m);  // -dU0, element (i, j): MN-major operand (k = i, n = j)
-    });
-    ok = run(sy, [&] {
-      const uint32_t id = tc::idesc_bf16(D, D, true, true);
-      const tc::Op qH{tc::smem_u32(qbh), C, true}, qL{tc::smem_u32(qbl), C, true};
-      const tc::Op oH{tc::smem_u32(doh), C, true}, oL{tc::smem_u32(dol), C, true};
-      const tc::Op wH{tc::smem_u32(wh), C, true}, wL{tc::smem_u32(wl), C, true};
-      const tc::Op uH{tc::smem_u32(duh), C, true}, uL{tc::smem_u32(dul), C, true};
-      mma3(tb + 192, qH, qL, oH, oL, C, id, false, EX);
-      mma3(tb + 192, wH, wL, uH, uL, C, id, true, false);
-    });
-  }
-  if (ok) {
-    // X goes where the forward kept B (dead once the forward scans are done), slice-major for the
-    // reverse scan's bulk loads
-    float* X = ws.Bc + base * D * D;
-    acc_read<D, D>(tb, 192, [&](int c, int j0, const float* v) {
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(X + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-    });
-  }
   tc::fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
@@ -960,12 +934,16 @@ struct BdqTcSmem {
   static constexpr size_t Pt = R + 4 * CDb + 2 * DDb;
   static constexpr size_t Stage = Pt + 2 * CCb;  // bf16 inputs: the chunk's q and k rows (pitch kStagePitch)
   static constexpr size_t StB = size_t(C) * tck::kStagePitch * 2;
-  static constexpr size_t total = Stage + 2 * StB;
+  static constexpr size_t Scr = Stage + 2 * StB;  // 4 x D fp32 scratch of the gate accumulation
+  static constexpr size_t total = Scr + sizeof(float) * 4 * D;
+  // epilogue, inside R: row buffer (C x LD fp32), fp32 staging of q and k (fp32 inputs), column partials
+  static constexpr size_t Part = sizeof(float) * C * LD + 2 * sizeof(float) * C * tck::kStagePitch;
+  static_assert(Part + sizeof(float) * 8 * D <= 4 * CDb + 2 * DDb, "epilogue scratch exceeds R");
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
 template <typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     kda_bwd_dq_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
                   const Tin* __restrict__ g_, const Tin* __restrict__ do_, Tout* __restrict__ dq_, KdaWs ws,
                   int chunk0 = 0) {
@@ -1002,26 +980,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bf16: the chunk's q and k rows into shared memory while the gates load and accumulate
   [[maybe_unused]] __nv_bfloat16* stq = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
   [[maybe_unused]] __nv_bfloat16* stk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
-  if constexpr (EX) {
-    stage_rows_async(stq, q_, srow, H, h, n);
-    stage_rows_async(stk, k_, srow, H, h, n);
-  }
-  load_gate(sG, LD, g_, srow, H, h, n);
-  __syncthreads();
-  cumsum_ref(sG, LD, n, sref, nullptr);
-  if constexpr (EX) tc::cp_async_wait<0>();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tb = tslot;
-  Sync sy{&bar, 0u, ws.status};
   auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   auto row_do = [&](int a) -> const Tin* {
     return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
   };
+  if constexpr (EX) {  // dO straight into its operand tile (raw bf16: no lo part)
+    stage_rows_async(stq, q_, srow, H, h, n);
+    stage_rows_async(stk, k_, srow, H, h, n);
+    tile_async_bf16<C, D>(doh, row_do, do_);
+  }
+  load_gate(sG, LD, g_, srow, H, h, n);
+  __syncthreads();
+  cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(tsm + S::Scr));
+  if constexpr (EX) tc::cp_async_wait<0>();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = tslot;
+  Sync sy{&bar, 0u, ws.status};
   // TMEM columns: Tq [0,128), T1 [128,256), RS [256,384), dP [384,448) then CS [384,512)
   constexpr int cTq = 0, cT1 = 128, cRS = 256, cCS = 384;
-  build_tile_ld<C, D, !EX, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
+  if constexpr (!EX) build_tile_ld<C, D, true, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
   const tc::Op oH{tc::smem_u32(doh), C, false}, oL{tc::smem_u32(dol), C, false};
   const tc::Op uH{tc::smem_u32(uh), C, false}, uL{tc::smem_u32(ul), C, false};
   const tc::Op sH{tc::smem_u32(sh), D, false}, sL{tc::smem_u32(sl), D, false};
@@ -1043,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ld_state_tile(ld, sh, sl, ws.dS, base);
     }
     const float* gC = sG + (n - 1) * LD;
-    auto khf = [&](int i, int c, float x) { return x * expf(gC[c] - sG[i * LD + c]); };
+    auto khf = [&](int i, int c, float x) { return x * tc::ex2(gC[c] - sG[i * LD + c]); };
     if constexpr (EX) build_tile_st<C, D, true>(doh, dol, stk, khf);
     else build_tile_ld<C, D, true, Tin>(doh, dol, row_k, khf);
     ok = ld_wait(ld);
@@ -1074,8 +1053,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
       put16<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
     });
-    auto bff = [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); };
-    auto qff = [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); };
+    auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
+    auto qff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
     if constexpr (EX) {
       build_tile_st<C, D, true>(bh, bl, stk, bff);
       build_tile_st<C, D, true>(qh, ql, stq, qff);
@@ -1107,10 +1086,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage_rows(sk, k_, srow, H, h, n);
     }
     __syncthreads();
-    const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
+    const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
     const int r = lane < 16 ? 16 * sp + lane : -1;
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
-    for (int c0 = grp * 16; c0 < D; c0 += 32) {
+    for (int c0 = grp * 16; c0 < D; c0 += 16 * kTcGroups) {
       float tq[16], t1[16], rs[16], cs[16];
       tc::tmem_ld16(la + cTq + c0, tq);
       tc::tmem_ld16(la + cT1 + c0, t1);
@@ -1124,9 +1103,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) {
         const int c = c0 + j;
         const float Gr = sG[r * LD + c], G0 = sref[c], GC = sG[(n - 1) * LD + c];
-        dq[j] = expf(Gr) * tq[j] + expf(Gr - G0) * rs[j];
-        const float dks = expf(GC - Gr) * t1[j];
-        dk[j] = dks + expf(G0 - Gr) * cs[j];
+        dq[j] = tc::ex2(Gr) * tq[j] + tc::ex2(Gr - G0) * rs[j];
+        const float dks = tc::ex2(GC - Gr) * t1[j];
+        dk[j] = dks + tc::ex2(G0 - Gr) * cs[j];
         dG[j] = qv[j] * dq[j] - kv[j] * dk[j];
         sbuf[r * LD + c] = r < n ? kv[j] * dks : 0.f;
       }
@@ -1135,11 +1114,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (r >= ch.n_replay && r < n) st16_out(dq_ + ((size_t)srow[r] * H + h) * D + c0, dq);
     }
     __syncthreads();
-    for (int c = tid; c < D; c += blockDim.x) {
-      float acc = 0.f;
-      for (int i = 0; i < n; ++i) acc += sbuf[i * LD + c];
-      const float acc2 = state_row_dot(ws.dS, ws.S0, base, c);  // sum_j dS_cj S0_cj
-      pdG[(n - 1) * D + c] += acc + expf(sG[(n - 1) * LD + c]) * acc2;
+    // per column c: sum over rows of the row buffer and sum_j dS_cj S0_cj, each split over four
+    // threads (rows and j in quarters) and combined in a fixed order
+    static_assert(kTcThreads == 4 * D, "four threads per column");
+    float* part = reinterpret_cast<float*>(tsm + S::R + S::Part);  // [2][4][D]
+    {
+      const int c = tid % D, q4 = tid / D;
+      float a = 0.f;
+      for (int i = 16 * q4; i < 16 * q4 + 16; ++i) a += sbuf[i * LD + c];  // rows >= n hold zeros
+      part[q4 * D + c] = a;
+      part[(4 + q4) * D + c] = state_row_dot(ws.dS, ws.S0, base, c, 32 * q4, 32 * q4 + 32);
+    }
+    __syncthreads();
+    if (tid < D) {
+      const int c = tid;
+      const float acc = (part[c] + part[D + c]) + (part[2 * D + c] + part[3 * D + c]);
+      const float acc2 = (part[4 * D + c] + part[5 * D + c]) + (part[6 * D + c] + part[7 * D + c]);
+      pdG[(n - 1) * D + c] += acc + tc::ex2(sG[(n - 1) * LD + c]) * acc2;
     }
   }
   if (tid == 0) tc::bulk_wait_all();
@@ -1164,8 +1155,8 @@ struct BdkvTcSmemT {
   static constexpr int C = kTcC, D = kTcD, LD = D + 1, LC = C + 1;
   static constexpr size_t G = 0;
   static constexpr size_t At = G + sizeof(float) * C * LD;        // Atilde fp32 [C][LC]
-  static constexpr size_t vec = At + sizeof(float) * C * LC;      // beta[C], ref[D], dbeta parts[6][C]
-  static constexpr size_t Ks = (vec + sizeof(float) * (C + D + 6 * C) + 15) & ~size_t(15);      // staged k rows
+  static constexpr size_t vec = At + sizeof(float) * C * LC;      // beta[C], ref[D], dbeta parts[3][groups][C]
+  static constexpr size_t Ks = (vec + sizeof(float) * (C + D + 3 * kTcGroups * C) + 15) & ~size_t(15);  // staged k
   static constexpr size_t Tt = (Ks + (kStageK ? sizeof(Tin) * C * tck::kStagePitch : 0) + 1023) & ~size_t(1023);  // T tile
   static constexpr size_t CCb = size_t(C) * C * 2, CDb = size_t(C) * D * 2, DDb = size_t(D) * D * 2;
   static constexpr size_t R = Tt + 2 * CCb;
@@ -1186,7 +1177,7 @@ struct BdkvTcSmemT {
 };
 
 template <typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     kda_bwd_dkv_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, Tout* __restrict__ dk_,
                    Tout* __restrict__ dv_, float* __restrict__ dg_, float* __restrict__ dbeta_, KdaWs ws,
@@ -1203,15 +1194,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sAt = reinterpret_cast<float*>(tsm + S::At);
   float* sb = reinterpret_cast<float*>(tsm + S::vec);
   float* sref = sb + C;
-  float* sdb = sref + D;  // [6][C] partial dbeta (dB_k, dB_v, dA parts per warp group), fixed-order sum
+  float* sdb = sref + D;  // [3][kTcGroups][C] partial dbeta (dB_k, dB_v, dA parts per warp group), fixed-order sum
   uint8_t* tTh = tsm + S::Tt;
   uint8_t* tTl = tTh + S::CCb;
   uint8_t* R = tsm + S::R;
   __shared__ int srow[C];
+  // where row r's gradients go: kind 0 the replay partials (row idx), 1 the target staging (row idx),
+  // 2 the outputs (row idx = srow)
+  __shared__ int skind[C], sidx[C];
   __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
-  for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
+  for (int i = tid; i < C; i += blockDim.x) {
+    const int row = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
+    srow[i] = row;
+    int kind = 2, idx = row;
+    if (i < ch.n_replay) {
+      kind = 0;
+      idx = ch.replay_base + i;
+    } else if (i < n) {
+      const int tg = t.row_tgt[row];
+      if (tg >= 0) {
+        kind = 1;
+        idx = tg;
+      }
+    }
+    skind[i] = kind;
+    sidx[i] = idx;
+  }
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
   Ld ld{&bar_ld, 0u, ws.status};
   if (tid == 0) {
@@ -1221,9 +1231,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
-  for (int e = tid; e < 6 * C; e += blockDim.x) sdb[e] = 0.f;
+  for (int e = tid; e < 3 * kTcGroups * C; e += blockDim.x) sdb[e] = 0.f;
   Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
-  if constexpr (S::kStageK) stage_rows_async(reinterpret_cast<__nv_bfloat16*>(sk), reinterpret_cast<const __nv_bfloat16*>(k_), srow, H, h, n);
+  auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  if constexpr (S::kStageK) {
+    stage_rows_async(reinterpret_cast<__nv_bfloat16*>(sk), reinterpret_cast<const __nv_bfloat16*>(k_), srow, H, h, n);
+    tile_async_bf16<C, D>(R + S::p2_V, row_v, v_);  // V straight into its phase-2a operand tile
+  }
   {  // Atilde (fp32, padded rows) by 4-byte asynchronous copies; T (hi/lo tile) by a bulk copy
     const size_t cb = (size_t)ci * H + h;
     const float* Ag = ws.At + cb * C * C;
@@ -1236,14 +1250,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   load_gate(sG, LD, g_, srow, H, h, n);
   __syncthreads();
-  cumsum_ref(sG, LD, n, sref, nullptr);
-  tc::cp_async_wait<0>();  // staged k and Atilde
+  cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(R));  // (R's first phase comes later)
+  tc::cp_async_wait<0>();  // staged k, V and Atilde
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   // 16 values of k row r from column c0 on (zero for r >= n)
   auto k16 = [&](int r, int c0, float(&kv)[16]) {
     if constexpr (S::kStageK) {
@@ -1266,8 +1279,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const size_t base = (size_t)ci * H + h;
   float* pdk = ws.pdk + base * C * D;
   float* pdG = ws.pdG + base * C * D;
-  const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = (w >> 2) & 1;
+  const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
   const int myrow = lane < 16 ? 16 * sp + lane : -1;  // M = 64 accumulator row of this thread
+  // 16 gradient values of row r from column c0 on, to where the row's gradients go
+  auto out16 = [&](float* replay_buf, float* tgt_buf, Tout* out, int r, int c0, const float(&v)[16]) {
+    const size_t o = ((size_t)sidx[r] * H + h) * D + c0;
+    if (skind[r] == 0) st16g(replay_buf + o, v);
+    else if (skind[r] == 1) st16g(tgt_buf + o, v);
+    else st16_out(out + o, v);
+  };
   const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
   // TMEM columns
   // dB_k [0, 128) stays in TMEM until the last phase; CS reuses the dB_v columns [128, 256)
@@ -1286,10 +1306,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *tph = R + S::p2_Tp, *tpl = tph + S::CCb, *kbh = R + S::p2_Kb, *kbl = kbh + S::CDb, *vh = R + S::p2_V,
             *vl = vh + S::CDb;
     build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return tval(r, i) * sb[i]; });
-    auto kbf = [&](int i, int c, float x) { return x * expf(sG[i * LD + c]); };
+    auto kbf = [&](int i, int c, float x) { return x * tc::ex2(sG[i * LD + c]); };
     if constexpr (S::kStageK) build_tile_st<C, D, true>(kbh, kbl, reinterpret_cast<const __nv_bfloat16*>(sk), kbf);
     else build_tile_ld<C, D, true, Tin>(kbh, kbl, row_k, kbf);
-    build_tile_ld<C, D, !EX, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
+    if constexpr (!EX) build_tile_ld<C, D, true, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
     ok = run(sy, [&] {
       const uint32_t id = tc::idesc_bf16(C, D, false, true);
       const tc::Op tH{tc::smem_u32(tph), C, false}, tL{tc::smem_u32(tpl), C, false};
@@ -1338,7 +1358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // ---- read dB: dB tile for dA; dv; dk / dG / dbeta contributions
     uint8_t *dbh = R + S::p4_dB, *dbl = dbh + 2 * S::CDb;
-    for (int c0 = grp * 16; c0 < 2 * D; c0 += 32) {
+    for (int c0 = grp * 16; c0 < 2 * D; c0 += 16 * kTcGroups) {
       float v[16];
       tc::tmem_ld16(la + cdB + c0, v);
       if (myrow < 0) continue;
@@ -1349,7 +1369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float kv[16];
         k16(i, c0, kv);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) part = fmaf(v[j], kv[j] * expf(sG[i * LD + c0 + j]), part);
+        for (int j = 0; j < 16; ++j) part = fmaf(v[j], kv[j] * tc::ex2(sG[i * LD + c0 + j]), part);
       } else if (i < n) {
         const int c1 = c0 - D;
         float vv[16], val[16];
@@ -1371,15 +1391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           part = fmaf(v[j], vv[j], part);
           val[j] = sb[i] * v[j];
         }
-        if (i < ch.n_replay) {
-          st16g(ws.rdv + ((size_t)(ch.replay_base + i) * H + h) * D + c1, val);
-        } else {
-          const int tg = t.row_tgt[srow[i]];
-          if (tg >= 0) st16g(ws.tdv + ((size_t)tg * H + h) * D + c1, val);
-          else st16_out(dv_ + ((size_t)srow[i] * H + h) * D + c1, val);
-        }
+        out16(ws.rdv, ws.tdv, dv_, i, c1, val);
       }
-      sdb[((c0 < D ? 0 : 2) + grp) * C + i] += part;  // one slot per (half, warp group)
+      sdb[((c0 < D ? 0 : 1) * kTcGroups + grp) * C + i] += part;  // one slot per (half, warp group)
     }
     uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb;
     ok = run(sy, [&] {
@@ -1391,7 +1405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // ---- dA = -(dB X^T) strict lower; dAt = beta dA (tile); dbeta += rowsum(dA Atilde)
     uint8_t *dah = R + S::p5_dA, *dal = dah + S::CCb;
-    for (int c0 = grp * 16; c0 < C; c0 += 32) {
+    for (int c0 = grp * 16; c0 < C; c0 += 16 * kTcGroups) {
       float v[16];
       tc::tmem_ld16(la + cdA + c0, v);
       if (myrow < 0) continue;
@@ -1404,12 +1418,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         m[j] = sb[r] * dA;
       }
       put16<C, true>(dah, dal, r, c0, m);  // element (r, i)
-      sdb[(4 + grp) * C + r] += part;
+      sdb[(2 * kTcGroups + grp) * C + r] += part;
     }
     // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
     uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
-    auto bff = [&](int i, int c, float x) { return x * expf(sref[c] - sG[i * LD + c]); };
-    auto aff = [&](int r, int c, float x) { return x * expf(sG[r * LD + c] - sref[c]); };
+    auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
+    auto aff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
     if constexpr (S::kStageK) {
       build_tile_st<C, D, true>(bfh, bfl, reinterpret_cast<const __nv_bfloat16*>(sk), bff);
       build_tile_st<C, D, true>(afh, afl, reinterpret_cast<const __nv_bfloat16*>(sk), aff);
@@ -1429,7 +1443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // ---- final: dk, dG = partials + dB_k terms + gated terms; dG staged for the reverse cumulative sum
     float* sdG = reinterpret_cast<float*>(R);  // [C][LD]
-    for (int c0 = grp * 16; c0 < D; c0 += 32) {
+    for (int c0 = grp * 16; c0 < D; c0 += 16 * kTcGroups) {
       float rs[16], cs[16], dbk[16];
       tc::tmem_ld16(la + cRS + c0, rs);
       tc::tmem_ld16(la + cCS + c0, cs);
@@ -1444,45 +1458,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) {
         const int c = c0 + j;
         const float Gr = sG[r * LD + c], G0 = sref[c];
-        const float a = expf(Gr - G0) * rs[j], b = expf(G0 - Gr) * cs[j];
-        const float wb = expf(Gr) * sb[r] * dbk[j];
+        const float a = tc::ex2(Gr - G0) * rs[j], b = tc::ex2(G0 - Gr) * cs[j];
+        const float wb = tc::ex2(Gr) * sb[r] * dbk[j];
         dkv[j] += wb + (a + b);
         sdG[r * LD + c] = r < n ? pg[j] + kv[j] * (wb + (a - b)) : 0.f;
       }
-      if (r < n) {
-        if (r < ch.n_replay) {
-          st16g(ws.rdk + ((size_t)(ch.replay_base + r) * H + h) * D + c0, dkv);
-        } else {
-          const int tg = t.row_tgt[srow[r]];
-          if (tg >= 0) st16g(ws.tdk + ((size_t)tg * H + h) * D + c0, dkv);
-          else st16_out(dk_ + ((size_t)srow[r] * H + h) * D + c0, dkv);
-        }
-      }
+      if (r < n) out16(ws.rdk, ws.tdk, dk_, r, c0, dkv);
     }
     __syncthreads();
-    for (int c = tid; c < D; c += blockDim.x) {
+    // dg = reverse cumulative sum of dG over the chunk's rows: four threads per column, each a
+    // quarter of the rows; the quarters' totals first, then each quarter's running sum from below
+    static_assert(kTcThreads == 4 * D, "four threads per column");
+    float* qsum = sdG + C * LD;  // [4][D]
+    const int c = tid % D, q4 = tid / D, r_lo = 16 * q4;
+    {
+      float a = 0.f;
+#pragma unroll
+      for (int r = r_lo; r < r_lo + 16; ++r) a += sdG[r * LD + c];  // rows >= n hold zeros
+      qsum[q4 * D + c] = a;
+    }
+    __syncthreads();
+    {
       float acc = 0.f;
-      for (int r = n - 1; r >= 0; --r) {
+      for (int q = 3; q > q4; --q) acc += qsum[q * D + c];
+      for (int r = r_lo + 15; r >= r_lo; --r) {
         acc += sdG[r * LD + c];
-        if (r < ch.n_replay) {
-          ws.rdg[((size_t)(ch.replay_base + r) * H + h) * D + c] = acc;
-        } else {
-          const int tg = t.row_tgt[srow[r]];
-          if (tg >= 0) ws.tdg[((size_t)tg * H + h) * D + c] = acc;
-          else dg_[((size_t)srow[r] * H + h) * D + c] = acc;
+        if (r < n) {
+          float* dst = skind[r] == 0 ? ws.rdg : (skind[r] == 1 ? ws.tdg : dg_);
+          dst[((size_t)sidx[r] * H + h) * D + c] = acc;
         }
       }
     }
     for (int r = tid; r < n; r += blockDim.x) {
-      const float db = ((sdb[0 * C + r] + sdb[1 * C + r]) + (sdb[2 * C + r] + sdb[3 * C + r])) +
-                       (sdb[4 * C + r] + sdb[5 * C + r]);
-      if (r < ch.n_replay) {
-        ws.rdb[(size_t)(ch.replay_base + r) * H + h] = db;
-      } else {
-        const int tg = t.row_tgt[srow[r]];
-        if (tg >= 0) ws.tdb[(size_t)tg * H + h] = db;
-        else dbeta_[(size_t)srow[r] * H + h] = db;
-      }
+      float db = 0.f;
+      for (int q = 0; q < 3 * kTcGroups; ++q) db += sdb[q * C + r];
+      float* dst = skind[r] == 0 ? ws.rdb : (skind[r] == 1 ? ws.tdb : dbeta_);
+      dst[(size_t)sidx[r] * H + h] = db;
     }
   }
   tc::fence_before_sync();

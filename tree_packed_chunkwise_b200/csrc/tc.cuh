@@ -9,6 +9,14 @@
 namespace tpc {
 namespace tc {
 
+// 2^x by the hardware approximation (ex2.approx.ftz.f32: relative error about 2^-22, subnormal
+// results flushed to zero)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

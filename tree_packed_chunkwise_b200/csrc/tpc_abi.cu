@@ -238,7 +238,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       if (c1 > c0)
         TPC_LAUNCH("kda_fwd_prep_tc", st,
-                   (kda_fwd_prep_tc<Tin><<<dim3(c1 - c0, H), kThreads, PrepTcSmemT<Tin>::total, st>>>(p.dt, H, k, v, g, b,
+                   (kda_fwd_prep_tc<Tin><<<dim3(c1 - c0, H), kTcThreads, PrepTcSmemT<Tin>::total, st>>>(p.dt, H, k, v, g, b,
                                                                                                   w, c0)));
       TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
       if (s1 > s0)
@@ -256,7 +256,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       TPC_CUDA(cudaEventDestroy(scans[r - 1]));
       if (c1 > c0)
         TPC_LAUNCH("kda_fwd_out_tc", st,
-                   (kda_fwd_out_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, OutTcSmem::total, st>>>(
+                   (kda_fwd_out_tc<Tin, Tout><<<dim3(c1 - c0, H), kTcThreads, OutTcSmem::total, st>>>(
                        p.dt, H, q, k, g, static_cast<Tout*>(io->o), w, c0)));
     }
   } else {
@@ -321,10 +321,10 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
       TPC_CUDA(cudaEventDestroy(scans[i]));
       if (c1 > c0) {
         TPC_LAUNCH("kda_bwd_dq_tc", st,
-                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdqTcSmem::total, st>>>(
+                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(c1 - c0, H), kTcThreads, BdqTcSmem::total, st>>>(
                        p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w, c0)));
         TPC_LAUNCH("kda_bwd_dkv_tc", st,
-                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(c1 - c0, H), kThreads, BdkvTcSmemT<Tin>::total, st>>>(
+                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(c1 - c0, H), kTcThreads, BdkvTcSmemT<Tin>::total, st>>>(
                        p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg,
                        io->dbeta, w, c0)));
       }
