@@ -119,32 +119,70 @@ __device__ __forceinline__ void build_tile_ld(uint8_t* hi, uint8_t* lo, RP rowp,
   }
 }
 
-// Two tiles (hi/lo) of the same rows, values f1(a, b, x) and f2(a, b, x), from one load of the rows
-template <int A, int B, typename T, class RP, class F1, class F2>
-__device__ __forceinline__ void build_tile2_ld(uint8_t* hi1, uint8_t* lo1, uint8_t* hi2, uint8_t* lo2, RP rowp, F1 f1,
-                                               F2 f2) {
-  constexpr int NCH = A * (B / 8), NT = kTcThreads;
-  static_assert(NCH % NT == 0, "tile chunks must be a multiple of the CTA size");
-  constexpr int IT = NCH / NT;
-  float x[IT][8];
+// The 16-byte pieces of a tile's rows (the element -> thread map of build_tile_ld), loaded early into
+// registers (raw_ld) and converted into tiles later (build_tile_raw, build_tile2_raw), so that the
+// loads overlap other work
+template <typename T, int A, int B>
+struct RawTile {
+  static constexpr int IT = A * (B / 8) / kTcThreads, Q = sizeof(T) / 2;  // uint4 per 8 values
+  uint4 u[IT][Q];
+};
+template <typename T, int A, int B, class RP>
+__device__ __forceinline__ void raw_ld(RawTile<T, A, B>& rt, RP rowp) {
+  using RT = RawTile<T, A, B>;
 #pragma unroll
-  for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * NT, a = e % A, b0 = (e / A) * 8;
+  for (int it = 0; it < RT::IT; ++it) {
+    const int e = threadIdx.x + it * kTcThreads, a = e % A, b0 = (e / A) * 8;
     const T* p = rowp(a);
-    if (p) ld8(p + b0, x[it]);
-    else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) x[it][j] = 0.f;
+    for (int q = 0; q < RT::Q; ++q)
+      rt.u[it][q] = p ? __ldg(reinterpret_cast<const uint4*>(p + b0) + q) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+template <typename T>
+__device__ __forceinline__ void raw_get(const uint4* u, float (&x)[8]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(&u[0]), b = *reinterpret_cast<const float4*>(&u[1]);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else {
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u[0]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(b2[j]);
+      x[2 * j] = f.x;
+      x[2 * j + 1] = f.y;
     }
   }
+}
+template <int A, int B, typename T, class F>
+__device__ __forceinline__ void build_tile_raw(uint8_t* hi, uint8_t* lo, const RawTile<T, A, B>& rt, F f) {
+  using RT = RawTile<T, A, B>;
 #pragma unroll
-  for (int it = 0; it < IT; ++it) {
-    const int e = threadIdx.x + it * NT, a = e % A, b0 = (e / A) * 8;
+  for (int it = 0; it < RT::IT; ++it) {
+    const int e = threadIdx.x + it * kTcThreads, a = e % A, b0 = (e / A) * 8;
+    float x[8];
+    raw_get<T>(rt.u[it], x);
+    __align__(16) __nv_bfloat16 hh[8], ll[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) split_bf16(f(a, b0 + j, x[j]), hh[j], ll[j]);
+    *reinterpret_cast<uint4*>(hi + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(hh);
+    *reinterpret_cast<uint4*>(lo + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(ll);
+  }
+}
+template <int A, int B, typename T, class F1, class F2>
+__device__ __forceinline__ void build_tile2_raw(uint8_t* hi1, uint8_t* lo1, uint8_t* hi2, uint8_t* lo2,
+                                                const RawTile<T, A, B>& rt, F1 f1, F2 f2) {
+  using RT = RawTile<T, A, B>;
+#pragma unroll
+  for (int it = 0; it < RT::IT; ++it) {
+    const int e = threadIdx.x + it * kTcThreads, a = e % A, b0 = (e / A) * 8;
+    float x[8];
+    raw_get<T>(rt.u[it], x);
     __align__(16) __nv_bfloat16 h1[8], l1[8], h2[8], l2[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      split_bf16(f1(a, b0 + j, x[it][j]), h1[j], l1[j]);
-      split_bf16(f2(a, b0 + j, x[it][j]), h2[j], l2[j]);
+      split_bf16(f1(a, b0 + j, x[j]), h1[j], l1[j]);
+      split_bf16(f2(a, b0 + j, x[j]), h2[j], l2[j]);
     }
     const uint32_t off = cm_off(a, b0, A);
     *reinterpret_cast<uint4*>(hi1 + off) = *reinterpret_cast<const uint4*>(h1);
@@ -154,25 +192,31 @@ __device__ __forceinline__ void build_tile2_ld(uint8_t* hi1, uint8_t* lo1, uint8
   }
 }
 
-// Gate rows of the chunk into G (fp32, pitch LD): every thread issues its 16-byte loads first;
-// neighbouring threads take neighbouring rows (conflict-free stores).  Rows >= n are zero.
+// Gate rows of the chunk into G (fp32, pitch LD) in two steps, so that a kernel issues these loads
+// before its larger copies and stores them once they arrive: gate_ld (16-byte loads into registers)
+// and gate_st (neighbouring threads take neighbouring rows: conflict-free stores).  Rows >= n are zero.
+struct GateRegs {
+  float x[kTcC * (kTcD / 8) / kTcThreads][8];
+};
 template <typename T>
-__device__ __forceinline__ void load_gate(float* G, int LD, const T* g_, const int* rows, int H, int h, int n) {
-  constexpr int NCH = kTcC * (kTcD / 8), IT = NCH / kTcThreads;
-  float x[IT][8];
+__device__ __forceinline__ void gate_ld(GateRegs& gr, const T* g_, const int* rows, int H, int h, int n) {
+  constexpr int IT = kTcC * (kTcD / 8) / kTcThreads;
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const int e = threadIdx.x + it * kTcThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
-    if (a < n) ld8(g_ + ((size_t)rows[a] * H + h) * kTcD + b0, x[it]);
+    if (a < n) ld8(g_ + ((size_t)rows[a] * H + h) * kTcD + b0, gr.x[it]);
     else
 #pragma unroll
-      for (int j = 0; j < 8; ++j) x[it][j] = 0.f;
+      for (int j = 0; j < 8; ++j) gr.x[it][j] = 0.f;
   }
+}
+__device__ __forceinline__ void gate_st(float* G, int LD, const GateRegs& gr) {
+  constexpr int IT = kTcC * (kTcD / 8) / kTcThreads;
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const int e = threadIdx.x + it * kTcThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) G[a * LD + b0 + j] = x[it][j];
+    for (int j = 0; j < 8; ++j) G[a * LD + b0 + j] = gr.x[it][j];
   }
 }
 
@@ -247,6 +291,21 @@ __device__ __forceinline__ void tile_async_bf16(uint8_t* hi, RP rowp, const void
   tc::cp_async_commit();
 }
 
+// 8 values (a, b0 .. b0 + 7) of a K-major hi/lo tile in shared memory, as fp32 (hi + lo)
+template <int A>
+__device__ __forceinline__ void tile8(const uint8_t* hi, const uint8_t* lo, int a, int b0, float (&v)[8]) {
+  const uint32_t off = cm_off(a, b0, A);
+  const uint4 hq = *reinterpret_cast<const uint4*>(hi + off), lq = *reinterpret_cast<const uint4*>(lo + off);
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
+  const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lq);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 x = __bfloat1622float2(h2[k]), y = __bfloat1622float2(l2[k]);
+    v[2 * k] = x.x + y.x;
+    v[2 * k + 1] = x.y + y.y;
+  }
+}
+
 // 16 values (a, b0 .. b0 + 15) of a K-major hi/lo tile in shared memory, as fp32 (hi + lo)
 template <int A>
 __device__ __forceinline__ void tile16(const uint8_t* hi, const uint8_t* lo, int a, int b0, float (&v)[16]) {
@@ -261,6 +320,25 @@ __device__ __forceinline__ void tile16(const uint8_t* hi, const uint8_t* lo, int
       const float2 x = __bfloat1622float2(h2[k]), y = __bfloat1622float2(l2[k]);
       v[8 * half + 2 * k] = x.x + y.x;
       v[8 * half + 2 * k + 1] = x.y + y.y;
+    }
+  }
+}
+
+// 8 consecutive values of a staged row as fp32
+template <typename T>
+__device__ __forceinline__ void staged8(const T* st, int r, int c0, float (&v)[8]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 u = *reinterpret_cast<const float4*>(st + r * kStagePitch + c0);
+    const float4 u2 = *reinterpret_cast<const float4*>(st + r * kStagePitch + c0 + 4);
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w; v[4] = u2.x; v[5] = u2.y; v[6] = u2.z; v[7] = u2.w;
+  } else {
+    const uint4 u = *reinterpret_cast<const uint4*>(st + r * kStagePitch + c0);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(b2[k]);
+      v[2 * k] = f.x;
+      v[2 * k + 1] = f.y;
     }
   }
 }
@@ -289,6 +367,25 @@ __device__ __forceinline__ void staged16(const T* st, int r, int c0, float (&v)[
   }
 }
 
+__device__ __forceinline__ void ld8g(const float* p, float (&v)[8]) {
+  const float4 u = *reinterpret_cast<const float4*>(p), u2 = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w; v[4] = u2.x; v[5] = u2.y; v[6] = u2.z; v[7] = u2.w;
+}
+__device__ __forceinline__ void st8g(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <typename T>
+__device__ __forceinline__ void st8_out(T* p, const float* v) {
+  if constexpr (sizeof(T) == 4) {
+    st8g(reinterpret_cast<float*>(p), v);
+  } else {
+    __align__(16) __nv_bfloat16 b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) b[j] = __float2bfloat16_rn(v[j]);
+    *reinterpret_cast<uint4*>(p) = *reinterpret_cast<const uint4*>(b);
+  }
+}
 __device__ __forceinline__ void ld16g(const float* p, float (&v)[16]) {
 #pragma unroll
   for (int j = 0; j < 16; j += 4) {
@@ -313,18 +410,58 @@ __device__ __forceinline__ void st16_out(T* p, const float* v) {
   }
 }
 
-// Reads an M x N fp32 accumulator (N a multiple of 16) starting at TMEM column col0:
-// f(m, n0, v) gets 16 consecutive columns n0 .. n0+15 of row m.  Warp w reads the lanes of
-// sub-partition w % 4; the kTcGroups groups of four warps take interleaved 16-column chunks.
+// The rows of an M = 64 accumulator sit in TMEM lanes 0-15 of each sub-partition.  After a 16-column
+// read, lanes 16-31 take columns 8-15 of the row of lane - 16 (one shuffle per value), so that every
+// lane of the warp handles 8 values: row 16 * sp + lane % 16, columns 8 * (lane / 16) + 0 .. 7.
+__device__ __forceinline__ void share8u(const uint32_t (&v)[16], float (&w)[8]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t x = __shfl_sync(0xffffffffu, v[8 + j], lane & 15);
+    w[j] = __uint_as_float(lane < 16 ? v[j] : x);
+  }
+}
+__device__ __forceinline__ void share8(const float (&v)[16], float (&w)[8]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float x = __shfl_sync(0xffffffffu, v[8 + j], lane & 15);
+    w[j] = lane < 16 ? v[j] : x;
+  }
+}
+
+// Reads an M x N fp32 accumulator (N a multiple of 16) starting at TMEM column col0.  Warp w reads
+// the lanes of sub-partition w % 4; the kTcGroups groups of four warps take interleaved 16-column
+// chunks.  M = 128: f(m, n0, v) gets 16 consecutive columns n0 .. n0+15 of row m.  M = 64: every lane
+// takes 8 of them (share8): f(m, n0, v) gets columns n0 .. n0+7.
 template <int M, int N, class F>
 __device__ __forceinline__ void acc_read(uint32_t tbase, int col0, F f) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, sp = w & 3, grp = w >> 2;
   for (int c = grp * 16; c < N; c += 16 * kTcGroups) {
     float v[16];
     tmem_ld16(tbase + ((uint32_t)(32 * sp) << 16) + (uint32_t)(col0 + c), v);
-    const int m = (M == 128) ? 32 * sp + lane : (lane < 16 ? 16 * sp + lane : -1);
-    if (m >= 0) f(m, c, v);
+    if constexpr (M == 128) {
+      f(32 * sp + lane, c, v);
+    } else {
+      float h8[8];
+      share8(v, h8);
+      f(16 * sp + (lane & 15), c + 8 * (lane >> 4), h8);
+    }
   }
+}
+
+// Writes 8 values into a K-major/MN-major tile as bf16 hi/lo at (a, b0..b0+7) (b0 a multiple of 8).
+template <int A, bool SPLIT>
+__device__ __forceinline__ void put8(uint8_t* hi, uint8_t* lo, int a, int b0, const float* v) {
+  __align__(16) __nv_bfloat16 h[8];
+  __align__(16) __nv_bfloat16 l[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (SPLIT) split_bf16(v[j], h[j], l[j]);
+    else h[j] = __float2bfloat16_rn(v[j]);
+  }
+  *reinterpret_cast<uint4*>(hi + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(h);
+  if (SPLIT) *reinterpret_cast<uint4*>(lo + cm_off(a, b0, A)) = *reinterpret_cast<const uint4*>(l);
 }
 
 // Writes 16 values (one row chunk) into a K-major/MN-major tile as bf16 hi/lo at (a, b0..b0+15).
@@ -499,58 +636,29 @@ __device__ __forceinline__ void mma4(uint32_t d, const Op& ah, const Op& al, con
 }
 
 // T = (I + L)^{-1} for strictly lower-triangular L (64 x 64, pitch LC), fp32, in smem.
-// Diagonal 16 x 16 blocks: (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) (N^16 = 0);
+// Diagonal 16 x 16 blocks by forward substitution, one thread per block column (64 threads) with the
+// column in registers: T_pp[r][c] = [r == c] - sum_{k < r} L_pp[r][k] T_pp[k][c];
 // off-diagonal blocks: T_pq = -T_pp sum_{q <= s < p} L_ps T_sq, by increasing p - q.
-// W1, W2: 4 scratch 16 x 16 blocks each (pitch 17).
+// Row r of T depends on rows <= r of L only.  W1: 4 scratch 16 x 16 blocks (pitch 17).
 template <int LC>
-__device__ __forceinline__ void block_inverse(float* T, const float* L, float* W1, float* W2) {
-  constexpr int B = 16, P = 17, BB = B * P;
+__device__ __forceinline__ void block_inverse(float* T, const float* L, float* W1) {
+  constexpr int P = 17, BB = 16 * P;
   const int tid = threadIdx.x;
-  // diagonal blocks, all four at once: element e -> (block, row, col)
-  auto blk = [&](int e, int& p, int& r, int& c) { p = e >> 8; r = (e >> 4) & 15; c = e & 15; };
-  // W1_p = N_p (strict lower), T_pp = I - N_p
-  for (int e = tid; e < 4 * 256; e += blockDim.x) {
-    int p, r, c;
-    blk(e, p, r, c);
-    const float n = (c < r) ? L[(16 * p + r) * LC + 16 * p + c] : 0.f;
-    W1[p * BB + r * P + c] = n;
-    T[(16 * p + r) * LC + 16 * p + c] = (r == c ? 1.f : 0.f) - n;
+  if (tid < 64) {
+    const int p = tid >> 4, c = tid & 15;
+    const float* Lp = L + (16 * p) * LC + 16 * p;
+    float col[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float acc = (r == c) ? 1.f : 0.f;
+#pragma unroll
+      for (int k = 0; k < r; ++k) acc = fmaf(-Lp[r * LC + k], col[k], acc);
+      col[r] = acc;
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) T[(16 * p + r) * LC + 16 * p + c] = col[r];
   }
   __syncthreads();
-  for (int level = 0; level < 3; ++level) {
-    // W2 = W1 * W1  (N^2, N^4, N^8)
-    for (int e = tid; e < 4 * 256; e += blockDim.x) {
-      int p, r, c;
-      blk(e, p, r, c);
-      float acc = 0.f;
-      for (int k = c + 1; k < r; ++k) acc = fmaf(W1[p * BB + r * P + k], W1[p * BB + k * P + c], acc);
-      W2[p * BB + r * P + c] = acc;
-    }
-    __syncthreads();
-    // T_pp <- T_pp (I + W2): row r of T times (I + W2)
-    float out[4];
-    int cnt = 0;
-    for (int e = tid; e < 4 * 256; e += blockDim.x, ++cnt) {
-      int p, r, c;
-      blk(e, p, r, c);
-      float acc = T[(16 * p + r) * LC + 16 * p + c];
-      for (int k = c + 1; k <= r; ++k) acc = fmaf(T[(16 * p + r) * LC + 16 * p + k], W2[p * BB + k * P + c], acc);
-      out[cnt] = acc;
-    }
-    __syncthreads();
-    cnt = 0;
-    for (int e = tid; e < 4 * 256; e += blockDim.x, ++cnt) {
-      int p, r, c;
-      blk(e, p, r, c);
-      T[(16 * p + r) * LC + 16 * p + c] = out[cnt];
-    }
-    for (int e = tid; e < 4 * 256; e += blockDim.x) {
-      int p, r, c;
-      blk(e, p, r, c);
-      W1[p * BB + r * P + c] = W2[p * BB + r * P + c];
-    }
-    __syncthreads();
-  }
   // off-diagonal blocks by distance d = p - q: T_pq = -T_pp * (sum_s L_ps T_sq)
   for (int d = 1; d < 4; ++d) {
     const int nb = 4 - d;  // blocks (p, p - d), p = d .. 3
@@ -653,7 +761,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* sA = reinterpret_cast<float*>(tsm + S::A);
   float* sT = reinterpret_cast<float*>(tsm + S::T);
   float* sW1 = reinterpret_cast<float*>(tsm + S::W1);
-  float* sW2 = reinterpret_cast<float*>(tsm + S::W2);
   float* sb = reinterpret_cast<float*>(tsm + S::vec);
   float* sref = sb + C;
   uint8_t* tl = tsm + S::tiles;
@@ -673,12 +780,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // bf16: the chunk's k and v rows into shared memory while the gates load and accumulate
   [[maybe_unused]] __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
   [[maybe_unused]] __nv_bfloat16* sv = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
+  GateRegs gr;
+  gate_ld(gr, g_, srow, H, h, n);  // gates and beta first
+  const float bv = tid < n ? to_f(beta_[(size_t)srow[tid] * H + h]) : 0.f;
   if constexpr (EX) {
     stage_rows_async(sk, k_, srow, H, h, n);
     stage_rows_async(sv, v_, srow, H, h, n);
   }
-  for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
-  load_gate(sG, LD, g_, srow, H, h, n);
+  gate_st(sG, LD, gr);
+  if (tid < C) sb[tid] = bv;
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, ws.status, reinterpret_cast<float*>(tl));  // (tiles not yet in use)
   if constexpr (EX) tc::cp_async_wait<0>();
@@ -705,19 +815,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok) {
       float* Ag = ws.At + ((size_t)ci * H + h) * C * C;  // kept for the backward
       acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
-        float a[16];
-        for (int j = 0; j < 16; ++j) {
+        float a[8];
+        for (int j = 0; j < 8; ++j) {
           const int i = i0 + j;
           a[j] = (i < r) ? v[j] : 0.f;
           sA[r * LC + i] = sb[r] * a[j];  // L = diag(beta) Atilde, strict lower
         }
-        st16g(Ag + r * C + i0, a);
+        st8g(Ag + r * C + i0, a);
       });
     }
   }
   if (ok) {
     __syncthreads();
-    block_inverse<LC>(sT, sA, sW1, sW2);
+    block_inverse<LC>(sT, sA, sW1);
     // T as a hi/lo tile (element (r, i) at cm_off(r, i, C)) for the backward, built where L was
     uint8_t *ttH = reinterpret_cast<uint8_t*>(sA), *ttL = ttH + S::CCb;
     build_tile<C, C, true>(ttH, ttL, [&](int r, int i) { return sT[r * LC + i]; });
@@ -745,8 +855,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               *khl = tl + 5 * S::CDb;
       // W and U' as hi/lo tiles, element (i, c) at cm_off(i, c, C): the operands of this phase and,
       // stored as they are, of the output and backward kernels
-      acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) { put16<C, true>(wth, wtl, r, c0, v); });
-      acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) { put16<C, true>(uth, utl, r, c0, v); });
+      acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) { put8<C, true>(wth, wtl, r, c0, v); });
+      acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) { put8<C, true>(uth, utl, r, c0, v); });
       const float* gC = sG + (n - 1) * LD;
       k_tile(khh, khl, [&](int i, int c, float x) { return x * tc::ex2(gC[c] - sG[i * LD + c]); });
       ok = run(sy, [&] {
@@ -826,28 +936,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc::mbar_init(&bar, 1);
     tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  GateRegs gr;
+  gate_ld(gr, g_, srow, H, h, n);  // gates, q and k first, then the workspace tiles
+  RawTile<Tin, C, D> rq, rk;
+  raw_ld(rq, row_q);
+  raw_ld(rk, row_k);
+  if (tid == 0) {
     ld_expect(ld, kStateTileBytes + kCDTileBytes);
     ld_state_tile(ld, s0h, s0l, ws.S0, base);  // the chunk-start state, as the scan left it
     ld_cd_tile(ld, tsm + S::Wq, tsm + S::Wq + S::CDb, ws.W, base);  // W, as the prep kernel left it
   }
-  __syncthreads();
-  load_gate(sG, LD, g_, srow, H, h, n);
+  gate_st(sG, LD, gr);
   __syncthreads();
   uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb;
   cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(qbh));  // (the Qbar tile comes later)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
-  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   // TMEM: P [0,64), W S0 [64,192), O [192,320), P W [320,448)
   uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
   uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb;
   // qf = q e^{G - ref} and Qbar = q e^G from one load of q; bf = k e^{ref - G}
-  build_tile2_ld<C, D, Tin>(
-      qfh, qfl, qbh, qbl, row_q, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); },
+  build_tile2_raw<C, D, Tin>(
+      qfh, qfl, qbh, qbl, rq, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); },
       [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c]); });
-  build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
+  build_tile_raw<C, D, Tin>(bfh, bfl, rk, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
   const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
   bool ok = ld_wait(ld);
   ok = ok && run(sy, [&] {
@@ -864,18 +981,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ld_cd_tile(ld, uh, ul, ws.U, base);
     }
     acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
-      float m[16];
-      for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
-      put16<C, true>(ph, pl, r, i0, m);  // kept (as this tile) for the backward
+      float m[8];
+      for (int j = 0; j < 8; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+      put8<C, true>(ph, pl, r, i0, m);  // kept (as this tile) for the backward
     });
     ok = ld_wait(ld);
   }
   if (ok) {
     acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
-      float u[16];
-      tile16<C>(uh, ul, i, j0, u);  // U'
-      for (int j = 0; j < 16; ++j) u[j] -= v[j];
-      put16<C, true>(uh, ul, i, j0, u);  // U, element (i, j): MN-major (k = i); kept for the backward
+      float u[8];
+      tile8<C>(uh, ul, i, j0, u);  // U'
+      for (int j = 0; j < 8; ++j) u[j] -= v[j];
+      put8<C, true>(uh, ul, i, j0, u);  // U, element (i, j): MN-major (k = i); kept for the backward
     });
     ok = run(sy, [&] {
       store_cc_tile(ws.Pm, base, ph, pl);
@@ -892,15 +1009,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     });
     if (ok) {
       acc_read<C, D>(tb, 192, [&](int r, int j0, const float* v) {
-        if (r >= ch.n_replay && r < n) st16_out(o_ + ((size_t)srow[r] * H + h) * D + j0, v);
+        if (r >= ch.n_replay && r < n) st8_out(o_ + ((size_t)srow[r] * H + h) * D + j0, v);
       });
       // Qeff = Qbar - P W (element (r, c)) into the S0 buffer, which the products above consumed
       uint8_t *eh = s0h, *el = s0h + S::CDb;
       acc_read<C, D>(tb, 320, [&](int r, int c0, const float* v) {
-        float e[16];
-        tile16<C>(qbh, qbl, r, c0, e);  // Qbar
-        for (int j = 0; j < 16; ++j) e[j] -= v[j];
-        put16<C, true>(eh, el, r, c0, e);
+        float e[8];
+        tile8<C>(qbh, qbl, r, c0, e);  // Qbar
+        for (int j = 0; j < 8; ++j) e[j] -= v[j];
+        put8<C, true>(eh, el, r, c0, e);
       });
       tc::fence_async_smem();
       __syncthreads();
@@ -924,8 +1041,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 struct BdqTcSmem {
   static constexpr int C = kTcC, D = kTcD, LD = D + 1;
   static constexpr size_t G = 0;
-  static constexpr size_t vec = G + sizeof(float) * C * LD;  // ref[D]
-  static constexpr size_t tiles = (vec + sizeof(float) * D + 1023) & ~size_t(1023);
+  static constexpr size_t vec = G + sizeof(float) * C * LD;  // ref[D], e0[D] = 2^{G_0}, eC0[D] = 2^{G_C - G_0}
+  static constexpr size_t tiles = (vec + sizeof(float) * 3 * D + 1023) & ~size_t(1023);
   static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2, DDb = size_t(D) * D * 2;
   // phase 1: dO (K-major) | U (K-major) | S0 (K-major D x D); phase 2: dS in the S0 slot;
   // phase 3: dP | bf (MN) | qf (MN) over the dO/U/S0 space; epilogue row buffer (C x LD fp32) after.
@@ -971,12 +1088,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc::mbar_init(&bar, 1);
     tc::mbar_init(&bar_ld, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  GateRegs gr;
+  gate_ld(gr, g_, srow, H, h, n);  // gates first, then the workspace tiles and the row gathers
+  if (tid == 0) {
     ld_expect(ld, kStateTileBytes + kCDTileBytes + kCCTileBytes);
     ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
     ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
     ld_cc_tile(ld, tsm + S::Pt, tsm + S::Pt + S::CCb, ws.Pm, base);  // P, as the output kernel left it
   }
-  __syncthreads();
   // bf16: the chunk's q and k rows into shared memory while the gates load and accumulate
   [[maybe_unused]] __nv_bfloat16* stq = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
   [[maybe_unused]] __nv_bfloat16* stk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
@@ -990,9 +1111,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     stage_rows_async(stk, k_, srow, H, h, n);
     tile_async_bf16<C, D>(doh, row_do, do_);
   }
-  load_gate(sG, LD, g_, srow, H, h, n);
+  gate_st(sG, LD, gr);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(tsm + S::Scr));
+  float* se0 = sref + D;  // per channel 2^{G_0} and 2^{G_C - G_0} (ready long before the epilogue)
+  float* seC0 = se0 + D;
+  for (int c = tid; c < D; c += blockDim.x) {
+    se0[c] = tc::ex2(sref[c]);
+    seC0[c] = tc::ex2(sG[(n - 1) * LD + c] - sref[c]);
+  }
   if constexpr (EX) tc::cp_async_wait<0>();
   __syncthreads();
   tc::fence_after_sync();
@@ -1035,7 +1162,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok) {
       // dU = dU0 + Khat dS as a hi/lo tile (element (i, j) at cm_off(i, j, C), in the consumed Khat
       // slot) for the dk / dv kernel
-      acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) { put16<C, true>(doh, dol, i, j0, v); });
+      acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) { put8<C, true>(doh, dol, i, j0, v); });
       tc::fence_async_smem();
       __syncthreads();
       if (tid == 0) {
@@ -1049,9 +1176,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *ql = qh + S::CDb;
   if (ok) {
     acc_read<C, C>(tb, cCS, [&](int r, int i0, const float* v) {
-      float m[16];
-      for (int j = 0; j < 16; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
-      put16<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
+      float m[8];
+      for (int j = 0; j < 8; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+      put8<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
     });
     auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
     auto qff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
@@ -1087,31 +1214,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     __syncthreads();
     const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
-    const int r = lane < 16 ? 16 * sp + lane : -1;
+    const int r = 16 * sp + (lane & 15);  // accumulator row; this lane's 8 columns: share8
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
-    for (int c0 = grp * 16; c0 < D; c0 += 16 * kTcGroups) {
-      float tq[16], t1[16], rs[16], cs[16];
-      tc::tmem_ld16(la + cTq + c0, tq);
-      tc::tmem_ld16(la + cT1 + c0, t1);
-      tc::tmem_ld16(la + cRS + c0, rs);
-      tc::tmem_ld16(la + cCS + c0, cs);
-      if (r < 0) continue;
-      float qv[16], kv[16], dq[16], dk[16], dG[16];
-      staged16(sq, r, c0, qv);
-      staged16(sk, r, c0, kv);
+    for (int cc = grp * 16; cc < D; cc += 16 * kTcGroups) {
+      float tq[8], t1[8], rs[8], cs[8];
+      {
+        uint32_t a0[16], a1[16], a2[16], a3[16];  // four loads in flight, one wait
+        tc::tmem_ld16_nowait(la + cTq + cc, a0);
+        tc::tmem_ld16_nowait(la + cT1 + cc, a1);
+        tc::tmem_ld16_nowait(la + cRS + cc, a2);
+        tc::tmem_ld16_nowait(la + cCS + cc, a3);
+        tc::tmem_wait_ld();
+        tc::tmem_regs16(a0);
+        tc::tmem_regs16(a1);
+        tc::tmem_regs16(a2);
+        tc::tmem_regs16(a3);
+        share8u(a0, tq);
+        share8u(a1, t1);
+        share8u(a2, rs);
+        share8u(a3, cs);
+      }
+      const int c0 = cc + 8 * (lane >> 4);
+      float qv[8], kv[8], dq[8], dk[8], dG[8];
+      staged8(sq, r, c0, qv);
+      staged8(sk, r, c0, kv);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int c = c0 + j;
-        const float Gr = sG[r * LD + c], G0 = sref[c], GC = sG[(n - 1) * LD + c];
-        dq[j] = tc::ex2(Gr) * tq[j] + tc::ex2(Gr - G0) * rs[j];
-        const float dks = tc::ex2(GC - Gr) * t1[j];
-        dk[j] = dks + tc::ex2(G0 - Gr) * cs[j];
+        // a = 2^{G_r - G_0} (bounded by the chunk's decay check), 1/a = 2^{G_0 - G_r};
+        // 2^{G_r} = 2^{G_0} a and 2^{G_C - G_r} = 2^{G_C - G_0} / a
+        const float a = tc::ex2(sG[r * LD + c] - sref[c]), ia = tc::rcp_approx(a);
+        dq[j] = a * fmaf(se0[c], tq[j], rs[j]);
+        const float dks = seC0[c] * ia * t1[j];
+        dk[j] = fmaf(ia, cs[j], dks);
         dG[j] = qv[j] * dq[j] - kv[j] * dk[j];
         sbuf[r * LD + c] = r < n ? kv[j] * dks : 0.f;
       }
-      st16g(pdk + r * D + c0, dk);
-      st16g(pdG + r * D + c0, dG);
-      if (r >= ch.n_replay && r < n) st16_out(dq_ + ((size_t)srow[r] * H + h) * D + c0, dq);
+      st8g(pdk + r * D + c0, dk);
+      st8g(pdG + r * D + c0, dG);
+      if (r >= ch.n_replay && r < n) st8_out(dq_ + ((size_t)srow[r] * H + h) * D + c0, dq);
     }
     __syncthreads();
     // per column c: sum over rows of the row buffer and sum_j dS_cj S0_cj, each split over four
@@ -1155,8 +1296,9 @@ struct BdkvTcSmemT {
   static constexpr int C = kTcC, D = kTcD, LD = D + 1, LC = C + 1;
   static constexpr size_t G = 0;
   static constexpr size_t At = G + sizeof(float) * C * LD;        // Atilde fp32 [C][LC]
-  static constexpr size_t vec = At + sizeof(float) * C * LC;      // beta[C], ref[D], dbeta parts[3][groups][C]
-  static constexpr size_t Ks = (vec + sizeof(float) * (C + D + 3 * kTcGroups * C) + 15) & ~size_t(15);  // staged k
+  // beta[C], ref[D], dbeta parts[3][groups][C], e0[D] = 2^{G_0}
+  static constexpr size_t vec = At + sizeof(float) * C * LC;
+  static constexpr size_t Ks = (vec + sizeof(float) * (C + 2 * D + 3 * kTcGroups * C) + 15) & ~size_t(15);  // staged k
   static constexpr size_t Tt = (Ks + (kStageK ? sizeof(Tin) * C * tck::kStagePitch : 0) + 1023) & ~size_t(1023);  // T tile
   static constexpr size_t CCb = size_t(C) * C * 2, CDb = size_t(C) * D * 2, DDb = size_t(D) * D * 2;
   static constexpr size_t R = Tt + 2 * CCb;
@@ -1167,11 +1309,11 @@ struct BdkvTcSmemT {
   static constexpr size_t inv_L = 0, inv_T = inv_L + sizeof(float) * C * LC;           // fp32 L, T
   static constexpr size_t inv_W1 = inv_T + sizeof(float) * C * LC, inv_W2 = inv_W1 + sizeof(float) * 4 * 16 * 17;
   static constexpr size_t p2_Tp = 44 * 1024, p2_Kb = p2_Tp + 2 * CCb, p2_V = p2_Kb + 2 * CDb;  // T', Kbar, V
-  static constexpr size_t p2_dU = 0, p2_S0 = 2 * CDb;                                  // dU (K), S0 (K)
+  static constexpr size_t p2_S0 = 0;                                                   // S0 (K); dU in dX
   static constexpr size_t p3_X = 0, p3_dX = 4 * CDb;                                   // X (K, C x 2D), dX (MN)
   static constexpr size_t p4_dB = 4 * CDb;                                             // dB (K, C x 2D)
   static constexpr size_t p5_dA = 0, p5_bf = 2 * CCb, p5_af = p5_bf + 2 * CDb;         // dAt, bf (MN), af (MN)
-  static_assert(p2_V + 2 * CDb <= Rbytes && p2_S0 + 2 * DDb <= Rbytes && p3_dX + 4 * CDb <= Rbytes, "R");
+  static_assert(p2_V + 2 * CDb <= Rbytes && p2_S0 + 2 * DDb <= p3_dX && p3_dX + 4 * CDb <= Rbytes, "R");
   static_assert(inv_W2 + sizeof(float) * 4 * 16 * 17 <= p2_Tp, "inverse scratch overlaps T'");
   static_assert(total <= 227 * 1024, "shared memory");
 };
@@ -1230,7 +1372,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  for (int i = tid; i < C; i += blockDim.x) sb[i] = i < n ? to_f(beta_[(size_t)srow[i] * H + h]) : 0.f;
+  GateRegs gr;
+  gate_ld(gr, g_, srow, H, h, n);  // gates and beta first, then the copies
+  const float bv = tid < n ? to_f(beta_[(size_t)srow[tid] * H + h]) : 0.f;
   for (int e = tid; e < 3 * kTcGroups * C; e += blockDim.x) sdb[e] = 0.f;
   Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
   auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
@@ -1248,45 +1392,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ld_cc_tile(ld, tTh, tTl, ws.Tm, cb);
     }
   }
-  load_gate(sG, LD, g_, srow, H, h, n);
+  gate_st(sG, LD, gr);
+  if (tid < C) sb[tid] = bv;
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(R));  // (R's first phase comes later)
+  float* se0 = sdb + 3 * kTcGroups * C;  // per channel 2^{G_0}
+  for (int c = tid; c < D; c += blockDim.x) se0[c] = tc::ex2(sref[c]);
   tc::cp_async_wait<0>();  // staged k, V and Atilde
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  // 16 values of k row r from column c0 on (zero for r >= n)
-  auto k16 = [&](int r, int c0, float(&kv)[16]) {
+  // 8 values of k row r from column c0 on (zero for r >= n)
+  auto k8 = [&](int r, int c0, float(&kv)[8]) {
     if constexpr (S::kStageK) {
-      staged16(sk, r, c0, kv);
+      staged8(sk, r, c0, kv);
     } else if (r < n) {
-      const Tin* p = k_ + ((size_t)srow[r] * H + h) * D + c0;
-      float a[8], b[8];
-      ld8(p, a);
-      ld8(p + 8, b);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        kv[j] = a[j];
-        kv[j + 8] = b[j];
-      }
+      ld8(k_ + ((size_t)srow[r] * H + h) * D + c0, kv);
     } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) kv[j] = 0.f;
+      for (int j = 0; j < 8; ++j) kv[j] = 0.f;
     }
   };
   const size_t base = (size_t)ci * H + h;
   float* pdk = ws.pdk + base * C * D;
   float* pdG = ws.pdG + base * C * D;
   const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
-  const int myrow = lane < 16 ? 16 * sp + lane : -1;  // M = 64 accumulator row of this thread
-  // 16 gradient values of row r from column c0 on, to where the row's gradients go
-  auto out16 = [&](float* replay_buf, float* tgt_buf, Tout* out, int r, int c0, const float(&v)[16]) {
+  const int myrow = 16 * sp + (lane & 15);  // M = 64 accumulator row; this lane's 8 columns: share8
+  const int half8 = 8 * (lane >> 4);
+  // 8 gradient values of row r from column c0 on, to where the row's gradients go
+  auto out8 = [&](float* replay_buf, float* tgt_buf, Tout* out, int r, int c0, const float* v) {
     const size_t o = ((size_t)sidx[r] * H + h) * D + c0;
-    if (skind[r] == 0) st16g(replay_buf + o, v);
-    else if (skind[r] == 1) st16g(tgt_buf + o, v);
-    else st16_out(out + o, v);
+    if (skind[r] == 0) st8g(replay_buf + o, v);
+    else if (skind[r] == 1) st8g(tgt_buf + o, v);
+    else st8_out(out + o, v);
   };
   const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
   // TMEM columns
@@ -1320,8 +1460,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     });
   }
   if (ok) {
-    // ---- phase 2b: dW' = dU S0^T
-    uint8_t *duh = R + S::p2_dU, *dul = duh + S::CDb, *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
+    // ---- phase 2b: dW' = dU S0^T.  dU is loaded where phase 3's dX keeps its columns [D, 2D) (a
+    // C x D sub-tile of the K-major C x 2D layout is itself a C x D K-major tile), S0 where X goes.
+    uint8_t *dxh0 = R + S::p3_dX, *dxl0 = dxh0 + 2 * S::CDb;
+    uint8_t *duh = dxh0 + tc::cm_off(0, D, C), *dul = dxl0 + tc::cm_off(0, D, C);
+    uint8_t *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
     if (tid == 0) {  // the phase 2a operands are consumed
       ld_expect(ld, kStateTileBytes + kCDTileBytes);
       ld_state_tile(ld, s0h, s0l, ws.S0, base);
@@ -1337,19 +1480,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (ok) {
     // ---- phase 3: X (K-major, rows i, columns n in [0, 2D)) and dX (MN-major, k = r, n)
     uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb, *dxh = R + S::p3_dX, *dxl = dxh + 2 * S::CDb;
-    acc_read<C, D>(tb, cW, [&](int i, int c0, const float* v) { put16<C, true>(xh, xl, i, c0, v); });
-    acc_read<C, D>(tb, cU, [&](int i, int c0, const float* v) { put16<C, true>(xh, xl, i, D + c0, v); });
+    acc_read<C, D>(tb, cW, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, c0, v); });
+    acc_read<C, D>(tb, cU, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, D + c0, v); });
     acc_read<C, D>(tb, cdW, [&](int r, int c0, const float* v) {
-      float m[16];
-      for (int j = 0; j < 16; ++j) m[j] = -v[j];
-      put16<C, true>(dxh, dxl, r, c0, m);
+      float m[8];
+      for (int j = 0; j < 8; ++j) m[j] = -v[j];
+      put8<C, true>(dxh, dxl, r, c0, m);
     });
-    if (tid == 0) {
-      ld_expect(ld, kCDTileBytes);
-      ld_cd_tile(ld, dxh + tc::cm_off(0, D, C), dxl + tc::cm_off(0, D, C), ws.dUt, base);
-    }
-    ok = ld_wait(ld);
-    ok = ok && run(sy, [&] {
+    // (dX columns [D, 2D) = dU, loaded in phase 2b)
+    ok = run(sy, [&] {
       const tc::Op aH{tc::smem_u32(tTh), C, true}, aL{tc::smem_u32(tTl), C, true};
       const tc::Op bH{tc::smem_u32(dxh), C, true}, bL{tc::smem_u32(dxl), C, true};
       mma4(tb + cdB, aH, aL, bH, bL, C, tc::idesc_bf16(C, 2 * D, true, true), false, false, false);
@@ -1358,42 +1497,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (ok) {
     // ---- read dB: dB tile for dA; dv; dk / dG / dbeta contributions
     uint8_t *dbh = R + S::p4_dB, *dbl = dbh + 2 * S::CDb;
-    for (int c0 = grp * 16; c0 < 2 * D; c0 += 16 * kTcGroups) {
-      float v[16];
-      tc::tmem_ld16(la + cdB + c0, v);
-      if (myrow < 0) continue;
-      const int i = myrow;
-      put16<C, true>(dbh, dbl, i, c0, v);
+    for (int cc = grp * 16; cc < 2 * D; cc += 16 * kTcGroups) {
+      float v[8];
+      {
+        float v16[16];
+        tc::tmem_ld16(la + cdB + cc, v16);
+        share8(v16, v);
+      }
+      const int i = myrow, c0 = cc + half8;
+      put8<C, true>(dbh, dbl, i, c0, v);
       float part = 0.f;
-      if (c0 < D) {  // (the dk / dG terms of dB_k are added in the last phase, from TMEM)
-        float kv[16];
-        k16(i, c0, kv);
+      if (cc < D) {  // (the dk / dG terms of dB_k are added in the last phase, from TMEM)
+        float kv[8];
+        k8(i, c0, kv);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) part = fmaf(v[j], kv[j] * tc::ex2(sG[i * LD + c0 + j]), part);
+        for (int j = 0; j < 8; ++j) part = fmaf(v[j], kv[j] * tc::ex2(sG[i * LD + c0 + j]), part);
       } else if (i < n) {
         const int c1 = c0 - D;
-        float vv[16], val[16];
-        if constexpr (sizeof(Tin) == 2) {
-          const uint4* src = reinterpret_cast<const uint4*>(v_ + ((size_t)srow[i] * H + h) * D + c1);
-          const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
-          const __nv_bfloat162* b0 = reinterpret_cast<const __nv_bfloat162*>(&u0);
-          const __nv_bfloat162* b1 = reinterpret_cast<const __nv_bfloat162*>(&u1);
+        float vv[8], val[8];
+        ld8(v_ + ((size_t)srow[i] * H + h) * D + c1, vv);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f0 = __bfloat1622float2(b0[k]), f1 = __bfloat1622float2(b1[k]);
-            vv[2 * k] = f0.x; vv[2 * k + 1] = f0.y; vv[8 + 2 * k] = f1.x; vv[8 + 2 * k + 1] = f1.y;
-          }
-        } else {
-          ld16g(reinterpret_cast<const float*>(v_) + ((size_t)srow[i] * H + h) * D + c1, vv);
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           part = fmaf(v[j], vv[j], part);
           val[j] = sb[i] * v[j];
         }
-        out16(ws.rdv, ws.tdv, dv_, i, c1, val);
+        out8(ws.rdv, ws.tdv, dv_, i, c1, val);
       }
-      sdb[((c0 < D ? 0 : 1) * kTcGroups + grp) * C + i] += part;  // one slot per (half, warp group)
+      part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);  // columns 0-7 + 8-15 of the chunk
+      if (lane < 16) sdb[((cc < D ? 0 : 1) * kTcGroups + grp) * C + i] += part;  // one slot per (half, group)
     }
     uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb;
     ok = run(sy, [&] {
@@ -1405,20 +1536,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (ok) {
     // ---- dA = -(dB X^T) strict lower; dAt = beta dA (tile); dbeta += rowsum(dA Atilde)
     uint8_t *dah = R + S::p5_dA, *dal = dah + S::CCb;
-    for (int c0 = grp * 16; c0 < C; c0 += 16 * kTcGroups) {
-      float v[16];
-      tc::tmem_ld16(la + cdA + c0, v);
-      if (myrow < 0) continue;
-      const int r = myrow;
-      float m[16], part = 0.f;
-      for (int j = 0; j < 16; ++j) {
+    for (int cc = grp * 16; cc < C; cc += 16 * kTcGroups) {
+      float v[8];
+      {
+        float v16[16];
+        tc::tmem_ld16(la + cdA + cc, v16);
+        share8(v16, v);
+      }
+      const int r = myrow, c0 = cc + half8;
+      float m[8], part = 0.f;
+      for (int j = 0; j < 8; ++j) {
         const int i = c0 + j;
         const float dA = (i < r) ? -v[j] : 0.f;
         part = fmaf(dA, sAt[r * LC + i], part);
         m[j] = sb[r] * dA;
       }
-      put16<C, true>(dah, dal, r, c0, m);  // element (r, i)
-      sdb[(2 * kTcGroups + grp) * C + r] += part;
+      put8<C, true>(dah, dal, r, c0, m);  // element (r, i)
+      part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);
+      if (lane < 16) sdb[(2 * kTcGroups + grp) * C + r] += part;
     }
     // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
     uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
@@ -1443,27 +1578,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (ok) {
     // ---- final: dk, dG = partials + dB_k terms + gated terms; dG staged for the reverse cumulative sum
     float* sdG = reinterpret_cast<float*>(R);  // [C][LD]
-    for (int c0 = grp * 16; c0 < D; c0 += 16 * kTcGroups) {
-      float rs[16], cs[16], dbk[16];
-      tc::tmem_ld16(la + cRS + c0, rs);
-      tc::tmem_ld16(la + cCS + c0, cs);
-      tc::tmem_ld16(la + cdB + c0, dbk);
-      if (myrow < 0) continue;
-      const int r = myrow;
-      float kv[16], dkv[16], pg[16];
-      k16(r, c0, kv);
-      ld16g(pdk + r * D + c0, dkv);
-      ld16g(pdG + r * D + c0, pg);
+    for (int cc = grp * 16; cc < D; cc += 16 * kTcGroups) {
+      float rs[8], cs[8], dbk[8];
+      {
+        uint32_t a0[16], a1[16], a2[16];  // three loads in flight, one wait
+        tc::tmem_ld16_nowait(la + cRS + cc, a0);
+        tc::tmem_ld16_nowait(la + cCS + cc, a1);
+        tc::tmem_ld16_nowait(la + cdB + cc, a2);
+        tc::tmem_wait_ld();
+        tc::tmem_regs16(a0);
+        tc::tmem_regs16(a1);
+        tc::tmem_regs16(a2);
+        share8u(a0, rs);
+        share8u(a1, cs);
+        share8u(a2, dbk);
+      }
+      const int r = myrow, c0 = cc + half8;
+      float kv[8], dkv[8], pg[8];
+      k8(r, c0, kv);
+      ld8g(pdk + r * D + c0, dkv);
+      ld8g(pdG + r * D + c0, pg);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int c = c0 + j;
-        const float Gr = sG[r * LD + c], G0 = sref[c];
-        const float a = tc::ex2(Gr - G0) * rs[j], b = tc::ex2(G0 - Gr) * cs[j];
-        const float wb = tc::ex2(Gr) * sb[r] * dbk[j];
+        // e = 2^{G_r - G_0} (bounded by the chunk's decay check), 1/e = 2^{G_0 - G_r}, 2^{G_r} = 2^{G_0} e
+        const float e = tc::ex2(sG[r * LD + c] - sref[c]), ie = tc::rcp_approx(e);
+        const float a = e * rs[j], b = ie * cs[j];
+        const float wb = se0[c] * e * sb[r] * dbk[j];
         dkv[j] += wb + (a + b);
         sdG[r * LD + c] = r < n ? pg[j] + kv[j] * (wb + (a - b)) : 0.f;
       }
-      if (r < n) out16(ws.rdk, ws.tdk, dk_, r, c0, dkv);
+      if (r < n) out8(ws.rdk, ws.tdk, dk_, r, c0, dkv);
     }
     __syncthreads();
     // dg = reverse cumulative sum of dG over the chunk's rows: four threads per column, each a
