@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     tc::mbar_wait(&bar_m[0], 0, 200000000ull);
   }
   if constexpr (REVERSE && EX) tc::cp_async_wait<0>();
-  if (c == 0) tc::bulk_wait_all();
+  if (c == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
   tc::fence_before_sync();
   __syncthreads();
   if ((c >> 5) == 0) tc::tmem_dealloc(tb, 32);

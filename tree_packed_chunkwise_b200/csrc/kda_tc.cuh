@@ -544,7 +544,8 @@ __device__ __forceinline__ void ld_cc_tile(Ld& l, uint8_t* hi, uint8_t* lo, cons
   tc::bulk_g2s(lo, src + kCCTileBytes / 2, kCCTileBytes / 2, l.bar);
 }
 // bulk stores (issuing thread, after the tile writes were fenced and synchronised; the caller waits
-// with bulk_wait_read / bulk_wait_all before the shared buffers are reused or the CTA exits)
+// with bulk_wait_read before the shared buffers are reused or the CTA exits; the global writes
+// complete with the grid)
 __device__ __forceinline__ void store_cd_tile(float* tiles, size_t base, const uint8_t* hi, const uint8_t* lo) {
   uint8_t* dst = reinterpret_cast<uint8_t*>(tiles) + base * kCDTileBytes;
   tc::bulk_s2g(dst, hi, kCDTileBytes / 2);
@@ -885,7 +886,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   }
-  if (tid == 0) tc::bulk_wait_all();
+  if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
   tc::fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
@@ -1024,7 +1025,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (tid == 0) store_cd_tile(ws.W, base, eh, el);
     }
   }
-  if (tid == 0) tc::bulk_wait_all();
+  if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
   tc::fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
@@ -1274,7 +1275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       pdG[(n - 1) * D + c] += acc + tc::ex2(sG[(n - 1) * LD + c]) * acc2;
     }
   }
-  if (tid == 0) tc::bulk_wait_all();
+  if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
   tc::fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
