@@ -1,5 +1,6 @@
 // C ABI of the tree-packed chunkwise KDA library: compact MoE routing with occurrence counts.
 // Declarations and contracts in include/tpc.h.
+#include <algorithm>
 #include <cuda_runtime.h>
 
 #include <string>
@@ -41,20 +42,21 @@ int tpc_moe_route(const tpc_plan* plan, const void* h, const void* w_router, int
   auto* part_load = reinterpret_cast<long long*>(sc);
   auto* part_prob = reinterpret_cast<float*>(sc + a256((size_t)parts * E * 8));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int npt = (tpc::kMoeRows * E + tpc::kMoeThreads - 1) / tpc::kMoeThreads;
-  auto go = [&](auto np) -> int {
-    constexpr int NPT = decltype(np)::value;
-    TPC_CUDA(set_smem(tpc::moe_route_kernel<NPT>, tpc::MoeSmem::total));
-    TPC_LAUNCH("moe_route", st, (tpc::moe_route_kernel<NPT><<<parts, tpc::kMoeThreads, tpc::MoeSmem::total, st>>>(
+  // rows per thread of the logits tiling: 32 rows x QP expert quads over the CTA's threads
+  const int rt = std::max(1, tpc::kMoeRows * tpc::moe_quads_p2(E) / tpc::kMoeThreads);
+  auto go = [&](auto rpt) -> int {
+    constexpr int RT = decltype(rpt)::value;
+    TPC_CUDA(set_smem(tpc::moe_route_kernel<RT>, tpc::MoeSmem::total));
+    TPC_LAUNCH("moe_route", st, (tpc::moe_route_kernel<RT><<<parts, tpc::kMoeThreads, tpc::MoeSmem::total, st>>>(
                                     plan->p.dt, (const __nv_bfloat16*)h, (const __nv_bfloat16*)w_router, (int)Dh, E, k,
                                     N, logits, lse, topk_idx, topk_gate, part_load, part_prob)));
     return TPC_OK;
   };
   int rc;
-  if (npt <= 4) rc = go(std::integral_constant<int, 4>{});
-  else if (npt <= 8) rc = go(std::integral_constant<int, 8>{});
-  else if (npt <= 16) rc = go(std::integral_constant<int, 16>{});
-  else rc = go(std::integral_constant<int, 32>{});
+  if (rt <= 1) rc = go(std::integral_constant<int, 1>{});
+  else if (rt <= 2) rc = go(std::integral_constant<int, 2>{});
+  else if (rt <= 4) rc = go(std::integral_constant<int, 4>{});
+  else rc = go(std::integral_constant<int, 8>{});
   if (rc) return rc;
   TPC_LAUNCH("moe_reduce", st, (tpc::moe_reduce_kernel<<<E, tpc::kMoeThreads, 0, st>>>(
                                    part_load, part_prob, parts, E, (long long*)expert_load, prob_sum)));

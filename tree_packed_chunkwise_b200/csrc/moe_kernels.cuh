@@ -23,10 +23,13 @@ constexpr int kMoeThreads = 256;
 constexpr int kMoeCK = 64;        // hidden-dimension chunk staged in shared memory
 constexpr int kMoeMaxE = 256, kMoeMaxK = 8;
 
+// Expert columns padded to a multiple of 4 (float4 reads) plus 4 (fewer bank conflicts on the stores)
+constexpr int kMoeMaxEp = kMoeMaxE + 4;
+
 struct MoeSmem {
   static constexpr size_t hs = 0;                                           // [rows][CK] fp32
-  static constexpr size_t ws = hs + sizeof(float) * kMoeRows * kMoeCK;       // [CK][E] fp32
-  static constexpr size_t zs = ws + sizeof(float) * kMoeCK * kMoeMaxE;       // [rows][E] fp32 logits
+  static constexpr size_t ws = hs + sizeof(float) * kMoeRows * kMoeCK;       // [CK][Ep] fp32
+  static constexpr size_t zs = ws + sizeof(float) * kMoeCK * kMoeMaxEp;      // [rows][E] fp32 logits
   static constexpr size_t sel = zs + sizeof(float) * kMoeRows * kMoeMaxE;    // [rows][K] int
   static constexpr size_t lse = sel + sizeof(int) * kMoeRows * kMoeMaxK;     // [rows] fp32
   static constexpr size_t total = lse + sizeof(float) * kMoeRows;
@@ -42,9 +45,18 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+// number of expert quads rounded up to a power of two (the thread tiling of the logits)
+__host__ __device__ __forceinline__ int moe_quads_p2(int E) {
+  int q = 1;
+  while (q < (E + 3) / 4) q <<= 1;
+  return q;
+}
+
 // Routing of kMoeRows rows per CTA: logits, lse, top-k experts and gates per row, and this CTA's
-// partial occurrence-weighted expert loads and probability sums.
-template <int NPT>  // (row, expert) pairs per thread: kMoeRows * E / kMoeThreads, rounded up
+// partial occurrence-weighted expert loads and probability sums.  Logits: thread (quad q, row group tr)
+// owns experts 4q .. 4q+3 of rows tr, tr + TR, ... (RT rows); per hidden index c it reads one float4
+// of router weights and RT hidden values and updates 4 RT sums, each in the order c = 0, 1, ...
+template <int RT>  // rows per thread: max(1, 32 * QP / 256), QP = moe_quads_p2(E)
 __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(DevTables t, const __nv_bfloat16* __restrict__ h,
                                                                 const __nv_bfloat16* __restrict__ w, int Dh, int E,
                                                                 int k, int N, float* __restrict__ logits,
@@ -59,39 +71,51 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(DevTables t, con
   int* sel = reinterpret_cast<int*>(msm + MoeSmem::sel);
   float* slse = reinterpret_cast<float*>(msm + MoeSmem::lse);
   const int tid = threadIdx.x, r0 = blockIdx.x * kMoeRows, nr = min(kMoeRows, N - r0);
-  const int pairs = kMoeRows * E;
-  float acc[NPT];
+  const int QP = moe_quads_p2(E), Ep = 4 * QP + 4, TR = kMoeThreads / QP;
+  const int q = tid % QP, tr = tid / QP;
+  float acc[RT][4];
 #pragma unroll
-  for (int i = 0; i < NPT; ++i) acc[i] = 0.f;
+  for (int m = 0; m < RT; ++m)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[m][j] = 0.f;
   for (int c0 = 0; c0 < Dh; c0 += kMoeCK) {
     for (int e = tid; e < kMoeRows * kMoeCK; e += kMoeThreads) {
       const int r = e / kMoeCK, c = e % kMoeCK;
       hs[e] = (r < nr) ? __bfloat162float(h[(size_t)(r0 + r) * Dh + c0 + c]) : 0.f;
     }
-    for (int e = tid; e < E * kMoeCK; e += kMoeThreads) {
+    for (int e = tid; e < 4 * QP * kMoeCK; e += kMoeThreads) {
       const int x = e / kMoeCK, c = e % kMoeCK;
-      wsm[c * E + x] = __bfloat162float(w[(size_t)x * Dh + c0 + c]);
+      wsm[c * Ep + x] = x < E ? __bfloat162float(w[(size_t)x * Dh + c0 + c]) : 0.f;
     }
     __syncthreads();
-    for (int c = 0; c < kMoeCK; ++c) {
+    if (tr < kMoeRows) {
+#pragma unroll 4
+      for (int c = 0; c < kMoeCK; ++c) {
+        const float4 wv = *reinterpret_cast<const float4*>(wsm + c * Ep + 4 * q);
 #pragma unroll
-      for (int i = 0; i < NPT; ++i) {
-        const int p = tid + kMoeThreads * i;
-        if (p < pairs) {
-          const int r = p / E, x = p - r * E;
-          acc[i] = __fadd_rn(acc[i], __fmul_rn(hs[r * kMoeCK + c], wsm[c * E + x]));
+        for (int m = 0; m < RT; ++m) {
+          const float hv = hs[(tr + TR * m) * kMoeCK + c];
+          acc[m][0] = __fadd_rn(acc[m][0], __fmul_rn(hv, wv.x));
+          acc[m][1] = __fadd_rn(acc[m][1], __fmul_rn(hv, wv.y));
+          acc[m][2] = __fadd_rn(acc[m][2], __fmul_rn(hv, wv.z));
+          acc[m][3] = __fadd_rn(acc[m][3], __fmul_rn(hv, wv.w));
         }
       }
     }
     __syncthreads();
   }
+  if (tr < kMoeRows) {
 #pragma unroll
-  for (int i = 0; i < NPT; ++i) {
-    const int p = tid + kMoeThreads * i;
-    if (p < pairs) {
-      const int r = p / E, x = p - r * E;
-      zs[r * E + x] = acc[i];
-      if (r < nr) logits[(size_t)(r0 + r) * E + x] = acc[i];
+    for (int m = 0; m < RT; ++m) {
+      const int r = tr + TR * m;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int x = 4 * q + j;
+        if (x < E) {
+          zs[r * E + x] = acc[m][j];
+          if (r < nr) logits[(size_t)(r0 + r) * E + x] = acc[m][j];
+        }
+      }
     }
   }
   __syncthreads();
