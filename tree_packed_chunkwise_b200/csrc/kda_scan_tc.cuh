@@ -154,6 +154,14 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     const int ci = chunk_at(q);
     load_mtile(mbuf[q & 1], mtile(ci), xbuf[q & 1], xsrc(ci), (uint32_t)S::XB, &bar_m[q & 1]);
   };
+  // thread 0: the operands of a later chunk into L2 (the M tile once per (sequence, head), by the
+  // first slice's CTA), so that the shared-memory copy a step ahead finds them there
+  auto prefetch_l2 = [&](int q) {
+    if (q >= nch) return;
+    const int ci = chunk_at(q);
+    if (blockIdx.z == 0) tc::bulk_prefetch_l2(mtile(ci), kMtileBytes);
+    tc::bulk_prefetch_l2(xsrc(ci), (uint32_t)S::XB);
+  };
   auto prefetch_do = [&](int q) {  // every thread
     if constexpr (REVERSE) {
       const ChunkRec ch = t.chunks[chunk_at(q)];
@@ -173,7 +181,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     else
       for (int j = 0; j < 32; ++j) s[j] = 0.f;
   }
-  if (c == 0) prefetch(0);
+  constexpr int kL2Ahead = 3;  // chunks prefetched into L2 ahead of the current one
+  if (c == 0) {
+    prefetch(0);
+    for (int q = 1; q < kL2Ahead; ++q) prefetch_l2(q);
+  }
   prefetch_do(0);
   uint32_t mma_phase = 0;
   bool ok = true;
@@ -193,7 +205,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
     put_state(sth, stl, c, s);
     if constexpr (REVERSE && EX) tc::cp_async_wait<0>();  // this chunk's dO slice (issued a step ago)
-    if (c == 0 && q + 1 < nch) prefetch(q + 1);
+    if (c == 0) {
+      if (q + 1 < nch) prefetch(q + 1);
+      prefetch_l2(q + kL2Ahead);
+    }
     if (q + 1 < nch) prefetch_do(q + 1);
     ok = wait_all(&bar_m[q & 1], (q >> 1) & 1, ws.status);
     if (!ok) break;
