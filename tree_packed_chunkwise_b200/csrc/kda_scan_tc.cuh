@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   __shared__ __align__(8) uint64_t bar_m[2];
   __shared__ __align__(8) uint64_t bar_mma;
   __shared__ uint32_t tslot;
+  __shared__ int s_ok;  // thread 0's bounded waits, read by every thread after the following barrier
   const int c = threadIdx.x;  // state row / TMEM lane
   if ((c >> 5) == 0) tc::tmem_alloc(&tslot, 32);
   if (c == 0) {
@@ -189,6 +190,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   prefetch_do(0);
   uint32_t mma_phase = 0;
   bool ok = true;
+  // Per step: thread 0 alone waits (bounded) on the mbarriers and publishes the outcome in s_ok; two
+  // barriers per step (operands ready; products done, and the state tile's bulk store has read it).
   for (int q = 0; q < nch && ok; ++q) {
     const int ci = chunk_at(q);
     const size_t base = (size_t)ci * H + h;
@@ -208,34 +211,30 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     if (c == 0) {
       if (q + 1 < nch) prefetch(q + 1);
       prefetch_l2(q + kL2Ahead);
+      const bool w = tc::mbar_wait(&bar_m[q & 1], (q >> 1) & 1);
+      if (!w) set_status(ws.status, kStatusTimeout);
+      s_ok = w ? 1 : 0;
     }
     if (q + 1 < nch) prefetch_do(q + 1);
-    ok = wait_all(&bar_m[q & 1], (q >> 1) & 1, ws.status);
+    tc::fence_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();  // state tile written, this chunk's operands arrived
+    tc::fence_after_sync();
+    ok = s_ok != 0;
     if (!ok) break;
-    float add[32];  // forward: B of this chunk, row c of the slice
+    float add[32];  // forward: B of this chunk, row c of the slice (16-byte groups permuted by c mod 8)
     if constexpr (!REVERSE) {
       const float* ab = reinterpret_cast<const float*>(xbuf[q & 1]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 u = reinterpret_cast<const float4*>(ab + c * DVT)[i];
+        const float4 u = reinterpret_cast<const float4*>(ab + c * DVT)[i ^ (c & 7)];
         add[4 * i] = u.x; add[4 * i + 1] = u.y; add[4 * i + 2] = u.z; add[4 * i + 3] = u.w;
       }
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) add[j] = 0.f;
     }
-    tc::fence_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
     if (c == 0) {
-      // the state slice tile goes to the chunk kernels as it is: forward the chunk-start state S0,
-      // reverse the gradient of the chunk-end state (hi/lo operand tiles, this slice's 8 KB of each)
-      uint8_t* dst = reinterpret_cast<uint8_t*>(REVERSE ? ws.dS : ws.S0) + base * kStateTileBytes +
-                     (size_t)blockIdx.z * S::StB;
-      tc::bulk_s2g(dst, sth, (uint32_t)S::StB);
-      tc::bulk_s2g(dst + kStateTileBytes / 2, stl, (uint32_t)S::StB);
-      tc::bulk_commit();
       const tc::Op mH{tc::smem_u32(mbuf[q & 1]), D, REVERSE}, mL{tc::smem_u32(mbuf[q & 1] + kMtileBytes / 2), D, REVERSE};
       const tc::Op sH{tc::smem_u32(sth), D, true}, sL{tc::smem_u32(stl), D, true};
       mma4(tb, mH, mL, sH, sL, D, tc::idesc_bf16(D, DVT, REVERSE, true), false, false, false);
@@ -245,11 +244,24 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         mma4(tb, eH, eL, oH, oL, C, tc::idesc_bf16(D, DVT, true, true), true, false, EX);
       }
       tc::commit(&bar_mma);
+      // the state slice tile goes to the chunk kernels as it is: forward the chunk-start state S0,
+      // reverse the gradient of the chunk-end state (hi/lo operand tiles, this slice's 8 KB of each)
+      uint8_t* dst = reinterpret_cast<uint8_t*>(REVERSE ? ws.dS : ws.S0) + base * kStateTileBytes +
+                     (size_t)blockIdx.z * S::StB;
+      tc::bulk_s2g(dst, sth, (uint32_t)S::StB);
+      tc::bulk_s2g(dst + kStateTileBytes / 2, stl, (uint32_t)S::StB);
+      tc::bulk_commit();
+      const bool w = tc::mbar_wait(&bar_mma, mma_phase);
+      if (!w) set_status(ws.status, kStatusTimeout);
+      tc::bulk_wait_read();  // (read while the products ran)
+      s_ok = w ? 1 : 0;
     }
-    ok = wait_all(&bar_mma, mma_phase, ws.status);
     mma_phase ^= 1u;
-    if (!ok) break;
+    tc::fence_before_sync();
+    __syncthreads();  // products in TMEM; this chunk's M buffer free again
     tc::fence_after_sync();
+    ok = s_ok != 0;
+    if (!ok) break;
     float acc[32];
     tc::tmem_ld32(la, acc);
     for (int j = 0; j < 32; ++j) s[j] = acc[j] + add[j];
@@ -257,9 +269,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       const int slot = t.chunks[ci].export_slot;
       if (slot >= 0) st32g(ws.slot + ((size_t)slot * H + h) * D * D + c * D + j0, s);
     }
-    if (c == 0) tc::bulk_wait_read();
-    tc::fence_before_sync();
-    __syncthreads();  // the state tile and this M buffer are free again
   }
   if (ok) {
     if (!REVERSE) {

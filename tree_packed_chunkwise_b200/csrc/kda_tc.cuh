@@ -37,10 +37,12 @@ enum : int { kStatusTimeout = 8 };
 // state scans: CTA size and width of the d_v slice one CTA owns
 constexpr int kScanThreads = 128, kScanDVT = 32;
 
-// offset (floats) of element (c, j) of a chunk-head's d x d additive term (B or X) in the
-// slice-major layout [slice][row][32] that the scans read by bulk copies
+// offset (floats) of element (c, j) of a chunk-head's d x d additive term B in the slice-major layout
+// [slice][row][32] that the forward scan reads by bulk copies; within a row the eight 16-byte groups
+// are permuted by (row mod 8) so that the scan's threads (one row each) read them without bank conflicts
 __host__ __device__ __forceinline__ size_t slice_major(int c, int j) {
-  return ((size_t)(j / kScanDVT) * kTcD + c) * kScanDVT + (j % kScanDVT);
+  const int jj = j % kScanDVT;
+  return ((size_t)(j / kScanDVT) * kTcD + c) * kScanDVT + ((((jj >> 2) ^ (c & 7)) << 2) | (jj & 3));
 }
 
 namespace tck {
@@ -871,18 +873,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mma4(tb + 128, kH, kL, uH, uL, C, id, false, false, false);  // Khat^T U'
       });
       if (ok) {
+        // M (tile) and B (slice-major) are assembled in the consumed tile space (and the staging rows,
+        // when they exist) and bulk-stored, once the W and U' stores have read their tiles
         uint8_t* Mt = reinterpret_cast<uint8_t*>(ws.Mt) + base * kMtileBytes;
         float* Bg = ws.Bc + base * D * D;
+        constexpr bool kBsm = 6 * S::CDb + 2 * S::StB >= kMtileBytes + sizeof(float) * D * D;
+        uint8_t* mts = tl;
+        float* bs = reinterpret_cast<float*>(tl + kMtileBytes);
+        if (tid == 0) tc::bulk_wait_read();
+        __syncthreads();
         acc_read<D, D>(tb, 0, [&](int c, int c0, const float* v) {
           float m[16];
           const float gam = tc::ex2(gC[c]);
           for (int j = 0; j < 16; ++j) m[j] = (c0 + j == c ? gam : 0.f) - v[j];
-          put16<D, true>(Mt, Mt + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
+          put16<D, true>(mts, mts + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
         });
         acc_read<D, D>(tb, 128, [&](int c, int j0, const float* v) {  // slice-major for the scan's bulk loads
+          float* dst = kBsm ? bs : Bg;
           for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(Bg + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            *reinterpret_cast<float4*>(dst + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         });
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+          constexpr uint32_t kPiece = 16384;
+          for (uint32_t o = 0; o < kMtileBytes; o += kPiece) tc::bulk_s2g(Mt + o, mts + o, kPiece);
+          if constexpr (kBsm)
+            for (uint32_t o = 0; o < sizeof(float) * D * D; o += kPiece)
+              tc::bulk_s2g(reinterpret_cast<uint8_t*>(Bg) + o, reinterpret_cast<const uint8_t*>(bs) + o, kPiece);
+          tc::bulk_commit();
+        }
       }
     }
   }
@@ -1422,6 +1442,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
   const int myrow = 16 * sp + (lane & 15);  // M = 64 accumulator row; this lane's 8 columns: share8
   const int half8 = 8 * (lane >> 4);
+  float pre_dk[2][8], pre_dG[2][8];  // the final phase's dq-kernel partials (loaded ahead)
   // 8 gradient values of row r from column c0 on, to where the row's gradients go
   auto out8 = [&](float* replay_buf, float* tgt_buf, Tout* out, int r, int c0, const float* v) {
     const size_t o = ((size_t)sidx[r] * H + h) * D + c0;
@@ -1556,6 +1577,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);
       if (lane < 16) sdb[(2 * kTcGroups + grp) * C + r] += part;
     }
+    // the dq kernel's partials of this lane's final-phase rows and columns, loaded ahead of phase 5
+    static_assert(D == 2 * 16 * kTcGroups, "two 16-column chunks per warp group in the final phase");
+    for (int it = 0; it < 2; ++it) {
+      const int c0 = grp * 16 + 16 * kTcGroups * it + half8;
+      ld8g(pdk + myrow * D + c0, pre_dk[it]);
+      ld8g(pdG + myrow * D + c0, pre_dG[it]);
+    }
     // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
     uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
     auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
@@ -1579,7 +1607,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (ok) {
     // ---- final: dk, dG = partials + dB_k terms + gated terms; dG staged for the reverse cumulative sum
     float* sdG = reinterpret_cast<float*>(R);  // [C][LD]
-    for (int cc = grp * 16; cc < D; cc += 16 * kTcGroups) {
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int cc = grp * 16 + 16 * kTcGroups * it;
       float rs[8], cs[8], dbk[8];
       {
         uint32_t a0[16], a1[16], a2[16];  // three loads in flight, one wait
@@ -1597,8 +1627,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int r = myrow, c0 = cc + half8;
       float kv[8], dkv[8], pg[8];
       k8(r, c0, kv);
-      ld8g(pdk + r * D + c0, dkv);
-      ld8g(pdG + r * D + c0, pg);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        dkv[j] = pre_dk[it][j];
+        pg[j] = pre_dG[it][j];
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int c = c0 + j;
