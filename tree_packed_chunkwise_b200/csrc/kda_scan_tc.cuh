@@ -50,10 +50,8 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* st
 __device__ __forceinline__ void load_mtile(uint8_t* dst, const uint8_t* src, uint8_t* x_dst, const uint8_t* x_src,
                                            uint32_t x_bytes, uint64_t* bar) {
   tc::mbar_arrive_expect_tx(bar, kMtileBytes + x_bytes);
-#pragma unroll
-  for (int p = 0; p < 4; ++p) tc::bulk_g2s(dst + p * (kMtileBytes / 4), src + p * (kMtileBytes / 4), kMtileBytes / 4, bar);
-  tc::bulk_g2s(x_dst, x_src, x_bytes / 2, bar);
-  tc::bulk_g2s(x_dst + x_bytes / 2, x_src + x_bytes / 2, x_bytes / 2, bar);
+  tc::bulk_g2s(dst, src, kMtileBytes, bar);
+  tc::bulk_g2s(x_dst, x_src, x_bytes, bar);
 }
 
 // This CTA's 32 columns (j0 ..) of the chunk's dO rows as an MN-major operand tile (k = chunk row,

@@ -326,6 +326,32 @@ __device__ __forceinline__ void tile16(const uint8_t* hi, const uint8_t* lo, int
   }
 }
 
+// Two A x B tiles (hi/lo) from the same staged bf16 rows: f(a, b, x) returns both values (float2)
+template <int A, int B, class F>
+__device__ __forceinline__ void build_tile2_st(uint8_t* hi1, uint8_t* lo1, uint8_t* hi2, uint8_t* lo2,
+                                               const __nv_bfloat16* st, F f) {
+  for (int e = threadIdx.x; e < A * (B / 8); e += blockDim.x) {
+    const int a = e % A, b0 = (e / A) * 8;
+    const uint4 u = *reinterpret_cast<const uint4*>(st + a * kStagePitch + b0);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    __align__(16) __nv_bfloat16 h1[8], l1[8], h2[8], l2[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 x = __bfloat1622float2(b2[j]);
+      const float2 y0 = f(a, b0 + 2 * j, x.x), y1 = f(a, b0 + 2 * j + 1, x.y);
+      split_bf16(y0.x, h1[2 * j], l1[2 * j]);
+      split_bf16(y1.x, h1[2 * j + 1], l1[2 * j + 1]);
+      split_bf16(y0.y, h2[2 * j], l2[2 * j]);
+      split_bf16(y1.y, h2[2 * j + 1], l2[2 * j + 1]);
+    }
+    const uint32_t off = cm_off(a, b0, A);
+    *reinterpret_cast<uint4*>(hi1 + off) = *reinterpret_cast<const uint4*>(h1);
+    *reinterpret_cast<uint4*>(lo1 + off) = *reinterpret_cast<const uint4*>(l1);
+    *reinterpret_cast<uint4*>(hi2 + off) = *reinterpret_cast<const uint4*>(h2);
+    *reinterpret_cast<uint4*>(lo2 + off) = *reinterpret_cast<const uint4*>(l2);
+  }
+}
+
 // 8 consecutive values of a staged row as fp32
 template <typename T>
 __device__ __forceinline__ void staged8(const T* st, int r, int c0, float (&v)[8]) {
@@ -810,8 +836,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // phase 1: Atilde = af bf^T with af = k e^{G - ref}, bf = k e^{ref - G}
   {
     uint8_t *afh = tl, *afl = tl + S::CDb, *bfh = tl + 2 * S::CDb, *bfl = tl + 3 * S::CDb;
-    k_tile(afh, afl, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); });
-    k_tile(bfh, bfl, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
+    if constexpr (EX) {  // e = 2^{G - ref} (bounded by the decay check), 2^{ref - G} = 1 / e
+      build_tile2_st<C, D>(afh, afl, bfh, bfl, sk, [&](int r, int c, float x) {
+        const float e = tc::ex2(sG[r * LD + c] - sref[c]);
+        return make_float2(x * e, x * tc::rcp_approx(e));
+      });
+    } else {
+      k_tile(afh, afl, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); });
+      k_tile(bfh, bfl, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
+    }
     const tc::Op ah{tc::smem_u32(afh), C, false}, al{tc::smem_u32(afl), C, false};
     const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
     ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
@@ -1588,9 +1621,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
     auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
     auto aff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
-    if constexpr (S::kStageK) {
-      build_tile_st<C, D, true>(bfh, bfl, reinterpret_cast<const __nv_bfloat16*>(sk), bff);
-      build_tile_st<C, D, true>(afh, afl, reinterpret_cast<const __nv_bfloat16*>(sk), aff);
+    if constexpr (S::kStageK) {  // e = 2^{G - ref} (bounded by the decay check), 2^{ref - G} = 1 / e
+      build_tile2_st<C, D>(afh, afl, bfh, bfl, reinterpret_cast<const __nv_bfloat16*>(sk), [&](int r, int c, float x) {
+        const float e = tc::ex2(sG[r * LD + c] - sref[c]);
+        return make_float2(x * e, x * tc::rcp_approx(e));
+      });
     } else {
       build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, bff);
       build_tile_ld<C, D, true, Tin>(afh, afl, row_k, aff);

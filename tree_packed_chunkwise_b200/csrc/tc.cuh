@@ -76,10 +76,26 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
       "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 
-// D (+)= A (M x K) * B (K x N), K a multiple of 16; issued by one thread.
+// Advance of a descriptor's start-address field per 16-wide K step (the field holds address >> 4 in its
+// low 14 bits; the tiles live below 256 KB of shared memory, so the sum never carries out of it).
+__device__ __forceinline__ uint64_t op_desc_step(const Op& o) {
+  return o.mn ? (uint64_t)((2u * 128u) >> 4) : (uint64_t)((2u * (uint32_t)(o.A >> 3) * 128u) >> 4);
+}
+
+// D (+)= A (M x K) * B (K x N), K a multiple of 16; issued by one thread.  The descriptors of step s
+// are those of step 0 advanced s times (one 64-bit add per operand and step).
 __device__ __forceinline__ void mma_chain(uint32_t d_tmem, const Op& a, const Op& b, int K, uint32_t idesc,
                                           bool accumulate) {
-  for (int s = 0; s < K / 16; ++s) mma_bf16(d_tmem, op_desc(a, s), op_desc(b, s), idesc, (accumulate || s) ? 1u : 0u);
+  uint64_t da = op_desc(a, 0), db = op_desc(b, 0);
+  const uint64_t ia = op_desc_step(a), ib = op_desc_step(b);
+  const int n = K / 16;
+  mma_bf16(d_tmem, da, db, idesc, accumulate ? 1u : 0u);
+#pragma unroll 4
+  for (int s = 1; s < n; ++s) {
+    da += ia;
+    db += ib;
+    mma_bf16(d_tmem, da, db, idesc, 1u);
+  }
 }
 
 // D (+)= A B with A (M x 16) read from tensor memory: row m of A in TMEM lane m, two bf16 per
