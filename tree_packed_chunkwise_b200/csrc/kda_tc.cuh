@@ -438,6 +438,35 @@ __device__ __forceinline__ void st16_out(T* p, const float* v) {
   }
 }
 
+// The chunk-head item of this launch that starts about one CTA lifetime after this one (the CTAs of a
+// launch start roughly in linear order, one per SM, so the item %nsmid places later); its workspace
+// tiles are prefetched into L2 so that its first loads do not wait for HBM.  False if there is none.
+__device__ __forceinline__ bool next_item(int chunk0, int& ci_next, int& h_next) {
+  uint32_t nsm;
+  asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
+  const long long lin = (long long)blockIdx.x + (long long)gridDim.x * blockIdx.y + nsm;
+  if (lin >= (long long)gridDim.x * gridDim.y) return false;
+  ci_next = chunk0 + (int)(lin % gridDim.x);
+  h_next = (int)(lin / gridDim.x);
+  return true;
+}
+__device__ __forceinline__ void prefetch_tile(const float* tiles, size_t item, uint32_t bytes) {
+  tc::bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(tiles) + item * bytes, bytes);
+}
+
+// The dq kernel's per-chunk partials of dk and dG (C x D fp32 each) go to the dk/dv kernel in the
+// order of the two kernels' epilogue lanes (the same element -> lane map in both): the 8 values of
+// (warp w, iteration it, lane l) are the float4 pair pd_frag(w, it, l) and pd_frag(w, it, l) + 32, so
+// that each store or load instruction of a warp covers 512 contiguous bytes.  Epilogue lane map
+// (512 threads, an M = 64 accumulator read 16 columns at a time with share8): row 16 (w % 4) + l % 16,
+// columns 16 (w / 4) + 64 it + 8 (l / 16) + 0 .. 7.
+__device__ __forceinline__ int pd_frag(int w, int it, int lane) { return (w * 2 + it) * 64 + lane; }
+// float offset of element (r, c) of a chunk's partials in that order
+__device__ __forceinline__ int pd_index(int r, int c) {
+  const int w = ((c >> 4) & 3) * 4 + (r >> 4), it = c >> 6, lane = (r & 15) + 16 * ((c >> 3) & 1), v = c & 7;
+  return ((pd_frag(w, it, lane) + 32 * (v >> 2)) << 2) + (v & 3);
+}
+
 // The rows of an M = 64 accumulator sit in TMEM lanes 0-15 of each sub-partition.  After a 16-column
 // read, lanes 16-31 take columns 8-15 of the row of lane - 16 (one shuffle per value), so that every
 // lane of the warp handles 8 values: row 16 * sp + lane % 16, columns 8 * (lane / 16) + 0 .. 7.
@@ -1003,6 +1032,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ld_expect(ld, kStateTileBytes + kCDTileBytes);
     ld_state_tile(ld, s0h, s0l, ws.S0, base);  // the chunk-start state, as the scan left it
     ld_cd_tile(ld, tsm + S::Wq, tsm + S::Wq + S::CDb, ws.W, base);  // W, as the prep kernel left it
+    int cn, hn;
+    if (next_item(chunk0, cn, hn)) {
+      const size_t nb = (size_t)cn * H + hn;
+      prefetch_tile(ws.S0, nb, kStateTileBytes);
+      prefetch_tile(ws.W, nb, kCDTileBytes);
+      prefetch_tile(ws.U, nb, kCDTileBytes);
+    }
   }
   gate_st(sG, LD, gr);
   __syncthreads();
@@ -1151,6 +1187,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
     ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
     ld_cc_tile(ld, tsm + S::Pt, tsm + S::Pt + S::CCb, ws.Pm, base);  // P, as the output kernel left it
+    int cn, hn;
+    if (next_item(chunk0, cn, hn)) {
+      const size_t nb = (size_t)cn * H + hn;
+      prefetch_tile(ws.S0, nb, kStateTileBytes);
+      prefetch_tile(ws.U, nb, kCDTileBytes);
+      prefetch_tile(ws.Pm, nb, kCCTileBytes);
+      prefetch_tile(ws.dS, nb, kStateTileBytes);
+    }
   }
   // bf16: the chunk's q and k rows into shared memory while the gates load and accumulate
   [[maybe_unused]] __nv_bfloat16* stq = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
@@ -1270,7 +1314,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
     const int r = 16 * sp + (lane & 15);  // accumulator row; this lane's 8 columns: share8
     const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
-    for (int cc = grp * 16; cc < D; cc += 16 * kTcGroups) {
+    static_assert(D == 2 * 16 * kTcGroups && C == 64 && kTcGroups == 4, "the pd_frag lane map");
+    for (int it = 0; it < 2; ++it) {
+      const int cc = grp * 16 + 16 * kTcGroups * it;
       float tq[8], t1[8], rs[8], cs[8];
       {
         uint32_t a0[16], a1[16], a2[16], a3[16];  // four loads in flight, one wait
@@ -1304,8 +1350,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         dG[j] = qv[j] * dq[j] - kv[j] * dk[j];
         sbuf[r * LD + c] = r < n ? kv[j] * dks : 0.f;
       }
-      st8g(pdk + r * D + c0, dk);
-      st8g(pdG + r * D + c0, dG);
+      {
+        float4* pk = reinterpret_cast<float4*>(pdk) + pd_frag(w, it, lane);
+        float4* pg = reinterpret_cast<float4*>(pdG) + pd_frag(w, it, lane);
+        pk[0] = make_float4(dk[0], dk[1], dk[2], dk[3]);
+        pk[32] = make_float4(dk[4], dk[5], dk[6], dk[7]);
+        pg[0] = make_float4(dG[0], dG[1], dG[2], dG[3]);
+        pg[32] = make_float4(dG[4], dG[5], dG[6], dG[7]);
+      }
       if (r >= ch.n_replay && r < n) st8_out(dq_ + ((size_t)srow[r] * H + h) * D + c0, dq);
     }
     __syncthreads();
@@ -1325,7 +1377,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int c = tid;
       const float acc = (part[c] + part[D + c]) + (part[2 * D + c] + part[3 * D + c]);
       const float acc2 = (part[4 * D + c] + part[5 * D + c]) + (part[6 * D + c] + part[7 * D + c]);
-      pdG[(n - 1) * D + c] += acc + tc::ex2(sG[(n - 1) * LD + c]) * acc2;
+      pdG[pd_index(n - 1, c)] += acc + tc::ex2(sG[(n - 1) * LD + c]) * acc2;
     }
   }
   if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
@@ -1444,6 +1496,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (tid == 0) {
       ld_expect(ld, kCCTileBytes);
       ld_cc_tile(ld, tTh, tTl, ws.Tm, cb);
+      int cn, hn;
+      if (next_item(chunk0, cn, hn)) {
+        const size_t nb = (size_t)cn * H + hn;
+        prefetch_tile(ws.At, nb, sizeof(float) * C * C);
+        prefetch_tile(ws.Tm, nb, kCCTileBytes);
+        prefetch_tile(ws.S0, nb, kStateTileBytes);
+        prefetch_tile(ws.dUt, nb, kCDTileBytes);
+        prefetch_tile(ws.pdk, nb, sizeof(float) * C * D);
+        prefetch_tile(ws.pdG, nb, sizeof(float) * C * D);
+      }
     }
   }
   gate_st(sG, LD, gr);
@@ -1612,10 +1674,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // the dq kernel's partials of this lane's final-phase rows and columns, loaded ahead of phase 5
     static_assert(D == 2 * 16 * kTcGroups, "two 16-column chunks per warp group in the final phase");
-    for (int it = 0; it < 2; ++it) {
-      const int c0 = grp * 16 + 16 * kTcGroups * it + half8;
-      ld8g(pdk + myrow * D + c0, pre_dk[it]);
-      ld8g(pdG + myrow * D + c0, pre_dG[it]);
+    for (int it = 0; it < 2; ++it) {  // (the pd_frag order of the dq kernel's epilogue)
+      const float4* pk = reinterpret_cast<const float4*>(pdk) + pd_frag(w, it, lane);
+      const float4* pg = reinterpret_cast<const float4*>(pdG) + pd_frag(w, it, lane);
+      const float4 a0 = pk[0], a1 = pk[32], b0 = pg[0], b1 = pg[32];
+      pre_dk[it][0] = a0.x; pre_dk[it][1] = a0.y; pre_dk[it][2] = a0.z; pre_dk[it][3] = a0.w;
+      pre_dk[it][4] = a1.x; pre_dk[it][5] = a1.y; pre_dk[it][6] = a1.z; pre_dk[it][7] = a1.w;
+      pre_dG[it][0] = b0.x; pre_dG[it][1] = b0.y; pre_dG[it][2] = b0.z; pre_dG[it][3] = b0.w;
+      pre_dG[it][4] = b1.x; pre_dG[it][5] = b1.y; pre_dG[it][6] = b1.z; pre_dG[it][7] = b1.w;
     }
     // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
     uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
