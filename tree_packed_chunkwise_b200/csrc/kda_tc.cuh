@@ -438,22 +438,6 @@ __device__ __forceinline__ void st16_out(T* p, const float* v) {
   }
 }
 
-// The chunk-head item of this launch that starts about one CTA lifetime after this one (the CTAs of a
-// launch start roughly in linear order, one per SM, so the item %nsmid places later); its workspace
-// tiles are prefetched into L2 so that its first loads do not wait for HBM.  False if there is none.
-__device__ __forceinline__ bool next_item(int chunk0, int& ci_next, int& h_next) {
-  uint32_t nsm;
-  asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
-  const long long lin = (long long)blockIdx.x + (long long)gridDim.x * blockIdx.y + nsm;
-  if (lin >= (long long)gridDim.x * gridDim.y) return false;
-  ci_next = chunk0 + (int)(lin % gridDim.x);
-  h_next = (int)(lin / gridDim.x);
-  return true;
-}
-__device__ __forceinline__ void prefetch_tile(const float* tiles, size_t item, uint32_t bytes) {
-  tc::bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(tiles) + item * bytes, bytes);
-}
-
 // The dq kernel's per-chunk partials of dk and dG (C x D fp32 each) go to the dk/dv kernel in the
 // order of the two kernels' epilogue lanes (the same element -> lane map in both): the 8 values of
 // (warp w, iteration it, lane l) are the float4 pair pd_frag(w, it, l) and pd_frag(w, it, l) + 32, so
@@ -1032,13 +1016,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ld_expect(ld, kStateTileBytes + kCDTileBytes);
     ld_state_tile(ld, s0h, s0l, ws.S0, base);  // the chunk-start state, as the scan left it
     ld_cd_tile(ld, tsm + S::Wq, tsm + S::Wq + S::CDb, ws.W, base);  // W, as the prep kernel left it
-    int cn, hn;
-    if (next_item(chunk0, cn, hn)) {
-      const size_t nb = (size_t)cn * H + hn;
-      prefetch_tile(ws.S0, nb, kStateTileBytes);
-      prefetch_tile(ws.W, nb, kCDTileBytes);
-      prefetch_tile(ws.U, nb, kCDTileBytes);
-    }
   }
   gate_st(sG, LD, gr);
   __syncthreads();
@@ -1187,14 +1164,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
     ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
     ld_cc_tile(ld, tsm + S::Pt, tsm + S::Pt + S::CCb, ws.Pm, base);  // P, as the output kernel left it
-    int cn, hn;
-    if (next_item(chunk0, cn, hn)) {
-      const size_t nb = (size_t)cn * H + hn;
-      prefetch_tile(ws.S0, nb, kStateTileBytes);
-      prefetch_tile(ws.U, nb, kCDTileBytes);
-      prefetch_tile(ws.Pm, nb, kCCTileBytes);
-      prefetch_tile(ws.dS, nb, kStateTileBytes);
-    }
   }
   // bf16: the chunk's q and k rows into shared memory while the gates load and accumulate
   [[maybe_unused]] __nv_bfloat16* stq = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
@@ -1496,16 +1465,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (tid == 0) {
       ld_expect(ld, kCCTileBytes);
       ld_cc_tile(ld, tTh, tTl, ws.Tm, cb);
-      int cn, hn;
-      if (next_item(chunk0, cn, hn)) {
-        const size_t nb = (size_t)cn * H + hn;
-        prefetch_tile(ws.At, nb, sizeof(float) * C * C);
-        prefetch_tile(ws.Tm, nb, kCCTileBytes);
-        prefetch_tile(ws.S0, nb, kStateTileBytes);
-        prefetch_tile(ws.dUt, nb, kCDTileBytes);
-        prefetch_tile(ws.pdk, nb, sizeof(float) * C * D);
-        prefetch_tile(ws.pdG, nb, sizeof(float) * C * D);
-      }
     }
   }
   gate_st(sG, LD, gr);
