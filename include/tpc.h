@@ -537,7 +537,7 @@ int tpc_group_status(const tpc_plan* plan, const tpc_group_shape* shape, void* w
  *   Sizes: problems whose tables + workspace exceed TPC_STATIC_SCRATCH_BYTES are rejected with
  *       TPC_ERR_WORKSPACE and a message giving the bytes needed.
  *   Set-up: the first call on a device looks up the array's device address (with that device
- *       current); make that first call before any stream capture.
+ *       current).
  *   Sharing: every call uses the same array and it keeps the previous call's contents; the call
  *       clears its status word itself (tpc_kda_static_status reads it).  Calls that overlap on the GPU (other streams, other host
  *       threads) race on the array: serialise them.  tpc_kda_backward cannot follow this call (the

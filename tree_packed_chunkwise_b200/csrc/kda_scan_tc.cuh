@@ -16,24 +16,26 @@
 
 namespace tpc {
 
-// bytes of one chunk-head's additive-term slice (128 rows x 32 fp32)
-constexpr uint32_t kScanAddBytes = kTcD * kScanDVT * 4;
-
-template <bool REVERSE>
+// Slice width W of d_v per CTA: 32 (128 threads) or 64 (256 threads; half the CTAs, the same M
+// tile traffic per CTA, used when the round has more (sequence, head) pairs than fit in one wave of
+// 32-column CTAs).  Thread c owns row c % 128 of the state and columns 32 (c / 128) .. + 31 of the
+// slice.
+template <bool REVERSE, int W>
 struct ScanTcSmemT {
+  static constexpr int NT = 128 * (W / 32);
   static constexpr size_t M0 = 0, M1 = kMtileBytes;              // double-buffered M tiles
   static constexpr size_t St = 2 * size_t(kMtileBytes);          // state slice hi/lo (MN-major, K = 128)
-  static constexpr size_t StB = size_t(kTcD) * kScanDVT * 2;
-  // double-buffered: forward the B slices, reverse the Qeff tiles (hi/lo, C x D)
+  static constexpr size_t StB = size_t(kTcD) * W * 2;            // one half (hi or lo) of it
+  // forward: B columns [j0, j0 + W) (W / 32 consecutive 32-column slices); reverse: the Qeff tile
+  static constexpr size_t XB = REVERSE ? size_t(2) * kTcC * kTcD * 2 : size_t(kTcD) * W * 4;
+  static constexpr int NX = (REVERSE && W == 64) ? 1 : 2;       // X buffers (one where two do not fit)
   static constexpr size_t X = St + 2 * StB;
-  static constexpr size_t XB = REVERSE ? size_t(2) * kTcC * kTcD * 2 : size_t(kScanAddBytes);
-  // reverse: double-buffered dO slices, hi/lo operand tiles of C rows x 32 columns (k = row, n = column)
-  static constexpr size_t dO = X + 2 * XB;
-  static constexpr size_t dOB = REVERSE ? size_t(kTcC) * kScanDVT * 2 : 0;
+  // reverse: double-buffered dO slices, hi/lo operand tiles of C rows x W columns (k = row, n = column)
+  static constexpr size_t dOB = REVERSE ? size_t(kTcC) * W * 2 : 0;
+  static constexpr size_t dO = X + NX * XB;
   static constexpr size_t total = dO + 2 * 2 * dOB;
-  static_assert(total <= 227 * 1024, "shared memory");
+  static_assert(total <= 224 * 1024, "shared memory");
 };
-
 
 namespace tck {
 
@@ -49,21 +51,21 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* st
 // mbarrier with one expected-bytes arrival
 __device__ __forceinline__ void load_mtile(uint8_t* dst, const uint8_t* src, uint8_t* x_dst, const uint8_t* x_src,
                                            uint32_t x_bytes, uint64_t* bar) {
-  tc::mbar_arrive_expect_tx(bar, kMtileBytes + x_bytes);
+  tc::mbar_arrive_expect_tx(bar, kMtileBytes + (x_dst ? x_bytes : 0u));
   tc::bulk_g2s(dst, src, kMtileBytes, bar);
-  tc::bulk_g2s(x_dst, x_src, x_bytes, bar);
+  if (x_dst) tc::bulk_g2s(x_dst, x_src, x_bytes, bar);
 }
 
-// This CTA's 32 columns (j0 ..) of the chunk's dO rows as an MN-major operand tile (k = chunk row,
+// This CTA's W columns (j0 ..) of the chunk's dO rows as an MN-major operand tile (k = chunk row,
 // n = column; element (r, j) at cm_off(r, j, C)), hi (and lo for fp32 data); rows that are replays
 // or past the chunk's end are zero.  bf16: asynchronous 16-byte copies (completed by the caller with
 // cp_async_wait); fp32: loaded, split and stored now.
-template <typename Tin>
+template <typename Tin, int W>
 __device__ __forceinline__ void load_do_slice(uint8_t* hi, uint8_t* lo, const Tin* d_o, const ChunkRec& ch, int H,
                                               int h, int j0) {
-  constexpr int C = kTcC;
-  for (int p = threadIdx.x; p < C * (kScanDVT / 8); p += blockDim.x) {
-    const int r = p >> 2, g = p & 3;
+  constexpr int C = kTcC, G = W / 8;
+  for (int p = threadIdx.x; p < C * G; p += blockDim.x) {
+    const int r = p / G, g = p % G;
     const bool own = r >= ch.n_replay && r < ch.n_rows;
     const size_t row = own ? (size_t)(ch.row_start + (r - ch.n_replay)) : 0;
     const Tin* src = d_o + (row * H + h) * kTcD + j0 + 8 * g;
@@ -85,10 +87,11 @@ __device__ __forceinline__ void load_do_slice(uint8_t* hi, uint8_t* lo, const Ti
   if constexpr (sizeof(Tin) == 2) tc::cp_async_commit();
 }
 
-// state slice (row c = this thread, 32 columns) -> MN-major hi/lo operand tile (k = c, n = j)
-__device__ __forceinline__ void put_state(uint8_t* hi, uint8_t* lo, int c, const float (&s)[32]) {
-  put16<kTcD, true>(hi, lo, c, 0, s);
-  put16<kTcD, true>(hi, lo, c, 16, s + 16);
+// this thread's part of the state slice (row c, 32 columns from n0) -> MN-major hi/lo operand tile
+// (k = c, n = j)
+__device__ __forceinline__ void put_state(uint8_t* hi, uint8_t* lo, int c, int n0, const float (&s)[32]) {
+  put16<kTcD, true>(hi, lo, c, n0, s);
+  put16<kTcD, true>(hi, lo, c, n0 + 16, s + 16);
 }
 
 __device__ __forceinline__ void ld32g(const float* p, float (&v)[32]) {
@@ -107,51 +110,60 @@ __device__ __forceinline__ void st32g(float* p, const float (&v)[32]) {
 }  // namespace tck
 
 // REVERSE: d_o [N, H, D] (Tin) is the output gradient; forward: unused
-template <bool REVERSE, typename Tin>
-__global__ void __launch_bounds__(kScanThreads, 1)
+template <bool REVERSE, int W, typename Tin>
+__global__ void __launch_bounds__(128 * (W / 32), 1)
     kda_scan_tc(DevTables t, int seq0, int H, const float* __restrict__ init, float* __restrict__ final_state,
                 const float* __restrict__ d_final, KdaWs ws, const Tin* __restrict__ d_o) {
   using namespace tck;
-  using S = ScanTcSmemT<REVERSE>;
-  constexpr int D = kTcD, C = kTcC, DVT = kScanDVT;
+  using S = ScanTcSmemT<REVERSE, W>;
+  constexpr int D = kTcD, C = kTcC;
   constexpr bool EX = sizeof(Tin) == 2;  // bf16 dO: exact operand, no lo part
-  const int si = seq0 + blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVT;
+  const int si = seq0 + blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * W;
   const SeqRec sq = t.seqs[si];
   extern __shared__ __align__(1024) uint8_t tsm[];
   uint8_t* mbuf[2] = {tsm + S::M0, tsm + S::M1};
-  uint8_t* xbuf[2] = {tsm + S::X, tsm + S::X + S::XB};
+  uint8_t* xbuf[2] = {tsm + S::X, tsm + S::X + (S::NX == 2 ? S::XB : 0)};
   uint8_t* dobuf[2] = {tsm + S::dO, tsm + S::dO + 2 * S::dOB};  // hi, then lo at + dOB
   uint8_t *sth = tsm + S::St, *stl = sth + S::StB;
   __shared__ __align__(8) uint64_t bar_m[2];
+  __shared__ __align__(8) uint64_t bar_x;  // the single X buffer (S::NX == 1)
   __shared__ __align__(8) uint64_t bar_mma;
   __shared__ uint32_t tslot;
   __shared__ int s_ok;  // thread 0's bounded waits, read by every thread after the following barrier
-  const int c = threadIdx.x;  // state row / TMEM lane
-  if ((c >> 5) == 0) tc::tmem_alloc(&tslot, 32);
-  if (c == 0) {
+  const int c = threadIdx.x & 127, half = threadIdx.x >> 7;  // state row / TMEM lane; 32-column half
+  const int jc = j0 + 32 * half;                              // this thread's first column
+  const bool lead = threadIdx.x == 0;
+  if ((threadIdx.x >> 5) == 0) tc::tmem_alloc(&tslot, W);
+  if (lead) {
     tc::mbar_init(&bar_m[0], 1);
     tc::mbar_init(&bar_m[1], 1);
+    tc::mbar_init(&bar_x, 1);
     tc::mbar_init(&bar_mma, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tb = tslot;
-  const uint32_t la = tb + ((uint32_t)(32 * (c >> 5)) << 16);
+  const uint32_t la = tb + ((uint32_t)(32 * ((threadIdx.x >> 5) & 3)) << 16) + (uint32_t)(32 * half);
   float s[32];
   const int nch = sq.n_chunks;
   auto chunk_at = [&](int q) { return REVERSE ? sq.chunk_begin + nch - 1 - q : sq.chunk_begin + q; };
   auto mtile = [&](int ci) {
     return reinterpret_cast<const uint8_t*>(ws.Mt) + ((size_t)ci * H + h) * kMtileBytes;
   };
-  // forward: this CTA's slice of B; reverse: the chunk's Qeff tile (kept where the forward kept W)
+  // forward: this CTA's columns of B (consecutive 32-column slices); reverse: the chunk's Qeff tile
+  // (kept where the forward kept W)
   auto xsrc = [&](int ci) -> const uint8_t* {
     if (REVERSE) return reinterpret_cast<const uint8_t*>(ws.W) + ((size_t)ci * H + h) * S::XB;
-    return reinterpret_cast<const uint8_t*>(ws.Bc + ((size_t)ci * H + h) * D * D + (size_t)blockIdx.z * D * DVT);
+    return reinterpret_cast<const uint8_t*>(ws.Bc + ((size_t)ci * H + h) * D * D + (size_t)j0 * D);
   };
-  auto prefetch = [&](int q) {  // thread 0: bulk copies
+  auto prefetch = [&](int q) {  // thread 0: bulk copies (the M tile, and X when it is double-buffered)
     const int ci = chunk_at(q);
-    load_mtile(mbuf[q & 1], mtile(ci), xbuf[q & 1], xsrc(ci), (uint32_t)S::XB, &bar_m[q & 1]);
+    load_mtile(mbuf[q & 1], mtile(ci), S::NX == 2 ? xbuf[q & 1] : nullptr, xsrc(ci), (uint32_t)S::XB, &bar_m[q & 1]);
+  };
+  auto load_x_single = [&](int q) {  // thread 0, S::NX == 1: once the previous chunk's products are done
+    tc::mbar_arrive_expect_tx(&bar_x, (uint32_t)S::XB);
+    tc::bulk_g2s(xbuf[0], xsrc(chunk_at(q)), (uint32_t)S::XB, &bar_x);
   };
   // thread 0: the operands of a later chunk into L2 (the M tile once per (sequence, head), by the
   // first slice's CTA), so that the shared-memory copy a step ahead finds them there
@@ -164,7 +176,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   auto prefetch_do = [&](int q) {  // every thread
     if constexpr (REVERSE) {
       const ChunkRec ch = t.chunks[chunk_at(q)];
-      load_do_slice<Tin>(dobuf[q & 1], dobuf[q & 1] + S::dOB, d_o, ch, H, h, j0);
+      load_do_slice<Tin, W>(dobuf[q & 1], dobuf[q & 1] + S::dOB, d_o, ch, H, h, j0);
     }
   };
   // initial value: forward -> initial / imported state; reverse -> gradient of the final state
@@ -176,13 +188,14 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     } else if (d_final && sq.leaf >= 0) {  // a sequence ending at an internal node has no final state
       src = d_final + ((size_t)sq.leaf * H + h) * D * D;
     }
-    if (src) ld32g(src + c * D + j0, s);
+    if (src) ld32g(src + c * D + jc, s);
     else
       for (int j = 0; j < 32; ++j) s[j] = 0.f;
   }
   constexpr int kL2Ahead = 3;  // chunks prefetched into L2 ahead of the current one
-  if (c == 0) {
+  if (lead) {
     prefetch(0);
+    if constexpr (S::NX == 1) load_x_single(0);
     for (int q = 1; q < kL2Ahead; ++q) prefetch_l2(q);
   }
   prefetch_do(0);
@@ -193,23 +206,25 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   for (int q = 0; q < nch && ok; ++q) {
     const int ci = chunk_at(q);
     const size_t base = (size_t)ci * H + h;
+    uint8_t* xq = xbuf[S::NX == 2 ? (q & 1) : 0];
     if (REVERSE) {
       const int slot = t.chunks[ci].export_slot;
       if (slot >= 0) {  // gradients of the exported boundary state, consumers in a fixed order
         const SlotRec sr = t.slots[slot];
         for (int m = 0; m < sr.n_cons; ++m) {
           float g2[32];
-          ld32g(ws.dS0seq + ((size_t)t.slot_cons[sr.cons_begin + m] * H + h) * D * D + c * D + j0, g2);
+          ld32g(ws.dS0seq + ((size_t)t.slot_cons[sr.cons_begin + m] * H + h) * D * D + c * D + jc, g2);
           for (int j = 0; j < 32; ++j) s[j] += g2[j];
         }
       }
     }
-    put_state(sth, stl, c, s);
+    put_state(sth, stl, c, 32 * half, s);
     if constexpr (REVERSE && EX) tc::cp_async_wait<0>();  // this chunk's dO slice (issued a step ago)
-    if (c == 0) {
+    if (lead) {
       if (q + 1 < nch) prefetch(q + 1);
       prefetch_l2(q + kL2Ahead);
-      const bool w = tc::mbar_wait(&bar_m[q & 1], (q >> 1) & 1);
+      bool w = tc::mbar_wait(&bar_m[q & 1], (q >> 1) & 1);
+      if constexpr (S::NX == 1) w = w && tc::mbar_wait(&bar_x, q & 1);
       if (!w) set_status(ws.status, kStatusTimeout);
       s_ok = w ? 1 : 0;
     }
@@ -220,30 +235,32 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     tc::fence_after_sync();
     ok = s_ok != 0;
     if (!ok) break;
-    float add[32];  // forward: B of this chunk, row c of the slice (16-byte groups permuted by c mod 8)
+    float add[32];  // forward: B of this chunk, row c of this thread's 32-column slice (16-byte groups
+                    // permuted by c mod 8)
     if constexpr (!REVERSE) {
-      const float* ab = reinterpret_cast<const float*>(xbuf[q & 1]);
+      const float* ab = reinterpret_cast<const float*>(xq) + ((size_t)half * D + c) * 32;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 u = reinterpret_cast<const float4*>(ab + c * DVT)[i ^ (c & 7)];
+        const float4 u = reinterpret_cast<const float4*>(ab)[i ^ (c & 7)];
         add[4 * i] = u.x; add[4 * i + 1] = u.y; add[4 * i + 2] = u.z; add[4 * i + 3] = u.w;
       }
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) add[j] = 0.f;
     }
-    if (c == 0) {
+    if (lead) {
       const tc::Op mH{tc::smem_u32(mbuf[q & 1]), D, REVERSE}, mL{tc::smem_u32(mbuf[q & 1] + kMtileBytes / 2), D, REVERSE};
       const tc::Op sH{tc::smem_u32(sth), D, true}, sL{tc::smem_u32(stl), D, true};
-      mma4(tb, mH, mL, sH, sL, D, tc::idesc_bf16(D, DVT, REVERSE, true), false, false, false);
+      mma4(tb, mH, mL, sH, sL, D, tc::idesc_bf16(D, W, REVERSE, true), false, false, false);
       if constexpr (REVERSE) {  // + Qeff^T dO (A: the Qeff tile read MN-major, k = chunk row)
-        const tc::Op eH{tc::smem_u32(xbuf[q & 1]), C, true}, eL{tc::smem_u32(xbuf[q & 1] + S::XB / 2), C, true};
+        const tc::Op eH{tc::smem_u32(xq), C, true}, eL{tc::smem_u32(xq + S::XB / 2), C, true};
         const tc::Op oH{tc::smem_u32(dobuf[q & 1]), C, true}, oL{tc::smem_u32(dobuf[q & 1] + S::dOB), C, true};
-        mma4(tb, eH, eL, oH, oL, C, tc::idesc_bf16(D, DVT, true, true), true, false, EX);
+        mma4(tb, eH, eL, oH, oL, C, tc::idesc_bf16(D, W, true, true), true, false, EX);
       }
       tc::commit(&bar_mma);
       // the state slice tile goes to the chunk kernels as it is: forward the chunk-start state S0,
-      // reverse the gradient of the chunk-end state (hi/lo operand tiles, this slice's 8 KB of each)
+      // reverse the gradient of the chunk-end state (hi/lo operand tiles; this slice's columns are
+      // contiguous in each half)
       uint8_t* dst = reinterpret_cast<uint8_t*>(REVERSE ? ws.dS : ws.S0) + base * kStateTileBytes +
                      (size_t)blockIdx.z * S::StB;
       tc::bulk_s2g(dst, sth, (uint32_t)S::StB);
@@ -256,33 +273,35 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
     mma_phase ^= 1u;
     tc::fence_before_sync();
-    __syncthreads();  // products in TMEM; this chunk's M buffer free again
+    __syncthreads();  // products in TMEM; this chunk's M buffer (and the single X buffer) free again
     tc::fence_after_sync();
     ok = s_ok != 0;
     if (!ok) break;
+    if constexpr (S::NX == 1)
+      if (lead && q + 1 < nch) load_x_single(q + 1);
     float acc[32];
     tc::tmem_ld32(la, acc);
     for (int j = 0; j < 32; ++j) s[j] = acc[j] + add[j];
     if (!REVERSE) {
       const int slot = t.chunks[ci].export_slot;
-      if (slot >= 0) st32g(ws.slot + ((size_t)slot * H + h) * D * D + c * D + j0, s);
+      if (slot >= 0) st32g(ws.slot + ((size_t)slot * H + h) * D * D + c * D + jc, s);
     }
   }
   if (ok) {
     if (!REVERSE) {
-      if (final_state && sq.leaf >= 0) st32g(final_state + ((size_t)sq.leaf * H + h) * D * D + c * D + j0, s);
+      if (final_state && sq.leaf >= 0) st32g(final_state + ((size_t)sq.leaf * H + h) * D * D + c * D + jc, s);
     } else {
-      st32g(ws.dS0seq + ((size_t)si * H + h) * D * D + c * D + j0, s);
+      st32g(ws.dS0seq + ((size_t)si * H + h) * D * D + c * D + jc, s);
     }
-  } else {
+  } else if (lead) {
     // give copies still in flight a last bounded chance before the shared memory is released
     tc::mbar_wait(&bar_m[0], 0, 200000000ull);
   }
   if constexpr (REVERSE && EX) tc::cp_async_wait<0>();
-  if (c == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
+  if (lead) tc::bulk_wait_read();  // (the stores complete with the grid)
   tc::fence_before_sync();
   __syncthreads();
-  if ((c >> 5) == 0) tc::tmem_dealloc(tb, 32);
+  if ((threadIdx.x >> 5) == 0) tc::tmem_dealloc(tb, W);
 }
 
 }  // namespace tpc

@@ -204,6 +204,11 @@ int stream_after(cudaStream_t to, cudaStream_t from) {
   return TPC_OK;
 }
 
+// State scans of a round: 64-column CTAs (half as many, each reading the M tile once for twice the
+// columns) when the round's (sequence, head) pairs would take more than one wave of 32-column CTAs
+// (one scan CTA per SM); 32-column CTAs otherwise (more CTAs for a short round's latency-bound chain)
+bool scan_wide(int n_seqs, int H) { return (long long)n_seqs * H * (tpc::kTcD / 32) > tpc_abi::sm_count(); }
+
 template <int C, int D, typename Tin, typename Tout, bool TC>
 int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_io* io, void* ws, cudaStream_t st) {
   using namespace tpc;
@@ -229,7 +234,8 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     // stream after prep(r) and scan(r - 1).  The caller's stream runs prep(1..R), out(1..R) in that
     // order, so the later rounds' prep overlaps scan(1) and out(r) overlaps scan(r + 1).
     TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmemT<Tin>::total));
-    TPC_CUDA(set_smem(kda_scan_tc<false, Tin>, ScanTcSmemT<false>::total));
+    TPC_CUDA(set_smem(kda_scan_tc<false, 32, Tin>, ScanTcSmemT<false, 32>::total));
+    TPC_CUDA(set_smem(kda_scan_tc<false, 64, Tin>, ScanTcSmemT<false, 64>::total));
     TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
     cudaStream_t hs = scan_stream();
     if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
@@ -241,11 +247,16 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
                    (kda_fwd_prep_tc<Tin><<<dim3(c1 - c0, H), kTcThreads, PrepTcSmemT<Tin>::total, st>>>(p.dt, H, k, v, g, b,
                                                                                                   w, c0)));
       TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
-      if (s1 > s0)
-        TPC_LAUNCH("kda_fwd_scan_tc", hs,
-                   (kda_scan_tc<false, Tin><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads,
-                                              ScanTcSmemT<false>::total, hs>>>(p.dt, s0, H, io->init_state,
-                                                                              io->final_state, nullptr, w, nullptr)));
+      if (s1 > s0) {
+        if (scan_wide(s1 - s0, H))
+          TPC_LAUNCH("kda_fwd_scan_tc", hs,
+                     (kda_scan_tc<false, 64, Tin><<<dim3(s1 - s0, H, D / 64), 256, ScanTcSmemT<false, 64>::total, hs>>>(
+                         p.dt, s0, H, io->init_state, io->final_state, nullptr, w, nullptr)));
+        else
+          TPC_LAUNCH("kda_fwd_scan_tc", hs,
+                     (kda_scan_tc<false, 32, Tin><<<dim3(s1 - s0, H, D / 32), 128, ScanTcSmemT<false, 32>::total, hs>>>(
+                         p.dt, s0, H, io->init_state, io->final_state, nullptr, w, nullptr)));
+      }
       scans.emplace_back();
       TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
@@ -299,7 +310,8 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
     // Rounds in reverse: the reverse scan(r) (which also forms the output's contribution Qeff^T dO)
     // on the high-priority scan stream after the caller's prior work and scan(r + 1); then dq(r),
     // dk/dv(r) on the caller's stream after scan(r), so dq / dk-dv(r) overlap scan(r - 1).
-    TPC_CUDA(set_smem(kda_scan_tc<true, Tin>, ScanTcSmemT<true>::total));
+    TPC_CUDA(set_smem(kda_scan_tc<true, 32, Tin>, ScanTcSmemT<true, 32>::total));
+    TPC_CUDA(set_smem(kda_scan_tc<true, 64, Tin>, ScanTcSmemT<true, 64>::total));
     TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
     TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmemT<Tin>::total));
     cudaStream_t hs = scan_stream();
@@ -307,10 +319,16 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
     TPC_TRY_ABI(stream_after(hs, st));  // the scans after the caller's prior work (forward, d_o)
     for (int r = p.n_rounds; r >= 1; --r) {
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-      if (s1 > s0)
-        TPC_LAUNCH("kda_bwd_scan_tc", hs,
-                   (kda_scan_tc<true, Tin><<<dim3(s1 - s0, H, D / kScanDVT), kScanThreads, ScanTcSmemT<true>::total,
-                                             hs>>>(p.dt, s0, H, nullptr, nullptr, io->d_final, w, dO)));
+      if (s1 > s0) {
+        if (scan_wide(s1 - s0, H))
+          TPC_LAUNCH("kda_bwd_scan_tc", hs,
+                     (kda_scan_tc<true, 64, Tin><<<dim3(s1 - s0, H, D / 64), 256, ScanTcSmemT<true, 64>::total, hs>>>(
+                         p.dt, s0, H, nullptr, nullptr, io->d_final, w, dO)));
+        else
+          TPC_LAUNCH("kda_bwd_scan_tc", hs,
+                     (kda_scan_tc<true, 32, Tin><<<dim3(s1 - s0, H, D / 32), 128, ScanTcSmemT<true, 32>::total, hs>>>(
+                         p.dt, s0, H, nullptr, nullptr, io->d_final, w, dO)));
+      }
       scans.emplace_back();
       TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
