@@ -701,33 +701,40 @@ __device__ __forceinline__ void block_inverse(float* T, const float* L, float* W
     for (int r = 0; r < 16; ++r) T[(16 * p + r) * LC + 16 * p + c] = col[r];
   }
   __syncthreads();
-  // off-diagonal blocks by distance d = p - q: T_pq = -T_pp * (sum_s L_ps T_sq)
+  // off-diagonal blocks by distance d = p - q: T_pq = -T_pp * (sum_s L_ps T_sq); the distance loop is
+  // unrolled so that every inner sum has a constant length (T_pp is zero above its diagonal, so the
+  // second product runs over all 16 columns)
+#pragma unroll
   for (int d = 1; d < 4; ++d) {
     const int nb = 4 - d;  // blocks (p, p - d), p = d .. 3
     // W1[j] = sum_{s=q}^{p-1} L_ps T_sq
     for (int e = tid; e < nb * 256; e += blockDim.x) {
       const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
       const int p = d + j, q = j;
+      const float* Lr = L + (16 * p + r) * LC + 16 * q;
+      const float* Tc = T + (16 * q) * LC + 16 * q + c;
       float acc = 0.f;
-      for (int s = q; s < p; ++s)
-        for (int k = 0; k < 16; ++k)
-          acc = fmaf(L[(16 * p + r) * LC + 16 * s + k], T[(16 * s + k) * LC + 16 * q + c], acc);
+#pragma unroll
+      for (int k = 0; k < 16 * d; ++k) acc = fmaf(Lr[k], Tc[k * LC], acc);
       W1[j * BB + r * P + c] = acc;
     }
     __syncthreads();
     for (int e = tid; e < nb * 256; e += blockDim.x) {
       const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
       const int p = d + j, q = j;
+      const float* Tr = T + (16 * p + r) * LC + 16 * p;
       float acc = 0.f;
-      for (int k = 0; k <= r; ++k) acc = fmaf(T[(16 * p + r) * LC + 16 * p + k], W1[j * BB + k * P + c], acc);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc = fmaf(Tr[k], W1[j * BB + k * P + c], acc);
       T[(16 * p + r) * LC + 16 * q + c] = -acc;
     }
     __syncthreads();
   }
-  // upper blocks are zero
-  for (int e = tid; e < 64 * 64; e += blockDim.x) {
-    const int r = e >> 6, c = e & 63;
-    if ((c >> 4) > (r >> 4)) T[r * LC + c] = 0.f;
+  // upper blocks (p < q) are zero
+  for (int e = tid; e < 6 * 256; e += blockDim.x) {
+    const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
+    const int p = b < 3 ? 0 : (b < 5 ? 1 : 2), q = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
+    T[(16 * p + r) * LC + 16 * q + c] = 0.f;
   }
   __syncthreads();
 }
