@@ -197,28 +197,32 @@ __device__ __forceinline__ void build_tile2_raw(uint8_t* hi1, uint8_t* lo1, uint
 // Gate rows of the chunk into G (fp32, pitch LD) in two steps, so that a kernel issues these loads
 // before its larger copies and stores them once they arrive: gate_ld (16-byte loads into registers)
 // and gate_st (neighbouring threads take neighbouring rows: conflict-free stores).  Rows >= n are zero.
+// (the loaded 16-byte pieces stay raw until gate_st, so that nothing waits for them before then)
+template <typename T>
 struct GateRegs {
-  float x[kTcC * (kTcD / 8) / kTcThreads][8];
+  static constexpr int IT = kTcC * (kTcD / 8) / kTcThreads, Q = sizeof(T) / 2;  // uint4 per 8 values
+  uint4 u[IT][Q];
 };
 template <typename T>
-__device__ __forceinline__ void gate_ld(GateRegs& gr, const T* g_, const int* rows, int H, int h, int n) {
-  constexpr int IT = kTcC * (kTcD / 8) / kTcThreads;
+__device__ __forceinline__ void gate_ld(GateRegs<T>& gr, const T* g_, const int* rows, int H, int h, int n) {
 #pragma unroll
-  for (int it = 0; it < IT; ++it) {
+  for (int it = 0; it < GateRegs<T>::IT; ++it) {
     const int e = threadIdx.x + it * kTcThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
-    if (a < n) ld8(g_ + ((size_t)rows[a] * H + h) * kTcD + b0, gr.x[it]);
-    else
+    const T* p = g_ + ((size_t)(a < n ? rows[a] : 0) * H + h) * kTcD + b0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) gr.x[it][j] = 0.f;
+    for (int q = 0; q < GateRegs<T>::Q; ++q)
+      gr.u[it][q] = a < n ? __ldg(reinterpret_cast<const uint4*>(p) + q) : make_uint4(0u, 0u, 0u, 0u);
   }
 }
-__device__ __forceinline__ void gate_st(float* G, int LD, const GateRegs& gr) {
-  constexpr int IT = kTcC * (kTcD / 8) / kTcThreads;
+template <typename T>
+__device__ __forceinline__ void gate_st(float* G, int LD, const GateRegs<T>& gr) {
 #pragma unroll
-  for (int it = 0; it < IT; ++it) {
+  for (int it = 0; it < GateRegs<T>::IT; ++it) {
     const int e = threadIdx.x + it * kTcThreads, a = e % kTcC, b0 = (e / kTcC) * 8;
+    float x[8];
+    raw_get<T>(gr.u[it], x);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) G[a * LD + b0 + j] = gr.x[it][j];
+    for (int j = 0; j < 8; ++j) G[a * LD + b0 + j] = x[j];
   }
 }
 
@@ -829,15 +833,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // bf16: the chunk's k and v rows into shared memory while the gates load and accumulate
   [[maybe_unused]] __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
   [[maybe_unused]] __nv_bfloat16* sv = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
-  GateRegs gr;
+  GateRegs<Tin> gr;
   gate_ld(gr, g_, srow, H, h, n);  // gates and beta first
-  const float bv = tid < n ? to_f(beta_[(size_t)srow[tid] * H + h]) : 0.f;
+  const Tin bv = tid < n ? beta_[(size_t)srow[tid] * H + h] : Tin(0.f);  // (converted when stored)
   if constexpr (EX) {
     stage_rows_async(sk, k_, srow, H, h, n);
     stage_rows_async(sv, v_, srow, H, h, n);
   }
   gate_st(sG, LD, gr);
-  if (tid < C) sb[tid] = bv;
+  if (tid < C) sb[tid] = to_f(bv);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, ws.status, reinterpret_cast<float*>(tl));  // (tiles not yet in use)
   if constexpr (EX) tc::cp_async_wait<0>();
@@ -1014,7 +1018,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
   auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  GateRegs gr;
+  GateRegs<Tin> gr;
   gate_ld(gr, g_, srow, H, h, n);  // gates, q and k first, then the workspace tiles
   RawTile<Tin, C, D> rq, rk;
   raw_ld(rq, row_q);
@@ -1164,7 +1168,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  GateRegs gr;
+  GateRegs<Tin> gr;
   gate_ld(gr, g_, srow, H, h, n);  // gates first, then the workspace tiles and the row gathers
   if (tid == 0) {
     ld_expect(ld, kStateTileBytes + kCDTileBytes + kCCTileBytes);
@@ -1454,9 +1458,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  GateRegs gr;
+  GateRegs<Tin> gr;
   gate_ld(gr, g_, srow, H, h, n);  // gates and beta first, then the copies
-  const float bv = tid < n ? to_f(beta_[(size_t)srow[tid] * H + h]) : 0.f;
+  const Tin bv = tid < n ? beta_[(size_t)srow[tid] * H + h] : Tin(0.f);  // (converted when stored)
   for (int e = tid; e < 3 * kTcGroups * C; e += blockDim.x) sdb[e] = 0.f;
   Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
   auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
@@ -1475,7 +1479,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   gate_st(sG, LD, gr);
-  if (tid < C) sb[tid] = bv;
+  if (tid < C) sb[tid] = to_f(bv);
   __syncthreads();
   cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(R));  // (R's first phase comes later)
   float* se0 = sdb + 3 * kTcGroups * C;  // per channel 2^{G_0}
