@@ -572,6 +572,10 @@ __device__ __forceinline__ void ld_expect(Ld& l, uint32_t bytes) { tc::mbar_arri
 // one chunk-head's state tile (S0 or dS: hi half then lo half, kStateTileBytes) into hi and lo
 __device__ __forceinline__ void ld_state_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
   const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kStateTileBytes;
+  if (lo == hi + kStateTileBytes / 2) {  // halves adjacent in shared memory: one copy
+    tc::bulk_g2s(hi, src, kStateTileBytes, l.bar);
+    return;
+  }
   tc::bulk_g2s(hi, src, kStateTileBytes / 2, l.bar);
   tc::bulk_g2s(lo, src + kStateTileBytes / 2, kStateTileBytes / 2, l.bar);
 }
@@ -580,11 +584,19 @@ __device__ __forceinline__ void ld_state_tile(Ld& l, uint8_t* hi, uint8_t* lo, c
 constexpr uint32_t kCDTileBytes = 2u * kTcC * kTcD * 2u, kCCTileBytes = 2u * kTcC * kTcC * 2u;
 __device__ __forceinline__ void ld_cd_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
   const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kCDTileBytes;
+  if (lo == hi + kCDTileBytes / 2) {  // halves adjacent in shared memory: one copy
+    tc::bulk_g2s(hi, src, kCDTileBytes, l.bar);
+    return;
+  }
   tc::bulk_g2s(hi, src, kCDTileBytes / 2, l.bar);
   tc::bulk_g2s(lo, src + kCDTileBytes / 2, kCDTileBytes / 2, l.bar);
 }
 __device__ __forceinline__ void ld_cc_tile(Ld& l, uint8_t* hi, uint8_t* lo, const float* tiles, size_t base) {
   const uint8_t* src = reinterpret_cast<const uint8_t*>(tiles) + base * kCCTileBytes;
+  if (lo == hi + kCCTileBytes / 2) {  // halves adjacent in shared memory: one copy
+    tc::bulk_g2s(hi, src, kCCTileBytes, l.bar);
+    return;
+  }
   tc::bulk_g2s(hi, src, kCCTileBytes / 2, l.bar);
   tc::bulk_g2s(lo, src + kCCTileBytes / 2, kCCTileBytes / 2, l.bar);
 }
@@ -593,14 +605,22 @@ __device__ __forceinline__ void ld_cc_tile(Ld& l, uint8_t* hi, uint8_t* lo, cons
 // complete with the grid)
 __device__ __forceinline__ void store_cd_tile(float* tiles, size_t base, const uint8_t* hi, const uint8_t* lo) {
   uint8_t* dst = reinterpret_cast<uint8_t*>(tiles) + base * kCDTileBytes;
-  tc::bulk_s2g(dst, hi, kCDTileBytes / 2);
-  tc::bulk_s2g(dst + kCDTileBytes / 2, lo, kCDTileBytes / 2);
+  if (lo == hi + kCDTileBytes / 2) {  // halves adjacent in shared memory: one copy
+    tc::bulk_s2g(dst, hi, kCDTileBytes);
+  } else {
+    tc::bulk_s2g(dst, hi, kCDTileBytes / 2);
+    tc::bulk_s2g(dst + kCDTileBytes / 2, lo, kCDTileBytes / 2);
+  }
   tc::bulk_commit();
 }
 __device__ __forceinline__ void store_cc_tile(float* tiles, size_t base, const uint8_t* hi, const uint8_t* lo) {
   uint8_t* dst = reinterpret_cast<uint8_t*>(tiles) + base * kCCTileBytes;
-  tc::bulk_s2g(dst, hi, kCCTileBytes / 2);
-  tc::bulk_s2g(dst + kCCTileBytes / 2, lo, kCCTileBytes / 2);
+  if (lo == hi + kCCTileBytes / 2) {  // halves adjacent in shared memory: one copy
+    tc::bulk_s2g(dst, hi, kCCTileBytes);
+  } else {
+    tc::bulk_s2g(dst, hi, kCCTileBytes / 2);
+    tc::bulk_s2g(dst + kCCTileBytes / 2, lo, kCCTileBytes / 2);
+  }
   tc::bulk_commit();
 }
 // element (i, c) of a C x D hi/lo tile in global memory, 16 consecutive c from c0, as fp32 (hi + lo)
@@ -945,20 +965,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int j = 0; j < 16; ++j) m[j] = (c0 + j == c ? gam : 0.f) - v[j];
           put16<D, true>(mts, mts + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
         });
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {  // M leaves while B is assembled
+          tc::bulk_s2g(Mt, mts, kMtileBytes);
+          tc::bulk_commit();
+        }
         acc_read<D, D>(tb, 128, [&](int c, int j0, const float* v) {  // slice-major for the scan's bulk loads
           float* dst = kBsm ? bs : Bg;
           for (int j = 0; j < 16; j += 4)
             *reinterpret_cast<float4*>(dst + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         });
-        tc::fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-          constexpr uint32_t kPiece = 16384;
-          for (uint32_t o = 0; o < kMtileBytes; o += kPiece) tc::bulk_s2g(Mt + o, mts + o, kPiece);
-          if constexpr (kBsm)
-            for (uint32_t o = 0; o < sizeof(float) * D * D; o += kPiece)
-              tc::bulk_s2g(reinterpret_cast<uint8_t*>(Bg) + o, reinterpret_cast<const uint8_t*>(bs) + o, kPiece);
-          tc::bulk_commit();
+        if constexpr (kBsm) {
+          tc::fence_async_smem();
+          __syncthreads();
+          if (tid == 0) {
+            tc::bulk_s2g(Bg, bs, sizeof(float) * D * D);
+            tc::bulk_commit();
+          }
         }
       }
     }
@@ -1433,23 +1457,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
-  for (int i = tid; i < C; i += blockDim.x) {
-    const int row = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
-    srow[i] = row;
-    int kind = 2, idx = row;
-    if (i < ch.n_replay) {
-      kind = 0;
-      idx = ch.replay_base + i;
-    } else if (i < n) {
-      const int tg = t.row_tgt[row];
-      if (tg >= 0) {
-        kind = 1;
-        idx = tg;
-      }
-    }
-    skind[i] = kind;
-    sidx[i] = idx;
-  }
+  for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
   Ld ld{&bar_ld, 0u, ws.status};
   if (tid == 0) {
@@ -1477,6 +1485,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ld_expect(ld, kCCTileBytes);
       ld_cc_tile(ld, tTh, tTl, ws.Tm, cb);
     }
+  }
+  if (tid < C) {  // where row tid's gradients go (read while the gates are in flight)
+    const int i = tid, row = srow[i];
+    int kind = 2, idx = row;
+    if (i < ch.n_replay) {
+      kind = 0;
+      idx = ch.replay_base + i;
+    } else if (i < n) {
+      const int tg = t.row_tgt[row];
+      if (tg >= 0) {
+        kind = 1;
+        idx = tg;
+      }
+    }
+    skind[i] = kind;
+    sidx[i] = idx;
   }
   gate_st(sG, LD, gr);
   if (tid < C) sb[tid] = to_f(bv);
