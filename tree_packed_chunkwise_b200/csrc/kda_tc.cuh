@@ -1532,6 +1532,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int myrow = 16 * sp + (lane & 15);  // M = 64 accumulator row; this lane's 8 columns: share8
   const int half8 = 8 * (lane >> 4);
   float pre_dk[2][8], pre_dG[2][8];  // the final phase's dq-kernel partials (loaded ahead)
+  uint4 vraw[2][sizeof(Tin) / 2];     // phase 4's v values (loaded ahead, raw)
   // 8 gradient values of row r from column c0 on, to where the row's gradients go
   auto out8 = [&](float* replay_buf, float* tgt_buf, Tout* out, int r, int c0, const float* v) {
     const size_t o = ((size_t)sidx[r] * H + h) * D + c0;
@@ -1591,6 +1592,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (ok) {
     // ---- phase 3: X (K-major, rows i, columns n in [0, 2D)) and dX (MN-major, k = r, n)
     uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb, *dxh = R + S::p3_dX, *dxl = dxh + 2 * S::CDb;
+    // this lane's v values for phase 4 (its rows' columns of dB_v), loaded now and converted there
+    static_assert(2 * D == 4 * 16 * kTcGroups, "four 16-column chunks of dB per warp group");
+    for (int t2 = 0; t2 < 2; ++t2) {
+      const int c1 = grp * 16 + 16 * kTcGroups * t2 + half8;
+      const Tin* p = v_ + ((size_t)srow[myrow] * H + h) * D + c1;
+#pragma unroll
+      for (int q = 0; q < (int)(sizeof(Tin) / 2); ++q)
+        vraw[t2][q] = myrow < n ? __ldg(reinterpret_cast<const uint4*>(p) + q) : make_uint4(0u, 0u, 0u, 0u);
+    }
     acc_read<C, D>(tb, cW, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, c0, v); });
     acc_read<C, D>(tb, cU, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, D + c0, v); });
     acc_read<C, D>(tb, cdW, [&](int r, int c0, const float* v) {
@@ -1608,7 +1618,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (ok) {
     // ---- read dB: dB tile for dA; dv; dk / dG / dbeta contributions
     uint8_t *dbh = R + S::p4_dB, *dbl = dbh + 2 * S::CDb;
-    for (int cc = grp * 16; cc < 2 * D; cc += 16 * kTcGroups) {
+#pragma unroll
+    for (int t4 = 0; t4 < 4; ++t4) {
+      const int cc = grp * 16 + 16 * kTcGroups * t4;
       float v[8];
       {
         float v16[16];
@@ -1618,7 +1630,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int i = myrow, c0 = cc + half8;
       put8<C, true>(dbh, dbl, i, c0, v);
       float part = 0.f;
-      if (cc < D) {  // (the dk / dG terms of dB_k are added in the last phase, from TMEM)
+      if (t4 < 2) {  // columns < D: dB_k (its dk / dG terms are added in the last phase, from TMEM)
         float kv[8];
         k8(i, c0, kv);
 #pragma unroll
@@ -1626,7 +1638,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       } else if (i < n) {
         const int c1 = c0 - D;
         float vv[8], val[8];
-        ld8(v_ + ((size_t)srow[i] * H + h) * D + c1, vv);
+        raw_get<Tin>(vraw[t4 - 2], vv);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           part = fmaf(v[j], vv[j], part);
@@ -1635,7 +1647,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         out8(ws.rdv, ws.tdv, dv_, i, c1, val);
       }
       part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);  // columns 0-7 + 8-15 of the chunk
-      if (lane < 16) sdb[((cc < D ? 0 : 1) * kTcGroups + grp) * C + i] += part;  // one slot per (half, group)
+      if (lane < 16) sdb[((t4 < 2 ? 0 : 1) * kTcGroups + grp) * C + i] += part;  // one slot per (half, group)
     }
     uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb;
     ok = run(sy, [&] {
