@@ -518,6 +518,7 @@ def measure_agentic(args, world, rank, tpc, torch):
             ems = kda_step_timer(tpc, torch, eplan, xe, H, d, world, 2, 2)
             out["expanded_path"] = {"ms_per_step": ems, "speedup_tree_vs_expanded": ems / ms,
                                     "target_speedup": info["n_expanded"] / info["n_seq_tokens"],
+                                    "chunk_ratio": eplan.info["n_chunks"] / info["n_chunks"],
                                     "expanded_chunks": eplan.info["n_chunks"]}
             del xe
         else:
@@ -730,9 +731,11 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world) / ek
+        # (the kernels work in whole chunks, so the chunk-count ratio bounds the speed-up they can reach)
         expanded = {"ms_per_step": ems, "expanded_tokens_per_s": world * info["n_expanded"] / (ems / 1e3),
                     "speedup_tree_vs_expanded": ems / ms_step,
-                    "target_speedup": info["n_expanded"] / info["n_seq_tokens"]}
+                    "target_speedup": info["n_expanded"] / info["n_seq_tokens"],
+                    "chunk_ratio": eplan.info["n_chunks"] / info["n_chunks"]}
         del ews, xe, eg
 
     # ---- end to end through the C ABI with host buffers: every step uploads its inputs from pinned
