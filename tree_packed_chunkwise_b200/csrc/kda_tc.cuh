@@ -826,7 +826,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using S = PrepTcSmemT<Tin>;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -1019,7 +1019,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using namespace tck;
   using S = OutTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD;
-  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -1170,7 +1170,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using S = BdqTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -1438,7 +1438,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using S = BdkvTcSmemT<Tin>;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = chunk0 + (int)blockIdx.x, h = blockIdx.y;
+  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];

@@ -204,6 +204,11 @@ int stream_after(cudaStream_t to, cudaStream_t from) {
   return TPC_OK;
 }
 
+// Chunk kernels run on grids (heads, chunks): the heads of one chunk are neighbouring CTAs, so the
+// CTAs in flight read whole token rows ([N, H, D] inputs) and consecutive workspace tiles; a round
+// with more chunks than a grid's y extent allows is launched in pieces.
+constexpr int kMaxGridY = 65535;
+
 // State scans of a round: 64-column CTAs (half as many, each reading the M tile once for twice the
 // columns) when the round's (sequence, head) pairs would take more than one wave of 32-column CTAs
 // (one scan CTA per SM); 32-column CTAs otherwise (more CTAs for a short round's latency-bound chain)
@@ -242,10 +247,10 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     for (int r = 1; r <= p.n_rounds; ++r) {
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-      if (c1 > c0)
+      for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_fwd_prep_tc", st,
-                   (kda_fwd_prep_tc<Tin><<<dim3(c1 - c0, H), kTcThreads, PrepTcSmemT<Tin>::total, st>>>(p.dt, H, k, v, g, b,
-                                                                                                  w, c0)));
+                   (kda_fwd_prep_tc<Tin><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads, PrepTcSmemT<Tin>::total,
+                                           st>>>(p.dt, H, k, v, g, b, w, a)));
       TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
       if (s1 > s0) {
         if (scan_wide(s1 - s0, H))
@@ -265,10 +270,10 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       TPC_CUDA(cudaStreamWaitEvent(st, scans[r - 1], 0));
       TPC_CUDA(cudaEventDestroy(scans[r - 1]));
-      if (c1 > c0)
+      for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_fwd_out_tc", st,
-                   (kda_fwd_out_tc<Tin, Tout><<<dim3(c1 - c0, H), kTcThreads, OutTcSmem::total, st>>>(
-                       p.dt, H, q, k, g, static_cast<Tout*>(io->o), w, c0)));
+                   (kda_fwd_out_tc<Tin, Tout><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads, OutTcSmem::total, st>>>(
+                       p.dt, H, q, k, g, static_cast<Tout*>(io->o), w, a)));
     }
   } else {
     TPC_LAUNCH("kda_fwd_prep", st,
@@ -337,15 +342,16 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       TPC_CUDA(cudaStreamWaitEvent(st, scans[i], 0));
       TPC_CUDA(cudaEventDestroy(scans[i]));
-      if (c1 > c0) {
+      for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_bwd_dq_tc", st,
-                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(c1 - c0, H), kTcThreads, BdqTcSmem::total, st>>>(
-                       p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w, c0)));
+                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads, BdqTcSmem::total, st>>>(
+                       p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w, a)));
+      for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_bwd_dkv_tc", st,
-                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(c1 - c0, H), kTcThreads, BdkvTcSmemT<Tin>::total, st>>>(
+                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads,
+                                                BdkvTcSmemT<Tin>::total, st>>>(
                        p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg,
-                       io->dbeta, w, c0)));
-      }
+                       io->dbeta, w, a)));
     }
   } else {
     TPC_LAUNCH("kda_bwd_prep", st,
