@@ -23,18 +23,21 @@ namespace tpc {
 template <bool REVERSE, int W>
 struct ScanTcSmemT {
   static constexpr int NT = 128 * (W / 32);
-  static constexpr size_t M0 = 0, M1 = kMtileBytes;              // double-buffered M tiles
-  static constexpr size_t St = 2 * size_t(kMtileBytes);          // state slice hi/lo (MN-major, K = 128)
+  // M tiles double-buffered, except at W = 128 (one buffer, reloaded after each step's products)
+  static constexpr int NM = W == 128 ? 1 : 2;
+  static constexpr size_t M0 = 0, M1 = NM == 2 ? kMtileBytes : 0;
+  static constexpr size_t St = NM * size_t(kMtileBytes);         // state slice hi/lo (MN-major, K = 128)
   static constexpr size_t StB = size_t(kTcD) * W * 2;            // one half (hi or lo) of it
   // forward: B columns [j0, j0 + W) (W / 32 consecutive 32-column slices); reverse: the Qeff tile
   static constexpr size_t XB = REVERSE ? size_t(2) * kTcC * kTcD * 2 : size_t(kTcD) * W * 4;
-  static constexpr int NX = (REVERSE && W == 64) ? 1 : 2;       // X buffers (one where two do not fit)
+  static constexpr int NX = ((REVERSE && W == 64) || W == 128) ? 1 : 2;  // X buffers (one where two do not fit)
   static constexpr size_t X = St + 2 * StB;
   // reverse: double-buffered dO slices, hi/lo operand tiles of C rows x W columns (k = row, n = column)
   static constexpr size_t dOB = REVERSE ? size_t(kTcC) * W * 2 : 0;
   static constexpr size_t dO = X + NX * XB;
   static constexpr size_t total = dO + 2 * 2 * dOB;
   static_assert(total <= 224 * 1024, "shared memory");
+  static_assert(W == 32 || W == 64 || W == 128, "slice width");
 };
 
 namespace tck {
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(128 * (W / 32), 1)
   uint8_t* dobuf[2] = {tsm + S::dO, tsm + S::dO + 2 * S::dOB};  // hi, then lo at + dOB
   uint8_t *sth = tsm + S::St, *stl = sth + S::StB;
   __shared__ __align__(8) uint64_t bar_m[2];
-  __shared__ __align__(8) uint64_t bar_x;  // the single X buffer (S::NX == 1)
+  __shared__ __align__(8) uint64_t bar_x;  // the single-buffered operands (S::NX == 1, S::NM == 1)
   __shared__ __align__(8) uint64_t bar_mma;
   __shared__ uint32_t tslot;
   __shared__ int s_ok;  // thread 0's bounded waits, read by every thread after the following barrier
@@ -161,9 +164,13 @@ __global__ void __launch_bounds__(128 * (W / 32), 1)
     const int ci = chunk_at(q);
     load_mtile(mbuf[q & 1], mtile(ci), S::NX == 2 ? xbuf[q & 1] : nullptr, xsrc(ci), (uint32_t)S::XB, &bar_m[q & 1]);
   };
-  auto load_x_single = [&](int q) {  // thread 0, S::NX == 1: once the previous chunk's products are done
-    tc::mbar_arrive_expect_tx(&bar_x, (uint32_t)S::XB);
-    tc::bulk_g2s(xbuf[0], xsrc(chunk_at(q)), (uint32_t)S::XB, &bar_x);
+  // thread 0: the single-buffered operands (X; and M at W = 128), once the previous chunk's products
+  // are done with them
+  auto load_x_single = [&](int q) {
+    const int ci = chunk_at(q);
+    tc::mbar_arrive_expect_tx(&bar_x, (uint32_t)S::XB + (S::NM == 1 ? kMtileBytes : 0u));
+    if constexpr (S::NM == 1) tc::bulk_g2s(mbuf[0], mtile(ci), kMtileBytes, &bar_x);
+    tc::bulk_g2s(xbuf[0], xsrc(ci), (uint32_t)S::XB, &bar_x);
   };
   // thread 0: the operands of a later chunk into L2 (the M tile once per (sequence, head), by the
   // first slice's CTA), so that the shared-memory copy a step ahead finds them there
@@ -194,7 +201,7 @@ __global__ void __launch_bounds__(128 * (W / 32), 1)
   }
   constexpr int kL2Ahead = 3;  // chunks prefetched into L2 ahead of the current one
   if (lead) {
-    prefetch(0);
+    if constexpr (S::NM == 2) prefetch(0);
     if constexpr (S::NX == 1) load_x_single(0);
     for (int q = 1; q < kL2Ahead; ++q) prefetch_l2(q);
   }
@@ -207,6 +214,7 @@ __global__ void __launch_bounds__(128 * (W / 32), 1)
     const int ci = chunk_at(q);
     const size_t base = (size_t)ci * H + h;
     uint8_t* xq = xbuf[S::NX == 2 ? (q & 1) : 0];
+    uint8_t* mq = mbuf[S::NM == 2 ? (q & 1) : 0];
     if (REVERSE) {
       const int slot = t.chunks[ci].export_slot;
       if (slot >= 0) {  // gradients of the exported boundary state, consumers in a fixed order
@@ -221,9 +229,9 @@ __global__ void __launch_bounds__(128 * (W / 32), 1)
     put_state(sth, stl, c, 32 * half, s);
     if constexpr (REVERSE && EX) tc::cp_async_wait<0>();  // this chunk's dO slice (issued a step ago)
     if (lead) {
-      if (q + 1 < nch) prefetch(q + 1);
+      if (S::NM == 2 && q + 1 < nch) prefetch(q + 1);
       prefetch_l2(q + kL2Ahead);
-      bool w = tc::mbar_wait(&bar_m[q & 1], (q >> 1) & 1);
+      bool w = S::NM == 1 || tc::mbar_wait(&bar_m[q & 1], (q >> 1) & 1);
       if constexpr (S::NX == 1) w = w && tc::mbar_wait(&bar_x, q & 1);
       if (!w) set_status(ws.status, kStatusTimeout);
       s_ok = w ? 1 : 0;
@@ -249,7 +257,7 @@ __global__ void __launch_bounds__(128 * (W / 32), 1)
       for (int j = 0; j < 32; ++j) add[j] = 0.f;
     }
     if (lead) {
-      const tc::Op mH{tc::smem_u32(mbuf[q & 1]), D, REVERSE}, mL{tc::smem_u32(mbuf[q & 1] + kMtileBytes / 2), D, REVERSE};
+      const tc::Op mH{tc::smem_u32(mq), D, REVERSE}, mL{tc::smem_u32(mq + kMtileBytes / 2), D, REVERSE};
       const tc::Op sH{tc::smem_u32(sth), D, true}, sL{tc::smem_u32(stl), D, true};
       mma4(tb, mH, mL, sH, sL, D, tc::idesc_bf16(D, W, REVERSE, true), false, false, false);
       if constexpr (REVERSE) {  // + Qeff^T dO (A: the Qeff tile read MN-major, k = chunk row)
@@ -295,7 +303,7 @@ __global__ void __launch_bounds__(128 * (W / 32), 1)
     }
   } else if (lead) {
     // give copies still in flight a last bounded chance before the shared memory is released
-    tc::mbar_wait(&bar_m[0], 0, 200000000ull);
+    if constexpr (S::NM == 2) tc::mbar_wait(&bar_m[0], 0, 200000000ull);
   }
   if constexpr (REVERSE && EX) tc::cp_async_wait<0>();
   if (lead) tc::bulk_wait_read();  // (the stores complete with the grid)

@@ -209,10 +209,40 @@ int stream_after(cudaStream_t to, cudaStream_t from) {
 // with more chunks than a grid's y extent allows is launched in pieces.
 constexpr int kMaxGridY = 65535;
 
-// State scans of a round: 64-column CTAs (half as many, each reading the M tile once for twice the
-// columns) when the round's (sequence, head) pairs would take more than one wave of 32-column CTAs
-// (one scan CTA per SM); 32-column CTAs otherwise (more CTAs for a short round's latency-bound chain)
-bool scan_wide(int n_seqs, int H) { return (long long)n_seqs * H * (tpc::kTcD / 32) > tpc_abi::sm_count(); }
+// Columns per state-scan CTA (one scan CTA per SM).  With several rounds the scans overlap the chunk
+// kernels of neighbouring rounds, so they take 128 columns (fewest CTAs: each reads the M tile once for
+// all columns, and the most SMs stay with the chunk kernels).  A plan of one round has nothing to
+// overlap: its scan takes the narrowest width whose CTAs fit one wave (more CTAs, a shorter chain
+// step), 128 if none does.  (Measured on the single-fork and agentic trees: 128 columns for every
+// round beat 32 / 64 by 2-4 % of the step.)
+int scan_width(int n_seqs, int H, int n_rounds) {
+  if (n_rounds > 1) return 128;
+  const long long pairs = (long long)n_seqs * H, sm = tpc_abi::sm_count();
+  for (int W = 32; W < 128; W *= 2)
+    if (pairs * (tpc::kTcD / W) <= sm) return W;
+  return 128;
+}
+
+// launches the state scan of a round with the chosen width
+template <bool REVERSE, typename Tin>
+int launch_scan(cudaStream_t hs, const tpc::Plan& p, int s0, int s1, int H, const float* init, float* final_state,
+                const float* d_final, const tpc::KdaWs& w, const Tin* dO) {
+  using namespace tpc;
+  const char* name = REVERSE ? "kda_bwd_scan_tc" : "kda_fwd_scan_tc";
+  auto go = [&](auto wc) -> int {
+    constexpr int W = decltype(wc)::value;
+    TPC_CUDA(set_smem(kda_scan_tc<REVERSE, W, Tin>, ScanTcSmemT<REVERSE, W>::total));
+    TPC_LAUNCH(name, hs,
+               (kda_scan_tc<REVERSE, W, Tin><<<dim3(s1 - s0, H, kTcD / W), 128 * (W / 32), ScanTcSmemT<REVERSE, W>::total,
+                                               hs>>>(p.dt, s0, H, init, final_state, d_final, w, dO)));
+    return TPC_OK;
+  };
+  switch (scan_width(s1 - s0, H, p.n_rounds)) {
+    case 128: return go(std::integral_constant<int, 128>{});
+    case 64: return go(std::integral_constant<int, 64>{});
+    default: return go(std::integral_constant<int, 32>{});
+  }
+}
 
 template <int C, int D, typename Tin, typename Tout, bool TC>
 int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_io* io, void* ws, cudaStream_t st) {
@@ -239,8 +269,6 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     // stream after prep(r) and scan(r - 1).  The caller's stream runs prep(1..R), out(1..R) in that
     // order, so the later rounds' prep overlaps scan(1) and out(r) overlaps scan(r + 1).
     TPC_CUDA(set_smem(kda_fwd_prep_tc<Tin>, PrepTcSmemT<Tin>::total));
-    TPC_CUDA(set_smem(kda_scan_tc<false, 32, Tin>, ScanTcSmemT<false, 32>::total));
-    TPC_CUDA(set_smem(kda_scan_tc<false, 64, Tin>, ScanTcSmemT<false, 64>::total));
     TPC_CUDA(set_smem(kda_fwd_out_tc<Tin, Tout>, OutTcSmem::total));
     cudaStream_t hs = scan_stream();
     if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
@@ -252,16 +280,9 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
                    (kda_fwd_prep_tc<Tin><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads, PrepTcSmemT<Tin>::total,
                                            st>>>(p.dt, H, k, v, g, b, w, a)));
       TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
-      if (s1 > s0) {
-        if (scan_wide(s1 - s0, H))
-          TPC_LAUNCH("kda_fwd_scan_tc", hs,
-                     (kda_scan_tc<false, 64, Tin><<<dim3(s1 - s0, H, D / 64), 256, ScanTcSmemT<false, 64>::total, hs>>>(
-                         p.dt, s0, H, io->init_state, io->final_state, nullptr, w, nullptr)));
-        else
-          TPC_LAUNCH("kda_fwd_scan_tc", hs,
-                     (kda_scan_tc<false, 32, Tin><<<dim3(s1 - s0, H, D / 32), 128, ScanTcSmemT<false, 32>::total, hs>>>(
-                         p.dt, s0, H, io->init_state, io->final_state, nullptr, w, nullptr)));
-      }
+      if (s1 > s0)
+        TPC_TRY_ABI((launch_scan<false, Tin>(hs, p, s0, s1, H, io->init_state, io->final_state, nullptr, w,
+                                             static_cast<const Tin*>(nullptr))));
       scans.emplace_back();
       TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
@@ -315,8 +336,6 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
     // Rounds in reverse: the reverse scan(r) (which also forms the output's contribution Qeff^T dO)
     // on the high-priority scan stream after the caller's prior work and scan(r + 1); then dq(r),
     // dk/dv(r) on the caller's stream after scan(r), so dq / dk-dv(r) overlap scan(r - 1).
-    TPC_CUDA(set_smem(kda_scan_tc<true, 32, Tin>, ScanTcSmemT<true, 32>::total));
-    TPC_CUDA(set_smem(kda_scan_tc<true, 64, Tin>, ScanTcSmemT<true, 64>::total));
     TPC_CUDA(set_smem(kda_bwd_dq_tc<Tin, Tout>, BdqTcSmem::total));
     TPC_CUDA(set_smem(kda_bwd_dkv_tc<Tin, Tout>, BdkvTcSmemT<Tin>::total));
     cudaStream_t hs = scan_stream();
@@ -324,16 +343,7 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
     TPC_TRY_ABI(stream_after(hs, st));  // the scans after the caller's prior work (forward, d_o)
     for (int r = p.n_rounds; r >= 1; --r) {
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
-      if (s1 > s0) {
-        if (scan_wide(s1 - s0, H))
-          TPC_LAUNCH("kda_bwd_scan_tc", hs,
-                     (kda_scan_tc<true, 64, Tin><<<dim3(s1 - s0, H, D / 64), 256, ScanTcSmemT<true, 64>::total, hs>>>(
-                         p.dt, s0, H, nullptr, nullptr, io->d_final, w, dO)));
-        else
-          TPC_LAUNCH("kda_bwd_scan_tc", hs,
-                     (kda_scan_tc<true, 32, Tin><<<dim3(s1 - s0, H, D / 32), 128, ScanTcSmemT<true, 32>::total, hs>>>(
-                         p.dt, s0, H, nullptr, nullptr, io->d_final, w, dO)));
-      }
+      if (s1 > s0) TPC_TRY_ABI((launch_scan<true, Tin>(hs, p, s0, s1, H, nullptr, nullptr, io->d_final, w, dO)));
       scans.emplace_back();
       TPC_CUDA(cudaEventCreateWithFlags(&scans.back(), cudaEventDisableTiming));
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
