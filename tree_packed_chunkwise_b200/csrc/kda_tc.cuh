@@ -312,23 +312,6 @@ __device__ __forceinline__ void tile8(const uint8_t* hi, const uint8_t* lo, int 
   }
 }
 
-// 16 values (a, b0 .. b0 + 15) of a K-major hi/lo tile in shared memory, as fp32 (hi + lo)
-template <int A>
-__device__ __forceinline__ void tile16(const uint8_t* hi, const uint8_t* lo, int a, int b0, float (&v)[16]) {
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const uint32_t off = cm_off(a, b0 + 8 * half, A);
-    const uint4 hq = *reinterpret_cast<const uint4*>(hi + off), lq = *reinterpret_cast<const uint4*>(lo + off);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
-    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lq);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 x = __bfloat1622float2(h2[k]), y = __bfloat1622float2(l2[k]);
-      v[8 * half + 2 * k] = x.x + y.x;
-      v[8 * half + 2 * k + 1] = x.y + y.y;
-    }
-  }
-}
 
 // Two A x B tiles (hi/lo) from the same staged bf16 rows: f(a, b, x) returns both values (float2)
 template <int A, int B, class F>
@@ -375,29 +358,6 @@ __device__ __forceinline__ void staged8(const T* st, int r, int c0, float (&v)[8
   }
 }
 
-// 16 consecutive values of a staged row as fp32
-template <typename T>
-__device__ __forceinline__ void staged16(const T* st, int r, int c0, float (&v)[16]) {
-  if constexpr (sizeof(T) == 4) {
-#pragma unroll
-    for (int j = 0; j < 16; j += 4) {
-      const float4 u = *reinterpret_cast<const float4*>(st + r * kStagePitch + c0 + j);
-      v[j] = u.x; v[j + 1] = u.y; v[j + 2] = u.z; v[j + 3] = u.w;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 16; j += 8) {
-      const uint4 u = *reinterpret_cast<const uint4*>(st + r * kStagePitch + c0 + j);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 f = __bfloat1622float2(b2[k]);
-        v[j + 2 * k] = f.x;
-        v[j + 2 * k + 1] = f.y;
-      }
-    }
-  }
-}
 
 __device__ __forceinline__ void ld8g(const float* p, float (&v)[8]) {
   const float4 u = *reinterpret_cast<const float4*>(p), u2 = *reinterpret_cast<const float4*>(p + 4);
@@ -416,29 +376,6 @@ __device__ __forceinline__ void st8_out(T* p, const float* v) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) b[j] = __float2bfloat16_rn(v[j]);
     *reinterpret_cast<uint4*>(p) = *reinterpret_cast<const uint4*>(b);
-  }
-}
-__device__ __forceinline__ void ld16g(const float* p, float (&v)[16]) {
-#pragma unroll
-  for (int j = 0; j < 16; j += 4) {
-    const float4 u = *reinterpret_cast<const float4*>(p + j);
-    v[j] = u.x; v[j + 1] = u.y; v[j + 2] = u.z; v[j + 3] = u.w;
-  }
-}
-__device__ __forceinline__ void st16g(float* p, const float* v) {
-#pragma unroll
-  for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(p + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-}
-template <typename T>
-__device__ __forceinline__ void st16_out(T* p, const float* v) {
-  if constexpr (sizeof(T) == 4) {
-    st16g(reinterpret_cast<float*>(p), v);
-  } else {
-    __align__(16) __nv_bfloat16 b[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) b[j] = __float2bfloat16_rn(v[j]);
-    reinterpret_cast<uint4*>(p)[0] = reinterpret_cast<const uint4*>(b)[0];
-    reinterpret_cast<uint4*>(p)[1] = reinterpret_cast<const uint4*>(b)[1];
   }
 }
 
@@ -623,24 +560,6 @@ __device__ __forceinline__ void store_cc_tile(float* tiles, size_t base, const u
   }
   tc::bulk_commit();
 }
-// element (i, c) of a C x D hi/lo tile in global memory, 16 consecutive c from c0, as fp32 (hi + lo)
-__device__ __forceinline__ void cd_tile16(const float* tiles, size_t base, int i, int c0, float (&v)[16]) {
-  const uint8_t* t = reinterpret_cast<const uint8_t*>(tiles) + base * kCDTileBytes;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const uint32_t off = cm_off(i, c0 + 8 * half, kTcC);
-    const uint4 h = __ldg(reinterpret_cast<const uint4*>(t + off));
-    const uint4 l = __ldg(reinterpret_cast<const uint4*>(t + kCDTileBytes / 2 + off));
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&h);
-    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&l);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 a = __bfloat1622float2(h2[k]), b = __bfloat1622float2(l2[k]);
-      v[8 * half + 2 * k] = a.x + b.x;
-      v[8 * half + 2 * k + 1] = a.y + b.y;
-    }
-  }
-}
 
 // bounded wait for the loads issued on l (CTA-wide vote); false on every thread after recording
 // TPC_ERR_TIMEOUT
@@ -789,10 +708,6 @@ __device__ __forceinline__ void cumsum_ref(float* G, int LD, int n, float* ref, 
   if (q == 0 && status && !(G[c] - G[(kTcC - 1) * LD + c] <= kMaxChunkDecay * kLog2e)) set_status(status, kStatusRange);
 }
 
-template <typename T>
-__device__ __forceinline__ float ld_in(const T* base, const int* rows, int H, int h, int n, int r, int c) {
-  return r < n ? to_f(base[((size_t)rows[r] * H + h) * kTcD + c]) : 0.f;
-}
 
 }  // namespace tck
 
@@ -806,8 +721,7 @@ struct PrepTcSmemT {
   static constexpr size_t A = G + sizeof(float) * C * LD;
   static constexpr size_t T = A + sizeof(float) * C * LC;
   static constexpr size_t W1 = T + sizeof(float) * C * LC;
-  static constexpr size_t W2 = W1 + sizeof(float) * 4 * 16 * 17;
-  static constexpr size_t vec = W2 + sizeof(float) * 4 * 16 * 17;       // beta[C], ref[D], gC[D]
+  static constexpr size_t vec = W1 + sizeof(float) * 4 * 16 * 17;       // beta[C], ref[D], gC[D]
   static constexpr size_t tiles = (vec + sizeof(float) * (C + 2 * D) + 1023) & ~size_t(1023);
   // phase 1: af hi/lo, bf hi/lo (C x D each); phase 2: T' hi/lo (C x C), Kbar hi/lo, V hi/lo (C x D)
   static constexpr size_t CDb = size_t(C) * D * 2, CCb = size_t(C) * C * 2;
@@ -1415,16 +1329,12 @@ struct BdkvTcSmemT {
   static constexpr size_t Rbytes = 128 * 1024;
   static constexpr size_t total = R + Rbytes;
   // offsets inside R by phase
-  static constexpr size_t p1_af = 0, p1_bf = 2 * CDb;                                 // K-major af, bf
-  static constexpr size_t inv_L = 0, inv_T = inv_L + sizeof(float) * C * LC;           // fp32 L, T
-  static constexpr size_t inv_W1 = inv_T + sizeof(float) * C * LC, inv_W2 = inv_W1 + sizeof(float) * 4 * 16 * 17;
   static constexpr size_t p2_Tp = 44 * 1024, p2_Kb = p2_Tp + 2 * CCb, p2_V = p2_Kb + 2 * CDb;  // T', Kbar, V
   static constexpr size_t p2_S0 = 0;                                                   // S0 (K); dU in dX
   static constexpr size_t p3_X = 0, p3_dX = 4 * CDb;                                   // X (K, C x 2D), dX (MN)
   static constexpr size_t p4_dB = 4 * CDb;                                             // dB (K, C x 2D)
   static constexpr size_t p5_dA = 0, p5_bf = 2 * CCb, p5_af = p5_bf + 2 * CDb;         // dAt, bf (MN), af (MN)
   static_assert(p2_V + 2 * CDb <= Rbytes && p2_S0 + 2 * DDb <= p3_dX && p3_dX + 4 * CDb <= Rbytes, "R");
-  static_assert(inv_W2 + sizeof(float) * 4 * 16 * 17 <= p2_Tp, "inverse scratch overlaps T'");
   static_assert(total <= 227 * 1024, "shared memory");
 };
 
