@@ -570,6 +570,41 @@ long long tpc_launch_count(void);
  */
 int tpc_debug_wait_timeout(int32_t* status, int64_t timeout_ns, tpc_stream_t stream);
 
+/* ------------------------------------------------------------------ index and bounds mode */
+/*
+ * Every kernel of this library indexes rows, chunks, boundary-state slots and replayed rows through
+ * the plan's uploaded tables (HARTS Figure 2(c): the rounds' packed calls, the exported and imported
+ * boundary states, the replay from the last aligned boundary).  With the mode on, each call that
+ * reads those tables (KDA forward / backward / export, attention, the layer group, log-prob
+ * recovery, MoE routing, the row maps) first bounds every index field of every table on the device
+ * with one kernel and waits for it: a bad entry makes the call return TPC_ERR_DEVICE_CHECK (the
+ * message names the table, the record and the bound) before any compute kernel is launched.  The
+ * check reads only inside the tables.  The mode costs one launch and one host synchronisation per
+ * call.  Off by default; the environment variable TPC_CHECKS=1 turns it on at the first call.
+ */
+void tpc_checks_enable(int on);
+int tpc_checks_enabled(void);
+/* Runs the table check once, whatever the mode: TPC_OK, TPC_ERR_DEVICE_CHECK or TPC_ERR_STATE
+ * (tables not uploaded).  Synchronises `stream`. */
+int tpc_plan_check_device(const tpc_plan* plan, tpc_stream_t stream);
+/* The same checks on the host copy of the tables (no GPU, no upload needed), with word `word` of
+ * table `table` (numbering of tpc_debug_poke_table) replaced by `value` when table >= 0: TPC_OK or
+ * TPC_ERR_DEVICE_CHECK (same message as the device check); TPC_ERR_BAD_SHAPE for a word outside
+ * the table. */
+int tpc_plan_check_host(const tpc_plan* plan, int32_t table, int64_t word, int32_t value);
+/*
+ * Test hook: overwrites int32 word `word` of uploaded table `table` (blob order: 0 sequences
+ * (8 words per record), 1 chunks (8), 2 slots (4), 3 slot consumers, 4 root-consumer offsets,
+ * 5 root consumers, 6 replayed rows, 7 replay-target rows, 8 target offsets, 9 target parts,
+ * 10 row-to-target map, 11 expanded rows, 12 occurrence offsets, 13 occurrence list,
+ * 14 occurrence counts, 15 attention nodes (8), 16 attention ranges (2), 17 query tiles (4),
+ * 18 key tiles (4)) with `value`, returning the previous value in *old_value (may be NULL).
+ * `table` and `word` are checked against the plan on the host (TPC_ERR_BAD_SHAPE).  Synchronises
+ * `stream`.  A plan whose tables were changed this way is only safe to use with the mode on.
+ */
+int tpc_debug_poke_table(tpc_plan* plan, int32_t table, int64_t word, int32_t value, int32_t* old_value,
+                         tpc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

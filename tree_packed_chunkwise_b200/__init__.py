@@ -152,6 +152,12 @@ SIGNATURES = {
     "tpc_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_size_t]),
     "tpc_launch_count": (ctypes.c_longlong, []),
     "tpc_debug_wait_timeout": (ctypes.c_int, [_V, ctypes.c_int64, _V]),
+    "tpc_checks_enable": (None, [ctypes.c_int]),
+    "tpc_checks_enabled": (ctypes.c_int, []),
+    "tpc_plan_check_device": (ctypes.c_int, [_V, _V]),
+    "tpc_plan_check_host": (ctypes.c_int, [_V, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32]),
+    "tpc_debug_poke_table": (ctypes.c_int, [_V, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                            _P(ctypes.c_int32), _V]),
 }
 
 _lib = None
@@ -257,6 +263,22 @@ class Plan:
         _check(lib().tpc_plan_upload(self._h, _ptr(buf), nbytes, _stream_ptr(stream)))
         self.dev_tables = buf
         return self
+
+    def check_device(self, stream=None):
+        """Bounds every index field of the uploaded tables on the device (tpc_plan_check_device); raises
+        TpcError(TPC_ERR_DEVICE_CHECK) naming the first bad entry."""
+        _check(lib().tpc_plan_check_device(self._h, _stream_ptr(stream)))
+
+    def check_host(self, table: int = -1, word: int = 0, value: int = 0):
+        """The device-table checks on the host copy of the tables, with one word replaced when table >= 0."""
+        _check(lib().tpc_plan_check_host(self._h, int(table), int(word), int(value)))
+
+    def poke_table(self, table: int, word: int, value: int, stream=None) -> int:
+        """Test hook: overwrites one int32 word of an uploaded table; returns the previous value."""
+        old = ctypes.c_int32(0)
+        _check(lib().tpc_debug_poke_table(self._h, int(table), int(word), int(value), ctypes.byref(old),
+                                          _stream_ptr(stream)))
+        return int(old.value)
 
     def compact_source_rows(self, node_start: np.ndarray, length: np.ndarray) -> np.ndarray:
         """For every compact row, the node-order row (rows of node 0, node 1, ...) it holds."""
@@ -515,6 +537,15 @@ def tpc_profile_read() -> dict:
 
 def tpc_launch_count() -> int:
     return int(lib().tpc_launch_count())
+
+
+def tpc_checks_enable(on: bool) -> None:
+    """Index and bounds mode: every call that reads plan tables checks them on the device first."""
+    lib().tpc_checks_enable(1 if on else 0)
+
+
+def tpc_checks_enabled() -> bool:
+    return bool(lib().tpc_checks_enabled())
 
 
 def tpc_debug_wait_timeout(status, timeout_ns=1_000_000, stream=None):

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtpc.so")
-SOURCES = ["planner.cpp", "microbatch.cpp", "tpc_abi.cu", "abi_dense.cu", "abi_attn.cu", "abi_moe.cu", "group.cu"]
+SOURCES = ["planner.cpp", "microbatch.cpp", "tpc_abi.cu", "abi_dense.cu", "abi_attn.cu", "abi_moe.cu", "abi_checks.cu", "group.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-shared"]

@@ -39,6 +39,8 @@ int tpc_tree_attn_forward(const tpc_plan* plan, const tpc_attn_shape* s, const v
   const tpc_attn_lo L = lo ? *lo : tpc_attn_lo{};
   const bool split = L.q || L.k || L.v;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_tree_attn_forward");
   const tpc::Plan& p = plan->p;
   const dim3 grid((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest
   using bf = __nv_bfloat16;
@@ -73,6 +75,8 @@ int tpc_tree_attn_backward(const tpc_plan* plan, const tpc_attn_shape* s, const 
   const tpc_attn_lo L = lo ? *lo : tpc_attn_lo{};
   const bool split = L.q || L.k || L.v || L.d_o;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_tree_attn_backward");
   const tpc::Plan& p = plan->p;
   using bf = __nv_bfloat16;
   const dim3 gq((unsigned)(p.attn_qtiles.size() * (size_t)s->H));  // (query tile, head), query tiles fastest

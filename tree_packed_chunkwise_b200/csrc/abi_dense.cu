@@ -130,6 +130,8 @@ int tpc_logprob_forward(const tpc_plan* plan, const void* h, const void* W, int6
   if (int rc = logprob_check(plan, h, W, V, Dh, targets, scratch, scratch_bytes, chunk_rows)) return rc;
   if (!logp || !lse) return fail(TPC_ERR_NULL, "logprob: logp and lse are required");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_logprob_forward");
   const tpc::Plan& p = plan->p;
   const int tiles = (int)((V + tpc::kGemmBN - 1) / tpc::kGemmBN);
   float2* part = static_cast<float2*>(scratch);
@@ -158,6 +160,8 @@ int tpc_logprob_backward(const tpc_plan* plan, const void* h, const void* W, int
   if (int rc = logprob_check(plan, h, W, V, Dh, targets, scratch, scratch_bytes, chunk_rows)) return rc;
   if (!dlogp || !lse || !dh || !dW) return fail(TPC_ERR_NULL, "logprob backward: dlogp, lse, dh and dW are required");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_logprob_backward");
   const tpc::Plan& p = plan->p;
   const int64_t N = p.n_unique, NE = p.n_expanded;
   char* sc = static_cast<char*>(scratch);

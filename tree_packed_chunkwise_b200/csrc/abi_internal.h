@@ -2,7 +2,9 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
+#include <cstdio>
 #include <string>
 #include <vector>
 
@@ -24,6 +26,26 @@ template <class KernelT>
 cudaError_t set_smem(KernelT k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
+
+// Index and bounds mode (TPC_CHECKS=1 or tpc_checks_enable): every index field of the plan's
+// device tables is bounded on the device before a call that reads them launches anything; returns
+// TPC_OK when the mode is off or the tables pass, else TPC_ERR_DEVICE_CHECK (nothing launched).
+bool checks_on();
+int plan_checks(const tpc_plan* plan, cudaStream_t st);
+
+// NVTX range over a scope (calls and rounds show up on an Nsight Systems timeline; a few
+// nanoseconds when no tool is attached)
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  NvtxRange(const char* name, int round) {
+    char buf[48];
+    snprintf(buf, sizeof(buf), "%s round %d", name, round);
+    nvtxRangePushA(buf);
+  }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // multiprocessors of the current device (persistent grids)
 int sm_count();

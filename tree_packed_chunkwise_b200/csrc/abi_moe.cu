@@ -42,6 +42,8 @@ int tpc_moe_route(const tpc_plan* plan, const void* h, const void* w_router, int
   auto* part_load = reinterpret_cast<long long*>(sc);
   auto* part_prob = reinterpret_cast<float*>(sc + a256((size_t)parts * E * 8));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_moe_route");
   // rows per thread of the logits tiling: 32 rows x QP expert quads over the CTA's threads
   const int rt = std::max(1, tpc::kMoeRows * tpc::moe_quads_p2(E) / tpc::kMoeThreads);
   auto go = [&](auto rpt) -> int {
@@ -79,6 +81,8 @@ int tpc_moe_router_loss(const tpc_plan* plan, const float* logits, const float* 
   auto* part_z = reinterpret_cast<float*>(sc + a256((size_t)parts * E * 8) + a256((size_t)parts * E * 4));
   const int rows_per = tpc::kMoeThreads / 32, nblk = (N + rows_per - 1) / rows_per;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_moe_router_loss");
   TPC_LAUNCH("moe_loss_grad", st, (tpc::moe_loss_grad_kernel<<<nblk, tpc::kMoeThreads, 0, st>>>(
                                       plan->p.dt, logits, lse, (const long long*)expert_load, E, N, a * alpha,
                                       (float)(b / n_exp), dlogits, part_z)));

@@ -273,6 +273,8 @@ int tpc_group_forward(const tpc_plan* plan, const tpc_group_shape* s, const tpc_
   TPC_TRY(check_group(plan, s, w, ws, ws_bytes, &b));
   if (!x || !y || (s->n_kda > 0 && !h)) return fail(TPC_ERR_NULL, "x, y or h is NULL");
   cudaStream_t st = stream;
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_group_forward");
   const size_t ND = (size_t)plan->p.n_unique * kGrpD;
   TPC_CUDA(cudaMemsetAsync(b.status, 0, 4, st));
   TPC_TRY(tpc_rope_positions(plan, b.pos, st));
@@ -296,6 +298,8 @@ int tpc_group_backward(const tpc_plan* plan, const tpc_group_shape* s, const tpc
     if (!g->kda[l].w_in || !g->kda[l].w_o) return fail(TPC_ERR_NULL, "KDA weight gradient is NULL");
   if (!g->mla.w_a || !g->mla.w_b || !g->mla.w_o) return fail(TPC_ERR_NULL, "MLA weight gradient is NULL");
   cudaStream_t st = stream;
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_group_backward");
   const size_t ND = (size_t)plan->p.n_unique * kGrpD;
   TPC_CUDA(cudaMemsetAsync(b.status, 0, 4, st));
   TPC_TRY(tpc_rope_positions(plan, b.pos, st));

@@ -273,6 +273,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
     cudaStream_t hs = scan_stream();
     if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
     for (int r = 1; r <= p.n_rounds; ++r) {
+      tpc_abi::NvtxRange nvtx_round("kda forward prep + scan", r);
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       for (int a = c0; a < c1; a += kMaxGridY)
@@ -288,6 +289,7 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
     }
     for (int r = 1; r <= p.n_rounds; ++r) {
+      tpc_abi::NvtxRange nvtx_round("kda forward out", r);
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       TPC_CUDA(cudaStreamWaitEvent(st, scans[r - 1], 0));
       TPC_CUDA(cudaEventDestroy(scans[r - 1]));
@@ -342,6 +344,7 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
     if (!hs) return fail(TPC_ERR_CUDA, "could not create the library's scan stream");
     TPC_TRY_ABI(stream_after(hs, st));  // the scans after the caller's prior work (forward, d_o)
     for (int r = p.n_rounds; r >= 1; --r) {
+      tpc_abi::NvtxRange nvtx_round("kda backward scan", r);
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
       if (s1 > s0) TPC_TRY_ABI((launch_scan<true, Tin>(hs, p, s0, s1, H, nullptr, nullptr, io->d_final, w, dO)));
       scans.emplace_back();
@@ -349,6 +352,7 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
       TPC_CUDA(cudaEventRecord(scans.back(), hs));
     }
     for (int r = p.n_rounds, i = 0; r >= 1; --r, ++i) {
+      tpc_abi::NvtxRange nvtx_round("kda backward dq + dkv", r);
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       TPC_CUDA(cudaStreamWaitEvent(st, scans[i], 0));
       TPC_CUDA(cudaEventDestroy(scans[i]));
@@ -649,6 +653,8 @@ int tpc_kda_forward(const tpc_plan* plan, const tpc_kda_shape* s, const tpc_kda_
   if (ws_bytes < tpc_kda_workspace_bytes(plan, s)) return fail(TPC_ERR_WORKSPACE, "workspace too small");
   if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(TPC_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_kda_forward");
   return dispatch(plan, s, [&](auto CC, auto DD, auto tin, auto tout, auto tc) {
     return forward_impl<decltype(CC)::value, decltype(DD)::value, decltype(tin), decltype(tout), decltype(tc)::value>(
         plan->p, s, io, ws, st);
@@ -663,6 +669,8 @@ int tpc_kda_backward_window(const tpc_plan* plan, const tpc_kda_shape* s, const 
     return fail(TPC_ERR_NULL, "backward: inputs, d_o, gradient outputs and ws are required");
   if (ws_bytes < tpc_kda_workspace_bytes(plan, s)) return fail(TPC_ERR_WORKSPACE, "workspace too small");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_kda_backward_window");
   // the external consumers' start-state gradients enter the reverse scans like in-tree consumers'
   const tpc::Plan& pl = plan->p;
   if (!pl.ext_slot.empty()) {
@@ -693,6 +701,7 @@ int tpc_kda_export_states(const tpc_plan* plan, const tpc_kda_shape* s, const vo
   const WsLayout L = ws_layout(pl, s->H, pl.C, s->dk);
   const size_t per = (size_t)s->H * s->dk * s->dv * 4;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
   for (size_t e = 0; e < pl.ext_slot.size(); ++e)
     TPC_CUDA(cudaMemcpyAsync(reinterpret_cast<char*>(states) + e * per,
                              static_cast<const char*>(ws) + L.slot + (size_t)pl.ext_slot[e] * per, per,
@@ -743,6 +752,7 @@ int tpc_reduce_expanded_to_unique(const tpc_plan* plan, const float* x_exp, floa
   if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
   if (width < 1) return fail(TPC_ERR_BAD_SHAPE, "width must be >= 1");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
   const int64_t N = plan->p.n_unique;
   TPC_LAUNCH("reduce_expanded", st,
              (tpc::reduce_expanded_kernel<<<(unsigned)N, 128, 0, st>>>(plan->p.dt, x_exp, x_unique, width)));
@@ -755,6 +765,7 @@ int tpc_gather_expanded(const tpc_plan* plan, const void* x_unique, void* x_exp,
   if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
   if (width < 1 || (elem_bytes != 2 && elem_bytes != 4)) return fail(TPC_ERR_BAD_SHAPE, "width >= 1, elem_bytes 2 or 4");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
   const int64_t M = plan->p.n_expanded;
   if (elem_bytes == 2)
     TPC_LAUNCH("gather_expanded", st,
@@ -771,6 +782,7 @@ int tpc_occurrence_counts(const tpc_plan* plan, int32_t* counts, tpc_stream_t st
   if (!plan || !counts) return fail(TPC_ERR_NULL, "plan or counts NULL");
   if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
   const int64_t N = plan->p.n_unique;
   TPC_LAUNCH("occurrence_count", st,
              (tpc::occurrence_count_kernel<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(plan->p.dt, counts, N)));
@@ -781,6 +793,7 @@ int tpc_rope_positions(const tpc_plan* plan, int32_t* pos, tpc_stream_t stream) 
   if (!plan || !pos) return fail(TPC_ERR_NULL, "plan or pos is NULL");
   if (!plan->p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
   TPC_LAUNCH("rope_positions", st, (tpc::rope_positions_kernel<<<plan->p.n, 128, 0, st>>>(plan->p.dt, pos)));
   return TPC_OK;
 }
@@ -829,6 +842,8 @@ int tpc_kda_forward_static(const tpc_plan* plan, const tpc_kda_shape* s, const t
   char* base = nullptr;
   if (int rc = static_base(&base)) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
+  tpc_abi::NvtxRange nvtx_call("tpc_kda_forward_static");
   // plan tables after the status word (pageable source: staged before cudaMemcpyAsync returns)
   std::vector<uint8_t> blob;
   tpc::pack_device_blob(p, off, blob);
