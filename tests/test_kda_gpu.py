@@ -208,3 +208,41 @@ def test_bounded_device_wait_reports_timeout(tpc):
     status.zero_()
     assert torch.ones(4, device="cuda").sum().item() == 4.0
 
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_outputs_written_exactly_inside_nan_canaries(tpc, out):
+    """Every output of the forward and backward is a view into a NaN-filled buffer with 4096 NaN
+    elements on both sides: afterwards the padding is still all NaN (no write outside an output) and
+    the outputs hold no NaN (every element written).  Tensor-core path, replay rows, initial states."""
+    import torch
+    w = synth.workload("agentic_small")
+    t = w.tree
+    case = Case(t, 2, 128, 64, "bf16", w.seed + 31, with_init=True)
+    plan = tpc.Plan(t.parent, t.length, 64).upload()
+    x = to_torch_compact(case, plan)
+    N, H, d = x["q"].shape
+    pad = 4096
+    odt = torch.float32 if out == "f32" else torch.bfloat16
+    bufs = []
+
+    def canary(shape, dtype):
+        n = int(np.prod(shape))
+        buf = torch.full((pad + n + pad,), float("nan"), dtype=dtype, device="cuda")
+        bufs.append((buf, n))
+        return buf[pad:pad + n].view(shape)
+
+    o = canary((N, H, d), odt)
+    fin = canary((plan.info["n_leaves"], H, d, d), torch.float32)
+    _, _, ws = tpc.tpc_kda_forward(plan, x["q"], x["k"], x["v"], x["g"], x["beta"], x["init"], out_dtype=odt,
+                                   o=o, final_state=fin)
+    grads = dict(dq=canary((N, H, d), odt), dk=canary((N, H, d), odt), dv=canary((N, H, d), odt),
+                 dg=canary((N, H, d), torch.float32), dbeta=canary((N, H), torch.float32),
+                 d_init=canary((plan.info["n_roots"], H, d, d), torch.float32))
+    tpc.tpc_kda_backward(plan, ws, x["q"], x["k"], x["v"], x["g"], x["beta"], x["d_o"], x["d_final"], x["init"],
+                         out_dtype=odt, grads=grads)
+    torch.cuda.synchronize()
+    tpc.tpc_status(plan, ws, H, d)
+    for i, (buf, n) in enumerate(bufs):
+        assert torch.isnan(buf[:pad]).all() and torch.isnan(buf[pad + n:]).all(), f"write outside output {i}"
+        assert not torch.isnan(buf[pad:pad + n]).any(), f"output {i} not fully written"
