@@ -200,9 +200,9 @@ int report(const std::vector<Named>& all, unsigned long long first) {
                                         std::to_string(rec) + "]: " + all[id].what);
 }
 
-int run_checks(const tpc::Plan& p, cudaStream_t st) {
-  if (!p.dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
-  const std::vector<Named> all = plan_checks_list(p, p.blob_offsets);
+int run_checks(const tpc::Plan& p, const void* dev, const std::vector<size_t>& off, cudaStream_t st) {
+  if (!dev) return fail(TPC_ERR_STATE, "plan tables not uploaded");
+  const std::vector<Named> all = plan_checks_list(p, off);
   if (int rc = bound_reads(p, all)) return rc;
   CheckList list{};
   list.n = (int)all.size();
@@ -216,7 +216,7 @@ int run_checks(const tpc::Plan& p, cudaStream_t st) {
   TPC_CUDA(cudaMemcpyToSymbolAsync(g_check_first, &none, sizeof(none), 0, cudaMemcpyHostToDevice, st));
   const unsigned gx = (unsigned)std::min<int64_t>((most + 255) / 256, 4 * (int64_t)tpc_abi::sm_count());
   TPC_LAUNCH("table_check", st, table_check_kernel<<<dim3(gx, list.n), 256, 0, st>>>(
-                                    static_cast<const int32_t*>(p.dev), list));
+                                    static_cast<const int32_t*>(dev), list));
   unsigned long long first = none;
   TPC_CUDA(cudaMemcpyFromSymbolAsync(&first, g_check_first, sizeof(first), 0, cudaMemcpyDeviceToHost, st));
   TPC_CUDA(cudaStreamSynchronize(st));
@@ -272,7 +272,11 @@ bool checks_on() {
 
 int plan_checks(const tpc_plan* plan, cudaStream_t st) {
   if (!checks_on()) return TPC_OK;
-  return run_checks(plan->p, st);
+  return run_checks(plan->p, plan->p.dev, plan->p.blob_offsets, st);
+}
+
+int table_checks_at(const tpc::Plan& p, const void* dev, const std::vector<size_t>& off, cudaStream_t st) {
+  return run_checks(p, dev, off, st);
 }
 }  // namespace tpc_abi
 
@@ -284,7 +288,7 @@ int tpc_checks_enabled(void) { return tpc_abi::checks_on() ? 1 : 0; }
 
 int tpc_plan_check_device(const tpc_plan* plan, tpc_stream_t stream) {
   if (!plan) return fail(TPC_ERR_NULL, "plan is NULL");
-  return run_checks(plan->p, reinterpret_cast<cudaStream_t>(stream));
+  return run_checks(plan->p, plan->p.dev, plan->p.blob_offsets, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int tpc_plan_check_host(const tpc_plan* plan, int32_t table, int64_t word, int32_t value) {

@@ -32,6 +32,8 @@ cudaError_t set_smem(KernelT k, size_t bytes) {
 // TPC_OK when the mode is off or the tables pass, else TPC_ERR_DEVICE_CHECK (nothing launched).
 bool checks_on();
 int plan_checks(const tpc_plan* plan, cudaStream_t st);
+// the same check of a copy of the plan's tables at `dev` (layout offsets `off`), whatever the mode
+int table_checks_at(const tpc::Plan& p, const void* dev, const std::vector<size_t>& off, cudaStream_t st);
 
 // NVTX range over a scope (calls and rounds show up on an Nsight Systems timeline; a few
 // nanoseconds when no tool is attached)

@@ -929,11 +929,13 @@ struct OutTcSmem {
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kTcThreads, 1)
     kda_fwd_out_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
-                   const Tin* __restrict__ g_, Tout* __restrict__ o_, KdaWs ws, int chunk0 = 0) {
+                   const Tin* __restrict__ g_, Tout* __restrict__ o_, KdaWs ws, int chunk0 = 0, int hpc = 1) {
   using namespace tck;
   using S = OutTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD;
-  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
+  // grid (heads / hpc, chunks): a CTA runs hpc heads of one chunk in turn, the next head's gates, q
+  // and k loaded into registers while the current head's products and epilogues run
+  const int ci = chunk0 + (int)blockIdx.y, h0 = (int)blockIdx.x * hpc;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -943,7 +945,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
-  const size_t base = (size_t)ci * H + h;
   uint8_t *s0h = tsm + S::S0, *s0l = s0h + S::DDb;
   for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
   if ((tid >> 5) == 0) tc::tmem_alloc(&tslot, 512);
@@ -954,95 +955,109 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+  int hl = h0;  // the head whose inputs are being loaded
+  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + hl) * D : nullptr; };
+  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + hl) * D : nullptr; };
   GateRegs<Tin> gr;
-  gate_ld(gr, g_, srow, H, h, n);  // gates, q and k first, then the workspace tiles
+  gate_ld(gr, g_, srow, H, hl, n);  // gates, q and k first, then the workspace tiles
   RawTile<Tin, C, D> rq, rk;
   raw_ld(rq, row_q);
   raw_ld(rk, row_k);
-  if (tid == 0) {
-    ld_expect(ld, kStateTileBytes + kCDTileBytes);
-    ld_state_tile(ld, s0h, s0l, ws.S0, base);  // the chunk-start state, as the scan left it
-    ld_cd_tile(ld, tsm + S::Wq, tsm + S::Wq + S::CDb, ws.W, base);  // W, as the prep kernel left it
-  }
-  gate_st(sG, LD, gr);
-  __syncthreads();
-  uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb;
-  cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(qbh));  // (the Qbar tile comes later)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
-  // TMEM: P [0,64), W S0 [64,192), O [192,320), P W [320,448)
-  uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
-  uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb;
-  // qf = q e^{G - ref} and Qbar = q e^G from one load of q; bf = k e^{ref - G}
-  build_tile2_raw<C, D, Tin>(
-      qfh, qfl, qbh, qbl, rq, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); },
-      [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c]); });
-  build_tile_raw<C, D, Tin>(bfh, bfl, rk, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
-  const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
-  bool ok = ld_wait(ld);
-  ok = ok && run(sy, [&] {
-    const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
-    const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
-    const tc::Op wH{tc::smem_u32(wh), C, false}, wL{tc::smem_u32(wl), C, false};
-    mma4(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false, false);
-    mma4(tb + 64, wH, wL, sH, sL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
-  });
-  uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
-  if (ok) {
-    if (tid == 0) {  // U' (as the prep kernel left it) into the consumed qf / bf space
-      ld_expect(ld, kCDTileBytes);
-      ld_cd_tile(ld, uh, ul, ws.U, base);
+  bool ok = true;
+  for (int hi = 0; hi < hpc && ok; ++hi) {
+    const int h = h0 + hi;
+    const size_t base = (size_t)ci * H + h;
+    if (tid == 0) {
+      ld_expect(ld, kStateTileBytes + kCDTileBytes);
+      ld_state_tile(ld, s0h, s0l, ws.S0, base);  // the chunk-start state, as the scan left it
+      ld_cd_tile(ld, tsm + S::Wq, tsm + S::Wq + S::CDb, ws.W, base);  // W, as the prep kernel left it
     }
-    acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
-      float m[8];
-      for (int j = 0; j < 8; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
-      put8<C, true>(ph, pl, r, i0, m);  // kept (as this tile) for the backward
-    });
+    gate_st(sG, LD, gr);
+    __syncthreads();
+    uint8_t *qbh = tsm + S::Qb, *qbl = qbh + S::CDb;
+    cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(qbh));  // (the Qbar tile comes later)
+    // TMEM: P [0,64), W S0 [64,192), O [192,320), P W [320,448)
+    uint8_t *qfh = tsm + S::R, *qfl = qfh + S::CDb, *bfh = qfl + S::CDb, *bfl = bfh + S::CDb;
+    uint8_t *wh = tsm + S::Wq, *wl = wh + S::CDb;
+    // qf = q e^{G - ref} and Qbar = q e^G from one load of q; bf = k e^{ref - G}
+    build_tile2_raw<C, D, Tin>(
+        qfh, qfl, qbh, qbl, rq, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); },
+        [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c]); });
+    build_tile_raw<C, D, Tin>(bfh, bfl, rk, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
+    if (hi + 1 < hpc) {  // the next head's inputs, into the registers just consumed
+      hl = h + 1;
+      gate_ld(gr, g_, srow, H, hl, n);
+      raw_ld(rq, row_q);
+      raw_ld(rk, row_k);
+    }
+    const tc::Op sH{tc::smem_u32(s0h), D, true}, sL{tc::smem_u32(s0l), D, true};
     ok = ld_wait(ld);
-  }
-  if (ok) {
-    acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
-      float u[8];
-      tile8<C>(uh, ul, i, j0, u);  // U'
-      for (int j = 0; j < 8; ++j) u[j] -= v[j];
-      put8<C, true>(uh, ul, i, j0, u);  // U, element (i, j): MN-major (k = i); kept for the backward
+    ok = ok && run(sy, [&] {
+      const tc::Op ah{tc::smem_u32(qfh), C, false}, al{tc::smem_u32(qfl), C, false};
+      const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
+      const tc::Op wH{tc::smem_u32(wh), C, false}, wL{tc::smem_u32(wl), C, false};
+      mma4(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false, false);
+      mma4(tb + 64, wH, wL, sH, sL, D, tc::idesc_bf16(C, D, false, true), false, false, false);
     });
-    ok = run(sy, [&] {
-      store_cc_tile(ws.Pm, base, ph, pl);
-      store_cd_tile(ws.U, base, uh, ul);  // U replaces U'
-
-      const uint32_t id = tc::idesc_bf16(C, D, false, true);
-      const tc::Op qH{tc::smem_u32(qbh), C, false}, qL{tc::smem_u32(qbl), C, false};
-      const tc::Op pH{tc::smem_u32(ph), C, false}, pL{tc::smem_u32(pl), C, false};
-      const tc::Op uH{tc::smem_u32(uh), C, true}, uL{tc::smem_u32(ul), C, true};
-      const tc::Op wH{tc::smem_u32(wh), C, true}, wL{tc::smem_u32(wl), C, true};  // W as B (k = i, n = c)
-      mma4(tb + 192, qH, qL, sH, sL, D, id, false, false, false);
-      mma4(tb + 192, pH, pL, uH, uL, C, id, true, false, false);
-      mma4(tb + 320, pH, pL, wH, wL, C, id, false, false, false);
-    });
+    uint8_t *ph = tsm + S::R, *pl = ph + S::CCb, *uh = pl + S::CCb, *ul = uh + S::CDb;
     if (ok) {
-      acc_read<C, D>(tb, 192, [&](int r, int j0, const float* v) {
-        if (r >= ch.n_replay && r < n) st8_out(o_ + ((size_t)srow[r] * H + h) * D + j0, v);
+      if (tid == 0) {  // U' (as the prep kernel left it) into the consumed qf / bf space
+        ld_expect(ld, kCDTileBytes);
+        ld_cd_tile(ld, uh, ul, ws.U, base);
+      }
+      acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
+        float m[8];
+        for (int j = 0; j < 8; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+        put8<C, true>(ph, pl, r, i0, m);  // kept (as this tile) for the backward
       });
-      // Qeff = Qbar - P W (element (r, c)) into the S0 buffer, which the products above consumed
-      uint8_t *eh = s0h, *el = s0h + S::CDb;
-      acc_read<C, D>(tb, 320, [&](int r, int c0, const float* v) {
-        float e[8];
-        tile8<C>(qbh, qbl, r, c0, e);  // Qbar
-        for (int j = 0; j < 8; ++j) e[j] -= v[j];
-        put8<C, true>(eh, el, r, c0, e);
-      });
-      tc::fence_async_smem();
-      __syncthreads();
-      if (tid == 0) store_cd_tile(ws.W, base, eh, el);
+      ok = ld_wait(ld);
     }
+    if (ok) {
+      acc_read<C, D>(tb, 64, [&](int i, int j0, const float* v) {
+        float u[8];
+        tile8<C>(uh, ul, i, j0, u);  // U'
+        for (int j = 0; j < 8; ++j) u[j] -= v[j];
+        put8<C, true>(uh, ul, i, j0, u);  // U, element (i, j): MN-major (k = i); kept for the backward
+      });
+      ok = run(sy, [&] {
+        store_cc_tile(ws.Pm, base, ph, pl);
+        store_cd_tile(ws.U, base, uh, ul);  // U replaces U'
+
+        const uint32_t id = tc::idesc_bf16(C, D, false, true);
+        const tc::Op qH{tc::smem_u32(qbh), C, false}, qL{tc::smem_u32(qbl), C, false};
+        const tc::Op pH{tc::smem_u32(ph), C, false}, pL{tc::smem_u32(pl), C, false};
+        const tc::Op uH{tc::smem_u32(uh), C, true}, uL{tc::smem_u32(ul), C, true};
+        const tc::Op wH{tc::smem_u32(wh), C, true}, wL{tc::smem_u32(wl), C, true};  // W as B (k = i, n = c)
+        mma4(tb + 192, qH, qL, sH, sL, D, id, false, false, false);
+        mma4(tb + 192, pH, pL, uH, uL, C, id, true, false, false);
+        mma4(tb + 320, pH, pL, wH, wL, C, id, false, false, false);
+      });
+      if (ok) {
+        acc_read<C, D>(tb, 192, [&](int r, int j0, const float* v) {
+          if (r >= ch.n_replay && r < n) st8_out(o_ + ((size_t)srow[r] * H + h) * D + j0, v);
+        });
+        // Qeff = Qbar - P W (element (r, c)) into the S0 buffer, which the products above consumed
+        uint8_t *eh = s0h, *el = s0h + S::CDb;
+        acc_read<C, D>(tb, 320, [&](int r, int c0, const float* v) {
+          float e[8];
+          tile8<C>(qbh, qbl, r, c0, e);  // Qbar
+          for (int j = 0; j < 8; ++j) e[j] -= v[j];
+          put8<C, true>(eh, el, r, c0, e);
+        });
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) store_cd_tile(ws.W, base, eh, el);
+      }
+    }
+    // the bulk stores have read the tiles before the next head overwrites them
+    if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
   }
-  if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
-  tc::fence_before_sync();
-  __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
 }
 

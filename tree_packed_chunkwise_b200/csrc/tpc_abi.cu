@@ -158,6 +158,15 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
   return w;
 }
 
+// Heads one chunk CTA runs in turn (the largest divisor of H up to `most`): the next head's inputs
+// load while the current head computes, and the CTA's set-up is paid once.
+constexpr int kOutHeadsPerCta = 2;
+int heads_per_cta(int H, int most) {
+  for (int k = most; k > 1; --k)
+    if (H % k == 0) return k;
+  return 1;
+}
+
 bool shape_supported(int C, int D) { return (C == 16 && D == 32) || (C == 64 && D == 128) || (C == 32 && D == 64); }
 
 int check_shape(const tpc_plan* plan, const tpc_kda_shape* s) {
@@ -293,10 +302,12 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       TPC_CUDA(cudaStreamWaitEvent(st, scans[r - 1], 0));
       TPC_CUDA(cudaEventDestroy(scans[r - 1]));
+      const int hpc = heads_per_cta(H, kOutHeadsPerCta);
       for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_fwd_out_tc", st,
-                   (kda_fwd_out_tc<Tin, Tout><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads, OutTcSmem::total, st>>>(
-                       p.dt, H, q, k, g, static_cast<Tout*>(io->o), w, a)));
+                   (kda_fwd_out_tc<Tin, Tout><<<dim3(H / hpc, std::min(c1 - a, kMaxGridY)), kTcThreads,
+                                                OutTcSmem::total, st>>>(p.dt, H, q, k, g,
+                                                                         static_cast<Tout*>(io->o), w, a, hpc)));
     }
   } else {
     TPC_LAUNCH("kda_fwd_prep", st,
@@ -842,13 +853,14 @@ int tpc_kda_forward_static(const tpc_plan* plan, const tpc_kda_shape* s, const t
   char* base = nullptr;
   if (int rc = static_base(&base)) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (int rc = tpc_abi::plan_checks(plan, st)) return rc;
   tpc_abi::NvtxRange nvtx_call("tpc_kda_forward_static");
   // plan tables after the status word (pageable source: staged before cudaMemcpyAsync returns)
   std::vector<uint8_t> blob;
   tpc::pack_device_blob(p, off, blob);
   char* tables = base + kStaticStatusBytes;
   TPC_CUDA(cudaMemcpyAsync(tables, blob.data(), table_bytes, cudaMemcpyHostToDevice, st));
+  if (tpc_abi::checks_on())  // the copy of the tables this call reads
+    if (int rc = tpc_abi::table_checks_at(p, tables, off, st)) return rc;
   const tpc::DevTables dt = tpc::device_view(p, tables, off);
   tpc::KdaWs w;
   static_ws_layout(p, s->H, p.C, s->dk, kStaticStatusBytes + a256(table_bytes), &w, base);
