@@ -735,12 +735,15 @@ struct PrepTcSmemT {
 template <typename Tin>
 __global__ void __launch_bounds__(kTcThreads, 1)
     kda_fwd_prep_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
-                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, KdaWs ws, int chunk0 = 0) {
+                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, KdaWs ws, int chunk0 = 0,
+                    int hpc = 1) {
   using namespace tck;
   using S = PrepTcSmemT<Tin>;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
+  // grid (heads / hpc, chunks): a CTA runs hpc heads of one chunk in turn, the next head's gates and
+  // beta loaded into registers while the current head computes
+  const int ci = chunk0 + (int)blockIdx.y, h0 = (int)blockIdx.x * hpc;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -768,142 +771,152 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   [[maybe_unused]] __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
   [[maybe_unused]] __nv_bfloat16* sv = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
   GateRegs<Tin> gr;
-  gate_ld(gr, g_, srow, H, h, n);  // gates and beta first
-  const Tin bv = tid < n ? beta_[(size_t)srow[tid] * H + h] : Tin(0.f);  // (converted when stored)
-  if constexpr (EX) {
-    stage_rows_async(sk, k_, srow, H, h, n);
-    stage_rows_async(sv, v_, srow, H, h, n);
-  }
-  gate_st(sG, LD, gr);
-  if (tid < C) sb[tid] = to_f(bv);
-  __syncthreads();
-  cumsum_ref(sG, LD, n, sref, ws.status, reinterpret_cast<float*>(tl));  // (tiles not yet in use)
-  if constexpr (EX) tc::cp_async_wait<0>();
-  __syncthreads();
+  gate_ld(gr, g_, srow, H, h0, n);  // gates and beta first
+  Tin bv = tid < n ? beta_[(size_t)srow[tid] * H + h0] : Tin(0.f);  // (converted when stored)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
-  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  // a C x D tile of k (or v) transformed by f, from the staged rows (bf16) or from global memory
-  auto k_tile = [&](uint8_t* hi, uint8_t* lo, auto f) {
-    if constexpr (EX) build_tile_st<C, D, true>(hi, lo, sk, f);
-    else build_tile_ld<C, D, true, Tin>(hi, lo, row_k, f);
-  };
   bool ok = true;
-  // phase 1: Atilde = af bf^T with af = k e^{G - ref}, bf = k e^{ref - G}
-  {
-    uint8_t *afh = tl, *afl = tl + S::CDb, *bfh = tl + 2 * S::CDb, *bfl = tl + 3 * S::CDb;
-    if constexpr (EX) {  // e = 2^{G - ref} (bounded by the decay check), 2^{ref - G} = 1 / e
-      build_tile2_st<C, D>(afh, afl, bfh, bfl, sk, [&](int r, int c, float x) {
-        const float e = tc::ex2(sG[r * LD + c] - sref[c]);
-        return make_float2(x * e, x * tc::rcp_approx(e));
-      });
-    } else {
-      k_tile(afh, afl, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); });
-      k_tile(bfh, bfl, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
+  for (int hk = 0; hk < hpc && ok; ++hk) {
+    const int h = h0 + hk;
+    if constexpr (EX) {
+      stage_rows_async(sk, k_, srow, H, h, n);
+      stage_rows_async(sv, v_, srow, H, h, n);
     }
-    const tc::Op ah{tc::smem_u32(afh), C, false}, al{tc::smem_u32(afl), C, false};
-    const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
-    ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
-    if (ok) {
-      float* Ag = ws.At + ((size_t)ci * H + h) * C * C;  // kept for the backward
-      acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
-        float a[8];
-        for (int j = 0; j < 8; ++j) {
-          const int i = i0 + j;
-          a[j] = (i < r) ? v[j] : 0.f;
-          sA[r * LC + i] = sb[r] * a[j];  // L = diag(beta) Atilde, strict lower
-        }
-        st8g(Ag + r * C + i0, a);
-      });
+    gate_st(sG, LD, gr);
+    if (tid < C) sb[tid] = to_f(bv);
+    if (hk + 1 < hpc) {  // the next head's gates and beta, into the registers just consumed
+      gate_ld(gr, g_, srow, H, h + 1, n);
+      bv = tid < n ? beta_[(size_t)srow[tid] * H + h + 1] : Tin(0.f);
     }
-  }
-  if (ok) {
     __syncthreads();
-    block_inverse<LC>(sT, sA, sW1);
-    // T as a hi/lo tile (element (r, i) at cm_off(r, i, C)) for the backward, built where L was
-    uint8_t *ttH = reinterpret_cast<uint8_t*>(sA), *ttL = ttH + S::CCb;
-    build_tile<C, C, true>(ttH, ttL, [&](int r, int i) { return sT[r * LC + i]; });
-    // phase 2: W = T' Kbar and U' = T' V with T' = T diag(beta)
-    uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
-            *vl = vh + S::CDb;
-    build_tile<C, C, true>(th, tlo, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
-    k_tile(kh, kl, [&](int i, int c, float x) { return x * tc::ex2(sG[i * LD + c]); });
-    if constexpr (EX) build_tile_st<C, D, false>(vh, vl, sv, [&](int, int, float x) { return x; });
-    else build_tile_ld<C, D, true, Tin>(vh, vl, row_v, [&](int, int, float x) { return x; });
-    const tc::Op tH{tc::smem_u32(th), C, false}, tL{tc::smem_u32(tlo), C, false};
-    const tc::Op kH{tc::smem_u32(kh), C, true}, kL{tc::smem_u32(kl), C, true};
-    const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
-    const uint32_t id = tc::idesc_bf16(C, D, false, true);
-    ok = run(sy, [&] {
-      store_cc_tile(ws.Tm, ((size_t)ci * H + h), ttH, ttL);
-      mma3(tb + 64, tH, tL, kH, kL, C, id, false, false);
-      mma3(tb + 192, tH, tL, vH, vL, C, id, false, EX);
-    });
+    cumsum_ref(sG, LD, n, sref, ws.status, reinterpret_cast<float*>(tl));  // (tiles not yet in use)
+    if constexpr (EX) tc::cp_async_wait<0>();
+    __syncthreads();
+    tc::fence_after_sync();
+    auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+    auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+    // a C x D tile of k (or v) transformed by f, from the staged rows (bf16) or from global memory
+    auto k_tile = [&](uint8_t* hi, uint8_t* lo, auto f) {
+      if constexpr (EX) build_tile_st<C, D, true>(hi, lo, sk, f);
+      else build_tile_ld<C, D, true, Tin>(hi, lo, row_k, f);
+    };
+    // phase 1: Atilde = af bf^T with af = k e^{G - ref}, bf = k e^{ref - G}
+    {
+      uint8_t *afh = tl, *afl = tl + S::CDb, *bfh = tl + 2 * S::CDb, *bfl = tl + 3 * S::CDb;
+      if constexpr (EX) {  // e = 2^{G - ref} (bounded by the decay check), 2^{ref - G} = 1 / e
+        build_tile2_st<C, D>(afh, afl, bfh, bfl, sk, [&](int r, int c, float x) {
+          const float e = tc::ex2(sG[r * LD + c] - sref[c]);
+          return make_float2(x * e, x * tc::rcp_approx(e));
+        });
+      } else {
+        k_tile(afh, afl, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); });
+        k_tile(bfh, bfl, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
+      }
+      const tc::Op ah{tc::smem_u32(afh), C, false}, al{tc::smem_u32(afl), C, false};
+      const tc::Op bh{tc::smem_u32(bfh), C, false}, bl{tc::smem_u32(bfl), C, false};
+      ok = run(sy, [&] { mma3(tb, ah, al, bh, bl, D, tc::idesc_bf16(C, C, false, false), false, false); });
+      if (ok) {
+        float* Ag = ws.At + ((size_t)ci * H + h) * C * C;  // kept for the backward
+        acc_read<C, C>(tb, 0, [&](int r, int i0, const float* v) {
+          float a[8];
+          for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j;
+            a[j] = (i < r) ? v[j] : 0.f;
+            sA[r * LC + i] = sb[r] * a[j];  // L = diag(beta) Atilde, strict lower
+          }
+          st8g(Ag + r * C + i0, a);
+        });
+      }
+    }
     if (ok) {
-      // phase 3: the chunk's state transition S_end = M S_0 + B with M = Diag(e^{G_C}) - Khat^T W and
-      // B = Khat^T U' (Khat = k e^{G_C - G})
-      const size_t base = (size_t)ci * H + h;
-      uint8_t *wth = tl, *wtl = tl + S::CDb, *uth = tl + 2 * S::CDb, *utl = tl + 3 * S::CDb, *khh = tl + 4 * S::CDb,
-              *khl = tl + 5 * S::CDb;
-      // W and U' as hi/lo tiles, element (i, c) at cm_off(i, c, C): the operands of this phase and,
-      // stored as they are, of the output and backward kernels
-      acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) { put8<C, true>(wth, wtl, r, c0, v); });
-      acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) { put8<C, true>(uth, utl, r, c0, v); });
-      const float* gC = sG + (n - 1) * LD;
-      k_tile(khh, khl, [&](int i, int c, float x) { return x * tc::ex2(gC[c] - sG[i * LD + c]); });
+      __syncthreads();
+      block_inverse<LC>(sT, sA, sW1);
+      // T as a hi/lo tile (element (r, i) at cm_off(r, i, C)) for the backward, built where L was
+      uint8_t *ttH = reinterpret_cast<uint8_t*>(sA), *ttL = ttH + S::CCb;
+      build_tile<C, C, true>(ttH, ttL, [&](int r, int i) { return sT[r * LC + i]; });
+      // phase 2: W = T' Kbar and U' = T' V with T' = T diag(beta)
+      uint8_t *th = tl, *tlo = tl + S::CCb, *kh = tl + 2 * S::CCb, *kl = kh + S::CDb, *vh = kl + S::CDb,
+              *vl = vh + S::CDb;
+      build_tile<C, C, true>(th, tlo, [&](int r, int i) { return sT[r * LC + i] * sb[i]; });
+      k_tile(kh, kl, [&](int i, int c, float x) { return x * tc::ex2(sG[i * LD + c]); });
+      if constexpr (EX) build_tile_st<C, D, false>(vh, vl, sv, [&](int, int, float x) { return x; });
+      else build_tile_ld<C, D, true, Tin>(vh, vl, row_v, [&](int, int, float x) { return x; });
+      const tc::Op tH{tc::smem_u32(th), C, false}, tL{tc::smem_u32(tlo), C, false};
+      const tc::Op kH{tc::smem_u32(kh), C, true}, kL{tc::smem_u32(kl), C, true};
+      const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
+      const uint32_t id = tc::idesc_bf16(C, D, false, true);
       ok = run(sy, [&] {
-        store_cd_tile(ws.W, base, wth, wtl);
-        store_cd_tile(ws.U, base, uth, utl);
-        const uint32_t id = tc::idesc_bf16(D, D, true, true);
-        const tc::Op kH{tc::smem_u32(khh), C, true}, kL{tc::smem_u32(khl), C, true};
-        const tc::Op wH{tc::smem_u32(wth), C, true}, wL{tc::smem_u32(wtl), C, true};
-        const tc::Op uH{tc::smem_u32(uth), C, true}, uL{tc::smem_u32(utl), C, true};
-        mma4(tb, kH, kL, wH, wL, C, id, false, false, false);        // Khat^T W
-        mma4(tb + 128, kH, kL, uH, uL, C, id, false, false, false);  // Khat^T U'
+        store_cc_tile(ws.Tm, ((size_t)ci * H + h), ttH, ttL);
+        mma3(tb + 64, tH, tL, kH, kL, C, id, false, false);
+        mma3(tb + 192, tH, tL, vH, vL, C, id, false, EX);
       });
       if (ok) {
-        // M (tile) and B (slice-major) are assembled in the consumed tile space (and the staging rows,
-        // when they exist) and bulk-stored, once the W and U' stores have read their tiles
-        uint8_t* Mt = reinterpret_cast<uint8_t*>(ws.Mt) + base * kMtileBytes;
-        float* Bg = ws.Bc + base * D * D;
-        constexpr bool kBsm = 6 * S::CDb + 2 * S::StB >= kMtileBytes + sizeof(float) * D * D;
-        uint8_t* mts = tl;
-        float* bs = reinterpret_cast<float*>(tl + kMtileBytes);
-        if (tid == 0) tc::bulk_wait_read();
-        __syncthreads();
-        acc_read<D, D>(tb, 0, [&](int c, int c0, const float* v) {
-          float m[16];
-          const float gam = tc::ex2(gC[c]);
-          for (int j = 0; j < 16; ++j) m[j] = (c0 + j == c ? gam : 0.f) - v[j];
-          put16<D, true>(mts, mts + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
+        // phase 3: the chunk's state transition S_end = M S_0 + B with M = Diag(e^{G_C}) - Khat^T W and
+        // B = Khat^T U' (Khat = k e^{G_C - G})
+        const size_t base = (size_t)ci * H + h;
+        uint8_t *wth = tl, *wtl = tl + S::CDb, *uth = tl + 2 * S::CDb, *utl = tl + 3 * S::CDb, *khh = tl + 4 * S::CDb,
+                *khl = tl + 5 * S::CDb;
+        // W and U' as hi/lo tiles, element (i, c) at cm_off(i, c, C): the operands of this phase and,
+        // stored as they are, of the output and backward kernels
+        acc_read<C, D>(tb, 64, [&](int r, int c0, const float* v) { put8<C, true>(wth, wtl, r, c0, v); });
+        acc_read<C, D>(tb, 192, [&](int r, int c0, const float* v) { put8<C, true>(uth, utl, r, c0, v); });
+        const float* gC = sG + (n - 1) * LD;
+        k_tile(khh, khl, [&](int i, int c, float x) { return x * tc::ex2(gC[c] - sG[i * LD + c]); });
+        ok = run(sy, [&] {
+          store_cd_tile(ws.W, base, wth, wtl);
+          store_cd_tile(ws.U, base, uth, utl);
+          const uint32_t id = tc::idesc_bf16(D, D, true, true);
+          const tc::Op kH{tc::smem_u32(khh), C, true}, kL{tc::smem_u32(khl), C, true};
+          const tc::Op wH{tc::smem_u32(wth), C, true}, wL{tc::smem_u32(wtl), C, true};
+          const tc::Op uH{tc::smem_u32(uth), C, true}, uL{tc::smem_u32(utl), C, true};
+          mma4(tb, kH, kL, wH, wL, C, id, false, false, false);        // Khat^T W
+          mma4(tb + 128, kH, kL, uH, uL, C, id, false, false, false);  // Khat^T U'
         });
-        tc::fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {  // M leaves while B is assembled
-          tc::bulk_s2g(Mt, mts, kMtileBytes);
-          tc::bulk_commit();
-        }
-        acc_read<D, D>(tb, 128, [&](int c, int j0, const float* v) {  // slice-major for the scan's bulk loads
-          float* dst = kBsm ? bs : Bg;
-          for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(dst + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        });
-        if constexpr (kBsm) {
+        if (ok) {
+          // M (tile) and B (slice-major) are assembled in the consumed tile space (and the staging rows,
+          // when they exist) and bulk-stored, once the W and U' stores have read their tiles
+          uint8_t* Mt = reinterpret_cast<uint8_t*>(ws.Mt) + base * kMtileBytes;
+          float* Bg = ws.Bc + base * D * D;
+          constexpr bool kBsm = 6 * S::CDb + 2 * S::StB >= kMtileBytes + sizeof(float) * D * D;
+          uint8_t* mts = tl;
+          float* bs = reinterpret_cast<float*>(tl + kMtileBytes);
+          if (tid == 0) tc::bulk_wait_read();
+          __syncthreads();
+          acc_read<D, D>(tb, 0, [&](int c, int c0, const float* v) {
+            float m[16];
+            const float gam = tc::ex2(gC[c]);
+            for (int j = 0; j < 16; ++j) m[j] = (c0 + j == c ? gam : 0.f) - v[j];
+            put16<D, true>(mts, mts + kMtileBytes / 2, c, c0, m);  // element (c, c'): K-major A (M = c)
+          });
           tc::fence_async_smem();
           __syncthreads();
-          if (tid == 0) {
-            tc::bulk_s2g(Bg, bs, sizeof(float) * D * D);
+          if (tid == 0) {  // M leaves while B is assembled
+            tc::bulk_s2g(Mt, mts, kMtileBytes);
             tc::bulk_commit();
+          }
+          acc_read<D, D>(tb, 128, [&](int c, int j0, const float* v) {  // slice-major for the scan's bulk loads
+            float* dst = kBsm ? bs : Bg;
+            for (int j = 0; j < 16; j += 4)
+              *reinterpret_cast<float4*>(dst + slice_major(c, j0 + j)) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          });
+          if constexpr (kBsm) {
+            tc::fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+              tc::bulk_s2g(Bg, bs, sizeof(float) * D * D);
+              tc::bulk_commit();
+            }
           }
         }
       }
     }
+    // the bulk stores have read the tiles and staging rows before the next head overwrites them
+    if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
   }
-  if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
-  tc::fence_before_sync();
-  __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
 }
 
@@ -967,8 +980,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
   bool ok = true;
-  for (int hi = 0; hi < hpc && ok; ++hi) {
-    const int h = h0 + hi;
+  for (int hk = 0; hk < hpc && ok; ++hk) {
+    const int h = h0 + hk;
     const size_t base = (size_t)ci * H + h;
     if (tid == 0) {
       ld_expect(ld, kStateTileBytes + kCDTileBytes);
@@ -987,7 +1000,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         qfh, qfl, qbh, qbl, rq, [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); },
         [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c]); });
     build_tile_raw<C, D, Tin>(bfh, bfl, rk, [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); });
-    if (hi + 1 < hpc) {  // the next head's inputs, into the registers just consumed
+    if (hk + 1 < hpc) {  // the next head's inputs, into the registers just consumed
       hl = h + 1;
       gate_ld(gr, g_, srow, H, hl, n);
       raw_ld(rq, row_q);

@@ -160,7 +160,7 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
 
 // Heads one chunk CTA runs in turn (the largest divisor of H up to `most`): the next head's inputs
 // load while the current head computes, and the CTA's set-up is paid once.
-constexpr int kOutHeadsPerCta = 2;
+constexpr int kOutHeadsPerCta = 2, kPrepHeadsPerCta = 2;
 int heads_per_cta(int H, int most) {
   for (int k = most; k > 1; --k)
     if (H % k == 0) return k;
@@ -285,10 +285,11 @@ int forward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_fwd_i
       tpc_abi::NvtxRange nvtx_round("kda forward prep + scan", r);
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       const int s0 = p.round_seq_begin[r - 1], s1 = p.round_seq_begin[r];
+      const int hpc = heads_per_cta(H, kPrepHeadsPerCta);
       for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_fwd_prep_tc", st,
-                   (kda_fwd_prep_tc<Tin><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads, PrepTcSmemT<Tin>::total,
-                                           st>>>(p.dt, H, k, v, g, b, w, a)));
+                   (kda_fwd_prep_tc<Tin><<<dim3(H / hpc, std::min(c1 - a, kMaxGridY)), kTcThreads,
+                                           PrepTcSmemT<Tin>::total, st>>>(p.dt, H, k, v, g, b, w, a, hpc)));
       TPC_TRY_ABI(stream_after(hs, st));  // scan(r) after prep(r)
       if (s1 > s0)
         TPC_TRY_ABI((launch_scan<false, Tin>(hs, p, s0, s1, H, io->init_state, io->final_state, nullptr, w,
