@@ -1107,12 +1107,14 @@ template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kTcThreads, 1)
     kda_bwd_dq_tc(DevTables t, int H, const Tin* __restrict__ q_, const Tin* __restrict__ k_,
                   const Tin* __restrict__ g_, const Tin* __restrict__ do_, Tout* __restrict__ dq_, KdaWs ws,
-                  int chunk0 = 0) {
+                  int chunk0 = 0, int hpc = 1) {
   using namespace tck;
   using S = BdqTcSmem;
   constexpr int C = S::C, D = S::D, LD = S::LD;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
+  // grid (heads / hpc, chunks): a CTA runs hpc heads of one chunk in turn, the next head's gates
+  // loaded into registers while the current head computes
+  const int ci = chunk0 + (int)blockIdx.y, h0 = (int)blockIdx.x * hpc;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -1122,7 +1124,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t bar, bar_ld;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x;
-  const size_t base = (size_t)ci * H + h;
   uint8_t *doh = tsm + S::R, *dol = doh + S::CDb, *uh = dol + S::CDb, *ul = uh + S::CDb;
   uint8_t *sh = ul + S::CDb, *sl = sh + S::DDb;
   for (int i = tid; i < C; i += blockDim.x) srow[i] = i < n ? chunk_row(ch, t.replay_rows, i) : 0;
@@ -1135,200 +1136,209 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   __syncthreads();
   GateRegs<Tin> gr;
-  gate_ld(gr, g_, srow, H, h, n);  // gates first, then the workspace tiles and the row gathers
-  if (tid == 0) {
-    ld_expect(ld, kStateTileBytes + kCDTileBytes + kCCTileBytes);
-    ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
-    ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
-    ld_cc_tile(ld, tsm + S::Pt, tsm + S::Pt + S::CCb, ws.Pm, base);  // P, as the output kernel left it
-  }
-  // bf16: the chunk's q and k rows into shared memory while the gates load and accumulate
-  [[maybe_unused]] __nv_bfloat16* stq = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
-  [[maybe_unused]] __nv_bfloat16* stk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
-  auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  auto row_do = [&](int a) -> const Tin* {
-    return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
-  };
-  if constexpr (EX) {  // dO straight into its operand tile (raw bf16: no lo part)
-    stage_rows_async(stq, q_, srow, H, h, n);
-    stage_rows_async(stk, k_, srow, H, h, n);
-    tile_async_bf16<C, D>(doh, row_do, do_);
-  }
-  gate_st(sG, LD, gr);
-  __syncthreads();
-  cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(tsm + S::Scr));
-  float* se0 = sref + D;  // per channel 2^{G_0} and 2^{G_C - G_0} (ready long before the epilogue)
-  float* seC0 = se0 + D;
-  for (int c = tid; c < D; c += blockDim.x) {
-    se0[c] = tc::ex2(sref[c]);
-    seC0[c] = tc::ex2(sG[(n - 1) * LD + c] - sref[c]);
-  }
-  if constexpr (EX) tc::cp_async_wait<0>();
-  __syncthreads();
+  gate_ld(gr, g_, srow, H, h0, n);  // gates first, then the workspace tiles and the row gathers
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
-  // TMEM columns: Tq [0,128), T1 [128,256), RS [256,384), dP [384,448) then CS [384,512)
-  constexpr int cTq = 0, cT1 = 128, cRS = 256, cCS = 384;
-  if constexpr (!EX) build_tile_ld<C, D, true, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
-  const tc::Op oH{tc::smem_u32(doh), C, false}, oL{tc::smem_u32(dol), C, false};
-  const tc::Op uH{tc::smem_u32(uh), C, false}, uL{tc::smem_u32(ul), C, false};
-  const tc::Op sH{tc::smem_u32(sh), D, false}, sL{tc::smem_u32(sl), D, false};
-  bool ok = ld_wait(ld);
-  ok = ok && run(sy, [&] {
-    mma4(tb + cCS, oH, oL, uH, uL, D, tc::idesc_bf16(C, C, false, false), false, EX, false);   // dP (raw)
-    {  // dU = P^T dO, accumulated further in phase 2 (P^T: the P tile read MN-major; dO read MN-major)
-      const tc::Op pH{tc::smem_u32(tsm + S::Pt), C, true}, pL{tc::smem_u32(tsm + S::Pt + S::CCb), C, true};
-      const tc::Op dH{tc::smem_u32(doh), C, true}, dL{tc::smem_u32(dol), C, true};
-      mma4(tb + cRS, pH, pL, dH, dL, C, tc::idesc_bf16(C, D, true, true), false, false, EX);
-    }
-    mma4(tb + cTq, oH, oL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, EX, false);  // Tq
-  });
-  if (ok) {
-    // phase 2: T1 = U dS^T and dU = dU0 + Khat dS (Khat = k e^{G_C - G}, K-major in the dO slot);
-    // the gradient of the chunk-end state replaces S0 in its buffer
+  bool ok = true;
+  for (int hk = 0; hk < hpc && ok; ++hk) {
+    const int h = h0 + hk;
+    const size_t base = (size_t)ci * H + h;
     if (tid == 0) {
-      ld_expect(ld, kStateTileBytes);
-      ld_state_tile(ld, sh, sl, ws.dS, base);
+      ld_expect(ld, kStateTileBytes + kCDTileBytes + kCCTileBytes);
+      ld_state_tile(ld, sh, sl, ws.S0, base);  // chunk-start state
+      ld_cd_tile(ld, uh, ul, ws.U, base);        // U, as the output kernel left it
+      ld_cc_tile(ld, tsm + S::Pt, tsm + S::Pt + S::CCb, ws.Pm, base);  // P, as the output kernel left it
     }
-    const float* gC = sG + (n - 1) * LD;
-    auto khf = [&](int i, int c, float x) { return x * tc::ex2(gC[c] - sG[i * LD + c]); };
-    if constexpr (EX) build_tile_st<C, D, true>(doh, dol, stk, khf);
-    else build_tile_ld<C, D, true, Tin>(doh, dol, row_k, khf);
+    // bf16: the chunk's q and k rows into shared memory while the gates load and accumulate
+    [[maybe_unused]] __nv_bfloat16* stq = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage);
+    [[maybe_unused]] __nv_bfloat16* stk = reinterpret_cast<__nv_bfloat16*>(tsm + S::Stage + S::StB);
+    auto row_q = [&](int a) -> const Tin* { return a < n ? q_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+    auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+    auto row_do = [&](int a) -> const Tin* {
+      return (a >= ch.n_replay && a < n) ? do_ + ((size_t)srow[a] * H + h) * D : nullptr;
+    };
+    if constexpr (EX) {  // dO straight into its operand tile (raw bf16: no lo part)
+      stage_rows_async(stq, q_, srow, H, h, n);
+      stage_rows_async(stk, k_, srow, H, h, n);
+      tile_async_bf16<C, D>(doh, row_do, do_);
+    }
+    gate_st(sG, LD, gr);
+    if (hk + 1 < hpc) gate_ld(gr, g_, srow, H, h + 1, n);  // the next head's gates
+    __syncthreads();
+    cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(tsm + S::Scr));
+    float* se0 = sref + D;  // per channel 2^{G_0} and 2^{G_C - G_0} (ready long before the epilogue)
+    float* seC0 = se0 + D;
+    for (int c = tid; c < D; c += blockDim.x) {
+      se0[c] = tc::ex2(sref[c]);
+      seC0[c] = tc::ex2(sG[(n - 1) * LD + c] - sref[c]);
+    }
+    if constexpr (EX) tc::cp_async_wait<0>();
+    __syncthreads();
+    tc::fence_after_sync();
+    // TMEM columns: Tq [0,128), T1 [128,256), RS [256,384), dP [384,448) then CS [384,512)
+    constexpr int cTq = 0, cT1 = 128, cRS = 256, cCS = 384;
+    if constexpr (!EX) build_tile_ld<C, D, true, Tin>(doh, dol, row_do, [&](int, int, float x) { return x; });
+    const tc::Op oH{tc::smem_u32(doh), C, false}, oL{tc::smem_u32(dol), C, false};
+    const tc::Op uH{tc::smem_u32(uh), C, false}, uL{tc::smem_u32(ul), C, false};
+    const tc::Op sH{tc::smem_u32(sh), D, false}, sL{tc::smem_u32(sl), D, false};
     ok = ld_wait(ld);
     ok = ok && run(sy, [&] {
-      mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
-      const tc::Op kH{tc::smem_u32(doh), C, false}, kL{tc::smem_u32(dol), C, false};
-      const tc::Op dH{tc::smem_u32(sh), D, true}, dL{tc::smem_u32(sl), D, true};
-      mma4(tb + cRS, kH, kL, dH, dL, D, tc::idesc_bf16(C, D, false, true), true, false, false);
+      mma4(tb + cCS, oH, oL, uH, uL, D, tc::idesc_bf16(C, C, false, false), false, EX, false);   // dP (raw)
+      {  // dU = P^T dO, accumulated further in phase 2 (P^T: the P tile read MN-major; dO read MN-major)
+        const tc::Op pH{tc::smem_u32(tsm + S::Pt), C, true}, pL{tc::smem_u32(tsm + S::Pt + S::CCb), C, true};
+        const tc::Op dH{tc::smem_u32(doh), C, true}, dL{tc::smem_u32(dol), C, true};
+        mma4(tb + cRS, pH, pL, dH, dL, C, tc::idesc_bf16(C, D, true, true), false, false, EX);
+      }
+      mma4(tb + cTq, oH, oL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, EX, false);  // Tq
     });
     if (ok) {
-      // dU = dU0 + Khat dS as a hi/lo tile (element (i, j) at cm_off(i, j, C), in the consumed Khat
-      // slot) for the dk / dv kernel
-      acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) { put8<C, true>(doh, dol, i, j0, v); });
-      tc::fence_async_smem();
-      __syncthreads();
+      // phase 2: T1 = U dS^T and dU = dU0 + Khat dS (Khat = k e^{G_C - G}, K-major in the dO slot);
+      // the gradient of the chunk-end state replaces S0 in its buffer
       if (tid == 0) {
-        store_cd_tile(ws.dUt, base, doh, dol);
-        tc::bulk_wait_read();
+        ld_expect(ld, kStateTileBytes);
+        ld_state_tile(ld, sh, sl, ws.dS, base);
+      }
+      const float* gC = sG + (n - 1) * LD;
+      auto khf = [&](int i, int c, float x) { return x * tc::ex2(gC[c] - sG[i * LD + c]); };
+      if constexpr (EX) build_tile_st<C, D, true>(doh, dol, stk, khf);
+      else build_tile_ld<C, D, true, Tin>(doh, dol, row_k, khf);
+      ok = ld_wait(ld);
+      ok = ok && run(sy, [&] {
+        mma4(tb + cT1, uH, uL, sH, sL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
+        const tc::Op kH{tc::smem_u32(doh), C, false}, kL{tc::smem_u32(dol), C, false};
+        const tc::Op dH{tc::smem_u32(sh), D, true}, dL{tc::smem_u32(sl), D, true};
+        mma4(tb + cRS, kH, kL, dH, dL, D, tc::idesc_bf16(C, D, false, true), true, false, false);
+      });
+      if (ok) {
+        // dU = dU0 + Khat dS as a hi/lo tile (element (i, j) at cm_off(i, j, C), in the consumed Khat
+        // slot) for the dk / dv kernel
+        acc_read<C, D>(tb, cRS, [&](int i, int j0, const float* v) { put8<C, true>(doh, dol, i, j0, v); });
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+          store_cd_tile(ws.dUt, base, doh, dol);
+          tc::bulk_wait_read();
+        }
+        __syncthreads();
+      }
+    }
+    uint8_t *pH8 = tsm + S::R, *pL8 = pH8 + S::CCb, *bh = pL8 + S::CCb, *bl = bh + S::CDb, *qh = bl + S::CDb,
+            *ql = qh + S::CDb;
+    if (ok) {
+      acc_read<C, C>(tb, cCS, [&](int r, int i0, const float* v) {
+        float m[8];
+        for (int j = 0; j < 8; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
+        put8<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
+      });
+      auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
+      auto qff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
+      if constexpr (EX) {
+        build_tile_st<C, D, true>(bh, bl, stk, bff);
+        build_tile_st<C, D, true>(qh, ql, stq, qff);
+      } else {
+        build_tile_ld<C, D, true, Tin>(bh, bl, row_k, bff);
+        build_tile_ld<C, D, true, Tin>(qh, ql, row_q, qff);
+      }
+      ok = run(sy, [&] {
+        const uint32_t id = tc::idesc_bf16(C, D, false, true), idT = tc::idesc_bf16(C, D, true, true);
+        const tc::Op pK{tc::smem_u32(pH8), C, false}, pKl{tc::smem_u32(pL8), C, false};  // dP (r, i), K-major
+        const tc::Op pM{tc::smem_u32(pH8), C, true}, pMl{tc::smem_u32(pL8), C, true};    // dP^T (i, r), MN-major
+        const tc::Op bH{tc::smem_u32(bh), C, true}, bL{tc::smem_u32(bl), C, true};
+        const tc::Op qH{tc::smem_u32(qh), C, true}, qL{tc::smem_u32(ql), C, true};
+        mma4(tb + cRS, pK, pKl, bH, bL, C, id, false, false, false);
+        mma4(tb + cCS, pM, pMl, qH, qL, C, idT, false, false, false);
+      });
+    }
+    if (ok) {
+      float* pdk = ws.pdk + base * C * D;
+      float* pdG = ws.pdG + base * C * D;
+      float* sbuf = reinterpret_cast<float*>(tsm + S::R);  // [C][LD]: k e^{G_C - G} T1 per row
+      Tin* sq = reinterpret_cast<Tin*>(tsm + S::R + sizeof(float) * C * LD);
+      Tin* sk = sq + C * kStagePitch;
+      if constexpr (EX) {  // staged at the start
+        sq = reinterpret_cast<Tin*>(stq);
+        sk = reinterpret_cast<Tin*>(stk);
+      } else {
+        stage_rows(sq, q_, srow, H, h, n);
+        stage_rows(sk, k_, srow, H, h, n);
       }
       __syncthreads();
-    }
-  }
-  uint8_t *pH8 = tsm + S::R, *pL8 = pH8 + S::CCb, *bh = pL8 + S::CCb, *bl = bh + S::CDb, *qh = bl + S::CDb,
-          *ql = qh + S::CDb;
-  if (ok) {
-    acc_read<C, C>(tb, cCS, [&](int r, int i0, const float* v) {
-      float m[8];
-      for (int j = 0; j < 8; ++j) m[j] = (i0 + j <= r) ? v[j] : 0.f;
-      put8<C, true>(pH8, pL8, r, i0, m);  // element (r, i)
-    });
-    auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
-    auto qff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
-    if constexpr (EX) {
-      build_tile_st<C, D, true>(bh, bl, stk, bff);
-      build_tile_st<C, D, true>(qh, ql, stq, qff);
-    } else {
-      build_tile_ld<C, D, true, Tin>(bh, bl, row_k, bff);
-      build_tile_ld<C, D, true, Tin>(qh, ql, row_q, qff);
-    }
-    ok = run(sy, [&] {
-      const uint32_t id = tc::idesc_bf16(C, D, false, true), idT = tc::idesc_bf16(C, D, true, true);
-      const tc::Op pK{tc::smem_u32(pH8), C, false}, pKl{tc::smem_u32(pL8), C, false};  // dP (r, i), K-major
-      const tc::Op pM{tc::smem_u32(pH8), C, true}, pMl{tc::smem_u32(pL8), C, true};    // dP^T (i, r), MN-major
-      const tc::Op bH{tc::smem_u32(bh), C, true}, bL{tc::smem_u32(bl), C, true};
-      const tc::Op qH{tc::smem_u32(qh), C, true}, qL{tc::smem_u32(ql), C, true};
-      mma4(tb + cRS, pK, pKl, bH, bL, C, id, false, false, false);
-      mma4(tb + cCS, pM, pMl, qH, qL, C, idT, false, false, false);
-    });
-  }
-  if (ok) {
-    float* pdk = ws.pdk + base * C * D;
-    float* pdG = ws.pdG + base * C * D;
-    float* sbuf = reinterpret_cast<float*>(tsm + S::R);  // [C][LD]: k e^{G_C - G} T1 per row
-    Tin* sq = reinterpret_cast<Tin*>(tsm + S::R + sizeof(float) * C * LD);
-    Tin* sk = sq + C * kStagePitch;
-    if constexpr (EX) {  // staged at the start
-      sq = reinterpret_cast<Tin*>(stq);
-      sk = reinterpret_cast<Tin*>(stk);
-    } else {
-      stage_rows(sq, q_, srow, H, h, n);
-      stage_rows(sk, k_, srow, H, h, n);
-    }
-    __syncthreads();
-    const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
-    const int r = 16 * sp + (lane & 15);  // accumulator row; this lane's 8 columns: share8
-    const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
-    static_assert(D == 2 * 16 * kTcGroups && C == 64 && kTcGroups == 4, "the pd_frag lane map");
-    for (int it = 0; it < 2; ++it) {
-      const int cc = grp * 16 + 16 * kTcGroups * it;
-      float tq[8], t1[8], rs[8], cs[8];
+      const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
+      const int r = 16 * sp + (lane & 15);  // accumulator row; this lane's 8 columns: share8
+      const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
+      static_assert(D == 2 * 16 * kTcGroups && C == 64 && kTcGroups == 4, "the pd_frag lane map");
+      for (int it = 0; it < 2; ++it) {
+        const int cc = grp * 16 + 16 * kTcGroups * it;
+        float tq[8], t1[8], rs[8], cs[8];
+        {
+          uint32_t a0[16], a1[16], a2[16], a3[16];  // four loads in flight, one wait
+          tc::tmem_ld16_nowait(la + cTq + cc, a0);
+          tc::tmem_ld16_nowait(la + cT1 + cc, a1);
+          tc::tmem_ld16_nowait(la + cRS + cc, a2);
+          tc::tmem_ld16_nowait(la + cCS + cc, a3);
+          tc::tmem_wait_ld();
+          tc::tmem_regs16(a0);
+          tc::tmem_regs16(a1);
+          tc::tmem_regs16(a2);
+          tc::tmem_regs16(a3);
+          share8u(a0, tq);
+          share8u(a1, t1);
+          share8u(a2, rs);
+          share8u(a3, cs);
+        }
+        const int c0 = cc + 8 * (lane >> 4);
+        float qv[8], kv[8], dq[8], dk[8], dG[8];
+        staged8(sq, r, c0, qv);
+        staged8(sk, r, c0, kv);
+  #pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = c0 + j;
+          // a = 2^{G_r - G_0} (bounded by the chunk's decay check), 1/a = 2^{G_0 - G_r};
+          // 2^{G_r} = 2^{G_0} a and 2^{G_C - G_r} = 2^{G_C - G_0} / a
+          const float a = tc::ex2(sG[r * LD + c] - sref[c]), ia = tc::rcp_approx(a);
+          dq[j] = a * fmaf(se0[c], tq[j], rs[j]);
+          const float dks = seC0[c] * ia * t1[j];
+          dk[j] = fmaf(ia, cs[j], dks);
+          dG[j] = qv[j] * dq[j] - kv[j] * dk[j];
+          sbuf[r * LD + c] = r < n ? kv[j] * dks : 0.f;
+        }
+        {
+          float4* pk = reinterpret_cast<float4*>(pdk) + pd_frag(w, it, lane);
+          float4* pg = reinterpret_cast<float4*>(pdG) + pd_frag(w, it, lane);
+          pk[0] = make_float4(dk[0], dk[1], dk[2], dk[3]);
+          pk[32] = make_float4(dk[4], dk[5], dk[6], dk[7]);
+          pg[0] = make_float4(dG[0], dG[1], dG[2], dG[3]);
+          pg[32] = make_float4(dG[4], dG[5], dG[6], dG[7]);
+        }
+        if (r >= ch.n_replay && r < n) st8_out(dq_ + ((size_t)srow[r] * H + h) * D + c0, dq);
+      }
+      __syncthreads();
+      // per column c: sum over rows of the row buffer and sum_j dS_cj S0_cj, each split over four
+      // threads (rows and j in quarters) and combined in a fixed order
+      static_assert(kTcThreads == 4 * D, "four threads per column");
+      float* part = reinterpret_cast<float*>(tsm + S::R + S::Part);  // [2][4][D]
       {
-        uint32_t a0[16], a1[16], a2[16], a3[16];  // four loads in flight, one wait
-        tc::tmem_ld16_nowait(la + cTq + cc, a0);
-        tc::tmem_ld16_nowait(la + cT1 + cc, a1);
-        tc::tmem_ld16_nowait(la + cRS + cc, a2);
-        tc::tmem_ld16_nowait(la + cCS + cc, a3);
-        tc::tmem_wait_ld();
-        tc::tmem_regs16(a0);
-        tc::tmem_regs16(a1);
-        tc::tmem_regs16(a2);
-        tc::tmem_regs16(a3);
-        share8u(a0, tq);
-        share8u(a1, t1);
-        share8u(a2, rs);
-        share8u(a3, cs);
+        const int c = tid % D, q4 = tid / D;
+        float a = 0.f;
+        for (int i = 16 * q4; i < 16 * q4 + 16; ++i) a += sbuf[i * LD + c];  // rows >= n hold zeros
+        part[q4 * D + c] = a;
+        part[(4 + q4) * D + c] = state_row_dot(ws.dS, ws.S0, base, c, 32 * q4, 32 * q4 + 32);
       }
-      const int c0 = cc + 8 * (lane >> 4);
-      float qv[8], kv[8], dq[8], dk[8], dG[8];
-      staged8(sq, r, c0, qv);
-      staged8(sk, r, c0, kv);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = c0 + j;
-        // a = 2^{G_r - G_0} (bounded by the chunk's decay check), 1/a = 2^{G_0 - G_r};
-        // 2^{G_r} = 2^{G_0} a and 2^{G_C - G_r} = 2^{G_C - G_0} / a
-        const float a = tc::ex2(sG[r * LD + c] - sref[c]), ia = tc::rcp_approx(a);
-        dq[j] = a * fmaf(se0[c], tq[j], rs[j]);
-        const float dks = seC0[c] * ia * t1[j];
-        dk[j] = fmaf(ia, cs[j], dks);
-        dG[j] = qv[j] * dq[j] - kv[j] * dk[j];
-        sbuf[r * LD + c] = r < n ? kv[j] * dks : 0.f;
+      __syncthreads();
+      if (tid < D) {
+        const int c = tid;
+        const float acc = (part[c] + part[D + c]) + (part[2 * D + c] + part[3 * D + c]);
+        const float acc2 = (part[4 * D + c] + part[5 * D + c]) + (part[6 * D + c] + part[7 * D + c]);
+        pdG[pd_index(n - 1, c)] += acc + tc::ex2(sG[(n - 1) * LD + c]) * acc2;
       }
-      {
-        float4* pk = reinterpret_cast<float4*>(pdk) + pd_frag(w, it, lane);
-        float4* pg = reinterpret_cast<float4*>(pdG) + pd_frag(w, it, lane);
-        pk[0] = make_float4(dk[0], dk[1], dk[2], dk[3]);
-        pk[32] = make_float4(dk[4], dk[5], dk[6], dk[7]);
-        pg[0] = make_float4(dG[0], dG[1], dG[2], dG[3]);
-        pg[32] = make_float4(dG[4], dG[5], dG[6], dG[7]);
-      }
-      if (r >= ch.n_replay && r < n) st8_out(dq_ + ((size_t)srow[r] * H + h) * D + c0, dq);
     }
+    // the bulk stores have read their tiles before the next head overwrites them
+    if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
+    tc::fence_before_sync();
     __syncthreads();
-    // per column c: sum over rows of the row buffer and sum_j dS_cj S0_cj, each split over four
-    // threads (rows and j in quarters) and combined in a fixed order
-    static_assert(kTcThreads == 4 * D, "four threads per column");
-    float* part = reinterpret_cast<float*>(tsm + S::R + S::Part);  // [2][4][D]
-    {
-      const int c = tid % D, q4 = tid / D;
-      float a = 0.f;
-      for (int i = 16 * q4; i < 16 * q4 + 16; ++i) a += sbuf[i * LD + c];  // rows >= n hold zeros
-      part[q4 * D + c] = a;
-      part[(4 + q4) * D + c] = state_row_dot(ws.dS, ws.S0, base, c, 32 * q4, 32 * q4 + 32);
-    }
-    __syncthreads();
-    if (tid < D) {
-      const int c = tid;
-      const float acc = (part[c] + part[D + c]) + (part[2 * D + c] + part[3 * D + c]);
-      const float acc2 = (part[4 * D + c] + part[5 * D + c]) + (part[6 * D + c] + part[7 * D + c]);
-      pdG[pd_index(n - 1, c)] += acc + tc::ex2(sG[(n - 1) * LD + c]) * acc2;
-    }
+    tc::fence_after_sync();
   }
-  if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
-  tc::fence_before_sync();
-  __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
 }
 
@@ -1371,12 +1381,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     kda_bwd_dkv_tc(DevTables t, int H, const Tin* __restrict__ k_, const Tin* __restrict__ v_,
                    const Tin* __restrict__ g_, const Tin* __restrict__ beta_, Tout* __restrict__ dk_,
                    Tout* __restrict__ dv_, float* __restrict__ dg_, float* __restrict__ dbeta_, KdaWs ws,
-                   int chunk0 = 0) {
+                   int chunk0 = 0, int hpc = 1) {
   using namespace tck;
   using S = BdkvTcSmemT<Tin>;
   constexpr int C = S::C, D = S::D, LD = S::LD, LC = S::LC;
   constexpr bool EX = std::is_same<Tin, __nv_bfloat16>::value;
-  const int ci = chunk0 + (int)blockIdx.y, h = blockIdx.x;  // grid (heads, chunks)
+  // grid (heads / hpc, chunks): a CTA runs hpc heads of one chunk in turn, the next head's gates
+  // loaded into registers while the current head computes
+  const int ci = chunk0 + (int)blockIdx.y, h0 = (int)blockIdx.x * hpc;
   const ChunkRec ch = t.chunks[ci];
   const int n = ch.n_rows;
   extern __shared__ __align__(1024) uint8_t tsm[];
@@ -1405,323 +1417,335 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   __syncthreads();
   GateRegs<Tin> gr;
-  gate_ld(gr, g_, srow, H, h, n);  // gates and beta first, then the copies
-  const Tin bv = tid < n ? beta_[(size_t)srow[tid] * H + h] : Tin(0.f);  // (converted when stored)
-  for (int e = tid; e < 3 * kTcGroups * C; e += blockDim.x) sdb[e] = 0.f;
-  Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
-  auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  if constexpr (S::kStageK) {
-    stage_rows_async(reinterpret_cast<__nv_bfloat16*>(sk), reinterpret_cast<const __nv_bfloat16*>(k_), srow, H, h, n);
-    tile_async_bf16<C, D>(R + S::p2_V, row_v, v_);  // V straight into its phase-2a operand tile
-  }
-  {  // Atilde (fp32, padded rows) by 4-byte asynchronous copies; T (hi/lo tile) by a bulk copy
-    const size_t cb = (size_t)ci * H + h;
-    const float* Ag = ws.At + cb * C * C;
-    for (int e = tid; e < C * C; e += blockDim.x) tc::cp_async4(sAt + (e / C) * LC + (e % C), Ag + e, 4u);
-    tc::cp_async_commit();
-    if (tid == 0) {
-      ld_expect(ld, kCCTileBytes);
-      ld_cc_tile(ld, tTh, tTl, ws.Tm, cb);
-    }
-  }
-  if (tid < C) {  // where row tid's gradients go (read while the gates are in flight)
-    const int i = tid, row = srow[i];
-    int kind = 2, idx = row;
-    if (i < ch.n_replay) {
-      kind = 0;
-      idx = ch.replay_base + i;
-    } else if (i < n) {
-      const int tg = t.row_tgt[row];
-      if (tg >= 0) {
-        kind = 1;
-        idx = tg;
-      }
-    }
-    skind[i] = kind;
-    sidx[i] = idx;
-  }
-  gate_st(sG, LD, gr);
-  if (tid < C) sb[tid] = to_f(bv);
-  __syncthreads();
-  cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(R));  // (R's first phase comes later)
-  float* se0 = sdb + 3 * kTcGroups * C;  // per channel 2^{G_0}
-  for (int c = tid; c < D; c += blockDim.x) se0[c] = tc::ex2(sref[c]);
-  tc::cp_async_wait<0>();  // staged k, V and Atilde
-  __syncthreads();
+  gate_ld(gr, g_, srow, H, h0, n);  // gates and beta first, then the copies
+  Tin bv = tid < n ? beta_[(size_t)srow[tid] * H + h0] : Tin(0.f);  // (converted when stored)
   tc::fence_after_sync();
   const uint32_t tb = tslot;
   Sync sy{&bar, 0u, ws.status};
-  auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
-  // 8 values of k row r from column c0 on (zero for r >= n)
-  auto k8 = [&](int r, int c0, float(&kv)[8]) {
+  bool ok = true;
+  for (int hk = 0; hk < hpc && ok; ++hk) {
+    const int h = h0 + hk;
+    const size_t base = (size_t)ci * H + h;
+    for (int e = tid; e < 3 * kTcGroups * C; e += blockDim.x) sdb[e] = 0.f;
+    Tin* sk = reinterpret_cast<Tin*>(tsm + S::Ks);
+    auto row_v = [&](int a) -> const Tin* { return a < n ? v_ + ((size_t)srow[a] * H + h) * D : nullptr; };
     if constexpr (S::kStageK) {
-      staged8(sk, r, c0, kv);
-    } else if (r < n) {
-      ld8(k_ + ((size_t)srow[r] * H + h) * D + c0, kv);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) kv[j] = 0.f;
+      stage_rows_async(reinterpret_cast<__nv_bfloat16*>(sk), reinterpret_cast<const __nv_bfloat16*>(k_), srow, H, h, n);
+      tile_async_bf16<C, D>(R + S::p2_V, row_v, v_);  // V straight into its phase-2a operand tile
     }
-  };
-  const size_t base = (size_t)ci * H + h;
-  float* pdk = ws.pdk + base * C * D;
-  float* pdG = ws.pdG + base * C * D;
-  const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
-  const int myrow = 16 * sp + (lane & 15);  // M = 64 accumulator row; this lane's 8 columns: share8
-  const int half8 = 8 * (lane >> 4);
-  float pre_dk[2][8], pre_dG[2][8];  // the final phase's dq-kernel partials (loaded ahead)
-  uint4 vraw[2][sizeof(Tin) / 2];     // phase 4's v values (loaded ahead, raw)
-  // 8 gradient values of row r from column c0 on, to where the row's gradients go
-  auto out8 = [&](float* replay_buf, float* tgt_buf, Tout* out, int r, int c0, const float* v) {
-    const size_t o = ((size_t)sidx[r] * H + h) * D + c0;
-    if (skind[r] == 0) st8g(replay_buf + o, v);
-    else if (skind[r] == 1) st8g(tgt_buf + o, v);
-    else st8_out(out + o, v);
-  };
-  const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
-  // TMEM columns
-  // dB_k [0, 128) stays in TMEM until the last phase; CS reuses the dB_v columns [128, 256)
-  constexpr int cW = 64, cU = 192, cdW = 320, cdB = 0, cdA = 256, cRS = 320, cCS = 128;
-
-  // ---- phase 1: Atilde and T as the forward left them (loaded above)
-  bool ok = ld_wait(ld);
-  // element (r, i) of T from its hi/lo tile
-  auto tval = [&](int r, int i) {
-    const uint32_t o = cm_off(r, i, C);
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tTh + o)) +
-           __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tTl + o));
-  };
-  if (ok) {
-    // ---- phase 2a: W = T' Kbar, U' = T' V (T' = T diag(beta)); the T tile for T^T dX
-    uint8_t *tph = R + S::p2_Tp, *tpl = tph + S::CCb, *kbh = R + S::p2_Kb, *kbl = kbh + S::CDb, *vh = R + S::p2_V,
-            *vl = vh + S::CDb;
-    build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return tval(r, i) * sb[i]; });
-    auto kbf = [&](int i, int c, float x) { return x * tc::ex2(sG[i * LD + c]); };
-    if constexpr (S::kStageK) build_tile_st<C, D, true>(kbh, kbl, reinterpret_cast<const __nv_bfloat16*>(sk), kbf);
-    else build_tile_ld<C, D, true, Tin>(kbh, kbl, row_k, kbf);
-    if constexpr (!EX) build_tile_ld<C, D, true, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
-    ok = run(sy, [&] {
-      const uint32_t id = tc::idesc_bf16(C, D, false, true);
-      const tc::Op tH{tc::smem_u32(tph), C, false}, tL{tc::smem_u32(tpl), C, false};
-      const tc::Op kH{tc::smem_u32(kbh), C, true}, kL{tc::smem_u32(kbl), C, true};
-      const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
-      mma4(tb + cW, tH, tL, kH, kL, C, id, false, false, false);
-      mma4(tb + cU, tH, tL, vH, vL, C, id, false, false, EX);
-    });
-  }
-  if (ok) {
-    // ---- phase 2b: dW' = dU S0^T.  dU is loaded where phase 3's dX keeps its columns [D, 2D) (a
-    // C x D sub-tile of the K-major C x 2D layout is itself a C x D K-major tile), S0 where X goes.
-    uint8_t *dxh0 = R + S::p3_dX, *dxl0 = dxh0 + 2 * S::CDb;
-    uint8_t *duh = dxh0 + tc::cm_off(0, D, C), *dul = dxl0 + tc::cm_off(0, D, C);
-    uint8_t *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
-    if (tid == 0) {  // the phase 2a operands are consumed
-      ld_expect(ld, kStateTileBytes + kCDTileBytes);
-      ld_state_tile(ld, s0h, s0l, ws.S0, base);
-      ld_cd_tile(ld, duh, dul, ws.dUt, base);
-    }
-    ok = ld_wait(ld);
-    ok = ok && run(sy, [&] {
-      const tc::Op aH{tc::smem_u32(duh), C, false}, aL{tc::smem_u32(dul), C, false};
-      const tc::Op bH{tc::smem_u32(s0h), D, false}, bL{tc::smem_u32(s0l), D, false};
-      mma4(tb + cdW, aH, aL, bH, bL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
-    });
-  }
-  if (ok) {
-    // ---- phase 3: X (K-major, rows i, columns n in [0, 2D)) and dX (MN-major, k = r, n)
-    uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb, *dxh = R + S::p3_dX, *dxl = dxh + 2 * S::CDb;
-    // this lane's v values for phase 4 (its rows' columns of dB_v), loaded now and converted there
-    static_assert(2 * D == 4 * 16 * kTcGroups, "four 16-column chunks of dB per warp group");
-    for (int t2 = 0; t2 < 2; ++t2) {
-      const int c1 = grp * 16 + 16 * kTcGroups * t2 + half8;
-      const Tin* p = v_ + ((size_t)srow[myrow] * H + h) * D + c1;
-#pragma unroll
-      for (int q = 0; q < (int)(sizeof(Tin) / 2); ++q)
-        vraw[t2][q] = myrow < n ? __ldg(reinterpret_cast<const uint4*>(p) + q) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    acc_read<C, D>(tb, cW, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, c0, v); });
-    acc_read<C, D>(tb, cU, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, D + c0, v); });
-    acc_read<C, D>(tb, cdW, [&](int r, int c0, const float* v) {
-      float m[8];
-      for (int j = 0; j < 8; ++j) m[j] = -v[j];
-      put8<C, true>(dxh, dxl, r, c0, m);
-    });
-    // (dX columns [D, 2D) = dU, loaded in phase 2b)
-    ok = run(sy, [&] {
-      const tc::Op aH{tc::smem_u32(tTh), C, true}, aL{tc::smem_u32(tTl), C, true};
-      const tc::Op bH{tc::smem_u32(dxh), C, true}, bL{tc::smem_u32(dxl), C, true};
-      mma4(tb + cdB, aH, aL, bH, bL, C, tc::idesc_bf16(C, 2 * D, true, true), false, false, false);
-    });
-  }
-  if (ok) {
-    // ---- read dB: dB tile for dA; dv; dk / dG / dbeta contributions
-    uint8_t *dbh = R + S::p4_dB, *dbl = dbh + 2 * S::CDb;
-#pragma unroll
-    for (int t4 = 0; t4 < 4; ++t4) {
-      const int cc = grp * 16 + 16 * kTcGroups * t4;
-      float v[8];
-      {
-        float v16[16];
-        tc::tmem_ld16(la + cdB + cc, v16);
-        share8(v16, v);
+    {  // Atilde (fp32, padded rows) by 4-byte asynchronous copies; T (hi/lo tile) by a bulk copy
+      const size_t cb = (size_t)ci * H + h;
+      const float* Ag = ws.At + cb * C * C;
+      for (int e = tid; e < C * C; e += blockDim.x) tc::cp_async4(sAt + (e / C) * LC + (e % C), Ag + e, 4u);
+      tc::cp_async_commit();
+      if (tid == 0) {
+        ld_expect(ld, kCCTileBytes);
+        ld_cc_tile(ld, tTh, tTl, ws.Tm, cb);
       }
-      const int i = myrow, c0 = cc + half8;
-      put8<C, true>(dbh, dbl, i, c0, v);
-      float part = 0.f;
-      if (t4 < 2) {  // columns < D: dB_k (its dk / dG terms are added in the last phase, from TMEM)
-        float kv[8];
-        k8(i, c0, kv);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) part = fmaf(v[j], kv[j] * tc::ex2(sG[i * LD + c0 + j]), part);
+    }
+    if (tid < C) {  // where row tid's gradients go (read while the gates are in flight)
+      const int i = tid, row = srow[i];
+      int kind = 2, idx = row;
+      if (i < ch.n_replay) {
+        kind = 0;
+        idx = ch.replay_base + i;
       } else if (i < n) {
-        const int c1 = c0 - D;
-        float vv[8], val[8];
-        raw_get<Tin>(vraw[t4 - 2], vv);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          part = fmaf(v[j], vv[j], part);
-          val[j] = sb[i] * v[j];
+        const int tg = t.row_tgt[row];
+        if (tg >= 0) {
+          kind = 1;
+          idx = tg;
         }
-        out8(ws.rdv, ws.tdv, dv_, i, c1, val);
       }
-      part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);  // columns 0-7 + 8-15 of the chunk
-      if (lane < 16) sdb[((t4 < 2 ? 0 : 1) * kTcGroups + grp) * C + i] += part;  // one slot per (half, group)
+      skind[i] = kind;
+      sidx[i] = idx;
     }
-    uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb;
-    ok = run(sy, [&] {
-      const tc::Op aH{tc::smem_u32(dbh), C, false}, aL{tc::smem_u32(dbl), C, false};
-      const tc::Op bH{tc::smem_u32(xh), C, false}, bL{tc::smem_u32(xl), C, false};
-      mma4(tb + cdA, aH, aL, bH, bL, 2 * D, tc::idesc_bf16(C, C, false, false), false, false, false);
-    });
-  }
-  if (ok) {
-    // ---- dA = -(dB X^T) strict lower; dAt = beta dA (tile); dbeta += rowsum(dA Atilde)
-    uint8_t *dah = R + S::p5_dA, *dal = dah + S::CCb;
-    for (int cc = grp * 16; cc < C; cc += 16 * kTcGroups) {
-      float v[8];
-      {
-        float v16[16];
-        tc::tmem_ld16(la + cdA + cc, v16);
-        share8(v16, v);
+    gate_st(sG, LD, gr);
+    if (tid < C) sb[tid] = to_f(bv);
+    if (hk + 1 < hpc) {  // the next head's gates and beta, into the registers just consumed
+      gate_ld(gr, g_, srow, H, h + 1, n);
+      bv = tid < n ? beta_[(size_t)srow[tid] * H + h + 1] : Tin(0.f);
+    }
+    __syncthreads();
+    cumsum_ref(sG, LD, n, sref, nullptr, reinterpret_cast<float*>(R));  // (R's first phase comes later)
+    float* se0 = sdb + 3 * kTcGroups * C;  // per channel 2^{G_0}
+    for (int c = tid; c < D; c += blockDim.x) se0[c] = tc::ex2(sref[c]);
+    tc::cp_async_wait<0>();  // staged k, V and Atilde
+    __syncthreads();
+    tc::fence_after_sync();
+    auto row_k = [&](int a) -> const Tin* { return a < n ? k_ + ((size_t)srow[a] * H + h) * D : nullptr; };
+    // 8 values of k row r from column c0 on (zero for r >= n)
+    auto k8 = [&](int r, int c0, float(&kv)[8]) {
+      if constexpr (S::kStageK) {
+        staged8(sk, r, c0, kv);
+      } else if (r < n) {
+        ld8(k_ + ((size_t)srow[r] * H + h) * D + c0, kv);
+      } else {
+  #pragma unroll
+        for (int j = 0; j < 8; ++j) kv[j] = 0.f;
       }
-      const int r = myrow, c0 = cc + half8;
-      float m[8], part = 0.f;
-      for (int j = 0; j < 8; ++j) {
-        const int i = c0 + j;
-        const float dA = (i < r) ? -v[j] : 0.f;
-        part = fmaf(dA, sAt[r * LC + i], part);
-        m[j] = sb[r] * dA;
-      }
-      put8<C, true>(dah, dal, r, c0, m);  // element (r, i)
-      part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);
-      if (lane < 16) sdb[(2 * kTcGroups + grp) * C + r] += part;
-    }
-    // the dq kernel's partials of this lane's final-phase rows and columns, loaded ahead of phase 5
-    static_assert(D == 2 * 16 * kTcGroups, "two 16-column chunks per warp group in the final phase");
-    for (int it = 0; it < 2; ++it) {  // (the pd_frag order of the dq kernel's epilogue)
-      const float4* pk = reinterpret_cast<const float4*>(pdk) + pd_frag(w, it, lane);
-      const float4* pg = reinterpret_cast<const float4*>(pdG) + pd_frag(w, it, lane);
-      const float4 a0 = pk[0], a1 = pk[32], b0 = pg[0], b1 = pg[32];
-      pre_dk[it][0] = a0.x; pre_dk[it][1] = a0.y; pre_dk[it][2] = a0.z; pre_dk[it][3] = a0.w;
-      pre_dk[it][4] = a1.x; pre_dk[it][5] = a1.y; pre_dk[it][6] = a1.z; pre_dk[it][7] = a1.w;
-      pre_dG[it][0] = b0.x; pre_dG[it][1] = b0.y; pre_dG[it][2] = b0.z; pre_dG[it][3] = b0.w;
-      pre_dG[it][4] = b1.x; pre_dG[it][5] = b1.y; pre_dG[it][6] = b1.z; pre_dG[it][7] = b1.w;
-    }
-    // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
-    uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
-    auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
-    auto aff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
-    if constexpr (S::kStageK) {  // e = 2^{G - ref} (bounded by the decay check), 2^{ref - G} = 1 / e
-      build_tile2_st<C, D>(afh, afl, bfh, bfl, reinterpret_cast<const __nv_bfloat16*>(sk), [&](int r, int c, float x) {
-        const float e = tc::ex2(sG[r * LD + c] - sref[c]);
-        return make_float2(x * e, x * tc::rcp_approx(e));
+    };
+    float* pdk = ws.pdk + base * C * D;
+    float* pdG = ws.pdG + base * C * D;
+    const int w = tid >> 5, lane = tid & 31, sp = w & 3, grp = w >> 2;
+    const int myrow = 16 * sp + (lane & 15);  // M = 64 accumulator row; this lane's 8 columns: share8
+    const int half8 = 8 * (lane >> 4);
+    float pre_dk[2][8], pre_dG[2][8];  // the final phase's dq-kernel partials (loaded ahead)
+    uint4 vraw[2][sizeof(Tin) / 2];     // phase 4's v values (loaded ahead, raw)
+    // 8 gradient values of row r from column c0 on, to where the row's gradients go
+    auto out8 = [&](float* replay_buf, float* tgt_buf, Tout* out, int r, int c0, const float* v) {
+      const size_t o = ((size_t)sidx[r] * H + h) * D + c0;
+      if (skind[r] == 0) st8g(replay_buf + o, v);
+      else if (skind[r] == 1) st8g(tgt_buf + o, v);
+      else st8_out(out + o, v);
+    };
+    const uint32_t la = tb + ((uint32_t)(32 * sp) << 16);
+    // TMEM columns
+    // dB_k [0, 128) stays in TMEM until the last phase; CS reuses the dB_v columns [128, 256)
+    constexpr int cW = 64, cU = 192, cdW = 320, cdB = 0, cdA = 256, cRS = 320, cCS = 128;
+
+    // ---- phase 1: Atilde and T as the forward left them (loaded above)
+    ok = ld_wait(ld);
+    // element (r, i) of T from its hi/lo tile
+    auto tval = [&](int r, int i) {
+      const uint32_t o = cm_off(r, i, C);
+      return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tTh + o)) +
+             __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tTl + o));
+    };
+    if (ok) {
+      // ---- phase 2a: W = T' Kbar, U' = T' V (T' = T diag(beta)); the T tile for T^T dX
+      uint8_t *tph = R + S::p2_Tp, *tpl = tph + S::CCb, *kbh = R + S::p2_Kb, *kbl = kbh + S::CDb, *vh = R + S::p2_V,
+              *vl = vh + S::CDb;
+      build_tile<C, C, true>(tph, tpl, [&](int r, int i) { return tval(r, i) * sb[i]; });
+      auto kbf = [&](int i, int c, float x) { return x * tc::ex2(sG[i * LD + c]); };
+      if constexpr (S::kStageK) build_tile_st<C, D, true>(kbh, kbl, reinterpret_cast<const __nv_bfloat16*>(sk), kbf);
+      else build_tile_ld<C, D, true, Tin>(kbh, kbl, row_k, kbf);
+      if constexpr (!EX) build_tile_ld<C, D, true, Tin>(vh, vl, row_v, [&](int i, int c, float x) { return x; });
+      ok = run(sy, [&] {
+        const uint32_t id = tc::idesc_bf16(C, D, false, true);
+        const tc::Op tH{tc::smem_u32(tph), C, false}, tL{tc::smem_u32(tpl), C, false};
+        const tc::Op kH{tc::smem_u32(kbh), C, true}, kL{tc::smem_u32(kbl), C, true};
+        const tc::Op vH{tc::smem_u32(vh), C, true}, vL{tc::smem_u32(vl), C, true};
+        mma4(tb + cW, tH, tL, kH, kL, C, id, false, false, false);
+        mma4(tb + cU, tH, tL, vH, vL, C, id, false, false, EX);
       });
-    } else {
-      build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, bff);
-      build_tile_ld<C, D, true, Tin>(afh, afl, row_k, aff);
     }
-    ok = run(sy, [&] {
-      const tc::Op pK{tc::smem_u32(dah), C, false}, pKl{tc::smem_u32(dal), C, false};
-      const tc::Op pM{tc::smem_u32(dah), C, true}, pMl{tc::smem_u32(dal), C, true};
-      const tc::Op bH{tc::smem_u32(bfh), C, true}, bL{tc::smem_u32(bfl), C, true};
-      const tc::Op aH{tc::smem_u32(afh), C, true}, aL{tc::smem_u32(afl), C, true};
-      mma4(tb + cRS, pK, pKl, bH, bL, C, tc::idesc_bf16(C, D, false, true), false, false, false);
-      mma4(tb + cCS, pM, pMl, aH, aL, C, tc::idesc_bf16(C, D, true, true), false, false, false);
-    });
-  }
-  if (ok) {
-    // ---- final: dk, dG = partials + dB_k terms + gated terms; dG staged for the reverse cumulative sum
-    float* sdG = reinterpret_cast<float*>(R);  // [C][LD]
-#pragma unroll
-    for (int it = 0; it < 2; ++it) {
-      const int cc = grp * 16 + 16 * kTcGroups * it;
-      float rs[8], cs[8], dbk[8];
+    if (ok) {
+      // ---- phase 2b: dW' = dU S0^T.  dU is loaded where phase 3's dX keeps its columns [D, 2D) (a
+      // C x D sub-tile of the K-major C x 2D layout is itself a C x D K-major tile), S0 where X goes.
+      uint8_t *dxh0 = R + S::p3_dX, *dxl0 = dxh0 + 2 * S::CDb;
+      uint8_t *duh = dxh0 + tc::cm_off(0, D, C), *dul = dxl0 + tc::cm_off(0, D, C);
+      uint8_t *s0h = R + S::p2_S0, *s0l = s0h + S::DDb;
+      if (tid == 0) {  // the phase 2a operands are consumed
+        ld_expect(ld, kStateTileBytes + kCDTileBytes);
+        ld_state_tile(ld, s0h, s0l, ws.S0, base);
+        ld_cd_tile(ld, duh, dul, ws.dUt, base);
+      }
+      ok = ld_wait(ld);
+      ok = ok && run(sy, [&] {
+        const tc::Op aH{tc::smem_u32(duh), C, false}, aL{tc::smem_u32(dul), C, false};
+        const tc::Op bH{tc::smem_u32(s0h), D, false}, bL{tc::smem_u32(s0l), D, false};
+        mma4(tb + cdW, aH, aL, bH, bL, D, tc::idesc_bf16(C, D, false, false), false, false, false);
+      });
+    }
+    if (ok) {
+      // ---- phase 3: X (K-major, rows i, columns n in [0, 2D)) and dX (MN-major, k = r, n)
+      uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb, *dxh = R + S::p3_dX, *dxl = dxh + 2 * S::CDb;
+      // this lane's v values for phase 4 (its rows' columns of dB_v), loaded now and converted there
+      static_assert(2 * D == 4 * 16 * kTcGroups, "four 16-column chunks of dB per warp group");
+      for (int t2 = 0; t2 < 2; ++t2) {
+        const int c1 = grp * 16 + 16 * kTcGroups * t2 + half8;
+        const Tin* p = v_ + ((size_t)srow[myrow] * H + h) * D + c1;
+  #pragma unroll
+        for (int q = 0; q < (int)(sizeof(Tin) / 2); ++q)
+          vraw[t2][q] = myrow < n ? __ldg(reinterpret_cast<const uint4*>(p) + q) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      acc_read<C, D>(tb, cW, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, c0, v); });
+      acc_read<C, D>(tb, cU, [&](int i, int c0, const float* v) { put8<C, true>(xh, xl, i, D + c0, v); });
+      acc_read<C, D>(tb, cdW, [&](int r, int c0, const float* v) {
+        float m[8];
+        for (int j = 0; j < 8; ++j) m[j] = -v[j];
+        put8<C, true>(dxh, dxl, r, c0, m);
+      });
+      // (dX columns [D, 2D) = dU, loaded in phase 2b)
+      ok = run(sy, [&] {
+        const tc::Op aH{tc::smem_u32(tTh), C, true}, aL{tc::smem_u32(tTl), C, true};
+        const tc::Op bH{tc::smem_u32(dxh), C, true}, bL{tc::smem_u32(dxl), C, true};
+        mma4(tb + cdB, aH, aL, bH, bL, C, tc::idesc_bf16(C, 2 * D, true, true), false, false, false);
+      });
+    }
+    if (ok) {
+      // ---- read dB: dB tile for dA; dv; dk / dG / dbeta contributions
+      uint8_t *dbh = R + S::p4_dB, *dbl = dbh + 2 * S::CDb;
+  #pragma unroll
+      for (int t4 = 0; t4 < 4; ++t4) {
+        const int cc = grp * 16 + 16 * kTcGroups * t4;
+        float v[8];
+        {
+          float v16[16];
+          tc::tmem_ld16(la + cdB + cc, v16);
+          share8(v16, v);
+        }
+        const int i = myrow, c0 = cc + half8;
+        put8<C, true>(dbh, dbl, i, c0, v);
+        float part = 0.f;
+        if (t4 < 2) {  // columns < D: dB_k (its dk / dG terms are added in the last phase, from TMEM)
+          float kv[8];
+          k8(i, c0, kv);
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) part = fmaf(v[j], kv[j] * tc::ex2(sG[i * LD + c0 + j]), part);
+        } else if (i < n) {
+          const int c1 = c0 - D;
+          float vv[8], val[8];
+          raw_get<Tin>(vraw[t4 - 2], vv);
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            part = fmaf(v[j], vv[j], part);
+            val[j] = sb[i] * v[j];
+          }
+          out8(ws.rdv, ws.tdv, dv_, i, c1, val);
+        }
+        part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);  // columns 0-7 + 8-15 of the chunk
+        if (lane < 16) sdb[((t4 < 2 ? 0 : 1) * kTcGroups + grp) * C + i] += part;  // one slot per (half, group)
+      }
+      uint8_t *xh = R + S::p3_X, *xl = xh + 2 * S::CDb;
+      ok = run(sy, [&] {
+        const tc::Op aH{tc::smem_u32(dbh), C, false}, aL{tc::smem_u32(dbl), C, false};
+        const tc::Op bH{tc::smem_u32(xh), C, false}, bL{tc::smem_u32(xl), C, false};
+        mma4(tb + cdA, aH, aL, bH, bL, 2 * D, tc::idesc_bf16(C, C, false, false), false, false, false);
+      });
+    }
+    if (ok) {
+      // ---- dA = -(dB X^T) strict lower; dAt = beta dA (tile); dbeta += rowsum(dA Atilde)
+      uint8_t *dah = R + S::p5_dA, *dal = dah + S::CCb;
+      for (int cc = grp * 16; cc < C; cc += 16 * kTcGroups) {
+        float v[8];
+        {
+          float v16[16];
+          tc::tmem_ld16(la + cdA + cc, v16);
+          share8(v16, v);
+        }
+        const int r = myrow, c0 = cc + half8;
+        float m[8], part = 0.f;
+        for (int j = 0; j < 8; ++j) {
+          const int i = c0 + j;
+          const float dA = (i < r) ? -v[j] : 0.f;
+          part = fmaf(dA, sAt[r * LC + i], part);
+          m[j] = sb[r] * dA;
+        }
+        put8<C, true>(dah, dal, r, c0, m);  // element (r, i)
+        part += __shfl_sync(0xffffffffu, part, (lane + 16) & 31);
+        if (lane < 16) sdb[(2 * kTcGroups + grp) * C + r] += part;
+      }
+      // the dq kernel's partials of this lane's final-phase rows and columns, loaded ahead of phase 5
+      static_assert(D == 2 * 16 * kTcGroups, "two 16-column chunks per warp group in the final phase");
+      for (int it = 0; it < 2; ++it) {  // (the pd_frag order of the dq kernel's epilogue)
+        const float4* pk = reinterpret_cast<const float4*>(pdk) + pd_frag(w, it, lane);
+        const float4* pg = reinterpret_cast<const float4*>(pdG) + pd_frag(w, it, lane);
+        const float4 a0 = pk[0], a1 = pk[32], b0 = pg[0], b1 = pg[32];
+        pre_dk[it][0] = a0.x; pre_dk[it][1] = a0.y; pre_dk[it][2] = a0.z; pre_dk[it][3] = a0.w;
+        pre_dk[it][4] = a1.x; pre_dk[it][5] = a1.y; pre_dk[it][6] = a1.z; pre_dk[it][7] = a1.w;
+        pre_dG[it][0] = b0.x; pre_dG[it][1] = b0.y; pre_dG[it][2] = b0.z; pre_dG[it][3] = b0.w;
+        pre_dG[it][4] = b1.x; pre_dG[it][5] = b1.y; pre_dG[it][6] = b1.z; pre_dG[it][7] = b1.w;
+      }
+      // ---- phase 5: RS = dAt bf, CS = dAt^T af (bf, af as MN-major B operands)
+      uint8_t *bfh = R + S::p5_bf, *bfl = bfh + S::CDb, *afh = R + S::p5_af, *afl = afh + S::CDb;
+      auto bff = [&](int i, int c, float x) { return x * tc::ex2(sref[c] - sG[i * LD + c]); };
+      auto aff = [&](int r, int c, float x) { return x * tc::ex2(sG[r * LD + c] - sref[c]); };
+      if constexpr (S::kStageK) {  // e = 2^{G - ref} (bounded by the decay check), 2^{ref - G} = 1 / e
+        build_tile2_st<C, D>(afh, afl, bfh, bfl, reinterpret_cast<const __nv_bfloat16*>(sk), [&](int r, int c, float x) {
+          const float e = tc::ex2(sG[r * LD + c] - sref[c]);
+          return make_float2(x * e, x * tc::rcp_approx(e));
+        });
+      } else {
+        build_tile_ld<C, D, true, Tin>(bfh, bfl, row_k, bff);
+        build_tile_ld<C, D, true, Tin>(afh, afl, row_k, aff);
+      }
+      ok = run(sy, [&] {
+        const tc::Op pK{tc::smem_u32(dah), C, false}, pKl{tc::smem_u32(dal), C, false};
+        const tc::Op pM{tc::smem_u32(dah), C, true}, pMl{tc::smem_u32(dal), C, true};
+        const tc::Op bH{tc::smem_u32(bfh), C, true}, bL{tc::smem_u32(bfl), C, true};
+        const tc::Op aH{tc::smem_u32(afh), C, true}, aL{tc::smem_u32(afl), C, true};
+        mma4(tb + cRS, pK, pKl, bH, bL, C, tc::idesc_bf16(C, D, false, true), false, false, false);
+        mma4(tb + cCS, pM, pMl, aH, aL, C, tc::idesc_bf16(C, D, true, true), false, false, false);
+      });
+    }
+    if (ok) {
+      // ---- final: dk, dG = partials + dB_k terms + gated terms; dG staged for the reverse cumulative sum
+      float* sdG = reinterpret_cast<float*>(R);  // [C][LD]
+  #pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        const int cc = grp * 16 + 16 * kTcGroups * it;
+        float rs[8], cs[8], dbk[8];
+        {
+          uint32_t a0[16], a1[16], a2[16];  // three loads in flight, one wait
+          tc::tmem_ld16_nowait(la + cRS + cc, a0);
+          tc::tmem_ld16_nowait(la + cCS + cc, a1);
+          tc::tmem_ld16_nowait(la + cdB + cc, a2);
+          tc::tmem_wait_ld();
+          tc::tmem_regs16(a0);
+          tc::tmem_regs16(a1);
+          tc::tmem_regs16(a2);
+          share8u(a0, rs);
+          share8u(a1, cs);
+          share8u(a2, dbk);
+        }
+        const int r = myrow, c0 = cc + half8;
+        float kv[8], dkv[8], pg[8];
+        k8(r, c0, kv);
+  #pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          dkv[j] = pre_dk[it][j];
+          pg[j] = pre_dG[it][j];
+        }
+  #pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = c0 + j;
+          // e = 2^{G_r - G_0} (bounded by the chunk's decay check), 1/e = 2^{G_0 - G_r}, 2^{G_r} = 2^{G_0} e
+          const float e = tc::ex2(sG[r * LD + c] - sref[c]), ie = tc::rcp_approx(e);
+          const float a = e * rs[j], b = ie * cs[j];
+          const float wb = se0[c] * e * sb[r] * dbk[j];
+          dkv[j] += wb + (a + b);
+          sdG[r * LD + c] = r < n ? pg[j] + kv[j] * (wb + (a - b)) : 0.f;
+        }
+        if (r < n) out8(ws.rdk, ws.tdk, dk_, r, c0, dkv);
+      }
+      __syncthreads();
+      // dg = reverse cumulative sum of dG over the chunk's rows: four threads per column, each a
+      // quarter of the rows; the quarters' totals first, then each quarter's running sum from below
+      static_assert(kTcThreads == 4 * D, "four threads per column");
+      float* qsum = sdG + C * LD;  // [4][D]
+      const int c = tid % D, q4 = tid / D, r_lo = 16 * q4;
       {
-        uint32_t a0[16], a1[16], a2[16];  // three loads in flight, one wait
-        tc::tmem_ld16_nowait(la + cRS + cc, a0);
-        tc::tmem_ld16_nowait(la + cCS + cc, a1);
-        tc::tmem_ld16_nowait(la + cdB + cc, a2);
-        tc::tmem_wait_ld();
-        tc::tmem_regs16(a0);
-        tc::tmem_regs16(a1);
-        tc::tmem_regs16(a2);
-        share8u(a0, rs);
-        share8u(a1, cs);
-        share8u(a2, dbk);
+        float a = 0.f;
+  #pragma unroll
+        for (int r = r_lo; r < r_lo + 16; ++r) a += sdG[r * LD + c];  // rows >= n hold zeros
+        qsum[q4 * D + c] = a;
       }
-      const int r = myrow, c0 = cc + half8;
-      float kv[8], dkv[8], pg[8];
-      k8(r, c0, kv);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        dkv[j] = pre_dk[it][j];
-        pg[j] = pre_dG[it][j];
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = c0 + j;
-        // e = 2^{G_r - G_0} (bounded by the chunk's decay check), 1/e = 2^{G_0 - G_r}, 2^{G_r} = 2^{G_0} e
-        const float e = tc::ex2(sG[r * LD + c] - sref[c]), ie = tc::rcp_approx(e);
-        const float a = e * rs[j], b = ie * cs[j];
-        const float wb = se0[c] * e * sb[r] * dbk[j];
-        dkv[j] += wb + (a + b);
-        sdG[r * LD + c] = r < n ? pg[j] + kv[j] * (wb + (a - b)) : 0.f;
-      }
-      if (r < n) out8(ws.rdk, ws.tdk, dk_, r, c0, dkv);
-    }
-    __syncthreads();
-    // dg = reverse cumulative sum of dG over the chunk's rows: four threads per column, each a
-    // quarter of the rows; the quarters' totals first, then each quarter's running sum from below
-    static_assert(kTcThreads == 4 * D, "four threads per column");
-    float* qsum = sdG + C * LD;  // [4][D]
-    const int c = tid % D, q4 = tid / D, r_lo = 16 * q4;
-    {
-      float a = 0.f;
-#pragma unroll
-      for (int r = r_lo; r < r_lo + 16; ++r) a += sdG[r * LD + c];  // rows >= n hold zeros
-      qsum[q4 * D + c] = a;
-    }
-    __syncthreads();
-    {
-      float acc = 0.f;
-      for (int q = 3; q > q4; --q) acc += qsum[q * D + c];
-      for (int r = r_lo + 15; r >= r_lo; --r) {
-        acc += sdG[r * LD + c];
-        if (r < n) {
-          float* dst = skind[r] == 0 ? ws.rdg : (skind[r] == 1 ? ws.tdg : dg_);
-          dst[((size_t)sidx[r] * H + h) * D + c] = acc;
+      __syncthreads();
+      {
+        float acc = 0.f;
+        for (int q = 3; q > q4; --q) acc += qsum[q * D + c];
+        for (int r = r_lo + 15; r >= r_lo; --r) {
+          acc += sdG[r * LD + c];
+          if (r < n) {
+            float* dst = skind[r] == 0 ? ws.rdg : (skind[r] == 1 ? ws.tdg : dg_);
+            dst[((size_t)sidx[r] * H + h) * D + c] = acc;
+          }
         }
       }
+      for (int r = tid; r < n; r += blockDim.x) {
+        float db = 0.f;
+        for (int q = 0; q < 3 * kTcGroups; ++q) db += sdb[q * C + r];
+        float* dst = skind[r] == 0 ? ws.rdb : (skind[r] == 1 ? ws.tdb : dbeta_);
+        dst[(size_t)sidx[r] * H + h] = db;
+      }
     }
-    for (int r = tid; r < n; r += blockDim.x) {
-      float db = 0.f;
-      for (int q = 0; q < 3 * kTcGroups; ++q) db += sdb[q * C + r];
-      float* dst = skind[r] == 0 ? ws.rdb : (skind[r] == 1 ? ws.tdb : dbeta_);
-      dst[(size_t)sidx[r] * H + h] = db;
-    }
+    // the bulk stores have read their tiles before the next head overwrites them
+    if (tid == 0) tc::bulk_wait_read();  // (the stores complete with the grid)
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
   }
-  tc::fence_before_sync();
-  __syncthreads();
   if ((tid >> 5) == 0) tc::tmem_dealloc(tb, 512);
 }
 

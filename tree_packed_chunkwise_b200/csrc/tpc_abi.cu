@@ -160,7 +160,7 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
 
 // Heads one chunk CTA runs in turn (the largest divisor of H up to `most`): the next head's inputs
 // load while the current head computes, and the CTA's set-up is paid once.
-constexpr int kOutHeadsPerCta = 2, kPrepHeadsPerCta = 2;
+constexpr int kOutHeadsPerCta = 2, kPrepHeadsPerCta = 2, kBwdHeadsPerCta = 2;
 int heads_per_cta(int H, int most) {
   for (int k = most; k > 1; --k)
     if (H % k == 0) return k;
@@ -368,16 +368,18 @@ int backward_impl(const tpc::Plan& p, const tpc_kda_shape* s, const tpc_kda_bwd_
       const int c0 = p.round_chunk_begin[r - 1], c1 = p.round_chunk_begin[r];
       TPC_CUDA(cudaStreamWaitEvent(st, scans[i], 0));
       TPC_CUDA(cudaEventDestroy(scans[i]));
+      const int hpc = heads_per_cta(H, kBwdHeadsPerCta);
       for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_bwd_dq_tc", st,
-                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads, BdqTcSmem::total, st>>>(
-                       p.dt, H, q, k, g, dO, static_cast<Tout*>(io->dq), w, a)));
+                   (kda_bwd_dq_tc<Tin, Tout><<<dim3(H / hpc, std::min(c1 - a, kMaxGridY)), kTcThreads,
+                                               BdqTcSmem::total, st>>>(p.dt, H, q, k, g, dO,
+                                                                       static_cast<Tout*>(io->dq), w, a, hpc)));
       for (int a = c0; a < c1; a += kMaxGridY)
         TPC_LAUNCH("kda_bwd_dkv_tc", st,
-                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(H, std::min(c1 - a, kMaxGridY)), kTcThreads,
+                   (kda_bwd_dkv_tc<Tin, Tout><<<dim3(H / hpc, std::min(c1 - a, kMaxGridY)), kTcThreads,
                                                 BdkvTcSmemT<Tin>::total, st>>>(
                        p.dt, H, k, v, g, b, static_cast<Tout*>(io->dk), static_cast<Tout*>(io->dv), io->dg,
-                       io->dbeta, w, a)));
+                       io->dbeta, w, a, hpc)));
     }
   } else {
     TPC_LAUNCH("kda_bwd_prep", st,
