@@ -83,6 +83,21 @@ def test_random_forest_fp32(tpc, seed):
     check(case, run_case(tpc, case)[1], TOL["f32"])
 
 
+@pytest.mark.parametrize("H", [1, 3, 6])
+def test_tensor_core_path_head_counts(tpc, H):
+    """bf16 at chunk 64 / d 128 on a ragged forest (replays, several roots, partial chunks) with head
+    counts that the chunk kernels split differently over their CTAs: one head per CTA (H = 1, 3)
+    and two heads per CTA over an odd number of CTAs per chunk (H = 6)."""
+    rng = np.random.default_rng(40 + H)
+    n = 9
+    parent = [-1] + [(-1 if rng.random() < 0.15 else int(rng.integers(0, i))) for i in range(1, n)]
+    length = rng.integers(1, 150, size=n).astype(np.int32)
+    tree = synth.Tree(np.array(parent, np.int32), length)
+    case = Case(tree, H, 128, 64, "bf16", 300 + H, with_init=(H == 3))
+    errs = check(case, run_case(tpc, case)[1], TOL["bf16"])
+    print("head count", H, errs)
+
+
 def test_single_segment_and_short_tree(tpc):
     for tree in (synth.Tree(np.array([-1], np.int32), np.array([1], np.int32)),
                  synth.Tree(np.array([-1, 0, 0], np.int32), np.array([16, 16, 1], np.int32))):
