@@ -160,7 +160,7 @@ tpc::KdaWs ws_view(const WsLayout& L, void* ws) {
 
 // Heads one chunk CTA runs in turn (the largest divisor of H up to `most`): the next head's inputs
 // load while the current head computes, and the CTA's set-up is paid once.
-constexpr int kOutHeadsPerCta = 2, kPrepHeadsPerCta = 2, kBwdHeadsPerCta = 2;
+constexpr int kOutHeadsPerCta = 2, kPrepHeadsPerCta = 4, kBwdHeadsPerCta = 4;
 int heads_per_cta(int H, int most) {
   for (int k = most; k > 1; --k)
     if (H % k == 0) return k;
