@@ -66,14 +66,44 @@ def step_flops_per_token_head(C, d):
     return 3 * (10 * C * d + 6 * d * d)
 
 
+def _flat_numbers(j, prefix=""):
+    """{dotted.key: number} of a nested JSON object."""
+    out = {}
+    if isinstance(j, dict):
+        for k, v in j.items():
+            out.update(_flat_numbers(v, f"{prefix}{k}."))
+    elif isinstance(j, (int, float)) and not isinstance(j, bool):
+        out[prefix[:-1].lower()] = float(j)
+    return out
+
+
+def _pick(nums, must, avoid=()):
+    for k, v in nums.items():
+        if all(m in k for m in must) and not any(a in k for a in avoid) and v > 0:
+            return v
+    return None
+
+
 def load_peaks():
+    """Measured HBM copy bandwidth (GB/s) and bf16 dense throughput (TFLOP/s, burst and sustained) of
+    this machine's B200s from MEASURED_PEAKS.json when present (keys located by name: hbm_gbs,
+    bf16_tflops, bf16_tflops_sustained or the like); the pool's earlier measurement otherwise."""
+    fb = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+    if not os.path.exists(p):
+        return fb
+    try:
         with open(p) as f:
-            j = json.load(f)
-        return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"], sustained=j.get("bf16_tflops_sustained"),
-                    sm_max_mhz=j.get("sm_max_mhz", 1965.0), source="measured")
-    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+            nums = _flat_numbers(json.load(f))
+    except (OSError, ValueError):
+        return fb
+    hbm = nums.get("hbm_gbs") or _pick(nums, ("hbm",), ("util", "frac", "pct"))
+    bf16 = nums.get("bf16_tflops") or _pick(nums, ("bf16",), ("sustain", "util", "frac", "pct", "mhz", "clock"))
+    sus = nums.get("bf16_tflops_sustained") or _pick(nums, ("bf16", "sustain"), ("mhz", "clock", "util", "frac"))
+    if not hbm or not bf16:
+        return fb
+    return dict(hbm_gbs=hbm, bf16_tflops=bf16, sustained=sus, sm_max_mhz=nums.get("sm_max_mhz", 1965.0),
+                source="measured")
 
 
 class ClockSampler:
